@@ -1,0 +1,263 @@
+"""Pins of the float64 oracle against things other than itself.
+
+Each check compares the oracle (literal token recurrence + BPTT, "Gated Linear
+Attention Transformers with Hardware-Efficient Training", section 4.1) with a
+different formulation the paper fixes, a closed form, an invariant, or finite
+differences.  All run on the CPU in seconds.
+"""
+import json
+import os
+
+import numpy as np
+import pytest
+
+from oracle import forms
+
+RNG = np.random.default_rng(1234)
+
+
+def rand_head(T, K, V, gate_scale=1.0, rng=RNG):
+    q = rng.standard_normal((T, K))
+    k = rng.standard_normal((T, K)) / np.sqrt(K)
+    v = rng.standard_normal((T, V))
+    z = rng.standard_normal((T, K))
+    la = gate_scale * np.log(1.0 / (1.0 + np.exp(-z))) / 16.0
+    return q, k, v, la
+
+
+def one(oracle, q, k, v, la, h0=None, gate="vector"):
+    """Run the oracle on a single head given 2-D arrays."""
+    def e(x):
+        return None if x is None else x[None, None]
+    o, hT = oracle.fwd(e(q), e(k), e(v), e(la), h0=e(h0), gate=gate)
+    return o[0, 0], hT[0, 0]
+
+
+# ---------------------------------------------------------------- forward pins
+
+@pytest.mark.parametrize("T,K,V", [(1, 1, 1), (5, 3, 2), (8, 4, 4)])
+def test_brute_force_tiny(oracle_mod, T, K, V):
+    q, k, v, la = rand_head(T, K, V)
+    h0 = RNG.standard_normal((K, V))
+    for h in (None, h0):
+        o, _ = one(oracle_mod, q, k, v, la, h)
+        ref = forms.brute_force(q, k, v, la, h)
+        np.testing.assert_allclose(o, ref, rtol=0, atol=1e-12)
+
+
+def test_parallel_form(oracle_mod):
+    """C = L: masked parallel form ((Q.B)(K/B)^T . M) V (section 4.1)."""
+    q, k, v, la = rand_head(48, 8, 6)
+    h0 = RNG.standard_normal((8, 6))
+    o, _ = one(oracle_mod, q, k, v, la, h0)
+    np.testing.assert_allclose(o, forms.parallel_form(q, k, v, la, h0), rtol=1e-11, atol=1e-11)
+    o2, S2 = forms.chunkwise_two_level(q, k, v, la, C=48, c=16, h0=h0)
+    np.testing.assert_allclose(o, o2, rtol=1e-11, atol=1e-11)
+
+
+def test_chunk_size_one_is_recurrence(oracle_mod):
+    """C = 1 chunkwise recovers the recurrent form (section 2.2)."""
+    q, k, v, la = rand_head(37, 5, 7)
+    o, hT = one(oracle_mod, q, k, v, la)
+    o2, S2 = forms.chunkwise_two_level(q, k, v, la, C=1, c=1)
+    np.testing.assert_allclose(o, o2, rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(hT, S2, rtol=1e-11, atol=1e-12)
+
+
+@pytest.mark.parametrize("T,C,c", [(64, 16, 4), (100, 32, 8), (130, 64, 16), (256, 64, 16), (77, 8, 8)])
+def test_chunkwise_any_tiling(oracle_mod, T, C, c):
+    """Any chunk / sub-chunk size (incl. a ragged tail) gives the recurrence."""
+    q, k, v, la = rand_head(T, 12, 10, gate_scale=4.0)
+    h0 = RNG.standard_normal((12, 10))
+    o, hT = one(oracle_mod, q, k, v, la, h0)
+    o2, S2 = forms.chunkwise_two_level(q, k, v, la, C=C, c=c, h0=h0)
+    np.testing.assert_allclose(o, o2, rtol=1e-10, atol=1e-10)
+    np.testing.assert_allclose(hT, S2, rtol=1e-10, atol=1e-10)
+
+
+def test_strong_gates_long_sequence(oracle_mod):
+    """Decay products underflow in the naive parallel form; the oracle and the
+    log-space chunkwise form stay finite and agree."""
+    q, k, v, la = rand_head(300, 6, 5)
+    la = np.full_like(la, -5.0)
+    o, hT = one(oracle_mod, q, k, v, la)
+    assert np.all(np.isfinite(o))
+    o2, S2 = forms.chunkwise_two_level(q, k, v, la, C=64, c=16)
+    np.testing.assert_allclose(o, o2, rtol=1e-10, atol=1e-10)
+
+
+def test_ungated_is_linear_attention(oracle_mod):
+    """alpha == 1 reduces to (Q K^T . M) V (section 2.1), in both the 'none'
+    mode and a vector gate of exact zeros."""
+    q, k, v, _ = rand_head(40, 6, 9)
+    ref = forms.linear_attention(q, k, v)
+    o, _ = one(oracle_mod, q, k, v, None, gate="none")
+    np.testing.assert_allclose(o, ref, rtol=1e-11, atol=1e-11)
+    o, _ = one(oracle_mod, q, k, v, np.zeros_like(q))
+    np.testing.assert_allclose(o, ref, rtol=1e-11, atol=1e-11)
+
+
+def test_constant_scalar_gate_is_retnet(oracle_mod):
+    """A data-independent scalar decay gamma gives (Q K^T . D) V with
+    D[t,n] = gamma^(t-n)."""
+    q, k, v, _ = rand_head(50, 6, 4)
+    gamma = 0.93
+    la = np.full((50,), np.log(gamma))
+    o, _ = one(oracle_mod, q, k, v, la, gate="scalar")
+    np.testing.assert_allclose(o, forms.retnet_form(q, k, v, gamma), rtol=1e-11, atol=1e-11)
+
+
+def test_scalar_mode_equals_broadcast_vector(oracle_mod):
+    q, k, v, _ = rand_head(33, 5, 3)
+    las = RNG.standard_normal(33) * 0.1 - 0.05
+    o1, h1 = one(oracle_mod, q, k, v, las, gate="scalar")
+    o2, h2 = one(oracle_mod, q, k, v, np.repeat(las[:, None], 5, axis=1))
+    np.testing.assert_allclose(o1, o2, rtol=1e-13, atol=1e-13)
+    np.testing.assert_allclose(h1, h2, rtol=1e-13, atol=1e-13)
+
+
+def test_segment_concatenation(oracle_mod):
+    """h0 carries 'the previous segment's state' (section 2.2): running
+    [0,T1) then [T1,T) from its final state equals one run."""
+    q, k, v, la = rand_head(90, 7, 5)
+    o, hT = one(oracle_mod, q, k, v, la)
+    oa, ha = one(oracle_mod, q[:41], k[:41], v[:41], la[:41])
+    ob, hb = one(oracle_mod, q[41:], k[41:], v[41:], la[41:], h0=ha)
+    np.testing.assert_allclose(np.concatenate([oa, ob]), o, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(hb, hT, rtol=1e-12, atol=1e-12)
+
+
+def test_linearity_in_v_and_h0(oracle_mod):
+    q, k, v, la = rand_head(30, 4, 6)
+    v2 = RNG.standard_normal(v.shape)
+    h0 = RNG.standard_normal((4, 6))
+    h1 = RNG.standard_normal((4, 6))
+    a, b = 0.7, -1.3
+    o_ab, _ = one(oracle_mod, q, k, a * v + b * v2, la, a * h0 + b * h1)
+    o_a, _ = one(oracle_mod, q, k, v, la, h0)
+    o_b, _ = one(oracle_mod, q, k, v2, la, h1)
+    np.testing.assert_allclose(o_ab, a * o_a + b * o_b, rtol=1e-12, atol=1e-12)
+
+
+def test_golden_hand_computed(oracle_mod):
+    """Values worked out by hand from the recurrence (tests/golden/*.json)."""
+    gdir = os.path.join(os.path.dirname(__file__), "golden")
+    files = sorted(f for f in os.listdir(gdir) if f.startswith("hand_") and f.endswith(".json"))
+    assert files
+    for f in files:
+        case = json.load(open(os.path.join(gdir, f)))
+        q = np.array(case["q"], float)
+        k = np.array(case["k"], float)
+        v = np.array(case["v"], float)
+        la = np.log(np.array(case["alpha"], float))
+        h0 = None if case.get("h0") is None else np.array(case["h0"], float)
+        o, hT = one(oracle_mod, q, k, v, la, h0)
+        np.testing.assert_allclose(o, np.array(case["o"], float), rtol=0, atol=1e-12)
+        np.testing.assert_allclose(hT, np.array(case["h_final"], float), rtol=0, atol=1e-12)
+
+
+# --------------------------------------------------------------- backward pins
+
+def loss_of(oracle, q, k, v, la, h0, do, dhT, gate):
+    o, hT = oracle.fwd(q, k, v, la, h0=h0, gate=gate)
+    return float(np.sum(o * do) + np.sum(hT * dhT))
+
+
+@pytest.mark.parametrize("gate", ["vector", "scalar", "none"])
+def test_finite_differences(oracle_mod, gate):
+    """Central differences (step 1e-6, float64) of L = <o,do> + <h_T,dh_T>
+    against the BPTT gradients for every input."""
+    rng = np.random.default_rng(7)
+    B, H, T, K, V = 1, 2, 11, 3, 4
+    q = rng.standard_normal((B, H, T, K))
+    k = rng.standard_normal((B, H, T, K)) / np.sqrt(K)
+    v = rng.standard_normal((B, H, T, V))
+    if gate == "vector":
+        la = -np.abs(rng.standard_normal((B, H, T, K))) * 0.3
+    elif gate == "scalar":
+        la = -np.abs(rng.standard_normal((B, H, T))) * 0.3
+    else:
+        la = None
+    h0 = rng.standard_normal((B, H, K, V))
+    do = rng.standard_normal((B, H, T, V))
+    dhT = rng.standard_normal((B, H, K, V))
+    dq, dk, dv, dla, dh0 = oracle_mod.bwd(q, k, v, la, do, h0=h0, dh_final=dhT, gate=gate)
+    eps = 1e-6
+    named = {"q": (q, dq), "k": (k, dk), "v": (v, dv), "h0": (h0, dh0)}
+    if la is not None:
+        named["la"] = (la, dla)
+    for name, (x, g) in named.items():
+        flat = x.reshape(-1)
+        gflat = g.reshape(-1)
+        idx = rng.choice(flat.size, size=min(flat.size, 25), replace=False)
+        for i in idx:
+            old = flat[i]
+            flat[i] = old + eps
+            lp = loss_of(oracle_mod, q, k, v, la, h0, do, dhT, gate)
+            flat[i] = old - eps
+            lm = loss_of(oracle_mod, q, k, v, la, h0, do, dhT, gate)
+            flat[i] = old
+            fd = (lp - lm) / (2 * eps)
+            assert abs(fd - gflat[i]) <= 1e-6 * max(1.0, abs(fd)), (name, i, fd, gflat[i])
+
+
+@pytest.mark.parametrize("with_final", [False, True])
+def test_closed_form_gate_gradient(oracle_mod, with_final):
+    """The paper's closed form (section 4.3 / Appendix B): dlog b_t =
+    q_t.dq_t - k_t.dk_t and dlog alpha_t = sum_{i>=t} dlog b_i, with the extra
+    final-state term sum_j h_T[c,j] dh_T[c,j] when dh_T != 0 (derived from the
+    same recurrence), equals back-propagation through the token loop."""
+    rng = np.random.default_rng(11)
+    B, H, T, K, V = 2, 1, 70, 5, 6
+    q = rng.standard_normal((B, H, T, K))
+    k = rng.standard_normal((B, H, T, K)) / np.sqrt(K)
+    v = rng.standard_normal((B, H, T, V))
+    la = np.log(1 / (1 + np.exp(-rng.standard_normal((B, H, T, K))))) / 16
+    h0 = rng.standard_normal((B, H, K, V))
+    do = rng.standard_normal((B, H, T, V))
+    dhT = rng.standard_normal((B, H, K, V)) if with_final else None
+    dq, dk, dv, dla, dh0 = oracle_mod.bwd(q, k, v, la, do, h0=h0, dh_final=dhT)
+    dlogb = q * dq - k * dk
+    if with_final:
+        _, hT = oracle_mod.fwd(q, k, v, la, h0=h0)
+        dlogb[:, :, -1, :] += np.sum(hT * dhT, axis=-1)
+    closed = np.flip(np.cumsum(np.flip(dlogb, axis=2), axis=2), axis=2)
+    np.testing.assert_allclose(dla, closed, rtol=1e-10, atol=1e-10)
+
+
+def test_scalar_gate_gradient_sums_channels(oracle_mod):
+    rng = np.random.default_rng(3)
+    B, H, T, K, V = 1, 1, 20, 4, 3
+    q = rng.standard_normal((B, H, T, K))
+    k = rng.standard_normal((B, H, T, K))
+    v = rng.standard_normal((B, H, T, V))
+    las = -np.abs(rng.standard_normal((B, H, T))) * 0.2
+    do = rng.standard_normal((B, H, T, V))
+    _, _, _, dla_s, _ = oracle_mod.bwd(q, k, v, las, do, gate="scalar")
+    _, _, _, dla_v, _ = oracle_mod.bwd(q, k, v, np.repeat(las[..., None], K, -1), do, gate="vector")
+    np.testing.assert_allclose(dla_s, dla_v.sum(-1), rtol=1e-12, atol=1e-12)
+
+
+# ------------------------------------------------------ planted mistakes (CPU)
+
+def _pins_pass(orc):
+    """A compact run of the pins above against an oracle-like object."""
+    try:
+        test_brute_force_tiny(orc, 8, 4, 4)
+        test_chunkwise_any_tiling(orc, 100, 32, 8)
+        for gate in ("vector", "scalar"):
+            test_finite_differences(orc, gate)
+        test_closed_form_gate_gradient(orc, True)
+    except AssertionError:
+        return False
+    return True
+
+
+def test_pins_pass_on_oracle(oracle_mod):
+    assert _pins_pass(oracle_mod)
+
+
+@pytest.mark.parametrize("mutant", [1, 2, 3, 4])
+def test_pins_catch_planted_mistakes(mutant):
+    from oracle.oracle import Mutant
+    assert not _pins_pass(Mutant(mutant))
