@@ -1,0 +1,364 @@
+// f32_path.cu -- fp32 CUDA-core implementation of chunkwise GLA (forward + backward).
+//
+// This is the library's path for fp32 inputs.  It follows the chunkwise form of
+// "Gated Linear Attention Transformers with Hardware-Efficient Training",
+// section 4.2, with every chunk-level state materialised (section 3.3,
+// Figure 1b-c) and the intra-chunk scores formed pair by pair in log space
+// (exp(B_t - B_s) with B the chunk-local cumulative log-gate, s <= t), so it is
+// stable for any gate strength.  All arithmetic is fp32 on CUDA cores.
+//
+// Kernels (grid-parallel over heads and chunks except the two state walks,
+// which are parallel over heads and state elements and sequential over chunks):
+//   prep     B[t,c]   chunk-local inclusive cumsum of log_alpha
+//   states   H[n]     state before chunk n (H[N] = final state)
+//   scores   P[n]     C x C causal intra-chunk scores
+//   out      o        (q (.) e^B) H[n] + P V
+//   dstates  dH[n]    adjoint of the state after chunk n
+//   dscores  dP[n]    dO V^T (causal part)
+//   dqk      dq, dk, dlog_alpha (closed form, section 4.3, with the chunk
+//            boundary term sum_v S_n[c,v] dS_n[c,v])
+//   dv       dv
+#include <cuda_bf16.h>
+
+#include "internal.h"
+
+namespace gla {
+namespace {
+
+template <typename T>
+__device__ __forceinline__ float ld(const T *p);
+template <>
+__device__ __forceinline__ float ld<float>(const float *p) { return *p; }
+template <>
+__device__ __forceinline__ float ld<__nv_bfloat16>(const __nv_bfloat16 *p) { return __bfloat162float(*p); }
+
+template <typename T>
+__device__ __forceinline__ void st(T *p, float x);
+template <>
+__device__ __forceinline__ void st<float>(float *p, float x) { *p = x; }
+template <>
+__device__ __forceinline__ void st<__nv_bfloat16>(__nv_bfloat16 *p, float x) { *p = __float2bfloat16_rn(x); }
+
+struct Dims {
+  int T, K, V, C, N, gate;
+  long Tp;
+};
+
+// ---------------------------------------------------------------- forward
+
+// Bc[bh, t, c] = sum_{j in chunk(t), j <= t} log_alpha[bh, j, c]; rows t >= T add 0.
+__global__ void k_prep(const float *__restrict__ la, Dims d, float *__restrict__ Bc) {
+  const int c = threadIdx.x;
+  if (c >= d.K) return;
+  const long bh = blockIdx.y;
+  const int n = blockIdx.x;
+  float acc = 0.f;
+  for (int j = 0; j < d.C; ++j) {
+    const long t = (long)n * d.C + j;
+    float g = 0.f;
+    if (t < d.T) {
+      if (d.gate == GLA_GATE_VECTOR) g = la[(bh * d.T + t) * d.K + c];
+      else if (d.gate == GLA_GATE_SCALAR) g = la[bh * d.T + t];
+    }
+    acc += g;
+    Bc[(bh * d.Tp + t) * d.K + c] = acc;
+  }
+}
+
+// H[bh, n] = state before chunk n; H[bh, N] = final state.  Thread = (c, v).
+template <typename T>
+__global__ void k_states(const T *__restrict__ k, const T *__restrict__ v, const float *__restrict__ Bc,
+                         const float *__restrict__ h0, Dims d, float *__restrict__ Hs,
+                         float *__restrict__ hT) {
+  const int vi = blockIdx.x * blockDim.x + threadIdx.x;
+  const int c = blockIdx.y * blockDim.y + threadIdx.y;
+  const long bh = blockIdx.z;
+  if (vi >= d.V || c >= d.K) return;
+  const long KV = (long)d.K * d.V;
+  float S = h0 ? h0[bh * KV + (long)c * d.V + vi] : 0.f;
+  for (int n = 0; n < d.N; ++n) {
+    Hs[(bh * (d.N + 1) + n) * KV + (long)c * d.V + vi] = S;
+    const float blast = Bc[(bh * d.Tp + (long)n * d.C + d.C - 1) * d.K + c];
+    float acc = 0.f;
+    for (int j = 0; j < d.C; ++j) {
+      const long t = (long)n * d.C + j;
+      if (t >= d.T) break;
+      const float kk = ld(k + (bh * d.T + t) * d.K + c);
+      const float w = __expf(blast - Bc[(bh * d.Tp + t) * d.K + c]);
+      acc += kk * w * ld(v + (bh * d.T + t) * d.V + vi);
+    }
+    S = __expf(blast) * S + acc;
+  }
+  Hs[(bh * (d.N + 1) + d.N) * KV + (long)c * d.V + vi] = S;
+  if (hT) hT[bh * KV + (long)c * d.V + vi] = S;
+}
+
+// P[bh, n, t, s] = sum_c q_t[c] k_s[c] exp(B_t[c] - B_s[c]) for s <= t, else 0.
+template <typename T>
+__global__ void k_scores(const T *__restrict__ q, const T *__restrict__ k, const float *__restrict__ Bc,
+                         Dims d, float *__restrict__ P) {
+  const long bh = blockIdx.y;
+  const int n = blockIdx.x;
+  for (int idx = threadIdx.x; idx < d.C * d.C; idx += blockDim.x) {
+    const int ti = idx / d.C, si = idx % d.C;
+    const long t = (long)n * d.C + ti, s = (long)n * d.C + si;
+    float acc = 0.f;
+    if (si <= ti && t < d.T) {
+      for (int c = 0; c < d.K; ++c) {
+        const float e = __expf(Bc[(bh * d.Tp + t) * d.K + c] - Bc[(bh * d.Tp + s) * d.K + c]);
+        acc += ld(q + (bh * d.T + t) * d.K + c) * ld(k + (bh * d.T + s) * d.K + c) * e;
+      }
+    }
+    P[((bh * d.N + n) * d.C + ti) * d.C + si] = acc;
+  }
+}
+
+// o[t, v] = sum_c q_t[c] e^{B_t[c]} H[n][c, v] + sum_{s<=t} P[t, s] v_s[v]
+template <typename T>
+__global__ void k_out(const T *__restrict__ q, const T *__restrict__ v, const float *__restrict__ Bc,
+                      const float *__restrict__ Hs, const float *__restrict__ P, Dims d, T *__restrict__ o) {
+  const int vi = blockIdx.x * blockDim.x + threadIdx.x;
+  const int n = blockIdx.y;
+  const long bh = blockIdx.z;
+  if (vi >= d.V) return;
+  const long KV = (long)d.K * d.V;
+  const float *H = Hs + (bh * (d.N + 1) + n) * KV;
+  for (int ti = threadIdx.y; ti < d.C; ti += blockDim.y) {
+    const long t = (long)n * d.C + ti;
+    if (t >= d.T) break;
+    float acc = 0.f;
+    for (int c = 0; c < d.K; ++c)
+      acc += ld(q + (bh * d.T + t) * d.K + c) * __expf(Bc[(bh * d.Tp + t) * d.K + c]) * H[(long)c * d.V + vi];
+    const float *Pr = P + ((bh * d.N + n) * d.C + ti) * d.C;
+    for (int si = 0; si <= ti; ++si) acc += Pr[si] * ld(v + (bh * d.T + (long)n * d.C + si) * d.V + vi);
+    st(o + (bh * d.T + t) * d.V + vi, acc);
+  }
+}
+
+// ---------------------------------------------------------------- backward
+
+// dH[bh, n] = adjoint of the state after chunk n (through chunks > n and dh_final).
+template <typename T>
+__global__ void k_dstates(const T *__restrict__ q, const T *__restrict__ dout, const float *__restrict__ Bc,
+                          const float *__restrict__ dhT, Dims d, float *__restrict__ dHs,
+                          float *__restrict__ dh0) {
+  const int vi = blockIdx.x * blockDim.x + threadIdx.x;
+  const int c = blockIdx.y * blockDim.y + threadIdx.y;
+  const long bh = blockIdx.z;
+  if (vi >= d.V || c >= d.K) return;
+  const long KV = (long)d.K * d.V;
+  float dS = dhT ? dhT[bh * KV + (long)c * d.V + vi] : 0.f;
+  for (int n = d.N - 1; n >= 0; --n) {
+    dHs[(bh * d.N + n) * KV + (long)c * d.V + vi] = dS;
+    const float blast = Bc[(bh * d.Tp + (long)n * d.C + d.C - 1) * d.K + c];
+    float acc = 0.f;
+    for (int j = 0; j < d.C; ++j) {
+      const long t = (long)n * d.C + j;
+      if (t >= d.T) break;
+      acc += ld(q + (bh * d.T + t) * d.K + c) * __expf(Bc[(bh * d.Tp + t) * d.K + c]) *
+             ld(dout + (bh * d.T + t) * d.V + vi);
+    }
+    dS = __expf(blast) * dS + acc;
+  }
+  if (dh0) dh0[bh * KV + (long)c * d.V + vi] = dS;
+}
+
+// dP[bh, n, t, s] = sum_v do_t[v] v_s[v] for s <= t, else 0.
+template <typename T>
+__global__ void k_dscores(const T *__restrict__ dout, const T *__restrict__ v, Dims d, float *__restrict__ dP) {
+  const long bh = blockIdx.y;
+  const int n = blockIdx.x;
+  for (int idx = threadIdx.x; idx < d.C * d.C; idx += blockDim.x) {
+    const int ti = idx / d.C, si = idx % d.C;
+    const long t = (long)n * d.C + ti, s = (long)n * d.C + si;
+    float acc = 0.f;
+    if (si <= ti && t < d.T)
+      for (int j = 0; j < d.V; ++j) acc += ld(dout + (bh * d.T + t) * d.V + j) * ld(v + (bh * d.T + s) * d.V + j);
+    dP[((bh * d.N + n) * d.C + ti) * d.C + si] = acc;
+  }
+}
+
+// One block per (chunk, head), one thread per key channel c:
+//   dq_t = e^{B_t} (do_t H[n]^T) + sum_{s<=t} dP[t,s] k_s e^{B_t - B_s}
+//   dk_t = e^{B_last - B_t} (v_t dH[n]^T) + sum_{s>=t} dP[s,t] q_s e^{B_s - B_t}
+//   dlog b_t = q_t dq_t - k_t dk_t   (closed form, section 4.3)
+//   dlog alpha_t = sum_{i >= t in chunk} dlog b_i + G_n,  G_n[c] = sum_v S_n[c,v] dS_n[c,v]
+// (S_n = H[n+1] the state after chunk n, dS_n = dH[n] its adjoint), which is the
+// suffix of dlog b beyond the chunk, so no cross-chunk scan is needed.
+template <typename T>
+__global__ void k_dqk(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
+                      const T *__restrict__ dout, const float *__restrict__ Bc, const float *__restrict__ Hs,
+                      const float *__restrict__ dHs, const float *__restrict__ dP, Dims d, T *__restrict__ dq,
+                      T *__restrict__ dk, float *__restrict__ dgv) {
+  const int c = threadIdx.x;
+  if (c >= d.K) return;
+  const long bh = blockIdx.y;
+  const int n = blockIdx.x;
+  const long KV = (long)d.K * d.V;
+  const float *H = Hs + (bh * (d.N + 1) + n) * KV + (long)c * d.V;
+  const float *Hn = Hs + (bh * (d.N + 1) + n + 1) * KV + (long)c * d.V;
+  const float *dH = dHs + (bh * d.N + n) * KV + (long)c * d.V;
+  const float *dPc = dP + (bh * d.N + n) * (long)d.C * d.C;
+  const float blast = Bc[(bh * d.Tp + (long)n * d.C + d.C - 1) * d.K + c];
+  float G = 0.f;
+  for (int j = 0; j < d.V; ++j) G += Hn[j] * dH[j];
+  // pass 1: dlog b per token into dgv, dq and dk stored
+  for (int ti = 0; ti < d.C; ++ti) {
+    const long t = (long)n * d.C + ti;
+    if (t >= d.T) break;
+    const float Bt = Bc[(bh * d.Tp + t) * d.K + c];
+    float a1 = 0.f, a2 = 0.f;
+    for (int j = 0; j < d.V; ++j) {
+      a1 += ld(dout + (bh * d.T + t) * d.V + j) * H[j];
+      a2 += ld(v + (bh * d.T + t) * d.V + j) * dH[j];
+    }
+    float dqv = __expf(Bt) * a1;
+    float dkv = __expf(blast - Bt) * a2;
+    for (int si = 0; si <= ti; ++si) {
+      const long s = (long)n * d.C + si;
+      dqv += dPc[ti * d.C + si] * ld(k + (bh * d.T + s) * d.K + c) * __expf(Bt - Bc[(bh * d.Tp + s) * d.K + c]);
+    }
+    for (int si = ti; si < d.C; ++si) {
+      const long s = (long)n * d.C + si;
+      if (s >= d.T) break;
+      dkv += dPc[si * d.C + ti] * ld(q + (bh * d.T + s) * d.K + c) * __expf(Bc[(bh * d.Tp + s) * d.K + c] - Bt);
+    }
+    st(dq + (bh * d.T + t) * d.K + c, dqv);
+    st(dk + (bh * d.T + t) * d.K + c, dkv);
+    dgv[(bh * d.Tp + t) * d.K + c] = ld(q + (bh * d.T + t) * d.K + c) * dqv - ld(k + (bh * d.T + t) * d.K + c) * dkv;
+  }
+  // pass 2: reverse cumulative sum within the chunk plus the boundary term
+  float run = G;
+  for (int ti = d.C - 1; ti >= 0; --ti) {
+    const long t = (long)n * d.C + ti;
+    if (t >= d.T) continue;
+    run += dgv[(bh * d.Tp + t) * d.K + c];
+    dgv[(bh * d.Tp + t) * d.K + c] = run;
+  }
+}
+
+// dv_t = (k_t (.) e^{B_last - B_t}) dH[n] + sum_{s>=t} P[s,t] do_s
+template <typename T>
+__global__ void k_dv(const T *__restrict__ k, const T *__restrict__ dout, const float *__restrict__ Bc,
+                     const float *__restrict__ dHs, const float *__restrict__ P, Dims d, T *__restrict__ dv) {
+  const int vi = blockIdx.x * blockDim.x + threadIdx.x;
+  const int n = blockIdx.y;
+  const long bh = blockIdx.z;
+  if (vi >= d.V) return;
+  const long KV = (long)d.K * d.V;
+  const float *dH = dHs + (bh * d.N + n) * KV;
+  const float *Pc = P + (bh * d.N + n) * (long)d.C * d.C;
+  for (int ti = threadIdx.y; ti < d.C; ti += blockDim.y) {
+    const long t = (long)n * d.C + ti;
+    if (t >= d.T) break;
+    float acc = 0.f;
+    for (int c = 0; c < d.K; ++c) {
+      const float blast = Bc[(bh * d.Tp + (long)n * d.C + d.C - 1) * d.K + c];
+      acc += ld(k + (bh * d.T + t) * d.K + c) * __expf(blast - Bc[(bh * d.Tp + t) * d.K + c]) * dH[(long)c * d.V + vi];
+    }
+    for (int si = ti; si < d.C; ++si) {
+      const long s = (long)n * d.C + si;
+      if (s >= d.T) break;
+      acc += Pc[si * d.C + ti] * ld(dout + (bh * d.T + s) * d.V + vi);
+    }
+    st(dv + (bh * d.T + t) * d.V + vi, acc);
+  }
+}
+
+// Copy (vector gate) or channel-sum (scalar gate) the per-channel gate gradient.
+__global__ void k_dg_out(const float *__restrict__ dgv, Dims d, float *__restrict__ dla) {
+  const long bh = blockIdx.y;
+  const long t = (long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (t >= d.T) return;
+  if (d.gate == GLA_GATE_VECTOR) {
+    for (int c = 0; c < d.K; ++c) dla[(bh * d.T + t) * d.K + c] = dgv[(bh * d.Tp + t) * d.K + c];
+  } else {
+    float s = 0.f;
+    for (int c = 0; c < d.K; ++c) s += dgv[(bh * d.Tp + t) * d.K + c];
+    dla[bh * d.T + t] = s;
+  }
+}
+
+Dims dims_of(const Problem &p) { return Dims{p.T, p.K, p.V, p.C, p.N, p.gate, p.Tp}; }
+
+struct F32Ws {
+  float *Bc, *Hs, *P, *dHs, *dP, *dgv;
+  size_t bytes;
+};
+
+F32Ws carve(const Problem &p, void *ws, bool bwd) {
+  Carve cv(ws);
+  F32Ws w{};
+  w.Bc = cv.take<float>((size_t)p.BH * p.Tp * p.K);
+  w.Hs = cv.take<float>((size_t)p.BH * (p.N + 1) * p.K * p.V);
+  w.P = cv.take<float>((size_t)p.BH * p.N * p.C * p.C);
+  if (bwd) {
+    w.dHs = cv.take<float>((size_t)p.BH * p.N * p.K * p.V);
+    w.dP = cv.take<float>((size_t)p.BH * p.N * p.C * p.C);
+    w.dgv = cv.take<float>((size_t)p.BH * p.Tp * p.K);
+  }
+  w.bytes = cv.bytes();
+  return w;
+}
+
+template <typename T>
+int fwd_impl(const Problem &p, const T *q, const T *k, const T *v, const float *la, const float *h0, T *o,
+             float *hT, void *ws, cudaStream_t st) {
+  const Dims d = dims_of(p);
+  F32Ws w = carve(p, ws, false);
+  const int kth = (p.K + 31) / 32 * 32;
+  GLA_LAUNCH(K_F32_PREP, st, (k_prep<<<dim3(p.N, p.BH), kth, 0, st>>>(la, d, w.Bc)));
+  GLA_LAUNCH(K_F32_STATES, st,
+             (k_states<T><<<dim3((p.V + 31) / 32, (p.K + 7) / 8, p.BH), dim3(32, 8), 0, st>>>(k, v, w.Bc, h0, d, w.Hs, hT)));
+  GLA_LAUNCH(K_F32_SCORES, st, (k_scores<T><<<dim3(p.N, p.BH), 256, 0, st>>>(q, k, w.Bc, d, w.P)));
+  GLA_LAUNCH(K_F32_OUT, st,
+             (k_out<T><<<dim3((p.V + 63) / 64, p.N, p.BH), dim3(64, 4), 0, st>>>(q, v, w.Bc, w.Hs, w.P, d, o)));
+  return GLA_OK;
+}
+
+template <typename T>
+int bwd_impl(const Problem &p, const T *q, const T *k, const T *v, const float *la, const float *h0, const T *dout,
+             const float *dhT, T *dq, T *dk, T *dv, float *dla, float *dh0, void *ws, cudaStream_t st) {
+  const Dims d = dims_of(p);
+  F32Ws w = carve(p, ws, true);
+  const int kth = (p.K + 31) / 32 * 32;
+  GLA_LAUNCH(K_F32_PREP, st, (k_prep<<<dim3(p.N, p.BH), kth, 0, st>>>(la, d, w.Bc)));
+  GLA_LAUNCH(K_F32_STATES, st,
+             (k_states<T><<<dim3((p.V + 31) / 32, (p.K + 7) / 8, p.BH), dim3(32, 8), 0, st>>>(k, v, w.Bc, h0, d, w.Hs, nullptr)));
+  GLA_LAUNCH(K_F32_SCORES, st, (k_scores<T><<<dim3(p.N, p.BH), 256, 0, st>>>(q, k, w.Bc, d, w.P)));
+  GLA_LAUNCH(K_F32_DSTATES, st,
+             (k_dstates<T><<<dim3((p.V + 31) / 32, (p.K + 7) / 8, p.BH), dim3(32, 8), 0, st>>>(q, dout, w.Bc, dhT, d, w.dHs, dh0)));
+  GLA_LAUNCH(K_F32_DSCORES, st, (k_dscores<T><<<dim3(p.N, p.BH), 256, 0, st>>>(dout, v, d, w.dP)));
+  GLA_LAUNCH(K_F32_DQK, st,
+             (k_dqk<T><<<dim3(p.N, p.BH), kth, 0, st>>>(q, k, v, dout, w.Bc, w.Hs, w.dHs, w.dP, d, dq, dk, w.dgv)));
+  GLA_LAUNCH(K_F32_DV, st,
+             (k_dv<T><<<dim3((p.V + 63) / 64, p.N, p.BH), dim3(64, 4), 0, st>>>(k, dout, w.Bc, w.dHs, w.P, d, dv)));
+  if (p.gate != GLA_GATE_NONE)
+    GLA_LAUNCH(K_F32_DG_SCALAR, st, (k_dg_out<<<dim3((p.T + 127) / 128, p.BH), 128, 0, st>>>(w.dgv, d, dla)));
+  return GLA_OK;
+}
+
+}  // namespace
+
+size_t f32_workspace(const Problem &p, bool bwd) { return carve(p, nullptr, bwd).bytes; }
+
+int f32_fwd(const Problem &p, const void *q, const void *k, const void *v, const float *la, const float *h0, void *o,
+            float *hT, void *ws, cudaStream_t st) {
+  if (p.dtype == GLA_DTYPE_FP32)
+    return fwd_impl<float>(p, (const float *)q, (const float *)k, (const float *)v, la, h0, (float *)o, hT, ws, st);
+  return fwd_impl<__nv_bfloat16>(p, (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v, la,
+                                 h0, (__nv_bfloat16 *)o, hT, ws, st);
+}
+
+int f32_bwd(const Problem &p, const void *q, const void *k, const void *v, const float *la, const float *h0,
+            const void *dout, const float *dhT, void *dq, void *dk, void *dv, float *dla, float *dh0, void *ws,
+            cudaStream_t st) {
+  if (p.dtype == GLA_DTYPE_FP32)
+    return bwd_impl<float>(p, (const float *)q, (const float *)k, (const float *)v, la, h0, (const float *)dout, dhT,
+                           (float *)dq, (float *)dk, (float *)dv, dla, dh0, ws, st);
+  using bf = __nv_bfloat16;
+  return bwd_impl<bf>(p, (const bf *)q, (const bf *)k, (const bf *)v, la, h0, (const bf *)dout, dhT, (bf *)dq,
+                      (bf *)dk, (bf *)dv, dla, dh0, ws, st);
+}
+
+}  // namespace gla

@@ -1,0 +1,13 @@
+// tc_path.h -- bf16 tensor-core (tcgen05 / TMEM / TMA) path, sm_100a.
+#pragma once
+#include "internal.h"
+
+namespace gla {
+int tc_check(const Problem &p);
+size_t tc_workspace(const Problem &p, bool bwd);
+int tc_fwd(const Problem &p, const void *q, const void *k, const void *v, const float *la, const float *h0,
+           void *o, float *hT, void *ws, cudaStream_t st);
+int tc_bwd(const Problem &p, const void *q, const void *k, const void *v, const float *la, const float *h0,
+           const void *dout, const float *dhT, void *dq, void *dk, void *dv, float *dla, float *dh0, void *ws,
+           cudaStream_t st);
+}  // namespace gla

@@ -1,0 +1,207 @@
+"""Thin Python binding of the C ABI in include/gla.h (ctypes; argument marshalling only).
+
+Every step of the computation runs in the CUDA library ``libgla_b200.so`` built
+in-tree from ``csrc/``.  There is no fallback: if the library is missing or a
+call fails, an exception is raised.  PyTorch is used only to own device memory
+(inputs, outputs and the workspace) and to name the CUDA stream.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libgla_b200.so")
+
+GLA_OK = 0
+STATUS = {
+    0: "GLA_OK", -1: "GLA_ERR_INVALID_ARG", -2: "GLA_ERR_UNSUPPORTED_SHAPE", -3: "GLA_ERR_MISALIGNED",
+    -4: "GLA_ERR_WORKSPACE_TOO_SMALL", -5: "GLA_ERR_CUDA", -6: "GLA_ERR_TIMEOUT", -7: "GLA_ERR_GATE_RANGE",
+    -8: "GLA_ERR_NO_DEVICE",
+}
+DTYPE = {torch.bfloat16: 0, torch.float32: 1}
+GATE = {"vector": 0, "scalar": 1, "none": 2}
+VARIANT = {"auto": 0, "fused": 1, "materialized": 2}
+
+# Every exported symbol of include/gla.h.
+EXPORTS = ["gla_workspace_size", "gla_check", "gla_fwd", "gla_bwd", "gla_poll_status", "gla_status_string",
+           "gla_timing_enable", "gla_timing_collect", "gla_kernel_name", "gla_build_info"]
+
+
+class GLAError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where} failed: {STATUS.get(code, code)} ({status_string(code)})")
+
+
+class gla_desc(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("T", ctypes.c_int), ("dk", ctypes.c_int),
+                ("dv", ctypes.c_int), ("dtype", ctypes.c_int), ("gate", ctypes.c_int), ("subchunk", ctypes.c_int),
+                ("variant", ctypes.c_int), ("segments", ctypes.c_int), ("workspace", ctypes.c_void_p),
+                ("workspace_bytes", ctypes.c_size_t)]
+
+
+_lib = None
+
+
+def load(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libgla_b200.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"CUDA library not built: {path} (run chunkwise_linear_rnn_fwd_b200/build.py)")
+    lib = ctypes.CDLL(path)
+    vp, i, dp = ctypes.c_void_p, ctypes.c_int, ctypes.POINTER(gla_desc)
+    lib.gla_workspace_size.argtypes = [dp, i, i]
+    lib.gla_workspace_size.restype = ctypes.c_size_t
+    lib.gla_check.argtypes = [dp, i]
+    lib.gla_check.restype = i
+    lib.gla_fwd.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, i, vp]
+    lib.gla_fwd.restype = i
+    lib.gla_bwd.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, vp]
+    lib.gla_bwd.restype = i
+    lib.gla_poll_status.argtypes = [dp, vp]
+    lib.gla_poll_status.restype = i
+    lib.gla_status_string.argtypes = [i]
+    lib.gla_status_string.restype = ctypes.c_char_p
+    lib.gla_timing_enable.argtypes = [i]
+    lib.gla_timing_enable.restype = i
+    lib.gla_timing_collect.argtypes = [i, ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_float)]
+    lib.gla_timing_collect.restype = i
+    lib.gla_kernel_name.argtypes = [i]
+    lib.gla_kernel_name.restype = ctypes.c_char_p
+    lib.gla_build_info.argtypes = []
+    lib.gla_build_info.restype = ctypes.c_char_p
+    _lib = lib
+    return lib
+
+
+def status_string(code: int) -> str:
+    return load().gla_status_string(int(code)).decode()
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError("tensors passed to the GLA library must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_handle(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(int(stream.cuda_stream))
+
+
+def _gate_of(log_alpha, gate):
+    if gate is not None:
+        return gate
+    if log_alpha is None:
+        return "none"
+    return "vector" if log_alpha.dim() == 4 else "scalar"
+
+
+def make_desc(B, H, T, dk, dv, dtype, gate, *, subchunk=16, variant="auto", segments=0,
+              workspace: Optional[torch.Tensor] = None) -> gla_desc:
+    d = gla_desc()
+    d.B, d.H, d.T, d.dk, d.dv = int(B), int(H), int(T), int(dk), int(dv)
+    d.dtype = DTYPE[dtype] if isinstance(dtype, torch.dtype) else int(dtype)
+    d.gate = GATE[gate] if isinstance(gate, str) else int(gate)
+    d.subchunk = int(subchunk)
+    d.variant = VARIANT[variant] if isinstance(variant, str) else int(variant)
+    d.segments = int(segments)
+    if workspace is not None:
+        d.workspace = workspace.data_ptr()
+        d.workspace_bytes = workspace.numel() * workspace.element_size()
+    return d
+
+
+def workspace_size(B, H, T, dk, dv, dtype, gate, chunk=64, for_bwd=False, **kw) -> int:
+    d = make_desc(B, H, T, dk, dv, dtype, gate, **kw)
+    n = load().gla_workspace_size(ctypes.byref(d), int(chunk), int(bool(for_bwd)))
+    if n == 0:
+        raise GLAError(load().gla_check(ctypes.byref(d), int(chunk)), "gla_workspace_size")
+    return int(n)
+
+
+def alloc_workspace(nbytes: int, device) -> torch.Tensor:
+    """A caller-owned workspace (PyTorch memory, 256-byte aligned by the allocator)."""
+    return torch.empty(int(nbytes), dtype=torch.uint8, device=device)
+
+
+def gla_fwd(q, k, v, log_alpha=None, h0=None, *, chunk=64, gate=None, subchunk=16, variant="auto", segments=0,
+            o=None, h_final=None, want_final=True, workspace=None, stream=None):
+    """Forward.  Returns (o, h_final or None).  See include/gla.h."""
+    lib = load()
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    gate = _gate_of(log_alpha, gate)
+    if o is None:
+        o = torch.empty(B, H, T, dv, dtype=q.dtype, device=q.device)
+    if h_final is None and want_final:
+        h_final = torch.empty(B, H, dk, dv, dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = alloc_workspace(workspace_size(B, H, T, dk, dv, q.dtype, gate, chunk, False, subchunk=subchunk,
+                                                   variant=variant, segments=segments), q.device)
+    d = make_desc(B, H, T, dk, dv, q.dtype, gate, subchunk=subchunk, variant=variant, segments=segments,
+                  workspace=workspace)
+    r = lib.gla_fwd(ctypes.byref(d), _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(h0), _ptr(o), _ptr(h_final),
+                    int(chunk), _stream_handle(stream))
+    if r != GLA_OK:
+        raise GLAError(r, "gla_fwd")
+    return o, h_final
+
+
+def gla_bwd(q, k, v, log_alpha, do, h0=None, dh_final=None, *, chunk=64, gate=None, subchunk=16, dq=None, dk=None,
+            dv=None, dlog_alpha=None, dh0=None, want_dh0=True, workspace=None, stream=None):
+    """Backward.  Returns (dq, dk, dv, dlog_alpha or None, dh0 or None).  See include/gla.h."""
+    lib = load()
+    B, H, T, dk_ = q.shape
+    dv_ = v.shape[-1]
+    gate = _gate_of(log_alpha, gate)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    if dlog_alpha is None and gate != "none":
+        dlog_alpha = torch.empty_like(log_alpha)
+    if dh0 is None and want_dh0:
+        dh0 = torch.empty(B, H, dk_, dv_, dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = alloc_workspace(workspace_size(B, H, T, dk_, dv_, q.dtype, gate, chunk, True, subchunk=subchunk),
+                                    q.device)
+    d = make_desc(B, H, T, dk_, dv_, q.dtype, gate, subchunk=subchunk, workspace=workspace)
+    r = lib.gla_bwd(ctypes.byref(d), _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(h0), _ptr(do), _ptr(dh_final),
+                    _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dlog_alpha), _ptr(dh0), int(chunk), _stream_handle(stream))
+    if r != GLA_OK:
+        raise GLAError(r, "gla_bwd")
+    return dq, dk, dv, dlog_alpha, dh0
+
+
+def poll_status(workspace: torch.Tensor, stream=None) -> int:
+    """Synchronise and read/clear the device status word of a workspace (GLA_OK = 0)."""
+    d = gla_desc()
+    d.workspace = workspace.data_ptr()
+    d.workspace_bytes = workspace.numel()
+    return int(load().gla_poll_status(ctypes.byref(d), _stream_handle(stream)))
+
+
+def timing_enable(on: bool = True) -> None:
+    load().gla_timing_enable(int(bool(on)))
+
+
+def timing_collect(max_launches: int = 65536):
+    """[(kernel_name, ms), ...] for the launches recorded since the last collect."""
+    lib = load()
+    ids = (ctypes.c_int * max_launches)()
+    ms = (ctypes.c_float * max_launches)()
+    n = lib.gla_timing_collect(max_launches, ids, ms)
+    return [(lib.gla_kernel_name(ids[i]).decode(), float(ms[i])) for i in range(n)]
+
+
+def build_info() -> str:
+    return load().gla_build_info().decode()

@@ -1,0 +1,152 @@
+/*
+ * gla.h -- C ABI of the B200 (sm_100a) chunkwise Gated Linear Attention library.
+ *
+ * The operation is the GLA layer of "Gated Linear Attention Transformers with
+ * Hardware-Efficient Training" (Yang, Wang, Shen, Panda, Kim; arXiv:2312.06635),
+ * section 4.1: for every (batch b, head h) independently, with a d_k x d_v
+ * fp32 state S,
+ *
+ *     S_t = diag(alpha_t) S_{t-1} + k_t^T v_t ,     o_t = q_t S_t ,
+ *
+ * alpha_t in (0,1)^{d_k} a per-key-channel gate, given as log_alpha_t <= 0,
+ * S_0 = h0 (zero when h0 == NULL), and o_t reading the state after step t's own
+ * update.  gla_fwd evaluates it in the chunkwise-parallel form of sections 4.2
+ * and 4.3 (chunk size `chunk`, secondary sub-chunks of `subchunk` tokens);
+ * gla_bwd returns the gradients of a scalar loss L given dL/do and dL/dS_T, with
+ * the gate gradient from the paper's closed form (section 4.3):
+ * dlog b_t = q_t (.) dq_t - k_t (.) dk_t, dlog alpha_t = sum_{i>=t} dlog b_i.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Layout      contiguous row-major.  q, k, dq, dk: [B,H,T,d_k]; v, o, do, dv:
+ *             [B,H,T,d_v]; log_alpha, dlog_alpha: [B,H,T,d_k] (GLA_GATE_VECTOR)
+ *             or [B,H,T] (GLA_GATE_SCALAR, one gate shared by all key channels);
+ *             states h0, h_final, dh0, dh_final: [B,H,d_k,d_v] fp32.
+ * Dtypes      q, k, v, do and o, dq, dk, dv have the element type desc->dtype
+ *             (bf16 or fp32); log_alpha, dlog_alpha and every state are fp32.
+ * Ownership   the caller owns every buffer (device memory, e.g. from PyTorch).
+ *             The library never allocates device memory: all scratch space comes
+ *             from desc->workspace (size from gla_workspace_size).  Calls that
+ *             share one workspace must not overlap on the GPU.
+ * Execution   asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *             stream).  No implicit synchronisation.
+ * Nullable    h0 (zero state), h_final / dh0 (not written), dh_final (zero);
+ *             log_alpha / dlog_alpha must be NULL iff gate == GLA_GATE_NONE.
+ * Errors      every argument is validated before anything is enqueued: a call
+ *             that returns an error has launched nothing.  Errors found on the
+ *             device (a bounded wait that ran out, a gate outside the supported
+ *             range) are recorded in a status word inside the workspace and read
+ *             by gla_poll_status.
+ * Ragged T    any T >= 1.  The tail chunk is zero padded (q = k = v = 0,
+ *             log_alpha = 0 beyond T), which leaves the state unchanged.
+ */
+#ifndef GLA_B200_GLA_H
+#define GLA_B200_GLA_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Return codes (0 = success, negative = error). */
+#define GLA_OK 0
+#define GLA_ERR_INVALID_ARG (-1)        /* NULL where a buffer is required, bad enum, ... */
+#define GLA_ERR_UNSUPPORTED_SHAPE (-2)  /* shape / chunk / dtype combination not built  */
+#define GLA_ERR_MISALIGNED (-3)         /* a tensor pointer is not 16-byte aligned      */
+#define GLA_ERR_WORKSPACE_TOO_SMALL (-4)
+#define GLA_ERR_CUDA (-5)               /* a CUDA runtime / driver call failed          */
+#define GLA_ERR_TIMEOUT (-6)            /* a device-side bounded wait ran out           */
+#define GLA_ERR_GATE_RANGE (-7)         /* a gate too strong for the bf16 rescaling     */
+#define GLA_ERR_NO_DEVICE (-8)          /* no sm_100 device for the bf16 tensor path    */
+
+/* Element type of q, k, v, do and of o, dq, dk, dv. */
+#define GLA_DTYPE_BF16 0
+#define GLA_DTYPE_FP32 1
+
+/* Gate parameterisation (section 4.1 and the gate ablation of section 5):
+ * VECTOR  G_t = alpha_t^T 1 with alpha_t per key channel,
+ * SCALAR  G_t = gamma_t 1^T 1 (one gate per token and head),
+ * NONE    alpha == 1 (ungated linear attention, section 2.1). */
+#define GLA_GATE_VECTOR 0
+#define GLA_GATE_SCALAR 1
+#define GLA_GATE_NONE 2
+
+/* Forward variant (section 3.3, Figure 1):
+ * FUSED         the state is carried on chip across the chunks of a segment;
+ *               only the P segment-start states are materialised (AUTO picks P).
+ * MATERIALIZED  every chunk-level state S[n] is written to the workspace in fp32
+ *               first, then all chunk outputs are computed in parallel
+ *               ("sequence-level chunk parallelism").
+ * AUTO          FUSED with the segment count chosen to fill the GPU. */
+#define GLA_VARIANT_AUTO 0
+#define GLA_VARIANT_FUSED 1
+#define GLA_VARIANT_MATERIALIZED 2
+
+typedef struct gla_desc {
+  int B, H, T;          /* batch, heads, tokens (T >= 1)                                   */
+  int dk, dv;           /* key / value head dimensions                                     */
+  int dtype;            /* GLA_DTYPE_*                                                     */
+  int gate;             /* GLA_GATE_*                                                      */
+  int subchunk;         /* secondary chunk size; 0 = 16                                    */
+  int variant;          /* GLA_VARIANT_* (forward only)                                    */
+  int segments;         /* segments per sequence for the FUSED variant; 0 = automatic      */
+  void *workspace;      /* device scratch owned by the caller, 256-byte aligned            */
+  size_t workspace_bytes;
+} gla_desc;
+
+/* Bytes of workspace gla_fwd (for_bwd == 0) or gla_bwd (for_bwd != 0) needs for
+ * this descriptor and chunk size.  Returns 0 for an invalid descriptor (call
+ * gla_check to learn why).  Host-only; enqueues nothing. */
+size_t gla_workspace_size(const gla_desc *desc, int chunk, int for_bwd);
+
+/* Validate a descriptor + chunk without any pointer (GLA_OK or an error code).
+ * Host-only; enqueues nothing. */
+int gla_check(const gla_desc *desc, int chunk);
+
+/* Forward (sections 4.2-4.3; Algorithms 3 and 5 of Appendix B by title).
+ *   q, k [B,H,T,d_k], v [B,H,T,d_v], log_alpha (see layout), h0 [B,H,d_k,d_v] or NULL
+ *   o [B,H,T,d_v] (written), h_final [B,H,d_k,d_v] or NULL (written: S_T)
+ * chunk: C (64 for the bf16 tensor-core path; 16/32/64/128 for fp32).
+ * Returns GLA_OK or an error code; on error nothing was enqueued. */
+int gla_fwd(const gla_desc *desc, const void *q, const void *k, const void *v,
+            const float *log_alpha, const float *h0, void *o, float *h_final, int chunk,
+            void *stream);
+
+/* Backward (Algorithms 4 and 6 of Appendix B by title; closed-form gate
+ * gradient of section 4.3).  Chunk states are recomputed, not read from the
+ * forward.  The loss gradient enters through do [B,H,T,d_v] and dh_final
+ * (dL/dS_T, NULL = 0).  Outputs: dq, dk [B,H,T,d_k], dv [B,H,T,d_v],
+ * dlog_alpha (gate layout; NULL iff gate == NONE), dh0 (dL/dh0; NULL = not
+ * written).  With a SCALAR gate dlog_alpha_t is the sum over key channels. */
+int gla_bwd(const gla_desc *desc, const void *q, const void *k, const void *v,
+            const float *log_alpha, const float *h0, const void *do_, const float *dh_final,
+            void *dq, void *dk, void *dv, float *dlog_alpha, float *dh0, int chunk,
+            void *stream);
+
+/* Synchronise `stream`, then read and clear the device status word kept in
+ * desc->workspace.  Returns GLA_OK, GLA_ERR_TIMEOUT or GLA_ERR_GATE_RANGE (or
+ * GLA_ERR_CUDA if the stream itself failed). */
+int gla_poll_status(const gla_desc *desc, void *stream);
+
+/* Human-readable text for a return code (static storage). */
+const char *gla_status_string(int code);
+
+/* ---- instrumentation (benchmarking only) ------------------------------------
+ * When enabled, every kernel launch of gla_fwd / gla_bwd is bracketed by two
+ * CUDA events recorded on the launch stream.  gla_timing_collect synchronises
+ * those events and returns, for up to `max` launches since the last collect,
+ * the kernel id and its duration in milliseconds; it returns the count.
+ * Events are created by the CUDA runtime; no device memory is allocated. */
+int gla_timing_enable(int on);
+int gla_timing_collect(int max, int *kernel_ids, float *ms);
+const char *gla_kernel_name(int kernel_id);
+
+/* Build information: a static string naming the kernels and architecture. */
+const char *gla_build_info(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GLA_B200_GLA_H */

@@ -1,0 +1,104 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every function include/gla.h declares, and rejects bad arguments before
+enqueuing anything."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import chunkwise_linear_rnn_fwd_b200 as pkg
+from chunkwise_linear_rnn_fwd_b200 import gla as G
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from chunkwise_linear_rnn_fwd_b200 import build
+    build.build()
+    return pkg.load()
+
+
+def header_functions():
+    src = open(os.path.join(ROOT, "include", "gla.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(gla_[a-z_0-9]+)\s*\(", src)))
+
+
+def test_exports_every_declared_symbol(lib):
+    names = header_functions()
+    assert len(names) >= 9
+    for n in names:
+        assert hasattr(lib, n), n
+    assert sorted(G.EXPORTS) == names
+
+
+def test_status_strings(lib):
+    for code in (0, -1, -2, -3, -4, -5, -6, -7, -8):
+        assert G.status_string(code)
+    assert "unknown" in G.status_string(12345)
+
+
+def desc(**kw):
+    base = dict(B=2, H=4, T=300, dk=128, dv=256, dtype=0, gate="vector")
+    base.update(kw)
+    return G.make_desc(base.pop("B"), base.pop("H"), base.pop("T"), base.pop("dk"), base.pop("dv"),
+                       base.pop("dtype"), base.pop("gate"), **base)
+
+
+def test_check_and_workspace(lib):
+    d = desc()
+    assert lib.gla_check(ctypes.byref(d), 64) == 0
+    assert lib.gla_workspace_size(ctypes.byref(d), 64, 0) > 0
+    assert lib.gla_workspace_size(ctypes.byref(d), 64, 1) >= lib.gla_workspace_size(ctypes.byref(d), 64, 0)
+    assert lib.gla_check(ctypes.byref(d), 48) == -2            # chunk not supported
+    assert lib.gla_check(ctypes.byref(desc(T=0)), 64) == -1
+    assert lib.gla_check(ctypes.byref(desc(dtype=7)), 64) == -1
+    assert lib.gla_check(ctypes.byref(desc(gate=5)), 64) == -1
+    assert lib.gla_check(ctypes.byref(desc(dk=512)), 64) == -2
+    assert lib.gla_check(ctypes.byref(desc(subchunk=24)), 64) == -2
+    assert lib.gla_workspace_size(ctypes.byref(desc(T=0)), 64, 0) == 0
+    assert lib.gla_check(None, 64) == -1
+
+
+def test_bad_calls_enqueue_nothing(lib):
+    """Every one of these returns an error from host validation alone (no GPU
+    is touched: the status word is cleared only after validation passes)."""
+    vp = ctypes.c_void_p
+    a = vp(4096)           # aligned, never dereferenced
+    mis = vp(4096 + 4)     # misaligned
+    ws = vp(1 << 20)
+    d = desc(T=64, dk=128, dv=128)
+    d.workspace = 1 << 20
+    d.workspace_bytes = 1 << 40
+    f = lib.gla_fwd
+    assert f(ctypes.byref(d), None, a, a, a, None, a, None, 64, None) == -1      # q NULL
+    assert f(ctypes.byref(d), mis, a, a, a, None, a, None, 64, None) == -3       # q misaligned
+    assert f(ctypes.byref(d), a, a, a, None, None, a, None, 64, None) == -1      # vector gate without log_alpha
+    d.gate = 2
+    assert f(ctypes.byref(d), a, a, a, a, None, a, None, 64, None) == -1         # none gate with log_alpha
+    d.gate = 0
+    d.workspace_bytes = 16
+    assert f(ctypes.byref(d), a, a, a, a, None, a, None, 64, None) == -4         # workspace too small
+    d.workspace_bytes = 1 << 40
+    d.workspace = (1 << 20) + 8
+    assert f(ctypes.byref(d), a, a, a, a, None, a, None, 64, None) == -3         # workspace misaligned
+    d.workspace = 0
+    assert f(ctypes.byref(d), a, a, a, a, None, a, None, 64, None) == -1         # no workspace
+    d.workspace = 1 << 20
+    b = lib.gla_bwd
+    assert b(ctypes.byref(d), a, a, a, a, None, None, None, a, a, a, a, None, 64, None) == -1   # do NULL
+    assert b(ctypes.byref(d), a, a, a, a, None, a, None, a, a, a, None, None, 64, None) == -1   # dlog_alpha NULL
+    d.gate = 2
+    assert b(ctypes.byref(d), a, a, a, None, None, a, None, a, a, a, a, None, 64, None) == -1   # none gate with dla
+
+
+def test_oracle_not_imported_by_product():
+    """The product package never imports, loads or links the oracle."""
+    pkg_dir = os.path.join(ROOT, "chunkwise_linear_rnn_fwd_b200")
+    pat = re.compile(r"^\s*(from\s+oracle|import\s+oracle)|libgla_oracle|gla_oracle", re.M)
+    for root, _, files in os.walk(pkg_dir):
+        for f in files:
+            if f.endswith((".py", ".cu", ".h", ".cuh")):
+                assert not pat.search(open(os.path.join(root, f)).read()), f
