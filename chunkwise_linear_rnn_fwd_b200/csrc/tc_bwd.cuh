@@ -1,0 +1,463 @@
+// tc_bwd.cuh -- per-chunk backward kernel of the bf16 tensor-core path.
+//
+// One CTA per (chunk n, head).  Inputs: the recomputed chunk state h_n (state
+// before chunk n) and adjoint dh_n (gradient w.r.t. the state after chunk n),
+// both bf16 [K][V]; qg, kg, P^T and gam from the prep kernel; q, k, V, dO and
+// log_alpha.  With B the chunk-local cumulative log-gate:
+//   phase 1 (loop over d_v tiles of 64, accumulating in TMEM):
+//     dqh^T = h_n dO^T          dkh^T = dh_n V^T         dP = dO V^T
+//     dv    = kg dh_n + P^T dO  (stored per tile)
+//     R[c]  = sum_v h_n[c,v] dh_n[c,v]
+//   phase 2 (intra-chunk, sub-chunk reference points, all on tcgen05):
+//     dq_intra[t] = u_t (.) sum_{s<=t} dP[t,s] k_s e^{z_j(t) - B_s}
+//     dk_intra[s] = w_s (.) sum_{t>=s} dP[t,s] q_t e^{B_t - z_j(s)+1}
+//   epilogue per key channel:
+//     dq = e^{B} (.) dqh + dq_intra ,  dk = e^{B_63 - B} (.) dkh + dk_intra
+//     dlog b_t = q_t dq_t - k_t dk_t                       (section 4.3)
+//     dlog alpha_t = sum_{i>=t in chunk} dlog b_i + G_n,
+//     G_n = gam_n R + sum_t k_t (.) e^{B_63-B_t} dkh_t  ( = sum_v S_n dS_n, the
+//           part of the suffix sum that lies beyond the chunk).
+#pragma once
+
+#include "tc_kernels.cuh"
+
+namespace gla {
+namespace tc {
+
+inline size_t bwd_scratch_floats(long BH, int N, int K, int V) {
+  (void)BH; (void)N; (void)K; (void)V;
+  return 0;
+}
+
+struct BwdArgs {
+  int T, N, V, gate;
+  long Tp;
+  const bf16 *q, *k;
+  const float *la;
+  const float *gam;
+  bf16 *dq, *dk, *dv;
+  float *dla;
+  unsigned *status;
+};
+
+template <int K>
+struct BwdSmem {
+  static constexpr int BVb = 64;
+  static constexpr int kTileH = K * BVb * 2;
+  static constexpr int kTileV = 64 * BVb * 2;
+  static constexpr int kStage = 2 * kTileH + 2 * kTileV;   // h, dh, V, dO
+  static constexpr int kKg = 2 * kStage;                   // kg tile [64][K]
+  static constexpr int kPT = kKg + 64 * K * 2;             // P^T tile [64][64]
+  static constexpr int kPhase1End = kPT + 64 * 64 * 2;
+  // phase 2 (aliases the phase-1 stages)
+  static constexpr int kRowsW = 160;
+  static constexpr int kKh = 0;                            // key windows  [160][K]
+  static constexpr int kQh = kKh + kRowsW * K * 2;         // query windows [160][K]
+  static constexpr int kdP = kQh + kRowsW * K * 2;         // masked dP  [t][s]
+  static constexpr int kdPT = kdP + 64 * 64 * 2;           // masked dP^T [s][t]
+  static constexpr int kPhase2End = kdPT + 64 * 64 * 2;
+  static constexpr int kRed = (kPhase1End > kPhase2End ? kPhase1End : kPhase2End);  // scalar-gate reduction [8][64]
+  static constexpr int kBar = kRed + 8 * 64 * 4;
+  static constexpr int kBytes = kBar + 128;
+};
+
+template <int K>
+__global__ void __launch_bounds__(256, 1)
+    k_bwd_main(BwdArgs a, const __grid_constant__ CUtensorMap tmH, const __grid_constant__ CUtensorMap tmDH,
+               const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
+               const __grid_constant__ CUtensorMap tmKg, const __grid_constant__ CUtensorMap tmPT) {
+  using L = BwdSmem<K>;
+  constexpr int BVb = L::BVb;
+  constexpr int kMB = K / 128;
+  constexpr int cDQ = 0, cDK = 64 * kMB, cDP = 128 * kMB, cDV = cDP + 64;
+  constexpr int cQI = cDP, cKI = cQI + 64 * kMB;
+  constexpr int kTmemCols = (K == 256) ? 512 : 256;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint64_t *full = (uint64_t *)(smem + L::kBar);  // [0],[1] stages, [2] kg+PT
+  uint64_t *mma_bar = full + 3;
+  uint32_t *tslot = (uint32_t *)(full + 4);
+  float *red = (float *)(smem + L::kRed);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int n = blockIdx.x;
+  const long bh = blockIdx.y;
+  const int nvt = a.V / BVb;
+  const long hrow = bh * a.N + n;
+
+  if (warp == 0) dev::tmem_alloc(tslot, kTmemCols);
+  if (tid == 0) {
+    for (int i = 0; i < 3; ++i) dev::mbar_init(&full[i], 1);
+    dev::mbar_init(mma_bar, 1);
+    dev::fence_mbar_init();
+  }
+  dev::tc_fence_before();
+  __syncthreads();
+  dev::tc_fence_after();
+  const uint32_t tmem = *tslot;
+
+  auto stage = [&](int s) { return smem + s * L::kStage; };
+  auto issue_tile = [&](int i) {
+    const int s = i & 1;
+    uint8_t *st = stage(s);
+    const int v0 = i * BVb;
+    dev::mbar_arrive_expect_tx(&full[s], (uint32_t)L::kStage);
+    dev::tma_load_3d(st, &tmH, v0, 0, (int)hrow, &full[s]);
+    dev::tma_load_3d(st + L::kTileH, &tmDH, v0, 0, (int)hrow, &full[s]);
+    dev::tma_load_3d(st + 2 * L::kTileH, &tmV, v0, n * kC, (int)bh, &full[s]);
+    dev::tma_load_3d(st + 2 * L::kTileH + L::kTileV, &tmDO, v0, n * kC, (int)bh, &full[s]);
+  };
+  if (tid == 0) {
+    dev::mbar_arrive_expect_tx(&full[2], (uint32_t)(64 * K * 2 + 64 * 64 * 2));
+#pragma unroll
+    for (int cb = 0; cb < K / 64; ++cb)
+      dev::tma_load_3d(smem + L::kKg + cb * 64 * 128, &tmKg, cb * 64, n * kC, (int)bh, &full[2]);
+    dev::tma_load_3d(smem + L::kPT, &tmPT, 0, 0, (int)hrow, &full[2]);
+    issue_tile(0);
+    if (nvt > 1) issue_tile(1);
+  }
+
+  const int c = tid;  // key channel (valid when tid < K)
+  float R = 0.f;      // sum_v h[c,v] dh[c,v]
+  bool ok = dev::mbar_wait(&full[2], 0, a.status);
+
+  // ============================ phase 1 ============================
+  for (int i = 0; i < nvt; ++i) {
+    const int s = i & 1;
+    uint8_t *st = stage(s);
+    if (ok) ok = dev::mbar_wait(&full[s], (i >> 1) & 1, a.status);
+    if (tid < K) {
+      const uint32_t sh = dev::smem_u32(st), sdh = sh + L::kTileH;
+#pragma unroll
+      for (int c8 = 0; c8 < BVb / 8; ++c8) {
+        uint4 x, y;
+        asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];"
+                     : "=r"(x.x), "=r"(x.y), "=r"(x.z), "=r"(x.w)
+                     : "r"(sh + dev::sw128_chunk(K, c, c8)));
+        asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];"
+                     : "=r"(y.x), "=r"(y.y), "=r"(y.z), "=r"(y.w)
+                     : "r"(sdh + dev::sw128_chunk(K, c, c8)));
+        const __nv_bfloat162 *xh = reinterpret_cast<const __nv_bfloat162 *>(&x);
+        const __nv_bfloat162 *yh = reinterpret_cast<const __nv_bfloat162 *>(&y);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 xf = __bfloat1622float2(xh[e]), yf = __bfloat1622float2(yh[e]);
+          R += xf.x * yf.x + xf.y * yf.y;
+        }
+      }
+    }
+    dev::tc_fence_before();
+    __syncthreads();
+    dev::tc_fence_after();
+    if (tid == 0 && ok) {
+      const uint32_t sH = dev::smem_u32(st), sDH = sH + L::kTileH, sV = sDH + L::kTileH, sDO = sV + L::kTileV;
+      const uint32_t sKg = dev::smem_u32(smem + L::kKg), sPT = dev::smem_u32(smem + L::kPT);
+      constexpr uint32_t id_kk128 = dev::idesc_bf16(128, 64, false, false);
+      constexpr uint32_t id_kk64 = dev::idesc_bf16(64, 64, false, false);
+#pragma unroll
+      for (int kk = 0; kk < BVb / 16; ++kk) {
+        const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
+#pragma unroll
+        for (int m = 0; m < kMB; ++m) {
+          dev::umma_bf16(tmem + cDQ + 64 * m, dev::desc_kmajor(sH, K, 128 * m, kk * 16),
+                         dev::desc_kmajor(sDO, 64, 0, kk * 16), id_kk128, acc);
+          dev::umma_bf16(tmem + cDK + 64 * m, dev::desc_kmajor(sDH, K, 128 * m, kk * 16),
+                         dev::desc_kmajor(sV, 64, 0, kk * 16), id_kk128, acc);
+        }
+        dev::umma_bf16(tmem + cDP, dev::desc_kmajor(sDO, 64, 0, kk * 16), dev::desc_kmajor(sV, 64, 0, kk * 16),
+                       id_kk64, acc);
+      }
+      // dv tile = kg dh + P^T dO
+      constexpr uint32_t id_dv1 = dev::idesc_bf16(64, BVb, false, true);
+#pragma unroll
+      for (int kk = 0; kk < K / 16; ++kk)
+        dev::umma_bf16(tmem + cDV, dev::desc_kmajor(sKg, 64, 0, kk * 16), dev::desc_mnmajor(sDH, K, kk * 16, 0),
+                       id_dv1, kk > 0 ? 1u : 0u);
+      // A[m = t][k = s] = P[s][t] = P^T tile [t][s]: K-major
+      constexpr uint32_t id_dv2 = dev::idesc_bf16(64, BVb, false, true);
+#pragma unroll
+      for (int kk = 0; kk < kC / 16; ++kk)
+        dev::umma_bf16(tmem + cDV, dev::desc_kmajor(sPT, 64, 0, kk * 16), dev::desc_mnmajor(sDO, 64, kk * 16, 0),
+                       id_dv2, 1u);
+      dev::umma_commit(mma_bar);
+    }
+    if (ok) ok = dev::mbar_wait(mma_bar, i & 1, a.status);
+    dev::tc_fence_after();
+    if (tid == 0 && ok && i + 2 < nvt) issue_tile(i + 2);
+    // dv epilogue: rows t (M = 64 layout), warps 0-3 columns [0,32), warps 4-7 [32,64)
+    {
+      const int sub = warp & 3;
+      const int col0 = (warp >= 4) ? BVb / 2 : 0;
+      const int t = 16 * sub + lane;
+      const long tgl = (long)n * kC + t;
+#pragma unroll
+      for (int cb = 0; cb < BVb / 32; ++cb) {
+        float v[16];
+        dev::tmem_ld16(dev::tmem_addr(tmem, 32 * sub, cDV + col0 + cb * 16), v);
+        dev::tmem_wait_ld();
+        if (lane < 16 && tgl < a.T && ok) {
+          uint4 p0, p1;
+          p0.x = dev::pack_bf16(v[0], v[1]);
+          p0.y = dev::pack_bf16(v[2], v[3]);
+          p0.z = dev::pack_bf16(v[4], v[5]);
+          p0.w = dev::pack_bf16(v[6], v[7]);
+          p1.x = dev::pack_bf16(v[8], v[9]);
+          p1.y = dev::pack_bf16(v[10], v[11]);
+          p1.z = dev::pack_bf16(v[12], v[13]);
+          p1.w = dev::pack_bf16(v[14], v[15]);
+          uint4 *dst = reinterpret_cast<uint4 *>(a.dv + (bh * a.T + tgl) * (long)a.V + i * BVb + col0 + cb * 16);
+          dst[0] = p0;
+          dst[1] = p1;
+        }
+      }
+    }
+    dev::tc_fence_before();
+    __syncthreads();
+    dev::tc_fence_after();
+  }
+
+  // ============================ phase 2 ============================
+  // dP (rows t, TMEM M = 64 layout) -> masked bf16 tiles dP[t][s] and dP^T[s][t]
+  const uint32_t sdP = dev::smem_u32(smem + L::kdP), sdPT = dev::smem_u32(smem + L::kdPT);
+  if (warp < 4) {
+    const int t = 16 * warp + lane;
+    float row[kC];
+#pragma unroll
+    for (int cb = 0; cb < 4; ++cb) dev::tmem_ld16(dev::tmem_addr(tmem, 32 * warp, cDP + 16 * cb), row + 16 * cb);
+    dev::tmem_wait_ld();
+    if (lane < 16) {
+#pragma unroll
+      for (int s8 = 0; s8 < 8; ++s8) {
+        float m8[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) m8[e] = (s8 * 8 + e <= t && ok) ? row[s8 * 8 + e] : 0.f;
+        dev::st_shared_v4(sdP + dev::sw128_chunk(64, t, s8), dev::pack_bf16(m8[0], m8[1]),
+                          dev::pack_bf16(m8[2], m8[3]), dev::pack_bf16(m8[4], m8[5]), dev::pack_bf16(m8[6], m8[7]));
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const bf16 b = __float2bfloat16_rn(m8[e]);
+          dev::st_shared_u16(sdPT + dev::sw128_off(64, s8 * 8 + e, t), *reinterpret_cast<const uint16_t *>(&b));
+        }
+      }
+    }
+  }
+
+  // per key channel: cumulative log-gate and the rescaled operands
+  float Bv[kC];
+  float z[5], Gam[4], E[4];
+  const long qrow0 = bh * a.T + (long)n * kC;  // first token row of this chunk
+  auto qk_at = [&](int t, float &qf, float &kf) {
+    qf = 0.f;
+    kf = 0.f;
+    if ((long)n * kC + t < a.T) {
+      qf = __bfloat162float(a.q[(qrow0 + t) * K + c]);
+      kf = __bfloat162float(a.k[(qrow0 + t) * K + c]);
+    }
+  };
+  if (tid < K) {
+    float acc = 0.f;
+#pragma unroll
+    for (int t = 0; t < kC; ++t) {
+      float g = 0.f;
+      if ((long)n * kC + t < a.T) {
+        if (a.gate == GLA_GATE_VECTOR) g = __ldg(a.la + (qrow0 + t) * K + c);
+        else if (a.gate == GLA_GATE_SCALAR) g = __ldg(a.la + qrow0 + t);
+      }
+      acc += g;
+      Bv[t] = acc;
+    }
+    z[0] = 0.f;
+    z[1] = Bv[15];
+    z[2] = Bv[31];
+    z[3] = Bv[47];
+    z[4] = Bv[63];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      Gam[j] = __expf(z[j + 1] - z[j]);
+      E[j] = __expf(z[j]);
+    }
+    const uint32_t sKh = dev::smem_u32(smem + L::kKh), sQh = dev::smem_u32(smem + L::kQh);
+    const int wK[4] = {0, 16, 48, 96};   // key window j: row wK[j] + s, s in [0, 16(j+1))
+    const int wQ[4] = {0, 48, 80, 96};   // query window u: row wQ[u] + t, t in [16u, 64)
+#pragma unroll
+    for (int t = 0; t < kC; ++t) {
+      const int j = t >> 4;
+      float qf, kf;
+      qk_at(t, qf, kf);
+      const float u = __expf(Bv[t] - z[j]);
+      const float w = __expf(z[j + 1] - Bv[t]);
+      // key operand k_t e^{z_jq - B_t}, query sub-chunks jq >= j (one more Gam per step)
+      float f = kf * w / Gam[j];
+#pragma unroll
+      for (int jq = 0; jq < 4; ++jq) {
+        if (jq >= j) {
+          const bf16 b = __float2bfloat16_rn(f);
+          dev::st_shared_u16(sKh + dev::sw128_off(L::kRowsW, wK[jq] + t, c), *reinterpret_cast<const uint16_t *>(&b));
+          f *= Gam[jq];
+        }
+      }
+      // query operand q_t e^{B_t - z_{uu+1}}, key sub-chunks uu <= j (one more Gam per step down)
+      float g2 = qf * u / Gam[j];
+#pragma unroll
+      for (int uu = 3; uu >= 0; --uu) {
+        if (uu <= j) {
+          const bf16 b = __float2bfloat16_rn(g2);
+          dev::st_shared_u16(sQh + dev::sw128_off(L::kRowsW, wQ[uu] + t, c), *reinterpret_cast<const uint16_t *>(&b));
+          g2 *= Gam[uu];
+        }
+      }
+    }
+  }
+  dev::fence_proxy_async_smem();
+  dev::tc_fence_before();
+  __syncthreads();
+  dev::tc_fence_after();
+  if (tid == 0 && ok) {
+    const uint32_t sKh = dev::smem_u32(smem + L::kKh), sQh = dev::smem_u32(smem + L::kQh);
+    const int wK[4] = {0, 16, 48, 96};
+    const int wQ[4] = {0, 48, 80, 96};
+    constexpr uint32_t id = dev::idesc_bf16(128, 16, true, false);
+#pragma unroll
+    for (int m = 0; m < kMB; ++m) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+#pragma unroll
+        for (int kk = 0; kk <= j; ++kk)
+          dev::umma_bf16(tmem + cQI + 64 * m + 16 * j, dev::desc_mnmajor(sKh, L::kRowsW, wK[j] + 16 * kk, 128 * m),
+                         dev::desc_kmajor(sdP, 64, 16 * j, 16 * kk), id, kk > 0 ? 1u : 0u);
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int kk = u; kk < 4; ++kk)
+          dev::umma_bf16(tmem + cKI + 64 * m + 16 * u, dev::desc_mnmajor(sQh, L::kRowsW, wQ[u] + 16 * kk, 128 * m),
+                         dev::desc_kmajor(sdPT, 64, 16 * u, 16 * kk), id, kk > u ? 1u : 0u);
+    }
+    dev::umma_commit(mma_bar);
+  }
+  if (ok) ok = dev::mbar_wait(mma_bar, nvt & 1, a.status);
+  dev::tc_fence_after();
+
+  // ============================ epilogue ============================
+  const int mb = warp >> 2;
+  const uint32_t lanebase = 32 * (warp & 3);
+  // pass A: boundary term G_n = gam_n R + sum_t k_t dk_inter_t
+  float Gb = 0.f;
+  if (tid < K) {
+    Gb = a.gam[(bh * a.N + n) * K + c] * R;
+  }
+#pragma unroll
+  for (int t16 = 0; t16 < 4; ++t16) {
+    float xk[16];
+    dev::tmem_ld16(dev::tmem_addr(tmem, lanebase, cDK + 64 * mb + 16 * t16), xk);
+    dev::tmem_wait_ld();
+    if (tid < K) {
+      const int j = t16;
+      float Gafter = 1.f;
+#pragma unroll
+      for (int i2 = 1; i2 < 4; ++i2)
+        if (i2 > j) Gafter *= Gam[i2];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const int t = 16 * t16 + e;
+        float qf, kf;
+        qk_at(t, qf, kf);
+        Gb += kf * __expf(z[j + 1] - Bv[t]) * Gafter * xk[e];
+      }
+    }
+  }
+  // pass B: reverse over tokens; dq, dk, dlog b and its suffix sum
+  float run = Gb;
+#pragma unroll
+  for (int t16 = 3; t16 >= 0; --t16) {
+    float xq[16], xk[16], xqi[16], xki[16];
+    dev::tmem_ld16(dev::tmem_addr(tmem, lanebase, cDQ + 64 * mb + 16 * t16), xq);
+    dev::tmem_ld16(dev::tmem_addr(tmem, lanebase, cDK + 64 * mb + 16 * t16), xk);
+    dev::tmem_ld16(dev::tmem_addr(tmem, lanebase, cQI + 64 * mb + 16 * t16), xqi);
+    dev::tmem_ld16(dev::tmem_addr(tmem, lanebase, cKI + 64 * mb + 16 * t16), xki);
+    dev::tmem_wait_ld();
+    const int j = t16;
+    float Gafter = 1.f;
+#pragma unroll
+    for (int i2 = 1; i2 < 4; ++i2)
+      if (i2 > j) Gafter *= Gam[i2];
+#pragma unroll
+    for (int e = 15; e >= 0; --e) {
+      const int t = 16 * t16 + e;
+      const long tg = (long)n * kC + t;
+      float dlb = 0.f;
+      if (tid < K) {
+        float qf, kf;
+        qk_at(t, qf, kf);
+        const float u = __expf(Bv[t] - z[j]);
+        const float w = __expf(z[j + 1] - Bv[t]);
+        const float dqv = u * (E[j] * xq[e] + xqi[e]);
+        const float dkv = w * (Gafter * xk[e] + xki[e]);
+        run += qf * dqv - kf * dkv;
+        dlb = run;
+        if (tg < a.T && ok) {
+          a.dq[(qrow0 + t) * K + c] = __float2bfloat16_rn(dqv);
+          a.dk[(qrow0 + t) * K + c] = __float2bfloat16_rn(dkv);
+          if (a.gate == GLA_GATE_VECTOR) a.dla[(qrow0 + t) * K + c] = dlb;
+        }
+      }
+      if (a.gate == GLA_GATE_SCALAR) {
+        float x = dlb;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+        if (lane == 0) red[warp * 64 + t] = x;
+      }
+    }
+  }
+  if (a.gate == GLA_GATE_SCALAR) {
+    __syncthreads();
+    if (tid < kC) {
+      float ssum = 0.f;
+#pragma unroll
+      for (int w8 = 0; w8 < 8; ++w8) ssum += red[w8 * 64 + tid];
+      const long tg = (long)n * kC + tid;
+      if (tg < a.T && ok) a.dla[bh * a.T + tg] = ssum;
+    }
+  }
+  dev::tc_fence_before();
+  __syncthreads();
+  if (warp == 0) dev::tmem_dealloc(tmem, kTmemCols);
+}
+
+template <int K>
+int launch_bwd_main_k(const Problem &p, const BwdArgs &a, const CUtensorMap *maps, cudaStream_t st) {
+  const int smem = BwdSmem<K>::kBytes + 1024;
+  static bool attr = false;
+  if (!attr) {
+    if (cudaFuncSetAttribute(k_bwd_main<K>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+      return GLA_ERR_CUDA;
+    attr = true;
+  }
+  GLA_LAUNCH(K_TC_BWD, st,
+             (k_bwd_main<K><<<dim3(p.N, p.BH), 256, smem, st>>>(a, maps[0], maps[1], maps[2], maps[3], maps[4],
+                                                                 maps[5])));
+  return GLA_OK;
+}
+
+bool map3_bf16(CUtensorMap *m, const void *base, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t b0, uint32_t b1);
+
+inline int launch_bwd_main(const Problem &p, const bf16 *q, const bf16 *k, const bf16 *v, const float *la,
+                           const bf16 *dout, bf16 *dq, bf16 *dk, bf16 *dv, float *dla, const bf16 *qg,
+                           const bf16 *kg, const bf16 *PT, const float *gam, const bf16 *hb, const bf16 *dhb,
+                           float *scratch, unsigned *status, cudaStream_t st) {
+  (void)qg;
+  (void)scratch;
+  if (p.V % 64 != 0) return GLA_ERR_UNSUPPORTED_SHAPE;
+  CUtensorMap maps[6];
+  const uint64_t BH = (uint64_t)p.BH;
+  const bool ok = map3_bf16(&maps[0], hb, p.V, p.K, BH * p.N, 64, p.K) &&
+                  map3_bf16(&maps[1], dhb, p.V, p.K, BH * p.N, 64, p.K) &&
+                  map3_bf16(&maps[2], v, p.V, p.T, BH, 64, 64) && map3_bf16(&maps[3], dout, p.V, p.T, BH, 64, 64) &&
+                  map3_bf16(&maps[4], kg, p.K, p.Tp, BH, 64, 64) && map3_bf16(&maps[5], PT, 64, 64, BH * p.N, 64, 64);
+  if (!ok) return GLA_ERR_CUDA;
+  BwdArgs a{p.T, p.N, p.V, p.gate, p.Tp, q, k, la, gam, dq, dk, dv, dla, status};
+  if (p.K == 256) return launch_bwd_main_k<256>(p, a, maps, st);
+  return launch_bwd_main_k<128>(p, a, maps, st);
+}
+
+}  // namespace tc
+}  // namespace gla

@@ -1,0 +1,536 @@
+// tc_kernels.cuh -- bf16 tensor-core kernels of the chunkwise GLA path (sm_100a).
+//
+// Notation (one head): chunk size C = 64, sub-chunk c = 16, d_k = K, tile of
+// d_v = BV.  B_t is the chunk-local inclusive cumulative log-gate, z_j = B at
+// the last row before sub-chunk j (z_0 = 0, z_4 = B_63), Gam_j = e^{z_{j+1}-z_j}
+// the decay of sub-chunk j, u_t = e^{B_t - z_{j(t)}} and w_t = e^{z_{j(t)+1} - B_t}
+// (both in (0,1]).  Every rescaled operand is a product of such factors, so no
+// factor exceeds 1 except the diagonal-block key factor 1/Gam_j (section 4.2 /
+// Figure 3 of "Gated Linear Attention Transformers with Hardware-Efficient
+// Training": secondary chunking with a reference point at each query sub-chunk).
+#pragma once
+
+#include "tc_common.cuh"
+
+namespace gla {
+namespace tc {
+
+using bf16 = __nv_bfloat16;
+constexpr int kC = 64;    // chunk
+constexpr int kSub = 16;  // sub-chunk
+
+// ============================================================================
+// Prep: per (chunk, head).  Writes
+//   qg[t]  = q_t (.) e^{B_t}              (bf16, inter-chunk query operand)
+//   kg[t]  = k_t (.) e^{B_63 - B_t}       (bf16, state-update key operand)
+//   gam    = e^{B_63}                     (fp32 per key channel)
+//   PT[s][t] = causal intra-chunk score A[t][s] (bf16, transposed)
+// The strictly-lower sub-chunk blocks of A come from three tcgen05 MMAs
+// (M = 64 keys, N = 16 queries of sub-chunk j, reference point z_j); the four
+// diagonal 16 x 16 blocks are summed in fp32 on CUDA cores.
+// ============================================================================
+struct PrepArgs {
+  int T, N, gate;
+  long Tp;
+  const bf16 *q, *k;
+  const float *la;
+  bf16 *qg, *kg, *PT;
+  float *gam;
+  unsigned *status;
+};
+
+template <int K>
+struct PrepSmem {
+  static constexpr int kRowsKw = 112;                  // K-hat windows: rows [0,16) [16,48) [48,96) + pad
+  static constexpr int kQh = 0;                        // Q-hat tile, 64 rows
+  static constexpr int kKw = kQh + 64 * K * 2;         // key windows, 112 rows
+  static constexpr int kAf = kKw + kRowsKw * K * 2;    // fp32 a_t = q_t u_t    [64][K]
+  static constexpr int kBf = kAf + 64 * K * 4;         // fp32 b_s = k_s e^{z_j - B_s}
+  static constexpr int kPd = kBf + 64 * K * 4;         // fp32 diag partials [2][64][16]
+  static constexpr int kBar = kPd + 2 * 64 * 16 * 4;   // mbarrier + tmem slot
+  static constexpr int kBytes = kBar + 64;
+};
+
+// fp32 [64][K] tile with a 16-byte-chunk swizzle (bank-conflict-free for the
+// diagonal-block access pattern).
+template <int K>
+__device__ __forceinline__ int f32_swz(int r, int c) {
+  const int cc = c >> 2;
+  const int sw = (r ^ (r >> 3)) & 7;
+  return r * K + (((cc & ~7) | ((cc & 7) ^ sw)) << 2) + (c & 3);
+}
+
+template <int K>
+__global__ void __launch_bounds__(256, 1) k_prep(PrepArgs a) {
+  using L = PrepSmem<K>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  const uint32_t sQh = dev::smem_u32(smem + L::kQh);
+  const uint32_t sKw = dev::smem_u32(smem + L::kKw);
+  float *Af = (float *)(smem + L::kAf);
+  float *Bf = (float *)(smem + L::kBf);
+  float *Pd = (float *)(smem + L::kPd);
+  uint64_t *bar = (uint64_t *)(smem + L::kBar);
+  uint32_t *tslot = (uint32_t *)(smem + L::kBar + 16);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int n = blockIdx.x;
+  const long bh = blockIdx.y;
+
+  if (warp == 0) dev::tmem_alloc(tslot, 64);
+  if (tid == 0) {
+    dev::mbar_init(bar, 1);
+    dev::fence_mbar_init();
+  }
+
+  // ---- per key channel: cumulative log-gate and rescaled operands --------
+  if (tid < K) {
+    const int c = tid;
+    float Bv[kC];
+    float acc = 0.f;
+#pragma unroll
+    for (int t = 0; t < kC; ++t) {
+      const long tg = (long)n * kC + t;
+      float g = 0.f;
+      if (tg < a.T) {
+        if (a.gate == GLA_GATE_VECTOR) g = __ldg(a.la + (bh * a.T + tg) * K + c);
+        else if (a.gate == GLA_GATE_SCALAR) g = __ldg(a.la + bh * a.T + tg);
+      }
+      acc += g;
+      Bv[t] = acc;
+    }
+    float z[5];
+    z[0] = 0.f;
+    z[1] = Bv[15];
+    z[2] = Bv[31];
+    z[3] = Bv[47];
+    z[4] = Bv[63];
+    float Gam[4], E[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      Gam[j] = __expf(z[j + 1] - z[j]);
+      E[j] = __expf(z[j]);
+    }
+    if (Gam[0] < 1e-36f || Gam[1] < 1e-36f || Gam[2] < 1e-36f || Gam[3] < 1e-36f)
+      atomicOr(a.status, (unsigned)ST_GATE_RANGE);
+    // Gafter[j] = prod_{i>j} Gam_i = e^{B_63 - z_{j+1}}
+    float Gafter[4];
+    Gafter[3] = 1.f;
+    Gafter[2] = Gam[3];
+    Gafter[1] = Gam[3] * Gam[2];
+    Gafter[0] = Gam[3] * Gam[2] * Gam[1];
+    a.gam[(bh * a.N + n) * K + c] = __expf(z[4]);
+    const int wrow[4] = {0, 0, 16, 48};  // window start row of query sub-chunk j (j >= 1)
+#pragma unroll
+    for (int t = 0; t < kC; ++t) {
+      const int j = t >> 4;
+      const long tg = (long)n * kC + t;
+      float qf = 0.f, kf = 0.f;
+      if (tg < a.T) {
+        qf = __bfloat162float(a.q[(bh * a.T + tg) * K + c]);
+        kf = __bfloat162float(a.k[(bh * a.T + tg) * K + c]);
+      }
+      const float u = __expf(Bv[t] - z[j]);
+      const float w = __expf(z[j + 1] - Bv[t]);
+      const float qh = qf * u;
+      const float kw = kf * w;
+      a.qg[(bh * a.Tp + tg) * K + c] = __float2bfloat16_rn(qh * E[j]);
+      a.kg[(bh * a.Tp + tg) * K + c] = __float2bfloat16_rn(kw * Gafter[j]);
+      const bf16 qhb = __float2bfloat16_rn(qh);
+      dev::st_shared_u16(sQh + dev::sw128_off(64, t, c), *reinterpret_cast<const uint16_t *>(&qhb));
+      Af[f32_swz<K>(t, c)] = qh;
+      Bf[f32_swz<K>(t, c)] = kw / Gam[j];
+      // key operand for every later query sub-chunk jq: k_s e^{z_jq - B_s}
+      float f = kw;
+#pragma unroll
+      for (int jq = 1; jq < 4; ++jq) {
+        if (jq > j) {
+          const bf16 kb = __float2bfloat16_rn(f);
+          dev::st_shared_u16(sKw + dev::sw128_off(L::kRowsKw, wrow[jq] + t, c), *reinterpret_cast<const uint16_t *>(&kb));
+          f *= Gam[jq];
+        }
+      }
+    }
+    // rows 96..111 of the window buffer are read by window 3 only for keys >= 48
+    // (whose entries are discarded); keep them finite.
+    const bf16 zb = __float2bfloat16_rn(0.f);
+    for (int r = 96; r < L::kRowsKw; ++r)
+      dev::st_shared_u16(sKw + dev::sw128_off(L::kRowsKw, r, c), *reinterpret_cast<const uint16_t *>(&zb));
+  }
+  dev::fence_proxy_async_smem();
+  dev::tc_fence_before();
+  __syncthreads();
+  dev::tc_fence_after();
+  const uint32_t tmem = *tslot;
+
+  // ---- off-diagonal blocks on the tensor cores ----------------------------
+  if (tid == 0) {
+    constexpr uint32_t idesc = dev::idesc_bf16(64, 16, false, false);
+    const int wrow[4] = {0, 0, 16, 48};
+#pragma unroll
+    for (int j = 1; j < 4; ++j) {
+#pragma unroll
+      for (int kk = 0; kk < K / 16; ++kk) {
+        const uint64_t da = dev::desc_kmajor(sKw, L::kRowsKw, wrow[j], kk * 16);
+        const uint64_t db = dev::desc_kmajor(sQh, 64, 16 * j, kk * 16);
+        dev::umma_bf16(tmem + 16 * j, da, db, idesc, kk > 0 ? 1u : 0u);
+      }
+    }
+    dev::umma_commit(bar);
+  }
+
+  // ---- diagonal blocks in fp32 on CUDA cores ------------------------------
+  {
+    const int j = warp >> 1, half = warp & 1;
+    const int tg = lane >> 3, sp = lane & 7;
+    const int t0 = 16 * j + 4 * tg, s0 = 16 * j + 2 * sp;
+    float acc[4][2] = {};
+    const bool active = (s0 <= t0 + 3);
+    if (active) {
+      const int c_begin = half * (K / 2), c_end = c_begin + K / 2;
+      for (int c = c_begin; c < c_end; c += 4) {
+        float4 av[4], bv[2];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) av[i] = *reinterpret_cast<const float4 *>(Af + f32_swz<K>(t0 + i, c));
+#pragma unroll
+        for (int i = 0; i < 2; ++i) bv[i] = *reinterpret_cast<const float4 *>(Bf + f32_swz<K>(s0 + i, c));
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int m = 0; m < 2; ++m)
+            acc[i][m] += av[i].x * bv[m].x + av[i].y * bv[m].y + av[i].z * bv[m].z + av[i].w * bv[m].w;
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int m = 0; m < 2; ++m) Pd[(half * 64 + t0 + i) * 16 + (s0 + m - 16 * j)] = acc[i][m];
+  }
+  __syncthreads();
+
+  // ---- wait for the MMAs, assemble P^T rows (key s) and store -------------
+  const bool ok = dev::mbar_wait(bar, 0, a.status);
+  dev::tc_fence_after();
+  if (warp < 4) {
+    const int s = 16 * warp + lane;  // valid for lane < 16
+    const int js = warp;             // sub-chunk of key s
+    float row[kC];
+#pragma unroll
+    for (int cb = 0; cb < 4; ++cb) dev::tmem_ld16(dev::tmem_addr(tmem, 32 * warp, 16 * cb), row + 16 * cb);
+    dev::tmem_wait_ld();
+    if (lane < 16) {
+      bf16 *dst = a.PT + ((bh * a.N + n) * kC + s) * kC;
+#pragma unroll
+      for (int t8 = 0; t8 < kC / 8; ++t8) {
+        float v8[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const int t = t8 * 8 + e;
+          const int jt = t >> 4;
+          float val = 0.f;
+          if (jt > js) val = ok ? row[t] : 0.f;
+          else if (jt == js && t >= s) val = Pd[t * 16 + (s - 16 * js)] + Pd[(64 + t) * 16 + (s - 16 * js)];
+          v8[e] = val;
+        }
+        uint4 pk;
+        pk.x = dev::pack_bf16(v8[0], v8[1]);
+        pk.y = dev::pack_bf16(v8[2], v8[3]);
+        pk.z = dev::pack_bf16(v8[4], v8[5]);
+        pk.w = dev::pack_bf16(v8[6], v8[7]);
+        *reinterpret_cast<uint4 *>(dst + t8 * 8) = pk;
+      }
+    }
+  }
+  dev::tc_fence_before();
+  __syncthreads();
+  if (warp == 0) dev::tmem_dealloc(tmem, 64);
+}
+
+// ============================================================================
+// Walk: per (d_v tile, segment, head); carries the fp32 state tile S (K x BV)
+// in TMEM across the chunks of one segment.  Per chunk n (forward):
+//     [state out]  h_n = S                       (bf16 via TMA, or fp32)
+//     [output]     O_n = qg_n S_bf16 + A_n V_n   (tcgen05, M = 64)
+//     S = diag(gam_n) S + kg_n^T V_n             (tcgen05, M = 128 per 128 key rows)
+// Reverse (adjoint) walks run the chunks backwards with (qg, dO) in place of
+// (kg, V): dS_{n-1} = diag(gam_n) dS_n + qg_n^T dO_n.
+// ============================================================================
+struct WalkArgs {
+  int T, N, V, L;  // L = chunks per segment
+  int reverse, do_out, state_mode;  // state_mode: 0 none, 1 bf16 (TMA store), 2 fp32
+  const float *gam;                 // [BH][N][K]
+  const float *start;               // [BH][P][K][V] fp32 or null
+  const float *h0;                  // used by segment 0 when start == null
+  float *end;                       // [BH][P][K][V] fp32 or null (state after the segment)
+  float *h32;                       // [BH][N][K][V] fp32 states (state_mode 2)
+  bf16 *out;                        // [BH][T][V]
+  unsigned *status;
+};
+
+template <int K, int BV>
+struct WalkSmem {
+  static constexpr int kTileX = 64 * K * 2;   // kg or qg chunk tile
+  static constexpr int kTileY = 64 * BV * 2;  // V or dO tile
+  static constexpr int kTileQ = 64 * K * 2;   // qg for the output
+  static constexpr int kTileP = 64 * 64 * 2;  // P^T
+  static constexpr int kStage = kTileX + kTileY + kTileQ + kTileP;
+  static constexpr int kSb = 2 * kStage;      // bf16 state tile [K][BV]
+  static constexpr int kBar = kSb + K * BV * 2;
+  static constexpr int kBytes = kBar + 64;
+};
+
+template <int K, int BV>
+__global__ void __launch_bounds__(K, 1)
+    k_walk(WalkArgs a, const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmY,
+           const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmP,
+           const __grid_constant__ CUtensorMap tmH) {
+  using L = WalkSmem<K, BV>;
+  constexpr int kThreads = K;
+  constexpr int kMB = K / 128;         // 128-row blocks of the state
+  constexpr int kColO = kMB * BV;      // TMEM column of the output accumulator
+  constexpr int kTmemCols = (kColO + BV <= 256) ? 256 : 512;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint64_t *full = (uint64_t *)(smem + L::kBar);
+  uint64_t *mma_bar = full + 2;
+  uint32_t *tslot = (uint32_t *)(full + 3);
+  const uint32_t sSb = dev::smem_u32(smem + L::kSb);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int vt = blockIdx.x, seg = blockIdx.y;
+  const long bh = blockIdx.z;
+  const int v0 = vt * BV;
+  const int n_begin = seg * a.L;
+  const int n_end = min(a.N, n_begin + a.L);
+  const int nloc = n_end - n_begin;
+  const int P = gridDim.y;
+
+  if (warp == 0) dev::tmem_alloc(tslot, kTmemCols);
+  if (tid == 0) {
+    dev::mbar_init(&full[0], 1);
+    dev::mbar_init(&full[1], 1);
+    dev::mbar_init(mma_bar, 1);
+    dev::fence_mbar_init();
+    dev::prefetch_tmap(&tmX);
+    dev::prefetch_tmap(&tmY);
+    if (a.do_out) {
+      dev::prefetch_tmap(&tmQ);
+      dev::prefetch_tmap(&tmP);
+    }
+  }
+  dev::tc_fence_before();
+  __syncthreads();
+  dev::tc_fence_after();
+  const uint32_t tmem = *tslot;
+
+  auto chunk_of = [&](int i) { return a.reverse ? (n_end - 1 - i) : (n_begin + i); };
+  auto stage_ptr = [&](int s) { return smem + s * L::kStage; };
+  const uint32_t tx_bytes = (uint32_t)(L::kTileX + L::kTileY + (a.do_out ? L::kTileQ + L::kTileP : 0));
+
+  auto issue_loads = [&](int i) {
+    const int s = i & 1;
+    const int n = chunk_of(i);
+    uint8_t *st = stage_ptr(s);
+    dev::mbar_arrive_expect_tx(&full[s], tx_bytes);
+#pragma unroll
+    for (int cb = 0; cb < K / 64; ++cb) dev::tma_load_3d(st + cb * 64 * 128, &tmX, cb * 64, n * kC, (int)bh, &full[s]);
+#pragma unroll
+    for (int cb = 0; cb < BV / 64; ++cb)
+      dev::tma_load_3d(st + L::kTileX + cb * 64 * 128, &tmY, v0 + cb * 64, n * kC, (int)bh, &full[s]);
+    if (a.do_out) {
+#pragma unroll
+      for (int cb = 0; cb < K / 64; ++cb)
+        dev::tma_load_3d(st + L::kTileX + L::kTileY + cb * 64 * 128, &tmQ, cb * 64, n * kC, (int)bh, &full[s]);
+      dev::tma_load_3d(st + L::kTileX + L::kTileY + L::kTileQ, &tmP, 0, 0, (int)(bh * a.N + n), &full[s]);
+    }
+  };
+
+  if (tid == 0 && nloc > 0) {
+    issue_loads(0);
+    if (nloc > 1) issue_loads(1);
+  }
+
+  // thread -> state row c; TMEM lane block of its warp
+  const int mb = warp >> 2;
+  const int c = tid;  // state row (key channel)
+  const uint32_t tS = dev::tmem_addr(tmem, 32 * (warp & 3), mb * BV);
+  const long KV = (long)K * a.V;
+
+  // ---- initial state into TMEM --------------------------------------------
+  {
+    const float *src = nullptr;
+    if (a.start) src = a.start + ((bh * P + seg) * K + c) * (long)a.V + v0;
+    else if (seg == 0 && a.h0) src = a.h0 + bh * KV + (long)c * a.V + v0;
+#pragma unroll
+    for (int cb = 0; cb < BV / 16; ++cb) {
+      float v[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) v[e] = src ? __ldg(src + cb * 16 + e) : 0.f;
+      dev::tmem_st16(tS + cb * 16, v);
+    }
+    dev::tmem_wait_st();
+  }
+
+  bool ok = true;
+  for (int i = 0; i < nloc; ++i) {
+    const int s = i & 1;
+    const int n = chunk_of(i);
+    uint8_t *st = stage_ptr(s);
+    const float g = __ldg(a.gam + (bh * a.N + n) * K + c);
+    if (ok) ok = dev::mbar_wait(&full[s], (i >> 1) & 1, a.status);
+
+    // ---- S-pass: read S, publish bf16/fp32 copy, scale by gamma ---------------
+#pragma unroll
+    for (int cb = 0; cb < BV / 16; ++cb) {
+      float v[16];
+      dev::tmem_ld16(tS + cb * 16, v);
+      dev::tmem_wait_ld();
+      if (a.do_out || a.state_mode == 1) {
+        const uint32_t w0 = dev::pack_bf16(v[0], v[1]), w1 = dev::pack_bf16(v[2], v[3]);
+        const uint32_t w2 = dev::pack_bf16(v[4], v[5]), w3 = dev::pack_bf16(v[6], v[7]);
+        const uint32_t w4 = dev::pack_bf16(v[8], v[9]), w5 = dev::pack_bf16(v[10], v[11]);
+        const uint32_t w6 = dev::pack_bf16(v[12], v[13]), w7 = dev::pack_bf16(v[14], v[15]);
+        dev::st_shared_v4(sSb + dev::sw128_chunk(K, c, cb * 2), w0, w1, w2, w3);
+        dev::st_shared_v4(sSb + dev::sw128_chunk(K, c, cb * 2 + 1), w4, w5, w6, w7);
+      }
+      if (a.state_mode == 2) {
+        float4 *dst = reinterpret_cast<float4 *>(a.h32 + ((bh * a.N + n) * K + c) * (long)a.V + v0 + cb * 16);
+        dst[0] = make_float4(v[0], v[1], v[2], v[3]);
+        dst[1] = make_float4(v[4], v[5], v[6], v[7]);
+        dst[2] = make_float4(v[8], v[9], v[10], v[11]);
+        dst[3] = make_float4(v[12], v[13], v[14], v[15]);
+      }
+#pragma unroll
+      for (int e = 0; e < 16; ++e) v[e] *= g;
+      dev::tmem_st16(tS + cb * 16, v);
+    }
+    dev::tmem_wait_st();
+    dev::fence_proxy_async_smem();
+    dev::tc_fence_before();
+    __syncthreads();
+    dev::tc_fence_after();
+
+    // ---- MMA issue ---------------------------------------------------------
+    if (tid == 0 && ok) {
+      const uint32_t sX = dev::smem_u32(st);
+      const uint32_t sY = sX + L::kTileX;
+      const uint32_t sQ = sY + L::kTileY;
+      const uint32_t sP = sQ + L::kTileQ;
+      if (a.do_out) {
+        constexpr uint32_t id_qs = dev::idesc_bf16(64, BV, false, true);
+#pragma unroll
+        for (int kk = 0; kk < K / 16; ++kk)
+          dev::umma_bf16(tmem + kColO, dev::desc_kmajor(sQ, 64, 0, kk * 16), dev::desc_mnmajor(sSb, K, kk * 16, 0),
+                         id_qs, kk > 0 ? 1u : 0u);
+        constexpr uint32_t id_pv = dev::idesc_bf16(64, BV, true, true);
+#pragma unroll
+        for (int kk = 0; kk < kC / 16; ++kk)
+          dev::umma_bf16(tmem + kColO, dev::desc_mnmajor(sP, 64, kk * 16, 0), dev::desc_mnmajor(sY, 64, kk * 16, 0),
+                         id_pv, 1u);
+      }
+      constexpr uint32_t id_st = dev::idesc_bf16(128, BV, true, true);
+#pragma unroll
+      for (int m = 0; m < kMB; ++m)
+#pragma unroll
+        for (int kk = 0; kk < kC / 16; ++kk)
+          dev::umma_bf16(tmem + m * BV, dev::desc_mnmajor(sX, 64, kk * 16, 128 * m),
+                         dev::desc_mnmajor(sY, 64, kk * 16, 0), id_st, 1u);
+      dev::umma_commit(mma_bar);
+      if (a.state_mode == 1) {
+#pragma unroll
+        for (int cb = 0; cb < BV / 64; ++cb)
+          dev::tma_store_3d(&tmH, smem + L::kSb + cb * K * 128, v0 + cb * 64, 0, (int)(bh * a.N + n));
+        dev::tma_store_commit();
+      }
+    }
+    if (ok) ok = dev::mbar_wait(mma_bar, i & 1, a.status);
+    dev::tc_fence_after();
+    if (tid == 0 && ok && i + 2 < nloc) issue_loads(i + 2);
+
+    // ---- output epilogue -----------------------------------------------------
+    if (a.do_out) {
+      constexpr int kWarps = kThreads / 32;
+      constexpr int kColsPerWarp = (kWarps >= 8) ? BV / 2 : BV;
+      const int sub = warp & 3;
+      const int col0 = (kWarps >= 8 && warp >= 4) ? BV / 2 : 0;
+      const int t = 16 * sub + lane;
+      const long tgl = (long)n * kC + t;
+#pragma unroll
+      for (int cb = 0; cb < kColsPerWarp / 16; ++cb) {
+        float v[16];
+        dev::tmem_ld16(dev::tmem_addr(tmem, 32 * sub, kColO + col0 + cb * 16), v);
+        dev::tmem_wait_ld();
+        if (lane < 16 && tgl < a.T && ok) {
+          uint4 p0, p1;
+          p0.x = dev::pack_bf16(v[0], v[1]);
+          p0.y = dev::pack_bf16(v[2], v[3]);
+          p0.z = dev::pack_bf16(v[4], v[5]);
+          p0.w = dev::pack_bf16(v[6], v[7]);
+          p1.x = dev::pack_bf16(v[8], v[9]);
+          p1.y = dev::pack_bf16(v[10], v[11]);
+          p1.z = dev::pack_bf16(v[12], v[13]);
+          p1.w = dev::pack_bf16(v[14], v[15]);
+          uint4 *dst = reinterpret_cast<uint4 *>(a.out + (bh * a.T + tgl) * (long)a.V + v0 + col0 + cb * 16);
+          dst[0] = p0;
+          dst[1] = p1;
+        }
+      }
+    }
+    if (a.state_mode == 1 && tid == 0) dev::tma_store_wait_read();
+    dev::tc_fence_before();
+    __syncthreads();
+    dev::tc_fence_after();
+  }
+
+  // ---- final state of the segment ---------------------------------------------
+  if (a.end) {
+    float *dst = a.end + ((bh * P + seg) * K + c) * (long)a.V + v0;
+#pragma unroll
+    for (int cb = 0; cb < BV / 16; ++cb) {
+      float v[16];
+      dev::tmem_ld16(tS + cb * 16, v);
+      dev::tmem_wait_ld();
+      float4 *d4 = reinterpret_cast<float4 *>(dst + cb * 16);
+      d4[0] = make_float4(v[0], v[1], v[2], v[3]);
+      d4[1] = make_float4(v[4], v[5], v[6], v[7]);
+      d4[2] = make_float4(v[8], v[9], v[10], v[11]);
+      d4[3] = make_float4(v[12], v[13], v[14], v[15]);
+    }
+  }
+  if (a.state_mode == 1 && tid == 0) dev::tma_store_wait_all();
+  dev::tc_fence_before();
+  __syncthreads();
+  if (warp == 0) dev::tmem_dealloc(tmem, kTmemCols);
+}
+
+// ============================================================================
+// Scan over segments (elementwise over the K x V state, sequential over P):
+//   start[p] = S;  S = diag(prod_{n in p} gam_n) S + delta[p]
+// run forwards from h0 (forward pass) or backwards from dh_final (adjoint).
+// ============================================================================
+struct ScanArgs {
+  int K, V, N, L, P, reverse;
+  const float *gam, *delta, *init;
+  float *start, *final_out;
+};
+
+__global__ void k_scan(ScanArgs a) {
+  const long idx = (long)blockIdx.x * blockDim.x + threadIdx.x;
+  const long KV = (long)a.K * a.V;
+  const long bh = blockIdx.y;
+  if (idx >= KV) return;
+  const int c = (int)(idx / a.V);
+  float S = a.init ? a.init[bh * KV + idx] : 0.f;
+  for (int pi = 0; pi < a.P; ++pi) {
+    const int p = a.reverse ? a.P - 1 - pi : pi;
+    a.start[(bh * a.P + p) * KV + idx] = S;
+    const int nb = p * a.L, ne = min(a.N, nb + a.L);
+    float gs = 1.f;
+    for (int n = nb; n < ne; ++n) gs *= a.gam[(bh * a.N + n) * a.K + c];
+    S = gs * S + a.delta[(bh * a.P + p) * KV + idx];
+  }
+  if (a.final_out) a.final_out[bh * KV + idx] = S;
+}
+
+}  // namespace tc
+}  // namespace gla

@@ -1,16 +1,355 @@
-// tc_path.cu -- bf16 path entry points (temporary: CUDA-core kernels).
+// tc_path.cu -- host orchestration of the bf16 tensor-core path (sm_100a).
+//
+// Forward (section 4.2 chunkwise form, section 3.3 Figure 1 variants):
+//   prep                      qg, kg, gam, P^T per chunk (parallel over chunks)
+//   FUSED, P segments:        walk(no output) per segment from 0 -> delta_p,
+//                             scan -> segment start states and h_final,
+//                             walk(output) per segment from its start state
+//                             (P = 1: a single walk from h0 that also writes h_final)
+//   MATERIALIZED:             walk(fp32 chunk states) over whole sequences, then
+//                             walk(output, one chunk per CTA) from those states.
+// Backward: see tc_bwd.
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "tc_bwd.cuh"
+#include "tc_kernels.cuh"
 #include "tc_path.h"
 
 namespace gla {
-int tc_check(const Problem &p) { (void)p; return GLA_OK; }
-size_t tc_workspace(const Problem &p, bool bwd) { return f32_workspace(p, bwd); }
-int tc_fwd(const Problem &p, const void *q, const void *k, const void *v, const float *la, const float *h0,
-           void *o, float *hT, void *ws, cudaStream_t st) {
-  return f32_fwd(p, q, k, v, la, h0, o, hT, ws, st);
+namespace {
+
+using tc::bf16;
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = (PFN_cuTensorMapEncodeTiled_v12000)p;
+  });
+  return fn;
 }
+
+// 3-D bf16 tensor map: dims (d0 innermost, d1, d2), box (b0, b1, 1), 128-byte swizzle.
+bool map3(CUtensorMap *m, const void *base, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t b0, uint32_t b1) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {d0 * 2, d0 * d1 * 2};
+  cuuint32_t box[3] = {b0, b1, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+bool tc::map3_bf16(CUtensorMap *m, const void *base, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t b0, uint32_t b1) {
+  return map3(m, base, d0, d1, d2, b0, b1);
+}
+
+namespace {
+
+int device_ok() {
+  static int state = -1;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    int dev = 0, major = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+      state = 0;
+    else
+      state = (major == 10) ? 1 : 0;
+  });
+  return state;
+}
+
+int sm_count() {
+  static int n = 0;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  });
+  return n;
+}
+
+int bv_of(const Problem &p) { return (p.K == 256 || p.V % 128 != 0) ? 64 : 128; }
+
+// Segment count for the FUSED forward: enough CTAs to cover the SMs once.
+int segments_of(const Problem &p, int nvt) {
+  if (p.variant == GLA_VARIANT_MATERIALIZED) return 1;
+  int P = p.segments;
+  if (P <= 0) {
+    const long ctas = p.BH * nvt;
+    P = (int)std::max<long>(1, (sm_count() + ctas - 1) / ctas);
+  }
+  P = std::min(P, p.N);
+  const int L = (p.N + P - 1) / P;
+  return (p.N + L - 1) / L;
+}
+
+struct TcWs {
+  bf16 *qg, *kg, *PT;
+  float *gam;
+  float *delta, *start;  // [BH][P][K][V]
+  float *h32;            // materialised fp32 chunk states [BH][N][K][V]
+  // backward
+  bf16 *hb, *dhb;        // bf16 chunk states and adjoints [BH][N][K][V]
+  float *dstart, *ddelta;
+  float *dscratch;       // bwd per-chunk scratch
+  size_t bytes;
+};
+
+TcWs carve(const Problem &p, void *ws, bool bwd) {
+  Carve cv(ws);
+  TcWs w{};
+  const int nvt = p.V / bv_of(p);
+  w.qg = cv.take<bf16>((size_t)p.BH * p.Tp * p.K);
+  w.kg = cv.take<bf16>((size_t)p.BH * p.Tp * p.K);
+  w.PT = cv.take<bf16>((size_t)p.BH * p.N * tc::kC * tc::kC);
+  w.gam = cv.take<float>((size_t)p.BH * p.N * p.K);
+  if (!bwd) {
+    const int P = segments_of(p, nvt);
+    if (p.variant == GLA_VARIANT_MATERIALIZED) {
+      w.h32 = cv.take<float>((size_t)p.BH * p.N * p.K * p.V);
+    } else if (P > 1) {
+      w.delta = cv.take<float>((size_t)p.BH * P * p.K * p.V);
+      w.start = cv.take<float>((size_t)p.BH * P * p.K * p.V);
+    }
+  } else {
+    Problem pf = p;
+    pf.variant = GLA_VARIANT_FUSED;
+    pf.segments = 0;
+    const int P = segments_of(pf, nvt);
+    w.delta = cv.take<float>((size_t)p.BH * P * p.K * p.V);
+    w.start = cv.take<float>((size_t)p.BH * P * p.K * p.V);
+    w.ddelta = cv.take<float>((size_t)p.BH * P * p.K * p.V);
+    w.dstart = cv.take<float>((size_t)p.BH * P * p.K * p.V);
+    w.hb = cv.take<bf16>((size_t)p.BH * p.N * p.K * p.V);
+    w.dhb = cv.take<bf16>((size_t)p.BH * p.N * p.K * p.V);
+    w.dscratch = cv.take<float>(tc::bwd_scratch_floats(p.BH, p.N, p.K, p.V));
+  }
+  w.bytes = cv.bytes();
+  return w;
+}
+
+template <int K>
+int launch_prep(const Problem &p, const bf16 *q, const bf16 *k, const float *la, const TcWs &w, unsigned *status,
+                cudaStream_t st) {
+  tc::PrepArgs a{p.T, p.N, p.gate, p.Tp, q, k, la, w.qg, w.kg, w.PT, w.gam, status};
+  const int smem = tc::PrepSmem<K>::kBytes + 1024;
+  static bool attr = false;
+  if (!attr) {
+    if (cudaFuncSetAttribute(tc::k_prep<K>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+      return GLA_ERR_CUDA;
+    attr = true;
+  }
+  GLA_LAUNCH(K_TC_PREP, st, (tc::k_prep<K><<<dim3(p.N, p.BH), 256, smem, st>>>(a)));
+  return GLA_OK;
+}
+
+struct WalkMaps {
+  CUtensorMap X, Y, Q, P, H;
+};
+
+template <int K, int BV>
+int launch_walk(const Problem &p, const tc::WalkArgs &a, const WalkMaps &m, int P, cudaStream_t st) {
+  const int smem = tc::WalkSmem<K, BV>::kBytes + 1024;
+  static bool attr = false;
+  if (!attr) {
+    if (cudaFuncSetAttribute(tc::k_walk<K, BV>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+      return GLA_ERR_CUDA;
+    attr = true;
+  }
+  GLA_LAUNCH(K_TC_WALK, st,
+             (tc::k_walk<K, BV><<<dim3(p.V / BV, P, p.BH), K, smem, st>>>(a, m.X, m.Y, m.Q, m.P, m.H)));
+  return GLA_OK;
+}
+
+int launch_walk_any(const Problem &p, const tc::WalkArgs &a, const WalkMaps &m, int P, cudaStream_t st) {
+  const int BV = bv_of(p);
+  if (p.K == 256 && BV == 64) return launch_walk<256, 64>(p, a, m, P, st);
+  if (p.K == 128 && BV == 128) return launch_walk<128, 128>(p, a, m, P, st);
+  if (p.K == 128 && BV == 64) return launch_walk<128, 64>(p, a, m, P, st);
+  return GLA_ERR_UNSUPPORTED_SHAPE;
+}
+
+int launch_scan(const Problem &p, const float *gam, const float *delta, const float *init, float *start,
+                float *final_out, int P, int L, int reverse, cudaStream_t st) {
+  tc::ScanArgs a{p.K, p.V, p.N, L, P, reverse, gam, delta, init, start, final_out};
+  const long KV = (long)p.K * p.V;
+  GLA_LAUNCH(K_TC_SCAN, st, (tc::k_scan<<<dim3((unsigned)((KV + 255) / 256), p.BH), 256, 0, st>>>(a)));
+  return GLA_OK;
+}
+
+int launch_prep_any(const Problem &p, const bf16 *q, const bf16 *k, const float *la, const TcWs &w, unsigned *status,
+                    cudaStream_t st) {
+  if (p.K == 256) return launch_prep<256>(p, q, k, la, w, status, st);
+  return launch_prep<128>(p, q, k, la, w, status, st);
+}
+
+#define TRY(x)                      \
+  do {                              \
+    const int _r = (x);             \
+    if (_r != GLA_OK) return _r;    \
+  } while (0)
+
+}  // namespace
+
+int tc_check(const Problem &p) {
+  if (p.K != 128 && p.K != 256) return GLA_ERR_UNSUPPORTED_SHAPE;
+  if (p.V % 64 != 0) return GLA_ERR_UNSUPPORTED_SHAPE;
+  if (p.C != 64 || p.c != 16) return GLA_ERR_UNSUPPORTED_SHAPE;
+  return GLA_OK;
+}
+
+size_t tc_workspace(const Problem &p, bool bwd) { return carve(p, nullptr, bwd).bytes; }
+
+int tc_fwd(const Problem &p, const void *q, const void *k, const void *v, const float *la, const float *h0, void *o,
+           float *hT, void *ws, cudaStream_t st) {
+  if (device_ok() != 1) return GLA_ERR_NO_DEVICE;
+  TcWs w = carve(p, ws, false);
+  unsigned *status = (unsigned *)ws;
+  TRY(launch_prep_any(p, (const bf16 *)q, (const bf16 *)k, la, w, status, st));
+
+  const int BV = bv_of(p);
+  const int nvt = p.V / BV;
+  WalkMaps m;
+  const uint64_t BH = (uint64_t)p.BH;
+  bool okm = map3(&m.X, w.kg, p.K, p.Tp, BH, 64, 64) && map3(&m.Y, v, p.V, p.T, BH, 64, 64) &&
+             map3(&m.Q, w.qg, p.K, p.Tp, BH, 64, 64) && map3(&m.P, w.PT, 64, 64, BH * p.N, 64, 64);
+  m.H = m.X;
+  if (!okm) return GLA_ERR_CUDA;
+
+  tc::WalkArgs a{};
+  a.T = p.T;
+  a.N = p.N;
+  a.V = p.V;
+  a.gam = w.gam;
+  a.out = (bf16 *)o;
+  a.status = status;
+
+  if (p.variant == GLA_VARIANT_MATERIALIZED) {
+    // pass 1: all chunk states in fp32 (sequential over chunks per (head, d_v tile))
+    a.L = p.N;
+    a.state_mode = 2;
+    a.h32 = w.h32;
+    a.h0 = h0;
+    a.end = hT;
+    TRY(launch_walk_any(p, a, m, 1, st));
+    // pass 2: every chunk's output in parallel from its materialised state
+    tc::WalkArgs b = a;
+    b.L = 1;
+    b.state_mode = 0;
+    b.do_out = 1;
+    b.start = w.h32;
+    b.h0 = nullptr;
+    b.end = nullptr;
+    return launch_walk_any(p, b, m, p.N, st);
+  }
+
+  const int P = segments_of(p, nvt);
+  const int L = (p.N + P - 1) / P;
+  a.L = L;
+  if (P == 1) {
+    a.do_out = 1;
+    a.h0 = h0;
+    a.end = hT;
+    return launch_walk_any(p, a, m, 1, st);
+  }
+  // pre-pass: each segment's contribution from a zero state
+  tc::WalkArgs pre = a;
+  pre.end = w.delta;
+  TRY(launch_walk_any(p, pre, m, P, st));
+  TRY(launch_scan(p, w.gam, w.delta, h0, w.start, hT, P, L, 0, st));
+  a.do_out = 1;
+  a.start = w.start;
+  return launch_walk_any(p, a, m, P, st);
+}
+
 int tc_bwd(const Problem &p, const void *q, const void *k, const void *v, const float *la, const float *h0,
            const void *dout, const float *dhT, void *dq, void *dk, void *dv, float *dla, float *dh0, void *ws,
            cudaStream_t st) {
-  return f32_bwd(p, q, k, v, la, h0, dout, dhT, dq, dk, dv, dla, dh0, ws, st);
+  if (device_ok() != 1) return GLA_ERR_NO_DEVICE;
+  TcWs w = carve(p, ws, true);
+  unsigned *status = (unsigned *)ws;
+  TRY(launch_prep_any(p, (const bf16 *)q, (const bf16 *)k, la, w, status, st));
+  const int BV = bv_of(p);
+  const int nvt = p.V / BV;
+  Problem pf = p;
+  pf.variant = GLA_VARIANT_FUSED;
+  pf.segments = 0;
+  const int P = segments_of(pf, nvt);
+  const int L = (p.N + P - 1) / P;
+  const uint64_t BH = (uint64_t)p.BH;
+
+  // ---- chunk states h_n (bf16), recomputed ------------------------------------
+  WalkMaps mf;
+  bool okm = map3(&mf.X, w.kg, p.K, p.Tp, BH, 64, 64) && map3(&mf.Y, v, p.V, p.T, BH, 64, 64) &&
+             map3(&mf.H, w.hb, p.V, p.K, BH * p.N, 64, p.K);
+  mf.Q = mf.X;
+  mf.P = mf.X;
+  // ---- chunk adjoints dh_n (bf16) -----------------------------------------------
+  WalkMaps mr;
+  okm = okm && map3(&mr.X, w.qg, p.K, p.Tp, BH, 64, 64) && map3(&mr.Y, dout, p.V, p.T, BH, 64, 64) &&
+        map3(&mr.H, w.dhb, p.V, p.K, BH * p.N, 64, p.K);
+  mr.Q = mr.X;
+  mr.P = mr.X;
+  if (!okm) return GLA_ERR_CUDA;
+
+  tc::WalkArgs a{};
+  a.T = p.T;
+  a.N = p.N;
+  a.V = p.V;
+  a.L = L;
+  a.gam = w.gam;
+  a.status = status;
+  if (P > 1) {
+    tc::WalkArgs pre = a;
+    pre.end = w.delta;
+    TRY(launch_walk_any(p, pre, mf, P, st));
+    TRY(launch_scan(p, w.gam, w.delta, h0, w.start, nullptr, P, L, 0, st));
+    a.start = w.start;
+  } else {
+    a.h0 = h0;
+  }
+  a.state_mode = 1;
+  TRY(launch_walk_any(p, a, mf, P, st));
+
+  tc::WalkArgs r{};
+  r.T = p.T;
+  r.N = p.N;
+  r.V = p.V;
+  r.L = L;
+  r.reverse = 1;
+  r.gam = w.gam;
+  r.status = status;
+  if (P > 1) {
+    tc::WalkArgs pre = r;
+    pre.end = w.ddelta;
+    TRY(launch_walk_any(p, pre, mr, P, st));
+    TRY(launch_scan(p, w.gam, w.ddelta, dhT, w.dstart, dh0, P, L, 1, st));
+    r.start = w.dstart;
+  } else {
+    r.h0 = dhT;
+    r.end = dh0;
+  }
+  r.state_mode = 1;
+  TRY(launch_walk_any(p, r, mr, P, st));
+
+  // ---- per-chunk gradients --------------------------------------------------------
+  return tc::launch_bwd_main(p, (const bf16 *)q, (const bf16 *)k, (const bf16 *)v, la, (const bf16 *)dout,
+                             (bf16 *)dq, (bf16 *)dk, (bf16 *)dv, dla, w.qg, w.kg, w.PT, w.gam, w.hb, w.dhb,
+                             w.dscratch, status, st);
 }
+
 }  // namespace gla
