@@ -1,0 +1,359 @@
+"""Benchmark: chunkwise GLA forward + backward on B200 (one process per GPU).
+
+One step = gla_fwd + gla_bwd over one batch of the 1.3B-layer workload
+(B=2, H=4, T=4096, d_k=256, d_v=512, bf16, vector gates with z ~ N(-1,1)),
+inputs resident in HBM.  Prints one JSON line (rank 0).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+For N > 1 launch with torchrun; every rank runs its own replica of the workload
+(weak scaling, no collective on the data path).  --impl reference times the
+float64 CPU oracle (the only reference implementation) on a bounded sample.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "GLA fwd+bwd tokens/s and TFLOP/s vs T; % of B200 bf16 tensor peak / HBM BW"
+WORKLOAD = dict(B=2, H=4, T=4096, K=256, V=512, C=64, z_mean=-1.0, gate="vector")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "sm_max_mhz": 1965.0}
+
+
+def counted_flops(B, H, T, K, V, C):
+    """Contraction FLOPs per step (fwd 4KV + C(K+V), bwd 10KV + C(3K+2V) per token-head)."""
+    th = B * H * T
+    return th * (4 * K * V + C * (K + V)) + th * (10 * K * V + C * (3 * K + 2 * V))
+
+
+def algorithmic_bytes(B, H, T, K, V, gate="vector"):
+    """Inputs + outputs of fwd and bwd (bf16 q,k,v,o,do,dq,dk,dv; fp32 gates; no states)."""
+    th = B * H * T
+    g = 4 * K if gate == "vector" else (4 if gate == "scalar" else 0)
+    fwd = th * (2 * K + 2 * K + 2 * V + g + 2 * V)
+    bwd = th * (2 * K + 2 * K + 2 * V + g + 2 * V + 2 * K + 2 * K + 2 * V + g)
+    return fwd + bwd
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return None
+        busy = [x for x in sm if x > 0.5 * (smax or 1)] or sm
+        return {"sm_mhz": statistics.median(busy), "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+# ----------------------------------------------------------------------------------- oracle
+def oracle_sample_rate(w, T_sample=1024, seed=0):
+    """Time the float64 oracle (fwd + BPTT bwd) on all heads of the workload for the
+    first T_sample tokens; returns (tokens/s, seconds, threads, description)."""
+    import torch
+
+    from chunkwise_linear_rnn_fwd_b200.synth import make_inputs
+    from oracle import oracle
+
+    x = make_inputs(w["B"], w["H"], T_sample, w["K"], w["V"], dtype=torch.bfloat16, gate=w["gate"], seed=seed,
+                    z_mean=w["z_mean"])
+    f = lambda a: None if a is None else a.double().numpy()
+    q, k, v, la, do = f(x.q), f(x.k), f(x.v), f(x.log_alpha), f(x.do)
+    oracle.build()
+    t0 = time.perf_counter()
+    oracle.fwd(q, k, v, la, gate=w["gate"])
+    oracle.bwd(q, k, v, la, do, gate=w["gate"])
+    dt = time.perf_counter() - t0
+    threads = min(oracle.threads(), w["B"] * w["H"])
+    desc = (f"fwd+bwd of all {w['B'] * w['H']} heads over the first {T_sample} of {w['T']} tokens "
+            f"(d_k={w['K']}, d_v={w['V']}), float64, OpenMP over heads")
+    return w["B"] * T_sample / dt, dt, threads, desc
+
+
+def run_reference(args, w):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    for _ in range(args.warmup):
+        oracle_sample_rate(w, T_sample=args.ref_tokens)
+    rates, secs = [], 0.0
+    threads, desc = 1, ""
+    for _ in range(args.steps):
+        r, dt, threads, desc = oracle_sample_rate(w, T_sample=args.ref_tokens)
+        rates.append(r)
+        secs += dt
+    value = statistics.median(rates)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / max(1, args.steps),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "gla fwd+bwd, B=2 H=4 T=4096 d_k=256 d_v=512, vector gates z~N(-1,1)",
+                   "sample": desc},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": desc},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------------------------ ours
+def kernel_io_bytes(name, w):
+    """Bytes a launch of `name` must move at minimum (its own inputs + outputs, once)."""
+    B, H, T, K, V, C = w["B"], w["H"], w["T"], w["K"], w["V"], w["C"]
+    BH, N = B * H, -(-T // C)
+    Tp = N * C
+    g = 4 * K if w["gate"] == "vector" else (4 if w["gate"] == "scalar" else 0)
+    if name == "tc_prep":
+        return BH * T * (2 * K + 2 * K + g) + BH * Tp * 2 * (2 * K) + BH * N * (4 * K + 2 * C * C)
+    if name == "tc_bwd":
+        return (BH * N * K * V * 2 * 2 + BH * T * (2 * V * 2 + 2 * K * 2 + g) + BH * Tp * 2 * K
+                + BH * N * 2 * C * C + BH * T * (2 * K * 2 + 2 * V + g))
+    return None
+
+
+def run_ours(args, w):
+    import torch
+    import torch.distributed as dist
+
+    import chunkwise_linear_rnn_fwd_b200 as pkg
+    from chunkwise_linear_rnn_fwd_b200.synth import make_inputs
+
+    rank, world, local = dist_env()
+    if world > 1:
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pkg.load()
+
+    B, H, T, K, V, C = w["B"], w["H"], w["T"], w["K"], w["V"], w["C"]
+    x = make_inputs(B, H, T, K, V, dtype=torch.bfloat16, gate=w["gate"], seed=rank, z_mean=w["z_mean"])
+    q, k, v, la, do = (t.to(dev) for t in (x.q, x.k, x.v, x.log_alpha, x.do))
+    o = torch.empty(B, H, T, V, dtype=torch.bfloat16, device=dev)
+    hT = torch.empty(B, H, K, V, dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    dla = torch.empty_like(la)
+    ws_f = pkg.alloc_workspace(pkg.workspace_size(B, H, T, K, V, torch.bfloat16, w["gate"], C, False), dev)
+    ws_b = pkg.alloc_workspace(pkg.workspace_size(B, H, T, K, V, torch.bfloat16, w["gate"], C, True), dev)
+    stream = torch.cuda.current_stream()
+
+    def step(qq=q, kk=k, vv=v, ll=la, dd=do):
+        pkg.gla_fwd(qq, kk, vv, ll, None, chunk=C, o=o, h_final=hT, workspace=ws_f, stream=stream)
+        pkg.gla_bwd(qq, kk, vv, ll, dd, None, None, chunk=C, dq=dq, dk=dk, dv=dv, dlog_alpha=dla, want_dh0=False,
+                    workspace=ws_b, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+
+    # ---- timed region: K steps, device events, per-kernel events for the roofline ----
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    pkg.timing_enable(True)
+    pkg.timing_collect()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ms_local = e0.elapsed_time(e1)
+    launches = pkg.timing_collect()
+    pkg.timing_enable(False)
+    clocks = sampler.stop()
+    ms = ms_local
+    if world > 1:
+        t = torch.tensor([ms_local], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_per_step = ms / args.steps
+    tokens = B * T * world * args.steps
+    value = tokens / (ms / 1e3)
+
+    # ---- end to end through the public API with host buffers ----------------------------
+    pin = lambda t: t.cpu().pin_memory()
+    hq, hk, hv, hla, hdo = pin(x.q), pin(x.k), pin(x.v), pin(x.log_alpha), pin(x.do)
+    ho = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    hdq, hdk, hdv = (torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (dq, dk, dv))
+    hdla = torch.empty(dla.shape, dtype=dla.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hla, hdo))
+    d2h = sum(t.numel() * t.element_size() for t in (ho, hdq, hdk, hdv, hdla))
+
+    def e2e_step():
+        for dst, src in ((q, hq), (k, hk), (v, hv), (la, hla), (do, hdo)):
+            dst.copy_(src, non_blocking=True)
+        step()
+        for dst, src in ((ho, o), (hdq, dq), (hdk, dk), (hdv, dv), (hdla, dla)):
+            dst.copy_(src, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    n_e2e = max(1, args.steps // 2)
+    for _ in range(n_e2e):
+        e2e_step()
+    f1.record(stream)
+    torch.cuda.synchronize()
+    ems = f0.elapsed_time(f1)
+    if world > 1:
+        t = torch.tensor([ems], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ems = float(t.item())
+    e2e_value = B * T * world * n_e2e / (ems / 1e3)
+
+    # ---- roofline of the dominant kernel --------------------------------------------------
+    peaks, peak_src = load_peaks()
+    per_kernel = {}
+    for name, t in launches:
+        d = per_kernel.setdefault(name, [0, 0.0])
+        d[0] += 1
+        d[1] += t
+    dom = max(per_kernel.items(), key=lambda kv: kv[1][1])[0] if per_kernel else None
+    roofline = None
+    if dom is not None:
+        n_l, tot = per_kernel[dom]
+        avg_ms = tot / n_l
+        io = kernel_io_bytes(dom, w)
+        if io is not None:
+            achieved = io / (avg_ms / 1e3) / 1e9
+            peak = float(peaks["hbm_gbs"])
+            roofline = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peak, "unit": "GB/s",
+                        "frac": achieved / peak, "traffic": None, "peak_source": peak_src,
+                        "bytes_per_launch": io, "avg_launch_ms": avg_ms}
+    flops = counted_flops(B, H, T, K, V, C)
+    abytes = algorithmic_bytes(B, H, T, K, V, w["gate"])
+    t_tensor = flops / (float(peaks.get("bf16_tflops", 1590)) * 1e12)
+    t_hbm = abytes / (float(peaks["hbm_gbs"]) * 1e9)
+    step_s = ms_per_step / 1e3
+    step_roofline = {
+        "bound": "hbm" if t_hbm >= t_tensor else "tensor", "tflops": flops / step_s / 1e12,
+        "frac_of_tensor_peak": (flops / step_s) / (float(peaks.get("bf16_tflops", 1590)) * 1e12),
+        "gbs_algorithmic": abytes / step_s / 1e9, "frac_of_roofline": max(t_hbm, t_tensor) / step_s,
+        "flops_per_step": flops, "algorithmic_bytes_per_step": abytes, "peak_source": peak_src,
+    }
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        r, dt, threads, desc = oracle_sample_rate(w, T_sample=args.ref_tokens)
+        cpu = {"value": r, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": desc, "seconds": dt}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "gla fwd+bwd, B=2 H=4 T=4096 d_k=256 d_v=512 C=64, bf16, vector gates "
+                                   "z~N(-1,1), fp32 state",
+                       "global_batch": B * world, "seq_len": T, "parallelism": f"replicas x{world}",
+                       "l2": "inputs larger than L2 (~268 MB touched per step)"},
+            "tflops": step_roofline["tflops"], "step_roofline": step_roofline, "roofline": roofline,
+            "kernels": {k2: {"launches": v2[0], "ms_total": v2[1], "share": v2[1] / max(1e-9, sum(x[1] for x in per_kernel.values()))}
+                        for k2, v2 in sorted(per_kernel.items(), key=lambda kv: -kv[1][1])},
+            "gpu_launches": len(launches),
+            "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "clocks": clocks, "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--ref-tokens", type=int, default=1024, help="tokens per head in the oracle sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    w = dict(WORKLOAD)
+    if args.impl == "reference":
+        return run_reference(args, w)
+    return run_ours(args, w)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

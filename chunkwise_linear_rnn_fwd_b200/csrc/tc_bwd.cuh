@@ -8,9 +8,13 @@
 //     dqh^T = h_n dO^T          dkh^T = dh_n V^T         dP = dO V^T
 //     dv    = kg dh_n + P^T dO  (stored per tile)
 //     R[c]  = sum_v h_n[c,v] dh_n[c,v]
-//   phase 2 (intra-chunk, sub-chunk reference points, all on tcgen05):
-//     dq_intra[t] = u_t (.) sum_{s<=t} dP[t,s] k_s e^{z_j(t) - B_s}
-//     dk_intra[s] = w_s (.) sum_{t>=s} dP[t,s] q_t e^{B_t - z_j(s)+1}
+//   phase 2 (intra-chunk, secondary chunking):
+//     strictly-lower sub-chunk blocks on tcgen05 with reference points
+//       dq_off[t] = u_t (.) sum_{s in earlier sub-chunks} dP[t,s] k_s e^{z_j(t) - B_s}
+//       dk_off[s] = w_s (.) sum_{t in later sub-chunks}  dP[t,s] q_t e^{B_t - z_j(s)+1}
+//     diagonal 16 x 16 blocks in fp32 on CUDA cores (one thread per key channel),
+//       with the same fp32 pair factor q_t k_s e^{B_t - B_s} on the dq and the dk
+//       side, so the pair terms cancel exactly in the closed-form gate gradient
 //   epilogue per key channel:
 //     dq = e^{B} (.) dqh + dq_intra ,  dk = e^{B_63 - B} (.) dkh + dk_intra
 //     dlog b_t = q_t dq_t - k_t dk_t                       (section 4.3)
@@ -50,12 +54,13 @@ struct BwdSmem {
   static constexpr int kPT = kKg + 64 * K * 2;             // P^T tile [64][64]
   static constexpr int kPhase1End = kPT + 64 * 64 * 2;
   // phase 2 (aliases the phase-1 stages)
-  static constexpr int kRowsW = 160;
-  static constexpr int kKh = 0;                            // key windows  [160][K]
-  static constexpr int kQh = kKh + kRowsW * K * 2;         // query windows [160][K]
-  static constexpr int kdP = kQh + kRowsW * K * 2;         // masked dP  [t][s]
-  static constexpr int kdPT = kdP + 64 * 64 * 2;           // masked dP^T [s][t]
-  static constexpr int kPhase2End = kdPT + 64 * 64 * 2;
+  static constexpr int kRowsW = 96;
+  static constexpr int kKh = 0;                            // key windows  [96][K]
+  static constexpr int kQh = kKh + kRowsW * K * 2;         // query windows [96][K]
+  static constexpr int kdP = kQh + kRowsW * K * 2;         // dP, strictly-lower blocks  [t][s]
+  static constexpr int kdPT = kdP + 64 * 64 * 2;           // the same, transposed [s][t]
+  static constexpr int kdPd = kdPT + 64 * 64 * 2;          // fp32 diagonal blocks [64][16]
+  static constexpr int kPhase2End = kdPd + 64 * 16 * 4;
   static constexpr int kRed = (kPhase1End > kPhase2End ? kPhase1End : kPhase2End);  // scalar-gate reduction [8][64]
   static constexpr int kBar = kRed + 8 * 64 * 4;
   static constexpr int kBytes = kBar + 128;
@@ -217,8 +222,10 @@ __global__ void __launch_bounds__(256, 1)
   }
 
   // ============================ phase 2 ============================
-  // dP (rows t, TMEM M = 64 layout) -> masked bf16 tiles dP[t][s] and dP^T[s][t]
+  // dP (rows t, TMEM M = 64 layout) -> bf16 tiles of its strictly-lower sub-chunk
+  // blocks, dP[t][s] and dP^T[s][t], and fp32 copies of the four diagonal blocks.
   const uint32_t sdP = dev::smem_u32(smem + L::kdP), sdPT = dev::smem_u32(smem + L::kdPT);
+  float *dPd = (float *)(smem + L::kdPd);
   if (warp < 4) {
     const int t = 16 * warp + lane;
     float row[kC];
@@ -226,11 +233,12 @@ __global__ void __launch_bounds__(256, 1)
     for (int cb = 0; cb < 4; ++cb) dev::tmem_ld16(dev::tmem_addr(tmem, 32 * warp, cDP + 16 * cb), row + 16 * cb);
     dev::tmem_wait_ld();
     if (lane < 16) {
+      const int jt = warp;  // sub-chunk of t
 #pragma unroll
       for (int s8 = 0; s8 < 8; ++s8) {
         float m8[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) m8[e] = (s8 * 8 + e <= t && ok) ? row[s8 * 8 + e] : 0.f;
+        for (int e = 0; e < 8; ++e) m8[e] = ((s8 * 8 + e) < 16 * jt && ok) ? row[s8 * 8 + e] : 0.f;
         dev::st_shared_v4(sdP + dev::sw128_chunk(64, t, s8), dev::pack_bf16(m8[0], m8[1]),
                           dev::pack_bf16(m8[2], m8[3]), dev::pack_bf16(m8[4], m8[5]), dev::pack_bf16(m8[6], m8[7]));
 #pragma unroll
@@ -238,6 +246,11 @@ __global__ void __launch_bounds__(256, 1)
           const bf16 b = __float2bfloat16_rn(m8[e]);
           dev::st_shared_u16(sdPT + dev::sw128_off(64, s8 * 8 + e, t), *reinterpret_cast<const uint16_t *>(&b));
         }
+      }
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const int sidx = 16 * jt + e;
+        dPd[t * 16 + e] = (sidx <= t && ok) ? row[sidx] : 0.f;
       }
     }
   }
@@ -277,8 +290,8 @@ __global__ void __launch_bounds__(256, 1)
       E[j] = __expf(z[j]);
     }
     const uint32_t sKh = dev::smem_u32(smem + L::kKh), sQh = dev::smem_u32(smem + L::kQh);
-    const int wK[4] = {0, 16, 48, 96};   // key window j: row wK[j] + s, s in [0, 16(j+1))
-    const int wQ[4] = {0, 48, 80, 96};   // query window u: row wQ[u] + t, t in [16u, 64)
+    const int wK[4] = {0, 0, 16, 48};    // key window j >= 1: row wK[j] + s, s in [0, 16j)
+    const int wQ[4] = {-16, 16, 32, 0};  // query window u <= 2: row wQ[u] + t, t in [16(u+1), 64)
 #pragma unroll
     for (int t = 0; t < kC; ++t) {
       const int j = t >> 4;
@@ -286,21 +299,21 @@ __global__ void __launch_bounds__(256, 1)
       qk_at(t, qf, kf);
       const float u = __expf(Bv[t] - z[j]);
       const float w = __expf(z[j + 1] - Bv[t]);
-      // key operand k_t e^{z_jq - B_t}, query sub-chunks jq >= j (one more Gam per step)
-      float f = kf * w / Gam[j];
+      // key operand k_t e^{z_jq - B_t} for later query sub-chunks jq > j
+      float f = kf * w;
 #pragma unroll
-      for (int jq = 0; jq < 4; ++jq) {
-        if (jq >= j) {
+      for (int jq = 1; jq < 4; ++jq) {
+        if (jq > j) {
           const bf16 b = __float2bfloat16_rn(f);
           dev::st_shared_u16(sKh + dev::sw128_off(L::kRowsW, wK[jq] + t, c), *reinterpret_cast<const uint16_t *>(&b));
           f *= Gam[jq];
         }
       }
-      // query operand q_t e^{B_t - z_{uu+1}}, key sub-chunks uu <= j (one more Gam per step down)
-      float g2 = qf * u / Gam[j];
+      // query operand q_t e^{B_t - z_{uu+1}} for earlier key sub-chunks uu < j
+      float g2 = qf * u;
 #pragma unroll
-      for (int uu = 3; uu >= 0; --uu) {
-        if (uu <= j) {
+      for (int uu = 2; uu >= 0; --uu) {
+        if (uu < j) {
           const bf16 b = __float2bfloat16_rn(g2);
           dev::st_shared_u16(sQh + dev::sw128_off(L::kRowsW, wQ[uu] + t, c), *reinterpret_cast<const uint16_t *>(&b));
           g2 *= Gam[uu];
@@ -314,23 +327,23 @@ __global__ void __launch_bounds__(256, 1)
   dev::tc_fence_after();
   if (tid == 0 && ok) {
     const uint32_t sKh = dev::smem_u32(smem + L::kKh), sQh = dev::smem_u32(smem + L::kQh);
-    const int wK[4] = {0, 16, 48, 96};
-    const int wQ[4] = {0, 48, 80, 96};
+    const int wK[4] = {0, 0, 16, 48};
+    const int wQ[4] = {-16, 16, 32, 0};
     constexpr uint32_t id = dev::idesc_bf16(128, 16, true, false);
 #pragma unroll
     for (int m = 0; m < kMB; ++m) {
 #pragma unroll
-      for (int j = 0; j < 4; ++j)
+      for (int j = 1; j < 4; ++j)
 #pragma unroll
-        for (int kk = 0; kk <= j; ++kk)
+        for (int kk = 0; kk < j; ++kk)
           dev::umma_bf16(tmem + cQI + 64 * m + 16 * j, dev::desc_mnmajor(sKh, L::kRowsW, wK[j] + 16 * kk, 128 * m),
                          dev::desc_kmajor(sdP, 64, 16 * j, 16 * kk), id, kk > 0 ? 1u : 0u);
 #pragma unroll
-      for (int u = 0; u < 4; ++u)
+      for (int u = 0; u < 3; ++u)
 #pragma unroll
-        for (int kk = u; kk < 4; ++kk)
+        for (int kk = u + 1; kk < 4; ++kk)
           dev::umma_bf16(tmem + cKI + 64 * m + 16 * u, dev::desc_mnmajor(sQh, L::kRowsW, wQ[u] + 16 * kk, 128 * m),
-                         dev::desc_kmajor(sdPT, 64, 16 * u, 16 * kk), id, kk > u ? 1u : 0u);
+                         dev::desc_kmajor(sdPT, 64, 16 * u, 16 * kk), id, kk > u + 1 ? 1u : 0u);
     }
     dev::umma_commit(mma_bar);
   }
@@ -365,21 +378,64 @@ __global__ void __launch_bounds__(256, 1)
       }
     }
   }
-  // pass B: reverse over tokens; dq, dk, dlog b and its suffix sum
+  // pass B: reverse over sub-chunks and tokens; dq, dk, dlog b and its suffix sum
   float run = Gb;
 #pragma unroll
   for (int t16 = 3; t16 >= 0; --t16) {
+    const int j = t16;
     float xq[16], xk[16], xqi[16], xki[16];
     dev::tmem_ld16(dev::tmem_addr(tmem, lanebase, cDQ + 64 * mb + 16 * t16), xq);
     dev::tmem_ld16(dev::tmem_addr(tmem, lanebase, cDK + 64 * mb + 16 * t16), xk);
     dev::tmem_ld16(dev::tmem_addr(tmem, lanebase, cQI + 64 * mb + 16 * t16), xqi);
     dev::tmem_ld16(dev::tmem_addr(tmem, lanebase, cKI + 64 * mb + 16 * t16), xki);
     dev::tmem_wait_ld();
-    const int j = t16;
+    float dqd[16], dkd[16];
     float Gafter = 1.f;
 #pragma unroll
     for (int i2 = 1; i2 < 4; ++i2)
       if (i2 > j) Gafter *= Gam[i2];
+    if (tid < K) {
+      // diagonal block of sub-chunk j in fp32:
+      //   a_t = q_t e^{B_t - z_j},  b_s = k_s e^{z_j - B_s}
+      //   dq_t += e^{B_t - z_j} sum_{s<=t} dP[t,s] b_s ,  dk_s += e^{z_j - B_s} sum_{t>=s} dP[t,s] a_t
+      float av[16], bv[16], uu[16], ee[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const int t = 16 * j + e;
+        float qf, kf;
+        qk_at(t, qf, kf);
+        uu[e] = __expf(Bv[t] - z[j]);
+        ee[e] = __expf(z[j + 1] - Bv[t]) / Gam[j];
+        av[e] = qf * uu[e];
+        bv[e] = kf * ee[e];
+        dqd[e] = 0.f;
+        dkd[e] = 0.f;
+      }
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const int t = 16 * j + e;
+        const float4 *rowp = reinterpret_cast<const float4 *>(dPd + t * 16);
+        float pr[16];
+#pragma unroll
+        for (int x4 = 0; x4 < 4; ++x4) {
+          const float4 v4 = rowp[x4];
+          pr[4 * x4] = v4.x;
+          pr[4 * x4 + 1] = v4.y;
+          pr[4 * x4 + 2] = v4.z;
+          pr[4 * x4 + 3] = v4.w;
+        }
+#pragma unroll
+        for (int f = 0; f <= e; ++f) {
+          dqd[e] += pr[f] * bv[f];
+          dkd[f] += pr[f] * av[e];
+        }
+      }
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        dqd[e] *= uu[e];
+        dkd[e] *= ee[e];
+      }
+    }
 #pragma unroll
     for (int e = 15; e >= 0; --e) {
       const int t = 16 * t16 + e;
@@ -390,9 +446,13 @@ __global__ void __launch_bounds__(256, 1)
         qk_at(t, qf, kf);
         const float u = __expf(Bv[t] - z[j]);
         const float w = __expf(z[j + 1] - Bv[t]);
-        const float dqv = u * (E[j] * xq[e] + xqi[e]);
-        const float dkv = w * (Gafter * xk[e] + xki[e]);
-        run += qf * dqv - kf * dkv;
+        const float offq = (j > 0) ? xqi[e] : 0.f;
+        const float offk = (j < 3) ? xki[e] : 0.f;
+        const float dqr = u * (E[j] * xq[e] + offq);
+        const float dkr = w * (Gafter * xk[e] + offk);
+        const float dqv = dqr + dqd[e];
+        const float dkv = dkr + dkd[e];
+        run += (qf * dqr - kf * dkr) + (qf * dqd[e] - kf * dkd[e]);
         dlb = run;
         if (tg < a.T && ok) {
           a.dq[(qrow0 + t) * K + c] = __float2bfloat16_rn(dqv);
