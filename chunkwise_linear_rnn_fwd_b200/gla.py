@@ -25,10 +25,11 @@ STATUS = {
 DTYPE = {torch.bfloat16: 0, torch.float32: 1}
 GATE = {"vector": 0, "scalar": 1, "none": 2}
 VARIANT = {"auto": 0, "fused": 1, "materialized": 2}
+NOALLOC_SCRATCH_BYTES = 64 << 20  # GLA_NOALLOC_SCRATCH_BYTES in include/gla.h
 
 # Every exported symbol of include/gla.h.
 EXPORTS = ["gla_workspace_size", "gla_check", "gla_fwd", "gla_bwd", "gla_poll_status", "gla_status_string",
-           "gla_timing_enable", "gla_timing_collect", "gla_kernel_name", "gla_build_info"]
+           "gla_timing_enable", "gla_timing_collect", "gla_kernel_name", "gla_build_info", "gla_fwd_noalloc"]
 
 
 class GLAError(RuntimeError):
@@ -62,6 +63,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.gla_check.restype = i
     lib.gla_fwd.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, i, vp]
     lib.gla_fwd.restype = i
+    lib.gla_fwd_noalloc.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, i, vp]
+    lib.gla_fwd_noalloc.restype = i
     lib.gla_bwd.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, vp]
     lib.gla_bwd.restype = i
     lib.gla_poll_status.argtypes = [dp, vp]
@@ -154,6 +157,27 @@ def gla_fwd(q, k, v, log_alpha=None, h0=None, *, chunk=64, gate=None, subchunk=1
                     int(chunk), _stream_handle(stream))
     if r != GLA_OK:
         raise GLAError(r, "gla_fwd")
+    return o, h_final
+
+
+def gla_fwd_noalloc(q, k, v, log_alpha=None, h0=None, *, chunk=64, gate=None, subchunk=16, variant="auto",
+                    segments=0, o=None, h_final=None, want_final=True, stream=None):
+    """Forward without a workspace, for callers that cannot allocate device memory:
+    the library uses a fixed scratch array of its own (GLA_NOALLOC_SCRATCH_BYTES,
+    shared by all calls; calls must not overlap on the GPU).  Returns (o, h_final)."""
+    lib = load()
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    gate = _gate_of(log_alpha, gate)
+    if o is None:
+        o = torch.empty(B, H, T, dv, dtype=q.dtype, device=q.device)
+    if h_final is None and want_final:
+        h_final = torch.empty(B, H, dk, dv, dtype=torch.float32, device=q.device)
+    d = make_desc(B, H, T, dk, dv, q.dtype, gate, subchunk=subchunk, variant=variant, segments=segments)
+    r = lib.gla_fwd_noalloc(ctypes.byref(d), _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(h0), _ptr(o),
+                            _ptr(h_final), int(chunk), _stream_handle(stream))
+    if r != GLA_OK:
+        raise GLAError(r, "gla_fwd_noalloc")
     return o, h_final
 
 

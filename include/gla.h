@@ -124,6 +124,31 @@ int gla_bwd(const gla_desc *desc, const void *q, const void *k, const void *v,
             void *dq, void *dk, void *dv, float *dlog_alpha, float *dh0, int chunk,
             void *stream);
 
+/* ---- forward without a workspace ---------------------------------------------
+ * No counterpart in the paper: this entry point exists for callers that cannot
+ * allocate device memory -- a program whose device memory is all owned by
+ * another allocator (a fixed arena reserved up front), or a plain C caller with
+ * no device-memory management of its own -- and so cannot pass a workspace.
+ * It computes exactly what gla_fwd computes (same arguments; desc->workspace
+ * and desc->workspace_bytes are ignored), using as scratch a fixed array of
+ * GLA_NOALLOC_SCRATCH_BYTES in the library's own device memory, which every GPU
+ * that loads the library holds until the process exits.  It never allocates.
+ *   - Problems whose forward workspace (gla_workspace_size(desc, chunk, 0))
+ *     exceeds GLA_NOALLOC_SCRATCH_BYTES are rejected with
+ *     GLA_ERR_WORKSPACE_TOO_SMALL before anything is enqueued; other argument
+ *     errors are reported as by gla_fwd.
+ *   - All calls share the one array.  Calls that overlap on the GPU (on other
+ *     streams or from other host threads) race on it; the caller must
+ *     serialise them.  Each call clears the status word it needs zeroed.
+ *   - The first call on a device looks up the array's address for that device
+ *     (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   - gla_poll_status cannot reach this scratch; errors found on the device
+ *     are not reported by this entry point. */
+#define GLA_NOALLOC_SCRATCH_BYTES (64u << 20)
+int gla_fwd_noalloc(const gla_desc *desc, const void *q, const void *k, const void *v,
+                    const float *log_alpha, const float *h0, void *o, float *h_final, int chunk,
+                    void *stream);
+
 /* Synchronise `stream`, then read and clear the device status word kept in
  * desc->workspace.  Returns GLA_OK, GLA_ERR_TIMEOUT or GLA_ERR_GATE_RANGE (or
  * GLA_ERR_CUDA if the stream itself failed). */
