@@ -320,7 +320,7 @@ def run_ours(args, w):
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": "gla fwd+bwd, B=2 H=4 T=4096 d_k=256 d_v=512 C=64, bf16, vector gates "
+            "config": {"workload": f"gla fwd+bwd, B={B} H={H} T={T} d_k={K} d_v={V} C={C}, bf16, vector gates "
                                    "z~N(-1,1), fp32 state",
                        "global_batch": B * world, "seq_len": T, "parallelism": f"replicas x{world}",
                        "l2": "inputs larger than L2 (~268 MB touched per step)"},
@@ -346,10 +346,16 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--ref-tokens", type=int, default=1024, help="tokens per head in the oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--batch", type=int, default=None, help="override B (smaller profiling captures)")
+    ap.add_argument("--heads", type=int, default=None, help="override H")
+    ap.add_argument("--seqlen", type=int, default=None, help="override T")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     w = dict(WORKLOAD)
+    for key, val in (("B", args.batch), ("H", args.heads), ("T", args.seqlen)):
+        if val is not None:
+            w[key] = val
     if args.impl == "reference":
         return run_reference(args, w)
     return run_ours(args, w)

@@ -208,7 +208,7 @@ int gla_poll_status(const gla_desc *desc, void *stream) {
     return GLA_ERR_CUDA;
   if (cudaStreamSynchronize(st) != cudaSuccess) return GLA_ERR_CUDA;
   if (cudaMemsetAsync(desc->workspace, 0, sizeof(word), st) != cudaSuccess) return GLA_ERR_CUDA;
-  if (word & ST_TIMEOUT) return GLA_ERR_TIMEOUT;
+  if (word & (ST_TIMEOUT | ST_SMEM_ALIGN)) return GLA_ERR_TIMEOUT;
   if (word & ST_GATE_RANGE) return GLA_ERR_GATE_RANGE;
   return GLA_OK;
 }

@@ -44,7 +44,7 @@ struct Problem {
 };
 
 // Status word bits written by kernels into the workspace header.
-enum StatusBits : unsigned { ST_TIMEOUT = 1u, ST_GATE_RANGE = 2u };
+enum StatusBits : unsigned { ST_TIMEOUT = 1u, ST_GATE_RANGE = 2u, ST_SMEM_ALIGN = 4u };
 
 constexpr size_t kStatusBytes = 256;
 

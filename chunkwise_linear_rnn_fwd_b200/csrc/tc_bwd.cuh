@@ -60,7 +60,9 @@ struct BwdSmem {
   static constexpr int kdP = kQh + kRowsW * K * 2;         // dP, strictly-lower blocks  [t][s]
   static constexpr int kdPT = kdP + 64 * 64 * 2;           // the same, transposed [s][t]
   static constexpr int kdPd = kdPT + 64 * 64 * 2;          // fp32 diagonal blocks [64][16]
-  static constexpr int kPhase2End = kdPd + 64 * 16 * 4;
+  static constexpr int kQt = kdPd + 64 * 16 * 4;          // q tile [64][K] bf16 (TMA, after phase 1)
+  static constexpr int kKt = kQt + 64 * K * 2;             // k tile [64][K] bf16
+  static constexpr int kPhase2End = kKt + 64 * K * 2;
   static constexpr int kRed = (kPhase1End > kPhase2End ? kPhase1End : kPhase2End);  // scalar-gate reduction [8][64]
   static constexpr int kBar = kRed + 8 * 64 * 4;
   static constexpr int kBytes = kBar + 128;
@@ -70,7 +72,8 @@ template <int K>
 __global__ void __launch_bounds__(256, 1)
     k_bwd_main(BwdArgs a, const __grid_constant__ CUtensorMap tmH, const __grid_constant__ CUtensorMap tmDH,
                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
-               const __grid_constant__ CUtensorMap tmKg, const __grid_constant__ CUtensorMap tmPT) {
+               const __grid_constant__ CUtensorMap tmKg, const __grid_constant__ CUtensorMap tmPT,
+               const __grid_constant__ CUtensorMap tmQin, const __grid_constant__ CUtensorMap tmKin) {
   using L = BwdSmem<K>;
   constexpr int BVb = L::BVb;
   constexpr int kMB = K / 128;
@@ -79,9 +82,10 @@ __global__ void __launch_bounds__(256, 1)
   constexpr int kTmemCols = (K == 256) ? 512 : 256;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  uint64_t *full = (uint64_t *)(smem + L::kBar);  // [0],[1] stages, [2] kg+PT
+  uint64_t *full = (uint64_t *)(smem + L::kBar);  // [0],[1] stages, [2] kg+PT, [4] q/k tiles
   uint64_t *mma_bar = full + 3;
-  uint32_t *tslot = (uint32_t *)(full + 4);
+  uint64_t *qk_bar = full + 4;
+  uint32_t *tslot = (uint32_t *)(full + 5);
   float *red = (float *)(smem + L::kRed);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -94,6 +98,7 @@ __global__ void __launch_bounds__(256, 1)
   if (tid == 0) {
     for (int i = 0; i < 3; ++i) dev::mbar_init(&full[i], 1);
     dev::mbar_init(mma_bar, 1);
+    dev::mbar_init(qk_bar, 1);
     dev::fence_mbar_init();
   }
   dev::tc_fence_before();
@@ -222,6 +227,16 @@ __global__ void __launch_bounds__(256, 1)
   }
 
   // ============================ phase 2 ============================
+  // q and k tiles of this chunk into the space phase 1 no longer uses
+  if (tid == 0) {
+    dev::fence_proxy_async_smem();
+    dev::mbar_arrive_expect_tx(qk_bar, (uint32_t)(2 * 64 * K * 2));
+#pragma unroll
+    for (int cb = 0; cb < K / 64; ++cb) {
+      dev::tma_load_3d(smem + L::kQt + cb * 64 * 128, &tmQin, cb * 64, n * kC, (int)bh, qk_bar);
+      dev::tma_load_3d(smem + L::kKt + cb * 64 * 128, &tmKin, cb * 64, n * kC, (int)bh, qk_bar);
+    }
+  }
   // dP (rows t, TMEM M = 64 layout) -> bf16 tiles of its strictly-lower sub-chunk
   // blocks, dP[t][s] and dP^T[s][t], and fp32 copies of the four diagonal blocks.
   const uint32_t sdP = dev::smem_u32(smem + L::kdP), sdPT = dev::smem_u32(smem + L::kdPT);
@@ -259,16 +274,15 @@ __global__ void __launch_bounds__(256, 1)
   float Bv[kC];
   float z[5], Gam[4], E[4];
   const long qrow0 = bh * a.T + (long)n * kC;  // first token row of this chunk
+  const uint32_t sQt = dev::smem_u32(smem + L::kQt), sKt = dev::smem_u32(smem + L::kKt);
   auto qk_at = [&](int t, float &qf, float &kf) {
-    qf = 0.f;
-    kf = 0.f;
-    if ((long)n * kC + t < a.T) {
-      qf = __bfloat162float(a.q[(qrow0 + t) * K + c]);
-      kf = __bfloat162float(a.k[(qrow0 + t) * K + c]);
-    }
+    uint16_t qb, kb;
+    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(qb) : "r"(sQt + dev::sw128_off(64, t, c)));
+    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(kb) : "r"(sKt + dev::sw128_off(64, t, c)));
+    qf = __bfloat162float(*reinterpret_cast<const bf16 *>(&qb));
+    kf = __bfloat162float(*reinterpret_cast<const bf16 *>(&kb));
   };
   if (tid < K) {
-    float acc = 0.f;
 #pragma unroll
     for (int t = 0; t < kC; ++t) {
       float g = 0.f;
@@ -276,7 +290,12 @@ __global__ void __launch_bounds__(256, 1)
         if (a.gate == GLA_GATE_VECTOR) g = __ldg(a.la + (qrow0 + t) * K + c);
         else if (a.gate == GLA_GATE_SCALAR) g = __ldg(a.la + qrow0 + t);
       }
-      acc += g;
+      Bv[t] = g;
+    }
+    float acc = 0.f;
+#pragma unroll
+    for (int t = 0; t < kC; ++t) {
+      acc += Bv[t];
       Bv[t] = acc;
     }
     z[0] = 0.f;
@@ -289,6 +308,9 @@ __global__ void __launch_bounds__(256, 1)
       Gam[j] = __expf(z[j + 1] - z[j]);
       E[j] = __expf(z[j]);
     }
+  }
+  if (!dev::mbar_wait(qk_bar, 0, a.status)) ok = false;
+  if (tid < K) {
     const uint32_t sKh = dev::smem_u32(smem + L::kKh), sQh = dev::smem_u32(smem + L::kQh);
     const int wK[4] = {0, 0, 16, 48};    // key window j >= 1: row wK[j] + s, s in [0, 16j)
     const int wQ[4] = {-16, 16, 32, 0};  // query window u <= 2: row wQ[u] + t, t in [16(u+1), 64)
@@ -485,16 +507,18 @@ __global__ void __launch_bounds__(256, 1)
 
 template <int K>
 int launch_bwd_main_k(const Problem &p, const BwdArgs &a, const CUtensorMap *maps, cudaStream_t st) {
-  const int smem = BwdSmem<K>::kBytes + 1024;
-  static bool attr = false;
-  if (!attr) {
-    if (cudaFuncSetAttribute(k_bwd_main<K>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+  static int smem = 0;
+  if (!smem) {
+    const int want = BwdSmem<K>::kBytes + 1024;
+    if (cudaFuncSetAttribute(k_bwd_main<K>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem) != cudaSuccess)
       return GLA_ERR_CUDA;
-    attr = true;
+    const int got = smem_for_tmem(k_bwd_main<K>, 256, want, (K == 256) ? 512 : 256);
+    if (got < 0) return GLA_ERR_CUDA;
+    smem = got;
   }
   GLA_LAUNCH(K_TC_BWD, st,
              (k_bwd_main<K><<<dim3(p.N, p.BH), 256, smem, st>>>(a, maps[0], maps[1], maps[2], maps[3], maps[4],
-                                                                 maps[5])));
+                                                                 maps[5], maps[6], maps[7])));
   return GLA_OK;
 }
 
@@ -507,12 +531,13 @@ inline int launch_bwd_main(const Problem &p, const bf16 *q, const bf16 *k, const
   (void)qg;
   (void)scratch;
   if (p.V % 64 != 0) return GLA_ERR_UNSUPPORTED_SHAPE;
-  CUtensorMap maps[6];
+  CUtensorMap maps[8];
   const uint64_t BH = (uint64_t)p.BH;
   const bool ok = map3_bf16(&maps[0], hb, p.V, p.K, BH * p.N, 64, p.K) &&
                   map3_bf16(&maps[1], dhb, p.V, p.K, BH * p.N, 64, p.K) &&
                   map3_bf16(&maps[2], v, p.V, p.T, BH, 64, 64) && map3_bf16(&maps[3], dout, p.V, p.T, BH, 64, 64) &&
-                  map3_bf16(&maps[4], kg, p.K, p.Tp, BH, 64, 64) && map3_bf16(&maps[5], PT, 64, 64, BH * p.N, 64, 64);
+                  map3_bf16(&maps[4], kg, p.K, p.Tp, BH, 64, 64) && map3_bf16(&maps[5], PT, 64, 64, BH * p.N, 64, 64) &&
+                  map3_bf16(&maps[6], q, p.K, p.T, BH, 64, 64) && map3_bf16(&maps[7], k, p.K, p.T, BH, 64, 64);
   if (!ok) return GLA_ERR_CUDA;
   BwdArgs a{p.T, p.N, p.V, p.gate, p.Tp, q, k, la, gam, dq, dk, dv, dla, status};
   if (p.K == 256) return launch_bwd_main_k<256>(p, a, maps, st);

@@ -227,4 +227,28 @@ __device__ __forceinline__ void st_shared_u16(uint32_t addr, uint16_t v) {
 }
 
 }  // namespace dev
+
+// Largest dynamic shared memory a CTA may use on sm_100 (227 KiB).
+constexpr int kMaxDynSmem = 232448;
+
+// tcgen05.alloc does not wait for columns to free up: a CTA that asks for more
+// TMEM than its SM has left gets no usable allocation.  So every TMEM-using
+// kernel is launched with enough dynamic shared memory that at most
+// 512 / tmem_cols of its CTAs can be resident on one SM.
+template <typename Kern>
+inline int smem_for_tmem(Kern kernel, int threads, int smem, int tmem_cols) {
+  const int max_ctas = 512 / tmem_cols;
+  int dev = 0, per_sm = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
+  for (int guard = 0; guard < 64; ++guard) {
+    int nb = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kernel, threads, smem) != cudaSuccess) return -1;
+    if (nb <= max_ctas) return smem;
+    smem = per_sm / (max_ctas + 1) + 1;  // (max_ctas + 1) CTAs no longer fit
+    smem = (smem + 1023) & ~1023;
+  }
+  return -1;
+}
+
 }  // namespace gla

@@ -32,7 +32,6 @@ constexpr int kSub = 16;  // sub-chunk
 struct PrepArgs {
   int T, N, gate;
   long Tp;
-  const bf16 *q, *k;
   const float *la;
   bf16 *qg, *kg, *PT;
   float *gam;
@@ -41,18 +40,21 @@ struct PrepArgs {
 
 template <int K>
 struct PrepSmem {
-  static constexpr int kRowsKw = 112;                  // K-hat windows: rows [0,16) [16,48) [48,96) + pad
-  static constexpr int kQh = 0;                        // Q-hat tile, 64 rows
+  static constexpr int kRowsKw = 112;                  // key windows: rows [0,16) [16,48) [48,96) + pad
+  static constexpr int kQ = 0;                         // q tile [64][K] bf16 (TMA)
+  static constexpr int kK = kQ + 64 * K * 2;           // k tile [64][K] bf16 (TMA)
+  static constexpr int kQh = kK + 64 * K * 2;          // Q-hat tile, 64 rows
   static constexpr int kKw = kQh + 64 * K * 2;         // key windows, 112 rows
-  static constexpr int kAf = kKw + kRowsKw * K * 2;    // fp32 a_t = q_t u_t    [64][K]
-  static constexpr int kBf = kAf + 64 * K * 4;         // fp32 b_s = k_s e^{z_j - B_s}
-  static constexpr int kPd = kBf + 64 * K * 4;         // fp32 diag partials [2][64][16]
-  static constexpr int kBar = kPd + 2 * 64 * 16 * 4;   // mbarrier + tmem slot
+  static constexpr int kAf = kKw + kRowsKw * K * 2;    // fp32 a_t = q_t u_t of one sub-chunk [16][K]
+  static constexpr int kBf = kAf + 16 * K * 4;         // fp32 b_s = k_s e^{z_j - B_s} [16][K]
+  static constexpr int kRed = kBf + 16 * K * 4;        // per-warp partial diagonal blocks [8][16][16]
+  static constexpr int kPd = kRed + 8 * 256 * 4;       // fp32 diagonal blocks [64][16]
+  static constexpr int kBar = kPd + 64 * 16 * 4;       // mbarriers + tmem slot
   static constexpr int kBytes = kBar + 64;
 };
 
-// fp32 [64][K] tile with a 16-byte-chunk swizzle (bank-conflict-free for the
-// diagonal-block access pattern).
+// fp32 [rows][K] tile with a 16-byte-chunk swizzle (bank-conflict-free for the
+// diagonal-block access pattern: 4 rows 4 apart, or 8 rows 2 apart, per load).
 template <int K>
 __device__ __forceinline__ int f32_swz(int r, int c) {
   const int cc = c >> 2;
@@ -61,16 +63,20 @@ __device__ __forceinline__ int f32_swz(int r, int c) {
 }
 
 template <int K>
-__global__ void __launch_bounds__(256, 1) k_prep(PrepArgs a) {
+__global__ void __launch_bounds__(256, 1)
+    k_prep(PrepArgs a, const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk) {
   using L = PrepSmem<K>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  const uint32_t sQ = dev::smem_u32(smem + L::kQ);
+  const uint32_t sK = dev::smem_u32(smem + L::kK);
   const uint32_t sQh = dev::smem_u32(smem + L::kQh);
   const uint32_t sKw = dev::smem_u32(smem + L::kKw);
   float *Af = (float *)(smem + L::kAf);
   float *Bf = (float *)(smem + L::kBf);
+  float *red = (float *)(smem + L::kRed);
   float *Pd = (float *)(smem + L::kPd);
-  uint64_t *bar = (uint64_t *)(smem + L::kBar);
+  uint64_t *bar = (uint64_t *)(smem + L::kBar);  // [0] q/k loads, [1] MMA
   uint32_t *tslot = (uint32_t *)(smem + L::kBar + 16);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -79,33 +85,44 @@ __global__ void __launch_bounds__(256, 1) k_prep(PrepArgs a) {
 
   if (warp == 0) dev::tmem_alloc(tslot, 64);
   if (tid == 0) {
-    dev::mbar_init(bar, 1);
+    dev::mbar_init(&bar[0], 1);
+    dev::mbar_init(&bar[1], 1);
     dev::fence_mbar_init();
+    dev::mbar_arrive_expect_tx(&bar[0], (uint32_t)(2 * 64 * K * 2));
+#pragma unroll
+    for (int cb = 0; cb < K / 64; ++cb) {
+      dev::tma_load_3d(smem + L::kQ + cb * 64 * 128, &tmq, cb * 64, n * kC, (int)bh, &bar[0]);
+      dev::tma_load_3d(smem + L::kK + cb * 64 * 128, &tmk, cb * 64, n * kC, (int)bh, &bar[0]);
+    }
   }
+  __syncthreads();  // barriers initialised before anyone waits on them
 
-  // ---- per key channel: cumulative log-gate and rescaled operands --------
+  // ---- per key channel: chunk-local cumulative log-gate (all loads in flight) ----
+  const int c = tid;
+  float Bv[kC];
+  float z[5], Gam[4], E[4], Gafter[4];
   if (tid < K) {
-    const int c = tid;
-    float Bv[kC];
-    float acc = 0.f;
+    float g[kC];
 #pragma unroll
     for (int t = 0; t < kC; ++t) {
       const long tg = (long)n * kC + t;
-      float g = 0.f;
+      g[t] = 0.f;
       if (tg < a.T) {
-        if (a.gate == GLA_GATE_VECTOR) g = __ldg(a.la + (bh * a.T + tg) * K + c);
-        else if (a.gate == GLA_GATE_SCALAR) g = __ldg(a.la + bh * a.T + tg);
+        if (a.gate == GLA_GATE_VECTOR) g[t] = __ldg(a.la + (bh * a.T + tg) * K + c);
+        else if (a.gate == GLA_GATE_SCALAR) g[t] = __ldg(a.la + bh * a.T + tg);
       }
-      acc += g;
+    }
+    float acc = 0.f;
+#pragma unroll
+    for (int t = 0; t < kC; ++t) {
+      acc += g[t];
       Bv[t] = acc;
     }
-    float z[5];
     z[0] = 0.f;
     z[1] = Bv[15];
     z[2] = Bv[31];
     z[3] = Bv[47];
     z[4] = Bv[63];
-    float Gam[4], E[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       Gam[j] = __expf(z[j + 1] - z[j]);
@@ -113,49 +130,91 @@ __global__ void __launch_bounds__(256, 1) k_prep(PrepArgs a) {
     }
     if (Gam[0] < 1e-36f || Gam[1] < 1e-36f || Gam[2] < 1e-36f || Gam[3] < 1e-36f)
       atomicOr(a.status, (unsigned)ST_GATE_RANGE);
-    // Gafter[j] = prod_{i>j} Gam_i = e^{B_63 - z_{j+1}}
-    float Gafter[4];
     Gafter[3] = 1.f;
     Gafter[2] = Gam[3];
     Gafter[1] = Gam[3] * Gam[2];
     Gafter[0] = Gam[3] * Gam[2] * Gam[1];
     a.gam[(bh * a.N + n) * K + c] = __expf(z[4]);
-    const int wrow[4] = {0, 0, 16, 48};  // window start row of query sub-chunk j (j >= 1)
-#pragma unroll
-    for (int t = 0; t < kC; ++t) {
-      const int j = t >> 4;
-      const long tg = (long)n * kC + t;
-      float qf = 0.f, kf = 0.f;
-      if (tg < a.T) {
-        qf = __bfloat162float(a.q[(bh * a.T + tg) * K + c]);
-        kf = __bfloat162float(a.k[(bh * a.T + tg) * K + c]);
-      }
-      const float u = __expf(Bv[t] - z[j]);
-      const float w = __expf(z[j + 1] - Bv[t]);
-      const float qh = qf * u;
-      const float kw = kf * w;
-      a.qg[(bh * a.Tp + tg) * K + c] = __float2bfloat16_rn(qh * E[j]);
-      a.kg[(bh * a.Tp + tg) * K + c] = __float2bfloat16_rn(kw * Gafter[j]);
-      const bf16 qhb = __float2bfloat16_rn(qh);
-      dev::st_shared_u16(sQh + dev::sw128_off(64, t, c), *reinterpret_cast<const uint16_t *>(&qhb));
-      Af[f32_swz<K>(t, c)] = qh;
-      Bf[f32_swz<K>(t, c)] = kw / Gam[j];
-      // key operand for every later query sub-chunk jq: k_s e^{z_jq - B_s}
-      float f = kw;
-#pragma unroll
-      for (int jq = 1; jq < 4; ++jq) {
-        if (jq > j) {
-          const bf16 kb = __float2bfloat16_rn(f);
-          dev::st_shared_u16(sKw + dev::sw128_off(L::kRowsKw, wrow[jq] + t, c), *reinterpret_cast<const uint16_t *>(&kb));
-          f *= Gam[jq];
-        }
-      }
-    }
-    // rows 96..111 of the window buffer are read by window 3 only for keys >= 48
-    // (whose entries are discarded); keep them finite.
+    // rows 96..111 of the window buffer are read by window 3 only for keys >= 48,
+    // whose entries are discarded; keep them finite
     const bf16 zb = __float2bfloat16_rn(0.f);
     for (int r = 96; r < L::kRowsKw; ++r)
       dev::st_shared_u16(sKw + dev::sw128_off(L::kRowsKw, r, c), *reinterpret_cast<const uint16_t *>(&zb));
+  }
+  const bool ok_ld = dev::mbar_wait(&bar[0], 0, a.status);
+
+  bf16 *qg = a.qg + (bh * a.Tp + (long)n * kC) * K;
+  bf16 *kg = a.kg + (bh * a.Tp + (long)n * kC) * K;
+  const int wrow[4] = {0, 0, 16, 48};  // window start row of query sub-chunk j (j >= 1)
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    // ---- rescaled operands of sub-chunk j ----
+    if (tid < K) {
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const int t = 16 * j + e;
+        uint16_t qb, kb;
+        asm volatile("ld.shared.u16 %0, [%1];" : "=h"(qb) : "r"(sQ + dev::sw128_off(64, t, c)));
+        asm volatile("ld.shared.u16 %0, [%1];" : "=h"(kb) : "r"(sK + dev::sw128_off(64, t, c)));
+        const float qf = ok_ld ? __bfloat162float(*reinterpret_cast<const bf16 *>(&qb)) : 0.f;
+        const float kf = ok_ld ? __bfloat162float(*reinterpret_cast<const bf16 *>(&kb)) : 0.f;
+        const float u = __expf(Bv[t] - z[j]);
+        const float w = __expf(z[j + 1] - Bv[t]);
+        const float qh = qf * u;
+        const float kw = kf * w;
+        qg[(long)t * K + c] = __float2bfloat16_rn(qh * E[j]);
+        kg[(long)t * K + c] = __float2bfloat16_rn(kw * Gafter[j]);
+        const bf16 qhb = __float2bfloat16_rn(qh);
+        dev::st_shared_u16(sQh + dev::sw128_off(64, t, c), *reinterpret_cast<const uint16_t *>(&qhb));
+        Af[f32_swz<K>(e, c)] = qh;
+        Bf[f32_swz<K>(e, c)] = kw / Gam[j];
+        // key operand for every later query sub-chunk jq: k_s e^{z_jq - B_s}
+        float f = kw;
+#pragma unroll
+        for (int jq = 1; jq < 4; ++jq) {
+          if (jq > j) {
+            const bf16 b = __float2bfloat16_rn(f);
+            dev::st_shared_u16(sKw + dev::sw128_off(L::kRowsKw, wrow[jq] + t, c), *reinterpret_cast<const uint16_t *>(&b));
+            f *= Gam[jq];
+          }
+        }
+      }
+    }
+    __syncthreads();
+    // ---- diagonal block j in fp32: warp w sums its slice of key channels ----
+    {
+      constexpr int kCw = K / 8;
+      const int tg = lane >> 3, sp = lane & 7;
+      float acc[4][2] = {};
+      if (2 * sp <= 4 * tg + 3) {
+        const int c0 = warp * kCw;
+#pragma unroll 4
+        for (int cc = c0; cc < c0 + kCw; cc += 4) {
+          float4 av[4], bv[2];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) av[i] = *reinterpret_cast<const float4 *>(Af + f32_swz<K>(4 * tg + i, cc));
+#pragma unroll
+          for (int m = 0; m < 2; ++m) bv[m] = *reinterpret_cast<const float4 *>(Bf + f32_swz<K>(2 * sp + m, cc));
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int m = 0; m < 2; ++m)
+              acc[i][m] += av[i].x * bv[m].x + av[i].y * bv[m].y + av[i].z * bv[m].z + av[i].w * bv[m].w;
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int m = 0; m < 2; ++m) red[warp * 256 + (4 * tg + i) * 16 + 2 * sp + m] = acc[i][m];
+    }
+    __syncthreads();
+    {
+      const int tl = tid >> 4, sl = tid & 15;
+      float ssum = 0.f;
+#pragma unroll
+      for (int w8 = 0; w8 < 8; ++w8) ssum += red[w8 * 256 + tl * 16 + sl];
+      Pd[(16 * j + tl) * 16 + sl] = (sl <= tl) ? ssum : 0.f;
+    }
   }
   dev::fence_proxy_async_smem();
   dev::tc_fence_before();
@@ -166,7 +225,6 @@ __global__ void __launch_bounds__(256, 1) k_prep(PrepArgs a) {
   // ---- off-diagonal blocks on the tensor cores ----------------------------
   if (tid == 0) {
     constexpr uint32_t idesc = dev::idesc_bf16(64, 16, false, false);
-    const int wrow[4] = {0, 0, 16, 48};
 #pragma unroll
     for (int j = 1; j < 4; ++j) {
 #pragma unroll
@@ -176,41 +234,12 @@ __global__ void __launch_bounds__(256, 1) k_prep(PrepArgs a) {
         dev::umma_bf16(tmem + 16 * j, da, db, idesc, kk > 0 ? 1u : 0u);
       }
     }
-    dev::umma_commit(bar);
+    dev::umma_commit(&bar[1]);
   }
-
-  // ---- diagonal blocks in fp32 on CUDA cores ------------------------------
-  {
-    const int j = warp >> 1, half = warp & 1;
-    const int tg = lane >> 3, sp = lane & 7;
-    const int t0 = 16 * j + 4 * tg, s0 = 16 * j + 2 * sp;
-    float acc[4][2] = {};
-    const bool active = (s0 <= t0 + 3);
-    if (active) {
-      const int c_begin = half * (K / 2), c_end = c_begin + K / 2;
-      for (int c = c_begin; c < c_end; c += 4) {
-        float4 av[4], bv[2];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) av[i] = *reinterpret_cast<const float4 *>(Af + f32_swz<K>(t0 + i, c));
-#pragma unroll
-        for (int i = 0; i < 2; ++i) bv[i] = *reinterpret_cast<const float4 *>(Bf + f32_swz<K>(s0 + i, c));
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-          for (int m = 0; m < 2; ++m)
-            acc[i][m] += av[i].x * bv[m].x + av[i].y * bv[m].y + av[i].z * bv[m].z + av[i].w * bv[m].w;
-      }
-    }
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int m = 0; m < 2; ++m) Pd[(half * 64 + t0 + i) * 16 + (s0 + m - 16 * j)] = acc[i][m];
-  }
-  __syncthreads();
-
-  // ---- wait for the MMAs, assemble P^T rows (key s) and store -------------
-  const bool ok = dev::mbar_wait(bar, 0, a.status);
+  const bool ok = dev::mbar_wait(&bar[1], 0, a.status) && ok_ld;
   dev::tc_fence_after();
+
+  // ---- assemble P^T rows (key s) and store ------------------------------------
   if (warp < 4) {
     const int s = 16 * warp + lane;  // valid for lane < 16
     const int js = warp;             // sub-chunk of key s
@@ -229,7 +258,7 @@ __global__ void __launch_bounds__(256, 1) k_prep(PrepArgs a) {
           const int jt = t >> 4;
           float val = 0.f;
           if (jt > js) val = ok ? row[t] : 0.f;
-          else if (jt == js && t >= s) val = Pd[t * 16 + (s - 16 * js)] + Pd[(64 + t) * 16 + (s - 16 * js)];
+          else if (jt == js && t >= s) val = Pd[t * 16 + (s - 16 * js)];
           v8[e] = val;
         }
         uint4 pk;
@@ -262,25 +291,31 @@ struct WalkArgs {
   const float *start;               // [BH][P][K][V] fp32 or null
   const float *h0;                  // used by segment 0 when start == null
   float *end;                       // [BH][P][K][V] fp32 or null (state after the segment)
+  float *gseg;                      // [BH][P][K] product of gam over the segment (written by d_v tile 0) or null
   float *h32;                       // [BH][N][K][V] fp32 states (state_mode 2)
   bf16 *out;                        // [BH][T][V]
   unsigned *status;
 };
 
+// Shared-memory layout of a walk CTA.  Output walks stage (kg, V, qg, P^T) once
+// (two CTAs share an SM); state-only walks double-buffer (kg or qg, V or dO).
 template <int K, int BV>
 struct WalkSmem {
   static constexpr int kTileX = 64 * K * 2;   // kg or qg chunk tile
   static constexpr int kTileY = 64 * BV * 2;  // V or dO tile
   static constexpr int kTileQ = 64 * K * 2;   // qg for the output
   static constexpr int kTileP = 64 * 64 * 2;  // P^T
-  static constexpr int kStage = kTileX + kTileY + kTileQ + kTileP;
-  static constexpr int kSb = 2 * kStage;      // bf16 state tile [K][BV]
-  static constexpr int kBar = kSb + K * BV * 2;
-  static constexpr int kBytes = kBar + 64;
+  __host__ __device__ static constexpr int stages(bool out) { return out ? 1 : 2; }
+  __host__ __device__ static constexpr int stage_bytes(bool out) {
+    return kTileX + kTileY + (out ? kTileQ + kTileP : 0);
+  }
+  __host__ __device__ static constexpr int sb_off(bool out) { return stages(out) * stage_bytes(out); }
+  __host__ __device__ static constexpr int bar_off(bool out, bool sb) { return sb_off(out) + (sb ? K * BV * 2 : 0); }
+  __host__ __device__ static constexpr int bytes(bool out, bool sb) { return bar_off(out, sb) + 64; }
 };
 
 template <int K, int BV>
-__global__ void __launch_bounds__(K, 1)
+__global__ void __launch_bounds__(K, 2)
     k_walk(WalkArgs a, const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmY,
            const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmP,
            const __grid_constant__ CUtensorMap tmH) {
@@ -289,12 +324,24 @@ __global__ void __launch_bounds__(K, 1)
   constexpr int kMB = K / 128;         // 128-row blocks of the state
   constexpr int kColO = kMB * BV;      // TMEM column of the output accumulator
   constexpr int kTmemCols = (kColO + BV <= 256) ? 256 : 512;
+  // The dynamic shared-memory window is allocated without alignment slack (two
+  // CTAs must fit on one SM); its base is 1024-byte aligned when the kernel has
+  // no static shared memory.  Checked: a misaligned base would break the
+  // 128-byte swizzle, so the CTA reports it and does nothing.
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  uint64_t *full = (uint64_t *)(smem + L::kBar);
+  uint8_t *smem = smem_raw;
+  if ((dev::smem_u32(smem_raw) & 1023u) != 0) {
+    if (threadIdx.x == 0) atomicOr(a.status, (unsigned)ST_SMEM_ALIGN);
+    return;
+  }
+  const bool need_sb = a.do_out || a.state_mode == 1;
+  const int nst = L::stages(a.do_out);
+  const int kStage = L::stage_bytes(a.do_out);
+  uint64_t *full = (uint64_t *)(smem + L::bar_off(a.do_out, need_sb));
   uint64_t *mma_bar = full + 2;
   uint32_t *tslot = (uint32_t *)(full + 3);
-  const uint32_t sSb = dev::smem_u32(smem + L::kSb);
+  uint8_t *sb_ptr = smem + L::sb_off(a.do_out);
+  const uint32_t sSb = dev::smem_u32(sb_ptr);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int vt = blockIdx.x, seg = blockIdx.y;
@@ -324,11 +371,11 @@ __global__ void __launch_bounds__(K, 1)
   const uint32_t tmem = *tslot;
 
   auto chunk_of = [&](int i) { return a.reverse ? (n_end - 1 - i) : (n_begin + i); };
-  auto stage_ptr = [&](int s) { return smem + s * L::kStage; };
-  const uint32_t tx_bytes = (uint32_t)(L::kTileX + L::kTileY + (a.do_out ? L::kTileQ + L::kTileP : 0));
+  auto stage_ptr = [&](int s) { return smem + s * kStage; };
+  const uint32_t tx_bytes = (uint32_t)kStage;
 
   auto issue_loads = [&](int i) {
-    const int s = i & 1;
+    const int s = i % nst;
     const int n = chunk_of(i);
     uint8_t *st = stage_ptr(s);
     dev::mbar_arrive_expect_tx(&full[s], tx_bytes);
@@ -345,10 +392,8 @@ __global__ void __launch_bounds__(K, 1)
     }
   };
 
-  if (tid == 0 && nloc > 0) {
-    issue_loads(0);
-    if (nloc > 1) issue_loads(1);
-  }
+  if (tid == 0)
+    for (int i = 0; i < nst && i < nloc; ++i) issue_loads(i);
 
   // thread -> state row c; TMEM lane block of its warp
   const int mb = warp >> 2;
@@ -372,12 +417,14 @@ __global__ void __launch_bounds__(K, 1)
   }
 
   bool ok = true;
+  float gprod = 1.f;
   for (int i = 0; i < nloc; ++i) {
-    const int s = i & 1;
+    const int s = i % nst;
     const int n = chunk_of(i);
     uint8_t *st = stage_ptr(s);
     const float g = __ldg(a.gam + (bh * a.N + n) * K + c);
-    if (ok) ok = dev::mbar_wait(&full[s], (i >> 1) & 1, a.status);
+    gprod *= g;
+    if (ok) ok = dev::mbar_wait(&full[s], (uint32_t)((i / nst) & 1), a.status);
 
     // ---- S-pass: read S, publish bf16/fp32 copy, scale by gamma ---------------
 #pragma unroll
@@ -439,13 +486,13 @@ __global__ void __launch_bounds__(K, 1)
       if (a.state_mode == 1) {
 #pragma unroll
         for (int cb = 0; cb < BV / 64; ++cb)
-          dev::tma_store_3d(&tmH, smem + L::kSb + cb * K * 128, v0 + cb * 64, 0, (int)(bh * a.N + n));
+          dev::tma_store_3d(&tmH, sb_ptr + cb * K * 128, v0 + cb * 64, 0, (int)(bh * a.N + n));
         dev::tma_store_commit();
       }
     }
     if (ok) ok = dev::mbar_wait(mma_bar, i & 1, a.status);
     dev::tc_fence_after();
-    if (tid == 0 && ok && i + 2 < nloc) issue_loads(i + 2);
+    if (tid == 0 && ok && i + nst < nloc) issue_loads(i + nst);
 
     // ---- output epilogue -----------------------------------------------------
     if (a.do_out) {
@@ -483,6 +530,7 @@ __global__ void __launch_bounds__(K, 1)
   }
 
   // ---- final state of the segment ---------------------------------------------
+  if (a.gseg && vt == 0) a.gseg[(bh * P + seg) * K + c] = gprod;
   if (a.end) {
     float *dst = a.end + ((bh * P + seg) * K + c) * (long)a.V + v0;
 #pragma unroll
@@ -509,8 +557,8 @@ __global__ void __launch_bounds__(K, 1)
 // run forwards from h0 (forward pass) or backwards from dh_final (adjoint).
 // ============================================================================
 struct ScanArgs {
-  int K, V, N, L, P, reverse;
-  const float *gam, *delta, *init;
+  int K, V, P, reverse;
+  const float *gseg, *delta, *init;
   float *start, *final_out;
 };
 
@@ -524,10 +572,7 @@ __global__ void k_scan(ScanArgs a) {
   for (int pi = 0; pi < a.P; ++pi) {
     const int p = a.reverse ? a.P - 1 - pi : pi;
     a.start[(bh * a.P + p) * KV + idx] = S;
-    const int nb = p * a.L, ne = min(a.N, nb + a.L);
-    float gs = 1.f;
-    for (int n = nb; n < ne; ++n) gs *= a.gam[(bh * a.N + n) * a.K + c];
-    S = gs * S + a.delta[(bh * a.P + p) * KV + idx];
+    S = a.gseg[(bh * a.P + p) * a.K + c] * S + a.delta[(bh * a.P + p) * KV + idx];
   }
   if (a.final_out) a.final_out[bh * KV + idx] = S;
 }

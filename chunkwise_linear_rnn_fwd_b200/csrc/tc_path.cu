@@ -84,13 +84,14 @@ int sm_count() {
 
 int bv_of(const Problem &p) { return (p.K == 256 || p.V % 128 != 0) ? 64 : 128; }
 
-// Segment count for the FUSED forward: enough CTAs to cover the SMs once.
+// Segment count for the FUSED forward: as many segments as one wave of walk
+// CTAs (two per SM) can hold.
 int segments_of(const Problem &p, int nvt) {
   if (p.variant == GLA_VARIANT_MATERIALIZED) return 1;
   int P = p.segments;
   if (P <= 0) {
     const long ctas = p.BH * nvt;
-    P = (int)std::max<long>(1, (sm_count() + ctas - 1) / ctas);
+    P = (int)std::max<long>(1, (2L * sm_count()) / ctas);
   }
   P = std::min(P, p.N);
   const int L = (p.N + P - 1) / P;
@@ -101,6 +102,7 @@ struct TcWs {
   bf16 *qg, *kg, *PT;
   float *gam;
   float *delta, *start;  // [BH][P][K][V]
+  float *gseg;           // [BH][P][K] per-segment gate products
   float *h32;            // materialised fp32 chunk states [BH][N][K][V]
   // backward
   bf16 *hb, *dhb;        // bf16 chunk states and adjoints [BH][N][K][V]
@@ -124,6 +126,7 @@ TcWs carve(const Problem &p, void *ws, bool bwd) {
     } else if (P > 1) {
       w.delta = cv.take<float>((size_t)p.BH * P * p.K * p.V);
       w.start = cv.take<float>((size_t)p.BH * P * p.K * p.V);
+      w.gseg = cv.take<float>((size_t)p.BH * P * p.K);
     }
   } else {
     Problem pf = p;
@@ -134,6 +137,7 @@ TcWs carve(const Problem &p, void *ws, bool bwd) {
     w.start = cv.take<float>((size_t)p.BH * P * p.K * p.V);
     w.ddelta = cv.take<float>((size_t)p.BH * P * p.K * p.V);
     w.dstart = cv.take<float>((size_t)p.BH * P * p.K * p.V);
+    w.gseg = cv.take<float>((size_t)p.BH * P * p.K);
     w.hb = cv.take<bf16>((size_t)p.BH * p.N * p.K * p.V);
     w.dhb = cv.take<bf16>((size_t)p.BH * p.N * p.K * p.V);
     w.dscratch = cv.take<float>(tc::bwd_scratch_floats(p.BH, p.N, p.K, p.V));
@@ -145,15 +149,20 @@ TcWs carve(const Problem &p, void *ws, bool bwd) {
 template <int K>
 int launch_prep(const Problem &p, const bf16 *q, const bf16 *k, const float *la, const TcWs &w, unsigned *status,
                 cudaStream_t st) {
-  tc::PrepArgs a{p.T, p.N, p.gate, p.Tp, q, k, la, w.qg, w.kg, w.PT, w.gam, status};
-  const int smem = tc::PrepSmem<K>::kBytes + 1024;
-  static bool attr = false;
-  if (!attr) {
-    if (cudaFuncSetAttribute(tc::k_prep<K>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+  tc::PrepArgs a{p.T, p.N, p.gate, p.Tp, la, w.qg, w.kg, w.PT, w.gam, status};
+  CUtensorMap mq, mk;
+  if (!map3(&mq, q, p.K, p.T, (uint64_t)p.BH, 64, 64) || !map3(&mk, k, p.K, p.T, (uint64_t)p.BH, 64, 64))
+    return GLA_ERR_CUDA;
+  static int smem = 0;
+  if (!smem) {
+    const int want = tc::PrepSmem<K>::kBytes + 1024;
+    if (cudaFuncSetAttribute(tc::k_prep<K>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem) != cudaSuccess)
       return GLA_ERR_CUDA;
-    attr = true;
+    const int got = smem_for_tmem(tc::k_prep<K>, 256, want, 64);
+    if (got < 0) return GLA_ERR_CUDA;
+    smem = got;
   }
-  GLA_LAUNCH(K_TC_PREP, st, (tc::k_prep<K><<<dim3(p.N, p.BH), 256, smem, st>>>(a)));
+  GLA_LAUNCH(K_TC_PREP, st, (tc::k_prep<K><<<dim3(p.N, p.BH), 256, smem, st>>>(a, mq, mk)));
   return GLA_OK;
 }
 
@@ -163,13 +172,18 @@ struct WalkMaps {
 
 template <int K, int BV>
 int launch_walk(const Problem &p, const tc::WalkArgs &a, const WalkMaps &m, int P, cudaStream_t st) {
-  const int smem = tc::WalkSmem<K, BV>::kBytes + 1024;
+  using W = tc::WalkSmem<K, BV>;
+  constexpr int kTmemCols = ((K / 128) * BV + BV <= 256) ? 256 : 512;
   static bool attr = false;
   if (!attr) {
-    if (cudaFuncSetAttribute(tc::k_walk<K, BV>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    if (cudaFuncSetAttribute(tc::k_walk<K, BV>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem) !=
+        cudaSuccess)
       return GLA_ERR_CUDA;
     attr = true;
   }
+  const int smem = smem_for_tmem(tc::k_walk<K, BV>, K, W::bytes(a.do_out != 0, a.do_out || a.state_mode == 1),
+                                 kTmemCols);
+  if (smem < 0) return GLA_ERR_CUDA;
   GLA_LAUNCH(K_TC_WALK, st,
              (tc::k_walk<K, BV><<<dim3(p.V / BV, P, p.BH), K, smem, st>>>(a, m.X, m.Y, m.Q, m.P, m.H)));
   return GLA_OK;
@@ -183,9 +197,9 @@ int launch_walk_any(const Problem &p, const tc::WalkArgs &a, const WalkMaps &m, 
   return GLA_ERR_UNSUPPORTED_SHAPE;
 }
 
-int launch_scan(const Problem &p, const float *gam, const float *delta, const float *init, float *start,
-                float *final_out, int P, int L, int reverse, cudaStream_t st) {
-  tc::ScanArgs a{p.K, p.V, p.N, L, P, reverse, gam, delta, init, start, final_out};
+int launch_scan(const Problem &p, const float *gseg, const float *delta, const float *init, float *start,
+                float *final_out, int P, int reverse, cudaStream_t st) {
+  tc::ScanArgs a{p.K, p.V, P, reverse, gseg, delta, init, start, final_out};
   const long KV = (long)p.K * p.V;
   GLA_LAUNCH(K_TC_SCAN, st, (tc::k_scan<<<dim3((unsigned)((KV + 255) / 256), p.BH), 256, 0, st>>>(a)));
   return GLA_OK;
@@ -269,8 +283,9 @@ int tc_fwd(const Problem &p, const void *q, const void *k, const void *v, const 
   // pre-pass: each segment's contribution from a zero state
   tc::WalkArgs pre = a;
   pre.end = w.delta;
+  pre.gseg = w.gseg;
   TRY(launch_walk_any(p, pre, m, P, st));
-  TRY(launch_scan(p, w.gam, w.delta, h0, w.start, hT, P, L, 0, st));
+  TRY(launch_scan(p, w.gseg, w.delta, h0, w.start, hT, P, 0, st));
   a.do_out = 1;
   a.start = w.start;
   return launch_walk_any(p, a, m, P, st);
@@ -316,8 +331,9 @@ int tc_bwd(const Problem &p, const void *q, const void *k, const void *v, const 
   if (P > 1) {
     tc::WalkArgs pre = a;
     pre.end = w.delta;
+    pre.gseg = w.gseg;
     TRY(launch_walk_any(p, pre, mf, P, st));
-    TRY(launch_scan(p, w.gam, w.delta, h0, w.start, nullptr, P, L, 0, st));
+    TRY(launch_scan(p, w.gseg, w.delta, h0, w.start, nullptr, P, 0, st));
     a.start = w.start;
   } else {
     a.h0 = h0;
@@ -337,7 +353,7 @@ int tc_bwd(const Problem &p, const void *q, const void *k, const void *v, const 
     tc::WalkArgs pre = r;
     pre.end = w.ddelta;
     TRY(launch_walk_any(p, pre, mr, P, st));
-    TRY(launch_scan(p, w.gam, w.ddelta, dhT, w.dstart, dh0, P, L, 1, st));
+    TRY(launch_scan(p, w.gseg, w.ddelta, dhT, w.dstart, dh0, P, 1, st));
     r.start = w.dstart;
   } else {
     r.h0 = dhT;
