@@ -286,6 +286,9 @@ __global__ void __launch_bounds__(256, 1)
 // ============================================================================
 struct WalkArgs {
   int T, N, V, L;  // L = chunks per segment
+  int P;           // segments per sequence (the grid covers segments seg0 .. seg0 + gridDim.y - 1)
+  int seg0;
+  int end_seg;     // -1: every segment writes end[BH][P][K][V]; s >= 0: only segment s writes end[BH][K][V]
   int reverse, do_out, state_mode;  // state_mode: 0 none, 1 bf16 (TMA store), 2 fp32
   const float *gam;                 // [BH][N][K]
   const float *start;               // [BH][P][K][V] fp32 or null
@@ -344,13 +347,13 @@ __global__ void __launch_bounds__(K, 2)
   const uint32_t sSb = dev::smem_u32(sb_ptr);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int vt = blockIdx.x, seg = blockIdx.y;
+  const int vt = blockIdx.x, seg = blockIdx.y + a.seg0;
   const long bh = blockIdx.z;
   const int v0 = vt * BV;
   const int n_begin = seg * a.L;
   const int n_end = min(a.N, n_begin + a.L);
   const int nloc = n_end - n_begin;
-  const int P = gridDim.y;
+  const int P = a.P;
 
   if (warp == 0) dev::tmem_alloc(tslot, kTmemCols);
   if (tid == 0) {
@@ -409,8 +412,20 @@ __global__ void __launch_bounds__(K, 2)
 #pragma unroll
     for (int cb = 0; cb < BV / 16; ++cb) {
       float v[16];
+      if (src) {
+        const float4 *s4 = reinterpret_cast<const float4 *>(src + cb * 16);
 #pragma unroll
-      for (int e = 0; e < 16; ++e) v[e] = src ? __ldg(src + cb * 16 + e) : 0.f;
+        for (int e = 0; e < 4; ++e) {
+          const float4 x = __ldg(s4 + e);
+          v[4 * e] = x.x;
+          v[4 * e + 1] = x.y;
+          v[4 * e + 2] = x.z;
+          v[4 * e + 3] = x.w;
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 16; ++e) v[e] = 0.f;
+      }
       dev::tmem_st16(tS + cb * 16, v);
     }
     dev::tmem_wait_st();
@@ -418,38 +433,38 @@ __global__ void __launch_bounds__(K, 2)
 
   bool ok = true;
   float gprod = 1.f;
+  float g_next = (nloc > 0) ? __ldg(a.gam + (bh * a.N + chunk_of(0)) * K + c) : 1.f;
   for (int i = 0; i < nloc; ++i) {
     const int s = i % nst;
     const int n = chunk_of(i);
     uint8_t *st = stage_ptr(s);
-    const float g = __ldg(a.gam + (bh * a.N + n) * K + c);
+    const float g = g_next;
+    if (i + 1 < nloc) g_next = __ldg(a.gam + (bh * a.N + chunk_of(i + 1)) * K + c);
     gprod *= g;
     if (ok) ok = dev::mbar_wait(&full[s], (uint32_t)((i / nst) & 1), a.status);
 
     // ---- S-pass: read S, publish bf16/fp32 copy, scale by gamma ---------------
 #pragma unroll
-    for (int cb = 0; cb < BV / 16; ++cb) {
-      float v[16];
-      dev::tmem_ld16(tS + cb * 16, v);
+    for (int cb = 0; cb < BV / 32; ++cb) {
+      float v[32];
+      dev::tmem_ld32(tS + cb * 32, v);
       dev::tmem_wait_ld();
       if (a.do_out || a.state_mode == 1) {
-        const uint32_t w0 = dev::pack_bf16(v[0], v[1]), w1 = dev::pack_bf16(v[2], v[3]);
-        const uint32_t w2 = dev::pack_bf16(v[4], v[5]), w3 = dev::pack_bf16(v[6], v[7]);
-        const uint32_t w4 = dev::pack_bf16(v[8], v[9]), w5 = dev::pack_bf16(v[10], v[11]);
-        const uint32_t w6 = dev::pack_bf16(v[12], v[13]), w7 = dev::pack_bf16(v[14], v[15]);
-        dev::st_shared_v4(sSb + dev::sw128_chunk(K, c, cb * 2), w0, w1, w2, w3);
-        dev::st_shared_v4(sSb + dev::sw128_chunk(K, c, cb * 2 + 1), w4, w5, w6, w7);
+#pragma unroll
+        for (int h = 0; h < 4; ++h)
+          dev::st_shared_v4(sSb + dev::sw128_chunk(K, c, cb * 4 + h), dev::pack_bf16(v[8 * h], v[8 * h + 1]),
+                            dev::pack_bf16(v[8 * h + 2], v[8 * h + 3]), dev::pack_bf16(v[8 * h + 4], v[8 * h + 5]),
+                            dev::pack_bf16(v[8 * h + 6], v[8 * h + 7]));
       }
       if (a.state_mode == 2) {
-        float4 *dst = reinterpret_cast<float4 *>(a.h32 + ((bh * a.N + n) * K + c) * (long)a.V + v0 + cb * 16);
-        dst[0] = make_float4(v[0], v[1], v[2], v[3]);
-        dst[1] = make_float4(v[4], v[5], v[6], v[7]);
-        dst[2] = make_float4(v[8], v[9], v[10], v[11]);
-        dst[3] = make_float4(v[12], v[13], v[14], v[15]);
+        float4 *dst = reinterpret_cast<float4 *>(a.h32 + ((bh * a.N + n) * K + c) * (long)a.V + v0 + cb * 32);
+#pragma unroll
+        for (int h = 0; h < 8; ++h) dst[h] = make_float4(v[4 * h], v[4 * h + 1], v[4 * h + 2], v[4 * h + 3]);
       }
 #pragma unroll
-      for (int e = 0; e < 16; ++e) v[e] *= g;
-      dev::tmem_st16(tS + cb * 16, v);
+      for (int e = 0; e < 32; ++e) v[e] *= g;
+      dev::tmem_st16(tS + cb * 32, v);
+      dev::tmem_st16(tS + cb * 32 + 16, v + 16);
     }
     dev::tmem_wait_st();
     dev::fence_proxy_async_smem();
@@ -531,8 +546,9 @@ __global__ void __launch_bounds__(K, 2)
 
   // ---- final state of the segment ---------------------------------------------
   if (a.gseg && vt == 0) a.gseg[(bh * P + seg) * K + c] = gprod;
-  if (a.end) {
-    float *dst = a.end + ((bh * P + seg) * K + c) * (long)a.V + v0;
+  if (a.end && (a.end_seg < 0 || a.end_seg == seg)) {
+    float *dst = (a.end_seg < 0) ? a.end + ((bh * P + seg) * K + c) * (long)a.V + v0
+                                 : a.end + (bh * K + c) * (long)a.V + v0;
 #pragma unroll
     for (int cb = 0; cb < BV / 16; ++cb) {
       float v[16];
@@ -559,9 +575,13 @@ __global__ void __launch_bounds__(K, 2)
 struct ScanArgs {
   int K, V, P, reverse;
   const float *gseg, *delta, *init;
-  float *start, *final_out;
+  float *start;
 };
 
+// start[p] for every segment p.  Forward: start[0] = init (h0), start[p] =
+// gseg[p-1] start[p-1] + delta[p-1].  Reverse: start[P-1] = init (dh_final),
+// start[p] = gseg[p+1] start[p+1] + delta[p+1].  (The one segment whose delta no
+// start needs -- the last forward, the first in reverse -- is never read.)
 __global__ void k_scan(ScanArgs a) {
   const long idx = (long)blockIdx.x * blockDim.x + threadIdx.x;
   const long KV = (long)a.K * a.V;
@@ -572,9 +592,8 @@ __global__ void k_scan(ScanArgs a) {
   for (int pi = 0; pi < a.P; ++pi) {
     const int p = a.reverse ? a.P - 1 - pi : pi;
     a.start[(bh * a.P + p) * KV + idx] = S;
-    S = a.gseg[(bh * a.P + p) * a.K + c] * S + a.delta[(bh * a.P + p) * KV + idx];
+    if (pi + 1 < a.P) S = a.gseg[(bh * a.P + p) * a.K + c] * S + a.delta[(bh * a.P + p) * KV + idx];
   }
-  if (a.final_out) a.final_out[bh * KV + idx] = S;
 }
 
 }  // namespace tc

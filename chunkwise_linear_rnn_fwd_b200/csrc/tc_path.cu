@@ -186,6 +186,7 @@ int launch_walk(const Problem &p, const tc::WalkArgs &a, const WalkMaps &m, int 
   if (smem < 0) return GLA_ERR_CUDA;
   GLA_LAUNCH(K_TC_WALK, st,
              (tc::k_walk<K, BV><<<dim3(p.V / BV, P, p.BH), K, smem, st>>>(a, m.X, m.Y, m.Q, m.P, m.H)));
+  // P here is the number of segments this launch covers (a.seg0 .. a.seg0 + P - 1)
   return GLA_OK;
 }
 
@@ -197,9 +198,9 @@ int launch_walk_any(const Problem &p, const tc::WalkArgs &a, const WalkMaps &m, 
   return GLA_ERR_UNSUPPORTED_SHAPE;
 }
 
-int launch_scan(const Problem &p, const float *gseg, const float *delta, const float *init, float *start,
-                float *final_out, int P, int reverse, cudaStream_t st) {
-  tc::ScanArgs a{p.K, p.V, P, reverse, gseg, delta, init, start, final_out};
+int launch_scan(const Problem &p, const float *gseg, const float *delta, const float *init, float *start, int P,
+                int reverse, cudaStream_t st) {
+  tc::ScanArgs a{p.K, p.V, P, reverse, gseg, delta, init, start};
   const long KV = (long)p.K * p.V;
   GLA_LAUNCH(K_TC_SCAN, st, (tc::k_scan<<<dim3((unsigned)((KV + 255) / 256), p.BH), 256, 0, st>>>(a)));
   return GLA_OK;
@@ -251,18 +252,22 @@ int tc_fwd(const Problem &p, const void *q, const void *k, const void *v, const 
   a.gam = w.gam;
   a.out = (bf16 *)o;
   a.status = status;
+  a.end_seg = -1;
 
   if (p.variant == GLA_VARIANT_MATERIALIZED) {
     // pass 1: all chunk states in fp32 (sequential over chunks per (head, d_v tile))
     a.L = p.N;
+    a.P = 1;
     a.state_mode = 2;
     a.h32 = w.h32;
     a.h0 = h0;
     a.end = hT;
+    a.end_seg = 0;
     TRY(launch_walk_any(p, a, m, 1, st));
     // pass 2: every chunk's output in parallel from its materialised state
     tc::WalkArgs b = a;
     b.L = 1;
+    b.P = p.N;
     b.state_mode = 0;
     b.do_out = 1;
     b.start = w.h32;
@@ -274,19 +279,22 @@ int tc_fwd(const Problem &p, const void *q, const void *k, const void *v, const 
   const int P = segments_of(p, nvt);
   const int L = (p.N + P - 1) / P;
   a.L = L;
+  a.P = P;
+  a.do_out = 1;
+  a.end = hT;
+  a.end_seg = P - 1;
   if (P == 1) {
-    a.do_out = 1;
     a.h0 = h0;
-    a.end = hT;
     return launch_walk_any(p, a, m, 1, st);
   }
-  // pre-pass: each segment's contribution from a zero state
+  // pre-pass: the contribution of segments 0 .. P-2 from a zero state
   tc::WalkArgs pre = a;
+  pre.do_out = 0;
   pre.end = w.delta;
+  pre.end_seg = -1;
   pre.gseg = w.gseg;
-  TRY(launch_walk_any(p, pre, m, P, st));
-  TRY(launch_scan(p, w.gseg, w.delta, h0, w.start, hT, P, 0, st));
-  a.do_out = 1;
+  TRY(launch_walk_any(p, pre, m, P - 1, st));
+  TRY(launch_scan(p, w.gseg, w.delta, h0, w.start, P, 0, st));
   a.start = w.start;
   return launch_walk_any(p, a, m, P, st);
 }
@@ -326,14 +334,16 @@ int tc_bwd(const Problem &p, const void *q, const void *k, const void *v, const 
   a.N = p.N;
   a.V = p.V;
   a.L = L;
+  a.P = P;
   a.gam = w.gam;
   a.status = status;
+  a.end_seg = -1;
   if (P > 1) {
-    tc::WalkArgs pre = a;
+    tc::WalkArgs pre = a;  // segments 0 .. P-2, forward
     pre.end = w.delta;
     pre.gseg = w.gseg;
-    TRY(launch_walk_any(p, pre, mf, P, st));
-    TRY(launch_scan(p, w.gseg, w.delta, h0, w.start, nullptr, P, 0, st));
+    TRY(launch_walk_any(p, pre, mf, P - 1, st));
+    TRY(launch_scan(p, w.gseg, w.delta, h0, w.start, P, 0, st));
     a.start = w.start;
   } else {
     a.h0 = h0;
@@ -346,18 +356,23 @@ int tc_bwd(const Problem &p, const void *q, const void *k, const void *v, const 
   r.N = p.N;
   r.V = p.V;
   r.L = L;
+  r.P = P;
   r.reverse = 1;
   r.gam = w.gam;
   r.status = status;
+  r.end = dh0;
+  r.end_seg = 0;
   if (P > 1) {
-    tc::WalkArgs pre = r;
+    tc::WalkArgs pre = r;  // segments 1 .. P-1, backward
     pre.end = w.ddelta;
-    TRY(launch_walk_any(p, pre, mr, P, st));
-    TRY(launch_scan(p, w.gseg, w.ddelta, dhT, w.dstart, dh0, P, 1, st));
+    pre.end_seg = -1;
+    pre.seg0 = 1;
+    pre.gseg = w.gseg;
+    TRY(launch_walk_any(p, pre, mr, P - 1, st));
+    TRY(launch_scan(p, w.gseg, w.ddelta, dhT, w.dstart, P, 1, st));
     r.start = w.dstart;
   } else {
     r.h0 = dhT;
-    r.end = dh0;
   }
   r.state_mode = 1;
   TRY(launch_walk_any(p, r, mr, P, st));
