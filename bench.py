@@ -108,6 +108,22 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+def reduce_max_ms(ms_local: float, world: int, device=None) -> float:
+    """Max of a per-rank duration over all ranks (the slowest rank defines the step)."""
+    if world <= 1:
+        return ms_local
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([ms_local], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_value(tokens_per_rank_step: int, world: int, steps: int, ms_max: float) -> float:
+    """Whole-job throughput: every rank's tokens over the slowest rank's time."""
+    return tokens_per_rank_step * world * steps / (ms_max / 1e3)
+
+
 def dist_env():
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -201,14 +217,16 @@ def run_ours(args, w):
     hT = torch.empty(B, H, K, V, dtype=torch.float32, device=dev)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     dla = torch.empty_like(la)
-    ws_f = pkg.alloc_workspace(pkg.workspace_size(B, H, T, K, V, torch.bfloat16, w["gate"], C, False), dev)
-    ws_b = pkg.alloc_workspace(pkg.workspace_size(B, H, T, K, V, torch.bfloat16, w["gate"], C, True), dev)
+    # one workspace for both calls: the backward reuses the forward's per-chunk prep
+    # outputs (GLA_FLAG_REUSE_PREP); chunk states are recomputed by the backward
+    ws = pkg.alloc_workspace(max(pkg.workspace_size(B, H, T, K, V, torch.bfloat16, w["gate"], C, False),
+                                 pkg.workspace_size(B, H, T, K, V, torch.bfloat16, w["gate"], C, True)), dev)
     stream = torch.cuda.current_stream()
 
     def step(qq=q, kk=k, vv=v, ll=la, dd=do):
-        pkg.gla_fwd(qq, kk, vv, ll, None, chunk=C, o=o, h_final=hT, workspace=ws_f, stream=stream)
+        pkg.gla_fwd(qq, kk, vv, ll, None, chunk=C, o=o, h_final=hT, workspace=ws, stream=stream)
         pkg.gla_bwd(qq, kk, vv, ll, dd, None, None, chunk=C, dq=dq, dk=dk, dv=dv, dlog_alpha=dla, want_dh0=False,
-                    workspace=ws_b, stream=stream)
+                    workspace=ws, stream=stream, reuse_prep=True)
 
     for _ in range(args.warmup):
         step()
@@ -235,14 +253,9 @@ def run_ours(args, w):
     launches = pkg.timing_collect()
     pkg.timing_enable(False)
     clocks = sampler.stop()
-    ms = ms_local
-    if world > 1:
-        t = torch.tensor([ms_local], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = reduce_max_ms(ms_local, world, dev)
     ms_per_step = ms / args.steps
-    tokens = B * T * world * args.steps
-    value = tokens / (ms / 1e3)
+    value = aggregate_value(B * T, world, args.steps, ms)
 
     # ---- end to end through the public API with host buffers ----------------------------
     pin = lambda t: t.cpu().pin_memory()
@@ -272,12 +285,8 @@ def run_ours(args, w):
         e2e_step()
     f1.record(stream)
     torch.cuda.synchronize()
-    ems = f0.elapsed_time(f1)
-    if world > 1:
-        t = torch.tensor([ems], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ems = float(t.item())
-    e2e_value = B * T * world * n_e2e / (ems / 1e3)
+    ems = reduce_max_ms(f0.elapsed_time(f1), world, dev)
+    e2e_value = aggregate_value(B * T, world, n_e2e, ems)
 
     # ---- roofline of the dominant kernel --------------------------------------------------
     peaks, peak_src = load_peaks()

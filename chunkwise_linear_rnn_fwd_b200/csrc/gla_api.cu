@@ -72,6 +72,7 @@ int make_problem(const gla_desc *d, int chunk, Problem *p) {
   if (d->variant != GLA_VARIANT_AUTO && d->variant != GLA_VARIANT_FUSED && d->variant != GLA_VARIANT_MATERIALIZED)
     return GLA_ERR_INVALID_ARG;
   if (d->segments < 0) return GLA_ERR_INVALID_ARG;
+  if (d->flags & ~GLA_FLAG_REUSE_PREP) return GLA_ERR_INVALID_ARG;
   const int sub = d->subchunk == 0 ? 16 : d->subchunk;
   if (chunk != 16 && chunk != 32 && chunk != 64 && chunk != 128) return GLA_ERR_UNSUPPORTED_SHAPE;
   if (sub < 1 || chunk % sub != 0) return GLA_ERR_UNSUPPORTED_SHAPE;
@@ -89,6 +90,7 @@ int make_problem(const gla_desc *d, int chunk, Problem *p) {
   p->c = sub;
   p->variant = d->variant;
   p->segments = d->segments;
+  p->flags = d->flags;
   p->BH = (long)d->B * d->H;
   p->N = (d->T + chunk - 1) / chunk;
   p->Tp = (long)p->N * chunk;

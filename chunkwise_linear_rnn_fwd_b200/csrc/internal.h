@@ -37,7 +37,7 @@ void timing_end(int kid, cudaStream_t s);
 // Everything a launcher needs about one call.
 struct Problem {
   int B, H, T, K, V;
-  int dtype, gate, C, c, variant, segments;
+  int dtype, gate, C, c, variant, segments, flags;
   long BH;     // B*H
   int N;       // chunks per sequence
   long Tp;     // N*C (padded tokens per head)

@@ -305,7 +305,9 @@ int tc_bwd(const Problem &p, const void *q, const void *k, const void *v, const 
   if (device_ok() != 1) return GLA_ERR_NO_DEVICE;
   TcWs w = carve(p, ws, true);
   unsigned *status = (unsigned *)ws;
-  TRY(launch_prep_any(p, (const bf16 *)q, (const bf16 *)k, la, w, status, st));
+  // qg, kg, P^T and gam sit at the same workspace offsets for gla_fwd and gla_bwd,
+  // so a forward run on this workspace can hand them over
+  if (!(p.flags & GLA_FLAG_REUSE_PREP)) TRY(launch_prep_any(p, (const bf16 *)q, (const bf16 *)k, la, w, status, st));
   const int BV = bv_of(p);
   const int nvt = p.V / BV;
   Problem pf = p;

@@ -41,7 +41,8 @@ class GLAError(RuntimeError):
 class gla_desc(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("T", ctypes.c_int), ("dk", ctypes.c_int),
                 ("dv", ctypes.c_int), ("dtype", ctypes.c_int), ("gate", ctypes.c_int), ("subchunk", ctypes.c_int),
-                ("variant", ctypes.c_int), ("segments", ctypes.c_int), ("workspace", ctypes.c_void_p),
+                ("variant", ctypes.c_int), ("segments", ctypes.c_int), ("flags", ctypes.c_int),
+                ("workspace", ctypes.c_void_p),
                 ("workspace_bytes", ctypes.c_size_t)]
 
 
@@ -109,7 +110,10 @@ def _gate_of(log_alpha, gate):
     return "vector" if log_alpha.dim() == 4 else "scalar"
 
 
-def make_desc(B, H, T, dk, dv, dtype, gate, *, subchunk=16, variant="auto", segments=0,
+FLAG_REUSE_PREP = 1
+
+
+def make_desc(B, H, T, dk, dv, dtype, gate, *, subchunk=16, variant="auto", segments=0, flags=0,
               workspace: Optional[torch.Tensor] = None) -> gla_desc:
     d = gla_desc()
     d.B, d.H, d.T, d.dk, d.dv = int(B), int(H), int(T), int(dk), int(dv)
@@ -118,6 +122,7 @@ def make_desc(B, H, T, dk, dv, dtype, gate, *, subchunk=16, variant="auto", segm
     d.subchunk = int(subchunk)
     d.variant = VARIANT[variant] if isinstance(variant, str) else int(variant)
     d.segments = int(segments)
+    d.flags = int(flags)
     if workspace is not None:
         d.workspace = workspace.data_ptr()
         d.workspace_bytes = workspace.numel() * workspace.element_size()
@@ -182,8 +187,10 @@ def gla_fwd_noalloc(q, k, v, log_alpha=None, h0=None, *, chunk=64, gate=None, su
 
 
 def gla_bwd(q, k, v, log_alpha, do, h0=None, dh_final=None, *, chunk=64, gate=None, subchunk=16, dq=None, dk=None,
-            dv=None, dlog_alpha=None, dh0=None, want_dh0=True, workspace=None, stream=None):
-    """Backward.  Returns (dq, dk, dv, dlog_alpha or None, dh0 or None).  See include/gla.h."""
+            dv=None, dlog_alpha=None, dh0=None, want_dh0=True, workspace=None, stream=None, reuse_prep=False):
+    """Backward.  Returns (dq, dk, dv, dlog_alpha or None, dh0 or None).  See include/gla.h.
+    reuse_prep=True: `workspace` holds the prep outputs of a gla_fwd call on the same
+    inputs with this workspace (GLA_FLAG_REUSE_PREP)."""
     lib = load()
     B, H, T, dk_ = q.shape
     dv_ = v.shape[-1]
@@ -198,7 +205,8 @@ def gla_bwd(q, k, v, log_alpha, do, h0=None, dh_final=None, *, chunk=64, gate=No
     if workspace is None:
         workspace = alloc_workspace(workspace_size(B, H, T, dk_, dv_, q.dtype, gate, chunk, True, subchunk=subchunk),
                                     q.device)
-    d = make_desc(B, H, T, dk_, dv_, q.dtype, gate, subchunk=subchunk, workspace=workspace)
+    d = make_desc(B, H, T, dk_, dv_, q.dtype, gate, subchunk=subchunk, workspace=workspace,
+                  flags=FLAG_REUSE_PREP if reuse_prep else 0)
     r = lib.gla_bwd(ctypes.byref(d), _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(h0), _ptr(do), _ptr(dh_final),
                     _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dlog_alpha), _ptr(dh0), int(chunk), _stream_handle(stream))
     if r != GLA_OK:

@@ -79,6 +79,15 @@ extern "C" {
  *               first, then all chunk outputs are computed in parallel
  *               ("sequence-level chunk parallelism").
  * AUTO          FUSED with the segment count chosen to fill the GPU. */
+/* gla_bwd only: desc->workspace already holds the per-chunk prep outputs
+ * (gate-rescaled q and k, intra-chunk scores, chunk decays) that a gla_fwd call
+ * wrote into this same workspace for the same q, k, log_alpha, shape, gate and
+ * chunk, and nothing has written to the workspace since.  The backward then
+ * reads them instead of recomputing them (chunk states are still recomputed).
+ * The workspace must be sized for the backward (gla_workspace_size(.., 1)),
+ * which is at least the forward's size.  Ignored by the fp32 path. */
+#define GLA_FLAG_REUSE_PREP 1
+
 #define GLA_VARIANT_AUTO 0
 #define GLA_VARIANT_FUSED 1
 #define GLA_VARIANT_MATERIALIZED 2
@@ -91,6 +100,7 @@ typedef struct gla_desc {
   int subchunk;         /* secondary chunk size; 0 = 16                                    */
   int variant;          /* GLA_VARIANT_* (forward only)                                    */
   int segments;         /* segments per sequence for the FUSED variant; 0 = automatic      */
+  int flags;            /* GLA_FLAG_* (0 = none)                                           */
   void *workspace;      /* device scratch owned by the caller, 256-byte aligned            */
   size_t workspace_bytes;
 } gla_desc;

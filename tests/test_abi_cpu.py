@@ -60,6 +60,8 @@ def test_check_and_workspace(lib):
     assert lib.gla_check(ctypes.byref(desc(subchunk=24)), 64) == -2
     assert lib.gla_workspace_size(ctypes.byref(desc(T=0)), 64, 0) == 0
     assert lib.gla_check(None, 64) == -1
+    assert lib.gla_check(ctypes.byref(desc(flags=1)), 64) == 0
+    assert lib.gla_check(ctypes.byref(desc(flags=2)), 64) == -1
 
 
 def test_bad_calls_enqueue_nothing(lib):

@@ -109,3 +109,11 @@ def test_segment_counts_bf16(segments):
 def test_h0_and_dh_final_bf16_large_dims():
     errs = run_case(1, 3, 700, 256, 512, dtype=BF16, chunk=64, seed=7, with_h0=True, with_dh_final=True)
     assert_parity(errs, BF16)
+
+
+@pytest.mark.parametrize("gate", ["vector", "scalar"])
+def test_backward_reusing_forward_prep(gate):
+    """gla_bwd with GLA_FLAG_REUSE_PREP on the workspace its gla_fwd filled."""
+    errs = run_case(2, 2, 777, 256, 512, dtype=BF16, gate=gate, chunk=64, seed=8, with_h0=True,
+                    with_dh_final=True, reuse_prep=True)
+    assert_parity(errs, BF16)
