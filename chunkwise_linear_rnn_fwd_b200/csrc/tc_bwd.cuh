@@ -272,7 +272,7 @@ __global__ void __launch_bounds__(256, 1)
 
   // per key channel: cumulative log-gate and the rescaled operands
   float Bv[kC];
-  float z[5], Gam[4], E[4];
+  float z[5], Gam[4], E[4], Gafter[4];
   const long qrow0 = bh * a.T + (long)n * kC;  // first token row of this chunk
   const uint32_t sQt = dev::smem_u32(smem + L::kQt), sKt = dev::smem_u32(smem + L::kKt);
   auto qk_at = [&](int t, float &qf, float &kf) {
@@ -282,6 +282,10 @@ __global__ void __launch_bounds__(256, 1)
     qf = __bfloat162float(*reinterpret_cast<const bf16 *>(&qb));
     kf = __bfloat162float(*reinterpret_cast<const bf16 *>(&kb));
   };
+  // 128-row block of this warp's key channels; warps without channels (d_k = 128,
+  // warps 4-7) mirror block 0 so their warp-collective TMEM loads stay in bounds
+  const int mb = ((warp >> 2) < kMB) ? (warp >> 2) : 0;
+  const uint32_t lanebase = 32 * (warp & 3);
   if (tid < K) {
 #pragma unroll
     for (int t = 0; t < kC; ++t) {
@@ -308,39 +312,66 @@ __global__ void __launch_bounds__(256, 1)
       Gam[j] = __expf(z[j + 1] - z[j]);
       E[j] = __expf(z[j]);
     }
+    Gafter[3] = 1.f;
+    Gafter[2] = Gam[3];
+    Gafter[1] = Gam[3] * Gam[2];
+    Gafter[0] = Gam[3] * Gam[2] * Gam[1];
   }
   if (!dev::mbar_wait(qk_bar, 0, a.status)) ok = false;
+
+  // window construction + boundary term G_n = gam_n R + sum_t k_t dk_inter_t
+  float Gb = 0.f;
   if (tid < K) {
+    Gb = a.gam[(bh * a.N + n) * K + c] * R;
     const uint32_t sKh = dev::smem_u32(smem + L::kKh), sQh = dev::smem_u32(smem + L::kQh);
     const int wK[4] = {0, 0, 16, 48};    // key window j >= 1: row wK[j] + s, s in [0, 16j)
     const int wQ[4] = {-16, 16, 32, 0};  // query window u <= 2: row wQ[u] + t, t in [16(u+1), 64)
+#pragma unroll 1
+    for (int j = 0; j < 4; ++j) {
+      float Bc[16], xk[16];
+      dev::take16(Bv, j, Bc);
+      dev::tmem_ld16(dev::tmem_addr(tmem, lanebase, cDK + 64 * mb + 16 * j), xk);
+      dev::tmem_wait_ld();
+      const float zj = dev::sel4(j, z[0], z[1], z[2], z[3]);
+      const float zj1 = dev::sel4(j, z[1], z[2], z[3], z[4]);
+      const float GAj = dev::sel4(j, Gafter[0], Gafter[1], Gafter[2], Gafter[3]);
 #pragma unroll
-    for (int t = 0; t < kC; ++t) {
-      const int j = t >> 4;
-      float qf, kf;
-      qk_at(t, qf, kf);
-      const float u = __expf(Bv[t] - z[j]);
-      const float w = __expf(z[j + 1] - Bv[t]);
-      // key operand k_t e^{z_jq - B_t} for later query sub-chunks jq > j
-      float f = kf * w;
+      for (int e = 0; e < 16; ++e) {
+        const int t = 16 * j + e;
+        float qf, kf;
+        qk_at(t, qf, kf);
+        const float u = __expf(Bc[e] - zj);
+        const float w = __expf(zj1 - Bc[e]);
+        Gb += kf * w * GAj * xk[e];
+        // key operand k_t e^{z_jq - B_t} for later query sub-chunks jq > j
+        float f = kf * w;
 #pragma unroll
-      for (int jq = 1; jq < 4; ++jq) {
-        if (jq > j) {
-          const bf16 b = __float2bfloat16_rn(f);
-          dev::st_shared_u16(sKh + dev::sw128_off(L::kRowsW, wK[jq] + t, c), *reinterpret_cast<const uint16_t *>(&b));
-          f *= Gam[jq];
+        for (int jq = 1; jq < 4; ++jq) {
+          if (jq > j) {
+            const bf16 b = __float2bfloat16_rn(f);
+            dev::st_shared_u16(sKh + dev::sw128_off(L::kRowsW, wK[jq] + t, c), *reinterpret_cast<const uint16_t *>(&b));
+            f *= Gam[jq];
+          }
+        }
+        // query operand q_t e^{B_t - z_{uu+1}} for earlier key sub-chunks uu < j
+        float g2 = qf * u;
+#pragma unroll
+        for (int uu = 2; uu >= 0; --uu) {
+          if (uu < j) {
+            const bf16 b = __float2bfloat16_rn(g2);
+            dev::st_shared_u16(sQh + dev::sw128_off(L::kRowsW, wQ[uu] + t, c), *reinterpret_cast<const uint16_t *>(&b));
+            g2 *= Gam[uu];
+          }
         }
       }
-      // query operand q_t e^{B_t - z_{uu+1}} for earlier key sub-chunks uu < j
-      float g2 = qf * u;
-#pragma unroll
-      for (int uu = 2; uu >= 0; --uu) {
-        if (uu < j) {
-          const bf16 b = __float2bfloat16_rn(g2);
-          dev::st_shared_u16(sQh + dev::sw128_off(L::kRowsW, wQ[uu] + t, c), *reinterpret_cast<const uint16_t *>(&b));
-          g2 *= Gam[uu];
-        }
-      }
+    }
+  } else {
+    // warps without key channels still take part in the warp-collective TMEM loads
+#pragma unroll 1
+    for (int j = 0; j < 4; ++j) {
+      float xk[16];
+      dev::tmem_ld16(dev::tmem_addr(tmem, lanebase, cDK + 64 * mb + 16 * j), xk);
+      dev::tmem_wait_ld();
     }
   }
   dev::fence_proxy_async_smem();
@@ -373,36 +404,9 @@ __global__ void __launch_bounds__(256, 1)
   dev::tc_fence_after();
 
   // ============================ epilogue ============================
-  const int mb = warp >> 2;
-  const uint32_t lanebase = 32 * (warp & 3);
-  // pass A: boundary term G_n = gam_n R + sum_t k_t dk_inter_t
-  float Gb = 0.f;
-  if (tid < K) {
-    Gb = a.gam[(bh * a.N + n) * K + c] * R;
-  }
-#pragma unroll
-  for (int t16 = 0; t16 < 4; ++t16) {
-    float xk[16];
-    dev::tmem_ld16(dev::tmem_addr(tmem, lanebase, cDK + 64 * mb + 16 * t16), xk);
-    dev::tmem_wait_ld();
-    if (tid < K) {
-      const int j = t16;
-      float Gafter = 1.f;
-#pragma unroll
-      for (int i2 = 1; i2 < 4; ++i2)
-        if (i2 > j) Gafter *= Gam[i2];
-#pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        const int t = 16 * t16 + e;
-        float qf, kf;
-        qk_at(t, qf, kf);
-        Gb += kf * __expf(z[j + 1] - Bv[t]) * Gafter * xk[e];
-      }
-    }
-  }
-  // pass B: reverse over sub-chunks and tokens; dq, dk, dlog b and its suffix sum
+  // reverse over sub-chunks and tokens: dq, dk, dlog b and its suffix sum
   float run = Gb;
-#pragma unroll
+#pragma unroll 1
   for (int t16 = 3; t16 >= 0; --t16) {
     const int j = t16;
     float xq[16], xk[16], xqi[16], xki[16];
@@ -411,32 +415,33 @@ __global__ void __launch_bounds__(256, 1)
     dev::tmem_ld16(dev::tmem_addr(tmem, lanebase, cQI + 64 * mb + 16 * t16), xqi);
     dev::tmem_ld16(dev::tmem_addr(tmem, lanebase, cKI + 64 * mb + 16 * t16), xki);
     dev::tmem_wait_ld();
-    float dqd[16], dkd[16];
-    float Gafter = 1.f;
-#pragma unroll
-    for (int i2 = 1; i2 < 4; ++i2)
-      if (i2 > j) Gafter *= Gam[i2];
     if (tid < K) {
+      float Bc[16];
+      dev::take16(Bv, j, Bc);
+      const float zj = dev::sel4(j, z[0], z[1], z[2], z[3]);
+      const float zj1 = dev::sel4(j, z[1], z[2], z[3], z[4]);
+      const float Ej = dev::sel4(j, E[0], E[1], E[2], E[3]);
+      const float invGj = 1.f / dev::sel4(j, Gam[0], Gam[1], Gam[2], Gam[3]);
+      const float GAj = dev::sel4(j, Gafter[0], Gafter[1], Gafter[2], Gafter[3]);
+      const float offq_on = (j > 0) ? 1.f : 0.f;  // no off-diagonal MMA wrote sub-chunk 0's dq columns
+      const float offk_on = (j < 3) ? 1.f : 0.f;  // ... nor sub-chunk 3's dk columns
       // diagonal block of sub-chunk j in fp32:
       //   a_t = q_t e^{B_t - z_j},  b_s = k_s e^{z_j - B_s}
       //   dq_t += e^{B_t - z_j} sum_{s<=t} dP[t,s] b_s ,  dk_s += e^{z_j - B_s} sum_{t>=s} dP[t,s] a_t
-      float av[16], bv[16], uu[16], ee[16];
+      float uu[16], ww[16], qv[16], kv[16], av[16], bv[16], dqd[16], dkd[16];
 #pragma unroll
       for (int e = 0; e < 16; ++e) {
-        const int t = 16 * j + e;
-        float qf, kf;
-        qk_at(t, qf, kf);
-        uu[e] = __expf(Bv[t] - z[j]);
-        ee[e] = __expf(z[j + 1] - Bv[t]) / Gam[j];
-        av[e] = qf * uu[e];
-        bv[e] = kf * ee[e];
+        qk_at(16 * j + e, qv[e], kv[e]);
+        uu[e] = __expf(Bc[e] - zj);
+        ww[e] = __expf(zj1 - Bc[e]);
+        av[e] = qv[e] * uu[e];
+        bv[e] = kv[e] * ww[e] * invGj;
         dqd[e] = 0.f;
         dkd[e] = 0.f;
       }
 #pragma unroll
       for (int e = 0; e < 16; ++e) {
-        const int t = 16 * j + e;
-        const float4 *rowp = reinterpret_cast<const float4 *>(dPd + t * 16);
+        const float4 *rowp = reinterpret_cast<const float4 *>(dPd + (16 * j + e) * 16);
         float pr[16];
 #pragma unroll
         for (int x4 = 0; x4 < 4; ++x4) {
@@ -453,41 +458,30 @@ __global__ void __launch_bounds__(256, 1)
         }
       }
 #pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        dqd[e] *= uu[e];
-        dkd[e] *= ee[e];
-      }
-    }
-#pragma unroll
-    for (int e = 15; e >= 0; --e) {
-      const int t = 16 * t16 + e;
-      const long tg = (long)n * kC + t;
-      float dlb = 0.f;
-      if (tid < K) {
-        float qf, kf;
-        qk_at(t, qf, kf);
-        const float u = __expf(Bv[t] - z[j]);
-        const float w = __expf(z[j + 1] - Bv[t]);
-        const float offq = (j > 0) ? xqi[e] : 0.f;
-        const float offk = (j < 3) ? xki[e] : 0.f;
-        const float dqr = u * (E[j] * xq[e] + offq);
-        const float dkr = w * (Gafter * xk[e] + offk);
-        const float dqv = dqr + dqd[e];
-        const float dkv = dkr + dkd[e];
-        run += (qf * dqr - kf * dkr) + (qf * dqd[e] - kf * dkd[e]);
-        dlb = run;
+      for (int e = 15; e >= 0; --e) {
+        const int t = 16 * j + e;
+        const long tg = (long)n * kC + t;
+        const float dqd_e = dqd[e] * uu[e];
+        const float dkd_e = dkd[e] * ww[e] * invGj;
+        const float dqr = uu[e] * (Ej * xq[e] + offq_on * xqi[e]);
+        const float dkr = ww[e] * (GAj * xk[e] + offk_on * xki[e]);
+        run += (qv[e] * dqr - kv[e] * dkr) + (qv[e] * dqd_e - kv[e] * dkd_e);
         if (tg < a.T && ok) {
-          a.dq[(qrow0 + t) * K + c] = __float2bfloat16_rn(dqv);
-          a.dk[(qrow0 + t) * K + c] = __float2bfloat16_rn(dkv);
-          if (a.gate == GLA_GATE_VECTOR) a.dla[(qrow0 + t) * K + c] = dlb;
+          a.dq[(qrow0 + t) * K + c] = __float2bfloat16_rn(dqr + dqd_e);
+          a.dk[(qrow0 + t) * K + c] = __float2bfloat16_rn(dkr + dkd_e);
+          if (a.gate == GLA_GATE_VECTOR) a.dla[(qrow0 + t) * K + c] = run;
+        }
+        if (a.gate == GLA_GATE_SCALAR) {
+          float x = run;
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+          if (lane == 0) red[warp * 64 + t] = x;
         }
       }
-      if (a.gate == GLA_GATE_SCALAR) {
-        float x = dlb;
+    } else if (a.gate == GLA_GATE_SCALAR) {
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
-        if (lane == 0) red[warp * 64 + t] = x;
-      }
+      for (int e = 15; e >= 0; --e)
+        if (lane == 0) red[warp * 64 + 16 * j + e] = 0.f;
     }
   }
   if (a.gate == GLA_GATE_SCALAR) {

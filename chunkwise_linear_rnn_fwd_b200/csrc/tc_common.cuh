@@ -229,6 +229,33 @@ __device__ __forceinline__ uint32_t sw128_chunk(int R, int r, int c8) {
   return (uint32_t)(c8 >> 3) * (uint32_t)R * 128u + (uint32_t)r * 128u + ((uint32_t)((c8 & 7) ^ (r & 7)) << 4);
 }
 
+// v[j] for a run-time j in [0,4) without dynamic register indexing.
+__device__ __forceinline__ float sel4(int j, float a0, float a1, float a2, float a3) {
+  return j == 0 ? a0 : (j == 1 ? a1 : (j == 2 ? a2 : a3));
+}
+
+// dst[e] = src[16 j + e], e < 16, for a run-time j in [0,4) (src stays in registers).
+__device__ __forceinline__ void take16(const float *src, int j, float *dst) {
+  switch (j) {
+    case 0:
+#pragma unroll
+      for (int e = 0; e < 16; ++e) dst[e] = src[e];
+      break;
+    case 1:
+#pragma unroll
+      for (int e = 0; e < 16; ++e) dst[e] = src[16 + e];
+      break;
+    case 2:
+#pragma unroll
+      for (int e = 0; e < 16; ++e) dst[e] = src[32 + e];
+      break;
+    default:
+#pragma unroll
+      for (int e = 0; e < 16; ++e) dst[e] = src[48 + e];
+      break;
+  }
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t *>(&h);

@@ -146,10 +146,18 @@ __global__ void __launch_bounds__(256, 1)
   bf16 *qg = a.qg + (bh * a.Tp + (long)n * kC) * K;
   bf16 *kg = a.kg + (bh * a.Tp + (long)n * kC) * K;
   const int wrow[4] = {0, 0, 16, 48};  // window start row of query sub-chunk j (j >= 1)
-#pragma unroll
+#pragma unroll 1
   for (int j = 0; j < 4; ++j) {
     // ---- rescaled operands of sub-chunk j ----
     if (tid < K) {
+      float Bc[16];
+      dev::take16(Bv, j, Bc);
+      const float zj = dev::sel4(j, z[0], z[1], z[2], z[3]);
+      const float zj1 = dev::sel4(j, z[1], z[2], z[3], z[4]);
+      const float Ej = dev::sel4(j, E[0], E[1], E[2], E[3]);
+      const float Gj = dev::sel4(j, Gam[0], Gam[1], Gam[2], Gam[3]);
+      const float GAj = dev::sel4(j, Gafter[0], Gafter[1], Gafter[2], Gafter[3]);
+      const float invGj = 1.f / Gj;
 #pragma unroll
       for (int e = 0; e < 16; ++e) {
         const int t = 16 * j + e;
@@ -158,16 +166,16 @@ __global__ void __launch_bounds__(256, 1)
         asm volatile("ld.shared.u16 %0, [%1];" : "=h"(kb) : "r"(sK + dev::sw128_off(64, t, c)));
         const float qf = ok_ld ? __bfloat162float(*reinterpret_cast<const bf16 *>(&qb)) : 0.f;
         const float kf = ok_ld ? __bfloat162float(*reinterpret_cast<const bf16 *>(&kb)) : 0.f;
-        const float u = __expf(Bv[t] - z[j]);
-        const float w = __expf(z[j + 1] - Bv[t]);
+        const float u = __expf(Bc[e] - zj);
+        const float w = __expf(zj1 - Bc[e]);
         const float qh = qf * u;
         const float kw = kf * w;
-        qg[(long)t * K + c] = __float2bfloat16_rn(qh * E[j]);
-        kg[(long)t * K + c] = __float2bfloat16_rn(kw * Gafter[j]);
+        qg[(long)t * K + c] = __float2bfloat16_rn(qh * Ej);
+        kg[(long)t * K + c] = __float2bfloat16_rn(kw * GAj);
         const bf16 qhb = __float2bfloat16_rn(qh);
         dev::st_shared_u16(sQh + dev::sw128_off(64, t, c), *reinterpret_cast<const uint16_t *>(&qhb));
         Af[f32_swz<K>(e, c)] = qh;
-        Bf[f32_swz<K>(e, c)] = kw / Gam[j];
+        Bf[f32_swz<K>(e, c)] = kw * invGj;
         // key operand for every later query sub-chunk jq: k_s e^{z_jq - B_s}
         float f = kw;
 #pragma unroll
