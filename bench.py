@@ -182,11 +182,37 @@ def run_reference(args, w):
 
 
 # ------------------------------------------------------------------------------------ ours
-def kernel_io_bytes(name, w):
-    """Bytes a launch of `name` must move at minimum (its own inputs + outputs, once)."""
+def walk_segments(w, sms):
+    """Segment count the library picks for the walks (one wave of two CTAs per SM)."""
+    B, H, T, K, V, C = w["B"], w["H"], w["T"], w["K"], w["V"], w["C"]
+    N = -(-T // C)
+    bv = 64 if (K == 256 or V % 128) else 128
+    P = max(1, (2 * sms) // (B * H * (V // bv)))
+    P = min(P, N)
+    L = -(-N // P)
+    return -(-N // L)
+
+
+def kernel_io_bytes(name, w, sms=148):
+    """Bytes the launches of `name` in one fwd+bwd step must move at minimum (their own
+    inputs + outputs, each once), divided by the number of those launches."""
     B, H, T, K, V, C = w["B"], w["H"], w["T"], w["K"], w["V"], w["C"]
     BH, N = B * H, -(-T // C)
     Tp = N * C
+    if name == "tc_walk":
+        P = walk_segments(w, sms)
+        f = (P - 1) / P                       # share of chunks a pre-pass covers
+        kx = BH * Tp * K * 2                  # qg or kg
+        vy = BH * T * V * 2                   # V or dO
+        seg = BH * (P - 1) * K * V * 4        # segment contributions (written, then read)
+        states = BH * N * K * V * 2           # bf16 chunk states h_n or dh_n
+        pt = BH * N * C * C * 2
+        pre = f * (kx + vy) + seg
+        fwd_out = 2 * kx + vy + pt + seg + vy + BH * K * V * 4
+        h_walk = kx + vy + seg + states
+        launches = (2 if P > 1 else 0) + 1 + 2 + (1 if P > 1 else 0)
+        total = (pre if P > 1 else 0) + fwd_out + 2 * ((pre if P > 1 else 0) + h_walk)
+        return total / launches
     g = 4 * K if w["gate"] == "vector" else (4 if w["gate"] == "scalar" else 0)
     if name == "tc_prep":
         return BH * T * (2 * K + 2 * K + g) + BH * Tp * 2 * (2 * K) + BH * N * (4 * K + 2 * C * C)
@@ -300,7 +326,7 @@ def run_ours(args, w):
     if dom is not None:
         n_l, tot = per_kernel[dom]
         avg_ms = tot / n_l
-        io = kernel_io_bytes(dom, w)
+        io = kernel_io_bytes(dom, w, torch.cuda.get_device_properties(dev).multi_processor_count)
         if io is not None:
             achieved = io / (avg_ms / 1e3) / 1e9
             peak = float(peaks["hbm_gbs"])

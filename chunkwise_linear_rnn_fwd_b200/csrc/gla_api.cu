@@ -11,7 +11,7 @@ namespace gla {
 const char *kernel_name(int id) {
   static const char *names[K_COUNT] = {
       "f32_prep",  "f32_states", "f32_scores", "f32_out",    "f32_dstates", "f32_dscores", "f32_dqk",
-      "f32_dv",    "f32_dg_out", "tc_prep",    "tc_walk",    "tc_scan",     "tc_bwd",      "status_clear"};
+      "f32_dv",    "f32_dg_out", "tc_prep",    "tc_walk",    "tc_scan(unused)", "tc_bwd",  "status_clear"};
   if (id < 0 || id >= K_COUNT) return "unknown";
   return names[id];
 }

@@ -299,10 +299,14 @@ struct WalkArgs {
   int end_seg;     // -1: every segment writes end[BH][P][K][V]; s >= 0: only segment s writes end[BH][K][V]
   int reverse, do_out, state_mode;  // state_mode: 0 none, 1 bf16 (TMA store), 2 fp32
   const float *gam;                 // [BH][N][K]
-  const float *start;               // [BH][P][K][V] fp32 or null
-  const float *h0;                  // used by segment 0 when start == null
+  const float *start;               // [BH][P][K][V] fp32 start states or null
+  const float *delta;               // [BH][P][K][V] segment contributions from a zero state (or null):
+                                    // the start state is then composed in the kernel from h0 and the
+                                    // contributions of the segments before this one (after it, reverse)
+  const float *h0;                  // initial state of the whole walk (h0, or dh_final in reverse) or null
   float *end;                       // [BH][P][K][V] fp32 or null (state after the segment)
   float *gseg;                      // [BH][P][K] product of gam over the segment (written by d_v tile 0) or null
+  const float *gseg_in;             // the same products, read when composing start states
   float *h32;                       // [BH][N][K][V] fp32 states (state_mode 2)
   bf16 *out;                        // [BH][T][V]
   unsigned *status;
@@ -413,29 +417,41 @@ __global__ void __launch_bounds__(K, 2)
   const long KV = (long)K * a.V;
 
   // ---- initial state into TMEM --------------------------------------------
+  // Composed segment start: S = h0; then for every earlier segment p (later, in
+  // reverse) S = diag(gseg_p) S + delta_p -- the scan over segments, done per row.
   {
+    const bool compose = (a.delta != nullptr);
     const float *src = nullptr;
     if (a.start) src = a.start + ((bh * P + seg) * K + c) * (long)a.V + v0;
-    else if (seg == 0 && a.h0) src = a.h0 + bh * KV + (long)c * a.V + v0;
+    else if (a.h0 && (compose || seg == (a.reverse ? P - 1 : 0))) src = a.h0 + bh * KV + (long)c * a.V + v0;
+    float S[BV];
 #pragma unroll
-    for (int cb = 0; cb < BV / 16; ++cb) {
-      float v[16];
-      if (src) {
-        const float4 *s4 = reinterpret_cast<const float4 *>(src + cb * 16);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float4 x = __ldg(s4 + e);
-          v[4 * e] = x.x;
-          v[4 * e + 1] = x.y;
-          v[4 * e + 2] = x.z;
-          v[4 * e + 3] = x.w;
-        }
-      } else {
-#pragma unroll
-        for (int e = 0; e < 16; ++e) v[e] = 0.f;
-      }
-      dev::tmem_st16(tS + cb * 16, v);
+    for (int x = 0; x < BV / 4; ++x) {
+      const float4 v4 = src ? __ldg(reinterpret_cast<const float4 *>(src) + x) : make_float4(0.f, 0.f, 0.f, 0.f);
+      S[4 * x] = v4.x;
+      S[4 * x + 1] = v4.y;
+      S[4 * x + 2] = v4.z;
+      S[4 * x + 3] = v4.w;
     }
+    if (compose) {
+      const int np = a.reverse ? (P - 1 - seg) : seg;
+#pragma unroll 1
+      for (int i = 0; i < np; ++i) {
+        const int p = a.reverse ? (P - 1 - i) : i;
+        const float gs = __ldg(a.gseg_in + (bh * P + p) * K + c);
+        const float4 *d4 = reinterpret_cast<const float4 *>(a.delta + ((bh * P + p) * K + c) * (long)a.V + v0);
+#pragma unroll
+        for (int x = 0; x < BV / 4; ++x) {
+          const float4 v4 = __ldg(d4 + x);
+          S[4 * x] = gs * S[4 * x] + v4.x;
+          S[4 * x + 1] = gs * S[4 * x + 1] + v4.y;
+          S[4 * x + 2] = gs * S[4 * x + 2] + v4.z;
+          S[4 * x + 3] = gs * S[4 * x + 3] + v4.w;
+        }
+      }
+    }
+#pragma unroll
+    for (int cb = 0; cb < BV / 16; ++cb) dev::tmem_st16(tS + cb * 16, S + 16 * cb);
     dev::tmem_wait_st();
   }
 
@@ -573,35 +589,6 @@ __global__ void __launch_bounds__(K, 2)
   dev::tc_fence_before();
   __syncthreads();
   if (warp == 0) dev::tmem_dealloc(tmem, kTmemCols);
-}
-
-// ============================================================================
-// Scan over segments (elementwise over the K x V state, sequential over P):
-//   start[p] = S;  S = diag(prod_{n in p} gam_n) S + delta[p]
-// run forwards from h0 (forward pass) or backwards from dh_final (adjoint).
-// ============================================================================
-struct ScanArgs {
-  int K, V, P, reverse;
-  const float *gseg, *delta, *init;
-  float *start;
-};
-
-// start[p] for every segment p.  Forward: start[0] = init (h0), start[p] =
-// gseg[p-1] start[p-1] + delta[p-1].  Reverse: start[P-1] = init (dh_final),
-// start[p] = gseg[p+1] start[p+1] + delta[p+1].  (The one segment whose delta no
-// start needs -- the last forward, the first in reverse -- is never read.)
-__global__ void k_scan(ScanArgs a) {
-  const long idx = (long)blockIdx.x * blockDim.x + threadIdx.x;
-  const long KV = (long)a.K * a.V;
-  const long bh = blockIdx.y;
-  if (idx >= KV) return;
-  const int c = (int)(idx / a.V);
-  float S = a.init ? a.init[bh * KV + idx] : 0.f;
-  for (int pi = 0; pi < a.P; ++pi) {
-    const int p = a.reverse ? a.P - 1 - pi : pi;
-    a.start[(bh * a.P + p) * KV + idx] = S;
-    if (pi + 1 < a.P) S = a.gseg[(bh * a.P + p) * a.K + c] * S + a.delta[(bh * a.P + p) * KV + idx];
-  }
 }
 
 }  // namespace tc

@@ -2,10 +2,10 @@
 //
 // Forward (section 4.2 chunkwise form, section 3.3 Figure 1 variants):
 //   prep                      qg, kg, gam, P^T per chunk (parallel over chunks)
-//   FUSED, P segments:        walk(no output) per segment from 0 -> delta_p,
-//                             scan -> segment start states and h_final,
-//                             walk(output) per segment from its start state
-//                             (P = 1: a single walk from h0 that also writes h_final)
+//   FUSED, P segments:        walk(no output) over segments 0..P-2 from 0 -> delta_p,
+//                             walk(output) per segment, each CTA composing its start
+//                             state from h0 and the earlier delta_p; the last segment
+//                             writes h_final (P = 1: a single walk from h0)
 //   MATERIALIZED:             walk(fp32 chunk states) over whole sequences, then
 //                             walk(output, one chunk per CTA) from those states.
 // Backward: see tc_bwd.
@@ -101,12 +101,12 @@ int segments_of(const Problem &p, int nvt) {
 struct TcWs {
   bf16 *qg, *kg, *PT;
   float *gam;
-  float *delta, *start;  // [BH][P][K][V]
+  float *delta;          // [BH][P][K][V] segment contributions
   float *gseg;           // [BH][P][K] per-segment gate products
   float *h32;            // materialised fp32 chunk states [BH][N][K][V]
   // backward
   bf16 *hb, *dhb;        // bf16 chunk states and adjoints [BH][N][K][V]
-  float *dstart, *ddelta;
+  float *ddelta;
   float *dscratch;       // bwd per-chunk scratch
   size_t bytes;
 };
@@ -125,7 +125,6 @@ TcWs carve(const Problem &p, void *ws, bool bwd) {
       w.h32 = cv.take<float>((size_t)p.BH * p.N * p.K * p.V);
     } else if (P > 1) {
       w.delta = cv.take<float>((size_t)p.BH * P * p.K * p.V);
-      w.start = cv.take<float>((size_t)p.BH * P * p.K * p.V);
       w.gseg = cv.take<float>((size_t)p.BH * P * p.K);
     }
   } else {
@@ -134,9 +133,7 @@ TcWs carve(const Problem &p, void *ws, bool bwd) {
     pf.segments = 0;
     const int P = segments_of(pf, nvt);
     w.delta = cv.take<float>((size_t)p.BH * P * p.K * p.V);
-    w.start = cv.take<float>((size_t)p.BH * P * p.K * p.V);
     w.ddelta = cv.take<float>((size_t)p.BH * P * p.K * p.V);
-    w.dstart = cv.take<float>((size_t)p.BH * P * p.K * p.V);
     w.gseg = cv.take<float>((size_t)p.BH * P * p.K);
     w.hb = cv.take<bf16>((size_t)p.BH * p.N * p.K * p.V);
     w.dhb = cv.take<bf16>((size_t)p.BH * p.N * p.K * p.V);
@@ -196,14 +193,6 @@ int launch_walk_any(const Problem &p, const tc::WalkArgs &a, const WalkMaps &m, 
   if (p.K == 128 && BV == 128) return launch_walk<128, 128>(p, a, m, P, st);
   if (p.K == 128 && BV == 64) return launch_walk<128, 64>(p, a, m, P, st);
   return GLA_ERR_UNSUPPORTED_SHAPE;
-}
-
-int launch_scan(const Problem &p, const float *gseg, const float *delta, const float *init, float *start, int P,
-                int reverse, cudaStream_t st) {
-  tc::ScanArgs a{p.K, p.V, P, reverse, gseg, delta, init, start};
-  const long KV = (long)p.K * p.V;
-  GLA_LAUNCH(K_TC_SCAN, st, (tc::k_scan<<<dim3((unsigned)((KV + 255) / 256), p.BH), 256, 0, st>>>(a)));
-  return GLA_OK;
 }
 
 int launch_prep_any(const Problem &p, const bf16 *q, const bf16 *k, const float *la, const TcWs &w, unsigned *status,
@@ -294,8 +283,9 @@ int tc_fwd(const Problem &p, const void *q, const void *k, const void *v, const 
   pre.end_seg = -1;
   pre.gseg = w.gseg;
   TRY(launch_walk_any(p, pre, m, P - 1, st));
-  TRY(launch_scan(p, w.gseg, w.delta, h0, w.start, P, 0, st));
-  a.start = w.start;
+  a.delta = w.delta;
+  a.gseg_in = w.gseg;
+  a.h0 = h0;
   return launch_walk_any(p, a, m, P, st);
 }
 
@@ -345,11 +335,10 @@ int tc_bwd(const Problem &p, const void *q, const void *k, const void *v, const 
     pre.end = w.delta;
     pre.gseg = w.gseg;
     TRY(launch_walk_any(p, pre, mf, P - 1, st));
-    TRY(launch_scan(p, w.gseg, w.delta, h0, w.start, P, 0, st));
-    a.start = w.start;
-  } else {
-    a.h0 = h0;
+    a.delta = w.delta;
+    a.gseg_in = w.gseg;
   }
+  a.h0 = h0;
   a.state_mode = 1;
   TRY(launch_walk_any(p, a, mf, P, st));
 
@@ -371,11 +360,10 @@ int tc_bwd(const Problem &p, const void *q, const void *k, const void *v, const 
     pre.seg0 = 1;
     pre.gseg = w.gseg;
     TRY(launch_walk_any(p, pre, mr, P - 1, st));
-    TRY(launch_scan(p, w.gseg, w.ddelta, dhT, w.dstart, P, 1, st));
-    r.start = w.dstart;
-  } else {
-    r.h0 = dhT;
+    r.delta = w.ddelta;
+    r.gseg_in = w.gseg;
   }
+  r.h0 = dhT;
   r.state_mode = 1;
   TRY(launch_walk_any(p, r, mr, P, st));
 
