@@ -262,16 +262,15 @@ __global__ void __launch_bounds__(256, 1)
           dev::st_shared_u16(sdPT + dev::sw128_off(64, s8 * 8 + e, t), *reinterpret_cast<const uint16_t *>(&b));
         }
       }
+      float dg[16];
+      dev::take16(row, jt, dg);  // the diagonal block's 16 entries of this row
 #pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        const int sidx = 16 * jt + e;
-        dPd[t * 16 + e] = (sidx <= t && ok) ? row[sidx] : 0.f;
-      }
+      for (int e = 0; e < 16; ++e) dPd[t * 16 + e] = (16 * jt + e <= t && ok) ? dg[e] : 0.f;
     }
   }
 
-  // per key channel: cumulative log-gate and the rescaled operands
-  float Bv[kC];
+  // per key channel: sub-chunk boundary values of the cumulative log-gate; the 16
+  // values inside sub-chunk j are rebuilt from log_alpha when needed (gate16)
   float z[5], Gam[4], E[4], Gafter[4];
   const long qrow0 = bh * a.T + (long)n * kC;  // first token row of this chunk
   const uint32_t sQt = dev::smem_u32(smem + L::kQt), sKt = dev::smem_u32(smem + L::kKt);
@@ -282,31 +281,40 @@ __global__ void __launch_bounds__(256, 1)
     qf = __bfloat162float(*reinterpret_cast<const bf16 *>(&qb));
     kf = __bfloat162float(*reinterpret_cast<const bf16 *>(&kb));
   };
+  // log_alpha of token 16 j + e of this chunk (0 beyond T)
+  auto gate_at = [&](int t) -> float {
+    if ((long)n * kC + t >= a.T) return 0.f;
+    if (a.gate == GLA_GATE_VECTOR) return __ldg(a.la + (qrow0 + t) * K + c);
+    if (a.gate == GLA_GATE_SCALAR) return __ldg(a.la + qrow0 + t);
+    return 0.f;
+  };
+  // Bc[e] = B at token 16 j + e (cumulative log-gate inside the chunk)
+  auto gate16 = [&](int j, float zj, float *Bc) {
+    float g[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) g[e] = gate_at(16 * j + e);
+    float acc = zj;
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      acc += g[e];
+      Bc[e] = acc;
+    }
+  };
   // 128-row block of this warp's key channels; warps without channels (d_k = 128,
   // warps 4-7) mirror block 0 so their warp-collective TMEM loads stay in bounds
   const int mb = ((warp >> 2) < kMB) ? (warp >> 2) : 0;
   const uint32_t lanebase = 32 * (warp & 3);
   if (tid < K) {
+    float g[kC];
 #pragma unroll
-    for (int t = 0; t < kC; ++t) {
-      float g = 0.f;
-      if ((long)n * kC + t < a.T) {
-        if (a.gate == GLA_GATE_VECTOR) g = __ldg(a.la + (qrow0 + t) * K + c);
-        else if (a.gate == GLA_GATE_SCALAR) g = __ldg(a.la + qrow0 + t);
-      }
-      Bv[t] = g;
-    }
+    for (int t = 0; t < kC; ++t) g[t] = gate_at(t);
     float acc = 0.f;
+    z[0] = 0.f;
 #pragma unroll
     for (int t = 0; t < kC; ++t) {
-      acc += Bv[t];
-      Bv[t] = acc;
+      acc += g[t];
+      if ((t & 15) == 15) z[(t >> 4) + 1] = acc;
     }
-    z[0] = 0.f;
-    z[1] = Bv[15];
-    z[2] = Bv[31];
-    z[3] = Bv[47];
-    z[4] = Bv[63];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       Gam[j] = __expf(z[j + 1] - z[j]);
@@ -329,10 +337,10 @@ __global__ void __launch_bounds__(256, 1)
 #pragma unroll 1
     for (int j = 0; j < 4; ++j) {
       float Bc[16], xk[16];
-      dev::take16(Bv, j, Bc);
+      const float zj = dev::sel4(j, z[0], z[1], z[2], z[3]);
+      gate16(j, zj, Bc);
       dev::tmem_ld16(dev::tmem_addr(tmem, lanebase, cDK + 64 * mb + 16 * j), xk);
       dev::tmem_wait_ld();
-      const float zj = dev::sel4(j, z[0], z[1], z[2], z[3]);
       const float zj1 = dev::sel4(j, z[1], z[2], z[3], z[4]);
       const float GAj = dev::sel4(j, Gafter[0], Gafter[1], Gafter[2], Gafter[3]);
 #pragma unroll
@@ -417,8 +425,8 @@ __global__ void __launch_bounds__(256, 1)
     dev::tmem_wait_ld();
     if (tid < K) {
       float Bc[16];
-      dev::take16(Bv, j, Bc);
       const float zj = dev::sel4(j, z[0], z[1], z[2], z[3]);
+      gate16(j, zj, Bc);
       const float zj1 = dev::sel4(j, z[1], z[2], z[3], z[4]);
       const float Ej = dev::sel4(j, E[0], E[1], E[2], E[3]);
       const float invGj = 1.f / dev::sel4(j, Gam[0], Gam[1], Gam[2], Gam[3]);
@@ -439,6 +447,7 @@ __global__ void __launch_bounds__(256, 1)
         dqd[e] = 0.f;
         dkd[e] = 0.f;
       }
+      // dP rows hold zeros beyond the diagonal, so pairs (f, f+1) may run one past e
 #pragma unroll
       for (int e = 0; e < 16; ++e) {
         const float4 *rowp = reinterpret_cast<const float4 *>(dPd + (16 * j + e) * 16);
@@ -451,11 +460,13 @@ __global__ void __launch_bounds__(256, 1)
           pr[4 * x4 + 2] = v4.z;
           pr[4 * x4 + 3] = v4.w;
         }
+        float q0 = 0.f, q1 = 0.f;
 #pragma unroll
-        for (int f = 0; f <= e; ++f) {
-          dqd[e] += pr[f] * bv[f];
-          dkd[f] += pr[f] * av[e];
+        for (int f = 0; f <= e; f += 2) {
+          dev::ffma2(q0, q1, pr[f], pr[f + 1], bv[f], bv[f + 1]);
+          dev::ffma2(dkd[f], dkd[f + 1], pr[f], pr[f + 1], av[e], av[e]);
         }
+        dqd[e] = q0 + q1;
       }
 #pragma unroll
       for (int e = 15; e >= 0; --e) {

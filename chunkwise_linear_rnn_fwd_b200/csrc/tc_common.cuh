@@ -229,6 +229,16 @@ __device__ __forceinline__ uint32_t sw128_chunk(int R, int r, int c8) {
   return (uint32_t)(c8 >> 3) * (uint32_t)R * 128u + (uint32_t)r * 128u + ((uint32_t)((c8 & 7) ^ (r & 7)) << 4);
 }
 
+// (d0, d1) += (a0, a1) * (b0, b1) as one packed fp32x2 FMA (sm_100).
+__device__ __forceinline__ void ffma2(float &d0, float &d1, float a0, float a1, float b0, float b1) {
+  uint64_t d, a, b;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(a) : "f"(a0), "f"(a1));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(b) : "f"(b0), "f"(b1));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "f"(d0), "f"(d1));
+  asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(d) : "l"(a), "l"(b));
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(d0), "=f"(d1) : "l"(d));
+}
+
 // v[j] for a run-time j in [0,4) without dynamic register indexing.
 __device__ __forceinline__ float sel4(int j, float a0, float a1, float a2, float a3) {
   return j == 0 ? a0 : (j == 1 ? a1 : (j == 2 ? a2 : a3));

@@ -435,7 +435,7 @@ __global__ void __launch_bounds__(K, 2)
     }
     if (compose) {
       const int np = a.reverse ? (P - 1 - seg) : seg;
-#pragma unroll 1
+#pragma unroll 2
       for (int i = 0; i < np; ++i) {
         const int p = a.reverse ? (P - 1 - i) : i;
         const float gs = __ldg(a.gseg_in + (bh * P + p) * K + c);
