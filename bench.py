@@ -208,10 +208,12 @@ def kernel_io_bytes(name, w, sms=148):
         states = BH * N * K * V * 2           # bf16 chunk states h_n or dh_n
         pt = BH * N * C * C * 2
         pre = f * (kx + vy) + seg
-        fwd_out = 2 * kx + vy + pt + seg + vy + BH * K * V * 4
-        h_walk = kx + vy + seg + states
-        launches = (2 if P > 1 else 0) + 1 + 2 + (1 if P > 1 else 0)
-        total = (pre if P > 1 else 0) + fwd_out + 2 * ((pre if P > 1 else 0) + h_walk)
+        # forward: pre-pass + output walk that also stores h_n (saved states);
+        # backward: reverse pre-pass + adjoint walk storing dh_n
+        fwd_out = 2 * kx + vy + pt + seg + vy + BH * K * V * 4 + states
+        dh_walk = kx + vy + seg + states
+        launches = 2 * (2 if P > 1 else 1)
+        total = 2 * (pre if P > 1 else 0) + fwd_out + dh_walk
         return total / launches
     g = 4 * K if w["gate"] == "vector" else (4 if w["gate"] == "scalar" else 0)
     if name == "tc_prep":
@@ -243,16 +245,17 @@ def run_ours(args, w):
     hT = torch.empty(B, H, K, V, dtype=torch.float32, device=dev)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     dla = torch.empty_like(la)
-    # one workspace for both calls: the backward reuses the forward's per-chunk prep
-    # outputs (GLA_FLAG_REUSE_PREP); chunk states are recomputed by the backward
-    ws = pkg.alloc_workspace(max(pkg.workspace_size(B, H, T, K, V, torch.bfloat16, w["gate"], C, False),
-                                 pkg.workspace_size(B, H, T, K, V, torch.bfloat16, w["gate"], C, True)), dev)
+    # one workspace for both calls: the forward stores its bf16 chunk states there
+    # (GLA_FLAG_SAVE_STATES) and the backward reads them and the forward's per-chunk
+    # prep outputs (GLA_FLAG_REUSE_PREP) instead of recomputing them
+    flags = pkg.FLAG_REUSE_PREP | pkg.FLAG_SAVE_STATES
+    ws = pkg.alloc_workspace(pkg.workspace_size(B, H, T, K, V, torch.bfloat16, w["gate"], C, True, flags=flags), dev)
     stream = torch.cuda.current_stream()
 
     def step(qq=q, kk=k, vv=v, ll=la, dd=do):
-        pkg.gla_fwd(qq, kk, vv, ll, None, chunk=C, o=o, h_final=hT, workspace=ws, stream=stream)
+        pkg.gla_fwd(qq, kk, vv, ll, None, chunk=C, o=o, h_final=hT, workspace=ws, stream=stream, save_states=True)
         pkg.gla_bwd(qq, kk, vv, ll, dd, None, None, chunk=C, dq=dq, dk=dk, dv=dv, dlog_alpha=dla, want_dh0=False,
-                    workspace=ws, stream=stream, reuse_prep=True)
+                    workspace=ws, stream=stream, reuse_prep=True, saved_states=True)
 
     for _ in range(args.warmup):
         step()

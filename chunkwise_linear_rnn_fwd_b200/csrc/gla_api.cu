@@ -72,7 +72,7 @@ int make_problem(const gla_desc *d, int chunk, Problem *p) {
   if (d->variant != GLA_VARIANT_AUTO && d->variant != GLA_VARIANT_FUSED && d->variant != GLA_VARIANT_MATERIALIZED)
     return GLA_ERR_INVALID_ARG;
   if (d->segments < 0) return GLA_ERR_INVALID_ARG;
-  if (d->flags & ~GLA_FLAG_REUSE_PREP) return GLA_ERR_INVALID_ARG;
+  if (d->flags & ~(GLA_FLAG_REUSE_PREP | GLA_FLAG_SAVE_STATES)) return GLA_ERR_INVALID_ARG;
   const int sub = d->subchunk == 0 ? 16 : d->subchunk;
   if (chunk != 16 && chunk != 32 && chunk != 64 && chunk != 128) return GLA_ERR_UNSUPPORTED_SHAPE;
   if (sub < 1 || chunk % sub != 0) return GLA_ERR_UNSUPPORTED_SHAPE;
@@ -166,7 +166,8 @@ int gla_fwd(const gla_desc *desc, const void *q, const void *k, const void *v, c
   GLA_TRY(check_gate_ptr(p, log_alpha));
   GLA_TRY(check_opt(h0));
   GLA_TRY(check_opt(h_final));
-  GLA_TRY(check_ws(desc, p, false));
+  // a forward that saves states for the backward writes into the backward's layout
+  GLA_TRY(check_ws(desc, p, (p.flags & GLA_FLAG_SAVE_STATES) != 0));
   cudaStream_t st = (cudaStream_t)stream;
   GLA_TRY(clear_status(desc, st));
   if (p.dtype == GLA_DTYPE_BF16) return tc_fwd(p, q, k, v, log_alpha, h0, o, h_final, desc->workspace, st);

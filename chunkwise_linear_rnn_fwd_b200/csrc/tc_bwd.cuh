@@ -136,29 +136,9 @@ __global__ void __launch_bounds__(256, 1)
     const int s = i & 1;
     uint8_t *st = stage(s);
     if (ok) ok = dev::mbar_wait(&full[s], (i >> 1) & 1, a.status);
-    if (tid < K) {
-      const uint32_t sh = dev::smem_u32(st), sdh = sh + L::kTileH;
-#pragma unroll
-      for (int c8 = 0; c8 < BVb / 8; ++c8) {
-        uint4 x, y;
-        asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];"
-                     : "=r"(x.x), "=r"(x.y), "=r"(x.z), "=r"(x.w)
-                     : "r"(sh + dev::sw128_chunk(K, c, c8)));
-        asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];"
-                     : "=r"(y.x), "=r"(y.y), "=r"(y.z), "=r"(y.w)
-                     : "r"(sdh + dev::sw128_chunk(K, c, c8)));
-        const __nv_bfloat162 *xh = reinterpret_cast<const __nv_bfloat162 *>(&x);
-        const __nv_bfloat162 *yh = reinterpret_cast<const __nv_bfloat162 *>(&y);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float2 xf = __bfloat1622float2(xh[e]), yf = __bfloat1622float2(yh[e]);
-          R += xf.x * yf.x + xf.y * yf.y;
-        }
-      }
-    }
-    dev::tc_fence_before();
-    __syncthreads();
-    dev::tc_fence_after();
+    // the previous tile's dv epilogue has released the dv accumulator (barrier at
+    // the end of the last iteration); issue this tile's MMAs, then sum h (.) dh
+    // from the same shared-memory tiles while they run
     if (tid == 0 && ok) {
       const uint32_t sH = dev::smem_u32(st), sDH = sH + L::kTileH, sV = sDH + L::kTileH, sDO = sV + L::kTileV;
       const uint32_t sKg = dev::smem_u32(smem + L::kKg), sPT = dev::smem_u32(smem + L::kPT);
@@ -191,8 +171,29 @@ __global__ void __launch_bounds__(256, 1)
                        id_dv2, 1u);
       dev::umma_commit(mma_bar);
     }
+    if (tid < K) {
+      const uint32_t sh = dev::smem_u32(st), sdh = sh + L::kTileH;
+#pragma unroll
+      for (int c8 = 0; c8 < BVb / 8; ++c8) {
+        uint4 x, y;
+        asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];"
+                     : "=r"(x.x), "=r"(x.y), "=r"(x.z), "=r"(x.w)
+                     : "r"(sh + dev::sw128_chunk(K, c, c8)));
+        asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];"
+                     : "=r"(y.x), "=r"(y.y), "=r"(y.z), "=r"(y.w)
+                     : "r"(sdh + dev::sw128_chunk(K, c, c8)));
+        const __nv_bfloat162 *xh = reinterpret_cast<const __nv_bfloat162 *>(&x);
+        const __nv_bfloat162 *yh = reinterpret_cast<const __nv_bfloat162 *>(&y);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 xf = __bfloat1622float2(xh[e]), yf = __bfloat1622float2(yh[e]);
+          R += xf.x * yf.x + xf.y * yf.y;
+        }
+      }
+    }
     if (ok) ok = dev::mbar_wait(mma_bar, i & 1, a.status);
     dev::tc_fence_after();
+    __syncthreads();  // every thread has finished reading stage s (R sums)
     if (tid == 0 && ok && i + 2 < nvt) issue_tile(i + 2);
     // dv epilogue: rows t (M = 64 layout), warps 0-3 columns [0,32), warps 4-7 [32,64)
     {
@@ -288,11 +289,12 @@ __global__ void __launch_bounds__(256, 1)
     if (a.gate == GLA_GATE_SCALAR) return __ldg(a.la + qrow0 + t);
     return 0.f;
   };
-  // Bc[e] = B at token 16 j + e (cumulative log-gate inside the chunk)
-  auto gate16 = [&](int j, float zj, float *Bc) {
-    float g[16];
+  // g[e] = log_alpha of token 16 j + e; Bc[e] = z_j + g[0] + ... + g[e] (cumulative log-gate)
+  auto load16 = [&](int j, float *g) {
 #pragma unroll
     for (int e = 0; e < 16; ++e) g[e] = gate_at(16 * j + e);
+  };
+  auto cumsum16 = [&](const float *g, float zj, float *Bc) {
     float acc = zj;
 #pragma unroll
     for (int e = 0; e < 16; ++e) {
@@ -334,11 +336,14 @@ __global__ void __launch_bounds__(256, 1)
     const uint32_t sKh = dev::smem_u32(smem + L::kKh), sQh = dev::smem_u32(smem + L::kQh);
     const int wK[4] = {0, 0, 16, 48};    // key window j >= 1: row wK[j] + s, s in [0, 16j)
     const int wQ[4] = {-16, 16, 32, 0};  // query window u <= 2: row wQ[u] + t, t in [16(u+1), 64)
+    float gnext[16];
+    load16(0, gnext);
 #pragma unroll 1
     for (int j = 0; j < 4; ++j) {
       float Bc[16], xk[16];
       const float zj = dev::sel4(j, z[0], z[1], z[2], z[3]);
-      gate16(j, zj, Bc);
+      cumsum16(gnext, zj, Bc);
+      if (j < 3) load16(j + 1, gnext);  // prefetch the next sub-chunk's gates
       dev::tmem_ld16(dev::tmem_addr(tmem, lanebase, cDK + 64 * mb + 16 * j), xk);
       dev::tmem_wait_ld();
       const float zj1 = dev::sel4(j, z[1], z[2], z[3], z[4]);
@@ -414,6 +419,8 @@ __global__ void __launch_bounds__(256, 1)
   // ============================ epilogue ============================
   // reverse over sub-chunks and tokens: dq, dk, dlog b and its suffix sum
   float run = Gb;
+  float gnext[16];
+  if (tid < K) load16(3, gnext);
 #pragma unroll 1
   for (int t16 = 3; t16 >= 0; --t16) {
     const int j = t16;
@@ -426,7 +433,8 @@ __global__ void __launch_bounds__(256, 1)
     if (tid < K) {
       float Bc[16];
       const float zj = dev::sel4(j, z[0], z[1], z[2], z[3]);
-      gate16(j, zj, Bc);
+      cumsum16(gnext, zj, Bc);
+      if (j > 0) load16(j - 1, gnext);  // prefetch the previous sub-chunk's gates
       const float zj1 = dev::sel4(j, z[1], z[2], z[3], z[4]);
       const float Ej = dev::sel4(j, E[0], E[1], E[2], E[3]);
       const float invGj = 1.f / dev::sel4(j, Gam[0], Gam[1], Gam[2], Gam[3]);

@@ -465,9 +465,9 @@ __global__ void __launch_bounds__(K, 2)
     const float g = g_next;
     if (i + 1 < nloc) g_next = __ldg(a.gam + (bh * a.N + chunk_of(i + 1)) * K + c);
     gprod *= g;
-    if (ok) ok = dev::mbar_wait(&full[s], (uint32_t)((i / nst) & 1), a.status);
 
     // ---- S-pass: read S, publish bf16/fp32 copy, scale by gamma ---------------
+    // (needs only the previous chunk's MMAs: it runs while this chunk's tiles load)
 #pragma unroll
     for (int cb = 0; cb < BV / 32; ++cb) {
       float v[32];
@@ -492,6 +492,7 @@ __global__ void __launch_bounds__(K, 2)
     }
     dev::tmem_wait_st();
     dev::fence_proxy_async_smem();
+    if (ok) ok = dev::mbar_wait(&full[s], (uint32_t)((i / nst) & 1), a.status);
     dev::tc_fence_before();
     __syncthreads();
     dev::tc_fence_after();

@@ -111,6 +111,18 @@ struct TcWs {
   size_t bytes;
 };
 
+// Segment count of the backward walks (and of a forward that saves states):
+// the FUSED choice for this descriptor whatever its forward variant.
+int bwd_segments(const Problem &p, int nvt) {
+  Problem pf = p;
+  pf.variant = GLA_VARIANT_FUSED;
+  return segments_of(pf, nvt);
+}
+
+// Workspace layout.  The forward layout is a prefix of the backward one up to
+// gam; the backward layout (also used by a forward with GLA_FLAG_SAVE_STATES)
+// keeps every offset independent of the forward variant: the MATERIALIZED
+// fp32 states come last.
 TcWs carve(const Problem &p, void *ws, bool bwd) {
   Carve cv(ws);
   TcWs w{};
@@ -128,16 +140,15 @@ TcWs carve(const Problem &p, void *ws, bool bwd) {
       w.gseg = cv.take<float>((size_t)p.BH * P * p.K);
     }
   } else {
-    Problem pf = p;
-    pf.variant = GLA_VARIANT_FUSED;
-    pf.segments = 0;
-    const int P = segments_of(pf, nvt);
+    const int P = bwd_segments(p, nvt);
     w.delta = cv.take<float>((size_t)p.BH * P * p.K * p.V);
     w.ddelta = cv.take<float>((size_t)p.BH * P * p.K * p.V);
     w.gseg = cv.take<float>((size_t)p.BH * P * p.K);
     w.hb = cv.take<bf16>((size_t)p.BH * p.N * p.K * p.V);
     w.dhb = cv.take<bf16>((size_t)p.BH * p.N * p.K * p.V);
     w.dscratch = cv.take<float>(tc::bwd_scratch_floats(p.BH, p.N, p.K, p.V));
+    if (p.variant == GLA_VARIANT_MATERIALIZED && (p.flags & GLA_FLAG_SAVE_STATES))
+      w.h32 = cv.take<float>((size_t)p.BH * p.N * p.K * p.V);
   }
   w.bytes = cv.bytes();
   return w;
@@ -221,7 +232,8 @@ size_t tc_workspace(const Problem &p, bool bwd) { return carve(p, nullptr, bwd).
 int tc_fwd(const Problem &p, const void *q, const void *k, const void *v, const float *la, const float *h0, void *o,
            float *hT, void *ws, cudaStream_t st) {
   if (device_ok() != 1) return GLA_ERR_NO_DEVICE;
-  TcWs w = carve(p, ws, false);
+  const bool save = (p.flags & GLA_FLAG_SAVE_STATES) != 0;
+  TcWs w = carve(p, ws, save);
   unsigned *status = (unsigned *)ws;
   TRY(launch_prep_any(p, (const bf16 *)q, (const bf16 *)k, la, w, status, st));
 
@@ -232,6 +244,8 @@ int tc_fwd(const Problem &p, const void *q, const void *k, const void *v, const 
   bool okm = map3(&m.X, w.kg, p.K, p.Tp, BH, 64, 64) && map3(&m.Y, v, p.V, p.T, BH, 64, 64) &&
              map3(&m.Q, w.qg, p.K, p.Tp, BH, 64, 64) && map3(&m.P, w.PT, 64, 64, BH * p.N, 64, 64);
   m.H = m.X;
+  // the output walk's bf16 copy of each chunk-entry state goes to the backward's h_n
+  if (save) okm = okm && map3(&m.H, w.hb, p.V, p.K, BH * p.N, 64, p.K);
   if (!okm) return GLA_ERR_CUDA;
 
   tc::WalkArgs a{};
@@ -257,7 +271,7 @@ int tc_fwd(const Problem &p, const void *q, const void *k, const void *v, const 
     tc::WalkArgs b = a;
     b.L = 1;
     b.P = p.N;
-    b.state_mode = 0;
+    b.state_mode = save ? 1 : 0;
     b.do_out = 1;
     b.start = w.h32;
     b.h0 = nullptr;
@@ -265,11 +279,12 @@ int tc_fwd(const Problem &p, const void *q, const void *k, const void *v, const 
     return launch_walk_any(p, b, m, p.N, st);
   }
 
-  const int P = segments_of(p, nvt);
+  const int P = save ? bwd_segments(p, nvt) : segments_of(p, nvt);
   const int L = (p.N + P - 1) / P;
   a.L = L;
   a.P = P;
   a.do_out = 1;
+  a.state_mode = save ? 1 : 0;
   a.end = hT;
   a.end_seg = P - 1;
   if (P == 1) {
@@ -279,6 +294,7 @@ int tc_fwd(const Problem &p, const void *q, const void *k, const void *v, const 
   // pre-pass: the contribution of segments 0 .. P-2 from a zero state
   tc::WalkArgs pre = a;
   pre.do_out = 0;
+  pre.state_mode = 0;
   pre.end = w.delta;
   pre.end_seg = -1;
   pre.gseg = w.gseg;
@@ -298,12 +314,10 @@ int tc_bwd(const Problem &p, const void *q, const void *k, const void *v, const 
   // qg, kg, P^T and gam sit at the same workspace offsets for gla_fwd and gla_bwd,
   // so a forward run on this workspace can hand them over
   if (!(p.flags & GLA_FLAG_REUSE_PREP)) TRY(launch_prep_any(p, (const bf16 *)q, (const bf16 *)k, la, w, status, st));
+  const bool saved = (p.flags & GLA_FLAG_SAVE_STATES) != 0;
   const int BV = bv_of(p);
   const int nvt = p.V / BV;
-  Problem pf = p;
-  pf.variant = GLA_VARIANT_FUSED;
-  pf.segments = 0;
-  const int P = segments_of(pf, nvt);
+  const int P = bwd_segments(p, nvt);
   const int L = (p.N + P - 1) / P;
   const uint64_t BH = (uint64_t)p.BH;
 
@@ -330,17 +344,19 @@ int tc_bwd(const Problem &p, const void *q, const void *k, const void *v, const 
   a.gam = w.gam;
   a.status = status;
   a.end_seg = -1;
-  if (P > 1) {
-    tc::WalkArgs pre = a;  // segments 0 .. P-2, forward
-    pre.end = w.delta;
-    pre.gseg = w.gseg;
-    TRY(launch_walk_any(p, pre, mf, P - 1, st));
-    a.delta = w.delta;
-    a.gseg_in = w.gseg;
+  if (!saved) {  // else the forward stored h_n in w.hb
+    if (P > 1) {
+      tc::WalkArgs pre = a;  // segments 0 .. P-2, forward
+      pre.end = w.delta;
+      pre.gseg = w.gseg;
+      TRY(launch_walk_any(p, pre, mf, P - 1, st));
+      a.delta = w.delta;
+      a.gseg_in = w.gseg;
+    }
+    a.h0 = h0;
+    a.state_mode = 1;
+    TRY(launch_walk_any(p, a, mf, P, st));
   }
-  a.h0 = h0;
-  a.state_mode = 1;
-  TRY(launch_walk_any(p, a, mf, P, st));
 
   tc::WalkArgs r{};
   r.T = p.T;

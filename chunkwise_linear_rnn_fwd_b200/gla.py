@@ -111,6 +111,7 @@ def _gate_of(log_alpha, gate):
 
 
 FLAG_REUSE_PREP = 1
+FLAG_SAVE_STATES = 2
 
 
 def make_desc(B, H, T, dk, dv, dtype, gate, *, subchunk=16, variant="auto", segments=0, flags=0,
@@ -143,8 +144,11 @@ def alloc_workspace(nbytes: int, device) -> torch.Tensor:
 
 
 def gla_fwd(q, k, v, log_alpha=None, h0=None, *, chunk=64, gate=None, subchunk=16, variant="auto", segments=0,
-            o=None, h_final=None, want_final=True, workspace=None, stream=None):
-    """Forward.  Returns (o, h_final or None).  See include/gla.h."""
+            o=None, h_final=None, want_final=True, workspace=None, stream=None, save_states=False):
+    """Forward.  Returns (o, h_final or None).  See include/gla.h.
+    save_states=True: also store the bf16 chunk states in `workspace` (sized for
+    the backward) for a following gla_bwd(..., saved_states=True)
+    (GLA_FLAG_SAVE_STATES)."""
     lib = load()
     B, H, T, dk = q.shape
     dv = v.shape[-1]
@@ -153,11 +157,13 @@ def gla_fwd(q, k, v, log_alpha=None, h0=None, *, chunk=64, gate=None, subchunk=1
         o = torch.empty(B, H, T, dv, dtype=q.dtype, device=q.device)
     if h_final is None and want_final:
         h_final = torch.empty(B, H, dk, dv, dtype=torch.float32, device=q.device)
+    flags = FLAG_SAVE_STATES if save_states else 0
     if workspace is None:
-        workspace = alloc_workspace(workspace_size(B, H, T, dk, dv, q.dtype, gate, chunk, False, subchunk=subchunk,
-                                                   variant=variant, segments=segments), q.device)
+        workspace = alloc_workspace(workspace_size(B, H, T, dk, dv, q.dtype, gate, chunk, save_states,
+                                                   subchunk=subchunk, variant=variant, segments=segments,
+                                                   flags=flags), q.device)
     d = make_desc(B, H, T, dk, dv, q.dtype, gate, subchunk=subchunk, variant=variant, segments=segments,
-                  workspace=workspace)
+                  flags=flags, workspace=workspace)
     r = lib.gla_fwd(ctypes.byref(d), _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(h0), _ptr(o), _ptr(h_final),
                     int(chunk), _stream_handle(stream))
     if r != GLA_OK:
@@ -187,10 +193,13 @@ def gla_fwd_noalloc(q, k, v, log_alpha=None, h0=None, *, chunk=64, gate=None, su
 
 
 def gla_bwd(q, k, v, log_alpha, do, h0=None, dh_final=None, *, chunk=64, gate=None, subchunk=16, dq=None, dk=None,
-            dv=None, dlog_alpha=None, dh0=None, want_dh0=True, workspace=None, stream=None, reuse_prep=False):
+            dv=None, dlog_alpha=None, dh0=None, want_dh0=True, workspace=None, stream=None, reuse_prep=False,
+            saved_states=False, segments=0, variant="auto"):
     """Backward.  Returns (dq, dk, dv, dlog_alpha or None, dh0 or None).  See include/gla.h.
     reuse_prep=True: `workspace` holds the prep outputs of a gla_fwd call on the same
-    inputs with this workspace (GLA_FLAG_REUSE_PREP)."""
+    inputs with this workspace (GLA_FLAG_REUSE_PREP).  saved_states=True: it also
+    holds the chunk states of a gla_fwd(..., save_states=True) call with the same
+    segments and variant (GLA_FLAG_SAVE_STATES)."""
     lib = load()
     B, H, T, dk_ = q.shape
     dv_ = v.shape[-1]
@@ -202,11 +211,12 @@ def gla_bwd(q, k, v, log_alpha, do, h0=None, dh_final=None, *, chunk=64, gate=No
         dlog_alpha = torch.empty_like(log_alpha)
     if dh0 is None and want_dh0:
         dh0 = torch.empty(B, H, dk_, dv_, dtype=torch.float32, device=q.device)
+    flags = (FLAG_REUSE_PREP if reuse_prep else 0) | (FLAG_SAVE_STATES if saved_states else 0)
     if workspace is None:
-        workspace = alloc_workspace(workspace_size(B, H, T, dk_, dv_, q.dtype, gate, chunk, True, subchunk=subchunk),
-                                    q.device)
-    d = make_desc(B, H, T, dk_, dv_, q.dtype, gate, subchunk=subchunk, workspace=workspace,
-                  flags=FLAG_REUSE_PREP if reuse_prep else 0)
+        workspace = alloc_workspace(workspace_size(B, H, T, dk_, dv_, q.dtype, gate, chunk, True, subchunk=subchunk,
+                                                   segments=segments, variant=variant, flags=flags), q.device)
+    d = make_desc(B, H, T, dk_, dv_, q.dtype, gate, subchunk=subchunk, variant=variant, segments=segments,
+                  workspace=workspace, flags=flags)
     r = lib.gla_bwd(ctypes.byref(d), _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(h0), _ptr(do), _ptr(dh_final),
                     _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dlog_alpha), _ptr(dh0), int(chunk), _stream_handle(stream))
     if r != GLA_OK:

@@ -79,18 +79,33 @@ extern "C" {
  *               first, then all chunk outputs are computed in parallel
  *               ("sequence-level chunk parallelism").
  * AUTO          FUSED with the segment count chosen to fill the GPU. */
-/* gla_bwd only: desc->workspace already holds the per-chunk prep outputs
- * (gate-rescaled q and k, intra-chunk scores, chunk decays) that a gla_fwd call
- * wrote into this same workspace for the same q, k, log_alpha, shape, gate and
- * chunk, and nothing has written to the workspace since.  The backward then
- * reads them instead of recomputing them (chunk states are still recomputed).
- * The workspace must be sized for the backward (gla_workspace_size(.., 1)),
- * which is at least the forward's size.  Ignored by the fp32 path. */
-#define GLA_FLAG_REUSE_PREP 1
-
 #define GLA_VARIANT_AUTO 0
 #define GLA_VARIANT_FUSED 1
 #define GLA_VARIANT_MATERIALIZED 2
+
+/* Flags (desc->flags).  Both are ignored by the fp32 path, which recomputes.
+ *
+ * GLA_FLAG_REUSE_PREP (gla_bwd): desc->workspace already holds the per-chunk
+ * prep outputs (gate-rescaled q and k, intra-chunk scores, chunk decays) that a
+ * gla_fwd call wrote into this same workspace for the same q, k, log_alpha,
+ * shape, gate, segments and chunk, and nothing has written to the workspace
+ * since.  The backward reads them instead of recomputing them.
+ *
+ * GLA_FLAG_SAVE_STATES (gla_fwd and gla_bwd): on gla_fwd, the forward also
+ * stores every chunk-entry state S[n-1] in bf16 into the workspace (the bf16
+ * copy the inter-chunk output term already uses); on gla_bwd, the backward
+ * reads those states instead of recomputing them with a second forward walk.
+ * The backward's chunk states are bf16 either way, so results are unchanged.
+ * The gla_bwd call must follow a gla_fwd call with this flag on the same
+ * inputs (and h0), descriptor and workspace, with nothing written to the
+ * workspace in between; pass GLA_FLAG_REUSE_PREP with it to reuse the prep
+ * outputs too.
+ *
+ * With either flag the workspace must be sized for the backward
+ * (gla_workspace_size(desc, chunk, 1)) on both calls, the gla_fwd call
+ * included; that size is at least the forward's. */
+#define GLA_FLAG_REUSE_PREP 1
+#define GLA_FLAG_SAVE_STATES 2
 
 typedef struct gla_desc {
   int B, H, T;          /* batch, heads, tokens (T >= 1)                                   */

@@ -38,9 +38,11 @@ def _np(t):
 
 def run_case(B, H, T, K, V, *, dtype=torch.bfloat16, gate="vector", chunk=64, seed=0, z_mean=0.0, with_h0=False,
              with_dh_final=False, bwd=True, variant="auto", segments=0, gate_scale=None, log_alpha_const=None,
-             sample_b=None, device="cuda", reuse_prep=False):
+             sample_b=None, device="cuda", reuse_prep=False, save_states=False):
     """Returns {name: max rel err}.  sample_b: list of batch indices the oracle
-    checks (all when None); the GPU always runs the full batch."""
+    checks (all when None); the GPU always runs the full batch.  reuse_prep /
+    save_states: the backward reads the forward's prep outputs / chunk states
+    from a workspace the two calls share."""
     import chunkwise_linear_rnn_fwd_b200 as pkg
     from chunkwise_linear_rnn_fwd_b200.synth import make_inputs
     from oracle import oracle
@@ -51,16 +53,19 @@ def run_case(B, H, T, K, V, *, dtype=torch.bfloat16, gate="vector", chunk=64, se
     g = {n: (None if getattr(x, n) is None else getattr(x, n).to(dev))
          for n in ("q", "k", "v", "log_alpha", "do", "h0", "dh_final")}
     ws = None
-    if reuse_prep:
-        ws = pkg.alloc_workspace(max(pkg.workspace_size(B, H, T, K, V, dtype, gate, chunk, False, variant=variant,
-                                                        segments=segments),
-                                     pkg.workspace_size(B, H, T, K, V, dtype, gate, chunk, True)), dev)
-    o, hT = pkg.gla_fwd(g["q"], g["k"], g["v"], g["log_alpha"], g["h0"], chunk=chunk, gate=gate, variant=variant,
-                        segments=segments, workspace=ws)
+    shared = dict(variant=variant, segments=segments)
+    if reuse_prep or save_states:
+        flags = (pkg.FLAG_REUSE_PREP if reuse_prep else 0) | (pkg.FLAG_SAVE_STATES if save_states else 0)
+        ws = pkg.alloc_workspace(max(pkg.workspace_size(B, H, T, K, V, dtype, gate, chunk, False, **shared),
+                                     pkg.workspace_size(B, H, T, K, V, dtype, gate, chunk, True, flags=flags,
+                                                        **shared)), dev)
+    o, hT = pkg.gla_fwd(g["q"], g["k"], g["v"], g["log_alpha"], g["h0"], chunk=chunk, gate=gate, workspace=ws,
+                        save_states=save_states, **shared)
     out = {"o": o, "h_final": hT}
     if bwd:
         dq, dk, dv, dla, dh0 = pkg.gla_bwd(g["q"], g["k"], g["v"], g["log_alpha"], g["do"], g["h0"], g["dh_final"],
-                                           chunk=chunk, gate=gate, workspace=ws, reuse_prep=reuse_prep)
+                                           chunk=chunk, gate=gate, workspace=ws, reuse_prep=reuse_prep,
+                                           saved_states=save_states, **shared)
         out.update(dq=dq, dk=dk, dv=dv, dlog_alpha=dla, dh0=dh0)
     torch.cuda.synchronize()
     out = {k: _np(v) for k, v in out.items()}

@@ -61,7 +61,21 @@ def test_check_and_workspace(lib):
     assert lib.gla_workspace_size(ctypes.byref(desc(T=0)), 64, 0) == 0
     assert lib.gla_check(None, 64) == -1
     assert lib.gla_check(ctypes.byref(desc(flags=1)), 64) == 0
-    assert lib.gla_check(ctypes.byref(desc(flags=2)), 64) == -1
+    assert lib.gla_check(ctypes.byref(desc(flags=2)), 64) == 0
+    assert lib.gla_check(ctypes.byref(desc(flags=3)), 64) == 0
+    assert lib.gla_check(ctypes.byref(desc(flags=4)), 64) == -1
+
+
+def test_saved_state_workspace_layout(lib):
+    """A forward that saves states needs the backward's workspace; the
+    MATERIALIZED forward's fp32 states are appended after everything else."""
+    fwd = lib.gla_workspace_size(ctypes.byref(desc()), 64, 0)
+    bwd = lib.gla_workspace_size(ctypes.byref(desc()), 64, 1)
+    assert 0 < fwd < bwd
+    assert lib.gla_workspace_size(ctypes.byref(desc(flags=2)), 64, 1) == bwd
+    mat = lib.gla_workspace_size(ctypes.byref(desc(flags=2, variant=2)), 64, 1)
+    assert mat > bwd
+    assert lib.gla_workspace_size(ctypes.byref(desc(variant=2)), 64, 1) == bwd
 
 
 def test_bad_calls_enqueue_nothing(lib):

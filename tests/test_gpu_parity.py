@@ -117,3 +117,20 @@ def test_backward_reusing_forward_prep(gate):
     errs = run_case(2, 2, 777, 256, 512, dtype=BF16, gate=gate, chunk=64, seed=8, with_h0=True,
                     with_dh_final=True, reuse_prep=True)
     assert_parity(errs, BF16)
+
+
+@pytest.mark.parametrize("variant,segments,reuse_prep", [("fused", 0, True), ("fused", 3, False),
+                                                         ("fused", 1, True), ("materialized", 0, True)])
+def test_backward_reading_saved_states(variant, segments, reuse_prep):
+    """gla_fwd with GLA_FLAG_SAVE_STATES stores the chunk states; gla_bwd with the
+    same flag reads them instead of recomputing them."""
+    errs = run_case(2, 2, 777, 256, 512, dtype=BF16, gate="vector", chunk=64, seed=9, with_h0=True,
+                    with_dh_final=True, variant=variant, segments=segments, reuse_prep=reuse_prep,
+                    save_states=True)
+    assert_parity(errs, BF16)
+
+
+def test_saved_states_k128():
+    errs = run_case(1, 3, 300, 128, 256, dtype=BF16, gate="scalar", chunk=64, seed=10, with_h0=True,
+                    reuse_prep=True, save_states=True)
+    assert_parity(errs, BF16)
