@@ -132,9 +132,10 @@ def dist_env():
 
 
 # ----------------------------------------------------------------------------------- oracle
-def oracle_sample_rate(w, T_sample=1024, seed=0):
+def oracle_sample_rate(w, T_sample=1024, seed=0, min_seconds=0.0):
     """Time the float64 oracle (fwd + BPTT bwd) on all heads of the workload for the
-    first T_sample tokens; returns (tokens/s, seconds, threads, description)."""
+    first T_sample tokens, repeated until at least min_seconds have passed; returns
+    (tokens/s, seconds, threads, description)."""
     import torch
 
     from chunkwise_linear_rnn_fwd_b200.synth import make_inputs
@@ -145,14 +146,17 @@ def oracle_sample_rate(w, T_sample=1024, seed=0):
     f = lambda a: None if a is None else a.double().numpy()
     q, k, v, la, do = f(x.q), f(x.k), f(x.v), f(x.log_alpha), f(x.do)
     oracle.build()
-    t0 = time.perf_counter()
-    oracle.fwd(q, k, v, la, gate=w["gate"])
-    oracle.bwd(q, k, v, la, do, gate=w["gate"])
-    dt = time.perf_counter() - t0
+    reps, dt = 0, 0.0
+    while reps == 0 or dt < min_seconds:
+        t0 = time.perf_counter()
+        oracle.fwd(q, k, v, la, gate=w["gate"])
+        oracle.bwd(q, k, v, la, do, gate=w["gate"])
+        dt += time.perf_counter() - t0
+        reps += 1
     threads = min(oracle.threads(), w["B"] * w["H"])
     desc = (f"fwd+bwd of all {w['B'] * w['H']} heads over the first {T_sample} of {w['T']} tokens "
-            f"(d_k={w['K']}, d_v={w['V']}), float64, OpenMP over heads")
-    return w["B"] * T_sample / dt, dt, threads, desc
+            f"(d_k={w['K']}, d_v={w['V']}), float64, OpenMP over heads, {reps} repetition(s)")
+    return reps * w["B"] * T_sample / dt, dt, threads, desc
 
 
 def run_reference(args, w):
@@ -350,7 +354,7 @@ def run_ours(args, w):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        r, dt, threads, desc = oracle_sample_rate(w, T_sample=args.ref_tokens)
+        r, dt, threads, desc = oracle_sample_rate(w, T_sample=w["T"], min_seconds=args.cpu_seconds)
         cpu = {"value": r, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": desc, "seconds": dt}
 
     if rank == 0:
@@ -384,6 +388,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--ref-tokens", type=int, default=1024, help="tokens per head in the oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0, help="minimum oracle time of the CPU baseline")
     ap.add_argument("--batch", type=int, default=None, help="override B (smaller profiling captures)")
     ap.add_argument("--heads", type=int, default=None, help="override H")
     ap.add_argument("--seqlen", type=int, default=None, help="override T")

@@ -44,6 +44,15 @@ def test_config4_bf16_fwd_bwd(variant):
     assert_parity(errs, BF16)
 
 
+def test_config4_bench_launch_configuration():
+    """Config 4 at full size, launched as bench.py times it: one workspace shared by
+    gla_fwd and gla_bwd, the forward saving its bf16 chunk states and the backward
+    reading them and the forward's prep outputs."""
+    errs = run_case(2, 4, 4096, 256, 512, dtype=BF16, gate="vector", chunk=64, z_mean=-1.0, bwd=True,
+                    reuse_prep=True, save_states=True)
+    assert_parity(errs, BF16)
+
+
 @pytest.mark.parametrize("T", [1024, 2048, 4096, 8192, 16384])
 @pytest.mark.parametrize("gate", ["vector", "scalar", "none"])
 def test_config5_sweep(T, gate):
