@@ -1,12 +1,13 @@
 // tc_bwd.cuh -- per-chunk backward kernel of the bf16 tensor-core path.
 //
-// One CTA per (chunk n, head).  Inputs: the recomputed chunk state h_n (state
-// before chunk n) and adjoint dh_n (gradient w.r.t. the state after chunk n),
-// both bf16 [K][V]; qg, kg, P^T and gam from the prep kernel; q, k, V, dO and
-// log_alpha.  With B the chunk-local cumulative log-gate:
+// One CTA per (chunk n, head, half of the key channels): 128 threads, one per key
+// channel c of its half.  Inputs: the chunk state h_n (state before chunk n) and
+// adjoint dh_n (gradient w.r.t. the state after chunk n), both bf16 in the
+// chunk-state layout [K/128][V/8][128][8]; gam from the prep kernel; q, k, V, dO
+// and log_alpha.  (dv comes from the reverse walk, which holds dh_n on chip.)
+// With B the chunk-local cumulative log-gate:
 //   phase 1 (loop over d_v tiles of 64, accumulating in TMEM):
 //     dqh^T = h_n dO^T          dkh^T = dh_n V^T         dP = dO V^T
-//     dv    = kg dh_n + P^T dO  (stored per tile)
 //     R[c]  = sum_v h_n[c,v] dh_n[c,v]
 //   phase 2 (intra-chunk, secondary chunking):
 //     strictly-lower sub-chunk blocks on tcgen05 with reference points
@@ -21,6 +22,10 @@
 //     dlog alpha_t = sum_{i>=t in chunk} dlog b_i + G_n,
 //     G_n = gam_n R + sum_t k_t (.) e^{B_63-B_t} dkh_t  ( = sum_v S_n dS_n, the
 //           part of the suffix sum that lies beyond the chunk).
+// A CTA needs 256 TMEM columns and ~100 KB of shared memory, so two share an SM
+// and one's load phase overlaps the other's CUDA-core phase.  dP is formed by both
+// halves of a chunk (it is tiny); with a scalar gate the two halves' channel sums
+// of dlog alpha meet in one atomic add onto a zeroed output (exact: 0 + a + b).
 #pragma once
 
 #include "tc_kernels.cuh"
@@ -28,10 +33,7 @@
 namespace gla {
 namespace tc {
 
-inline size_t bwd_scratch_floats(long BH, int N, int K, int V) {
-  (void)BH; (void)N; (void)K; (void)V;
-  return 0;
-}
+constexpr int kBwdKH = 128;  // key channels per backward CTA
 
 struct BwdArgs {
   int T, N, V, gate;
@@ -39,149 +41,140 @@ struct BwdArgs {
   const bf16 *q, *k;
   const float *la;
   const float *gam;
-  bf16 *dq, *dk, *dv;
+  const bf16 *hb, *dhb;  // chunk states / adjoints, [BH][N][K/128][V/8][128][8]
+  bf16 *dq, *dk;
   float *dla;
   unsigned *status;
 };
 
-template <int K>
 struct BwdSmem {
   static constexpr int BVb = 64;
-  static constexpr int kTileH = K * BVb * 2;
-  static constexpr int kTileV = 64 * BVb * 2;
-  static constexpr int kStage = 2 * kTileH + 2 * kTileV;   // h, dh, V, dO
-  static constexpr int kKg = 2 * kStage;                   // kg tile [64][K]
-  static constexpr int kPT = kKg + 64 * K * 2;             // P^T tile [64][64]
-  static constexpr int kPhase1End = kPT + 64 * 64 * 2;
+  static constexpr int kTileH = kBwdKH * BVb * 2;         // h or dh half-tile, [8][128][8] bf16
+  static constexpr int kTileV = 64 * BVb * 2;             // V or dO tile, SW128
+  static constexpr int kStage = 2 * kTileH + 2 * kTileV;  // h, dh, V, dO
+  static constexpr int kPhase1End = 2 * kStage;
   // phase 2 (aliases the phase-1 stages)
   static constexpr int kRowsW = 96;
-  static constexpr int kKh = 0;                            // key windows  [96][K]
-  static constexpr int kQh = kKh + kRowsW * K * 2;         // query windows [96][K]
-  static constexpr int kdP = kQh + kRowsW * K * 2;         // dP, strictly-lower blocks  [t][s]
-  static constexpr int kdPT = kdP + 64 * 64 * 2;           // the same, transposed [s][t]
-  static constexpr int kdPd = kdPT + 64 * 64 * 2;          // fp32 diagonal blocks [64][16]
-  static constexpr int kQt = kdPd + 64 * 16 * 4;          // q tile [64][K] bf16 (TMA, after phase 1)
-  static constexpr int kKt = kQt + 64 * K * 2;             // k tile [64][K] bf16
-  static constexpr int kPhase2End = kKt + 64 * K * 2;
-  static constexpr int kRed = (kPhase1End > kPhase2End ? kPhase1End : kPhase2End);  // scalar-gate reduction [8][64]
-  static constexpr int kBar = kRed + 8 * 64 * 4;
+  static constexpr int kKh = 0;                               // key windows  [96][128]
+  static constexpr int kQh = kKh + kRowsW * kBwdKH * 2;       // query windows [96][128]
+  static constexpr int kdP = kQh + kRowsW * kBwdKH * 2;       // dP, strictly-lower blocks  [t][s]
+  static constexpr int kdPT = kdP + 64 * 64 * 2;              // the same, transposed [s][t]
+  static constexpr int kdPd = kdPT + 64 * 64 * 2;             // fp32 diagonal blocks [64][16]
+  static constexpr int kQt = kdPd + 64 * 16 * 4;              // q tile [64][128] bf16 (TMA, after phase 1)
+  static constexpr int kKt = kQt + 64 * kBwdKH * 2;           // k tile [64][128] bf16
+  static constexpr int kPhase2End = kKt + 64 * kBwdKH * 2;
+  static constexpr int kRed = (kPhase1End > kPhase2End ? kPhase1End : kPhase2End);  // scalar-gate sums [4][64]
+  static constexpr int kBar = kRed + 4 * 64 * 4;
   static constexpr int kBytes = kBar + 128;
 };
 
+__device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   dev::smem_u32(dst)),
+               "l"(src), "r"(bytes), "r"(dev::smem_u32(bar))
+               : "memory");
+}
+
 template <int K>
-__global__ void __launch_bounds__(256, 1)
-    k_bwd_main(BwdArgs a, const __grid_constant__ CUtensorMap tmH, const __grid_constant__ CUtensorMap tmDH,
-               const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
-               const __grid_constant__ CUtensorMap tmKg, const __grid_constant__ CUtensorMap tmPT,
+__global__ void __launch_bounds__(kBwdKH, 2)
+    k_bwd_main(BwdArgs a, const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
                const __grid_constant__ CUtensorMap tmQin, const __grid_constant__ CUtensorMap tmKin) {
-  using L = BwdSmem<K>;
+  using L = BwdSmem;
   constexpr int BVb = L::BVb;
-  constexpr int kMB = K / 128;
-  constexpr int cDQ = 0, cDK = 64 * kMB, cDP = 128 * kMB, cDV = cDP + 64;
-  constexpr int cQI = cDP, cKI = cQI + 64 * kMB;
-  constexpr int kTmemCols = (K == 256) ? 512 : 256;
+  constexpr int kH = K / kBwdKH;  // CTAs per chunk
+  constexpr int cDQ = 0, cDK = 64, cDP = 128;
+  constexpr int cQI = cDP, cKI = 192;
+  constexpr int kTmemCols = 256;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  uint64_t *full = (uint64_t *)(smem + L::kBar);  // [0],[1] stages, [2] kg+PT, [4] q/k tiles
-  uint64_t *mma_bar = full + 3;
-  uint64_t *qk_bar = full + 4;
-  uint32_t *tslot = (uint32_t *)(full + 5);
+  uint64_t *full = (uint64_t *)(smem + L::kBar);  // [0],[1] stages
+  uint64_t *mma_bar = full + 2;
+  uint64_t *qk_bar = full + 3;
+  uint32_t *tslot = (uint32_t *)(full + 4);
   float *red = (float *)(smem + L::kRed);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int n = blockIdx.x;
   const long bh = blockIdx.y;
+  const int half = blockIdx.z;
+  const int c0 = half * kBwdKH;
   const int nvt = a.V / BVb;
   const long hrow = bh * a.N + n;
 
   if (warp == 0) dev::tmem_alloc(tslot, kTmemCols);
   if (tid == 0) {
-    for (int i = 0; i < 3; ++i) dev::mbar_init(&full[i], 1);
+    dev::mbar_init(&full[0], 1);
+    dev::mbar_init(&full[1], 1);
     dev::mbar_init(mma_bar, 1);
     dev::mbar_init(qk_bar, 1);
     dev::fence_mbar_init();
+    dev::prefetch_tmap(&tmV);
+    dev::prefetch_tmap(&tmDO);
   }
   dev::tc_fence_before();
   __syncthreads();
   dev::tc_fence_after();
   const uint32_t tmem = *tslot;
 
+  // this CTA's 128 rows of h_n / dh_n for d_v tile i: 16 contiguous KB
+  const long half_tile = (long)kBwdKH * BVb;  // bf16 elements
+  const bf16 *h_src = a.hb + (hrow * kH + half) * (long)a.V * kBwdKH;
+  const bf16 *dh_src = a.dhb + (hrow * kH + half) * (long)a.V * kBwdKH;
   auto stage = [&](int s) { return smem + s * L::kStage; };
   auto issue_tile = [&](int i) {
     const int s = i & 1;
     uint8_t *st = stage(s);
     const int v0 = i * BVb;
     dev::mbar_arrive_expect_tx(&full[s], (uint32_t)L::kStage);
-    dev::tma_load_3d(st, &tmH, v0, 0, (int)hrow, &full[s]);
-    dev::tma_load_3d(st + L::kTileH, &tmDH, v0, 0, (int)hrow, &full[s]);
+    bulk_load(st, h_src + i * half_tile, (uint32_t)L::kTileH, &full[s]);
+    bulk_load(st + L::kTileH, dh_src + i * half_tile, (uint32_t)L::kTileH, &full[s]);
     dev::tma_load_3d(st + 2 * L::kTileH, &tmV, v0, n * kC, (int)bh, &full[s]);
     dev::tma_load_3d(st + 2 * L::kTileH + L::kTileV, &tmDO, v0, n * kC, (int)bh, &full[s]);
   };
   if (tid == 0) {
-    dev::mbar_arrive_expect_tx(&full[2], (uint32_t)(64 * K * 2 + 64 * 64 * 2));
-#pragma unroll
-    for (int cb = 0; cb < K / 64; ++cb)
-      dev::tma_load_3d(smem + L::kKg + cb * 64 * 128, &tmKg, cb * 64, n * kC, (int)bh, &full[2]);
-    dev::tma_load_3d(smem + L::kPT, &tmPT, 0, 0, (int)hrow, &full[2]);
     issue_tile(0);
     if (nvt > 1) issue_tile(1);
   }
 
-  const int c = tid;  // key channel (valid when tid < K)
-  float R = 0.f;      // sum_v h[c,v] dh[c,v]
-  bool ok = dev::mbar_wait(&full[2], 0, a.status);
+  const int cl = tid;     // key channel within this CTA's half
+  const int c = c0 + cl;  // key channel
+  float R = 0.f;          // sum_v h[c,v] dh[c,v]
+  bool ok = true;
 
   // ============================ phase 1 ============================
   for (int i = 0; i < nvt; ++i) {
     const int s = i & 1;
     uint8_t *st = stage(s);
     if (ok) ok = dev::mbar_wait(&full[s], (i >> 1) & 1, a.status);
-    // the previous tile's dv epilogue has released the dv accumulator (barrier at
-    // the end of the last iteration); issue this tile's MMAs, then sum h (.) dh
-    // from the same shared-memory tiles while they run
+    // issue this tile's MMAs, then sum h (.) dh from the same shared-memory tiles
+    // while they run
     if (tid == 0 && ok) {
       const uint32_t sH = dev::smem_u32(st), sDH = sH + L::kTileH, sV = sDH + L::kTileH, sDO = sV + L::kTileV;
-      const uint32_t sKg = dev::smem_u32(smem + L::kKg), sPT = dev::smem_u32(smem + L::kPT);
       constexpr uint32_t id_kk128 = dev::idesc_bf16(128, 64, false, false);
       constexpr uint32_t id_kk64 = dev::idesc_bf16(64, 64, false, false);
 #pragma unroll
       for (int kk = 0; kk < BVb / 16; ++kk) {
         const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
-#pragma unroll
-        for (int m = 0; m < kMB; ++m) {
-          dev::umma_bf16(tmem + cDQ + 64 * m, dev::desc_kmajor(sH, K, 128 * m, kk * 16),
-                         dev::desc_kmajor(sDO, 64, 0, kk * 16), id_kk128, acc);
-          dev::umma_bf16(tmem + cDK + 64 * m, dev::desc_kmajor(sDH, K, 128 * m, kk * 16),
-                         dev::desc_kmajor(sV, 64, 0, kk * 16), id_kk128, acc);
-        }
+        dev::umma_bf16(tmem + cDQ, dev::desc_state_kmajor(sH, kBwdKH, 0, kk * 16),
+                       dev::desc_kmajor(sDO, 64, 0, kk * 16), id_kk128, acc);
+        dev::umma_bf16(tmem + cDK, dev::desc_state_kmajor(sDH, kBwdKH, 0, kk * 16),
+                       dev::desc_kmajor(sV, 64, 0, kk * 16), id_kk128, acc);
         dev::umma_bf16(tmem + cDP, dev::desc_kmajor(sDO, 64, 0, kk * 16), dev::desc_kmajor(sV, 64, 0, kk * 16),
                        id_kk64, acc);
       }
-      // dv tile = kg dh + P^T dO
-      constexpr uint32_t id_dv1 = dev::idesc_bf16(64, BVb, false, true);
-#pragma unroll
-      for (int kk = 0; kk < K / 16; ++kk)
-        dev::umma_bf16(tmem + cDV, dev::desc_kmajor(sKg, 64, 0, kk * 16), dev::desc_mnmajor(sDH, K, kk * 16, 0),
-                       id_dv1, kk > 0 ? 1u : 0u);
-      // A[m = t][k = s] = P[s][t] = P^T tile [t][s]: K-major
-      constexpr uint32_t id_dv2 = dev::idesc_bf16(64, BVb, false, true);
-#pragma unroll
-      for (int kk = 0; kk < kC / 16; ++kk)
-        dev::umma_bf16(tmem + cDV, dev::desc_kmajor(sPT, 64, 0, kk * 16), dev::desc_mnmajor(sDO, 64, kk * 16, 0),
-                       id_dv2, 1u);
       dev::umma_commit(mma_bar);
     }
-    if (tid < K) {
+    {
       const uint32_t sh = dev::smem_u32(st), sdh = sh + L::kTileH;
 #pragma unroll
       for (int c8 = 0; c8 < BVb / 8; ++c8) {
         uint4 x, y;
         asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];"
                      : "=r"(x.x), "=r"(x.y), "=r"(x.z), "=r"(x.w)
-                     : "r"(sh + dev::sw128_chunk(K, c, c8)));
+                     : "r"(sh + (uint32_t)(c8 * kBwdKH + cl) * 16u));
         asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];"
                      : "=r"(y.x), "=r"(y.y), "=r"(y.z), "=r"(y.w)
-                     : "r"(sdh + dev::sw128_chunk(K, c, c8)));
+                     : "r"(sdh + (uint32_t)(c8 * kBwdKH + cl) * 16u));
         const __nv_bfloat162 *xh = reinterpret_cast<const __nv_bfloat162 *>(&x);
         const __nv_bfloat162 *yh = reinterpret_cast<const __nv_bfloat162 *>(&y);
 #pragma unroll
@@ -195,54 +188,24 @@ __global__ void __launch_bounds__(256, 1)
     dev::tc_fence_after();
     __syncthreads();  // every thread has finished reading stage s (R sums)
     if (tid == 0 && ok && i + 2 < nvt) issue_tile(i + 2);
-    // dv epilogue: rows t (M = 64 layout), warps 0-3 columns [0,32), warps 4-7 [32,64)
-    {
-      const int sub = warp & 3;
-      const int col0 = (warp >= 4) ? BVb / 2 : 0;
-      const int t = 16 * sub + lane;
-      const long tgl = (long)n * kC + t;
-#pragma unroll
-      for (int cb = 0; cb < BVb / 32; ++cb) {
-        float v[16];
-        dev::tmem_ld16(dev::tmem_addr(tmem, 32 * sub, cDV + col0 + cb * 16), v);
-        dev::tmem_wait_ld();
-        if (lane < 16 && tgl < a.T && ok) {
-          uint4 p0, p1;
-          p0.x = dev::pack_bf16(v[0], v[1]);
-          p0.y = dev::pack_bf16(v[2], v[3]);
-          p0.z = dev::pack_bf16(v[4], v[5]);
-          p0.w = dev::pack_bf16(v[6], v[7]);
-          p1.x = dev::pack_bf16(v[8], v[9]);
-          p1.y = dev::pack_bf16(v[10], v[11]);
-          p1.z = dev::pack_bf16(v[12], v[13]);
-          p1.w = dev::pack_bf16(v[14], v[15]);
-          uint4 *dst = reinterpret_cast<uint4 *>(a.dv + (bh * a.T + tgl) * (long)a.V + i * BVb + col0 + cb * 16);
-          dst[0] = p0;
-          dst[1] = p1;
-        }
-      }
-    }
-    dev::tc_fence_before();
-    __syncthreads();
-    dev::tc_fence_after();
   }
 
   // ============================ phase 2 ============================
-  // q and k tiles of this chunk into the space phase 1 no longer uses
+  // q and k columns of this half into the space phase 1 no longer uses
   if (tid == 0) {
     dev::fence_proxy_async_smem();
-    dev::mbar_arrive_expect_tx(qk_bar, (uint32_t)(2 * 64 * K * 2));
+    dev::mbar_arrive_expect_tx(qk_bar, (uint32_t)(2 * 64 * kBwdKH * 2));
 #pragma unroll
-    for (int cb = 0; cb < K / 64; ++cb) {
-      dev::tma_load_3d(smem + L::kQt + cb * 64 * 128, &tmQin, cb * 64, n * kC, (int)bh, qk_bar);
-      dev::tma_load_3d(smem + L::kKt + cb * 64 * 128, &tmKin, cb * 64, n * kC, (int)bh, qk_bar);
+    for (int cb = 0; cb < kBwdKH / 64; ++cb) {
+      dev::tma_load_3d(smem + L::kQt + cb * 64 * 128, &tmQin, c0 + cb * 64, n * kC, (int)bh, qk_bar);
+      dev::tma_load_3d(smem + L::kKt + cb * 64 * 128, &tmKin, c0 + cb * 64, n * kC, (int)bh, qk_bar);
     }
   }
   // dP (rows t, TMEM M = 64 layout) -> bf16 tiles of its strictly-lower sub-chunk
   // blocks, dP[t][s] and dP^T[s][t], and fp32 copies of the four diagonal blocks.
   const uint32_t sdP = dev::smem_u32(smem + L::kdP), sdPT = dev::smem_u32(smem + L::kdPT);
   float *dPd = (float *)(smem + L::kdPd);
-  if (warp < 4) {
+  {
     const int t = 16 * warp + lane;
     float row[kC];
 #pragma unroll
@@ -271,18 +234,18 @@ __global__ void __launch_bounds__(256, 1)
   }
 
   // per key channel: sub-chunk boundary values of the cumulative log-gate; the 16
-  // values inside sub-chunk j are rebuilt from log_alpha when needed (gate16)
+  // values inside sub-chunk j are rebuilt from log_alpha when needed
   float z[5], Gam[4], E[4], Gafter[4];
   const long qrow0 = bh * a.T + (long)n * kC;  // first token row of this chunk
   const uint32_t sQt = dev::smem_u32(smem + L::kQt), sKt = dev::smem_u32(smem + L::kKt);
   auto qk_at = [&](int t, float &qf, float &kf) {
     uint16_t qb, kb;
-    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(qb) : "r"(sQt + dev::sw128_off(64, t, c)));
-    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(kb) : "r"(sKt + dev::sw128_off(64, t, c)));
+    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(qb) : "r"(sQt + dev::sw128_off(64, t, cl)));
+    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(kb) : "r"(sKt + dev::sw128_off(64, t, cl)));
     qf = __bfloat162float(*reinterpret_cast<const bf16 *>(&qb));
     kf = __bfloat162float(*reinterpret_cast<const bf16 *>(&kb));
   };
-  // log_alpha of token 16 j + e of this chunk (0 beyond T)
+  // log_alpha of token t of this chunk (0 beyond T)
   auto gate_at = [&](int t) -> float {
     if ((long)n * kC + t >= a.T) return 0.f;
     if (a.gate == GLA_GATE_VECTOR) return __ldg(a.la + (qrow0 + t) * K + c);
@@ -302,11 +265,8 @@ __global__ void __launch_bounds__(256, 1)
       Bc[e] = acc;
     }
   };
-  // 128-row block of this warp's key channels; warps without channels (d_k = 128,
-  // warps 4-7) mirror block 0 so their warp-collective TMEM loads stay in bounds
-  const int mb = ((warp >> 2) < kMB) ? (warp >> 2) : 0;
-  const uint32_t lanebase = 32 * (warp & 3);
-  if (tid < K) {
+  const uint32_t lanebase = 32 * warp;
+  {
     float g[kC];
 #pragma unroll
     for (int t = 0; t < kC; ++t) g[t] = gate_at(t);
@@ -330,9 +290,8 @@ __global__ void __launch_bounds__(256, 1)
   if (!dev::mbar_wait(qk_bar, 0, a.status)) ok = false;
 
   // window construction + boundary term G_n = gam_n R + sum_t k_t dk_inter_t
-  float Gb = 0.f;
-  if (tid < K) {
-    Gb = a.gam[(bh * a.N + n) * K + c] * R;
+  float Gb = a.gam[(bh * a.N + n) * K + c] * R;
+  {
     const uint32_t sKh = dev::smem_u32(smem + L::kKh), sQh = dev::smem_u32(smem + L::kQh);
     const int wK[4] = {0, 0, 16, 48};    // key window j >= 1: row wK[j] + s, s in [0, 16j)
     const int wQ[4] = {-16, 16, 32, 0};  // query window u <= 2: row wQ[u] + t, t in [16(u+1), 64)
@@ -344,7 +303,7 @@ __global__ void __launch_bounds__(256, 1)
       const float zj = dev::sel4(j, z[0], z[1], z[2], z[3]);
       cumsum16(gnext, zj, Bc);
       if (j < 3) load16(j + 1, gnext);  // prefetch the next sub-chunk's gates
-      dev::tmem_ld16(dev::tmem_addr(tmem, lanebase, cDK + 64 * mb + 16 * j), xk);
+      dev::tmem_ld16(dev::tmem_addr(tmem, lanebase, cDK + 16 * j), xk);
       dev::tmem_wait_ld();
       const float zj1 = dev::sel4(j, z[1], z[2], z[3], z[4]);
       const float GAj = dev::sel4(j, Gafter[0], Gafter[1], Gafter[2], Gafter[3]);
@@ -362,7 +321,8 @@ __global__ void __launch_bounds__(256, 1)
         for (int jq = 1; jq < 4; ++jq) {
           if (jq > j) {
             const bf16 b = __float2bfloat16_rn(f);
-            dev::st_shared_u16(sKh + dev::sw128_off(L::kRowsW, wK[jq] + t, c), *reinterpret_cast<const uint16_t *>(&b));
+            dev::st_shared_u16(sKh + dev::sw128_off(L::kRowsW, wK[jq] + t, cl),
+                               *reinterpret_cast<const uint16_t *>(&b));
             f *= Gam[jq];
           }
         }
@@ -372,19 +332,12 @@ __global__ void __launch_bounds__(256, 1)
         for (int uu = 2; uu >= 0; --uu) {
           if (uu < j) {
             const bf16 b = __float2bfloat16_rn(g2);
-            dev::st_shared_u16(sQh + dev::sw128_off(L::kRowsW, wQ[uu] + t, c), *reinterpret_cast<const uint16_t *>(&b));
+            dev::st_shared_u16(sQh + dev::sw128_off(L::kRowsW, wQ[uu] + t, cl),
+                               *reinterpret_cast<const uint16_t *>(&b));
             g2 *= Gam[uu];
           }
         }
       }
-    }
-  } else {
-    // warps without key channels still take part in the warp-collective TMEM loads
-#pragma unroll 1
-    for (int j = 0; j < 4; ++j) {
-      float xk[16];
-      dev::tmem_ld16(dev::tmem_addr(tmem, lanebase, cDK + 64 * mb + 16 * j), xk);
-      dev::tmem_wait_ld();
     }
   }
   dev::fence_proxy_async_smem();
@@ -397,20 +350,17 @@ __global__ void __launch_bounds__(256, 1)
     const int wQ[4] = {-16, 16, 32, 0};
     constexpr uint32_t id = dev::idesc_bf16(128, 16, true, false);
 #pragma unroll
-    for (int m = 0; m < kMB; ++m) {
+    for (int j = 1; j < 4; ++j)
 #pragma unroll
-      for (int j = 1; j < 4; ++j)
+      for (int kk = 0; kk < j; ++kk)
+        dev::umma_bf16(tmem + cQI + 16 * j, dev::desc_mnmajor(sKh, L::kRowsW, wK[j] + 16 * kk, 0),
+                       dev::desc_kmajor(sdP, 64, 16 * j, 16 * kk), id, kk > 0 ? 1u : 0u);
 #pragma unroll
-        for (int kk = 0; kk < j; ++kk)
-          dev::umma_bf16(tmem + cQI + 64 * m + 16 * j, dev::desc_mnmajor(sKh, L::kRowsW, wK[j] + 16 * kk, 128 * m),
-                         dev::desc_kmajor(sdP, 64, 16 * j, 16 * kk), id, kk > 0 ? 1u : 0u);
+    for (int u = 0; u < 3; ++u)
 #pragma unroll
-      for (int u = 0; u < 3; ++u)
-#pragma unroll
-        for (int kk = u + 1; kk < 4; ++kk)
-          dev::umma_bf16(tmem + cKI + 64 * m + 16 * u, dev::desc_mnmajor(sQh, L::kRowsW, wQ[u] + 16 * kk, 128 * m),
-                         dev::desc_kmajor(sdPT, 64, 16 * u, 16 * kk), id, kk > u + 1 ? 1u : 0u);
-    }
+      for (int kk = u + 1; kk < 4; ++kk)
+        dev::umma_bf16(tmem + cKI + 16 * u, dev::desc_mnmajor(sQh, L::kRowsW, wQ[u] + 16 * kk, 0),
+                       dev::desc_kmajor(sdPT, 64, 16 * u, 16 * kk), id, kk > u + 1 ? 1u : 0u);
     dev::umma_commit(mma_bar);
   }
   if (ok) ok = dev::mbar_wait(mma_bar, nvt & 1, a.status);
@@ -420,87 +370,80 @@ __global__ void __launch_bounds__(256, 1)
   // reverse over sub-chunks and tokens: dq, dk, dlog b and its suffix sum
   float run = Gb;
   float gnext[16];
-  if (tid < K) load16(3, gnext);
+  load16(3, gnext);
 #pragma unroll 1
-  for (int t16 = 3; t16 >= 0; --t16) {
-    const int j = t16;
+  for (int j = 3; j >= 0; --j) {
     float xq[16], xk[16], xqi[16], xki[16];
-    dev::tmem_ld16(dev::tmem_addr(tmem, lanebase, cDQ + 64 * mb + 16 * t16), xq);
-    dev::tmem_ld16(dev::tmem_addr(tmem, lanebase, cDK + 64 * mb + 16 * t16), xk);
-    dev::tmem_ld16(dev::tmem_addr(tmem, lanebase, cQI + 64 * mb + 16 * t16), xqi);
-    dev::tmem_ld16(dev::tmem_addr(tmem, lanebase, cKI + 64 * mb + 16 * t16), xki);
+    dev::tmem_ld16(dev::tmem_addr(tmem, lanebase, cDQ + 16 * j), xq);
+    dev::tmem_ld16(dev::tmem_addr(tmem, lanebase, cDK + 16 * j), xk);
+    dev::tmem_ld16(dev::tmem_addr(tmem, lanebase, cQI + 16 * j), xqi);
+    dev::tmem_ld16(dev::tmem_addr(tmem, lanebase, cKI + 16 * j), xki);
     dev::tmem_wait_ld();
-    if (tid < K) {
-      float Bc[16];
-      const float zj = dev::sel4(j, z[0], z[1], z[2], z[3]);
-      cumsum16(gnext, zj, Bc);
-      if (j > 0) load16(j - 1, gnext);  // prefetch the previous sub-chunk's gates
-      const float zj1 = dev::sel4(j, z[1], z[2], z[3], z[4]);
-      const float Ej = dev::sel4(j, E[0], E[1], E[2], E[3]);
-      const float invGj = 1.f / dev::sel4(j, Gam[0], Gam[1], Gam[2], Gam[3]);
-      const float GAj = dev::sel4(j, Gafter[0], Gafter[1], Gafter[2], Gafter[3]);
-      const float offq_on = (j > 0) ? 1.f : 0.f;  // no off-diagonal MMA wrote sub-chunk 0's dq columns
-      const float offk_on = (j < 3) ? 1.f : 0.f;  // ... nor sub-chunk 3's dk columns
-      // diagonal block of sub-chunk j in fp32:
-      //   a_t = q_t e^{B_t - z_j},  b_s = k_s e^{z_j - B_s}
-      //   dq_t += e^{B_t - z_j} sum_{s<=t} dP[t,s] b_s ,  dk_s += e^{z_j - B_s} sum_{t>=s} dP[t,s] a_t
-      float uu[16], ww[16], qv[16], kv[16], av[16], bv[16], dqd[16], dkd[16];
+    float Bc[16];
+    const float zj = dev::sel4(j, z[0], z[1], z[2], z[3]);
+    cumsum16(gnext, zj, Bc);
+    if (j > 0) load16(j - 1, gnext);  // prefetch the previous sub-chunk's gates
+    const float zj1 = dev::sel4(j, z[1], z[2], z[3], z[4]);
+    const float Ej = dev::sel4(j, E[0], E[1], E[2], E[3]);
+    const float invGj = 1.f / dev::sel4(j, Gam[0], Gam[1], Gam[2], Gam[3]);
+    const float GAj = dev::sel4(j, Gafter[0], Gafter[1], Gafter[2], Gafter[3]);
+    const float offq_on = (j > 0) ? 1.f : 0.f;  // no off-diagonal MMA wrote sub-chunk 0's dq columns
+    const float offk_on = (j < 3) ? 1.f : 0.f;  // ... nor sub-chunk 3's dk columns
+    // diagonal block of sub-chunk j in fp32:
+    //   a_t = q_t e^{B_t - z_j},  b_s = k_s e^{z_j - B_s}
+    //   dq_t += e^{B_t - z_j} sum_{s<=t} dP[t,s] b_s ,  dk_s += e^{z_j - B_s} sum_{t>=s} dP[t,s] a_t
+    float uu[16], ww[16], qv[16], kv[16], av[16], bv[16], dqd[16], dkd[16];
 #pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        qk_at(16 * j + e, qv[e], kv[e]);
-        uu[e] = __expf(Bc[e] - zj);
-        ww[e] = __expf(zj1 - Bc[e]);
-        av[e] = qv[e] * uu[e];
-        bv[e] = kv[e] * ww[e] * invGj;
-        dqd[e] = 0.f;
-        dkd[e] = 0.f;
+    for (int e = 0; e < 16; ++e) {
+      qk_at(16 * j + e, qv[e], kv[e]);
+      uu[e] = __expf(Bc[e] - zj);
+      ww[e] = __expf(zj1 - Bc[e]);
+      av[e] = qv[e] * uu[e];
+      bv[e] = kv[e] * ww[e] * invGj;
+      dqd[e] = 0.f;
+      dkd[e] = 0.f;
+    }
+    // dP rows hold zeros beyond the diagonal, so pairs (f, f+1) may run one past e
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      const float4 *rowp = reinterpret_cast<const float4 *>(dPd + (16 * j + e) * 16);
+      float pr[16];
+#pragma unroll
+      for (int x4 = 0; x4 < 4; ++x4) {
+        const float4 v4 = rowp[x4];
+        pr[4 * x4] = v4.x;
+        pr[4 * x4 + 1] = v4.y;
+        pr[4 * x4 + 2] = v4.z;
+        pr[4 * x4 + 3] = v4.w;
       }
-      // dP rows hold zeros beyond the diagonal, so pairs (f, f+1) may run one past e
+      float q0 = 0.f, q1 = 0.f;
 #pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        const float4 *rowp = reinterpret_cast<const float4 *>(dPd + (16 * j + e) * 16);
-        float pr[16];
-#pragma unroll
-        for (int x4 = 0; x4 < 4; ++x4) {
-          const float4 v4 = rowp[x4];
-          pr[4 * x4] = v4.x;
-          pr[4 * x4 + 1] = v4.y;
-          pr[4 * x4 + 2] = v4.z;
-          pr[4 * x4 + 3] = v4.w;
-        }
-        float q0 = 0.f, q1 = 0.f;
-#pragma unroll
-        for (int f = 0; f <= e; f += 2) {
-          dev::ffma2(q0, q1, pr[f], pr[f + 1], bv[f], bv[f + 1]);
-          dev::ffma2(dkd[f], dkd[f + 1], pr[f], pr[f + 1], av[e], av[e]);
-        }
-        dqd[e] = q0 + q1;
+      for (int f = 0; f <= e; f += 2) {
+        dev::ffma2(q0, q1, pr[f], pr[f + 1], bv[f], bv[f + 1]);
+        dev::ffma2(dkd[f], dkd[f + 1], pr[f], pr[f + 1], av[e], av[e]);
       }
+      dqd[e] = q0 + q1;
+    }
 #pragma unroll
-      for (int e = 15; e >= 0; --e) {
-        const int t = 16 * j + e;
-        const long tg = (long)n * kC + t;
-        const float dqd_e = dqd[e] * uu[e];
-        const float dkd_e = dkd[e] * ww[e] * invGj;
-        const float dqr = uu[e] * (Ej * xq[e] + offq_on * xqi[e]);
-        const float dkr = ww[e] * (GAj * xk[e] + offk_on * xki[e]);
-        run += (qv[e] * dqr - kv[e] * dkr) + (qv[e] * dqd_e - kv[e] * dkd_e);
-        if (tg < a.T && ok) {
-          a.dq[(qrow0 + t) * K + c] = __float2bfloat16_rn(dqr + dqd_e);
-          a.dk[(qrow0 + t) * K + c] = __float2bfloat16_rn(dkr + dkd_e);
-          if (a.gate == GLA_GATE_VECTOR) a.dla[(qrow0 + t) * K + c] = run;
-        }
-        if (a.gate == GLA_GATE_SCALAR) {
-          float x = run;
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
-          if (lane == 0) red[warp * 64 + t] = x;
-        }
+    for (int e = 15; e >= 0; --e) {
+      const int t = 16 * j + e;
+      const long tg = (long)n * kC + t;
+      const float dqd_e = dqd[e] * uu[e];
+      const float dkd_e = dkd[e] * ww[e] * invGj;
+      const float dqr = uu[e] * (Ej * xq[e] + offq_on * xqi[e]);
+      const float dkr = ww[e] * (GAj * xk[e] + offk_on * xki[e]);
+      run += (qv[e] * dqr - kv[e] * dkr) + (qv[e] * dqd_e - kv[e] * dkd_e);
+      if (tg < a.T && ok) {
+        a.dq[(qrow0 + t) * K + c] = __float2bfloat16_rn(dqr + dqd_e);
+        a.dk[(qrow0 + t) * K + c] = __float2bfloat16_rn(dkr + dkd_e);
+        if (a.gate == GLA_GATE_VECTOR) a.dla[(qrow0 + t) * K + c] = run;
       }
-    } else if (a.gate == GLA_GATE_SCALAR) {
+      if (a.gate == GLA_GATE_SCALAR) {
+        float x = run;
 #pragma unroll
-      for (int e = 15; e >= 0; --e)
-        if (lane == 0) red[warp * 64 + 16 * j + e] = 0.f;
+        for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+        if (lane == 0) red[warp * 64 + t] = x;
+      }
     }
   }
   if (a.gate == GLA_GATE_SCALAR) {
@@ -508,9 +451,12 @@ __global__ void __launch_bounds__(256, 1)
     if (tid < kC) {
       float ssum = 0.f;
 #pragma unroll
-      for (int w8 = 0; w8 < 8; ++w8) ssum += red[w8 * 64 + tid];
+      for (int w4 = 0; w4 < kBwdKH / 32; ++w4) ssum += red[w4 * 64 + tid];
       const long tg = (long)n * kC + tid;
-      if (tg < a.T && ok) a.dla[bh * a.T + tg] = ssum;
+      if (tg < a.T && ok) {
+        if (kH == 1) a.dla[bh * a.T + tg] = ssum;
+        else atomicAdd(a.dla + bh * a.T + tg, ssum);  // onto zero, two addends: exact and order-free
+      }
     }
   }
   dev::tc_fence_before();
@@ -522,37 +468,34 @@ template <int K>
 int launch_bwd_main_k(const Problem &p, const BwdArgs &a, const CUtensorMap *maps, cudaStream_t st) {
   static int smem = 0;
   if (!smem) {
-    const int want = BwdSmem<K>::kBytes + 1024;
+    const int want = BwdSmem::kBytes + 1024;
     if (cudaFuncSetAttribute(k_bwd_main<K>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem) != cudaSuccess)
       return GLA_ERR_CUDA;
-    const int got = smem_for_tmem(k_bwd_main<K>, 256, want, (K == 256) ? 512 : 256);
+    const int got = smem_for_tmem(k_bwd_main<K>, kBwdKH, want, 256);
     if (got < 0) return GLA_ERR_CUDA;
     smem = got;
   }
   GLA_LAUNCH(K_TC_BWD, st,
-             (k_bwd_main<K><<<dim3(p.N, p.BH), 256, smem, st>>>(a, maps[0], maps[1], maps[2], maps[3], maps[4],
-                                                                 maps[5], maps[6], maps[7])));
+             (k_bwd_main<K><<<dim3(p.N, p.BH, K / kBwdKH), kBwdKH, smem, st>>>(a, maps[0], maps[1], maps[2],
+                                                                                maps[3])));
   return GLA_OK;
 }
 
 bool map3_bf16(CUtensorMap *m, const void *base, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t b0, uint32_t b1);
 
 inline int launch_bwd_main(const Problem &p, const bf16 *q, const bf16 *k, const bf16 *v, const float *la,
-                           const bf16 *dout, bf16 *dq, bf16 *dk, bf16 *dv, float *dla, const bf16 *qg,
-                           const bf16 *kg, const bf16 *PT, const float *gam, const bf16 *hb, const bf16 *dhb,
-                           float *scratch, unsigned *status, cudaStream_t st) {
-  (void)qg;
-  (void)scratch;
-  if (p.V % 64 != 0) return GLA_ERR_UNSUPPORTED_SHAPE;
-  CUtensorMap maps[8];
+                           const bf16 *dout, bf16 *dq, bf16 *dk, float *dla, const float *gam, const bf16 *hb,
+                           const bf16 *dhb, unsigned *status, cudaStream_t st) {
+  if (p.V % 64 != 0 || p.K % kBwdKH != 0) return GLA_ERR_UNSUPPORTED_SHAPE;
+  CUtensorMap maps[4];
   const uint64_t BH = (uint64_t)p.BH;
-  const bool ok = map3_bf16(&maps[0], hb, p.V, p.K, BH * p.N, 64, p.K) &&
-                  map3_bf16(&maps[1], dhb, p.V, p.K, BH * p.N, 64, p.K) &&
-                  map3_bf16(&maps[2], v, p.V, p.T, BH, 64, 64) && map3_bf16(&maps[3], dout, p.V, p.T, BH, 64, 64) &&
-                  map3_bf16(&maps[4], kg, p.K, p.Tp, BH, 64, 64) && map3_bf16(&maps[5], PT, 64, 64, BH * p.N, 64, 64) &&
-                  map3_bf16(&maps[6], q, p.K, p.T, BH, 64, 64) && map3_bf16(&maps[7], k, p.K, p.T, BH, 64, 64);
+  const bool ok = map3_bf16(&maps[0], v, p.V, p.T, BH, 64, 64) && map3_bf16(&maps[1], dout, p.V, p.T, BH, 64, 64) &&
+                  map3_bf16(&maps[2], q, p.K, p.T, BH, 64, 64) && map3_bf16(&maps[3], k, p.K, p.T, BH, 64, 64);
   if (!ok) return GLA_ERR_CUDA;
-  BwdArgs a{p.T, p.N, p.V, p.gate, p.Tp, q, k, la, gam, dq, dk, dv, dla, status};
+  // with a scalar gate and two channel halves, dlog alpha is summed by atomic adds
+  if (p.gate == GLA_GATE_SCALAR && p.K > kBwdKH)
+    if (cudaMemsetAsync(dla, 0, (size_t)p.BH * p.T * sizeof(float), st) != cudaSuccess) return GLA_ERR_CUDA;
+  BwdArgs a{p.T, p.N, p.V, p.gate, p.Tp, q, k, la, gam, hb, dhb, dq, dk, dla, status};
   if (p.K == 256) return launch_bwd_main_k<256>(p, a, maps, st);
   return launch_bwd_main_k<128>(p, a, maps, st);
 }

@@ -199,6 +199,25 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo_bytes, ui
   return d;
 }
 
+// Shared-memory matrix descriptor without swizzle (layout type 0), version 1:
+// 8-row x 16-byte core matrices; lbo = byte distance between core matrices
+// adjacent along K, sbo = between core matrices adjacent along M/N.
+__device__ __forceinline__ uint64_t sdesc_noswz(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1 << 46;
+  return d;
+}
+
+// K-major operand view of a "chunk-state tile": R rows (M index) by 8*G columns
+// (K index) of bf16 stored as [G][R][8] (16-byte chunk (r, g) at (g*R + r)*16).
+//   row0 (multiple of 8) selects the first M row, k0 (multiple of 16) the K slice.
+__device__ __forceinline__ uint64_t desc_state_kmajor(uint32_t tile, int R, int row0, int k0) {
+  return sdesc_noswz(tile + (uint32_t)((k0 >> 3) * R + row0) * 16u, (uint32_t)R * 16u, 128u);
+}
+
 // Operand view of an SW128 tile with R rows per column block.
 // K-major: rows are the M/N index, the K index runs along columns.
 //   k0 (multiple of 16) selects the MMA's K slice; row0 (multiple of 8) the first M/N row.

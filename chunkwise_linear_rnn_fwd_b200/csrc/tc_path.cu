@@ -8,7 +8,8 @@
 //                             writes h_final (P = 1: a single walk from h0)
 //   MATERIALIZED:             walk(fp32 chunk states) over whole sequences, then
 //                             walk(output, one chunk per CTA) from those states.
-// Backward: see tc_bwd.
+// Backward: chunk states h_n (saved by the forward, or a forward walk), a reverse
+// walk for the adjoints dh_n that also writes dv, then the per-chunk kernel (tc_bwd).
 #include <cudaTypedefs.h>
 
 #include <algorithm>
@@ -101,13 +102,12 @@ int segments_of(const Problem &p, int nvt) {
 struct TcWs {
   bf16 *qg, *kg, *PT;
   float *gam;
-  float *delta;          // [BH][P][K][V] segment contributions
+  float *delta;          // [BH][P][V/4][K] float4 segment contributions
   float *gseg;           // [BH][P][K] per-segment gate products
   float *h32;            // materialised fp32 chunk states [BH][N][K][V]
   // backward
-  bf16 *hb, *dhb;        // bf16 chunk states and adjoints [BH][N][K][V]
+  bf16 *hb, *dhb;        // bf16 chunk states and adjoints [BH][N][K/128][V/8][128][8]
   float *ddelta;
-  float *dscratch;       // bwd per-chunk scratch
   size_t bytes;
 };
 
@@ -146,7 +146,6 @@ TcWs carve(const Problem &p, void *ws, bool bwd) {
     w.gseg = cv.take<float>((size_t)p.BH * P * p.K);
     w.hb = cv.take<bf16>((size_t)p.BH * p.N * p.K * p.V);
     w.dhb = cv.take<bf16>((size_t)p.BH * p.N * p.K * p.V);
-    w.dscratch = cv.take<float>(tc::bwd_scratch_floats(p.BH, p.N, p.K, p.V));
     if (p.variant == GLA_VARIANT_MATERIALIZED && (p.flags & GLA_FLAG_SAVE_STATES))
       w.h32 = cv.take<float>((size_t)p.BH * p.N * p.K * p.V);
   }
@@ -175,7 +174,7 @@ int launch_prep(const Problem &p, const bf16 *q, const bf16 *k, const float *la,
 }
 
 struct WalkMaps {
-  CUtensorMap X, Y, Q, P, H;
+  CUtensorMap X, Y, Q, P;
 };
 
 template <int K, int BV>
@@ -189,11 +188,10 @@ int launch_walk(const Problem &p, const tc::WalkArgs &a, const WalkMaps &m, int 
       return GLA_ERR_CUDA;
     attr = true;
   }
-  const int smem = smem_for_tmem(tc::k_walk<K, BV>, K, W::bytes(a.do_out != 0, a.do_out || a.state_mode == 1),
-                                 kTmemCols);
+  const int smem = smem_for_tmem(tc::k_walk<K, BV>, K, W::bytes(a.do_out != 0, a.do_out != 0), kTmemCols);
   if (smem < 0) return GLA_ERR_CUDA;
   GLA_LAUNCH(K_TC_WALK, st,
-             (tc::k_walk<K, BV><<<dim3(p.V / BV, P, p.BH), K, smem, st>>>(a, m.X, m.Y, m.Q, m.P, m.H)));
+             (tc::k_walk<K, BV><<<dim3(p.V / BV, P, p.BH), K, smem, st>>>(a, m.X, m.Y, m.Q, m.P)));
   // P here is the number of segments this launch covers (a.seg0 .. a.seg0 + P - 1)
   return GLA_OK;
 }
@@ -243,9 +241,6 @@ int tc_fwd(const Problem &p, const void *q, const void *k, const void *v, const 
   const uint64_t BH = (uint64_t)p.BH;
   bool okm = map3(&m.X, w.kg, p.K, p.Tp, BH, 64, 64) && map3(&m.Y, v, p.V, p.T, BH, 64, 64) &&
              map3(&m.Q, w.qg, p.K, p.Tp, BH, 64, 64) && map3(&m.P, w.PT, 64, 64, BH * p.N, 64, 64);
-  m.H = m.X;
-  // the output walk's bf16 copy of each chunk-entry state goes to the backward's h_n
-  if (save) okm = okm && map3(&m.H, w.hb, p.V, p.K, BH * p.N, 64, p.K);
   if (!okm) return GLA_ERR_CUDA;
 
   tc::WalkArgs a{};
@@ -256,6 +251,7 @@ int tc_fwd(const Problem &p, const void *q, const void *k, const void *v, const 
   a.out = (bf16 *)o;
   a.status = status;
   a.end_seg = -1;
+  a.hb = save ? w.hb : nullptr;  // the output walk's bf16 chunk-entry states go to the backward's h_n
 
   if (p.variant == GLA_VARIANT_MATERIALIZED) {
     // pass 1: all chunk states in fp32 (sequential over chunks per (head, d_v tile))
@@ -323,16 +319,13 @@ int tc_bwd(const Problem &p, const void *q, const void *k, const void *v, const 
 
   // ---- chunk states h_n (bf16), recomputed ------------------------------------
   WalkMaps mf;
-  bool okm = map3(&mf.X, w.kg, p.K, p.Tp, BH, 64, 64) && map3(&mf.Y, v, p.V, p.T, BH, 64, 64) &&
-             map3(&mf.H, w.hb, p.V, p.K, BH * p.N, 64, p.K);
+  bool okm = map3(&mf.X, w.kg, p.K, p.Tp, BH, 64, 64) && map3(&mf.Y, v, p.V, p.T, BH, 64, 64);
   mf.Q = mf.X;
   mf.P = mf.X;
-  // ---- chunk adjoints dh_n (bf16) -----------------------------------------------
+  // ---- chunk adjoints dh_n (bf16) and dv = kg_n dh_n + P_n^T dO_n ------------------
   WalkMaps mr;
   okm = okm && map3(&mr.X, w.qg, p.K, p.Tp, BH, 64, 64) && map3(&mr.Y, dout, p.V, p.T, BH, 64, 64) &&
-        map3(&mr.H, w.dhb, p.V, p.K, BH * p.N, 64, p.K);
-  mr.Q = mr.X;
-  mr.P = mr.X;
+        map3(&mr.Q, w.kg, p.K, p.Tp, BH, 64, 64) && map3(&mr.P, w.PT, 64, 64, BH * p.N, 64, 64);
   if (!okm) return GLA_ERR_CUDA;
 
   tc::WalkArgs a{};
@@ -355,6 +348,7 @@ int tc_bwd(const Problem &p, const void *q, const void *k, const void *v, const 
     }
     a.h0 = h0;
     a.state_mode = 1;
+    a.hb = w.hb;
     TRY(launch_walk_any(p, a, mf, P, st));
   }
 
@@ -381,12 +375,15 @@ int tc_bwd(const Problem &p, const void *q, const void *k, const void *v, const 
   }
   r.h0 = dhT;
   r.state_mode = 1;
+  r.hb = w.dhb;
+  r.do_out = 1;
+  r.p_kmajor = 1;
+  r.out = (bf16 *)dv;
   TRY(launch_walk_any(p, r, mr, P, st));
 
   // ---- per-chunk gradients --------------------------------------------------------
   return tc::launch_bwd_main(p, (const bf16 *)q, (const bf16 *)k, (const bf16 *)v, la, (const bf16 *)dout,
-                             (bf16 *)dq, (bf16 *)dk, (bf16 *)dv, dla, w.qg, w.kg, w.PT, w.gam, w.hb, w.dhb,
-                             w.dscratch, status, st);
+                             (bf16 *)dq, (bf16 *)dk, dla, w.gam, w.hb, w.dhb, status, st);
 }
 
 }  // namespace gla
