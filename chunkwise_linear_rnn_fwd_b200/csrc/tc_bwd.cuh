@@ -88,9 +88,10 @@ __global__ void __launch_bounds__(kBwdKH, 2)
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint64_t *full = (uint64_t *)(smem + L::kBar);  // [0],[1] stages
-  uint64_t *mma_bar = full + 2;
+  uint64_t *mma_bar = full + 2;   // phase-1 MMAs, three issuing threads
   uint64_t *qk_bar = full + 3;
-  uint32_t *tslot = (uint32_t *)(full + 4);
+  uint64_t *mma2_bar = full + 4;  // phase-2 MMAs, two issuing threads
+  uint32_t *tslot = (uint32_t *)(full + 5);
   float *red = (float *)(smem + L::kRed);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -105,8 +106,9 @@ __global__ void __launch_bounds__(kBwdKH, 2)
   if (tid == 0) {
     dev::mbar_init(&full[0], 1);
     dev::mbar_init(&full[1], 1);
-    dev::mbar_init(mma_bar, 1);
+    dev::mbar_init(mma_bar, 3);
     dev::mbar_init(qk_bar, 1);
+    dev::mbar_init(mma2_bar, 2);
     dev::fence_mbar_init();
     dev::prefetch_tmap(&tmV);
     dev::prefetch_tmap(&tmDO);
@@ -146,21 +148,25 @@ __global__ void __launch_bounds__(kBwdKH, 2)
     const int s = i & 1;
     uint8_t *st = stage(s);
     if (ok) ok = dev::mbar_wait(&full[s], (i >> 1) & 1, a.status);
-    // issue this tile's MMAs, then sum h (.) dh from the same shared-memory tiles
-    // while they run
-    if (tid == 0 && ok) {
+    // issue this tile's MMAs (lane 0 of warps 0, 1, 2: one accumulator each, since
+    // a tcgen05.mma costs its issuing thread tens of cycles), then sum h (.) dh from
+    // the same shared-memory tiles while they run
+    if (lane == 0 && warp < 3 && ok) {
       const uint32_t sH = dev::smem_u32(st), sDH = sH + L::kTileH, sV = sDH + L::kTileH, sDO = sV + L::kTileV;
       constexpr uint32_t id_kk128 = dev::idesc_bf16(128, 64, false, false);
       constexpr uint32_t id_kk64 = dev::idesc_bf16(64, 64, false, false);
 #pragma unroll
       for (int kk = 0; kk < BVb / 16; ++kk) {
         const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
-        dev::umma_bf16(tmem + cDQ, dev::desc_state_kmajor(sH, kBwdKH, 0, kk * 16),
-                       dev::desc_kmajor(sDO, 64, 0, kk * 16), id_kk128, acc);
-        dev::umma_bf16(tmem + cDK, dev::desc_state_kmajor(sDH, kBwdKH, 0, kk * 16),
-                       dev::desc_kmajor(sV, 64, 0, kk * 16), id_kk128, acc);
-        dev::umma_bf16(tmem + cDP, dev::desc_kmajor(sDO, 64, 0, kk * 16), dev::desc_kmajor(sV, 64, 0, kk * 16),
-                       id_kk64, acc);
+        if (warp == 0)
+          dev::umma_bf16(tmem + cDQ, dev::desc_state_kmajor(sH, kBwdKH, 0, kk * 16),
+                         dev::desc_kmajor(sDO, 64, 0, kk * 16), id_kk128, acc);
+        else if (warp == 1)
+          dev::umma_bf16(tmem + cDK, dev::desc_state_kmajor(sDH, kBwdKH, 0, kk * 16),
+                         dev::desc_kmajor(sV, 64, 0, kk * 16), id_kk128, acc);
+        else
+          dev::umma_bf16(tmem + cDP, dev::desc_kmajor(sDO, 64, 0, kk * 16), dev::desc_kmajor(sV, 64, 0, kk * 16),
+                         id_kk64, acc);
       }
       dev::umma_commit(mma_bar);
     }
@@ -344,26 +350,29 @@ __global__ void __launch_bounds__(kBwdKH, 2)
   dev::tc_fence_before();
   __syncthreads();
   dev::tc_fence_after();
-  if (tid == 0 && ok) {
+  if (lane == 0 && warp < 2 && ok) {  // dq blocks from warp 0, dk blocks from warp 1
     const uint32_t sKh = dev::smem_u32(smem + L::kKh), sQh = dev::smem_u32(smem + L::kQh);
     const int wK[4] = {0, 0, 16, 48};
     const int wQ[4] = {-16, 16, 32, 0};
     constexpr uint32_t id = dev::idesc_bf16(128, 16, true, false);
+    if (warp == 0) {
 #pragma unroll
-    for (int j = 1; j < 4; ++j)
+      for (int j = 1; j < 4; ++j)
 #pragma unroll
-      for (int kk = 0; kk < j; ++kk)
-        dev::umma_bf16(tmem + cQI + 16 * j, dev::desc_mnmajor(sKh, L::kRowsW, wK[j] + 16 * kk, 0),
-                       dev::desc_kmajor(sdP, 64, 16 * j, 16 * kk), id, kk > 0 ? 1u : 0u);
+        for (int kk = 0; kk < j; ++kk)
+          dev::umma_bf16(tmem + cQI + 16 * j, dev::desc_mnmajor(sKh, L::kRowsW, wK[j] + 16 * kk, 0),
+                         dev::desc_kmajor(sdP, 64, 16 * j, 16 * kk), id, kk > 0 ? 1u : 0u);
+    } else {
 #pragma unroll
-    for (int u = 0; u < 3; ++u)
+      for (int u = 0; u < 3; ++u)
 #pragma unroll
-      for (int kk = u + 1; kk < 4; ++kk)
-        dev::umma_bf16(tmem + cKI + 16 * u, dev::desc_mnmajor(sQh, L::kRowsW, wQ[u] + 16 * kk, 0),
-                       dev::desc_kmajor(sdPT, 64, 16 * u, 16 * kk), id, kk > u + 1 ? 1u : 0u);
-    dev::umma_commit(mma_bar);
+        for (int kk = u + 1; kk < 4; ++kk)
+          dev::umma_bf16(tmem + cKI + 16 * u, dev::desc_mnmajor(sQh, L::kRowsW, wQ[u] + 16 * kk, 0),
+                         dev::desc_kmajor(sdPT, 64, 16 * u, 16 * kk), id, kk > u + 1 ? 1u : 0u);
+    }
+    dev::umma_commit(mma2_bar);
   }
-  if (ok) ok = dev::mbar_wait(mma_bar, nvt & 1, a.status);
+  if (ok) ok = dev::mbar_wait(mma2_bar, 0, a.status);
   dev::tc_fence_after();
 
   // ============================ epilogue ============================

@@ -23,6 +23,7 @@ constexpr int kSub = 16;  // sub-chunk
 // Prep: per (chunk, head).  Writes
 //   qg[t]  = q_t (.) e^{B_t}              (bf16, inter-chunk query operand)
 //   kg[t]  = k_t (.) e^{B_63 - B_t}       (bf16, state-update key operand)
+//            (both written over the q / k tiles in shared memory, then TMA-stored)
 //   gam    = e^{B_63}                     (fp32 per key channel)
 //   PT[s][t] = causal intra-chunk score A[t][s] (bf16, transposed)
 // The strictly-lower sub-chunk blocks of A come from three tcgen05 MMAs
@@ -64,7 +65,8 @@ __device__ __forceinline__ int f32_swz(int r, int c) {
 
 template <int K>
 __global__ void __launch_bounds__(256, 1)
-    k_prep(PrepArgs a, const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk) {
+    k_prep(PrepArgs a, const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
+           const __grid_constant__ CUtensorMap tmqg, const __grid_constant__ CUtensorMap tmkg) {
   using L = PrepSmem<K>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -86,7 +88,7 @@ __global__ void __launch_bounds__(256, 1)
   if (warp == 0) dev::tmem_alloc(tslot, 64);
   if (tid == 0) {
     dev::mbar_init(&bar[0], 1);
-    dev::mbar_init(&bar[1], 1);
+    dev::mbar_init(&bar[1], 3);  // one arrival per MMA-issuing thread
     dev::fence_mbar_init();
     dev::mbar_arrive_expect_tx(&bar[0], (uint32_t)(2 * 64 * K * 2));
 #pragma unroll
@@ -143,8 +145,6 @@ __global__ void __launch_bounds__(256, 1)
   }
   const bool ok_ld = dev::mbar_wait(&bar[0], 0, a.status);
 
-  bf16 *qg = a.qg + (bh * a.Tp + (long)n * kC) * K;
-  bf16 *kg = a.kg + (bh * a.Tp + (long)n * kC) * K;
   const int wrow[4] = {0, 0, 16, 48};  // window start row of query sub-chunk j (j >= 1)
 #pragma unroll 1
   for (int j = 0; j < 4; ++j) {
@@ -170,8 +170,11 @@ __global__ void __launch_bounds__(256, 1)
         const float w = __expf(zj1 - Bc[e]);
         const float qh = qf * u;
         const float kw = kf * w;
-        qg[(long)t * K + c] = __float2bfloat16_rn(qh * Ej);
-        kg[(long)t * K + c] = __float2bfloat16_rn(kw * GAj);
+        // qg and kg replace q and k in their tiles (same thread, same element),
+        // which are then stored by TMA
+        const bf16 qgb = __float2bfloat16_rn(qh * Ej), kgb = __float2bfloat16_rn(kw * GAj);
+        dev::st_shared_u16(sQ + dev::sw128_off(64, t, c), *reinterpret_cast<const uint16_t *>(&qgb));
+        dev::st_shared_u16(sK + dev::sw128_off(64, t, c), *reinterpret_cast<const uint16_t *>(&kgb));
         const bf16 qhb = __float2bfloat16_rn(qh);
         dev::st_shared_u16(sQh + dev::sw128_off(64, t, c), *reinterpret_cast<const uint16_t *>(&qhb));
         Af[f32_swz<K>(e, c)] = qh;
@@ -230,42 +233,53 @@ __global__ void __launch_bounds__(256, 1)
   dev::tc_fence_after();
   const uint32_t tmem = *tslot;
 
-  // ---- off-diagonal blocks on the tensor cores ----------------------------
-  if (tid == 0) {
+  // ---- off-diagonal blocks on the tensor cores; qg, kg tiles out by TMA ------
+  // query sub-chunk j (1..3) from lane 0 of warp j - 1 (a tcgen05.mma costs its
+  // issuing thread tens of cycles; the three accumulators are independent)
+  if (lane == 0 && warp < 3) {
+    const int j = warp + 1;
     constexpr uint32_t idesc = dev::idesc_bf16(64, 16, false, false);
-#pragma unroll
-    for (int j = 1; j < 4; ++j) {
-#pragma unroll
-      for (int kk = 0; kk < K / 16; ++kk) {
-        const uint64_t da = dev::desc_kmajor(sKw, L::kRowsKw, wrow[j], kk * 16);
-        const uint64_t db = dev::desc_kmajor(sQh, 64, 16 * j, kk * 16);
-        dev::umma_bf16(tmem + 16 * j, da, db, idesc, kk > 0 ? 1u : 0u);
-      }
+#pragma unroll 4
+    for (int kk = 0; kk < K / 16; ++kk) {
+      const uint64_t da = dev::desc_kmajor(sKw, L::kRowsKw, j == 1 ? 0 : (j == 2 ? 16 : 48), kk * 16);
+      const uint64_t db = dev::desc_kmajor(sQh, 64, 16 * j, kk * 16);
+      dev::umma_bf16(tmem + 16 * j, da, db, idesc, kk > 0 ? 1u : 0u);
     }
     dev::umma_commit(&bar[1]);
+  }
+  if (tid == 32 * 3) {
+#pragma unroll
+    for (int cb = 0; cb < K / 64; ++cb) {
+      dev::tma_store_3d(&tmqg, smem + L::kQ + cb * 64 * 128, cb * 64, n * kC, (int)bh);
+      dev::tma_store_3d(&tmkg, smem + L::kK + cb * 64 * 128, cb * 64, n * kC, (int)bh);
+    }
+    dev::tma_store_commit();
   }
   const bool ok = dev::mbar_wait(&bar[1], 0, a.status) && ok_ld;
   dev::tc_fence_after();
 
-  // ---- assemble P^T rows (key s) and store ------------------------------------
-  if (warp < 4) {
-    const int s = 16 * warp + lane;  // valid for lane < 16
-    const int js = warp;             // sub-chunk of key s
-    float row[kC];
+  // ---- assemble P^T rows (key s) and store: warps w and w+4 share the rows of
+  // TMEM lane block w (columns t < 32 and t >= 32) -------------------------------
+  {
+    const int wb = warp & 3;
+    const int s = 16 * wb + lane;  // valid for lane < 16
+    const int js = wb;             // sub-chunk of key s
+    const int t0 = (warp >> 2) * 32;
+    float row[32];
 #pragma unroll
-    for (int cb = 0; cb < 4; ++cb) dev::tmem_ld16(dev::tmem_addr(tmem, 32 * warp, 16 * cb), row + 16 * cb);
+    for (int cb = 0; cb < 2; ++cb) dev::tmem_ld16(dev::tmem_addr(tmem, 32 * wb, t0 + 16 * cb), row + 16 * cb);
     dev::tmem_wait_ld();
     if (lane < 16) {
-      bf16 *dst = a.PT + ((bh * a.N + n) * kC + s) * kC;
+      bf16 *dst = a.PT + ((bh * a.N + n) * kC + s) * kC + t0;
 #pragma unroll
-      for (int t8 = 0; t8 < kC / 8; ++t8) {
+      for (int t8 = 0; t8 < 4; ++t8) {
         float v8[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          const int t = t8 * 8 + e;
+          const int t = t0 + t8 * 8 + e;
           const int jt = t >> 4;
           float val = 0.f;
-          if (jt > js) val = ok ? row[t] : 0.f;
+          if (jt > js) val = ok ? row[t8 * 8 + e] : 0.f;
           else if (jt == js && t >= s) val = Pd[t * 16 + (s - 16 * js)];
           v8[e] = val;
         }
@@ -278,6 +292,7 @@ __global__ void __launch_bounds__(256, 1)
       }
     }
   }
+  if (tid == 32 * 3) dev::tma_store_wait_all();  // the qg / kg tile stores are complete
   dev::tc_fence_before();
   __syncthreads();
   if (warp == 0) dev::tmem_dealloc(tmem, 64);

@@ -157,8 +157,9 @@ template <int K>
 int launch_prep(const Problem &p, const bf16 *q, const bf16 *k, const float *la, const TcWs &w, unsigned *status,
                 cudaStream_t st) {
   tc::PrepArgs a{p.T, p.N, p.gate, p.Tp, la, w.qg, w.kg, w.PT, w.gam, status};
-  CUtensorMap mq, mk;
-  if (!map3(&mq, q, p.K, p.T, (uint64_t)p.BH, 64, 64) || !map3(&mk, k, p.K, p.T, (uint64_t)p.BH, 64, 64))
+  CUtensorMap mq, mk, mqg, mkg;
+  if (!map3(&mq, q, p.K, p.T, (uint64_t)p.BH, 64, 64) || !map3(&mk, k, p.K, p.T, (uint64_t)p.BH, 64, 64) ||
+      !map3(&mqg, w.qg, p.K, p.Tp, (uint64_t)p.BH, 64, 64) || !map3(&mkg, w.kg, p.K, p.Tp, (uint64_t)p.BH, 64, 64))
     return GLA_ERR_CUDA;
   static int smem = 0;
   if (!smem) {
@@ -169,7 +170,7 @@ int launch_prep(const Problem &p, const bf16 *q, const bf16 *k, const float *la,
     if (got < 0) return GLA_ERR_CUDA;
     smem = got;
   }
-  GLA_LAUNCH(K_TC_PREP, st, (tc::k_prep<K><<<dim3(p.N, p.BH), 256, smem, st>>>(a, mq, mk)));
+  GLA_LAUNCH(K_TC_PREP, st, (tc::k_prep<K><<<dim3(p.N, p.BH), 256, smem, st>>>(a, mq, mk, mqg, mkg)));
   return GLA_OK;
 }
 
