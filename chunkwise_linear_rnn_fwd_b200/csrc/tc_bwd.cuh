@@ -34,6 +34,10 @@ namespace gla {
 namespace tc {
 
 constexpr int kBwdKH = 128;  // key channels per backward CTA
+#ifndef GLA_BWD_STAGGER_NS
+#define GLA_BWD_STAGGER_NS 8000
+#endif
+constexpr unsigned kBwdStaggerNs = GLA_BWD_STAGGER_NS;
 
 struct BwdArgs {
   int T, N, V, gate;
@@ -45,6 +49,10 @@ struct BwdArgs {
   bf16 *dq, *dk;
   float *dla;
   unsigned *status;
+  // CTAs with linear index in [stagger0, stagger1) start stagger_ns later, so
+  // that half of the first wave is loading while the other half computes
+  int stagger0, stagger1;
+  unsigned stagger_ns;
 };
 
 struct BwdSmem {
@@ -95,14 +103,15 @@ __global__ void __launch_bounds__(kBwdKH, 2)
   float *red = (float *)(smem + L::kRed);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int n = blockIdx.x;
-  const long bh = blockIdx.y;
-  const int half = blockIdx.z;
+  // grid (K/128, N, BH): the two channel halves of a chunk are neighbours in
+  // launch order and share the chunk's V and dO tiles through L2
+  const int half = blockIdx.x;
+  const int n = blockIdx.y;
+  const long bh = blockIdx.z;
   const int c0 = half * kBwdKH;
   const int nvt = a.V / BVb;
   const long hrow = bh * a.N + n;
 
-  if (warp == 0) dev::tmem_alloc(tslot, kTmemCols);
   if (tid == 0) {
     dev::mbar_init(&full[0], 1);
     dev::mbar_init(&full[1], 1);
@@ -113,6 +122,16 @@ __global__ void __launch_bounds__(kBwdKH, 2)
     dev::prefetch_tmap(&tmV);
     dev::prefetch_tmap(&tmDO);
   }
+  dev::pdl_launch_dependents();
+  {
+    const int lin = blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z);
+    if (lin >= a.stagger0 && lin < a.stagger1) {  // bounded: stagger_ns < 1 ms
+      const uint64_t t0 = dev::globaltimer();
+      while (dev::globaltimer() - t0 < a.stagger_ns) __nanosleep(256);
+    }
+  }
+  dev::pdl_wait();
+  if (warp == 0) dev::tmem_alloc(tslot, kTmemCols);
   dev::tc_fence_before();
   __syncthreads();
   dev::tc_fence_after();
@@ -485,8 +504,8 @@ int launch_bwd_main_k(const Problem &p, const BwdArgs &a, const CUtensorMap *map
     smem = got;
   }
   GLA_LAUNCH(K_TC_BWD, st,
-             (k_bwd_main<K><<<dim3(p.N, p.BH, K / kBwdKH), kBwdKH, smem, st>>>(a, maps[0], maps[1], maps[2],
-                                                                                maps[3])));
+             if (launch_pdl(k_bwd_main<K>, dim3(K / kBwdKH, p.N, p.BH), dim3(kBwdKH), smem, st, a, maps[0], maps[1],
+                            maps[2], maps[3]) != cudaSuccess) return GLA_ERR_CUDA);
   return GLA_OK;
 }
 
@@ -504,7 +523,15 @@ inline int launch_bwd_main(const Problem &p, const bf16 *q, const bf16 *k, const
   // with a scalar gate and two channel halves, dlog alpha is summed by atomic adds
   if (p.gate == GLA_GATE_SCALAR && p.K > kBwdKH)
     if (cudaMemsetAsync(dla, 0, (size_t)p.BH * p.T * sizeof(float), st) != cudaSuccess) return GLA_ERR_CUDA;
-  BwdArgs a{p.T, p.N, p.V, p.gate, p.Tp, q, k, la, gam, hb, dhb, dq, dk, dla, status};
+  BwdArgs a{p.T, p.N, p.V, p.gate, p.Tp, q, k, la, gam, hb, dhb, dq, dk, dla, status, 0, 0, 0u};
+  {
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    a.stagger0 = sms;  // the second CTA of each SM in the first wave
+    a.stagger1 = 2 * sms;
+    a.stagger_ns = kBwdStaggerNs;
+  }
   if (p.K == 256) return launch_bwd_main_k<256>(p, a, maps, st);
   return launch_bwd_main_k<128>(p, a, maps, st);
 }

@@ -85,11 +85,17 @@ __global__ void __launch_bounds__(256, 1)
   const int n = blockIdx.x;
   const long bh = blockIdx.y;
 
-  if (warp == 0) dev::tmem_alloc(tslot, 64);
   if (tid == 0) {
     dev::mbar_init(&bar[0], 1);
     dev::mbar_init(&bar[1], 3);  // one arrival per MMA-issuing thread
     dev::fence_mbar_init();
+    dev::prefetch_tmap(&tmq);
+    dev::prefetch_tmap(&tmk);
+  }
+  dev::pdl_launch_dependents();
+  dev::pdl_wait();
+  if (warp == 0) dev::tmem_alloc(tslot, 64);
+  if (tid == 0) {
     dev::mbar_arrive_expect_tx(&bar[0], (uint32_t)(2 * 64 * K * 2));
 #pragma unroll
     for (int cb = 0; cb < K / 64; ++cb) {
@@ -384,7 +390,6 @@ __global__ void __launch_bounds__(K, 2)
   const int nloc = n_end - n_begin;
   const int P = a.P;
 
-  if (warp == 0) dev::tmem_alloc(tslot, kTmemCols);
   if (tid == 0) {
     dev::mbar_init(&full[0], 1);
     dev::mbar_init(&full[1], 1);
@@ -397,6 +402,9 @@ __global__ void __launch_bounds__(K, 2)
       dev::prefetch_tmap(&tmP);
     }
   }
+  dev::pdl_launch_dependents();
+  dev::pdl_wait();
+  if (warp == 0) dev::tmem_alloc(tslot, kTmemCols);
   dev::tc_fence_before();
   __syncthreads();
   dev::tc_fence_after();

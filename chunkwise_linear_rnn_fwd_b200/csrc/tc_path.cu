@@ -170,7 +170,9 @@ int launch_prep(const Problem &p, const bf16 *q, const bf16 *k, const float *la,
     if (got < 0) return GLA_ERR_CUDA;
     smem = got;
   }
-  GLA_LAUNCH(K_TC_PREP, st, (tc::k_prep<K><<<dim3(p.N, p.BH), 256, smem, st>>>(a, mq, mk, mqg, mkg)));
+  GLA_LAUNCH(K_TC_PREP, st,
+             if (launch_pdl(tc::k_prep<K>, dim3(p.N, p.BH), dim3(256), smem, st, a, mq, mk, mqg, mkg) != cudaSuccess)
+                 return GLA_ERR_CUDA);
   return GLA_OK;
 }
 
@@ -192,7 +194,8 @@ int launch_walk(const Problem &p, const tc::WalkArgs &a, const WalkMaps &m, int 
   const int smem = smem_for_tmem(tc::k_walk<K, BV>, K, W::bytes(a.do_out != 0, a.do_out != 0), kTmemCols);
   if (smem < 0) return GLA_ERR_CUDA;
   GLA_LAUNCH(K_TC_WALK, st,
-             (tc::k_walk<K, BV><<<dim3(p.V / BV, P, p.BH), K, smem, st>>>(a, m.X, m.Y, m.Q, m.P)));
+             if (launch_pdl(tc::k_walk<K, BV>, dim3(p.V / BV, P, p.BH), dim3(K), smem, st, a, m.X, m.Y, m.Q, m.P) !=
+                 cudaSuccess) return GLA_ERR_CUDA);
   // P here is the number of segments this launch covers (a.seg0 .. a.seg0 + P - 1)
   return GLA_OK;
 }
@@ -223,6 +226,7 @@ int tc_check(const Problem &p) {
   if (p.K != 128 && p.K != 256) return GLA_ERR_UNSUPPORTED_SHAPE;
   if (p.V % 64 != 0) return GLA_ERR_UNSUPPORTED_SHAPE;
   if (p.C != 64 || p.c != 16) return GLA_ERR_UNSUPPORTED_SHAPE;
+  if (p.N > 65535) return GLA_ERR_UNSUPPORTED_SHAPE;  // chunk index is a grid y coordinate of the backward
   return GLA_OK;
 }
 
