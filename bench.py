@@ -48,7 +48,8 @@ def algorithmic_bytes(B, H, T, K, V, gate="vector"):
 # DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) measured by ncu on
 # the full-size workload, with the sha256 of the kernel sources it was measured on.  It is
 # reported only while the sources are unchanged (a changed kernel has unknown traffic).
-NCU_TRAFFIC = {"src_sha256": None, "per_launch_bytes": {}}
+NCU_TRAFFIC = {"src_sha256": "227cea49f4f7e35da7ec2e3369ef342a3a777f685c8173eb04c007e00b52eb72",
+               "per_launch_bytes": {"tc_walk": 117738560, "tc_bwd": 448079104, "tc_prep": 72913920}}
 
 
 def kernel_src_sha256():
