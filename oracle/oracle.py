@@ -127,6 +127,18 @@ def bwd(q, k, v, log_alpha, do, h0=None, dh_final=None, gate="vector", _lib_over
     return dq, dk, dv, dla, dh0
 
 
+def decode_step(q, k, v, log_alpha, state, gate="vector"):
+    """One recurrent decode step per (batch, head): the recurrence of section 4.1 at a
+    single token, S <- diag(alpha) S + k^T v, o = q S (the state after the update).
+    Shapes: q, k [B,H,K]; v [B,H,V]; log_alpha [B,H,K] (vector) / [B,H] (scalar) /
+    None (none); state [B,H,K,V] (None = zero).  Returns (o [B,H,V], new state
+    [B,H,K,V]) as float64; `state` itself is not modified."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    la = None if log_alpha is None else _f64(log_alpha)[:, :, None]
+    o, hT = fwd(q[:, :, None], k[:, :, None], v[:, :, None], la, h0=state, gate=gate)
+    return o[:, :, 0], hT
+
+
 class Mutant:
     """A planted-mistake build of the oracle (pin tests only)."""
 

@@ -156,6 +156,51 @@ def test_golden_hand_computed(oracle_mod):
         np.testing.assert_allclose(hT, np.array(case["h_final"], float), rtol=0, atol=1e-12)
 
 
+def test_decode_steps_reproduce_golden(oracle_mod):
+    """The decode step applied token by token reproduces the hand-computed outputs and
+    final state of tests/golden/*.json (the state carried between calls)."""
+    gdir = os.path.join(os.path.dirname(__file__), "golden")
+    files = sorted(f for f in os.listdir(gdir) if f.startswith("hand_") and f.endswith(".json"))
+    assert files
+    for f in files:
+        case = json.load(open(os.path.join(gdir, f)))
+        q = np.array(case["q"], float)
+        k = np.array(case["k"], float)
+        v = np.array(case["v"], float)
+        la = np.log(np.array(case["alpha"], float))
+        K, V = q.shape[1], v.shape[1]
+        S = np.zeros((1, 1, K, V)) if case.get("h0") is None else np.array(case["h0"], float)[None, None]
+        for t in range(q.shape[0]):
+            o, S = oracle_mod.decode_step(q[None, None, t], k[None, None, t], v[None, None, t],
+                                          la[None, None, t], S)
+            np.testing.assert_allclose(o[0, 0], np.array(case["o"], float)[t], rtol=0, atol=1e-12)
+        np.testing.assert_allclose(S[0, 0], np.array(case["h_final"], float), rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("gate", ["vector", "scalar", "none"])
+def test_decode_steps_match_sequence_forward(oracle_mod, gate):
+    """T decode steps from h0 equal one forward pass over the T tokens from h0, and the
+    step leaves its input state untouched."""
+    rng = np.random.default_rng(11)
+    B, H, T, K, V = 2, 3, 5, 4, 3
+    q, k, v = rng.normal(size=(B, H, T, K)), rng.normal(size=(B, H, T, K)), rng.normal(size=(B, H, T, V))
+    la = None
+    if gate == "vector":
+        la = -rng.uniform(0.01, 2.0, size=(B, H, T, K))
+    elif gate == "scalar":
+        la = -rng.uniform(0.01, 2.0, size=(B, H, T))
+    h0 = rng.normal(size=(B, H, K, V))
+    o_ref, hT_ref = oracle_mod.fwd(q, k, v, la, h0=h0, gate=gate)
+    S = h0.copy()
+    for t in range(T):
+        S_in, S_copy = S, S.copy()
+        o, S = oracle_mod.decode_step(q[:, :, t], k[:, :, t], v[:, :, t], None if la is None else la[:, :, t], S_in,
+                                      gate=gate)
+        np.testing.assert_array_equal(S_in, S_copy)
+        np.testing.assert_allclose(o, o_ref[:, :, t], rtol=1e-13, atol=1e-13)
+    np.testing.assert_allclose(S, hT_ref, rtol=1e-13, atol=1e-13)
+
+
 # --------------------------------------------------------------- backward pins
 
 def loss_of(oracle, q, k, v, la, h0, do, dhT, gate):
