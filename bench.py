@@ -252,6 +252,45 @@ def kernel_io_bytes(name, w, sms=148):
     return None
 
 
+DECODE_WORKLOAD = dict(B=128, H=4, K=256, V=512)
+
+
+def measure_decode(args, dev, stream, peaks, peak_src, seed=0):
+    """The recurrent decode step (one token per head, state updated in place) on a batch
+    whose fp32 state (256 MB) exceeds L2: device time per step and the HBM roofline of
+    its algorithmic bytes (state read + write, q, k, v, log alpha read, o written)."""
+    import torch
+
+    import chunkwise_linear_rnn_fwd_b200 as pkg
+    from chunkwise_linear_rnn_fwd_b200.synth import make_inputs
+
+    w = DECODE_WORKLOAD
+    B, H, K, V = w["B"], w["H"], w["K"], w["V"]
+    x = make_inputs(B, H, 1, K, V, dtype=torch.bfloat16, gate="vector", seed=seed, with_h0=True)
+    q, k, v = (t[:, :, 0].contiguous().to(dev) for t in (x.q, x.k, x.v))
+    la = x.log_alpha[:, :, 0].contiguous().to(dev)
+    S = x.h0.to(dev).contiguous()
+    o = torch.empty(B, H, V, dtype=torch.bfloat16, device=dev)
+    for _ in range(max(3, args.warmup)):
+        pkg.gla_decode_step(q, k, v, la, S, o=o, stream=stream)
+    torch.cuda.synchronize()
+    n = max(10, args.steps)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(n):
+        pkg.gla_decode_step(q, k, v, la, S, o=o, stream=stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / n
+    nbytes = B * H * (2 * K * V * 4 + 2 * K * 2 + V * 2 + K * 4 + V * 2)
+    gbs = nbytes / (ms / 1e3) / 1e9
+    peak = float(peaks["hbm_gbs"])
+    return {"workload": f"decode step, B={B} H={H} d_k={K} d_v={V}, bf16 q/k/v/o, fp32 state, vector gates",
+            "ms_per_step": ms, "tokens_per_s": B / (ms / 1e3), "bytes_per_step": nbytes,  # one token per sequence
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak,
+                         "peak_source": peak_src}}
+
+
 def run_ours(args, w):
     import torch
     import torch.distributed as dist
@@ -383,6 +422,8 @@ def run_ours(args, w):
         "flops_per_step": flops, "algorithmic_bytes_per_step": abytes, "peak_source": peak_src,
     }
 
+    decode = measure_decode(args, dev, stream, peaks, peak_src, seed=rank)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         r, dt, threads, desc = oracle_sample_rate(w, T_sample=w["T"], min_seconds=args.cpu_seconds)
@@ -403,7 +444,7 @@ def run_ours(args, w):
             "gpu_launches": len(launches),
             "kernel_timing": "separate pass of the same K steps with a CUDA-event pair around each launch",
             "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-            "clocks": clocks, "cpu_baseline": cpu,
+            "clocks": clocks, "cpu_baseline": cpu, "decode_step": decode,
         }
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -11,7 +11,8 @@ namespace gla {
 const char *kernel_name(int id) {
   static const char *names[K_COUNT] = {
       "f32_prep",  "f32_states", "f32_scores", "f32_out",    "f32_dstates", "f32_dscores", "f32_dqk",
-      "f32_dv",    "f32_dg_out", "tc_prep",    "tc_walk",    "tc_scan(unused)", "tc_bwd",  "status_clear"};
+      "f32_dv",    "f32_dg_out", "tc_prep",    "tc_walk",    "tc_scan(unused)", "tc_bwd",  "status_clear",
+      "decode"};
   if (id < 0 || id >= K_COUNT) return "unknown";
   return names[id];
 }
@@ -256,6 +257,27 @@ int gla_timing_collect(int max, int *kernel_ids, float *ms) {
 }
 
 const char *gla_kernel_name(int kernel_id) { return gla::kernel_name(kernel_id); }
+
+int gla_decode_step(const gla_desc *desc, const void *q, const void *k, const void *v, const float *log_alpha,
+                    float *state, void *o, void *stream) {
+  if (!desc) return GLA_ERR_INVALID_ARG;
+  if (desc->B < 1 || desc->H < 1 || desc->T != 1 || desc->dk < 1 || desc->dv < 1) return GLA_ERR_INVALID_ARG;
+  if (desc->dtype != GLA_DTYPE_BF16 && desc->dtype != GLA_DTYPE_FP32) return GLA_ERR_INVALID_ARG;
+  if (desc->gate != GLA_GATE_VECTOR && desc->gate != GLA_GATE_SCALAR && desc->gate != GLA_GATE_NONE)
+    return GLA_ERR_INVALID_ARG;
+  if (desc->dk > 4096 || desc->dv % 4 != 0 || (long)desc->B * desc->H > 65535) return GLA_ERR_UNSUPPORTED_SHAPE;
+  GLA_TRY(check_req(q));
+  GLA_TRY(check_req(k));
+  GLA_TRY(check_req(v));
+  GLA_TRY(check_req(o));
+  GLA_TRY(check_req(state));
+  if (desc->gate == GLA_GATE_NONE) {
+    if (log_alpha) return GLA_ERR_INVALID_ARG;
+  } else {
+    GLA_TRY(check_req(log_alpha));
+  }
+  return decode_step(desc, q, k, v, log_alpha, state, o, (cudaStream_t)stream);
+}
 
 const char *gla_build_info(void) {
   return "gla-b200: sm_100a; bf16 path tcgen05/TMEM/TMA; fp32 path CUDA cores";

@@ -25,6 +25,7 @@ enum KernelId : int {
   K_TC_SCAN,
   K_TC_BWD,
   K_STATUS_CLEAR,
+  K_DECODE,
   K_COUNT
 };
 
@@ -72,6 +73,10 @@ int f32_fwd(const Problem &p, const void *q, const void *k, const void *v, const
 int f32_bwd(const Problem &p, const void *q, const void *k, const void *v, const float *la,
             const float *h0, const void *dout, const float *dhT, void *dq, void *dk, void *dv,
             float *dla, float *dh0, void *ws, cudaStream_t st);
+
+// recurrent decode step (CUDA cores); arguments validated by the caller
+int decode_step(const gla_desc *d, const void *q, const void *k, const void *v, const float *la, float *state,
+                void *o, cudaStream_t st);
 
 }  // namespace gla
 

@@ -29,7 +29,8 @@ NOALLOC_SCRATCH_BYTES = 64 << 20  # GLA_NOALLOC_SCRATCH_BYTES in include/gla.h
 
 # Every exported symbol of include/gla.h.
 EXPORTS = ["gla_workspace_size", "gla_check", "gla_fwd", "gla_bwd", "gla_poll_status", "gla_status_string",
-           "gla_timing_enable", "gla_timing_collect", "gla_kernel_name", "gla_build_info", "gla_fwd_noalloc"]
+           "gla_timing_enable", "gla_timing_collect", "gla_kernel_name", "gla_build_info", "gla_fwd_noalloc",
+           "gla_decode_step"]
 
 
 class GLAError(RuntimeError):
@@ -66,6 +67,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.gla_fwd.restype = i
     lib.gla_fwd_noalloc.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, i, vp]
     lib.gla_fwd_noalloc.restype = i
+    lib.gla_decode_step.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp]
+    lib.gla_decode_step.restype = i
     lib.gla_bwd.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, vp]
     lib.gla_bwd.restype = i
     lib.gla_poll_status.argtypes = [dp, vp]
@@ -190,6 +193,25 @@ def gla_fwd_noalloc(q, k, v, log_alpha=None, h0=None, *, chunk=64, gate=None, su
     if r != GLA_OK:
         raise GLAError(r, "gla_fwd_noalloc")
     return o, h_final
+
+
+def gla_decode_step(q, k, v, log_alpha, state, *, gate=None, o=None, stream=None):
+    """One recurrent decode step per (batch, head): state <- diag(alpha) state + k^T v
+    (in place), o = q state.  q, k [B,H,d_k]; v [B,H,d_v]; log_alpha [B,H,d_k] or
+    [B,H] or None; state [B,H,d_k,d_v] fp32.  Returns o [B,H,d_v].  See include/gla.h."""
+    lib = load()
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    if gate is None:
+        gate = "none" if log_alpha is None else ("vector" if log_alpha.dim() == 3 else "scalar")
+    if o is None:
+        o = torch.empty(B, H, dv, dtype=q.dtype, device=q.device)
+    d = make_desc(B, H, 1, dk, dv, q.dtype, gate)
+    r = lib.gla_decode_step(ctypes.byref(d), _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(state), _ptr(o),
+                            _stream_handle(stream))
+    if r != GLA_OK:
+        raise GLAError(r, "gla_decode_step")
+    return o
 
 
 def gla_bwd(q, k, v, log_alpha, do, h0=None, dh_final=None, *, chunk=64, gate=None, subchunk=16, dq=None, dk=None,

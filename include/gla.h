@@ -149,6 +149,22 @@ int gla_bwd(const gla_desc *desc, const void *q, const void *k, const void *v,
             void *dq, void *dk, void *dv, float *dlog_alpha, float *dh0, int chunk,
             void *stream);
 
+/* ---- recurrent decode step ---------------------------------------------------
+ * One token per (batch, head) in the recurrent form of section 4.1 (the form the
+ * paper uses for generation), on the state the caller carries between calls:
+ *     S <- diag(alpha) S + k^T v ,     o = q S   (o reads the updated state).
+ *   q, k [B,H,d_k]; v, o [B,H,d_v] (element type desc->dtype); log_alpha
+ *   [B,H,d_k] (GLA_GATE_VECTOR) or [B,H] (GLA_GATE_SCALAR) or NULL
+ *   (GLA_GATE_NONE), fp32; state [B,H,d_k,d_v] fp32, read and overwritten in
+ *   place (it must not alias q, k, v, log_alpha or o).
+ * desc->T must be 1; d_k <= 4096 and d_v a multiple of 4.  desc->subchunk,
+ * variant, segments, flags and the workspace are ignored (no scratch memory).
+ * Every argument is validated before anything is enqueued; the call is
+ * asynchronous on `stream` and bound by HBM bandwidth on the state.
+ * Returns GLA_OK or an error code; on error nothing was enqueued. */
+int gla_decode_step(const gla_desc *desc, const void *q, const void *k, const void *v,
+                    const float *log_alpha, float *state, void *o, void *stream);
+
 /* ---- forward without a workspace ---------------------------------------------
  * No counterpart in the paper: this entry point exists for callers that cannot
  * allocate device memory -- a program whose device memory is all owned by

@@ -110,6 +110,32 @@ def test_bad_calls_enqueue_nothing(lib):
     assert b(ctypes.byref(d), a, a, a, None, None, a, None, a, a, a, a, None, 64, None) == -1   # none gate with dla
 
 
+def test_decode_step_validation_enqueues_nothing(lib):
+    """gla_decode_step rejects bad descriptors and pointers before any launch."""
+    vp = ctypes.c_void_p
+    a = vp(4096)
+    mis = vp(4096 + 4)
+    d = desc(T=1, dk=128, dv=128)
+    f = lib.gla_decode_step
+    f.argtypes = [ctypes.POINTER(type(d)), vp, vp, vp, vp, vp, vp, vp]
+    assert f(None, a, a, a, a, a, a, None) == -1                              # no descriptor
+    d.T = 2
+    assert f(ctypes.byref(d), a, a, a, a, a, a, None) == -1                   # T must be 1
+    d.T = 1
+    d.dv = 126
+    assert f(ctypes.byref(d), a, a, a, a, a, a, None) == -2                   # d_v not a multiple of 4
+    d.dv = 128
+    d.dk = 5000
+    assert f(ctypes.byref(d), a, a, a, a, a, a, None) == -2                   # d_k too large
+    d.dk = 128
+    assert f(ctypes.byref(d), a, a, a, None, a, a, None) == -1                # vector gate without log_alpha
+    assert f(ctypes.byref(d), a, a, a, a, None, a, None) == -1                # state NULL
+    assert f(ctypes.byref(d), a, a, a, a, mis, a, None) == -3                 # state misaligned
+    assert f(ctypes.byref(d), a, a, mis, a, a, a, None) == -3                 # v misaligned
+    d.gate = 2
+    assert f(ctypes.byref(d), a, a, a, a, a, a, None) == -1                   # none gate with log_alpha
+
+
 def test_oracle_not_imported_by_product():
     """The product package never imports, loads or links the oracle."""
     pkg_dir = os.path.join(ROOT, "chunkwise_linear_rnn_fwd_b200")
