@@ -454,6 +454,77 @@ def run_ours(args, w):
     return 0
 
 
+SWEEP = ([dict(name="config 2: fwd, B=8 H=4 T=2048 d_k=128 d_v=256", B=8, H=4, T=2048, K=128, V=256, gate=g,
+               z_mean=0.0, bwd=False) for g in ("vector", "none")]
+         + [dict(name="config 3: fwd+bwd, B=8 H=4 T=2048 d_k=128 d_v=256", B=8, H=4, T=2048, K=128, V=256,
+                 gate="vector", z_mean=0.0, bwd=True)]
+         + [dict(name="config 4: fwd+bwd, B=2 H=4 T=4096 d_k=256 d_v=512", B=2, H=4, T=4096, K=256, V=512,
+                 gate="vector", z_mean=-1.0, bwd=True)]
+         + [dict(name=f"config 5: fwd+bwd, B*T=32768 H=4 d_k=256 d_v=512, T={T}", B=32768 // T, H=4, T=T, K=256,
+                 V=512, gate=g, z_mean=0.0, bwd=True)
+            for T in (1024, 2048, 4096, 8192, 16384) for g in ("vector", "scalar", "none")])
+
+
+def run_sweep(args):
+    """Device time of every workload configuration (one JSON line, --sweep): the forward
+    (and backward) as bench.py's step launches them, inputs drawn once per shape on the
+    device with the workload's distributions (timing only; parity is in tests/)."""
+    import torch
+
+    import chunkwise_linear_rnn_fwd_b200 as pkg
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    pkg.load()
+    peaks, peak_src = load_peaks()
+    stream = torch.cuda.current_stream()
+    g = torch.Generator(device=dev)
+    g.manual_seed(0)
+    out = []
+    for c in SWEEP:
+        B, H, T, K, V, C = c["B"], c["H"], c["T"], c["K"], c["V"], 64
+        q = torch.randn(B, H, T, K, device=dev, generator=g).to(torch.bfloat16)
+        k = (torch.randn(B, H, T, K, device=dev, generator=g) / K ** 0.5).to(torch.bfloat16)
+        v = torch.randn(B, H, T, V, device=dev, generator=g).to(torch.bfloat16)
+        do = torch.randn(B, H, T, V, device=dev, generator=g).to(torch.bfloat16)
+        shape = {"vector": (B, H, T, K), "scalar": (B, H, T)}.get(c["gate"])
+        la = None if shape is None else torch.nn.functional.logsigmoid(
+            torch.randn(*shape, device=dev, generator=g) + c["z_mean"]) / 16
+        o = torch.empty_like(v)
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        dla = None if la is None else torch.empty_like(la)
+        flags = pkg.FLAG_REUSE_PREP | pkg.FLAG_SAVE_STATES if c["bwd"] else 0
+        ws = pkg.alloc_workspace(pkg.workspace_size(B, H, T, K, V, torch.bfloat16, c["gate"], C, c["bwd"],
+                                                    flags=flags), dev)
+
+        def step():
+            pkg.gla_fwd(q, k, v, la, None, chunk=C, gate=c["gate"], o=o, want_final=False, workspace=ws,
+                        stream=stream, save_states=c["bwd"])
+            if c["bwd"]:
+                pkg.gla_bwd(q, k, v, la, do, None, None, chunk=C, gate=c["gate"], dq=dq, dk=dk, dv=dv,
+                            dlog_alpha=dla, want_dh0=False, workspace=ws, stream=stream, reuse_prep=True,
+                            saved_states=True)
+
+        for _ in range(args.warmup):
+            step()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / args.steps
+        th = B * H * T
+        flops = th * (4 * K * V + C * (K + V)) + (th * (10 * K * V + C * (3 * K + 2 * V)) if c["bwd"] else 0)
+        out.append({"workload": c["name"], "gate": c["gate"], "ms_per_step": ms, "tokens_per_s": B * T / (ms / 1e3),
+                    "tflops": flops / (ms / 1e3) / 1e12,
+                    "frac_of_tensor_peak": flops / (ms / 1e3) / (float(peaks.get("bf16_tflops", 1590)) * 1e12)})
+        del q, k, v, do, la, o, dq, dk, dv, dla, ws
+    print(json.dumps({"metric": METRIC, "sweep": out, "peak_source": peak_src}), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -466,6 +537,7 @@ def main():
     ap.add_argument("--batch", type=int, default=None, help="override B (smaller profiling captures)")
     ap.add_argument("--heads", type=int, default=None, help="override H")
     ap.add_argument("--seqlen", type=int, default=None, help="override T")
+    ap.add_argument("--sweep", action="store_true", help="time every workload configuration (one JSON line)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -475,6 +547,8 @@ def main():
             w[key] = val
     if args.impl == "reference":
         return run_reference(args, w)
+    if args.sweep:
+        return run_sweep(args)
     return run_ours(args, w)
 
 
