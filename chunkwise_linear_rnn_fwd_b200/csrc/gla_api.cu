@@ -279,6 +279,12 @@ int gla_decode_step(const gla_desc *desc, const void *q, const void *k, const vo
   return decode_step(desc, q, k, v, log_alpha, state, o, (cudaStream_t)stream);
 }
 
+int gla_selftest_timeout(void *status_word, unsigned limit_us, void *stream) {
+  if (!status_word || limit_us < 1 || limit_us > 1000000) return GLA_ERR_INVALID_ARG;
+  if (((uintptr_t)status_word & 3u) != 0) return GLA_ERR_MISALIGNED;
+  return gla::selftest_timeout((unsigned *)status_word, limit_us, (cudaStream_t)stream);
+}
+
 const char *gla_build_info(void) {
   return "gla-b200: sm_100a; bf16 path tcgen05/TMEM/TMA; fp32 path CUDA cores";
 }

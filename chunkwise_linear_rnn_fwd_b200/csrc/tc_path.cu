@@ -222,6 +222,22 @@ int launch_prep_any(const Problem &p, const bf16 *q, const bf16 *k, const float 
 
 }  // namespace
 
+namespace {
+// One thread waits, with the library's bounded wait, on an mbarrier that nothing
+// will ever complete; the wait gives up after limit_ns and records ST_TIMEOUT.
+__global__ void k_selftest_timeout(unsigned *status, unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  dev::mbar_init(&bar, 1);
+  dev::fence_mbar_init();
+  (void)dev::mbar_wait(&bar, 0, status, limit_ns);
+}
+}  // namespace
+
+int selftest_timeout(unsigned *status, unsigned limit_us, cudaStream_t st) {
+  k_selftest_timeout<<<1, 1, 0, st>>>(status, 1000ull * limit_us);
+  return cudaGetLastError() == cudaSuccess ? GLA_OK : GLA_ERR_CUDA;
+}
+
 int tc_check(const Problem &p) {
   if (p.K != 128 && p.K != 256) return GLA_ERR_UNSUPPORTED_SHAPE;
   if (p.V % 64 != 0) return GLA_ERR_UNSUPPORTED_SHAPE;

@@ -4,6 +4,7 @@
 
 namespace gla {
 int tc_check(const Problem &p);
+int selftest_timeout(unsigned *status, unsigned limit_us, cudaStream_t st);
 size_t tc_workspace(const Problem &p, bool bwd);
 int tc_fwd(const Problem &p, const void *q, const void *k, const void *v, const float *la, const float *h0,
            void *o, float *hT, void *ws, cudaStream_t st);

@@ -30,7 +30,7 @@ NOALLOC_SCRATCH_BYTES = 64 << 20  # GLA_NOALLOC_SCRATCH_BYTES in include/gla.h
 # Every exported symbol of include/gla.h.
 EXPORTS = ["gla_workspace_size", "gla_check", "gla_fwd", "gla_bwd", "gla_poll_status", "gla_status_string",
            "gla_timing_enable", "gla_timing_collect", "gla_kernel_name", "gla_build_info", "gla_fwd_noalloc",
-           "gla_decode_step"]
+           "gla_decode_step", "gla_selftest_timeout"]
 
 
 class GLAError(RuntimeError):
@@ -69,6 +69,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.gla_fwd_noalloc.restype = i
     lib.gla_decode_step.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp]
     lib.gla_decode_step.restype = i
+    lib.gla_selftest_timeout.argtypes = [vp, ctypes.c_uint, vp]
+    lib.gla_selftest_timeout.restype = i
     lib.gla_bwd.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, vp]
     lib.gla_bwd.restype = i
     lib.gla_poll_status.argtypes = [dp, vp]
@@ -252,6 +254,15 @@ def poll_status(workspace: torch.Tensor, stream=None) -> int:
     d.workspace = workspace.data_ptr()
     d.workspace_bytes = workspace.numel()
     return int(load().gla_poll_status(ctypes.byref(d), _stream_handle(stream)))
+
+
+def selftest_timeout(workspace: torch.Tensor, limit_us: int = 20000, stream=None) -> None:
+    """Enqueue the bounded-wait self-test: a kernel whose wait on an mbarrier that
+    nothing completes runs out after limit_us and sets the timeout bit of the status
+    word at the start of `workspace` (read it with poll_status)."""
+    r = load().gla_selftest_timeout(ctypes.c_void_p(workspace.data_ptr()), int(limit_us), _stream_handle(stream))
+    if r != GLA_OK:
+        raise GLAError(r, "gla_selftest_timeout")
 
 
 def timing_enable(on: bool = True) -> None:

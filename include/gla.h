@@ -208,6 +208,15 @@ int gla_timing_enable(int on);
 int gla_timing_collect(int max, int *kernel_ids, float *ms);
 const char *gla_kernel_name(int kernel_id);
 
+/* Self-test of the device-side bounded waits (no counterpart in the paper).
+ * Enqueues one kernel whose single thread waits, with the same bounded wait
+ * every kernel of this library uses, on an mbarrier that nothing completes; the
+ * wait gives up after limit_us microseconds (1 .. 1e6) and sets the timeout bit
+ * in the 4-byte device word *status_word, which gla_poll_status reads when it is
+ * the first word of desc->workspace.  It faults nothing and leaves the context
+ * usable; it exists so that the timeout path can be tested. */
+int gla_selftest_timeout(void *status_word, unsigned limit_us, void *stream);
+
 /* Build information: a static string naming the kernels and architecture. */
 const char *gla_build_info(void);
 
