@@ -69,6 +69,14 @@ def measured_traffic(kernel):
     return NCU_TRAFFIC["per_launch_bytes"].get(kernel)
 
 
+def bench_config(w, world):
+    """The `config` object of the JSON line (the same for both arms)."""
+    return {"workload": f"gla fwd+bwd, B={w['B']} H={w['H']} T={w['T']} d_k={w['K']} d_v={w['V']} C={w['C']}, "
+                        f"bf16, {w['gate']} gates z~N({w['z_mean']:g},1), fp32 state",
+            "global_batch": w["B"] * world, "seq_len": w["T"], "parallelism": f"replicas x{world}",
+            "l2": "inputs larger than L2 (~268 MB touched per step)"}
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -201,8 +209,7 @@ def run_reference(args, w):
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / max(1, args.steps),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": "gla fwd+bwd, B=2 H=4 T=4096 d_k=256 d_v=512, vector gates z~N(-1,1)",
-                   "sample": desc},
+        "config": bench_config(w, world),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": desc},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -435,10 +442,7 @@ def run_ours(args, w):
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": f"gla fwd+bwd, B={B} H={H} T={T} d_k={K} d_v={V} C={C}, bf16, vector gates "
-                                   "z~N(-1,1), fp32 state",
-                       "global_batch": B * world, "seq_len": T, "parallelism": f"replicas x{world}",
-                       "l2": "inputs larger than L2 (~268 MB touched per step)"},
+            "config": bench_config(w, world),
             "tflops": step_roofline["tflops"], "step_roofline": step_roofline, "roofline": roofline,
             "kernels": {k2: {"launches": v2[0], "ms_total": v2[1], "share": v2[1] / max(1e-9, sum(x[1] for x in per_kernel.values()))}
                         for k2, v2 in sorted(per_kernel.items(), key=lambda kv: -kv[1][1])},
