@@ -201,6 +201,53 @@ def test_decode_steps_match_sequence_forward(oracle_mod, gate):
     np.testing.assert_allclose(S, hT_ref, rtol=1e-13, atol=1e-13)
 
 
+# ------------------------------------------------------- layer epilogue pins
+
+def test_epilogue_normalisation_and_gate_closed_forms():
+    """With w = 1, b = 0 each row of LN(o) has mean 0 and variance var/(var+eps);
+    the Swish gate at r = 0 is 0 and for large r tends to r; w and b act affinely."""
+    from oracle import epilogue
+    rng = np.random.default_rng(31)
+    o = rng.normal(size=(2, 3, 5, 16)) * 3 + 1
+    ones = np.ones_like(o)
+    n = epilogue.fwd(o, 50.0 * ones) / 50.0      # sigmoid(50) = 1 - 2e-22
+    np.testing.assert_allclose(n.mean(axis=-1), 0.0, atol=1e-12)
+    var = o.var(axis=-1)
+    np.testing.assert_allclose(n.var(axis=-1), var / (var + 1e-5), rtol=1e-12)
+    assert np.all(epilogue.fwd(o, 0.0 * ones) == 0.0)
+    w, b = rng.normal(size=16), rng.normal(size=16)
+    np.testing.assert_allclose(epilogue.fwd(o, 50.0 * ones, w, b) / 50.0, n * w + b, rtol=1e-12, atol=1e-12)
+    # Swish against its definition evaluated with Python's math module
+    import math
+    r = np.array([-4.0, -0.5, 0.0, 0.3, 2.0])
+    ref = [x / (1.0 + math.exp(-x)) for x in r]
+    np.testing.assert_allclose(epilogue.fwd(np.array([[1.0, -1.0]]).repeat(5, 0), r[:, None].repeat(2, 1))[:, 0],
+                               np.array(ref) * (1.0 / math.sqrt(1.0 + 1e-5)), rtol=1e-14)
+
+
+def test_epilogue_gradients_finite_differences():
+    """Every gradient of the epilogue against central differences of the forward."""
+    from oracle import epilogue
+    rng = np.random.default_rng(32)
+    o, r, dy = rng.normal(size=(2, 3, 8)), rng.normal(size=(2, 3, 8)), rng.normal(size=(2, 3, 8))
+    w, b = rng.normal(size=8), rng.normal(size=8)
+    do, dr, dw, db = epilogue.bwd(o, r, dy, w, b)
+    L = lambda o_, r_, w_, b_: float(np.sum(epilogue.fwd(o_, r_, w_, b_) * dy))
+    h = 1e-6
+    for name, x, g in (("o", o, do), ("r", r, dr), ("w", w, dw), ("b", b, db)):
+        num = np.zeros_like(x)
+        for idx in np.ndindex(x.shape):
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += h
+            xm[idx] -= h
+            args_p = {"o": o, "r": r, "w": w, "b": b}
+            args_m = dict(args_p)
+            args_p[name], args_m[name] = xp, xm
+            num[idx] = (L(args_p["o"], args_p["r"], args_p["w"], args_p["b"])
+                        - L(args_m["o"], args_m["r"], args_m["w"], args_m["b"])) / (2 * h)
+        np.testing.assert_allclose(g, num, rtol=1e-6, atol=1e-8, err_msg=name)
+
+
 # --------------------------------------------------------------- backward pins
 
 def loss_of(oracle, q, k, v, la, h0, do, dhT, gate):
