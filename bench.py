@@ -299,6 +299,56 @@ def measure_decode(args, dev, stream, peaks, peak_src, seed=0):
                          "peak_source": peak_src}}
 
 
+def measure_epilogue(args, w, dev, stream, peaks, peak_src, seed=0):
+    """The layer epilogue (LayerNorm of each head's output times the Swish output gate)
+    on the bench workload's output shape: device time of the forward and of the
+    backward (with dw, db) and their HBM rooflines on algorithmic bytes."""
+    import torch
+
+    import chunkwise_linear_rnn_fwd_b200 as pkg
+
+    B, H, T, V = w["B"], w["H"], w["T"], w["V"]
+    g = torch.Generator(device=dev)
+    g.manual_seed(seed)
+    o, r, dy = (torch.randn(B, H, T, V, device=dev, generator=g).to(torch.bfloat16) for _ in range(3))
+    wt = torch.ones(V, device=dev)
+    bs = torch.zeros(V, device=dev)
+    y = torch.empty_like(o)
+    lib = pkg.load()
+    d = pkg.gla.make_desc(B, H, T, 1, V, torch.bfloat16, "none")
+    ws = pkg.alloc_workspace(lib.gla_epilogue_workspace_size(__import__("ctypes").byref(d)), dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)  # twice the L2
+    res = {}
+    for name, fn in (("fwd", lambda: pkg.gla_epilogue_fwd(o, r, wt, bs, y=y, stream=stream)),
+                     ("bwd", lambda: pkg.gla_epilogue_bwd(o, r, dy, wt, bs, workspace=ws, stream=stream))):
+        for _ in range(max(3, args.warmup)):
+            fn()
+        torch.cuda.synchronize()
+        # device time of every launch (library events on the launch stream), L2 flushed
+        # before each call so that no input is served from the previous iteration's L2
+        n = max(10, args.steps)
+        pkg.timing_enable(True)
+        pkg.timing_collect()
+        for _ in range(n):
+            flush.fill_(1)  # on torch's current stream, which is the launch stream
+            fn()
+        torch.cuda.synchronize()
+        launches = pkg.timing_collect()
+        pkg.timing_enable(False)
+        per_kernel = {}
+        for kname, kms in launches:
+            per_kernel[kname] = per_kernel.get(kname, 0.0) + kms / n
+        ms = sum(per_kernel.values())
+        elems = B * H * T * V
+        nbytes = elems * 2 * (3 if name == "fwd" else 5) + 4 * 4 * V
+        gbs = nbytes / (ms / 1e3) / 1e9
+        res[name] = {"ms": ms, "kernels_ms": per_kernel, "bytes": nbytes, "achieved_gbs": gbs,
+                     "frac_of_hbm": gbs / float(peaks["hbm_gbs"]), "l2": "flushed before every call"}
+    res["workload"] = f"layer epilogue, B={B} H={H} T={T} d_v={V}, bf16 (fwd: o, r -> y; bwd: o, r, dy -> do, dr, dw, db)"
+    res["peak_source"] = peak_src
+    return res
+
+
 def run_ours(args, w):
     import torch
     import torch.distributed as dist
@@ -431,6 +481,7 @@ def run_ours(args, w):
     }
 
     decode = measure_decode(args, dev, stream, peaks, peak_src, seed=rank)
+    epilogue = measure_epilogue(args, w, dev, stream, peaks, peak_src, seed=rank)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -449,7 +500,7 @@ def run_ours(args, w):
             "gpu_launches": len(launches),
             "kernel_timing": "separate pass of the same K steps with a CUDA-event pair around each launch",
             "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-            "clocks": clocks, "cpu_baseline": cpu, "decode_step": decode,
+            "clocks": clocks, "cpu_baseline": cpu, "decode_step": decode, "layer_epilogue": epilogue,
         }
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -12,7 +12,7 @@ const char *kernel_name(int id) {
   static const char *names[K_COUNT] = {
       "f32_prep",  "f32_states", "f32_scores", "f32_out",    "f32_dstates", "f32_dscores", "f32_dqk",
       "f32_dv",    "f32_dg_out", "tc_prep",    "tc_walk",    "tc_scan(unused)", "tc_bwd",  "status_clear",
-      "decode"};
+      "decode",    "epilogue_fwd", "epilogue_bwd", "epilogue_reduce"};
   if (id < 0 || id >= K_COUNT) return "unknown";
   return names[id];
 }
@@ -277,6 +277,55 @@ int gla_decode_step(const gla_desc *desc, const void *q, const void *k, const vo
     GLA_TRY(check_req(log_alpha));
   }
   return decode_step(desc, q, k, v, log_alpha, state, o, (cudaStream_t)stream);
+}
+
+namespace {
+int check_epilogue_desc(const gla_desc *d) {
+  if (!d) return GLA_ERR_INVALID_ARG;
+  if (d->B < 1 || d->H < 1 || d->T < 1 || d->dv < 1) return GLA_ERR_INVALID_ARG;
+  if (d->dtype != GLA_DTYPE_BF16 && d->dtype != GLA_DTYPE_FP32) return GLA_ERR_INVALID_ARG;
+  if (d->dv % 8 != 0 || d->dv > 1024 || (long)d->B * d->H * d->T > (1L << 40)) return GLA_ERR_UNSUPPORTED_SHAPE;
+  return GLA_OK;
+}
+int check_eps(float eps) { return (eps > 0.f && eps < 1.f) ? GLA_OK : GLA_ERR_INVALID_ARG; }
+}  // namespace
+
+size_t gla_epilogue_workspace_size(const gla_desc *desc) {
+  if (check_epilogue_desc(desc) != GLA_OK) return 0;
+  return gla::epilogue_workspace(desc);
+}
+
+int gla_epilogue_fwd(const gla_desc *desc, const void *o, const void *r, const float *w, const float *b, float eps,
+                     void *y, void *stream) {
+  GLA_TRY(check_epilogue_desc(desc));
+  GLA_TRY(check_eps(eps));
+  GLA_TRY(check_req(o));
+  GLA_TRY(check_req(r));
+  GLA_TRY(check_req(y));
+  GLA_TRY(check_opt(w));
+  GLA_TRY(check_opt(b));
+  return gla::epilogue_fwd(desc, o, r, w, b, eps, y, (cudaStream_t)stream);
+}
+
+int gla_epilogue_bwd(const gla_desc *desc, const void *o, const void *r, const float *w, const float *b, float eps,
+                     const void *dy, void *do_, void *dr, float *dw, float *db, void *stream) {
+  GLA_TRY(check_epilogue_desc(desc));
+  GLA_TRY(check_eps(eps));
+  GLA_TRY(check_req(o));
+  GLA_TRY(check_req(r));
+  GLA_TRY(check_req(dy));
+  GLA_TRY(check_req(do_));
+  GLA_TRY(check_req(dr));
+  GLA_TRY(check_opt(w));
+  GLA_TRY(check_opt(b));
+  GLA_TRY(check_opt(dw));
+  GLA_TRY(check_opt(db));
+  if (dw || db) {
+    if (!desc->workspace) return GLA_ERR_INVALID_ARG;
+    if (((uintptr_t)desc->workspace & 255u) != 0) return GLA_ERR_MISALIGNED;
+    if (desc->workspace_bytes < gla::epilogue_workspace(desc)) return GLA_ERR_WORKSPACE_TOO_SMALL;
+  }
+  return gla::epilogue_bwd(desc, o, r, w, b, eps, dy, do_, dr, dw, db, (cudaStream_t)stream);
 }
 
 int gla_selftest_timeout(void *status_word, unsigned limit_us, void *stream) {

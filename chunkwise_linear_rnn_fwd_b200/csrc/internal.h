@@ -26,6 +26,9 @@ enum KernelId : int {
   K_TC_BWD,
   K_STATUS_CLEAR,
   K_DECODE,
+  K_EPI_FWD,
+  K_EPI_BWD,
+  K_EPI_REDUCE,
   K_COUNT
 };
 
@@ -77,6 +80,13 @@ int f32_bwd(const Problem &p, const void *q, const void *k, const void *v, const
 // recurrent decode step (CUDA cores); arguments validated by the caller
 int decode_step(const gla_desc *d, const void *q, const void *k, const void *v, const float *la, float *state,
                 void *o, cudaStream_t st);
+
+// layer epilogue (CUDA cores); arguments validated by the caller
+size_t epilogue_workspace(const gla_desc *d);
+int epilogue_fwd(const gla_desc *d, const void *o, const void *r, const float *w, const float *b, float eps,
+                 void *y, cudaStream_t st);
+int epilogue_bwd(const gla_desc *d, const void *o, const void *r, const float *w, const float *b, float eps,
+                 const void *dy, void *dout, void *dr, float *dw, float *db, cudaStream_t st);
 
 }  // namespace gla
 

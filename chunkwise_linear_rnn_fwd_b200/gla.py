@@ -30,7 +30,8 @@ NOALLOC_SCRATCH_BYTES = 64 << 20  # GLA_NOALLOC_SCRATCH_BYTES in include/gla.h
 # Every exported symbol of include/gla.h.
 EXPORTS = ["gla_workspace_size", "gla_check", "gla_fwd", "gla_bwd", "gla_poll_status", "gla_status_string",
            "gla_timing_enable", "gla_timing_collect", "gla_kernel_name", "gla_build_info", "gla_fwd_noalloc",
-           "gla_decode_step", "gla_selftest_timeout"]
+           "gla_decode_step", "gla_selftest_timeout", "gla_epilogue_workspace_size", "gla_epilogue_fwd",
+           "gla_epilogue_bwd"]
 
 
 class GLAError(RuntimeError):
@@ -71,6 +72,13 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.gla_decode_step.restype = i
     lib.gla_selftest_timeout.argtypes = [vp, ctypes.c_uint, vp]
     lib.gla_selftest_timeout.restype = i
+    f = ctypes.c_float
+    lib.gla_epilogue_workspace_size.argtypes = [dp]
+    lib.gla_epilogue_workspace_size.restype = ctypes.c_size_t
+    lib.gla_epilogue_fwd.argtypes = [dp, vp, vp, vp, vp, f, vp, vp]
+    lib.gla_epilogue_fwd.restype = i
+    lib.gla_epilogue_bwd.argtypes = [dp, vp, vp, vp, vp, f, vp, vp, vp, vp, vp, vp]
+    lib.gla_epilogue_bwd.restype = i
     lib.gla_bwd.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, vp]
     lib.gla_bwd.restype = i
     lib.gla_poll_status.argtypes = [dp, vp]
@@ -214,6 +222,41 @@ def gla_decode_step(q, k, v, log_alpha, state, *, gate=None, o=None, stream=None
     if r != GLA_OK:
         raise GLAError(r, "gla_decode_step")
     return o
+
+
+def gla_epilogue_fwd(o, r, w=None, b=None, *, eps=1e-5, y=None, stream=None):
+    """y = LayerNorm(o; w, b, eps) * Swish(r) per (batch, head, token) over d_v.
+    o, r [B,H,T,d_v]; w, b [d_v] fp32 or None.  See include/gla.h."""
+    lib = load()
+    B, H, T, dv = o.shape
+    if y is None:
+        y = torch.empty_like(o)
+    d = make_desc(B, H, T, 1, dv, o.dtype, "none")
+    r_ = lib.gla_epilogue_fwd(ctypes.byref(d), _ptr(o), _ptr(r), _ptr(w), _ptr(b), float(eps), _ptr(y),
+                              _stream_handle(stream))
+    if r_ != GLA_OK:
+        raise GLAError(r_, "gla_epilogue_fwd")
+    return y
+
+
+def gla_epilogue_bwd(o, r, dy, w=None, b=None, *, eps=1e-5, want_dwb=True, workspace=None, stream=None):
+    """Backward of gla_epilogue_fwd: (do, dr, dw or None, db or None)."""
+    lib = load()
+    B, H, T, dv = o.shape
+    do_, dr = torch.empty_like(o), torch.empty_like(r)
+    dw = db = None
+    d = make_desc(B, H, T, 1, dv, o.dtype, "none")
+    if want_dwb:
+        dw = torch.empty(dv, dtype=torch.float32, device=o.device)
+        db = torch.empty(dv, dtype=torch.float32, device=o.device)
+        if workspace is None:
+            workspace = alloc_workspace(lib.gla_epilogue_workspace_size(ctypes.byref(d)), o.device)
+        d = make_desc(B, H, T, 1, dv, o.dtype, "none", workspace=workspace)
+    r_ = lib.gla_epilogue_bwd(ctypes.byref(d), _ptr(o), _ptr(r), _ptr(w), _ptr(b), float(eps), _ptr(dy), _ptr(do_),
+                              _ptr(dr), _ptr(dw), _ptr(db), _stream_handle(stream))
+    if r_ != GLA_OK:
+        raise GLAError(r_, "gla_epilogue_bwd")
+    return do_, dr, dw, db
 
 
 def gla_bwd(q, k, v, log_alpha, do, h0=None, dh_final=None, *, chunk=64, gate=None, subchunk=16, dq=None, dk=None,

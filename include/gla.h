@@ -165,6 +165,31 @@ int gla_bwd(const gla_desc *desc, const void *q, const void *k, const void *v,
 int gla_decode_step(const gla_desc *desc, const void *q, const void *k, const void *v,
                     const float *log_alpha, float *state, void *o, void *stream);
 
+/* ---- layer epilogue -------------------------------------------------------------
+ * The step after the recurrence in the GLA layer of the paper: each head's output
+ * is normalised by a LayerNorm over its d_v channels and multiplied elementwise
+ * by the Swish output gate r (Swish(x) = x sigmoid(x)) before the output
+ * projection (not part of this library):
+ *     y = (w (.) (o - mean(o)) / sqrt(var(o) + eps) + b) (.) r sigmoid(r)
+ * mean and biased variance over the d_v channels of one (batch, head, token).
+ *   o, r, y, dy, do, dr: [B,H,T,d_v], element type desc->dtype (r is the gate's
+ *   pre-activation, given in o's layout); w, b, dw, db: [d_v] fp32, one weight and
+ *   bias shared by every head (w NULL = ones, b NULL = zeros; dw / db NULL = not
+ *   computed).  d_v a multiple of 8 and <= 1024; 0 < eps < 1 (the paper's layer
+ *   uses the usual 1e-5).  desc->dk, subchunk, variant, segments and flags are
+ *   ignored.
+ * gla_epilogue_bwd returns do, dr and, when asked, dw and db; the latter are
+ * summed over all rows in a fixed order (deterministic) through per-CTA partial
+ * sums in desc->workspace (size from gla_epilogue_workspace_size, 256-byte
+ * aligned; unused when dw and db are NULL).  Both calls validate every argument
+ * before enqueuing anything, run asynchronously on `stream` and are bound by HBM
+ * bandwidth. */
+size_t gla_epilogue_workspace_size(const gla_desc *desc);
+int gla_epilogue_fwd(const gla_desc *desc, const void *o, const void *r, const float *w, const float *b,
+                     float eps, void *y, void *stream);
+int gla_epilogue_bwd(const gla_desc *desc, const void *o, const void *r, const float *w, const float *b,
+                     float eps, const void *dy, void *do_, void *dr, float *dw, float *db, void *stream);
+
 /* ---- forward without a workspace ---------------------------------------------
  * No counterpart in the paper: this entry point exists for callers that cannot
  * allocate device memory -- a program whose device memory is all owned by

@@ -136,6 +136,34 @@ def test_decode_step_validation_enqueues_nothing(lib):
     assert f(ctypes.byref(d), a, a, a, a, a, a, None) == -1                   # none gate with log_alpha
 
 
+def test_epilogue_validation_enqueues_nothing(lib):
+    """gla_epilogue_fwd / _bwd reject bad descriptors, pointers and workspaces before
+    any launch."""
+    vp = ctypes.c_void_p
+    a = vp(4096)
+    mis = vp(4096 + 4)
+    d = desc(T=10, dv=512)
+    f, b = lib.gla_epilogue_fwd, lib.gla_epilogue_bwd
+    d.dv = 12
+    assert f(ctypes.byref(d), a, a, None, None, 1e-5, a, None) == -2          # d_v not a multiple of 8
+    d.dv = 2048
+    assert f(ctypes.byref(d), a, a, None, None, 1e-5, a, None) == -2          # d_v too large
+    d.dv = 512
+    assert f(ctypes.byref(d), a, a, None, None, 0.0, a, None) == -1           # eps must be positive
+    assert f(ctypes.byref(d), None, a, None, None, 1e-5, a, None) == -1       # o NULL
+    assert f(ctypes.byref(d), a, mis, None, None, 1e-5, a, None) == -3        # r misaligned
+    assert f(ctypes.byref(d), a, a, mis, None, 1e-5, a, None) == -3          # w misaligned
+    assert b(ctypes.byref(d), a, a, None, None, 1e-5, a, a, a, a, a, None) == -1   # dw asked, no workspace
+    d.workspace = (1 << 20) + 8
+    d.workspace_bytes = 1 << 30
+    assert b(ctypes.byref(d), a, a, None, None, 1e-5, a, a, a, a, a, None) == -3   # workspace misaligned
+    d.workspace = 1 << 20
+    d.workspace_bytes = 16
+    assert b(ctypes.byref(d), a, a, None, None, 1e-5, a, a, a, a, a, None) == -4   # workspace too small
+    assert lib.gla_epilogue_workspace_size(ctypes.byref(d)) > 16
+    assert b(ctypes.byref(d), a, a, None, None, 1e-5, None, a, a, a, a, None) == -1  # dy NULL
+
+
 def test_oracle_not_imported_by_product():
     """The product package never imports, loads or links the oracle."""
     pkg_dir = os.path.join(ROOT, "chunkwise_linear_rnn_fwd_b200")
