@@ -314,12 +314,10 @@ def measure_epilogue(args, w, dev, stream, peaks, peak_src, seed=0):
     wt = torch.ones(V, device=dev)
     bs = torch.zeros(V, device=dev)
     y = torch.empty_like(o)
-    lib = pkg.load()
-    d = pkg.gla.make_desc(B, H, T, 1, V, torch.bfloat16, "none")
-    ws = pkg.alloc_workspace(lib.gla_epilogue_workspace_size(__import__("ctypes").byref(d)), dev)
+    ws = pkg.alloc_workspace(pkg.epilogue_workspace_size(B, H, T, V, torch.bfloat16), dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)  # twice the L2
     res = {}
-    for name, fn in (("fwd", lambda: pkg.gla_epilogue_fwd(o, r, wt, bs, y=y, stream=stream)),
+    for name, fn in (("fwd", lambda: pkg.gla_epilogue_fwd(o, r, wt, bs, y=y, workspace=ws, stream=stream)),
                      ("bwd", lambda: pkg.gla_epilogue_bwd(o, r, dy, wt, bs, workspace=ws, stream=stream))):
         for _ in range(max(3, args.warmup)):
             fn()
@@ -593,6 +591,9 @@ def main():
     ap.add_argument("--heads", type=int, default=None, help="override H")
     ap.add_argument("--seqlen", type=int, default=None, help="override T")
     ap.add_argument("--sweep", action="store_true", help="time every workload configuration (one JSON line)")
+    ap.add_argument("--epilogue-once", action="store_true",
+                    help="run the layer epilogue forward and backward twice on the workload's output shape and "
+                         "exit (a small case for profiler captures; prints no bench line)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -604,7 +605,32 @@ def main():
         return run_reference(args, w)
     if args.sweep:
         return run_sweep(args)
+    if args.epilogue_once:
+        return run_epilogue_once(w)
     return run_ours(args, w)
+
+
+def run_epilogue_once(w):
+    """Two forward + backward calls of the layer epilogue on [B,H,T,d_v] bf16 inputs,
+    then the device status word.  Launch order: fwd, bwd, reduce, fwd, bwd, reduce."""
+    import torch
+
+    import chunkwise_linear_rnn_fwd_b200 as pkg
+
+    dev = torch.device("cuda", 0)
+    B, H, T, V = w["B"], w["H"], w["T"], w["V"]
+    g = torch.Generator(device=dev)
+    g.manual_seed(0)
+    o, r, dy = (torch.randn(B, H, T, V, device=dev, generator=g).to(torch.bfloat16) for _ in range(3))
+    wt, bs = torch.ones(V, device=dev), torch.zeros(V, device=dev)
+    ws = pkg.alloc_workspace(pkg.epilogue_workspace_size(B, H, T, V, torch.bfloat16), dev)
+    for _ in range(2):
+        pkg.gla_epilogue_fwd(o, r, wt, bs, workspace=ws)
+        pkg.gla_epilogue_bwd(o, r, dy, wt, bs, workspace=ws)
+    torch.cuda.synchronize()
+    st = pkg.poll_status(ws)
+    print(json.dumps({"epilogue_once": {"B": B, "H": H, "T": T, "d_v": V, "status": st}}))
+    return 0 if st == 0 else 1
 
 
 if __name__ == "__main__":

@@ -10,27 +10,55 @@
 // output store; the epilogue is its own pass, bound by HBM bandwidth (read o and
 // r once, write y once; the backward reads o, r, dy and writes do, dr).
 //
-// One warp per row (batch, head, token): lane l holds the 8-element chunks
-// l, l + 32, ... of the row (d_v <= 1024, a multiple of 8) in registers, so the
-// mean and the variance are two passes over registers with warp shuffles.  The
-// gradients of w and b are reduced deterministically: every CTA writes its
-// partial sums to the caller's workspace and a second kernel adds them in order.
+// Persistent grid (SMs x resident CTAs); every warp owns the rows
+// gw, gw + nw, gw + 2 nw, ... (gw its global warp index, nw the warp count) and a
+// ring of S shared-memory stages.  Lane 0 fills a stage with one bulk copy
+// (cp.async.bulk, the TMA engine) per input row and tensor, completing on the
+// stage's mbarrier; the warp waits on it (bounded), works on the row and lane 0
+// refills the stage with the row S steps ahead, so S - 1 rows per warp are in
+// flight while one is computed.  No stage is shared between warps, so there are
+// no block-wide barriers in the row loop.  Lane l holds the 8-element chunks
+// l, l + 32, ... of a row (d_v <= 1024, a multiple of 8): the mean and the
+// variance are two passes over registers with warp shuffles, and the outputs
+// leave as coalesced 16-byte stores.  The gradients of w and b are reduced
+// deterministically: every CTA writes its partial sums to the caller's workspace
+// and a second kernel adds them in order.
 #include <cuda_bf16.h>
 
 #include "internal.h"
+#include "tc_common.cuh"
 
 namespace gla {
 namespace {
 
-constexpr int kEpiThreads = 256;        // 8 warps
-constexpr int kEpiRowsPerWarp = 8;      // backward: rows per warp (per-CTA partials of dw, db)
+constexpr int kEpiWarps = 8;
+constexpr int kEpiThreads = 32 * kEpiWarps;
+constexpr int kEpiMaxStages = 4;
+constexpr int kEpiRingBudget = 24 * 1024;  // bytes of one warp's ring (stages x tensors x row)
+constexpr long kEpiMaxGrid = 1024;         // bound on CTAs, hence on the partial sums of dw, db
+
+struct EpiArgs {
+  long rows;
+  int V, S;
+  float eps;
+  const void *o, *r, *dy;
+  const float *w, *b;
+  void *out0, *out1;  // forward: y; backward: do, dr
+  float *part;        // backward: per-CTA partial sums [grid][2][V], or null
+  unsigned *status;
+};
 
 __device__ __forceinline__ void ld8(const float *p, float *x) {
   const float4 a = __ldg(reinterpret_cast<const float4 *>(p)), b = __ldg(reinterpret_cast<const float4 *>(p) + 1);
   x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
 }
-__device__ __forceinline__ void ld8(const __nv_bfloat16 *p, float *x) {
-  const uint4 u = __ldg(reinterpret_cast<const uint4 *>(p));
+// 8 consecutive elements from shared memory (the staged row), widened to fp32
+__device__ __forceinline__ void lds8(const float *p, float *x) {
+  const float4 a = reinterpret_cast<const float4 *>(p)[0], b = reinterpret_cast<const float4 *>(p)[1];
+  x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+}
+__device__ __forceinline__ void lds8(const __nv_bfloat16 *p, float *x) {
+  const uint4 u = *reinterpret_cast<const uint4 *>(p);
   const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
@@ -60,20 +88,43 @@ __device__ __forceinline__ float warp_sum(float x) {
   return x;
 }
 
-__device__ __forceinline__ float sigmoidf_(float x) { return 1.f / (1.f + __expf(-x)); }
+// sigmoid(x).  bf16 rows: (1 + tanh(x/2)) / 2 with the one-instruction tanh
+// approximation (relative error about 2^-11, below the output's bf16 rounding);
+// fp32 rows: 1 / (1 + e^-x) with the fast exponential and divide (about 1e-6).
+__device__ __forceinline__ float tanh_approx(float x) {
+  float y;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+template <typename T>
+__device__ __forceinline__ float sigm(float x) {
+  return __fdividef(1.f, 1.f + __expf(-x));
+}
+template <>
+__device__ __forceinline__ float sigm<__nv_bfloat16>(float x) {
+  return fmaf(0.5f, tanh_approx(0.5f * x), 0.5f);
+}
+
+// Global -> shared bulk copy (no multicast) completing on an mbarrier.
+__device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   dev::smem_u32(dst)),
+               "l"(src), "r"(bytes), "r"(dev::smem_u32(bar))
+               : "memory");
+}
 
 // Row statistics: mean and 1/sqrt(var + eps) of the row held in x (NCH chunks of 8
 // per lane; chunk i of lane l is element 8 (l + 32 i) .. +8, valid if < V).
 template <int NCH>
-__device__ __forceinline__ void row_stats(const float (&x)[NCH][8], int lane, int V, float eps, float &mu,
-                                          float &rstd) {
+__device__ __forceinline__ void row_stats(const float (&x)[NCH][8], int lane, int V, float inv_v, float eps,
+                                          float &mu, float &rstd) {
   float s = 0.f;
 #pragma unroll
   for (int i = 0; i < NCH; ++i)
     if (8 * (lane + 32 * i) < V)
 #pragma unroll
       for (int e = 0; e < 8; ++e) s += x[i][e];
-  mu = warp_sum(s) / (float)V;
+  mu = warp_sum(s) * inv_v;
   float q = 0.f;
 #pragma unroll
   for (int i = 0; i < NCH; ++i)
@@ -83,153 +134,266 @@ __device__ __forceinline__ void row_stats(const float (&x)[NCH][8], int lane, in
         const float d = x[i][e] - mu;
         q += d * d;
       }
-  rstd = rsqrtf(warp_sum(q) / (float)V + eps);
+  rstd = rsqrtf(warp_sum(q) * inv_v + eps);
 }
 
-template <typename T, int NCH>
-__global__ void __launch_bounds__(kEpiThreads)
-    k_epi_fwd(long rows, int V, float eps, const T *__restrict__ o, const T *__restrict__ r,
-              const float *__restrict__ w, const float *__restrict__ b, T *__restrict__ y) {
-  const int lane = threadIdx.x & 31;
-  const long row = (long)blockIdx.x * (kEpiThreads / 32) + (threadIdx.x >> 5);
-  if (row >= rows) return;
-  // o and r of the row are requested together, before the statistics need o
-  float x[NCH][8], rr[NCH][8];
-#pragma unroll
-  for (int i = 0; i < NCH; ++i) {
-    const int c = 8 * (lane + 32 * i);
-    if (c < V) {
-      ld8(o + row * V + c, x[i]);
-      ld8(r + row * V + c, rr[i]);
-    }
-  }
-  float mu, rstd;
-  row_stats<NCH>(x, lane, V, eps, mu, rstd);
-#pragma unroll
-  for (int i = 0; i < NCH; ++i) {
-    const int c = 8 * (lane + 32 * i);
-    if (c < V) {
-      float ww[8], bb[8], out[8];
-      if (w) ld8(w + c, ww);
-      if (b) ld8(b + c, bb);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const float n = (x[i][e] - mu) * rstd * (w ? ww[e] : 1.f) + (b ? bb[e] : 0.f);
-        out[e] = n * (rr[i][e] * sigmoidf_(rr[i][e]));
-      }
-      st8(y + row * V + c, out);
-    }
-  }
-}
+// One warp's staged row stream: NT tensors, S stages of one row each.
+template <typename T, int NT>
+struct RowRing {
+  uint8_t *ring;  // [S][NT][V] elements of T
+  uint64_t *bar;  // [S]
+  const T *src[NT];
+  long gw, nw, mine;  // first row, row stride, rows of this warp
+  int S;
+  uint32_t rowb;
 
-// Backward; every warp takes kEpiRowsPerWarp consecutive rows and the CTA writes
-// its partial sums of dw (= sum dn xhat) and db (= sum dn) to part[blockIdx.x][2][V].
-template <typename T, int NCH>
-__global__ void __launch_bounds__(kEpiThreads)
-    k_epi_bwd(long rows, int V, float eps, const T *__restrict__ o, const T *__restrict__ r,
-              const float *__restrict__ w, const float *__restrict__ b, const T *__restrict__ dy,
-              T *__restrict__ dout, T *__restrict__ dr, float *__restrict__ part) {
-  extern __shared__ float spart[];  // [8 warps][2][V]
+  __device__ uint8_t *stage(int s) const { return ring + (size_t)s * NT * rowb; }
+  // lane 0 only: row j of this warp into stage s (= j mod S)
+  __device__ void issue(long j, int s) const {
+    const long row = gw + j * nw;
+    uint8_t *st = stage(s);
+    dev::mbar_arrive_expect_tx(&bar[s], NT * rowb);
+#pragma unroll
+    for (int t = 0; t < NT; ++t) bulk_g2s(st + t * rowb, src[t] + row * (rowb / sizeof(T)), rowb, &bar[s]);
+  }
+  // every lane: wait for stage s to complete phase ph; false (warp-uniform) once
+  // the wait has run out
+  __device__ bool wait(int s, uint32_t ph, unsigned *status) const {
+    const bool ok = dev::mbar_wait(&bar[s], ph, status);
+    return __all_sync(0xffffffffu, ok);
+  }
+  // lane 0, after the wait for row j (stage s, phase ph) ran out: let the copies
+  // still in flight land
+  __device__ void drain(long j, int s, uint32_t ph, unsigned *status) const {
+    const long end = j + S < mine ? j + S : mine;
+    for (long i = j; i < end; ++i) {
+      dev::mbar_wait(&bar[s], ph, status);
+      if (++s == S) s = 0, ph ^= 1u;
+    }
+  }
+};
+
+// Shared memory: the warps' rings [8][S][NT][V], then scratch_b bytes per warp,
+// then the mbarriers [8][kEpiMaxStages].
+template <typename T, int NT>
+__device__ __forceinline__ RowRing<T, NT> make_ring(const EpiArgs &a, uint8_t *smem, const T *const (&src)[NT],
+                                                    uint32_t scratch_b = 0) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  RowRing<T, NT> q;
+  q.rowb = (uint32_t)(a.V * sizeof(T));
+  q.S = a.S;
+  q.ring = smem + (size_t)warp * a.S * NT * q.rowb;
+  q.bar = reinterpret_cast<uint64_t *>(smem + (size_t)kEpiWarps * (a.S * NT * q.rowb + scratch_b)) +
+          warp * kEpiMaxStages;
+#pragma unroll
+  for (int t = 0; t < NT; ++t) q.src[t] = src[t];
+  q.nw = (long)gridDim.x * kEpiWarps;
+  q.gw = (long)blockIdx.x * kEpiWarps + warp;
+  q.mine = q.gw < a.rows ? (a.rows - 1 - q.gw) / q.nw + 1 : 0;
+  if (lane == 0) {
+    for (int s = 0; s < a.S; ++s) dev::mbar_init(&q.bar[s], 1);
+    dev::fence_mbar_init();
+  }
+  __syncwarp();
+  if (lane == 0)
+    for (int j = 0; j < q.mine && j < a.S; ++j) q.issue(j, j);
+  return q;
+}
+
+template <typename T, int NCH>
+__global__ void __launch_bounds__(kEpiThreads) k_epi_fwd(EpiArgs a) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int lane = threadIdx.x & 31;
+  const int V = a.V;
+  const T *const src[2] = {(const T *)a.o, (const T *)a.r};
+  const RowRing<T, 2> q = make_ring<T, 2>(a, smem, src);
+  T *y = (T *)a.out0;
+  float wv[NCH][8], bv[NCH][8];
+#pragma unroll
+  for (int i = 0; i < NCH; ++i) {
+    const int c = 8 * (lane + 32 * i);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) wv[i][e] = 1.f, bv[i][e] = 0.f;
+    if (c < V) {
+      if (a.w) ld8(a.w + c, wv[i]);
+      if (a.b) ld8(a.b + c, bv[i]);
+    }
+  }
+  const float inv_v = 1.f / (float)V;
+  int s = 0;
+  uint32_t ph = 0;
+  for (long j = 0; j < q.mine; ++j) {
+    if (!q.wait(s, ph, a.status)) {
+      if (lane == 0) q.drain(j, s, ph, a.status);
+      return;
+    }
+    const long row = q.gw + j * q.nw;
+    const T *so = reinterpret_cast<const T *>(q.stage(s)), *sr = so + V;
+    float x[NCH][8];
+#pragma unroll
+    for (int i = 0; i < NCH; ++i) {
+      const int c = 8 * (lane + 32 * i);
+      if (c < V) lds8(so + c, x[i]);
+    }
+    float mu, rstd;
+    row_stats<NCH>(x, lane, V, inv_v, a.eps, mu, rstd);
+#pragma unroll
+    for (int i = 0; i < NCH; ++i) {
+      const int c = 8 * (lane + 32 * i);
+      if (c < V) {
+        float rr[8], out[8];
+        lds8(sr + c, rr);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float n = (x[i][e] - mu) * rstd * wv[i][e] + bv[i][e];
+          out[e] = n * (rr[e] * sigm<T>(rr[e]));
+        }
+        st8(y + row * V + c, out);
+      }
+    }
+    __syncwarp();  // every lane has read the stage
+    if (lane == 0 && j + q.S < q.mine) {
+      dev::fence_proxy_async_smem();
+      q.issue(j + q.S, s);
+    }
+    if (++s == q.S) s = 0, ph ^= 1u;
+  }
+}
+
+// Backward.  With dn = dy r sigmoid(r) (the gradient at the LayerNorm output),
+// x^ = (o - mean) rstd and g = dn w:  do = rstd (g - mean(g) - x^ mean(g x^)),
+// dr = dy n sigmoid(r) (1 + r (1 - sigmoid(r))), dw += dn x^, db += dn.
+template <typename T, int NCH>
+__global__ void __launch_bounds__(kEpiThreads) k_epi_bwd(EpiArgs a) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int lane = threadIdx.x & 31;
+  const int V = a.V;
+  const T *const src[3] = {(const T *)a.o, (const T *)a.r, (const T *)a.dy};
+  const RowRing<T, 3> q = make_ring<T, 3>(a, smem, src, 4u * V);
+  // this warp's fp32 row of g = dn w, written in pass 1 and read in pass 2
+  float *gs = reinterpret_cast<float *>(smem + (size_t)kEpiWarps * a.S * 3 * q.rowb) + (threadIdx.x >> 5) * V;
+  T *dout = (T *)a.out0, *dr = (T *)a.out1;
   float pw[NCH][8], pb[NCH][8];
 #pragma unroll
   for (int i = 0; i < NCH; ++i)
 #pragma unroll
     for (int e = 0; e < 8; ++e) pw[i][e] = pb[i][e] = 0.f;
-  const long row0 = ((long)blockIdx.x * (kEpiThreads / 32) + warp) * kEpiRowsPerWarp;
-#pragma unroll 1
-  for (int rr_ = 0; rr_ < kEpiRowsPerWarp; ++rr_) {
-    const long row = row0 + rr_;
-    if (row >= rows) break;
+  const float inv_v = 1.f / (float)V;
+  int s = 0;
+  uint32_t ph = 0;
+  for (long j = 0; j < q.mine; ++j) {
+    if (!q.wait(s, ph, a.status)) {
+      if (lane == 0) q.drain(j, s, ph, a.status);
+      break;
+    }
+    const long row = q.gw + j * q.nw;
+    const T *so = reinterpret_cast<const T *>(q.stage(s)), *sr = so + V, *sd = so + 2 * V;
     float x[NCH][8];
 #pragma unroll
     for (int i = 0; i < NCH; ++i) {
       const int c = 8 * (lane + 32 * i);
-      if (c < V) ld8(o + row * V + c, x[i]);
+      if (c < V) lds8(so + c, x[i]);
     }
     float mu, rstd;
-    row_stats<NCH>(x, lane, V, eps, mu, rstd);
-    // dxhat = dn w with dn = dy g; keep dxhat in x's registers after xhat is formed
-    float dxh[NCH][8];
+    row_stats<NCH>(x, lane, V, inv_v, a.eps, mu, rstd);
+    // pass 1: dr, g (parked in gs), the dw / db partials and the row means of g
+    // and g x^; x is replaced by x^
     float m1 = 0.f, m2 = 0.f;
 #pragma unroll
     for (int i = 0; i < NCH; ++i) {
       const int c = 8 * (lane + 32 * i);
       if (c < V) {
-        float rv[8], gy[8], ww[8], bb[8], drv[8];
-        ld8(r + row * V + c, rv);
-        ld8(dy + row * V + c, gy);
-        if (w) ld8(w + c, ww);
-        if (b) ld8(b + c, bb);
+        float rv[8], gy[8], ww[8], bb[8], drv[8], gg[8];
+        lds8(sr + c, rv);
+        lds8(sd + c, gy);
+        if (a.w) ld8(a.w + c, ww);
+        if (a.b) ld8(a.b + c, bb);
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           const float xh = (x[i][e] - mu) * rstd;
-          const float we = w ? ww[e] : 1.f;
-          const float n = xh * we + (b ? bb[e] : 0.f);
-          const float sg = sigmoidf_(rv[e]);
+          const float we = a.w ? ww[e] : 1.f;
+          const float n = xh * we + (a.b ? bb[e] : 0.f);
+          const float sg = sigm<T>(rv[e]);
           const float dn = gy[e] * (rv[e] * sg);
           drv[e] = gy[e] * n * (sg * (1.f + rv[e] * (1.f - sg)));
           pw[i][e] += dn * xh;
           pb[i][e] += dn;
-          dxh[i][e] = dn * we;
+          gg[e] = dn * we;
+          m1 += gg[e];
+          m2 += gg[e] * xh;
           x[i][e] = xh;
-          m1 += dxh[i][e];
-          m2 += dxh[i][e] * xh;
         }
         st8(dr + row * V + c, drv);
+        st8(gs + c, gg);
       }
     }
-    m1 = warp_sum(m1) / (float)V;
-    m2 = warp_sum(m2) / (float)V;
+    m1 = warp_sum(m1) * inv_v;
+    m2 = warp_sum(m2) * inv_v;
+    // pass 2: do (each lane reads back only the g it wrote)
 #pragma unroll
     for (int i = 0; i < NCH; ++i) {
       const int c = 8 * (lane + 32 * i);
       if (c < V) {
-        float d[8];
+        float gg[8], d[8];
+        lds8(gs + c, gg);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) d[e] = rstd * (dxh[i][e] - m1 - x[i][e] * m2);
+        for (int e = 0; e < 8; ++e) d[e] = rstd * (gg[e] - m1 - x[i][e] * m2);
         st8(dout + row * V + c, d);
       }
     }
+    __syncwarp();
+    if (lane == 0 && j + q.S < q.mine) {
+      dev::fence_proxy_async_smem();
+      q.issue(j + q.S, s);
+    }
+    if (++s == q.S) s = 0, ph ^= 1u;
   }
-  if (!part) return;
+  if (!a.part) return;
+  // The CTA's partial sums: every warp parks its lanes' sums in its own ring (idle
+  // now; a ring holds 3 S d_v >= 6 d_v elements of T, at least 2 d_v floats), then
+  // the CTA adds the 8 warps in order.  A warp that gave up on a wait parks its
+  // sums too; the status word already marks the call as failed.
+  float *mine = reinterpret_cast<float *>(q.ring);
 #pragma unroll
   for (int i = 0; i < NCH; ++i) {
     const int c = 8 * (lane + 32 * i);
     if (c < V)
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
-        spart[(warp * 2) * V + c + e] = pw[i][e];
-        spart[(warp * 2 + 1) * V + c + e] = pb[i][e];
+        mine[c + e] = pw[i][e];
+        mine[V + c + e] = pb[i][e];
       }
   }
   __syncthreads();
+  const size_t ring_floats = (size_t)a.S * 3 * q.rowb / sizeof(float);
+  const float *all = reinterpret_cast<const float *>(smem);
   for (int idx = threadIdx.x; idx < 2 * V; idx += kEpiThreads) {
     float s = 0.f;
 #pragma unroll
-    for (int w8 = 0; w8 < kEpiThreads / 32; ++w8) s += spart[w8 * 2 * V + idx];
-    part[(long)blockIdx.x * 2 * V + idx] = s;
+    for (int w8 = 0; w8 < kEpiWarps; ++w8) s += all[w8 * ring_floats + idx];
+    a.part[(long)blockIdx.x * 2 * V + idx] = s;
   }
 }
 
-// dw[c] = sum over CTAs of part[cta][0][c], db[c] likewise.  A CTA of 256 threads
-// takes 32 consecutive entries of [dw | db]; warp w adds the partials w, w + 8, ...
-// of its lane's entry and the 8 warp sums are added in warp order: a fixed order,
-// so the result does not depend on scheduling.
-__global__ void __launch_bounds__(256) k_epi_reduce(int nparts, int V, const float *__restrict__ part,
-                                                    float *__restrict__ dw, float *__restrict__ db) {
-  __shared__ float sred[8][32];
+// dw[c] = sum over CTAs of part[cta][0][c], db[c] likewise.  A CTA of 1024 threads
+// owns 32 consecutive entries of the 2 d_v sums: warp w adds the partials
+// w, w + 32, ... for its lane's entry, then warp 0 adds the 32 warp sums in order.
+constexpr int kReduceWarps = 32;
+__global__ void __launch_bounds__(32 * kReduceWarps) k_epi_reduce(int nparts, int V, const float *__restrict__ part,
+                                                                  float *__restrict__ dw, float *__restrict__ db) {
+  __shared__ float sred[kReduceWarps][32];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int idx = blockIdx.x * 32 + lane;
   float s = 0.f;
   if (idx < 2 * V)
-    for (int p = warp; p < nparts; p += 8) s += part[(long)p * 2 * V + idx];
+#pragma unroll 4
+    for (int p = warp; p < nparts; p += kReduceWarps) s += part[(long)p * 2 * V + idx];
   sred[warp][lane] = s;
   __syncthreads();
   if (warp == 0 && idx < 2 * V) {
     float t = sred[0][lane];
 #pragma unroll
-    for (int w8 = 1; w8 < 8; ++w8) t += sred[w8][lane];
+    for (int w = 1; w < kReduceWarps; ++w) t += sred[w][lane];
     if (idx < V) {
       if (dw) dw[idx] = t;
     } else if (db) {
@@ -238,78 +402,112 @@ __global__ void __launch_bounds__(256) k_epi_reduce(int nparts, int V, const flo
   }
 }
 
-template <int NCH>
+// Stages per warp, dynamic shared memory and the persistent grid of a launch.
+struct EpiShape {
+  int S;
+  size_t smem;
+  unsigned grid;
+};
+
+size_t stage_bytes(const gla_desc *d, int nt) { return (size_t)nt * d->dv * (d->dtype == GLA_DTYPE_BF16 ? 2 : 4); }
+
+int stages_for(size_t per_stage) {
+  const int S = (int)(kEpiRingBudget / per_stage);
+  return S < 2 ? 2 : (S > kEpiMaxStages ? kEpiMaxStages : S);
+}
+
+template <typename Kern>
+int epi_shape(Kern kernel, const gla_desc *d, int nt, size_t scratch_b, EpiShape *sh) {
+  const long rows = (long)d->B * d->H * d->T;
+  const size_t per_stage = stage_bytes(d, nt);
+  sh->S = stages_for(per_stage);
+  sh->smem = (size_t)kEpiWarps * (sh->S * per_stage + scratch_b) + (size_t)kEpiWarps * kEpiMaxStages * sizeof(uint64_t);
+  // the attribute belongs to the current device, so it is set on every call that needs it
+  if (sh->smem > 48 * 1024 &&
+      cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sh->smem) != cudaSuccess)
+    return GLA_ERR_CUDA;
+  int dev = 0, nsm = 0, occ = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kernel, kEpiThreads, sh->smem) != cudaSuccess)
+    return GLA_ERR_CUDA;
+  if (occ < 1) return GLA_ERR_UNSUPPORTED_SHAPE;
+  long g = (rows + kEpiWarps - 1) / kEpiWarps;
+  if (g > (long)nsm * occ) g = (long)nsm * occ;
+  if (g > kEpiMaxGrid) g = kEpiMaxGrid;
+  sh->grid = (unsigned)g;
+  return GLA_OK;
+}
+
+template <typename T, int NCH>
 int epi_fwd_n(const gla_desc *d, const void *o, const void *r, const float *w, const float *b, float eps, void *y,
               cudaStream_t st) {
-  const long rows = (long)d->B * d->H * d->T;
-  const unsigned grid = (unsigned)((rows + kEpiThreads / 32 - 1) / (kEpiThreads / 32));
-  if (d->dtype == GLA_DTYPE_BF16)
-    GLA_LAUNCH(K_EPI_FWD, st,
-               (k_epi_fwd<__nv_bfloat16, NCH><<<grid, kEpiThreads, 0, st>>>(
-                   rows, d->dv, eps, (const __nv_bfloat16 *)o, (const __nv_bfloat16 *)r, w, b, (__nv_bfloat16 *)y)));
-  else
-    GLA_LAUNCH(K_EPI_FWD, st,
-               (k_epi_fwd<float, NCH><<<grid, kEpiThreads, 0, st>>>(rows, d->dv, eps, (const float *)o,
-                                                                    (const float *)r, w, b, (float *)y)));
+  EpiShape sh;
+  if (const int e = epi_shape(k_epi_fwd<T, NCH>, d, 2, 0, &sh)) return e;
+  const EpiArgs a{(long)d->B * d->H * d->T, d->dv, sh.S, eps, o, r, nullptr, w, b, y, nullptr, nullptr,
+                  (unsigned *)d->workspace};
+  GLA_LAUNCH(K_EPI_FWD, st, (k_epi_fwd<T, NCH><<<sh.grid, kEpiThreads, sh.smem, st>>>(a)));
+  return GLA_OK;
+}
+
+template <typename T, int NCH>
+int epi_bwd_n(const gla_desc *d, const void *o, const void *r, const float *w, const float *b, float eps,
+              const void *dy, void *dout, void *dr, float *dw, float *db, cudaStream_t st) {
+  EpiShape sh;
+  if (const int e = epi_shape(k_epi_bwd<T, NCH>, d, 3, (size_t)4 * d->dv, &sh)) return e;
+  float *part = (dw || db) ? (float *)((char *)d->workspace + kStatusBytes) : nullptr;
+  const EpiArgs a{(long)d->B * d->H * d->T, d->dv, sh.S, eps, o, r, dy, w, b, dout, dr, part,
+                  (unsigned *)d->workspace};
+  GLA_LAUNCH(K_EPI_BWD, st, (k_epi_bwd<T, NCH><<<sh.grid, kEpiThreads, sh.smem, st>>>(a)));
+  if (part)
+    GLA_LAUNCH(K_EPI_REDUCE, st,
+               (k_epi_reduce<<<(2 * d->dv + 31) / 32, 32 * kReduceWarps, 0, st>>>((int)sh.grid, d->dv, part, dw, db)));
   return GLA_OK;
 }
 
 template <int NCH>
-int epi_bwd_n(const gla_desc *d, const void *o, const void *r, const float *w, const float *b, float eps,
+int epi_fwd_t(const gla_desc *d, const void *o, const void *r, const float *w, const float *b, float eps, void *y,
+              cudaStream_t st) {
+  return d->dtype == GLA_DTYPE_BF16 ? epi_fwd_n<__nv_bfloat16, NCH>(d, o, r, w, b, eps, y, st)
+                                    : epi_fwd_n<float, NCH>(d, o, r, w, b, eps, y, st);
+}
+
+template <int NCH>
+int epi_bwd_t(const gla_desc *d, const void *o, const void *r, const float *w, const float *b, float eps,
               const void *dy, void *dout, void *dr, float *dw, float *db, cudaStream_t st) {
-  const long rows = (long)d->B * d->H * d->T;
-  const long per_cta = (long)(kEpiThreads / 32) * kEpiRowsPerWarp;
-  const unsigned grid = (unsigned)((rows + per_cta - 1) / per_cta);
-  float *part = (dw || db) ? (float *)d->workspace : nullptr;
-  const size_t smem = (dw || db) ? (size_t)(kEpiThreads / 32) * 2 * d->dv * sizeof(float) : 0;
-  if (smem > 48 * 1024) {  // the attribute belongs to the current device, so it is set on every such call
-    const cudaError_t e = d->dtype == GLA_DTYPE_BF16
-                              ? cudaFuncSetAttribute(k_epi_bwd<__nv_bfloat16, NCH>,
-                                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)
-                              : cudaFuncSetAttribute(k_epi_bwd<float, NCH>,
-                                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return GLA_ERR_CUDA;
-  }
-  if (d->dtype == GLA_DTYPE_BF16)
-    GLA_LAUNCH(K_EPI_BWD, st,
-               (k_epi_bwd<__nv_bfloat16, NCH><<<grid, kEpiThreads, smem, st>>>(
-                   rows, d->dv, eps, (const __nv_bfloat16 *)o, (const __nv_bfloat16 *)r, w, b,
-                   (const __nv_bfloat16 *)dy, (__nv_bfloat16 *)dout, (__nv_bfloat16 *)dr, part)));
-  else
-    GLA_LAUNCH(K_EPI_BWD, st,
-               (k_epi_bwd<float, NCH><<<grid, kEpiThreads, smem, st>>>(rows, d->dv, eps, (const float *)o,
-                                                                       (const float *)r, w, b, (const float *)dy,
-                                                                       (float *)dout, (float *)dr, part)));
-  if (part)
-    GLA_LAUNCH(K_EPI_REDUCE, st,
-               (k_epi_reduce<<<(2 * d->dv + 31) / 32, 256, 0, st>>>((int)grid, d->dv, part, dw, db)));
-  return GLA_OK;
+  return d->dtype == GLA_DTYPE_BF16 ? epi_bwd_n<__nv_bfloat16, NCH>(d, o, r, w, b, eps, dy, dout, dr, dw, db, st)
+                                    : epi_bwd_n<float, NCH>(d, o, r, w, b, eps, dy, dout, dr, dw, db, st);
 }
 
 }  // namespace
 
 size_t epilogue_workspace(const gla_desc *d) {
   const long rows = (long)d->B * d->H * d->T;
-  const long per_cta = (long)(kEpiThreads / 32) * kEpiRowsPerWarp;
-  return (size_t)((rows + per_cta - 1) / per_cta) * 2 * d->dv * sizeof(float);
+  long g = (rows + kEpiWarps - 1) / kEpiWarps;
+  if (g > kEpiMaxGrid) g = kEpiMaxGrid;
+  return kStatusBytes + (size_t)g * 2 * d->dv * sizeof(float);
 }
 
 int epilogue_fwd(const gla_desc *d, const void *o, const void *r, const float *w, const float *b, float eps,
                  void *y, cudaStream_t st) {
-  const int nch = (d->dv + 255) / 256;
-  if (nch == 1) return epi_fwd_n<1>(d, o, r, w, b, eps, y, st);
-  if (nch == 2) return epi_fwd_n<2>(d, o, r, w, b, eps, y, st);
-  if (nch == 3) return epi_fwd_n<3>(d, o, r, w, b, eps, y, st);
-  return epi_fwd_n<4>(d, o, r, w, b, eps, y, st);
+  if (cudaMemsetAsync(d->workspace, 0, kStatusBytes, st) != cudaSuccess) return GLA_ERR_CUDA;
+  switch ((d->dv + 255) / 256) {
+    case 1: return epi_fwd_t<1>(d, o, r, w, b, eps, y, st);
+    case 2: return epi_fwd_t<2>(d, o, r, w, b, eps, y, st);
+    case 3: return epi_fwd_t<3>(d, o, r, w, b, eps, y, st);
+    default: return epi_fwd_t<4>(d, o, r, w, b, eps, y, st);
+  }
 }
 
 int epilogue_bwd(const gla_desc *d, const void *o, const void *r, const float *w, const float *b, float eps,
                  const void *dy, void *dout, void *dr, float *dw, float *db, cudaStream_t st) {
-  const int nch = (d->dv + 255) / 256;
-  if (nch == 1) return epi_bwd_n<1>(d, o, r, w, b, eps, dy, dout, dr, dw, db, st);
-  if (nch == 2) return epi_bwd_n<2>(d, o, r, w, b, eps, dy, dout, dr, dw, db, st);
-  if (nch == 3) return epi_bwd_n<3>(d, o, r, w, b, eps, dy, dout, dr, dw, db, st);
-  return epi_bwd_n<4>(d, o, r, w, b, eps, dy, dout, dr, dw, db, st);
+  if (cudaMemsetAsync(d->workspace, 0, kStatusBytes, st) != cudaSuccess) return GLA_ERR_CUDA;
+  switch ((d->dv + 255) / 256) {
+    case 1: return epi_bwd_t<1>(d, o, r, w, b, eps, dy, dout, dr, dw, db, st);
+    case 2: return epi_bwd_t<2>(d, o, r, w, b, eps, dy, dout, dr, dw, db, st);
+    case 3: return epi_bwd_t<3>(d, o, r, w, b, eps, dy, dout, dr, dw, db, st);
+    default: return epi_bwd_t<4>(d, o, r, w, b, eps, dy, dout, dr, dw, db, st);
+  }
 }
 
 }  // namespace gla

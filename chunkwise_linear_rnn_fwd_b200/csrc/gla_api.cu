@@ -288,6 +288,13 @@ int check_epilogue_desc(const gla_desc *d) {
   return GLA_OK;
 }
 int check_eps(float eps) { return (eps > 0.f && eps < 1.f) ? GLA_OK : GLA_ERR_INVALID_ARG; }
+// the epilogue's workspace: the status word always, the dw / db partial sums when asked
+int check_epilogue_ws(const gla_desc *d, bool partials) {
+  if (!d->workspace) return GLA_ERR_INVALID_ARG;
+  if (((uintptr_t)d->workspace & 255u) != 0) return GLA_ERR_MISALIGNED;
+  if (d->workspace_bytes < (partials ? gla::epilogue_workspace(d) : kStatusBytes)) return GLA_ERR_WORKSPACE_TOO_SMALL;
+  return GLA_OK;
+}
 }  // namespace
 
 size_t gla_epilogue_workspace_size(const gla_desc *desc) {
@@ -304,6 +311,7 @@ int gla_epilogue_fwd(const gla_desc *desc, const void *o, const void *r, const f
   GLA_TRY(check_req(y));
   GLA_TRY(check_opt(w));
   GLA_TRY(check_opt(b));
+  GLA_TRY(check_epilogue_ws(desc, false));
   return gla::epilogue_fwd(desc, o, r, w, b, eps, y, (cudaStream_t)stream);
 }
 
@@ -320,11 +328,7 @@ int gla_epilogue_bwd(const gla_desc *desc, const void *o, const void *r, const f
   GLA_TRY(check_opt(b));
   GLA_TRY(check_opt(dw));
   GLA_TRY(check_opt(db));
-  if (dw || db) {
-    if (!desc->workspace) return GLA_ERR_INVALID_ARG;
-    if (((uintptr_t)desc->workspace & 255u) != 0) return GLA_ERR_MISALIGNED;
-    if (desc->workspace_bytes < gla::epilogue_workspace(desc)) return GLA_ERR_WORKSPACE_TOO_SMALL;
-  }
+  GLA_TRY(check_epilogue_ws(desc, dw || db));
   return gla::epilogue_bwd(desc, o, r, w, b, eps, dy, do_, dr, dw, db, (cudaStream_t)stream);
 }
 

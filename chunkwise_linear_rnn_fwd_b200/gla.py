@@ -224,14 +224,22 @@ def gla_decode_step(q, k, v, log_alpha, state, *, gate=None, o=None, stream=None
     return o
 
 
-def gla_epilogue_fwd(o, r, w=None, b=None, *, eps=1e-5, y=None, stream=None):
+def epilogue_workspace_size(B, H, T, dv, dtype) -> int:
+    """Bytes of the layer epilogue's workspace (status word + dw/db partial sums)."""
+    d = make_desc(B, H, T, 1, dv, dtype, "none")
+    return int(load().gla_epilogue_workspace_size(ctypes.byref(d)))
+
+
+def gla_epilogue_fwd(o, r, w=None, b=None, *, eps=1e-5, y=None, workspace=None, stream=None):
     """y = LayerNorm(o; w, b, eps) * Swish(r) per (batch, head, token) over d_v.
     o, r [B,H,T,d_v]; w, b [d_v] fp32 or None.  See include/gla.h."""
     lib = load()
     B, H, T, dv = o.shape
     if y is None:
         y = torch.empty_like(o)
-    d = make_desc(B, H, T, 1, dv, o.dtype, "none")
+    if workspace is None:
+        workspace = alloc_workspace(256, o.device)
+    d = make_desc(B, H, T, 1, dv, o.dtype, "none", workspace=workspace)
     r_ = lib.gla_epilogue_fwd(ctypes.byref(d), _ptr(o), _ptr(r), _ptr(w), _ptr(b), float(eps), _ptr(y),
                               _stream_handle(stream))
     if r_ != GLA_OK:
@@ -245,13 +253,12 @@ def gla_epilogue_bwd(o, r, dy, w=None, b=None, *, eps=1e-5, want_dwb=True, works
     B, H, T, dv = o.shape
     do_, dr = torch.empty_like(o), torch.empty_like(r)
     dw = db = None
-    d = make_desc(B, H, T, 1, dv, o.dtype, "none")
     if want_dwb:
         dw = torch.empty(dv, dtype=torch.float32, device=o.device)
         db = torch.empty(dv, dtype=torch.float32, device=o.device)
-        if workspace is None:
-            workspace = alloc_workspace(lib.gla_epilogue_workspace_size(ctypes.byref(d)), o.device)
-        d = make_desc(B, H, T, 1, dv, o.dtype, "none", workspace=workspace)
+    if workspace is None:
+        workspace = alloc_workspace(epilogue_workspace_size(B, H, T, dv, o.dtype) if want_dwb else 256, o.device)
+    d = make_desc(B, H, T, 1, dv, o.dtype, "none", workspace=workspace)
     r_ = lib.gla_epilogue_bwd(ctypes.byref(d), _ptr(o), _ptr(r), _ptr(w), _ptr(b), float(eps), _ptr(dy), _ptr(do_),
                               _ptr(dr), _ptr(dw), _ptr(db), _stream_handle(stream))
     if r_ != GLA_OK:

@@ -179,11 +179,16 @@ int gla_decode_step(const gla_desc *desc, const void *q, const void *k, const vo
  *   uses the usual 1e-5).  desc->dk, subchunk, variant, segments and flags are
  *   ignored.
  * gla_epilogue_bwd returns do, dr and, when asked, dw and db; the latter are
- * summed over all rows in a fixed order (deterministic) through per-CTA partial
- * sums in desc->workspace (size from gla_epilogue_workspace_size, 256-byte
- * aligned; unused when dw and db are NULL).  Both calls validate every argument
- * before enqueuing anything, run asynchronously on `stream` and are bound by HBM
- * bandwidth. */
+ * summed over all rows in a fixed order (deterministic on a given GPU model)
+ * through per-CTA partial sums in desc->workspace.
+ *   desc->workspace: 256-byte aligned, caller-owned; at least
+ *   gla_epilogue_workspace_size(desc) bytes for a backward that returns dw or db,
+ *   at least 256 bytes otherwise.  Its first 256 bytes hold the status word that
+ *   every call clears and that gla_poll_status(desc, stream) reads (a device-side
+ *   bounded wait that ran out: GLA_ERR_TIMEOUT).  Calls that share a workspace
+ *   must not overlap on the GPU.
+ * Both calls validate every argument before enqueuing anything, run
+ * asynchronously on `stream` and are bound by HBM bandwidth. */
 size_t gla_epilogue_workspace_size(const gla_desc *desc);
 int gla_epilogue_fwd(const gla_desc *desc, const void *o, const void *r, const float *w, const float *b,
                      float eps, void *y, void *stream);

@@ -138,7 +138,7 @@ def test_decode_step_validation_enqueues_nothing(lib):
 
 def test_epilogue_validation_enqueues_nothing(lib):
     """gla_epilogue_fwd / _bwd reject bad descriptors, pointers and workspaces before
-    any launch."""
+    any launch (every call below fails validation: none reaches a kernel)."""
     vp = ctypes.c_void_p
     a = vp(4096)
     mis = vp(4096 + 4)
@@ -153,6 +153,16 @@ def test_epilogue_validation_enqueues_nothing(lib):
     assert f(ctypes.byref(d), None, a, None, None, 1e-5, a, None) == -1       # o NULL
     assert f(ctypes.byref(d), a, mis, None, None, 1e-5, a, None) == -3        # r misaligned
     assert f(ctypes.byref(d), a, a, mis, None, 1e-5, a, None) == -3          # w misaligned
+    assert f(ctypes.byref(d), a, a, None, None, 1e-5, a, None) == -1         # no workspace (status word)
+    d.workspace = (1 << 20) + 8
+    d.workspace_bytes = 1 << 30
+    assert f(ctypes.byref(d), a, a, None, None, 1e-5, a, None) == -3         # workspace misaligned
+    d.workspace = 1 << 20
+    d.workspace_bytes = 255
+    assert f(ctypes.byref(d), a, a, None, None, 1e-5, a, None) == -4         # smaller than the status word
+    assert b(ctypes.byref(d), a, a, None, None, 1e-5, a, a, a, None, None, None) == -4  # same, without dw/db
+    d.workspace = None
+    d.workspace_bytes = 0
     assert b(ctypes.byref(d), a, a, None, None, 1e-5, a, a, a, a, a, None) == -1   # dw asked, no workspace
     d.workspace = (1 << 20) + 8
     d.workspace_bytes = 1 << 30
@@ -161,6 +171,10 @@ def test_epilogue_validation_enqueues_nothing(lib):
     d.workspace_bytes = 16
     assert b(ctypes.byref(d), a, a, None, None, 1e-5, a, a, a, a, a, None) == -4   # workspace too small
     assert lib.gla_epilogue_workspace_size(ctypes.byref(d)) > 16
+    # status word + per-CTA partial sums of dw, db (at most 1024 CTAs of 8 rows)
+    assert lib.gla_epilogue_workspace_size(ctypes.byref(d)) == 256 + 10 * 2 * 512 * 4  # 80 rows, 10 CTAs
+    big = desc(T=1 << 20, dv=512)
+    assert lib.gla_epilogue_workspace_size(ctypes.byref(big)) == 256 + 1024 * 2 * 512 * 4
     assert b(ctypes.byref(d), a, a, None, None, 1e-5, None, a, a, a, a, None) == -1  # dy NULL
 
 

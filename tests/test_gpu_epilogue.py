@@ -66,3 +66,27 @@ def test_epilogue_backward_is_deterministic_and_optional():
     assert torch.equal(a[2], c[2]) and torch.equal(a[3], c[3])
     assert n[2] is None and n[3] is None
     assert torch.equal(a[0], n[0]) and torch.equal(a[1], n[1])
+
+
+@pytest.mark.parametrize("B,H,T,V,dtype", [(2, 4, 4096, 512, torch.bfloat16), (1, 4, 1000, 1024, torch.float32)])
+def test_epilogue_full_size_and_status(B, H, T, V, dtype):
+    """Every row at the layer's full output shape (bf16: 32768 rows, about 14 per warp,
+    so each warp's ring of staged rows wraps several times; fp32 at d_v = 1024: two
+    stages per warp), then a clean device status word."""
+    import chunkwise_linear_rnn_fwd_b200 as pkg
+    from oracle import epilogue
+    o, r, dy, w, b = _inputs(B, H, T, V, dtype, seed=7, affine=True)
+    dev = torch.device("cuda")
+    ws = pkg.alloc_workspace(pkg.epilogue_workspace_size(B, H, T, V, dtype), dev)
+    od, rd, dyd, wd, bd = (t.to(dev) for t in (o, r, dy, w, b))
+    y = pkg.gla_epilogue_fwd(od, rd, wd, bd, workspace=ws)
+    assert pkg.poll_status(ws) == 0
+    do_, dr, dw, db = pkg.gla_epilogue_bwd(od, rd, dyd, wd, bd, workspace=ws)
+    assert pkg.poll_status(ws) == 0
+    ry = epilogue.fwd(_np(o), _np(r), _np(w), _np(b))
+    rdo, rdr, rdw, rdb = epilogue.bwd(_np(o), _np(r), _np(dy), _np(w), _np(b))
+    errs = {"y": rel_err(_np(y), ry), "do": rel_err(_np(do_), rdo), "dr": rel_err(_np(dr), rdr),
+            "dw": rel_err(_np(dw), rdw), "db": rel_err(_np(db), rdb)}
+    print("epilogue full size", dtype, (B, H, T, V), {k: f"{v:.2e}" for k, v in errs.items()})
+    assert all(errs[k] <= TOL[dtype] for k in ("y", "do", "dr")), errs
+    assert errs["dw"] <= 5e-3 and errs["db"] <= 5e-3, errs
