@@ -48,8 +48,8 @@ def algorithmic_bytes(B, H, T, K, V, gate="vector"):
 # DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) measured by ncu on
 # the full-size workload, with the sha256 of the kernel sources it was measured on.  It is
 # reported only while the sources are unchanged (a changed kernel has unknown traffic).
-NCU_TRAFFIC = {"src_sha256": "373c1ff00950a7edc477e7959139d2348eeb5172f7d23eb6018db77d77ace777",
-               "per_launch_bytes": {"tc_walk": 117732032, "tc_bwd": 447953920, "tc_prep": 72997376}}
+NCU_TRAFFIC = {"src_sha256": "a475d8b4339b1eca5edf7f74ffd7dc56410fa7ea74928e5ee3938a59580546fa",
+               "per_launch_bytes": {"tc_walk": 117666176, "tc_bwd": 449001216, "tc_prep": 73192704}}
 
 
 def kernel_src_sha256():
@@ -347,6 +347,70 @@ def measure_epilogue(args, w, dev, stream, peaks, peak_src, seed=0):
     return res
 
 
+def measure_seqpar(args, w, dev, stream, seed=0, pieces=8):
+    """Sequence parallelism's cost per rank when the bench workload is one piece of a
+    sequence split over `pieces` ranks: a piece's whole training step (summaries,
+    folds over the gathered summaries of the other pieces -- the worst-placed rank
+    folds pieces - 1 -- and the reruns, one workspace, seqpar.LibraryOps) against the
+    plain step on the same inputs, both timed with events around `steps` steps.  The
+    all-gather itself needs several GPUs and is reported in bytes."""
+    import torch
+
+    import chunkwise_linear_rnn_fwd_b200 as pkg
+    from chunkwise_linear_rnn_fwd_b200 import seqpar
+    from chunkwise_linear_rnn_fwd_b200.synth import make_inputs
+
+    B, H, T, K, V = w["B"], w["H"], w["T"], w["K"], w["V"]
+    x = make_inputs(B, H, T, K, V, dtype=torch.bfloat16, gate=w["gate"], seed=seed, z_mean=w["z_mean"])
+    q, k, v, la, do = (t.to(dev) for t in (x.q, x.k, x.v, x.log_alpha, x.do))
+    g = torch.Generator(device=dev)
+    g.manual_seed(seed)
+    gammas = torch.rand(pieces, B, H, K, device=dev, generator=g)
+    deltas = torch.randn(pieces, B, H, K, V, device=dev, generator=g)
+    ops = seqpar.LibraryOps(w["C"], stream)
+    ws = pkg.alloc_workspace(pkg.workspace_size(B, H, T, K, V, torch.bfloat16, w["gate"], w["C"], True,
+                                                flags=pkg.FLAG_SAVE_STATES), dev)
+
+    def sp_step():
+        ops.fwd_state(q, k, v, la, None)
+        h_in = ops.state_scan(gammas, deltas, pieces - 1, False)
+        ops.fwd(q, k, v, la, h_in)
+        ops.bwd_state(q, k, la, do, None)
+        dh_out = ops.state_scan(gammas, deltas, 0, True)
+        ops.bwd(q, k, v, la, do, h_in, dh_out)
+
+    def plain_step():
+        pkg.gla_fwd(q, k, v, la, None, chunk=w["C"], workspace=ws, stream=stream, save_states=True)
+        pkg.gla_bwd(q, k, v, la, do, None, None, chunk=w["C"], workspace=ws, stream=stream, reuse_prep=True,
+                    saved_states=True)
+
+    res = {}
+    for name, fn in (("plain_step", plain_step), ("sp_step", sp_step)):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        n = max(5, min(args.steps, 20))
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(n):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        res[name + "_ms"] = e0.elapsed_time(e1) / n
+    pkg.timing_enable(True)
+    pkg.timing_collect()
+    sp_step()
+    torch.cuda.synchronize()
+    per = {}
+    for kname, kms in pkg.timing_collect():
+        per[kname] = per.get(kname, 0.0) + kms
+    pkg.timing_enable(False)
+    return {"workload": f"one piece of {pieces}: B={B} H={H} T={T} d_k={K} d_v={V} bf16, {w['gate']} gates",
+            **res, "overhead": res["sp_step_ms"] / res["plain_step_ms"] - 1.0,
+            "sp_step_kernels_ms": per,
+            "allgather_bytes_per_rank_per_direction": (B * H * K * V + B * H * K) * 4}
+
+
 def run_ours(args, w):
     import torch
     import torch.distributed as dist
@@ -480,6 +544,7 @@ def run_ours(args, w):
 
     decode = measure_decode(args, dev, stream, peaks, peak_src, seed=rank)
     epilogue = measure_epilogue(args, w, dev, stream, peaks, peak_src, seed=rank)
+    seqpar = measure_seqpar(args, w, dev, stream, seed=rank)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -499,6 +564,7 @@ def run_ours(args, w):
             "kernel_timing": "separate pass of the same K steps with a CUDA-event pair around each launch",
             "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "clocks": clocks, "cpu_baseline": cpu, "decode_step": decode, "layer_epilogue": epilogue,
+            "sequence_parallel": seqpar,
         }
         print(json.dumps(line), flush=True)
     if world > 1:

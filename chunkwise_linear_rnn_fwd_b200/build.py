@@ -8,7 +8,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libgla_b200.so")
-SOURCES = ["gla_api.cu", "f32_path.cu", "tc_path.cu", "gla_noalloc.cu", "decode.cu", "epilogue.cu"]
+SOURCES = ["gla_api.cu", "f32_path.cu", "tc_path.cu", "gla_noalloc.cu", "decode.cu", "epilogue.cu", "seqpar.cu"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
 

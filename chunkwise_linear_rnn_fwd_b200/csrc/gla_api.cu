@@ -12,7 +12,7 @@ const char *kernel_name(int id) {
   static const char *names[K_COUNT] = {
       "f32_prep",  "f32_states", "f32_scores", "f32_out",    "f32_dstates", "f32_dscores", "f32_dqk",
       "f32_dv",    "f32_dg_out", "tc_prep",    "tc_walk",    "tc_scan(unused)", "tc_bwd",  "status_clear",
-      "decode",    "epilogue_fwd", "epilogue_bwd", "epilogue_reduce"};
+      "decode",    "epilogue_fwd", "epilogue_bwd", "epilogue_reduce", "state_scan", "fold_segments"};
   if (id < 0 || id >= K_COUNT) return "unknown";
   return names[id];
 }
@@ -73,7 +73,7 @@ int make_problem(const gla_desc *d, int chunk, Problem *p) {
   if (d->variant != GLA_VARIANT_AUTO && d->variant != GLA_VARIANT_FUSED && d->variant != GLA_VARIANT_MATERIALIZED)
     return GLA_ERR_INVALID_ARG;
   if (d->segments < 0) return GLA_ERR_INVALID_ARG;
-  if (d->flags & ~(GLA_FLAG_REUSE_PREP | GLA_FLAG_SAVE_STATES)) return GLA_ERR_INVALID_ARG;
+  if (d->flags & ~(GLA_FLAG_REUSE_PREP | GLA_FLAG_SAVE_STATES | GLA_FLAG_REUSE_SEGMENTS)) return GLA_ERR_INVALID_ARG;
   const int sub = d->subchunk == 0 ? 16 : d->subchunk;
   if (chunk != 16 && chunk != 32 && chunk != 64 && chunk != 128) return GLA_ERR_UNSUPPORTED_SHAPE;
   if (sub < 1 || chunk % sub != 0) return GLA_ERR_UNSUPPORTED_SHAPE;
@@ -202,6 +202,58 @@ int gla_bwd(const gla_desc *desc, const void *q, const void *k, const void *v, c
   if (p.dtype == GLA_DTYPE_BF16)
     return tc_bwd(p, q, k, v, log_alpha, h0, do_, dh_final, dq, dk, dv, dlog_alpha, dh0, desc->workspace, st);
   return f32_bwd(p, q, k, v, log_alpha, h0, do_, dh_final, dq, dk, dv, dlog_alpha, dh0, desc->workspace, st);
+}
+
+int gla_fwd_state(const gla_desc *desc, const void *q, const void *k, const void *v, const float *log_alpha,
+                  const float *h0, float *delta, float *gamma, int chunk, void *stream) {
+  Problem p;
+  GLA_TRY(make_problem(desc, chunk, &p));
+  if (p.dtype != GLA_DTYPE_BF16) return GLA_ERR_UNSUPPORTED_SHAPE;
+  GLA_TRY(check_req(q));
+  GLA_TRY(check_req(k));
+  GLA_TRY(check_req(v));
+  GLA_TRY(check_gate_ptr(p, log_alpha));
+  GLA_TRY(check_opt(h0));
+  GLA_TRY(check_req(delta));
+  GLA_TRY(check_req(gamma));
+  GLA_TRY(check_ws(desc, p, false));
+  cudaStream_t st = (cudaStream_t)stream;
+  GLA_TRY(clear_status(desc, st));
+  return tc_fwd_state(p, q, k, v, log_alpha, h0, delta, gamma, desc->workspace, st);
+}
+
+int gla_bwd_state(const gla_desc *desc, const void *q, const void *k, const float *log_alpha, const void *do_,
+                  const float *dh_final, float *ddelta, float *gamma, int chunk, void *stream) {
+  Problem p;
+  GLA_TRY(make_problem(desc, chunk, &p));
+  if (p.dtype != GLA_DTYPE_BF16) return GLA_ERR_UNSUPPORTED_SHAPE;
+  GLA_TRY(check_req(q));
+  GLA_TRY(check_req(k));
+  GLA_TRY(check_gate_ptr(p, log_alpha));
+  GLA_TRY(check_req(do_));
+  GLA_TRY(check_opt(dh_final));
+  GLA_TRY(check_req(ddelta));
+  GLA_TRY(check_opt(gamma));
+  GLA_TRY(check_ws(desc, p, true));
+  cudaStream_t st = (cudaStream_t)stream;
+  GLA_TRY(clear_status(desc, st));
+  return tc_bwd_state(p, q, k, log_alpha, do_, dh_final, ddelta, gamma, desc->workspace, st);
+}
+
+int gla_state_scan(const gla_desc *desc, int nseg, int seg, int reverse, const float *gammas, const float *deltas,
+                   const float *init, float *out, void *stream) {
+  if (!desc || desc->B < 1 || desc->H < 1 || desc->dk < 1 || desc->dv < 1) return GLA_ERR_INVALID_ARG;
+  if (desc->dv % 4 != 0) return GLA_ERR_UNSUPPORTED_SHAPE;
+  if (nseg < 1 || seg < 0 || seg >= nseg || (reverse != 0 && reverse != 1)) return GLA_ERR_INVALID_ARG;
+  const bool empty = reverse ? seg == nseg - 1 : seg == 0;  // no piece to fold: out = init
+  if (!empty) {
+    GLA_TRY(check_req(gammas));
+    GLA_TRY(check_req(deltas));
+  }
+  GLA_TRY(check_opt(init));
+  GLA_TRY(check_req(out));
+  return gla::state_scan((long)desc->B * desc->H, desc->dk, desc->dv, nseg, seg, reverse, gammas, deltas, init, out,
+                         (cudaStream_t)stream);
 }
 
 int gla_poll_status(const gla_desc *desc, void *stream) {

@@ -29,6 +29,8 @@ enum KernelId : int {
   K_EPI_FWD,
   K_EPI_BWD,
   K_EPI_REDUCE,
+  K_STATE_SCAN,
+  K_FOLD_SEGMENTS,
   K_COUNT
 };
 
@@ -83,6 +85,11 @@ int decode_step(const gla_desc *d, const void *q, const void *k, const void *v, 
 
 // layer epilogue (CUDA cores); arguments validated by the caller
 size_t epilogue_workspace(const gla_desc *d);
+// sequence parallelism (seqpar.cu)
+int fold_segments(long BH, int K, int V, int P, int reverse, const float *gseg, const float *delta, const float *h0,
+                  float *out, float *gamma, cudaStream_t st);
+int state_scan(long BH, int K, int V, int nseg, int seg, int reverse, const float *gammas, const float *deltas,
+               const float *init, float *out, cudaStream_t st);
 int epilogue_fwd(const gla_desc *d, const void *o, const void *r, const float *w, const float *b, float eps,
                  void *y, cudaStream_t st);
 int epilogue_bwd(const gla_desc *d, const void *o, const void *r, const float *w, const float *b, float eps,

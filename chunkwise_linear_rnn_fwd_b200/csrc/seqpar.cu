@@ -1,0 +1,116 @@
+// seqpar.cu -- the two small kernels of sequence (context) parallelism.
+//
+// "Gated Linear Attention Transformers with Hardware-Efficient Training",
+// section 3.3 / 4.2: the chunk-level recurrence S_n = diag(gamma_n) S_{n-1} + dS_n
+// is a composition of affine maps, so a sequence split into consecutive pieces
+// (one per GPU) needs, per piece, only its summary: the gate product
+// gamma = prod_t alpha_t (per key channel) and the state it produces from zero.
+// The state entering piece r is the fold of the summaries of pieces 0 .. r-1 over
+// the initial state; in the backward, the state adjoint leaving piece r is the
+// fold of the reverse summaries of pieces r+1 .. P-1.
+//
+//   k_fold_segments  a piece's summary from the walk's segment contributions: the
+//                    zero-state pre-pass runs every segment of the piece in parallel
+//                    (contributions delta_p in the walk's float4-column layout, gate
+//                    products gseg_p); out = fold over p of S <- diag(gseg_p) S + delta_p
+//                    from h0 (dh_final in reverse), gamma = prod_p gseg_p
+//   k_state_scan     out = fold over the selected pieces of S <- diag(gamma_s) S + D_s
+//                    (elementwise per (bh, c, v), HBM-bound: one read of every D_s)
+#include "internal.h"
+
+namespace gla {
+namespace {
+
+// Thread (bh, v4, c), c fastest: the float4-column contributions
+// delta[bh][p][v4][c] are read coalesced; out[bh][c][4 v4 .. 4 v4 + 3].
+__global__ void __launch_bounds__(256) k_fold_segments(long BH, int K, int V, int P, int reverse,
+                                                       const float *__restrict__ gseg,
+                                                       const float4 *__restrict__ delta,
+                                                       const float *__restrict__ h0, float *__restrict__ out,
+                                                       float *__restrict__ gamma) {
+  const int V4 = V / 4;
+  const long i = (long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= BH * V4 * K) return;
+  const int c = (int)(i % K);
+  const int v4 = (int)((i / K) % V4);
+  const long bh = i / ((long)K * V4);
+  const long o = (bh * K + c) * (long)V + 4 * v4;
+  float4 S = h0 ? __ldg(reinterpret_cast<const float4 *>(h0 + o)) : make_float4(0.f, 0.f, 0.f, 0.f);
+  float gp = 1.f;
+  for (int j0 = 0; j0 < P; j0 += 4) {  // the loads of four segments in flight together
+    float g[4];
+    float4 d[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int j = j0 + u, p = reverse ? P - 1 - j : j;
+      g[u] = j < P ? __ldg(gseg + (bh * P + p) * K + c) : 1.f;
+      d[u] = j < P ? __ldg(delta + ((bh * P + p) * V4 + v4) * K + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      S.x = g[u] * S.x + d[u].x;
+      S.y = g[u] * S.y + d[u].y;
+      S.z = g[u] * S.z + d[u].z;
+      S.w = g[u] * S.w + d[u].w;
+      gp *= g[u];
+    }
+  }
+  *reinterpret_cast<float4 *>(out + o) = S;
+  if (gamma && v4 == 0) gamma[bh * K + c] = gp;
+}
+
+// Pieces s in [s_lo, s_hi), ascending (forward) or descending (reverse).
+__global__ void __launch_bounds__(256) k_state_scan(long BH, int K, int V, int s_lo, int s_hi, int reverse,
+                                                    const float *__restrict__ gammas,
+                                                    const float4 *__restrict__ deltas,
+                                                    const float4 *__restrict__ init, float4 *__restrict__ out) {
+  const long n4 = BH * K * (V / 4);
+  const long i = (long)blockIdx.x * blockDim.x + threadIdx.x;  // float4 index in [BH][K][V/4]
+  if (i >= n4) return;
+  const long row = i / (V / 4);  // bh * K + c
+  float4 S = init ? __ldg(init + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+  const int cnt = s_hi - s_lo;
+  for (int j0 = 0; j0 < cnt; j0 += 4) {  // the loads of four pieces in flight together
+    float g[4];
+    float4 d[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int j = j0 + u, s = reverse ? s_hi - 1 - j : s_lo + j;
+      g[u] = j < cnt ? __ldg(gammas + (long)s * BH * K + row) : 1.f;
+      d[u] = j < cnt ? __ldg(deltas + (long)s * n4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      S.x = g[u] * S.x + d[u].x;
+      S.y = g[u] * S.y + d[u].y;
+      S.z = g[u] * S.z + d[u].z;
+      S.w = g[u] * S.w + d[u].w;
+    }
+  }
+  out[i] = S;
+}
+
+}  // namespace
+
+int fold_segments(long BH, int K, int V, int P, int reverse, const float *gseg, const float *delta, const float *h0,
+                  float *out, float *gamma, cudaStream_t st) {
+  const long n = BH * (V / 4) * K;
+  GLA_LAUNCH(K_FOLD_SEGMENTS, st,
+             (k_fold_segments<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(BH, K, V, P, reverse, gseg,
+                                                                          (const float4 *)delta, h0, out, gamma)));
+  return GLA_OK;
+}
+
+int state_scan(long BH, int K, int V, int nseg, int seg, int reverse, const float *gammas, const float *deltas,
+               const float *init, float *out, cudaStream_t st) {
+  const int s_lo = reverse ? seg + 1 : 0;
+  const int s_hi = reverse ? nseg : seg;
+  const long n4 = BH * K * (V / 4);
+  GLA_LAUNCH(K_STATE_SCAN, st,
+             (k_state_scan<<<(unsigned)((n4 + 255) / 256), 256, 0, st>>>(
+                 BH, K, V, s_lo, s_hi, reverse, gammas, (const float4 *)deltas, (const float4 *)init,
+                 (float4 *)out)));
+  return GLA_OK;
+}
+
+}  // namespace gla

@@ -254,7 +254,7 @@ int tc_fwd(const Problem &p, const void *q, const void *k, const void *v, const 
   const bool save = (p.flags & GLA_FLAG_SAVE_STATES) != 0;
   TcWs w = carve(p, ws, save);
   unsigned *status = (unsigned *)ws;
-  TRY(launch_prep_any(p, (const bf16 *)q, (const bf16 *)k, la, w, status, st));
+  if (!(p.flags & GLA_FLAG_REUSE_PREP)) TRY(launch_prep_any(p, (const bf16 *)q, (const bf16 *)k, la, w, status, st));
 
   const int BV = bv_of(p);
   const int nvt = p.V / BV;
@@ -308,14 +308,17 @@ int tc_fwd(const Problem &p, const void *q, const void *k, const void *v, const 
     a.h0 = h0;
     return launch_walk_any(p, a, m, 1, st);
   }
-  // pre-pass: the contribution of segments 0 .. P-2 from a zero state
-  tc::WalkArgs pre = a;
-  pre.do_out = 0;
-  pre.state_mode = 0;
-  pre.end = w.delta;
-  pre.end_seg = -1;
-  pre.gseg = w.gseg;
-  TRY(launch_walk_any(p, pre, m, P - 1, st));
+  // pre-pass: the contribution of segments 0 .. P-2 from a zero state (already in
+  // the workspace after gla_fwd_state with GLA_FLAG_REUSE_SEGMENTS)
+  if (!(p.flags & GLA_FLAG_REUSE_SEGMENTS)) {
+    tc::WalkArgs pre = a;
+    pre.do_out = 0;
+    pre.state_mode = 0;
+    pre.end = w.delta;
+    pre.end_seg = -1;
+    pre.gseg = w.gseg;
+    TRY(launch_walk_any(p, pre, m, P - 1, st));
+  }
   a.delta = w.delta;
   a.gseg_in = w.gseg;
   a.h0 = h0;
@@ -385,12 +388,14 @@ int tc_bwd(const Problem &p, const void *q, const void *k, const void *v, const 
   r.end = dh0;
   r.end_seg = 0;
   if (P > 1) {
-    tc::WalkArgs pre = r;  // segments 1 .. P-1, backward
-    pre.end = w.ddelta;
-    pre.end_seg = -1;
-    pre.seg0 = 1;
-    pre.gseg = w.gseg;
-    TRY(launch_walk_any(p, pre, mr, P - 1, st));
+    if (!(p.flags & GLA_FLAG_REUSE_SEGMENTS)) {  // else gla_bwd_state left them in the workspace
+      tc::WalkArgs pre = r;  // segments 1 .. P-1, backward
+      pre.end = w.ddelta;
+      pre.end_seg = -1;
+      pre.seg0 = 1;
+      pre.gseg = w.gseg;
+      TRY(launch_walk_any(p, pre, mr, P - 1, st));
+    }
     r.delta = w.ddelta;
     r.gseg_in = w.gseg;
   }
@@ -405,6 +410,92 @@ int tc_bwd(const Problem &p, const void *q, const void *k, const void *v, const 
   // ---- per-chunk gradients --------------------------------------------------------
   return tc::launch_bwd_main(p, (const bf16 *)q, (const bf16 *)k, (const bf16 *)v, la, (const bf16 *)dout,
                              (bf16 *)dq, (bf16 *)dk, dla, w.gam, w.hb, w.dhb, status, st);
+}
+
+
+// ---- sequence summaries (sequence parallelism) ----------------------------------
+// Forward: the state after the whole sequence from h0 (zero if null), delta
+// [BH][K][V], and the product of its gates, gamma [BH][K].  The walk runs without
+// outputs over every segment in parallel from a zero state (the contributions stay
+// in the workspace where gla_fwd with GLA_FLAG_REUSE_SEGMENTS finds them), then
+// fold_segments composes them over h0.  Workspace layout and segment count are those
+// of gla_fwd with the same flags (GLA_FLAG_SAVE_STATES: the backward layout).
+int tc_fwd_state(const Problem &p, const void *q, const void *k, const void *v, const float *la, const float *h0,
+                 float *delta, float *gamma, void *ws, cudaStream_t st) {
+  if (device_ok() != 1) return GLA_ERR_NO_DEVICE;
+  const bool save = (p.flags & GLA_FLAG_SAVE_STATES) != 0;
+  Problem pf = p;
+  pf.variant = GLA_VARIANT_FUSED;
+  TcWs w = carve(pf, ws, save);
+  unsigned *status = (unsigned *)ws;
+  if (!(p.flags & GLA_FLAG_REUSE_PREP)) TRY(launch_prep_any(pf, (const bf16 *)q, (const bf16 *)k, la, w, status, st));
+  const int nvt = p.V / bv_of(p);
+  const int P = save ? bwd_segments(pf, nvt) : segments_of(pf, nvt);
+  const uint64_t BH = (uint64_t)p.BH;
+  WalkMaps m;
+  if (!(map3(&m.X, w.kg, p.K, p.Tp, BH, 64, 64) && map3(&m.Y, v, p.V, p.T, BH, 64, 64))) return GLA_ERR_CUDA;
+  m.Q = m.X;
+  m.P = m.X;
+  tc::WalkArgs a{};
+  a.T = p.T;
+  a.N = p.N;
+  a.V = p.V;
+  a.L = (p.N + P - 1) / P;
+  a.P = P;
+  a.gam = w.gam;
+  a.status = status;
+  if (P == 1) {  // one walk from h0 straight into delta; its gate product is gamma
+    a.h0 = h0;
+    a.end = delta;
+    a.end_seg = 0;
+    a.gseg = gamma;
+    return launch_walk_any(pf, a, m, 1, st);
+  }
+  a.end = w.delta;
+  a.end_seg = -1;
+  a.gseg = w.gseg;
+  TRY(launch_walk_any(pf, a, m, P, st));
+  return fold_segments(p.BH, p.K, p.V, P, 0, w.gseg, w.delta, h0, delta, gamma, st);
+}
+
+// Reverse: the state adjoint before the first token from dh_final (zero if null),
+// ddelta [BH][K][V] (what gla_bwd returns as dh0), and gamma as above (if not null).
+// The reverse walk over qg and dO without dv, every segment from zero (left in the
+// workspace for gla_bwd with GLA_FLAG_REUSE_SEGMENTS), folded over dh_final.
+int tc_bwd_state(const Problem &p, const void *q, const void *k, const float *la, const void *dout,
+                 const float *dhT, float *ddelta, float *gamma, void *ws, cudaStream_t st) {
+  if (device_ok() != 1) return GLA_ERR_NO_DEVICE;
+  TcWs w = carve(p, ws, true);
+  unsigned *status = (unsigned *)ws;
+  if (!(p.flags & GLA_FLAG_REUSE_PREP)) TRY(launch_prep_any(p, (const bf16 *)q, (const bf16 *)k, la, w, status, st));
+  const int nvt = p.V / bv_of(p);
+  const int P = bwd_segments(p, nvt);
+  const uint64_t BH = (uint64_t)p.BH;
+  WalkMaps m;
+  if (!(map3(&m.X, w.qg, p.K, p.Tp, BH, 64, 64) && map3(&m.Y, dout, p.V, p.T, BH, 64, 64))) return GLA_ERR_CUDA;
+  m.Q = m.X;
+  m.P = m.X;
+  tc::WalkArgs r{};
+  r.T = p.T;
+  r.N = p.N;
+  r.V = p.V;
+  r.L = (p.N + P - 1) / P;
+  r.P = P;
+  r.reverse = 1;
+  r.gam = w.gam;
+  r.status = status;
+  if (P == 1) {
+    r.h0 = dhT;
+    r.end = ddelta;
+    r.end_seg = 0;
+    r.gseg = gamma;
+    return launch_walk_any(p, r, m, 1, st);
+  }
+  r.end = w.ddelta;
+  r.end_seg = -1;
+  r.gseg = w.gseg;
+  TRY(launch_walk_any(p, r, m, P, st));
+  return fold_segments(p.BH, p.K, p.V, P, 1, w.gseg, w.ddelta, dhT, ddelta, gamma, st);
 }
 
 }  // namespace gla

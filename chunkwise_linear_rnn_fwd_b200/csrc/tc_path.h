@@ -11,4 +11,8 @@ int tc_fwd(const Problem &p, const void *q, const void *k, const void *v, const 
 int tc_bwd(const Problem &p, const void *q, const void *k, const void *v, const float *la, const float *h0,
            const void *dout, const float *dhT, void *dq, void *dk, void *dv, float *dla, float *dh0, void *ws,
            cudaStream_t st);
+int tc_fwd_state(const Problem &p, const void *q, const void *k, const void *v, const float *la, const float *h0,
+                 float *delta, float *gamma, void *ws, cudaStream_t st);
+int tc_bwd_state(const Problem &p, const void *q, const void *k, const float *la, const void *dout,
+                 const float *dhT, float *ddelta, float *gamma, void *ws, cudaStream_t st);
 }  // namespace gla

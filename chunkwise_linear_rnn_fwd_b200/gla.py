@@ -31,7 +31,7 @@ NOALLOC_SCRATCH_BYTES = 64 << 20  # GLA_NOALLOC_SCRATCH_BYTES in include/gla.h
 EXPORTS = ["gla_workspace_size", "gla_check", "gla_fwd", "gla_bwd", "gla_poll_status", "gla_status_string",
            "gla_timing_enable", "gla_timing_collect", "gla_kernel_name", "gla_build_info", "gla_fwd_noalloc",
            "gla_decode_step", "gla_selftest_timeout", "gla_epilogue_workspace_size", "gla_epilogue_fwd",
-           "gla_epilogue_bwd"]
+           "gla_epilogue_bwd", "gla_fwd_state", "gla_bwd_state", "gla_state_scan"]
 
 
 class GLAError(RuntimeError):
@@ -79,6 +79,12 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.gla_epilogue_fwd.restype = i
     lib.gla_epilogue_bwd.argtypes = [dp, vp, vp, vp, vp, f, vp, vp, vp, vp, vp, vp]
     lib.gla_epilogue_bwd.restype = i
+    lib.gla_fwd_state.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, i, vp]
+    lib.gla_fwd_state.restype = i
+    lib.gla_bwd_state.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, i, vp]
+    lib.gla_bwd_state.restype = i
+    lib.gla_state_scan.argtypes = [dp, i, i, i, vp, vp, vp, vp, vp]
+    lib.gla_state_scan.restype = i
     lib.gla_bwd.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, vp]
     lib.gla_bwd.restype = i
     lib.gla_poll_status.argtypes = [dp, vp]
@@ -125,6 +131,7 @@ def _gate_of(log_alpha, gate):
 
 FLAG_REUSE_PREP = 1
 FLAG_SAVE_STATES = 2
+FLAG_REUSE_SEGMENTS = 4
 
 
 def make_desc(B, H, T, dk, dv, dtype, gate, *, subchunk=16, variant="auto", segments=0, flags=0,
@@ -157,11 +164,14 @@ def alloc_workspace(nbytes: int, device) -> torch.Tensor:
 
 
 def gla_fwd(q, k, v, log_alpha=None, h0=None, *, chunk=64, gate=None, subchunk=16, variant="auto", segments=0,
-            o=None, h_final=None, want_final=True, workspace=None, stream=None, save_states=False):
+            o=None, h_final=None, want_final=True, workspace=None, stream=None, save_states=False,
+            reuse_prep=False, reuse_segments=False):
     """Forward.  Returns (o, h_final or None).  See include/gla.h.
     save_states=True: also store the bf16 chunk states in `workspace` (sized for
     the backward) for a following gla_bwd(..., saved_states=True)
-    (GLA_FLAG_SAVE_STATES)."""
+    (GLA_FLAG_SAVE_STATES).  reuse_prep / reuse_segments: `workspace` holds the prep
+    outputs / segment contributions of a gla_fwd_state call on the same inputs and
+    flags (GLA_FLAG_REUSE_PREP, GLA_FLAG_REUSE_SEGMENTS)."""
     lib = load()
     B, H, T, dk = q.shape
     dv = v.shape[-1]
@@ -170,7 +180,8 @@ def gla_fwd(q, k, v, log_alpha=None, h0=None, *, chunk=64, gate=None, subchunk=1
         o = torch.empty(B, H, T, dv, dtype=q.dtype, device=q.device)
     if h_final is None and want_final:
         h_final = torch.empty(B, H, dk, dv, dtype=torch.float32, device=q.device)
-    flags = FLAG_SAVE_STATES if save_states else 0
+    flags = ((FLAG_SAVE_STATES if save_states else 0) | (FLAG_REUSE_PREP if reuse_prep else 0)
+             | (FLAG_REUSE_SEGMENTS if reuse_segments else 0))
     if workspace is None:
         workspace = alloc_workspace(workspace_size(B, H, T, dk, dv, q.dtype, gate, chunk, save_states,
                                                    subchunk=subchunk, variant=variant, segments=segments,
@@ -182,6 +193,74 @@ def gla_fwd(q, k, v, log_alpha=None, h0=None, *, chunk=64, gate=None, subchunk=1
     if r != GLA_OK:
         raise GLAError(r, "gla_fwd")
     return o, h_final
+
+
+def gla_fwd_state(q, k, v, log_alpha=None, h0=None, *, chunk=64, gate=None, subchunk=16, segments=0,
+                  delta=None, gamma=None, workspace=None, stream=None, save_states=False, reuse_prep=False):
+    """Summary of this piece of the sequence: (delta, gamma) = (the state after the
+    piece from h0, the product of its gates per key channel).  See include/gla.h.
+    save_states: use the workspace layout of gla_fwd(..., save_states=True), so that
+    call can reuse the prep outputs and segment contributions left here."""
+    lib = load()
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    gate = _gate_of(log_alpha, gate)
+    if delta is None:
+        delta = torch.empty(B, H, dk, dv, dtype=torch.float32, device=q.device)
+    if gamma is None:
+        gamma = torch.empty(B, H, dk, dtype=torch.float32, device=q.device)
+    flags = (FLAG_SAVE_STATES if save_states else 0) | (FLAG_REUSE_PREP if reuse_prep else 0)
+    if workspace is None:
+        workspace = alloc_workspace(workspace_size(B, H, T, dk, dv, q.dtype, gate, chunk, bool(flags),
+                                                   subchunk=subchunk, segments=segments, flags=flags), q.device)
+    d = make_desc(B, H, T, dk, dv, q.dtype, gate, subchunk=subchunk, segments=segments, flags=flags,
+                  workspace=workspace)
+    r = lib.gla_fwd_state(ctypes.byref(d), _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(h0), _ptr(delta),
+                          _ptr(gamma), int(chunk), _stream_handle(stream))
+    if r != GLA_OK:
+        raise GLAError(r, "gla_fwd_state")
+    return delta, gamma
+
+
+def gla_bwd_state(q, k, log_alpha, do, dh_final=None, *, chunk=64, gate=None, subchunk=16, segments=0,
+                  ddelta=None, gamma=None, want_gamma=True, workspace=None, stream=None, reuse_prep=False):
+    """Reverse summary of this piece: (ddelta, gamma or None) = (the state adjoint
+    before the piece given dh_final after it, the gate product).  See include/gla.h."""
+    lib = load()
+    B, H, T, dk = q.shape
+    dv = do.shape[-1]
+    gate = _gate_of(log_alpha, gate)
+    if ddelta is None:
+        ddelta = torch.empty(B, H, dk, dv, dtype=torch.float32, device=q.device)
+    if gamma is None and want_gamma:
+        gamma = torch.empty(B, H, dk, dtype=torch.float32, device=q.device)
+    flags = FLAG_REUSE_PREP if reuse_prep else 0
+    if workspace is None:
+        workspace = alloc_workspace(workspace_size(B, H, T, dk, dv, q.dtype, gate, chunk, True, subchunk=subchunk,
+                                                   segments=segments), q.device)
+    d = make_desc(B, H, T, dk, dv, q.dtype, gate, subchunk=subchunk, segments=segments, flags=flags,
+                  workspace=workspace)
+    r = lib.gla_bwd_state(ctypes.byref(d), _ptr(q), _ptr(k), _ptr(log_alpha), _ptr(do), _ptr(dh_final), _ptr(ddelta),
+                          _ptr(gamma), int(chunk), _stream_handle(stream))
+    if r != GLA_OK:
+        raise GLAError(r, "gla_bwd_state")
+    return ddelta, gamma
+
+
+def gla_state_scan(gammas, deltas, seg, *, reverse=False, init=None, out=None, stream=None):
+    """Fold of gathered piece summaries: gammas [P,B,H,dk], deltas [P,B,H,dk,dv] fp32.
+    reverse=False: the state entering piece `seg` (pieces 0 .. seg-1 over init);
+    reverse=True: the adjoint leaving piece `seg` (pieces P-1 .. seg+1 over init)."""
+    lib = load()
+    P, B, H, dk, dv = deltas.shape
+    if out is None:
+        out = torch.empty(B, H, dk, dv, dtype=torch.float32, device=deltas.device)
+    d = make_desc(B, H, 1, dk, dv, torch.bfloat16, "vector")
+    r = lib.gla_state_scan(ctypes.byref(d), int(P), int(seg), int(bool(reverse)), _ptr(gammas), _ptr(deltas),
+                           _ptr(init), _ptr(out), _stream_handle(stream))
+    if r != GLA_OK:
+        raise GLAError(r, "gla_state_scan")
+    return out
 
 
 def gla_fwd_noalloc(q, k, v, log_alpha=None, h0=None, *, chunk=64, gate=None, subchunk=16, variant="auto",
@@ -268,12 +347,13 @@ def gla_epilogue_bwd(o, r, dy, w=None, b=None, *, eps=1e-5, want_dwb=True, works
 
 def gla_bwd(q, k, v, log_alpha, do, h0=None, dh_final=None, *, chunk=64, gate=None, subchunk=16, dq=None, dk=None,
             dv=None, dlog_alpha=None, dh0=None, want_dh0=True, workspace=None, stream=None, reuse_prep=False,
-            saved_states=False, segments=0, variant="auto"):
+            saved_states=False, reuse_segments=False, segments=0, variant="auto"):
     """Backward.  Returns (dq, dk, dv, dlog_alpha or None, dh0 or None).  See include/gla.h.
     reuse_prep=True: `workspace` holds the prep outputs of a gla_fwd call on the same
     inputs with this workspace (GLA_FLAG_REUSE_PREP).  saved_states=True: it also
     holds the chunk states of a gla_fwd(..., save_states=True) call with the same
-    segments and variant (GLA_FLAG_SAVE_STATES)."""
+    segments and variant (GLA_FLAG_SAVE_STATES).  reuse_segments=True: it holds the
+    segment contributions of a gla_bwd_state call (GLA_FLAG_REUSE_SEGMENTS)."""
     lib = load()
     B, H, T, dk_ = q.shape
     dv_ = v.shape[-1]
@@ -285,7 +365,8 @@ def gla_bwd(q, k, v, log_alpha, do, h0=None, dh_final=None, *, chunk=64, gate=No
         dlog_alpha = torch.empty_like(log_alpha)
     if dh0 is None and want_dh0:
         dh0 = torch.empty(B, H, dk_, dv_, dtype=torch.float32, device=q.device)
-    flags = (FLAG_REUSE_PREP if reuse_prep else 0) | (FLAG_SAVE_STATES if saved_states else 0)
+    flags = ((FLAG_REUSE_PREP if reuse_prep else 0) | (FLAG_SAVE_STATES if saved_states else 0)
+             | (FLAG_REUSE_SEGMENTS if reuse_segments else 0))
     if workspace is None:
         workspace = alloc_workspace(workspace_size(B, H, T, dk_, dv_, q.dtype, gate, chunk, True, subchunk=subchunk,
                                                    segments=segments, variant=variant, flags=flags), q.device)

@@ -103,9 +103,21 @@ extern "C" {
  *
  * With either flag the workspace must be sized for the backward
  * (gla_workspace_size(desc, chunk, 1)) on both calls, the gla_fwd call
- * included; that size is at least the forward's. */
+ * included; that size is at least the forward's.
+ *
+ * GLA_FLAG_REUSE_PREP also applies to gla_fwd, gla_fwd_state and gla_bwd_state:
+ * the prep outputs may come from any earlier call of these four on the same
+ * inputs and workspace (the sequence-parallel step runs prep once).
+ *
+ * GLA_FLAG_REUSE_SEGMENTS (gla_fwd, gla_bwd): the workspace holds the zero-state
+ * contributions of every segment written by gla_fwd_state (for gla_fwd) or
+ * gla_bwd_state (for gla_bwd) on the same inputs, descriptor and flags, and
+ * nothing but those calls (and a gla_fwd / gla_bwd with this flag) has written to
+ * the workspace since; the walks' pre-passes are skipped.  Ignored by the fp32
+ * path and by the materialized variant. */
 #define GLA_FLAG_REUSE_PREP 1
 #define GLA_FLAG_SAVE_STATES 2
+#define GLA_FLAG_REUSE_SEGMENTS 4
 
 typedef struct gla_desc {
   int B, H, T;          /* batch, heads, tokens (T >= 1)                                   */
@@ -194,6 +206,42 @@ int gla_epilogue_fwd(const gla_desc *desc, const void *o, const void *r, const f
                      float eps, void *y, void *stream);
 int gla_epilogue_bwd(const gla_desc *desc, const void *o, const void *r, const float *w, const float *b,
                      float eps, const void *dy, void *do_, void *dr, float *dw, float *db, void *stream);
+
+/* ---- sequence (context) parallelism ---------------------------------------------
+ * "Gated Linear Attention Transformers with Hardware-Efficient Training",
+ * sections 3.3 and 4.2: the chunk-level recurrence S_n = diag(gamma_n) S_{n-1} + dS_n
+ * composes affine maps, so a sequence split into consecutive pieces (one per GPU,
+ * piece r holding tokens [t_r, t_{r+1}) of every (batch, head)) needs, per piece,
+ * one summary: its gate product gamma = prod_t alpha_t (per key channel) and the
+ * state it produces.  One exchange of the summaries (an all-gather), a fold, and
+ * every piece reruns gla_fwd / gla_bwd with its incoming state.  Each call below
+ * describes one piece: desc->T is the piece's token count, the tensors hold only
+ * the piece's tokens.  bf16 path only (fp32 descriptors: GLA_ERR_UNSUPPORTED_SHAPE).
+ *
+ * gla_fwd_state: delta [B,H,dk,dv] fp32 = the state after the piece's tokens
+ *   starting from h0 (NULL = zero), i.e. the h_final of gla_fwd, without computing
+ *   o; gamma [B,H,dk] fp32 = prod over the piece's tokens of alpha_t (exp of the
+ *   summed log_alpha; all ones for GLA_GATE_NONE, the scalar gate broadcast over
+ *   dk).  Workspace: gla_workspace_size(desc, chunk, 0).
+ * gla_bwd_state: ddelta [B,H,dk,dv] fp32 = the state adjoint before the piece's
+ *   first token given dh_final (NULL = zero) after its last, i.e. the dh0 of
+ *   gla_bwd, without the token gradients; gamma (NULL = not written) as above.
+ *   Workspace: gla_workspace_size(desc, chunk, 1).
+ * gla_state_scan: the fold over gathered summaries.  gammas [nseg][B,H,dk],
+ *   deltas [nseg][B,H,dk,dv] fp32 (piece-major, as an all-gather stacks them);
+ *   S = init (NULL = zero), then S <- diag(gammas[s]) S + deltas[s] for
+ *   s = 0 .. seg-1 (reverse = 0: the state entering piece seg) or for
+ *   s = nseg-1 down to seg+1 (reverse = 1: the adjoint leaving piece seg); out = S.
+ *   Uses B, H, dk, dv of desc (dv a multiple of 4); no workspace.
+ * All three validate every argument before enqueuing anything and run
+ * asynchronously on `stream`; the first two report device errors through the
+ * status word like gla_fwd. */
+int gla_fwd_state(const gla_desc *desc, const void *q, const void *k, const void *v, const float *log_alpha,
+                  const float *h0, float *delta, float *gamma, int chunk, void *stream);
+int gla_bwd_state(const gla_desc *desc, const void *q, const void *k, const float *log_alpha, const void *do_,
+                  const float *dh_final, float *ddelta, float *gamma, int chunk, void *stream);
+int gla_state_scan(const gla_desc *desc, int nseg, int seg, int reverse, const float *gammas, const float *deltas,
+                   const float *init, float *out, void *stream);
 
 /* ---- forward without a workspace ---------------------------------------------
  * No counterpart in the paper: this entry point exists for callers that cannot

@@ -63,7 +63,8 @@ def test_check_and_workspace(lib):
     assert lib.gla_check(ctypes.byref(desc(flags=1)), 64) == 0
     assert lib.gla_check(ctypes.byref(desc(flags=2)), 64) == 0
     assert lib.gla_check(ctypes.byref(desc(flags=3)), 64) == 0
-    assert lib.gla_check(ctypes.byref(desc(flags=4)), 64) == -1
+    assert lib.gla_check(ctypes.byref(desc(flags=8)), 64) == -1               # unknown flag bit
+    assert lib.gla_check(ctypes.byref(desc(flags=4)), 64) == 0                # GLA_FLAG_REUSE_SEGMENTS
 
 
 def test_saved_state_workspace_layout(lib):
@@ -186,3 +187,38 @@ def test_oracle_not_imported_by_product():
         for f in files:
             if f.endswith((".py", ".cu", ".h", ".cuh")):
                 assert not pat.search(open(os.path.join(root, f)).read()), f
+
+
+def test_sequence_state_validation_enqueues_nothing(lib):
+    """gla_fwd_state / gla_bwd_state / gla_state_scan reject bad arguments before any
+    launch (every call below fails validation: none reaches a kernel)."""
+    vp = ctypes.c_void_p
+    a, mis = vp(4096), vp(4096 + 4)
+    d = desc(T=300, dk=256, dv=512)
+    fs, bs, sc = lib.gla_fwd_state, lib.gla_bwd_state, lib.gla_state_scan
+    d32 = desc(T=300, dk=256, dv=512, dtype=1)
+    assert fs(ctypes.byref(d32), a, a, a, a, None, a, a, 64, None) == -2      # fp32: bf16 path only
+    assert bs(ctypes.byref(d32), a, a, a, a, None, a, a, 64, None) == -2
+    assert fs(ctypes.byref(d), None, a, a, a, None, a, a, 64, None) == -1     # q NULL
+    assert fs(ctypes.byref(d), a, a, a, a, None, None, a, 64, None) == -1     # delta NULL
+    assert fs(ctypes.byref(d), a, a, a, a, None, a, None, 64, None) == -1     # gamma NULL
+    assert fs(ctypes.byref(d), a, a, a, a, mis, a, a, 64, None) == -3         # h0 misaligned
+    assert fs(ctypes.byref(d), a, a, a, a, None, a, a, 64, None) == -1        # no workspace
+    assert bs(ctypes.byref(d), a, a, a, None, None, a, None, 64, None) == -1  # do NULL
+    assert bs(ctypes.byref(d), a, a, a, a, None, None, None, 64, None) == -1  # ddelta NULL
+    assert bs(ctypes.byref(d), a, a, None, a, None, a, None, 64, None) == -1  # vector gate without log_alpha
+    assert bs(ctypes.byref(d), a, a, a, a, None, a, None, 64, None) == -1     # no workspace
+    d.workspace = 1 << 20
+    d.workspace_bytes = 16
+    assert fs(ctypes.byref(d), a, a, a, a, None, a, a, 64, None) == -4        # workspace too small
+    assert bs(ctypes.byref(d), a, a, a, a, None, a, None, 64, None) == -4
+    assert sc(ctypes.byref(d), 0, 0, 0, a, a, None, a, None) == -1            # no pieces
+    assert sc(ctypes.byref(d), 3, 3, 0, a, a, None, a, None) == -1            # seg out of range
+    assert sc(ctypes.byref(d), 3, -1, 0, a, a, None, a, None) == -1
+    assert sc(ctypes.byref(d), 3, 1, 2, a, a, None, a, None) == -1            # reverse not 0/1
+    assert sc(ctypes.byref(d), 3, 1, 0, None, a, None, a, None) == -1         # gammas NULL with a piece to fold
+    assert sc(ctypes.byref(d), 3, 1, 1, a, None, None, a, None) == -1         # deltas NULL
+    assert sc(ctypes.byref(d), 3, 1, 0, a, a, None, None, None) == -1         # out NULL
+    assert sc(ctypes.byref(d), 3, 1, 0, a, a, mis, a, None) == -3             # init misaligned
+    d.dv = 510
+    assert sc(ctypes.byref(d), 3, 1, 0, a, a, None, a, None) == -2            # d_v not a multiple of 4
