@@ -25,8 +25,16 @@
  * (unstable); instead the forward states are checkpointed every CKPT steps and
  * each segment is recomputed forward before it is walked backward.
  *
- * Layout: contiguous row-major [B,H,T,D] for q,k,v,o,do,dq,dk,dv and la/dla
- * ([B,H,T,d_k] vector, [B,H,T] scalar); states [B,H,d_k,d_v].
+ * General gate (appendix C of the paper, G_t = alpha_t^T beta_t): the
+ * gla_oracle_*_general entry points also take lb_t = log beta_t [T, d_v], a gate
+ * on the value side, so that column j of S is scaled by beta_t[j] as well:
+ *
+ *     S_t = diag(alpha_t) S_{t-1} diag(beta_t) + k_t^T v_t ,   o_t = q_t S_t .
+ *
+ * lb == NULL is beta == 1 and runs exactly the alpha-only arithmetic.
+ *
+ * Layout: contiguous row-major [B,H,T,D] for q,k,v,o,do,dq,dk,dv, la/dla
+ * ([B,H,T,d_k] vector, [B,H,T] scalar) and lb/dlb [B,H,T,d_v]; states [B,H,d_k,d_v].
  * All arithmetic is float64.  (b,h) pairs run in parallel with OpenMP.
  */
 #include <math.h>
@@ -55,10 +63,18 @@ static inline double gate_log(const double *la, int mode, long t, int K, int c) 
   return 0.0;
 }
 
-/* One recurrence step S <- diag(alpha_t) S + k_t^T v_t (section 4.1). */
-static void step_state(double *S, const double *q_unused, const double *kt, const double *vt,
+/* One recurrence step S <- diag(alpha_t) S diag(beta_t) + k_t^T v_t (section 4.1;
+ * appendix C for beta).  lbt = log beta_t [V] or NULL (beta == 1). */
+static void step_state(double *S, const double *lbt, const double *kt, const double *vt,
                        const double *la, int mode, long t, int K, int V) {
-  (void)q_unused;
+  if (lbt) {
+    for (int c = 0; c < K; ++c) {
+      const double a = exp(gate_log(la, mode, t, K, c));
+      double *row = S + (long)c * V;
+      for (int j = 0; j < V; ++j) row[j] = a * row[j] * exp(lbt[j]) + kt[c] * vt[j];
+    }
+    return;
+  }
   for (int c = 0; c < K; ++c) {
     const double a = exp(gate_log(la, mode, t, K, c));
     double *row = S + (long)c * V;
@@ -88,11 +104,12 @@ static long la_head_stride(int mode, long T, int K) {
 }
 
 /*
- * Forward.  h0 may be NULL (zero state); hT may be NULL (not written).
+ * Forward.  h0 may be NULL (zero state); hT may be NULL (not written); lb may be
+ * NULL (beta == 1).
  */
-void gla_oracle_fwd(int B, int H, long T, int K, int V, int mode,
-                    const double *q, const double *k, const double *v, const double *la,
-                    const double *h0, double *o, double *hT) {
+void gla_oracle_fwd_general(int B, int H, long T, int K, int V, int mode,
+                            const double *q, const double *k, const double *v, const double *la,
+                            const double *lb, const double *h0, double *o, double *hT) {
   const long BH = (long)B * H;
 #pragma omp parallel for schedule(dynamic, 1)
   for (long bh = 0; bh < BH; ++bh) {
@@ -101,19 +118,27 @@ void gla_oracle_fwd(int B, int H, long T, int K, int V, int mode,
     else memset(S, 0, sizeof(double) * K * V);
     const double *qh = q + bh * T * K, *kh = k + bh * T * K, *vh = v + bh * T * V;
     const double *lah = la ? la + bh * la_head_stride(mode, T, K) : NULL;
+    const double *lbh = lb ? lb + bh * T * V : NULL;
     double *oh = o + bh * T * V;
     for (long t = 0; t < T; ++t) {
+      const double *lbt = lbh ? lbh + t * V : NULL;
 #if GLA_ORACLE_MUTANT == 1
       read_out(S, qh + t * K, oh + t * V, K, V);
-      step_state(S, NULL, kh + t * K, vh + t * V, lah, mode, t, K, V);
+      step_state(S, lbt, kh + t * K, vh + t * V, lah, mode, t, K, V);
 #else
-      step_state(S, NULL, kh + t * K, vh + t * V, lah, mode, t, K, V);
+      step_state(S, lbt, kh + t * K, vh + t * V, lah, mode, t, K, V);
       read_out(S, qh + t * K, oh + t * V, K, V);
 #endif
     }
     if (hT) memcpy(hT + bh * K * V, S, sizeof(double) * K * V);
     free(S);
   }
+}
+
+void gla_oracle_fwd(int B, int H, long T, int K, int V, int mode,
+                    const double *q, const double *k, const double *v, const double *la,
+                    const double *h0, double *o, double *hT) {
+  gla_oracle_fwd_general(B, H, T, K, V, mode, q, k, v, la, NULL, h0, o, hT);
 }
 
 /*
@@ -124,16 +149,17 @@ void gla_oracle_fwd(int B, int H, long T, int K, int V, int mode,
  *     dq_t[c]  = sum_j S_t[c,j] do_t[j]
  *     dk_t[c]  = sum_j dS[c,j] v_t[j]           (S_t = ... + k_t^T v_t)
  *     dv_t[j]  = sum_c k_t[c] dS[c,j]
- *     dla_t[c] = alpha_t[c] sum_j S_{t-1}[c,j] dS[c,j]
- *     dS      <- diag(alpha_t) dS
+ *     dla_t[c] = alpha_t[c] sum_j S_{t-1}[c,j] beta_t[j] dS[c,j]
+ *     dlb_t[j] = beta_t[j] sum_c alpha_t[c] S_{t-1}[c,j] dS[c,j]
+ *     dS      <- diag(alpha_t) dS diag(beta_t)
  *   dh0 = dS
  * Scalar mode returns dla_t = sum_c dla_t[c]; NONE mode writes no dla.
- * dh_final, dla, dh0 may be NULL.
+ * dh_final, dla, dh0 may be NULL; lb == NULL is beta == 1 (dlb then unused).
  */
-void gla_oracle_bwd(int B, int H, long T, int K, int V, int mode,
-                    const double *q, const double *k, const double *v, const double *la,
-                    const double *h0, const double *dout, const double *dhT,
-                    double *dq, double *dk, double *dv, double *dla, double *dh0) {
+void gla_oracle_bwd_general(int B, int H, long T, int K, int V, int mode,
+                            const double *q, const double *k, const double *v, const double *la,
+                            const double *lb, const double *h0, const double *dout, const double *dhT,
+                            double *dq, double *dk, double *dv, double *dla, double *dlb, double *dh0) {
   const long BH = (long)B * H;
   const long nck = (T + CKPT - 1) / CKPT;
 #pragma omp parallel for schedule(dynamic, 1)
@@ -141,6 +167,8 @@ void gla_oracle_bwd(int B, int H, long T, int K, int V, int mode,
     const long KV = (long)K * V;
     const double *qh = q + bh * T * K, *kh = k + bh * T * K, *vh = v + bh * T * V;
     const double *lah = la ? la + bh * la_head_stride(mode, T, K) : NULL;
+    const double *lbh = lb ? lb + bh * T * V : NULL;
+    double *dlbh = (lb && dlb) ? dlb + bh * T * V : NULL;
     const double *doh = dout + bh * T * V;
     double *dqh = dq + bh * T * K, *dkh = dk + bh * T * K, *dvh = dv + bh * T * V;
     double *dlah = (dla && mode != GLA_ORACLE_GATE_NONE) ? dla + bh * la_head_stride(mode, T, K) : NULL;
@@ -152,7 +180,7 @@ void gla_oracle_bwd(int B, int H, long T, int K, int V, int mode,
     else memset(S, 0, sizeof(double) * KV);
     for (long t = 0; t < T; ++t) {
       if (t % CKPT == 0) memcpy(ck + (t / CKPT) * KV, S, sizeof(double) * KV);
-      step_state(S, NULL, kh + t * K, vh + t * V, lah, mode, t, K, V);
+      step_state(S, lbh ? lbh + t * V : NULL, kh + t * K, vh + t * V, lah, mode, t, K, V);
     }
 
     /* seg holds S after each token of the current segment: seg[i] = state after token t0+i */
@@ -168,7 +196,7 @@ void gla_oracle_bwd(int B, int H, long T, int K, int V, int mode,
       /* recompute the segment forward from its checkpoint */
       memcpy(S, ck + ci * KV, sizeof(double) * KV);
       for (long t = t0; t < t1; ++t) {
-        step_state(S, NULL, kh + t * K, vh + t * V, lah, mode, t, K, V);
+        step_state(S, lbh ? lbh + t * V : NULL, kh + t * K, vh + t * V, lah, mode, t, K, V);
         memcpy(seg + (t - t0) * KV, S, sizeof(double) * KV);
       }
       for (long t = t1 - 1; t >= t0; --t) {
@@ -193,8 +221,11 @@ void gla_oracle_bwd(int B, int H, long T, int K, int V, int mode,
           }
           dqh[t * K + c] = acc;
         }
-        /* S_t = diag(alpha_t) S_{t-1} + k_t^T v_t */
+        /* S_t = diag(alpha_t) S_{t-1} diag(beta_t) + k_t^T v_t */
+        const double *lbt = lbh ? lbh + t * V : NULL;
         for (int j = 0; j < V; ++j) dvh[t * V + j] = 0.0;
+        if (dlbh)
+          for (int j = 0; j < V; ++j) dlbh[t * V + j] = 0.0;
         for (int c = 0; c < K; ++c) {
           const double *drow = dS + (long)c * V;
           const double *prow = Sp + (long)c * V;
@@ -203,7 +234,9 @@ void gla_oracle_bwd(int B, int H, long T, int K, int V, int mode,
           for (int j = 0; j < V; ++j) {
             acck += drow[j] * vt[j];
             dvh[t * V + j] += kt[c] * drow[j];
-            accg += prow[j] * drow[j];
+            const double bj = lbt ? exp(lbt[j]) : 1.0;
+            accg += prow[j] * bj * drow[j];
+            if (dlbh) dlbh[t * V + j] += a * prow[j] * bj * drow[j];
           }
 #if GLA_ORACLE_MUTANT == 4
           dkh[t * K + c] = dla_vec[c];
@@ -228,7 +261,10 @@ void gla_oracle_bwd(int B, int H, long T, int K, int V, int mode,
         for (int c = 0; c < K; ++c) {
           const double a = exp(gate_log(lah, mode, t, K, c));
           double *drow = dS + (long)c * V;
-          for (int j = 0; j < V; ++j) drow[j] *= a;
+          if (lbt)
+            for (int j = 0; j < V; ++j) drow[j] *= a * exp(lbt[j]);
+          else
+            for (int j = 0; j < V; ++j) drow[j] *= a;
         }
       }
     }
@@ -239,6 +275,13 @@ void gla_oracle_bwd(int B, int H, long T, int K, int V, int mode,
     free(dS);
     free(dla_vec);
   }
+}
+
+void gla_oracle_bwd(int B, int H, long T, int K, int V, int mode,
+                    const double *q, const double *k, const double *v, const double *la,
+                    const double *h0, const double *dout, const double *dhT,
+                    double *dq, double *dk, double *dv, double *dla, double *dh0) {
+  gla_oracle_bwd_general(B, H, T, K, V, mode, q, k, v, la, NULL, h0, dout, dhT, dq, dk, dv, dla, NULL, dh0);
 }
 
 /* Threads OpenMP will use for the (b,h) loop. */

@@ -6,7 +6,8 @@ CPU-baseline leg of ``bench.py`` do.
 
 The arithmetic lives in ``gla_oracle.c`` (the literal token recurrence of
 "Gated Linear Attention Transformers with Hardware-Efficient Training",
-section 4.1, and back-propagation through it).  This module compiles that file
+section 4.1, its general-gate form of appendix C, and back-propagation through
+them).  This module compiles that file
 with the host C compiler on first use and marshals numpy float64 arrays.
 """
 from __future__ import annotations
@@ -53,6 +54,13 @@ def _open(path):
                                    ctypes.c_int, ctypes.c_int, dp, dp, dp, dp, dp, dp, dp,
                                    dp, dp, dp, dp, dp]
     lib.gla_oracle_bwd.restype = None
+    lib.gla_oracle_fwd_general.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_long, ctypes.c_int,
+                                           ctypes.c_int, ctypes.c_int, dp, dp, dp, dp, dp, dp, dp, dp]
+    lib.gla_oracle_fwd_general.restype = None
+    lib.gla_oracle_bwd_general.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_long, ctypes.c_int,
+                                           ctypes.c_int, ctypes.c_int, dp, dp, dp, dp, dp, dp, dp, dp,
+                                           dp, dp, dp, dp, dp, dp]
+    lib.gla_oracle_bwd_general.restype = None
     lib.gla_oracle_max_threads.restype = ctypes.c_int
     return lib
 
@@ -125,6 +133,46 @@ def bwd(q, k, v, log_alpha, do, h0=None, dh_final=None, gate="vector", _lib_over
     (_lib_override or _load()).gla_oracle_bwd(B, H, T, K, V, mode, _ptr(q), _ptr(k), _ptr(v), _ptr(la), _ptr(h0),
                            _ptr(do), _ptr(dhT), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dla), _ptr(dh0))
     return dq, dk, dv, dla, dh0
+
+
+def fwd_general(q, k, v, log_alpha, log_beta, h0=None, gate="vector", _lib_override=None):
+    """Recurrent form with the general gate G_t = alpha_t^T beta_t (appendix C):
+    S_t = diag(alpha_t) S_{t-1} diag(beta_t) + k_t^T v_t, o_t = q_t S_t.
+    log_beta [B,H,T,V] (None: beta == 1).  Returns (o, h_final) as float64."""
+    mode = _gate_mode(gate)
+    q, k, v, la, lb, h0 = _f64(q), _f64(k), _f64(v), _f64(log_alpha), _f64(log_beta), _f64(h0)
+    B, H, T, K = q.shape
+    V = v.shape[-1]
+    o = np.empty((B, H, T, V), np.float64)
+    hT = np.empty((B, H, K, V), np.float64)
+    if mode == GATE_NONE:
+        la = None
+    (_lib_override or _load()).gla_oracle_fwd_general(B, H, T, K, V, mode, _ptr(q), _ptr(k), _ptr(v), _ptr(la),
+                                                      _ptr(lb), _ptr(h0), _ptr(o), _ptr(hT))
+    return o, hT
+
+
+def bwd_general(q, k, v, log_alpha, log_beta, do, h0=None, dh_final=None, gate="vector", _lib_override=None):
+    """Back-propagation through the general-gate recurrence.  Returns
+    (dq, dk, dv, dlog_alpha or None, dlog_beta or None, dh0) as float64."""
+    mode = _gate_mode(gate)
+    q, k, v, la, lb, do = _f64(q), _f64(k), _f64(v), _f64(log_alpha), _f64(log_beta), _f64(do)
+    h0, dhT = _f64(h0), _f64(dh_final)
+    B, H, T, K = q.shape
+    V = v.shape[-1]
+    dq, dk, dv = np.empty_like(q), np.empty_like(k), np.empty_like(v)
+    if mode == GATE_VECTOR:
+        dla = np.empty((B, H, T, K), np.float64)
+    elif mode == GATE_SCALAR:
+        dla = np.empty((B, H, T), np.float64)
+    else:
+        dla, la = None, None
+    dlb = None if lb is None else np.empty((B, H, T, V), np.float64)
+    dh0 = np.empty((B, H, K, V), np.float64)
+    (_lib_override or _load()).gla_oracle_bwd_general(B, H, T, K, V, mode, _ptr(q), _ptr(k), _ptr(v), _ptr(la),
+                                                      _ptr(lb), _ptr(h0), _ptr(do), _ptr(dhT), _ptr(dq), _ptr(dk),
+                                                      _ptr(dv), _ptr(dla), _ptr(dlb), _ptr(dh0))
+    return dq, dk, dv, dla, dlb, dh0
 
 
 def decode_step(q, k, v, log_alpha, state, gate="vector"):

@@ -353,3 +353,112 @@ def test_pins_pass_on_oracle(oracle_mod):
 def test_pins_catch_planted_mistakes(mutant):
     from oracle.oracle import Mutant
     assert not _pins_pass(Mutant(mutant))
+
+
+# ------------------------------------------------------ general gate (appendix C)
+# S_t = diag(alpha_t) S_{t-1} diag(beta_t) + k_t^T v_t, o_t = q_t S_t.
+
+def _general_case(rng, T, K, V, with_state=True):
+    q = rng.standard_normal((1, 1, T, K))
+    k = rng.standard_normal((1, 1, T, K)) / np.sqrt(K)
+    v = rng.standard_normal((1, 1, T, V))
+    la = np.log(rng.uniform(0.6, 1.0, (1, 1, T, K)))
+    lb = np.log(rng.uniform(0.6, 1.0, (1, 1, T, V)))
+    h0 = rng.standard_normal((1, 1, K, V)) if with_state else None
+    return q, k, v, la, lb, h0
+
+
+def test_general_gate_with_unit_beta_is_the_alpha_only_oracle(oracle_mod):
+    """log beta = 0 reduces the general recurrence to the paper's per-key gate."""
+    rng = np.random.default_rng(21)
+    q, k, v, la, lb, h0 = _general_case(rng, 37, 5, 4)
+    do, dhT = rng.standard_normal((1, 1, 37, 4)), rng.standard_normal((1, 1, 5, 4))
+    zero = np.zeros_like(lb)
+    o1, h1 = oracle_mod.fwd(q, k, v, la, h0)
+    o2, h2 = oracle_mod.fwd_general(q, k, v, la, zero, h0)
+    np.testing.assert_array_equal(o1, o2)
+    np.testing.assert_array_equal(h1, h2)
+    g1 = oracle_mod.bwd(q, k, v, la, do, h0, dhT)
+    g2 = oracle_mod.bwd_general(q, k, v, la, zero, do, h0, dhT)
+    for a, b in zip(g1, (g2[0], g2[1], g2[2], g2[3], g2[5])):
+        np.testing.assert_allclose(a, b, rtol=1e-13, atol=1e-13)
+
+
+def test_general_gate_parallel_form(oracle_mod):
+    """The recurrence against the quadratic (parallel) form written with global
+    cumulative log-gates Ag (per key channel) and Eg (per value channel):
+    o_t[j] = sum_c q_t[c] e^{Ag_t[c]} h0[c,j] e^{Eg_t[j]}
+           + sum_{s<=t} sum_c q_t[c] k_s[c] e^{Ag_t[c]-Ag_s[c]} v_s[j] e^{Eg_t[j]-Eg_s[j]}."""
+    rng = np.random.default_rng(22)
+    T, K, V = 20, 5, 4
+    q, k, v, la, lb, h0 = _general_case(rng, T, K, V)
+    o, hT = oracle_mod.fwd_general(q, k, v, la, lb, h0)
+    Q, Kk, Vv, H0 = q[0, 0], k[0, 0], v[0, 0], h0[0, 0]
+    Ag, Eg = np.cumsum(la[0, 0], axis=0), np.cumsum(lb[0, 0], axis=0)
+    ref = np.zeros((T, V))
+    for t in range(T):
+        ref[t] = (Q[t] * np.exp(Ag[t])) @ H0 * np.exp(Eg[t])
+        for s in range(t + 1):
+            ref[t] += (Q[t] * Kk[s] * np.exp(Ag[t] - Ag[s])).sum() * Vv[s] * np.exp(Eg[t] - Eg[s])
+    refT = np.exp(Ag[-1])[:, None] * H0 * np.exp(Eg[-1])[None, :]
+    for s in range(T):
+        refT += np.outer(Kk[s] * np.exp(Ag[-1] - Ag[s]), Vv[s] * np.exp(Eg[-1] - Eg[s]))
+    np.testing.assert_allclose(o[0, 0], ref, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(hT[0, 0], refT, rtol=1e-12, atol=1e-12)
+
+
+def test_general_gate_transpose_symmetry(oracle_mod):
+    """S^T obeys the same recurrence with (k, alpha) and (v, beta) exchanged, so the
+    final state of the exchanged problem is the transpose (a swapped alpha / beta
+    in the state update fails this)."""
+    rng = np.random.default_rng(23)
+    T, K, V = 15, 4, 3
+    q, k, v, la, lb, h0 = _general_case(rng, T, K, V)
+    _, hT = oracle_mod.fwd_general(q, k, v, la, lb, h0)
+    qv = rng.standard_normal((1, 1, T, V))
+    _, hTt = oracle_mod.fwd_general(qv, v, k, lb, la, np.swapaxes(h0, 2, 3))
+    np.testing.assert_allclose(hTt, np.swapaxes(hT, 2, 3), rtol=1e-12, atol=1e-12)
+
+
+def test_general_gate_finite_differences(oracle_mod):
+    """Every gradient of L = sum(o W) + sum(h_final U), log beta and h0 included,
+    against central differences."""
+    rng = np.random.default_rng(24)
+    T, K, V = 6, 3, 2
+    q, k, v, la, lb, h0 = _general_case(rng, T, K, V)
+    W, U = rng.standard_normal((1, 1, T, V)), rng.standard_normal((1, 1, K, V))
+
+    def loss(q, k, v, la, lb, h0):
+        o, hT = oracle_mod.fwd_general(q, k, v, la, lb, h0)
+        return float((o * W).sum() + (hT * U).sum())
+
+    dq, dk, dv, dla, dlb, dh0 = oracle_mod.bwd_general(q, k, v, la, lb, W, h0, U)
+    args = [q, k, v, la, lb, h0]
+    for i, g in enumerate((dq, dk, dv, dla, dlb, dh0)):
+        fd = np.zeros_like(args[i])
+        for idx in np.ndindex(args[i].shape):
+            plus = [a.copy() for a in args]
+            minus = [a.copy() for a in args]
+            plus[i][idx] += 1e-6
+            minus[i][idx] -= 1e-6
+            fd[idx] = (loss(*plus) - loss(*minus)) / 2e-6
+        np.testing.assert_allclose(g, fd, rtol=1e-6, atol=1e-8)
+
+
+def test_general_gate_closed_form_gate_gradients(oracle_mod):
+    """The closed forms the CUDA path uses, against back-propagation:
+    dlog alpha_t[c] = sum_{i>=t} (q_i dq_i - k_i dk_i)[c] + sum_j hT[c,j] dhT[c,j]
+    dlog beta_t[j]  = sum_{i>=t} (o_i do_i - v_i dv_i)[j] + sum_c hT[c,j] dhT[c,j]
+    (log alpha_t enters through q_t e^{Ag_t} and k_t e^{-Ag_t}, log beta_t through
+    o_t = e^{Eg_t} (...) and v_t e^{-Eg_t}; the h_final terms are the suffix beyond T)."""
+    rng = np.random.default_rng(25)
+    T, K, V = 50, 4, 5
+    q, k, v, la, lb, h0 = _general_case(rng, T, K, V)
+    do, dhT = rng.standard_normal((1, 1, T, V)), rng.standard_normal((1, 1, K, V))
+    o, hT = oracle_mod.fwd_general(q, k, v, la, lb, h0)
+    dq, dk, dv, dla, dlb, _ = oracle_mod.bwd_general(q, k, v, la, lb, do, h0, dhT)
+    rev = lambda x: np.flip(np.cumsum(np.flip(x, axis=2), axis=2), axis=2)
+    cla = rev(q * dq - k * dk) + (hT * dhT).sum(axis=3)[:, :, None, :]
+    clb = rev(o * do - v * dv) + (hT * dhT).sum(axis=2)[:, :, None, :]
+    np.testing.assert_allclose(dla, cla, rtol=1e-10, atol=1e-10)
+    np.testing.assert_allclose(dlb, clb, rtol=1e-10, atol=1e-10)
