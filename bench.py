@@ -411,6 +411,42 @@ def measure_seqpar(args, w, dev, stream, seed=0, pieces=8):
             "allgather_bytes_per_rank_per_direction": (B * H * K * V + B * H * K) * 4}
 
 
+def measure_general_gate(args, w, dev, stream, seed=0):
+    """The general gate alpha_t^T beta_t (CUDA-core path, fp32 arithmetic) on the
+    bench workload with log beta drawn like log alpha: forward + backward step time
+    from events around `steps` steps (inputs larger than L2)."""
+    import torch
+
+    import chunkwise_linear_rnn_fwd_b200 as pkg
+    from chunkwise_linear_rnn_fwd_b200.synth import make_inputs
+
+    B, H, T, K, V = w["B"], w["H"], w["T"], w["K"], w["V"]
+    x = make_inputs(B, H, T, K, V, dtype=torch.bfloat16, gate=w["gate"], seed=seed, z_mean=w["z_mean"],
+                    with_log_beta=True)
+    q, k, v, la, lb, do = (t.to(dev) for t in (x.q, x.k, x.v, x.log_alpha, x.log_beta, x.do))
+    wsf = pkg.alloc_workspace(pkg.general_workspace_size(B, H, T, K, V, torch.bfloat16, w["gate"], w["C"]), dev)
+    wsb = pkg.alloc_workspace(pkg.general_workspace_size(B, H, T, K, V, torch.bfloat16, w["gate"], w["C"], True),
+                              dev)
+
+    def step():
+        pkg.gla_fwd_general(q, k, v, la, lb, chunk=w["C"], workspace=wsf, stream=stream)
+        pkg.gla_bwd_general(q, k, v, la, lb, do, chunk=w["C"], workspace=wsb, stream=stream)
+
+    step()
+    torch.cuda.synchronize()
+    n = 3
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(n):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / n
+    return {"workload": f"general gate, B={B} H={H} T={T} d_k={K} d_v={V} bf16 in/out, {w['gate']} alpha + vector beta",
+            "path": "CUDA cores, fp32 arithmetic, materialised chunk states", "ms_per_step": ms,
+            "tokens_per_s": B * T / (ms / 1e3)}
+
+
 def run_ours(args, w):
     import torch
     import torch.distributed as dist
@@ -545,6 +581,8 @@ def run_ours(args, w):
     decode = measure_decode(args, dev, stream, peaks, peak_src, seed=rank)
     epilogue = measure_epilogue(args, w, dev, stream, peaks, peak_src, seed=rank)
     seqpar = measure_seqpar(args, w, dev, stream, seed=rank)
+    general = measure_general_gate(args, w, dev, stream, seed=rank)
+    general["vs_alpha_only_step"] = general["ms_per_step"] / ms_per_step
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -564,7 +602,7 @@ def run_ours(args, w):
             "kernel_timing": "separate pass of the same K steps with a CUDA-event pair around each launch",
             "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "clocks": clocks, "cpu_baseline": cpu, "decode_step": decode, "layer_epilogue": epilogue,
-            "sequence_parallel": seqpar,
+            "sequence_parallel": seqpar, "general_gate": general,
         }
         print(json.dumps(line), flush=True)
     if world > 1:

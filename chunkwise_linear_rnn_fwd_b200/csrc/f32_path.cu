@@ -18,6 +18,16 @@
 //   dqk      dq, dk, dlog_alpha (closed form, section 4.3, with the chunk
 //            boundary term sum_v S_n[c,v] dS_n[c,v])
 //   dv       dv
+//
+// General gate (appendix C, G_t = alpha_t^T beta_t): with log beta [B,H,T,V] the
+// state is also scaled per value channel, S_t = diag(alpha_t) S_{t-1} diag(beta_t)
+// + k_t^T v_t.  Every kernel then takes E[t,v], the chunk-local cumulative log beta
+// (null: beta == 1, the arithmetic above unchanged), and the factors
+// exp(E_t[v] - E_s[v]) join the pairs (s, t) exactly as exp(B_t[c] - B_s[c]) do on
+// the key side.  The gate gradient of beta has the same closed form as alpha's on
+// the other index: dlog beta_t[v] = sum_{i>=t} (o_i[v] do_i[v] - v_i[v] dv_i[v])
+// with the chunk boundary term sum_c S_n[c,v] dS_n[c,v] (kernel k_dlb; o is
+// recomputed in fp32 for it).
 #include <cuda_bf16.h>
 
 #include "internal.h"
@@ -65,11 +75,25 @@ __global__ void k_prep(const float *__restrict__ la, Dims d, float *__restrict__
   }
 }
 
+// E[bh, t, v] = chunk-local inclusive cumsum of log_beta (rows t >= T add 0).
+__global__ void k_prep_beta(const float *__restrict__ lb, Dims d, float *__restrict__ Ec) {
+  const long bh = blockIdx.y;
+  const int n = blockIdx.x;
+  for (int v = threadIdx.x; v < d.V; v += blockDim.x) {
+    float acc = 0.f;
+    for (int j = 0; j < d.C; ++j) {
+      const long t = (long)n * d.C + j;
+      if (t < d.T) acc += lb[(bh * d.T + t) * d.V + v];
+      Ec[(bh * d.Tp + t) * d.V + v] = acc;
+    }
+  }
+}
+
 // H[bh, n] = state before chunk n; H[bh, N] = final state.  Thread = (c, v).
 template <typename T>
 __global__ void k_states(const T *__restrict__ k, const T *__restrict__ v, const float *__restrict__ Bc,
-                         const float *__restrict__ h0, Dims d, float *__restrict__ Hs,
-                         float *__restrict__ hT) {
+                         const float *__restrict__ Ec, const float *__restrict__ h0, Dims d,
+                         float *__restrict__ Hs, float *__restrict__ hT) {
   const int vi = blockIdx.x * blockDim.x + threadIdx.x;
   const int c = blockIdx.y * blockDim.y + threadIdx.y;
   const long bh = blockIdx.z;
@@ -79,15 +103,17 @@ __global__ void k_states(const T *__restrict__ k, const T *__restrict__ v, const
   for (int n = 0; n < d.N; ++n) {
     Hs[(bh * (d.N + 1) + n) * KV + (long)c * d.V + vi] = S;
     const float blast = Bc[(bh * d.Tp + (long)n * d.C + d.C - 1) * d.K + c];
+    const float elast = Ec ? Ec[(bh * d.Tp + (long)n * d.C + d.C - 1) * d.V + vi] : 0.f;
     float acc = 0.f;
     for (int j = 0; j < d.C; ++j) {
       const long t = (long)n * d.C + j;
       if (t >= d.T) break;
       const float kk = ld(k + (bh * d.T + t) * d.K + c);
-      const float w = __expf(blast - Bc[(bh * d.Tp + t) * d.K + c]);
+      float w = __expf(blast - Bc[(bh * d.Tp + t) * d.K + c]);
+      if (Ec) w *= __expf(elast - Ec[(bh * d.Tp + t) * d.V + vi]);
       acc += kk * w * ld(v + (bh * d.T + t) * d.V + vi);
     }
-    S = __expf(blast) * S + acc;
+    S = __expf(blast + elast) * S + acc;
   }
   Hs[(bh * (d.N + 1) + d.N) * KV + (long)c * d.V + vi] = S;
   if (hT) hT[bh * KV + (long)c * d.V + vi] = S;
@@ -114,9 +140,11 @@ __global__ void k_scores(const T *__restrict__ q, const T *__restrict__ k, const
 }
 
 // o[t, v] = sum_c q_t[c] e^{B_t[c]} H[n][c, v] + sum_{s<=t} P[t, s] v_s[v]
-template <typename T>
+// (general gate: the first term times e^{E_t[v]}, the pairs times e^{E_t[v] - E_s[v]})
+template <typename T, typename TO>
 __global__ void k_out(const T *__restrict__ q, const T *__restrict__ v, const float *__restrict__ Bc,
-                      const float *__restrict__ Hs, const float *__restrict__ P, Dims d, T *__restrict__ o) {
+                      const float *__restrict__ Ec, const float *__restrict__ Hs, const float *__restrict__ P,
+                      Dims d, TO *__restrict__ o) {
   const int vi = blockIdx.x * blockDim.x + threadIdx.x;
   const int n = blockIdx.y;
   const long bh = blockIdx.z;
@@ -130,7 +158,16 @@ __global__ void k_out(const T *__restrict__ q, const T *__restrict__ v, const fl
     for (int c = 0; c < d.K; ++c)
       acc += ld(q + (bh * d.T + t) * d.K + c) * __expf(Bc[(bh * d.Tp + t) * d.K + c]) * H[(long)c * d.V + vi];
     const float *Pr = P + ((bh * d.N + n) * d.C + ti) * d.C;
-    for (int si = 0; si <= ti; ++si) acc += Pr[si] * ld(v + (bh * d.T + (long)n * d.C + si) * d.V + vi);
+    if (Ec) {
+      const float Et = Ec[(bh * d.Tp + t) * d.V + vi];
+      acc *= __expf(Et);
+      for (int si = 0; si <= ti; ++si) {
+        const long s = (long)n * d.C + si;
+        acc += Pr[si] * ld(v + (bh * d.T + s) * d.V + vi) * __expf(Et - Ec[(bh * d.Tp + s) * d.V + vi]);
+      }
+    } else {
+      for (int si = 0; si <= ti; ++si) acc += Pr[si] * ld(v + (bh * d.T + (long)n * d.C + si) * d.V + vi);
+    }
     st(o + (bh * d.T + t) * d.V + vi, acc);
   }
 }
@@ -140,8 +177,8 @@ __global__ void k_out(const T *__restrict__ q, const T *__restrict__ v, const fl
 // dH[bh, n] = adjoint of the state after chunk n (through chunks > n and dh_final).
 template <typename T>
 __global__ void k_dstates(const T *__restrict__ q, const T *__restrict__ dout, const float *__restrict__ Bc,
-                          const float *__restrict__ dhT, Dims d, float *__restrict__ dHs,
-                          float *__restrict__ dh0) {
+                          const float *__restrict__ Ec, const float *__restrict__ dhT, Dims d,
+                          float *__restrict__ dHs, float *__restrict__ dh0) {
   const int vi = blockIdx.x * blockDim.x + threadIdx.x;
   const int c = blockIdx.y * blockDim.y + threadIdx.y;
   const long bh = blockIdx.z;
@@ -151,29 +188,39 @@ __global__ void k_dstates(const T *__restrict__ q, const T *__restrict__ dout, c
   for (int n = d.N - 1; n >= 0; --n) {
     dHs[(bh * d.N + n) * KV + (long)c * d.V + vi] = dS;
     const float blast = Bc[(bh * d.Tp + (long)n * d.C + d.C - 1) * d.K + c];
+    const float elast = Ec ? Ec[(bh * d.Tp + (long)n * d.C + d.C - 1) * d.V + vi] : 0.f;
     float acc = 0.f;
     for (int j = 0; j < d.C; ++j) {
       const long t = (long)n * d.C + j;
       if (t >= d.T) break;
-      acc += ld(q + (bh * d.T + t) * d.K + c) * __expf(Bc[(bh * d.Tp + t) * d.K + c]) *
-             ld(dout + (bh * d.T + t) * d.V + vi);
+      float x = ld(q + (bh * d.T + t) * d.K + c) * __expf(Bc[(bh * d.Tp + t) * d.K + c]) *
+                ld(dout + (bh * d.T + t) * d.V + vi);
+      if (Ec) x *= __expf(Ec[(bh * d.Tp + t) * d.V + vi]);
+      acc += x;
     }
-    dS = __expf(blast) * dS + acc;
+    dS = __expf(blast + elast) * dS + acc;
   }
   if (dh0) dh0[bh * KV + (long)c * d.V + vi] = dS;
 }
 
-// dP[bh, n, t, s] = sum_v do_t[v] v_s[v] for s <= t, else 0.
+// dP[bh, n, t, s] = sum_v do_t[v] v_s[v] (e^{E_t[v] - E_s[v]}) for s <= t, else 0.
 template <typename T>
-__global__ void k_dscores(const T *__restrict__ dout, const T *__restrict__ v, Dims d, float *__restrict__ dP) {
+__global__ void k_dscores(const T *__restrict__ dout, const T *__restrict__ v, const float *__restrict__ Ec, Dims d,
+                          float *__restrict__ dP) {
   const long bh = blockIdx.y;
   const int n = blockIdx.x;
   for (int idx = threadIdx.x; idx < d.C * d.C; idx += blockDim.x) {
     const int ti = idx / d.C, si = idx % d.C;
     const long t = (long)n * d.C + ti, s = (long)n * d.C + si;
     float acc = 0.f;
-    if (si <= ti && t < d.T)
-      for (int j = 0; j < d.V; ++j) acc += ld(dout + (bh * d.T + t) * d.V + j) * ld(v + (bh * d.T + s) * d.V + j);
+    if (si <= ti && t < d.T) {
+      if (Ec)
+        for (int j = 0; j < d.V; ++j)
+          acc += ld(dout + (bh * d.T + t) * d.V + j) * ld(v + (bh * d.T + s) * d.V + j) *
+                 __expf(Ec[(bh * d.Tp + t) * d.V + j] - Ec[(bh * d.Tp + s) * d.V + j]);
+      else
+        for (int j = 0; j < d.V; ++j) acc += ld(dout + (bh * d.T + t) * d.V + j) * ld(v + (bh * d.T + s) * d.V + j);
+    }
     dP[((bh * d.N + n) * d.C + ti) * d.C + si] = acc;
   }
 }
@@ -187,9 +234,9 @@ __global__ void k_dscores(const T *__restrict__ dout, const T *__restrict__ v, D
 // suffix of dlog b beyond the chunk, so no cross-chunk scan is needed.
 template <typename T>
 __global__ void k_dqk(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
-                      const T *__restrict__ dout, const float *__restrict__ Bc, const float *__restrict__ Hs,
-                      const float *__restrict__ dHs, const float *__restrict__ dP, Dims d, T *__restrict__ dq,
-                      T *__restrict__ dk, float *__restrict__ dgv) {
+                      const T *__restrict__ dout, const float *__restrict__ Bc, const float *__restrict__ Ec,
+                      const float *__restrict__ Hs, const float *__restrict__ dHs, const float *__restrict__ dP,
+                      Dims d, T *__restrict__ dq, T *__restrict__ dk, float *__restrict__ dgv) {
   const int c = threadIdx.x;
   if (c >= d.K) return;
   const long bh = blockIdx.y;
@@ -208,9 +255,18 @@ __global__ void k_dqk(const T *__restrict__ q, const T *__restrict__ k, const T 
     if (t >= d.T) break;
     const float Bt = Bc[(bh * d.Tp + t) * d.K + c];
     float a1 = 0.f, a2 = 0.f;
-    for (int j = 0; j < d.V; ++j) {
-      a1 += ld(dout + (bh * d.T + t) * d.V + j) * H[j];
-      a2 += ld(v + (bh * d.T + t) * d.V + j) * dH[j];
+    if (Ec) {
+      const float *Et = Ec + (bh * d.Tp + t) * d.V;
+      const float *El = Ec + (bh * d.Tp + (long)n * d.C + d.C - 1) * d.V;
+      for (int j = 0; j < d.V; ++j) {
+        a1 += ld(dout + (bh * d.T + t) * d.V + j) * H[j] * __expf(Et[j]);
+        a2 += ld(v + (bh * d.T + t) * d.V + j) * dH[j] * __expf(El[j] - Et[j]);
+      }
+    } else {
+      for (int j = 0; j < d.V; ++j) {
+        a1 += ld(dout + (bh * d.T + t) * d.V + j) * H[j];
+        a2 += ld(v + (bh * d.T + t) * d.V + j) * dH[j];
+      }
     }
     float dqv = __expf(Bt) * a1;
     float dkv = __expf(blast - Bt) * a2;
@@ -238,9 +294,12 @@ __global__ void k_dqk(const T *__restrict__ q, const T *__restrict__ k, const T 
 }
 
 // dv_t = (k_t (.) e^{B_last - B_t}) dH[n] + sum_{s>=t} P[s,t] do_s
+// (general gate: the first term times e^{E_last[v] - E_t[v]}, the pairs times
+// e^{E_s[v] - E_t[v]}; dvf, if not null, receives dv in fp32 for the beta gradient)
 template <typename T>
 __global__ void k_dv(const T *__restrict__ k, const T *__restrict__ dout, const float *__restrict__ Bc,
-                     const float *__restrict__ dHs, const float *__restrict__ P, Dims d, T *__restrict__ dv) {
+                     const float *__restrict__ Ec, const float *__restrict__ dHs, const float *__restrict__ P, Dims d,
+                     T *__restrict__ dv, float *__restrict__ dvf) {
   const int vi = blockIdx.x * blockDim.x + threadIdx.x;
   const int n = blockIdx.y;
   const long bh = blockIdx.z;
@@ -256,12 +315,49 @@ __global__ void k_dv(const T *__restrict__ k, const T *__restrict__ dout, const 
       const float blast = Bc[(bh * d.Tp + (long)n * d.C + d.C - 1) * d.K + c];
       acc += ld(k + (bh * d.T + t) * d.K + c) * __expf(blast - Bc[(bh * d.Tp + t) * d.K + c]) * dH[(long)c * d.V + vi];
     }
-    for (int si = ti; si < d.C; ++si) {
-      const long s = (long)n * d.C + si;
-      if (s >= d.T) break;
-      acc += Pc[si * d.C + ti] * ld(dout + (bh * d.T + s) * d.V + vi);
+    if (Ec) {
+      const float Et = Ec[(bh * d.Tp + t) * d.V + vi];
+      acc *= __expf(Ec[(bh * d.Tp + (long)n * d.C + d.C - 1) * d.V + vi] - Et);
+      for (int si = ti; si < d.C; ++si) {
+        const long s = (long)n * d.C + si;
+        if (s >= d.T) break;
+        acc += Pc[si * d.C + ti] * ld(dout + (bh * d.T + s) * d.V + vi) * __expf(Ec[(bh * d.Tp + s) * d.V + vi] - Et);
+      }
+    } else {
+      for (int si = ti; si < d.C; ++si) {
+        const long s = (long)n * d.C + si;
+        if (s >= d.T) break;
+        acc += Pc[si * d.C + ti] * ld(dout + (bh * d.T + s) * d.V + vi);
+      }
     }
     st(dv + (bh * d.T + t) * d.V + vi, acc);
+    if (dvf) dvf[(bh * d.T + t) * d.V + vi] = acc;
+  }
+}
+
+// dlog beta[bh, t, v] = sum_{i >= t in chunk} (o_i[v] do_i[v] - v_i[v] dv_i[v])
+//                      + sum_c S_n[c, v] dS_n[c, v]
+// (o and dv in fp32; S_n = H[n+1] the state after chunk n, dS_n = dH[n] its
+// adjoint: the suffix beyond the chunk, so no cross-chunk scan).  Thread = (v, chunk).
+template <typename T>
+__global__ void k_dlb(const T *__restrict__ v, const T *__restrict__ dout, const float *__restrict__ of,
+                      const float *__restrict__ dvf, const float *__restrict__ Hs, const float *__restrict__ dHs,
+                      Dims d, float *__restrict__ dlb) {
+  const int vi = blockIdx.x * blockDim.x + threadIdx.x;
+  const int n = blockIdx.y;
+  const long bh = blockIdx.z;
+  if (vi >= d.V) return;
+  const long KV = (long)d.K * d.V;
+  const float *Hn = Hs + (bh * (d.N + 1) + n + 1) * KV + vi;
+  const float *dH = dHs + (bh * d.N + n) * KV + vi;
+  float run = 0.f;
+  for (int c = 0; c < d.K; ++c) run += Hn[(long)c * d.V] * dH[(long)c * d.V];
+  for (int ti = d.C - 1; ti >= 0; --ti) {
+    const long t = (long)n * d.C + ti;
+    if (t >= d.T) continue;
+    const long i = (bh * d.T + t) * d.V + vi;
+    run += of[i] * ld(dout + i) - ld(v + i) * dvf[i];
+    dlb[i] = run;
   }
 }
 
@@ -283,10 +379,11 @@ Dims dims_of(const Problem &p) { return Dims{p.T, p.K, p.V, p.C, p.N, p.gate, p.
 
 struct F32Ws {
   float *Bc, *Hs, *P, *dHs, *dP, *dgv;
+  float *Ec, *of, *dvf;  // general gate only
   size_t bytes;
 };
 
-F32Ws carve(const Problem &p, void *ws, bool bwd) {
+F32Ws carve(const Problem &p, void *ws, bool bwd, bool general) {
   Carve cv(ws);
   F32Ws w{};
   w.Bc = cv.take<float>((size_t)p.BH * p.Tp * p.K);
@@ -297,68 +394,94 @@ F32Ws carve(const Problem &p, void *ws, bool bwd) {
     w.dP = cv.take<float>((size_t)p.BH * p.N * p.C * p.C);
     w.dgv = cv.take<float>((size_t)p.BH * p.Tp * p.K);
   }
+  if (general) {
+    w.Ec = cv.take<float>((size_t)p.BH * p.Tp * p.V);
+    if (bwd) {
+      w.of = cv.take<float>((size_t)p.BH * p.T * p.V);
+      w.dvf = cv.take<float>((size_t)p.BH * p.T * p.V);
+    }
+  }
   w.bytes = cv.bytes();
   return w;
 }
 
 template <typename T>
-int fwd_impl(const Problem &p, const T *q, const T *k, const T *v, const float *la, const float *h0, T *o,
-             float *hT, void *ws, cudaStream_t st) {
+int fwd_impl(const Problem &p, const T *q, const T *k, const T *v, const float *la, const float *lb, const float *h0,
+             T *o, float *hT, void *ws, cudaStream_t st) {
   const Dims d = dims_of(p);
-  F32Ws w = carve(p, ws, false);
+  F32Ws w = carve(p, ws, false, lb != nullptr);
   const int kth = (p.K + 31) / 32 * 32;
   GLA_LAUNCH(K_F32_PREP, st, (k_prep<<<dim3(p.N, p.BH), kth, 0, st>>>(la, d, w.Bc)));
+  if (lb) GLA_LAUNCH(K_F32_PREP, st, (k_prep_beta<<<dim3(p.N, p.BH), 256, 0, st>>>(lb, d, w.Ec)));
   GLA_LAUNCH(K_F32_STATES, st,
-             (k_states<T><<<dim3((p.V + 31) / 32, (p.K + 7) / 8, p.BH), dim3(32, 8), 0, st>>>(k, v, w.Bc, h0, d, w.Hs, hT)));
+             (k_states<T><<<dim3((p.V + 31) / 32, (p.K + 7) / 8, p.BH), dim3(32, 8), 0, st>>>(k, v, w.Bc, w.Ec, h0, d,
+                                                                                              w.Hs, hT)));
   GLA_LAUNCH(K_F32_SCORES, st, (k_scores<T><<<dim3(p.N, p.BH), 256, 0, st>>>(q, k, w.Bc, d, w.P)));
   GLA_LAUNCH(K_F32_OUT, st,
-             (k_out<T><<<dim3((p.V + 63) / 64, p.N, p.BH), dim3(64, 4), 0, st>>>(q, v, w.Bc, w.Hs, w.P, d, o)));
+             (k_out<T, T><<<dim3((p.V + 63) / 64, p.N, p.BH), dim3(64, 4), 0, st>>>(q, v, w.Bc, w.Ec, w.Hs, w.P, d,
+                                                                                     o)));
   return GLA_OK;
 }
 
 template <typename T>
-int bwd_impl(const Problem &p, const T *q, const T *k, const T *v, const float *la, const float *h0, const T *dout,
-             const float *dhT, T *dq, T *dk, T *dv, float *dla, float *dh0, void *ws, cudaStream_t st) {
+int bwd_impl(const Problem &p, const T *q, const T *k, const T *v, const float *la, const float *lb, const float *h0,
+             const T *dout, const float *dhT, T *dq, T *dk, T *dv, float *dla, float *dlb, float *dh0, void *ws,
+             cudaStream_t st) {
   const Dims d = dims_of(p);
-  F32Ws w = carve(p, ws, true);
+  F32Ws w = carve(p, ws, true, lb != nullptr);
   const int kth = (p.K + 31) / 32 * 32;
   GLA_LAUNCH(K_F32_PREP, st, (k_prep<<<dim3(p.N, p.BH), kth, 0, st>>>(la, d, w.Bc)));
+  if (lb) GLA_LAUNCH(K_F32_PREP, st, (k_prep_beta<<<dim3(p.N, p.BH), 256, 0, st>>>(lb, d, w.Ec)));
   GLA_LAUNCH(K_F32_STATES, st,
-             (k_states<T><<<dim3((p.V + 31) / 32, (p.K + 7) / 8, p.BH), dim3(32, 8), 0, st>>>(k, v, w.Bc, h0, d, w.Hs, nullptr)));
+             (k_states<T><<<dim3((p.V + 31) / 32, (p.K + 7) / 8, p.BH), dim3(32, 8), 0, st>>>(k, v, w.Bc, w.Ec, h0, d,
+                                                                                              w.Hs, nullptr)));
   GLA_LAUNCH(K_F32_SCORES, st, (k_scores<T><<<dim3(p.N, p.BH), 256, 0, st>>>(q, k, w.Bc, d, w.P)));
   GLA_LAUNCH(K_F32_DSTATES, st,
-             (k_dstates<T><<<dim3((p.V + 31) / 32, (p.K + 7) / 8, p.BH), dim3(32, 8), 0, st>>>(q, dout, w.Bc, dhT, d, w.dHs, dh0)));
-  GLA_LAUNCH(K_F32_DSCORES, st, (k_dscores<T><<<dim3(p.N, p.BH), 256, 0, st>>>(dout, v, d, w.dP)));
+             (k_dstates<T><<<dim3((p.V + 31) / 32, (p.K + 7) / 8, p.BH), dim3(32, 8), 0, st>>>(q, dout, w.Bc, w.Ec,
+                                                                                               dhT, d, w.dHs, dh0)));
+  GLA_LAUNCH(K_F32_DSCORES, st, (k_dscores<T><<<dim3(p.N, p.BH), 256, 0, st>>>(dout, v, w.Ec, d, w.dP)));
   GLA_LAUNCH(K_F32_DQK, st,
-             (k_dqk<T><<<dim3(p.N, p.BH), kth, 0, st>>>(q, k, v, dout, w.Bc, w.Hs, w.dHs, w.dP, d, dq, dk, w.dgv)));
+             (k_dqk<T><<<dim3(p.N, p.BH), kth, 0, st>>>(q, k, v, dout, w.Bc, w.Ec, w.Hs, w.dHs, w.dP, d, dq, dk,
+                                                         w.dgv)));
   GLA_LAUNCH(K_F32_DV, st,
-             (k_dv<T><<<dim3((p.V + 63) / 64, p.N, p.BH), dim3(64, 4), 0, st>>>(k, dout, w.Bc, w.dHs, w.P, d, dv)));
+             (k_dv<T><<<dim3((p.V + 63) / 64, p.N, p.BH), dim3(64, 4), 0, st>>>(k, dout, w.Bc, w.Ec, w.dHs, w.P, d, dv,
+                                                                                w.dvf)));
   if (p.gate != GLA_GATE_NONE)
     GLA_LAUNCH(K_F32_DG_SCALAR, st, (k_dg_out<<<dim3((p.T + 127) / 128, p.BH), 128, 0, st>>>(w.dgv, d, dla)));
+  if (lb) {
+    // o in fp32 for the beta gradient, then the closed form
+    GLA_LAUNCH(K_F32_OUT, st,
+               (k_out<T, float><<<dim3((p.V + 63) / 64, p.N, p.BH), dim3(64, 4), 0, st>>>(q, v, w.Bc, w.Ec, w.Hs, w.P,
+                                                                                          d, w.of)));
+    GLA_LAUNCH(K_F32_DLB, st,
+               (k_dlb<T><<<dim3((p.V + 63) / 64, p.N, p.BH), 64, 0, st>>>(v, dout, w.of, w.dvf, w.Hs, w.dHs, d, dlb)));
+  }
   return GLA_OK;
 }
 
 }  // namespace
 
-size_t f32_workspace(const Problem &p, bool bwd) { return carve(p, nullptr, bwd).bytes; }
+size_t f32_workspace(const Problem &p, bool bwd) { return carve(p, nullptr, bwd, false).bytes; }
+size_t f32_general_workspace(const Problem &p, bool bwd) { return carve(p, nullptr, bwd, true).bytes; }
 
-int f32_fwd(const Problem &p, const void *q, const void *k, const void *v, const float *la, const float *h0, void *o,
-            float *hT, void *ws, cudaStream_t st) {
+int f32_fwd(const Problem &p, const void *q, const void *k, const void *v, const float *la, const float *lb,
+            const float *h0, void *o, float *hT, void *ws, cudaStream_t st) {
   if (p.dtype == GLA_DTYPE_FP32)
-    return fwd_impl<float>(p, (const float *)q, (const float *)k, (const float *)v, la, h0, (float *)o, hT, ws, st);
-  return fwd_impl<__nv_bfloat16>(p, (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v, la,
-                                 h0, (__nv_bfloat16 *)o, hT, ws, st);
+    return fwd_impl<float>(p, (const float *)q, (const float *)k, (const float *)v, la, lb, h0, (float *)o, hT, ws,
+                           st);
+  using bf = __nv_bfloat16;
+  return fwd_impl<bf>(p, (const bf *)q, (const bf *)k, (const bf *)v, la, lb, h0, (bf *)o, hT, ws, st);
 }
 
-int f32_bwd(const Problem &p, const void *q, const void *k, const void *v, const float *la, const float *h0,
-            const void *dout, const float *dhT, void *dq, void *dk, void *dv, float *dla, float *dh0, void *ws,
-            cudaStream_t st) {
+int f32_bwd(const Problem &p, const void *q, const void *k, const void *v, const float *la, const float *lb,
+            const float *h0, const void *dout, const float *dhT, void *dq, void *dk, void *dv, float *dla,
+            float *dlb, float *dh0, void *ws, cudaStream_t st) {
   if (p.dtype == GLA_DTYPE_FP32)
-    return bwd_impl<float>(p, (const float *)q, (const float *)k, (const float *)v, la, h0, (const float *)dout, dhT,
-                           (float *)dq, (float *)dk, (float *)dv, dla, dh0, ws, st);
+    return bwd_impl<float>(p, (const float *)q, (const float *)k, (const float *)v, la, lb, h0, (const float *)dout,
+                           dhT, (float *)dq, (float *)dk, (float *)dv, dla, dlb, dh0, ws, st);
   using bf = __nv_bfloat16;
-  return bwd_impl<bf>(p, (const bf *)q, (const bf *)k, (const bf *)v, la, h0, (const bf *)dout, dhT, (bf *)dq,
-                      (bf *)dk, (bf *)dv, dla, dh0, ws, st);
+  return bwd_impl<bf>(p, (const bf *)q, (const bf *)k, (const bf *)v, la, lb, h0, (const bf *)dout, dhT, (bf *)dq,
+                      (bf *)dk, (bf *)dv, dla, dlb, dh0, ws, st);
 }
 
 }  // namespace gla

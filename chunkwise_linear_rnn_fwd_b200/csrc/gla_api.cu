@@ -12,7 +12,7 @@ const char *kernel_name(int id) {
   static const char *names[K_COUNT] = {
       "f32_prep",  "f32_states", "f32_scores", "f32_out",    "f32_dstates", "f32_dscores", "f32_dqk",
       "f32_dv",    "f32_dg_out", "tc_prep",    "tc_walk",    "tc_scan(unused)", "tc_bwd",  "status_clear",
-      "decode",    "epilogue_fwd", "epilogue_bwd", "epilogue_reduce", "state_scan", "fold_segments"};
+      "decode",    "epilogue_fwd", "epilogue_bwd", "epilogue_reduce", "state_scan", "fold_segments", "f32_dlog_beta"};
   if (id < 0 || id >= K_COUNT) return "unknown";
   return names[id];
 }
@@ -64,7 +64,9 @@ namespace {
 
 bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
 
-int make_problem(const gla_desc *d, int chunk, Problem *p) {
+// tensor_path: bf16 descriptors also pass the tensor-core path's shape limits
+// (false for the general gate, which runs on CUDA cores for both dtypes).
+int make_problem(const gla_desc *d, int chunk, Problem *p, bool tensor_path = true) {
   if (!d) return GLA_ERR_INVALID_ARG;
   if (d->B < 1 || d->H < 1 || d->T < 1 || d->dk < 1 || d->dv < 1) return GLA_ERR_INVALID_ARG;
   if (d->dtype != GLA_DTYPE_BF16 && d->dtype != GLA_DTYPE_FP32) return GLA_ERR_INVALID_ARG;
@@ -95,7 +97,7 @@ int make_problem(const gla_desc *d, int chunk, Problem *p) {
   p->BH = (long)d->B * d->H;
   p->N = (d->T + chunk - 1) / chunk;
   p->Tp = (long)p->N * chunk;
-  if (p->dtype == GLA_DTYPE_BF16) {
+  if (p->dtype == GLA_DTYPE_BF16 && tensor_path) {
     const int r = tc_check(*p);
     if (r != GLA_OK) return r;
   }
@@ -112,6 +114,13 @@ int check_ws(const gla_desc *d, const Problem &p, bool bwd) {
   if (!d->workspace) return GLA_ERR_INVALID_ARG;
   if (((uintptr_t)d->workspace & 255u) != 0) return GLA_ERR_MISALIGNED;
   if (d->workspace_bytes < need) return GLA_ERR_WORKSPACE_TOO_SMALL;
+  return GLA_OK;
+}
+
+int check_general_ws(const gla_desc *d, const Problem &p, bool bwd) {
+  if (!d->workspace) return GLA_ERR_INVALID_ARG;
+  if (((uintptr_t)d->workspace & 255u) != 0) return GLA_ERR_MISALIGNED;
+  if (d->workspace_bytes < f32_general_workspace(p, bwd)) return GLA_ERR_WORKSPACE_TOO_SMALL;
   return GLA_OK;
 }
 
@@ -172,7 +181,7 @@ int gla_fwd(const gla_desc *desc, const void *q, const void *k, const void *v, c
   cudaStream_t st = (cudaStream_t)stream;
   GLA_TRY(clear_status(desc, st));
   if (p.dtype == GLA_DTYPE_BF16) return tc_fwd(p, q, k, v, log_alpha, h0, o, h_final, desc->workspace, st);
-  return f32_fwd(p, q, k, v, log_alpha, h0, o, h_final, desc->workspace, st);
+  return f32_fwd(p, q, k, v, log_alpha, nullptr, h0, o, h_final, desc->workspace, st);
 }
 
 int gla_bwd(const gla_desc *desc, const void *q, const void *k, const void *v, const float *log_alpha,
@@ -201,7 +210,62 @@ int gla_bwd(const gla_desc *desc, const void *q, const void *k, const void *v, c
   GLA_TRY(clear_status(desc, st));
   if (p.dtype == GLA_DTYPE_BF16)
     return tc_bwd(p, q, k, v, log_alpha, h0, do_, dh_final, dq, dk, dv, dlog_alpha, dh0, desc->workspace, st);
-  return f32_bwd(p, q, k, v, log_alpha, h0, do_, dh_final, dq, dk, dv, dlog_alpha, dh0, desc->workspace, st);
+  return f32_bwd(p, q, k, v, log_alpha, nullptr, h0, do_, dh_final, dq, dk, dv, dlog_alpha, nullptr, dh0,
+                 desc->workspace, st);
+}
+
+size_t gla_general_workspace_size(const gla_desc *desc, int chunk, int for_bwd) {
+  Problem p;
+  if (make_problem(desc, chunk, &p, false) != GLA_OK) return 0;
+  return f32_general_workspace(p, for_bwd != 0);
+}
+
+int gla_fwd_general(const gla_desc *desc, const void *q, const void *k, const void *v, const float *log_alpha,
+                    const float *log_beta, const float *h0, void *o, float *h_final, int chunk, void *stream) {
+  Problem p;
+  GLA_TRY(make_problem(desc, chunk, &p, false));
+  GLA_TRY(check_req(q));
+  GLA_TRY(check_req(k));
+  GLA_TRY(check_req(v));
+  GLA_TRY(check_req(o));
+  GLA_TRY(check_gate_ptr(p, log_alpha));
+  GLA_TRY(check_req(log_beta));
+  GLA_TRY(check_opt(h0));
+  GLA_TRY(check_opt(h_final));
+  GLA_TRY(check_general_ws(desc, p, false));
+  cudaStream_t st = (cudaStream_t)stream;
+  GLA_TRY(clear_status(desc, st));
+  return f32_fwd(p, q, k, v, log_alpha, log_beta, h0, o, h_final, desc->workspace, st);
+}
+
+int gla_bwd_general(const gla_desc *desc, const void *q, const void *k, const void *v, const float *log_alpha,
+                    const float *log_beta, const float *h0, const void *do_, const float *dh_final, void *dq,
+                    void *dk, void *dv, float *dlog_alpha, float *dlog_beta, float *dh0, int chunk, void *stream) {
+  Problem p;
+  GLA_TRY(make_problem(desc, chunk, &p, false));
+  GLA_TRY(check_req(q));
+  GLA_TRY(check_req(k));
+  GLA_TRY(check_req(v));
+  GLA_TRY(check_req(do_));
+  GLA_TRY(check_req(dq));
+  GLA_TRY(check_req(dk));
+  GLA_TRY(check_req(dv));
+  GLA_TRY(check_gate_ptr(p, log_alpha));
+  if (p.gate == GLA_GATE_NONE) {
+    if (dlog_alpha) return GLA_ERR_INVALID_ARG;
+  } else {
+    GLA_TRY(check_req(dlog_alpha));
+  }
+  GLA_TRY(check_req(log_beta));
+  GLA_TRY(check_req(dlog_beta));
+  GLA_TRY(check_opt(h0));
+  GLA_TRY(check_opt(dh_final));
+  GLA_TRY(check_opt(dh0));
+  GLA_TRY(check_general_ws(desc, p, true));
+  cudaStream_t st = (cudaStream_t)stream;
+  GLA_TRY(clear_status(desc, st));
+  return f32_bwd(p, q, k, v, log_alpha, log_beta, h0, do_, dh_final, dq, dk, dv, dlog_alpha, dlog_beta, dh0,
+                 desc->workspace, st);
 }
 
 int gla_fwd_state(const gla_desc *desc, const void *q, const void *k, const void *v, const float *log_alpha,

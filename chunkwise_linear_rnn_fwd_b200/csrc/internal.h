@@ -31,6 +31,7 @@ enum KernelId : int {
   K_EPI_REDUCE,
   K_STATE_SCAN,
   K_FOLD_SEGMENTS,
+  K_F32_DLB,
   K_COUNT
 };
 
@@ -72,12 +73,14 @@ struct Carve {
 };
 
 // fp32 CUDA-core path (any element type; exact pairwise log-space intra-chunk math)
+// lb / dlb: log beta and its gradient of the general gate (null: beta == 1)
 size_t f32_workspace(const Problem &p, bool bwd);
-int f32_fwd(const Problem &p, const void *q, const void *k, const void *v, const float *la,
+size_t f32_general_workspace(const Problem &p, bool bwd);
+int f32_fwd(const Problem &p, const void *q, const void *k, const void *v, const float *la, const float *lb,
             const float *h0, void *o, float *hT, void *ws, cudaStream_t st);
-int f32_bwd(const Problem &p, const void *q, const void *k, const void *v, const float *la,
-            const float *h0, const void *dout, const float *dhT, void *dq, void *dk, void *dv,
-            float *dla, float *dh0, void *ws, cudaStream_t st);
+int f32_bwd(const Problem &p, const void *q, const void *k, const void *v, const float *la, const float *lb,
+            const float *h0, const void *dout, const float *dhT, void *dq, void *dk, void *dv, float *dla,
+            float *dlb, float *dh0, void *ws, cudaStream_t st);
 
 // recurrent decode step (CUDA cores); arguments validated by the caller
 int decode_step(const gla_desc *d, const void *q, const void *k, const void *v, const float *la, float *state,

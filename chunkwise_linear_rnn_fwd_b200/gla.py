@@ -31,7 +31,8 @@ NOALLOC_SCRATCH_BYTES = 64 << 20  # GLA_NOALLOC_SCRATCH_BYTES in include/gla.h
 EXPORTS = ["gla_workspace_size", "gla_check", "gla_fwd", "gla_bwd", "gla_poll_status", "gla_status_string",
            "gla_timing_enable", "gla_timing_collect", "gla_kernel_name", "gla_build_info", "gla_fwd_noalloc",
            "gla_decode_step", "gla_selftest_timeout", "gla_epilogue_workspace_size", "gla_epilogue_fwd",
-           "gla_epilogue_bwd", "gla_fwd_state", "gla_bwd_state", "gla_state_scan"]
+           "gla_epilogue_bwd", "gla_fwd_state", "gla_bwd_state", "gla_state_scan", "gla_general_workspace_size",
+           "gla_fwd_general", "gla_bwd_general"]
 
 
 class GLAError(RuntimeError):
@@ -85,6 +86,12 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.gla_bwd_state.restype = i
     lib.gla_state_scan.argtypes = [dp, i, i, i, vp, vp, vp, vp, vp]
     lib.gla_state_scan.restype = i
+    lib.gla_general_workspace_size.argtypes = [dp, i, i]
+    lib.gla_general_workspace_size.restype = ctypes.c_size_t
+    lib.gla_fwd_general.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp, i, vp]
+    lib.gla_fwd_general.restype = i
+    lib.gla_bwd_general.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, vp]
+    lib.gla_bwd_general.restype = i
     lib.gla_bwd.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, vp]
     lib.gla_bwd.restype = i
     lib.gla_poll_status.argtypes = [dp, vp]
@@ -193,6 +200,58 @@ def gla_fwd(q, k, v, log_alpha=None, h0=None, *, chunk=64, gate=None, subchunk=1
     if r != GLA_OK:
         raise GLAError(r, "gla_fwd")
     return o, h_final
+
+
+def general_workspace_size(B, H, T, dk, dv, dtype, gate, chunk=64, for_bwd=False) -> int:
+    d = make_desc(B, H, T, dk, dv, dtype, gate)
+    n = load().gla_general_workspace_size(ctypes.byref(d), int(chunk), int(bool(for_bwd)))
+    if n == 0:
+        raise GLAError(load().gla_check(ctypes.byref(d), int(chunk)), "gla_general_workspace_size")
+    return int(n)
+
+
+def gla_fwd_general(q, k, v, log_alpha, log_beta, h0=None, *, chunk=64, gate=None, o=None, h_final=None,
+                    want_final=True, workspace=None, stream=None):
+    """Forward with the general gate alpha_t^T beta_t (log_beta [B,H,T,d_v]).
+    Returns (o, h_final or None).  See include/gla.h."""
+    lib = load()
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    gate = _gate_of(log_alpha, gate)
+    if o is None:
+        o = torch.empty(B, H, T, dv, dtype=q.dtype, device=q.device)
+    if h_final is None and want_final:
+        h_final = torch.empty(B, H, dk, dv, dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = alloc_workspace(general_workspace_size(B, H, T, dk, dv, q.dtype, gate, chunk, False), q.device)
+    d = make_desc(B, H, T, dk, dv, q.dtype, gate, workspace=workspace)
+    r = lib.gla_fwd_general(ctypes.byref(d), _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(log_beta), _ptr(h0),
+                            _ptr(o), _ptr(h_final), int(chunk), _stream_handle(stream))
+    if r != GLA_OK:
+        raise GLAError(r, "gla_fwd_general")
+    return o, h_final
+
+
+def gla_bwd_general(q, k, v, log_alpha, log_beta, do, h0=None, dh_final=None, *, chunk=64, gate=None,
+                    want_dh0=True, workspace=None, stream=None):
+    """Backward of gla_fwd_general: (dq, dk, dv, dlog_alpha or None, dlog_beta, dh0 or None)."""
+    lib = load()
+    B, H, T, dk_ = q.shape
+    dv_ = v.shape[-1]
+    gate = _gate_of(log_alpha, gate)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    dla = None if gate == "none" else torch.empty_like(log_alpha)
+    dlb = torch.empty_like(log_beta)
+    dh0 = torch.empty(B, H, dk_, dv_, dtype=torch.float32, device=q.device) if want_dh0 else None
+    if workspace is None:
+        workspace = alloc_workspace(general_workspace_size(B, H, T, dk_, dv_, q.dtype, gate, chunk, True), q.device)
+    d = make_desc(B, H, T, dk_, dv_, q.dtype, gate, workspace=workspace)
+    r = lib.gla_bwd_general(ctypes.byref(d), _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(log_beta), _ptr(h0),
+                            _ptr(do), _ptr(dh_final), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dla), _ptr(dlb), _ptr(dh0),
+                            int(chunk), _stream_handle(stream))
+    if r != GLA_OK:
+        raise GLAError(r, "gla_bwd_general")
+    return dq, dk, dv, dla, dlb, dh0
 
 
 def gla_fwd_state(q, k, v, log_alpha=None, h0=None, *, chunk=64, gate=None, subchunk=16, segments=0,

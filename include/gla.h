@@ -207,6 +207,26 @@ int gla_epilogue_fwd(const gla_desc *desc, const void *o, const void *r, const f
 int gla_epilogue_bwd(const gla_desc *desc, const void *o, const void *r, const float *w, const float *b,
                      float eps, const void *dy, void *do_, void *dr, float *dw, float *db, void *stream);
 
+/* ---- general gate (value-side gate beta) -------------------------------------------
+ * "Gated Linear Attention Transformers with Hardware-Efficient Training",
+ * appendix C: the gate G_t = alpha_t^T beta_t, an outer product of a key-side
+ * gate alpha_t (per desc->gate, given as log_alpha exactly as for gla_fwd) and a
+ * value-side gate beta_t in (0,1]^{d_v}:
+ *     S_t = diag(alpha_t) S_{t-1} diag(beta_t) + k_t^T v_t ,   o_t = q_t S_t .
+ *   log_beta / dlog_beta: [B,H,T,dv] fp32, required (log_beta = 0 gives gla_fwd's
+ *   result).  Every other argument as for gla_fwd / gla_bwd.  dlog_beta is the
+ *   gradient of the loss with respect to log_beta.
+ * Runs on the CUDA-core path for either dtype (fp32 arithmetic, every chunk state
+ * materialised, intra-chunk pairs in log space, so any gate strength is stable).
+ * Workspace: gla_general_workspace_size(desc, chunk, for_bwd) bytes, 256-byte
+ * aligned; desc->flags, variant and segments are ignored.  Errors as for gla_fwd. */
+size_t gla_general_workspace_size(const gla_desc *desc, int chunk, int for_bwd);
+int gla_fwd_general(const gla_desc *desc, const void *q, const void *k, const void *v, const float *log_alpha,
+                    const float *log_beta, const float *h0, void *o, float *h_final, int chunk, void *stream);
+int gla_bwd_general(const gla_desc *desc, const void *q, const void *k, const void *v, const float *log_alpha,
+                    const float *log_beta, const float *h0, const void *do_, const float *dh_final, void *dq,
+                    void *dk, void *dv, float *dlog_alpha, float *dlog_beta, float *dh0, int chunk, void *stream);
+
 /* ---- sequence (context) parallelism ---------------------------------------------
  * "Gated Linear Attention Transformers with Hardware-Efficient Training",
  * sections 3.3 and 4.2: the chunk-level recurrence S_n = diag(gamma_n) S_{n-1} + dS_n

@@ -222,3 +222,23 @@ def test_sequence_state_validation_enqueues_nothing(lib):
     assert sc(ctypes.byref(d), 3, 1, 0, a, a, mis, a, None) == -3             # init misaligned
     d.dv = 510
     assert sc(ctypes.byref(d), 3, 1, 0, a, a, None, a, None) == -2            # d_v not a multiple of 4
+
+
+def test_general_gate_validation_enqueues_nothing(lib):
+    """gla_fwd_general / gla_bwd_general reject bad arguments before any launch
+    (every call below fails validation: none reaches a kernel)."""
+    vp = ctypes.c_void_p
+    a, mis = vp(4096), vp(4096 + 4)
+    d = desc(T=100, dk=64, dv=64)
+    f, b = lib.gla_fwd_general, lib.gla_bwd_general
+    assert lib.gla_general_workspace_size(ctypes.byref(d), 64, 1) > lib.gla_general_workspace_size(ctypes.byref(d), 64, 0)
+    assert f(ctypes.byref(d), a, a, a, a, None, None, a, None, 64, None) == -1      # log_beta NULL
+    assert f(ctypes.byref(d), a, a, a, a, mis, None, a, None, 64, None) == -3       # log_beta misaligned
+    assert f(ctypes.byref(d), a, a, a, None, a, None, a, None, 64, None) == -1      # vector gate without log_alpha
+    assert f(ctypes.byref(d), a, a, a, a, a, None, a, None, 64, None) == -1         # no workspace
+    assert b(ctypes.byref(d), a, a, a, a, a, None, a, None, a, a, a, a, None, None, 64, None) == -1  # dlog_beta NULL
+    assert b(ctypes.byref(d), a, a, a, a, a, None, a, None, a, a, a, None, a, None, 64, None) == -1  # dlog_alpha NULL
+    d.workspace = 1 << 20
+    d.workspace_bytes = 16
+    assert f(ctypes.byref(d), a, a, a, a, a, None, a, None, 64, None) == -4         # workspace too small
+    assert b(ctypes.byref(d), a, a, a, a, a, None, a, None, a, a, a, a, a, None, 64, None) == -4
