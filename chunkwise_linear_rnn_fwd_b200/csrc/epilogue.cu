@@ -19,8 +19,9 @@
 // flight while one is computed.  No stage is shared between warps, so there are
 // no block-wide barriers in the row loop.  Lane l holds the 8-element chunks
 // l, l + 32, ... of a row (d_v <= 1024, a multiple of 8): the mean and the
-// variance are two passes over registers with warp shuffles, and the outputs
-// leave as coalesced 16-byte stores.  The gradients of w and b are reduced
+// variance are two passes over registers with warp shuffles, the elementwise
+// arithmetic runs on packed fp32 pairs (f32x2 add / mul / fma: one instruction per
+// two values), and the outputs leave as coalesced 16-byte stores.  The gradients of w and b are reduced
 // deterministically: every CTA writes its partial sums to the caller's workspace
 // and a second kernel adds them in order.
 #include <cuda_bf16.h>
@@ -48,61 +49,137 @@ struct EpiArgs {
   unsigned *status;
 };
 
-__device__ __forceinline__ void ld8(const float *p, float *x) {
-  const float4 a = __ldg(reinterpret_cast<const float4 *>(p)), b = __ldg(reinterpret_cast<const float4 *>(p) + 1);
-  x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
-}
-// 8 consecutive elements from shared memory (the staged row), widened to fp32
-__device__ __forceinline__ void lds8(const float *p, float *x) {
-  const float4 a = reinterpret_cast<const float4 *>(p)[0], b = reinterpret_cast<const float4 *>(p)[1];
-  x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
-}
-__device__ __forceinline__ void lds8(const __nv_bfloat16 *p, float *x) {
-  const uint4 u = *reinterpret_cast<const uint4 *>(p);
-  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w[i]));
-    x[2 * i] = f.x;
-    x[2 * i + 1] = f.y;
-  }
-}
-__device__ __forceinline__ void st8(float *p, const float *x) {
-  reinterpret_cast<float4 *>(p)[0] = make_float4(x[0], x[1], x[2], x[3]);
-  reinterpret_cast<float4 *>(p)[1] = make_float4(x[4], x[5], x[6], x[7]);
-}
-__device__ __forceinline__ void st8(__nv_bfloat16 *p, const float *x) {
-  uint4 u;
-  uint32_t *w = reinterpret_cast<uint32_t *>(&u);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const __nv_bfloat162 h = __floats2bfloat162_rn(x[2 * i], x[2 * i + 1]);
-    w[i] = *reinterpret_cast<const uint32_t *>(&h);
-  }
-  *reinterpret_cast<uint4 *>(p) = u;
-}
-
 __device__ __forceinline__ float warp_sum(float x) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
   return x;
 }
 
-// sigmoid(x).  bf16 rows: (1 + tanh(x/2)) / 2 with the one-instruction tanh
-// approximation (relative error about 2^-11, below the output's bf16 rounding);
-// fp32 rows: 1 / (1 + e^-x) with the fast exponential and divide (about 1e-6).
+// tanh, one-instruction approximation (relative error about 2^-11, below the
+// bf16 rounding of the epilogue's outputs)
 __device__ __forceinline__ float tanh_approx(float x) {
   float y;
   asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+
+// ---- packed fp32 pairs (sm_100 f32x2 arithmetic: one instruction per two values)
+using f2 = uint64_t;
+__device__ __forceinline__ f2 pk(float lo, float hi) {
+  f2 r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void upk(f2 v, float &lo, float &hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ f2 add2(f2 a, f2 b) {
+  f2 d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ f2 mul2(f2 a, f2 b) {
+  f2 d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ f2 fma2(f2 a, f2 b, f2 c) {
+  f2 d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ float hsum(f2 v) {
+  float lo, hi;
+  upk(v, lo, hi);
+  return lo + hi;
+}
+// 8 consecutive elements as 4 pairs: from shared memory (the staged row) ...
+__device__ __forceinline__ f2 bf16pair(uint32_t w) {  // element 2i in the low half
+  return pk(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
+__device__ __forceinline__ void lds8p(const __nv_bfloat16 *p, f2 *x) {
+  const uint4 u = *reinterpret_cast<const uint4 *>(p);
+  x[0] = bf16pair(u.x);
+  x[1] = bf16pair(u.y);
+  x[2] = bf16pair(u.z);
+  x[3] = bf16pair(u.w);
+}
+__device__ __forceinline__ void lds8p(const float *p, f2 *x) {
+  const ulonglong2 a = reinterpret_cast<const ulonglong2 *>(p)[0], b = reinterpret_cast<const ulonglong2 *>(p)[1];
+  x[0] = a.x;
+  x[1] = a.y;
+  x[2] = b.x;
+  x[3] = b.y;
+}
+// ... from global memory (w, b) ...
+__device__ __forceinline__ void ldg8p(const float *p, f2 *x) {
+  const ulonglong2 a = __ldg(reinterpret_cast<const ulonglong2 *>(p)), b = __ldg(reinterpret_cast<const ulonglong2 *>(p) + 1);
+  x[0] = a.x;
+  x[1] = a.y;
+  x[2] = b.x;
+  x[3] = b.y;
+}
+// ... and back out (global or shared memory)
+__device__ __forceinline__ void st8p(float *p, const f2 *x) {
+  reinterpret_cast<ulonglong2 *>(p)[0] = make_ulonglong2(x[0], x[1]);
+  reinterpret_cast<ulonglong2 *>(p)[1] = make_ulonglong2(x[2], x[3]);
+}
+__device__ __forceinline__ void st8p(__nv_bfloat16 *p, const f2 *x) {
+  uint4 u;
+  uint32_t *w = reinterpret_cast<uint32_t *>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float lo, hi;
+    upk(x[i], lo, hi);
+    const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    w[i] = *reinterpret_cast<const uint32_t *>(&h);
+  }
+  *reinterpret_cast<uint4 *>(p) = u;
+}
+
+// Swish gate of a pair r: rs = r sigmoid(r) and sg = sigmoid(r).  bf16 rows:
+// h = r/2, t = tanh(h), sigmoid = (1 + t)/2, r sigmoid(r) = h + h t; fp32 rows:
+// the fast exponential and divide per element.
 template <typename T>
-__device__ __forceinline__ float sigm(float x) {
-  return __fdividef(1.f, 1.f + __expf(-x));
+__device__ __forceinline__ void gate2(f2 r, f2 &rs, f2 &sg) {
+  float lo, hi;
+  upk(r, lo, hi);
+  sg = pk(__fdividef(1.f, 1.f + __expf(-lo)), __fdividef(1.f, 1.f + __expf(-hi)));
+  rs = mul2(r, sg);
 }
 template <>
-__device__ __forceinline__ float sigm<__nv_bfloat16>(float x) {
-  return fmaf(0.5f, tanh_approx(0.5f * x), 0.5f);
+__device__ __forceinline__ void gate2<__nv_bfloat16>(f2 r, f2 &rs, f2 &sg) {
+  const f2 half = pk(0.5f, 0.5f);
+  const f2 h = mul2(r, half);
+  float lo, hi;
+  upk(h, lo, hi);
+  const f2 t = pk(tanh_approx(lo), tanh_approx(hi));
+  rs = fma2(h, t, h);
+  sg = fma2(t, half, half);
+}
+
+// Row statistics over packed chunks: mean, then 1/sqrt(biased variance + eps).
+template <int NCH>
+__device__ __forceinline__ void row_stats2(const f2 (&x)[NCH][4], int lane, int V, float inv_v, float eps, float &mu,
+                                           float &rstd) {
+  f2 s = pk(0.f, 0.f);
+#pragma unroll
+  for (int i = 0; i < NCH; ++i)
+    if (8 * (lane + 32 * i) < V)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) s = add2(s, x[i][e]);
+  mu = warp_sum(hsum(s)) * inv_v;
+  const f2 nmu = pk(-mu, -mu);
+  f2 q = pk(0.f, 0.f);
+#pragma unroll
+  for (int i = 0; i < NCH; ++i)
+    if (8 * (lane + 32 * i) < V)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const f2 d = add2(x[i][e], nmu);
+        q = fma2(d, d, q);
+      }
+  rstd = rsqrtf(warp_sum(hsum(q)) * inv_v + eps);
 }
 
 // Global -> shared bulk copy (no multicast) completing on an mbarrier.
@@ -111,30 +188,6 @@ __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t by
                    dev::smem_u32(dst)),
                "l"(src), "r"(bytes), "r"(dev::smem_u32(bar))
                : "memory");
-}
-
-// Row statistics: mean and 1/sqrt(var + eps) of the row held in x (NCH chunks of 8
-// per lane; chunk i of lane l is element 8 (l + 32 i) .. +8, valid if < V).
-template <int NCH>
-__device__ __forceinline__ void row_stats(const float (&x)[NCH][8], int lane, int V, float inv_v, float eps,
-                                          float &mu, float &rstd) {
-  float s = 0.f;
-#pragma unroll
-  for (int i = 0; i < NCH; ++i)
-    if (8 * (lane + 32 * i) < V)
-#pragma unroll
-      for (int e = 0; e < 8; ++e) s += x[i][e];
-  mu = warp_sum(s) * inv_v;
-  float q = 0.f;
-#pragma unroll
-  for (int i = 0; i < NCH; ++i)
-    if (8 * (lane + 32 * i) < V)
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const float d = x[i][e] - mu;
-        q += d * d;
-      }
-  rstd = rsqrtf(warp_sum(q) * inv_v + eps);
 }
 
 // One warp's staged row stream: NT tensors, S stages of one row each.
@@ -208,15 +261,15 @@ __global__ void __launch_bounds__(kEpiThreads) k_epi_fwd(EpiArgs a) {
   const T *const src[2] = {(const T *)a.o, (const T *)a.r};
   const RowRing<T, 2> q = make_ring<T, 2>(a, smem, src);
   T *y = (T *)a.out0;
-  float wv[NCH][8], bv[NCH][8];
+  f2 wv[NCH][4], bv[NCH][4];
 #pragma unroll
   for (int i = 0; i < NCH; ++i) {
     const int c = 8 * (lane + 32 * i);
 #pragma unroll
-    for (int e = 0; e < 8; ++e) wv[i][e] = 1.f, bv[i][e] = 0.f;
+    for (int e = 0; e < 4; ++e) wv[i][e] = pk(1.f, 1.f), bv[i][e] = pk(0.f, 0.f);
     if (c < V) {
-      if (a.w) ld8(a.w + c, wv[i]);
-      if (a.b) ld8(a.b + c, bv[i]);
+      if (a.w) ldg8p(a.w + c, wv[i]);
+      if (a.b) ldg8p(a.b + c, bv[i]);
     }
   }
   const float inv_v = 1.f / (float)V;
@@ -229,26 +282,29 @@ __global__ void __launch_bounds__(kEpiThreads) k_epi_fwd(EpiArgs a) {
     }
     const long row = q.gw + j * q.nw;
     const T *so = reinterpret_cast<const T *>(q.stage(s)), *sr = so + V;
-    float x[NCH][8];
+    f2 x[NCH][4];
 #pragma unroll
     for (int i = 0; i < NCH; ++i) {
       const int c = 8 * (lane + 32 * i);
-      if (c < V) lds8(so + c, x[i]);
+      if (c < V) lds8p(so + c, x[i]);
     }
     float mu, rstd;
-    row_stats<NCH>(x, lane, V, inv_v, a.eps, mu, rstd);
+    row_stats2<NCH>(x, lane, V, inv_v, a.eps, mu, rstd);
+    const f2 nmu = pk(-mu, -mu), rs2 = pk(rstd, rstd);
 #pragma unroll
     for (int i = 0; i < NCH; ++i) {
       const int c = 8 * (lane + 32 * i);
       if (c < V) {
-        float rr[8], out[8];
-        lds8(sr + c, rr);
+        f2 rr[4], out[4];
+        lds8p(sr + c, rr);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const float n = (x[i][e] - mu) * rstd * wv[i][e] + bv[i][e];
-          out[e] = n * (rr[e] * sigm<T>(rr[e]));
+        for (int e = 0; e < 4; ++e) {
+          const f2 n = fma2(mul2(add2(x[i][e], nmu), rs2), wv[i][e], bv[i][e]);
+          f2 rsw, sg;
+          gate2<T>(rr[e], rsw, sg);
+          out[e] = mul2(n, rsw);
         }
-        st8(y + row * V + c, out);
+        st8p(y + row * V + c, out);
       }
     }
     __syncwarp();  // every lane has read the stage
@@ -273,11 +329,12 @@ __global__ void __launch_bounds__(kEpiThreads) k_epi_bwd(EpiArgs a) {
   // this warp's fp32 row of g = dn w, written in pass 1 and read in pass 2
   float *gs = reinterpret_cast<float *>(smem + (size_t)kEpiWarps * a.S * 3 * q.rowb) + (threadIdx.x >> 5) * V;
   T *dout = (T *)a.out0, *dr = (T *)a.out1;
-  float pw[NCH][8], pb[NCH][8];
+  f2 pw[NCH][4], pb[NCH][4];
 #pragma unroll
   for (int i = 0; i < NCH; ++i)
 #pragma unroll
-    for (int e = 0; e < 8; ++e) pw[i][e] = pb[i][e] = 0.f;
+    for (int e = 0; e < 4; ++e) pw[i][e] = pb[i][e] = pk(0.f, 0.f);
+  const f2 one = pk(1.f, 1.f), zero = pk(0.f, 0.f);
   const float inv_v = 1.f / (float)V;
   int s = 0;
   uint32_t ph = 0;
@@ -288,57 +345,62 @@ __global__ void __launch_bounds__(kEpiThreads) k_epi_bwd(EpiArgs a) {
     }
     const long row = q.gw + j * q.nw;
     const T *so = reinterpret_cast<const T *>(q.stage(s)), *sr = so + V, *sd = so + 2 * V;
-    float x[NCH][8];
+    f2 x[NCH][4];
 #pragma unroll
     for (int i = 0; i < NCH; ++i) {
       const int c = 8 * (lane + 32 * i);
-      if (c < V) lds8(so + c, x[i]);
+      if (c < V) lds8p(so + c, x[i]);
     }
     float mu, rstd;
-    row_stats<NCH>(x, lane, V, inv_v, a.eps, mu, rstd);
+    row_stats2<NCH>(x, lane, V, inv_v, a.eps, mu, rstd);
+    const f2 nmu = pk(-mu, -mu), rs2 = pk(rstd, rstd);
     // pass 1: dr, g (parked in gs), the dw / db partials and the row means of g
     // and g x^; x is replaced by x^
-    float m1 = 0.f, m2 = 0.f;
+    f2 m1 = zero, m2 = zero;
 #pragma unroll
     for (int i = 0; i < NCH; ++i) {
       const int c = 8 * (lane + 32 * i);
       if (c < V) {
-        float rv[8], gy[8], ww[8], bb[8], drv[8], gg[8];
-        lds8(sr + c, rv);
-        lds8(sd + c, gy);
-        if (a.w) ld8(a.w + c, ww);
-        if (a.b) ld8(a.b + c, bb);
+        f2 rv[4], gy[4], ww[4], bb[4], drv[4], gg[4];
+        lds8p(sr + c, rv);
+        lds8p(sd + c, gy);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const float xh = (x[i][e] - mu) * rstd;
-          const float we = a.w ? ww[e] : 1.f;
-          const float n = xh * we + (a.b ? bb[e] : 0.f);
-          const float sg = sigm<T>(rv[e]);
-          const float dn = gy[e] * (rv[e] * sg);
-          drv[e] = gy[e] * n * (sg * (1.f + rv[e] * (1.f - sg)));
-          pw[i][e] += dn * xh;
-          pb[i][e] += dn;
-          gg[e] = dn * we;
-          m1 += gg[e];
-          m2 += gg[e] * xh;
+        for (int e = 0; e < 4; ++e) ww[e] = one, bb[e] = zero;
+        if (a.w) ldg8p(a.w + c, ww);
+        if (a.b) ldg8p(a.b + c, bb);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const f2 xh = mul2(add2(x[i][e], nmu), rs2);
+          const f2 n = fma2(xh, ww[e], bb[e]);
+          f2 rsw, sg;
+          gate2<T>(rv[e], rsw, sg);
+          const f2 dn = mul2(gy[e], rsw);
+          // d(r sigmoid(r))/dr = sigmoid (1 + r (1 - sigmoid))
+          const f2 dsw = mul2(sg, fma2(rv[e], add2(one, mul2(sg, pk(-1.f, -1.f))), one));
+          drv[e] = mul2(mul2(gy[e], n), dsw);
+          pw[i][e] = fma2(dn, xh, pw[i][e]);
+          pb[i][e] = add2(pb[i][e], dn);
+          gg[e] = mul2(dn, ww[e]);
+          m1 = add2(m1, gg[e]);
+          m2 = fma2(gg[e], xh, m2);
           x[i][e] = xh;
         }
-        st8(dr + row * V + c, drv);
-        st8(gs + c, gg);
+        st8p(dr + row * V + c, drv);
+        st8p(gs + c, gg);
       }
     }
-    m1 = warp_sum(m1) * inv_v;
-    m2 = warp_sum(m2) * inv_v;
-    // pass 2: do (each lane reads back only the g it wrote)
+    const float m1s = warp_sum(hsum(m1)) * inv_v, m2s = warp_sum(hsum(m2)) * inv_v;
+    // pass 2: do = rstd g - rstd m1 - x^ (rstd m2), each lane reading back only its g
+    const f2 c1 = pk(-rstd * m1s, -rstd * m1s), c2 = pk(-rstd * m2s, -rstd * m2s);
 #pragma unroll
     for (int i = 0; i < NCH; ++i) {
       const int c = 8 * (lane + 32 * i);
       if (c < V) {
-        float gg[8], d[8];
-        lds8(gs + c, gg);
+        f2 gg[4], d[4];
+        lds8p(gs + c, gg);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) d[e] = rstd * (gg[e] - m1 - x[i][e] * m2);
-        st8(dout + row * V + c, d);
+        for (int e = 0; e < 4; ++e) d[e] = fma2(x[i][e], c2, fma2(gg[e], rs2, c1));
+        st8p(dout + row * V + c, d);
       }
     }
     __syncwarp();
@@ -357,21 +419,19 @@ __global__ void __launch_bounds__(kEpiThreads) k_epi_bwd(EpiArgs a) {
 #pragma unroll
   for (int i = 0; i < NCH; ++i) {
     const int c = 8 * (lane + 32 * i);
-    if (c < V)
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        mine[c + e] = pw[i][e];
-        mine[V + c + e] = pb[i][e];
-      }
+    if (c < V) {
+      st8p(mine + c, pw[i]);
+      st8p(mine + V + c, pb[i]);
+    }
   }
   __syncthreads();
   const size_t ring_floats = (size_t)a.S * 3 * q.rowb / sizeof(float);
   const float *all = reinterpret_cast<const float *>(smem);
   for (int idx = threadIdx.x; idx < 2 * V; idx += kEpiThreads) {
-    float s = 0.f;
+    float sum = 0.f;
 #pragma unroll
-    for (int w8 = 0; w8 < kEpiWarps; ++w8) s += all[w8 * ring_floats + idx];
-    a.part[(long)blockIdx.x * 2 * V + idx] = s;
+    for (int w8 = 0; w8 < kEpiWarps; ++w8) sum += all[w8 * ring_floats + idx];
+    a.part[(long)blockIdx.x * 2 * V + idx] = sum;
   }
 }
 
