@@ -7,15 +7,17 @@
 // (exp(B_t - B_s) with B the chunk-local cumulative log-gate, s <= t), so it is
 // stable for any gate strength.  All arithmetic is fp32 on CUDA cores.
 //
-// Kernels (grid-parallel over heads and chunks except the two state walks,
+// Kernels (grid-parallel over heads and chunks except the two state scans,
 // which are parallel over heads and state elements and sequential over chunks):
 //   prep     B[t,c]   chunk-local inclusive cumsum of log_alpha
-//   states   H[n]     state before chunk n (H[N] = final state)
+//   states   H[n]     state before chunk n (H[N] = final state): each chunk's
+//                     contribution as a tiled fp32 GEMM over its tokens, then a scan
 //   scores   P[n]     C x C causal intra-chunk scores
 //   out      o        (q (.) e^B) H[n] + P V
-//   dstates  dH[n]    adjoint of the state after chunk n
+//   dstates  dH[n]    adjoint of the state after chunk n (GEMMs, then a reverse scan)
 //   dscores  dP[n]    dO V^T (causal part)
-//   dqk      dq, dk, dlog_alpha (closed form, section 4.3, with the chunk
+//   dqk      dq, dk, dlog_alpha (inter terms as tiled GEMMs over d_v; closed form,
+//            section 4.3, with the chunk
 //            boundary term sum_v S_n[c,v] dS_n[c,v])
 //   dv       dv
 //
@@ -54,6 +56,8 @@ struct Dims {
   long Tp;
 };
 
+constexpr int kQkTile = 64, kQkRed = 32;  // output tile and staged reduction tile of the fp32 GEMMs
+
 // ---------------------------------------------------------------- forward
 
 // Bc[bh, t, c] = sum_{j in chunk(t), j <= t} log_alpha[bh, j, c]; rows t >= T add 0.
@@ -89,34 +93,118 @@ __global__ void k_prep_beta(const float *__restrict__ lb, Dims d, float *__restr
   }
 }
 
-// H[bh, n] = state before chunk n; H[bh, N] = final state.  Thread = (c, v).
-template <typename T>
-__global__ void k_states(const T *__restrict__ k, const T *__restrict__ v, const float *__restrict__ Bc,
-                         const float *__restrict__ Ec, const float *__restrict__ h0, Dims d,
-                         float *__restrict__ Hs, float *__restrict__ hT) {
-  const int vi = blockIdx.x * blockDim.x + threadIdx.x;
-  const int c = blockIdx.y * blockDim.y + threadIdx.y;
+// H[bh, n] = state before chunk n; H[bh, N] = final state: the chunk contributions
+// by k_chunk_kv<MODE 0>, composed by k_states_scan.
+
+// Chunk contributions over the chunk's tokens, a tiled fp32 GEMM per (chunk, head):
+//   MODE 0 (states):  D_n[c, v] = sum_t k_t[c] e^{B_last[c] - B_t[c]} v_t[v] e^{E_last[v] - E_t[v]},
+//                     written to Hs slot n + 1 (k_states_scan composes it)
+//   MODE 1 (adjoints): D_n[c, v] = sum_t q_t[c] e^{B_t[c]} do_t[v] e^{E_t[v]},
+//                     written to dHs slot n (k_dstates_scan composes it)
+// CTA = 64 key x 64 value channels; token tiles of 32 staged in shared memory with
+// coalesced loads, each exp factor applied once per staged element; 256 threads,
+// 4 x 4 outputs each.  grid: x = chunk, y = channel tile, z = head.
+template <typename T, int MODE>
+__global__ void __launch_bounds__(256) k_chunk_kv(const T *__restrict__ a, const T *__restrict__ b,
+                                                  const float *__restrict__ Bc, const float *__restrict__ Ec, Dims d,
+                                                  float *__restrict__ out) {
+  __shared__ float Xs[kQkRed][kQkTile + 1];  // [t][c]
+  __shared__ float Ys[kQkRed][kQkTile + 1];  // [t][v]
+  const int n = blockIdx.x;
+  const int ctiles = (d.K + kQkTile - 1) / kQkTile;
+  const int c0 = (blockIdx.y % ctiles) * kQkTile, v0 = (blockIdx.y / ctiles) * kQkTile;
   const long bh = blockIdx.z;
-  if (vi >= d.V || c >= d.K) return;
   const long KV = (long)d.K * d.V;
-  float S = h0 ? h0[bh * KV + (long)c * d.V + vi] : 0.f;
-  for (int n = 0; n < d.N; ++n) {
-    Hs[(bh * (d.N + 1) + n) * KV + (long)c * d.V + vi] = S;
-    const float blast = Bc[(bh * d.Tp + (long)n * d.C + d.C - 1) * d.K + c];
-    const float elast = Ec ? Ec[(bh * d.Tp + (long)n * d.C + d.C - 1) * d.V + vi] : 0.f;
-    float acc = 0.f;
-    for (int j = 0; j < d.C; ++j) {
-      const long t = (long)n * d.C + j;
-      if (t >= d.T) break;
-      const float kk = ld(k + (bh * d.T + t) * d.K + c);
-      float w = __expf(blast - Bc[(bh * d.Tp + t) * d.K + c]);
-      if (Ec) w *= __expf(elast - Ec[(bh * d.Tp + t) * d.V + vi]);
-      acc += kk * w * ld(v + (bh * d.T + t) * d.V + vi);
+  const long last = bh * d.Tp + (long)n * d.C + d.C - 1;
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  float acc[4][4] = {};
+  for (int j0 = 0; j0 < d.C; j0 += kQkRed) {
+    for (int idx = threadIdx.x; idx < kQkRed * kQkTile; idx += 256) {
+      const int j = idx / kQkTile, r = idx % kQkTile;
+      const long t = (long)n * d.C + j0 + j;
+      const bool ok = j0 + j < d.C && t < d.T;
+      float x = 0.f, y = 0.f;
+      if (ok && c0 + r < d.K) {
+        const float Bt = Bc[(bh * d.Tp + t) * d.K + c0 + r];
+        x = ld(a + (bh * d.T + t) * d.K + c0 + r) * __expf(MODE == 0 ? Bc[last * d.K + c0 + r] - Bt : Bt);
+      }
+      if (ok && v0 + r < d.V) {
+        y = ld(b + (bh * d.T + t) * d.V + v0 + r);
+        if (Ec) {
+          const float Et = Ec[(bh * d.Tp + t) * d.V + v0 + r];
+          y *= __expf(MODE == 0 ? Ec[last * d.V + v0 + r] - Et : Et);
+        }
+      }
+      Xs[j][r] = x;
+      Ys[j][r] = y;
     }
-    S = __expf(blast + elast) * S + acc;
+    __syncthreads();
+#pragma unroll 8
+    for (int j = 0; j < kQkRed; ++j) {
+      float xa[4], ya[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) xa[u] = Xs[j][4 * ty + u], ya[u] = Ys[j][4 * tx + u];
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int w = 0; w < 4; ++w) acc[u][w] += xa[u] * ya[w];
+    }
+    __syncthreads();
   }
-  Hs[(bh * (d.N + 1) + d.N) * KV + (long)c * d.V + vi] = S;
-  if (hT) hT[bh * KV + (long)c * d.V + vi] = S;
+  float *D = out + (MODE == 0 ? bh * (d.N + 1) + n + 1 : bh * d.N + n) * KV;
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int c = c0 + 4 * ty + u;
+    if (c >= d.K) continue;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      const int vv = v0 + 4 * tx + w;
+      if (vv < d.V) D[(long)c * d.V + vv] = acc[u][w];
+    }
+  }
+}
+
+// Forward scan over chunks, in place: Hs[0] = h0; Hs[n+1] = e^{B_last+E_last} Hs[n] + D_n.
+__global__ void k_states_scan(const float *__restrict__ Bc, const float *__restrict__ Ec,
+                              const float *__restrict__ h0, Dims d, float *__restrict__ Hs,
+                              float *__restrict__ hT) {
+  const long KV = (long)d.K * d.V;
+  const long i = (long)blockIdx.x * blockDim.x + threadIdx.x;  // c * V + v
+  const long bh = blockIdx.y;
+  if (i >= KV) return;
+  const int c = (int)(i / d.V), vi = (int)(i % d.V);
+  float *H = Hs + bh * (d.N + 1) * KV + i;
+  float S = h0 ? h0[bh * KV + i] : 0.f;
+  H[0] = S;
+  for (int n = 0; n < d.N; ++n) {
+    const long last = bh * d.Tp + (long)n * d.C + d.C - 1;
+    const float g = Bc[last * d.K + c] + (Ec ? Ec[last * d.V + vi] : 0.f);
+    S = __expf(g) * S + H[(long)(n + 1) * KV];
+    H[(long)(n + 1) * KV] = S;
+  }
+  if (hT) hT[bh * KV + i] = S;
+}
+
+// Reverse scan, in place: dHs[n] holds D_n on entry; dHs[N-1] = dh_final,
+// dHs[n-1] = e^{B_last,n + E_last,n} dHs[n] + D_n, dh0 = e^{...0} dHs[0] + D_0.
+__global__ void k_dstates_scan(const float *__restrict__ Bc, const float *__restrict__ Ec,
+                               const float *__restrict__ dhT, Dims d, float *__restrict__ dHs,
+                               float *__restrict__ dh0) {
+  const long KV = (long)d.K * d.V;
+  const long i = (long)blockIdx.x * blockDim.x + threadIdx.x;
+  const long bh = blockIdx.y;
+  if (i >= KV) return;
+  const int c = (int)(i / d.V), vi = (int)(i % d.V);
+  float *dH = dHs + bh * d.N * KV + i;
+  float dS = dhT ? dhT[bh * KV + i] : 0.f;
+  for (int n = d.N - 1; n >= 0; --n) {
+    const float Dn = dH[(long)n * KV];
+    dH[(long)n * KV] = dS;
+    const long last = bh * d.Tp + (long)n * d.C + d.C - 1;
+    const float g = Bc[last * d.K + c] + (Ec ? Ec[last * d.V + vi] : 0.f);
+    dS = __expf(g) * dS + Dn;
+  }
+  if (dh0) dh0[bh * KV + i] = dS;
 }
 
 // P[bh, n, t, s] = sum_c q_t[c] k_s[c] exp(B_t[c] - B_s[c]) for s <= t, else 0.
@@ -174,34 +262,8 @@ __global__ void k_out(const T *__restrict__ q, const T *__restrict__ v, const fl
 
 // ---------------------------------------------------------------- backward
 
-// dH[bh, n] = adjoint of the state after chunk n (through chunks > n and dh_final).
-template <typename T>
-__global__ void k_dstates(const T *__restrict__ q, const T *__restrict__ dout, const float *__restrict__ Bc,
-                          const float *__restrict__ Ec, const float *__restrict__ dhT, Dims d,
-                          float *__restrict__ dHs, float *__restrict__ dh0) {
-  const int vi = blockIdx.x * blockDim.x + threadIdx.x;
-  const int c = blockIdx.y * blockDim.y + threadIdx.y;
-  const long bh = blockIdx.z;
-  if (vi >= d.V || c >= d.K) return;
-  const long KV = (long)d.K * d.V;
-  float dS = dhT ? dhT[bh * KV + (long)c * d.V + vi] : 0.f;
-  for (int n = d.N - 1; n >= 0; --n) {
-    dHs[(bh * d.N + n) * KV + (long)c * d.V + vi] = dS;
-    const float blast = Bc[(bh * d.Tp + (long)n * d.C + d.C - 1) * d.K + c];
-    const float elast = Ec ? Ec[(bh * d.Tp + (long)n * d.C + d.C - 1) * d.V + vi] : 0.f;
-    float acc = 0.f;
-    for (int j = 0; j < d.C; ++j) {
-      const long t = (long)n * d.C + j;
-      if (t >= d.T) break;
-      float x = ld(q + (bh * d.T + t) * d.K + c) * __expf(Bc[(bh * d.Tp + t) * d.K + c]) *
-                ld(dout + (bh * d.T + t) * d.V + vi);
-      if (Ec) x *= __expf(Ec[(bh * d.Tp + t) * d.V + vi]);
-      acc += x;
-    }
-    dS = __expf(blast + elast) * dS + acc;
-  }
-  if (dh0) dh0[bh * KV + (long)c * d.V + vi] = dS;
-}
+// dH[bh, n] = adjoint of the state after chunk n (through chunks > n and dh_final):
+// the chunk contributions by k_chunk_kv<MODE 1>, composed by k_dstates_scan.
 
 // dP[bh, n, t, s] = sum_v do_t[v] v_s[v] (e^{E_t[v] - E_s[v]}) for s <= t, else 0.
 template <typename T>
@@ -225,24 +287,93 @@ __global__ void k_dscores(const T *__restrict__ dout, const T *__restrict__ v, c
   }
 }
 
+// Inter-chunk terms of dq and dk, contractions over the d_v channels per chunk n:
+//   A1[t, c] = sum_v do_t[v] e^{E_t[v]} H[n][c, v]
+//   A2[t, c] = sum_v v_t[v] e^{E_last[v] - E_t[v]} dH[n][c, v]
+// (E null: no factors).  A tiled fp32 GEMM: CTA = 64 tokens x 64 channels of one
+// chunk, head and term; operand tiles of 32 value channels staged in shared memory
+// with coalesced loads (each exp factor applied once per staged element); 256
+// threads, 4 x 4 outputs each.
+template <typename T>
+__global__ void __launch_bounds__(256) k_inter_qk(const T *__restrict__ dout, const T *__restrict__ v,
+                                                  const float *__restrict__ Ec, const float *__restrict__ Hs,
+                                                  const float *__restrict__ dHs, Dims d, float *__restrict__ A1,
+                                                  float *__restrict__ A2) {
+  __shared__ float Xs[kQkRed][kQkTile + 1];  // [j][t]
+  __shared__ float Ys[kQkRed][kQkTile + 1];  // [j][c]
+  const int tpc = (d.C + kQkTile - 1) / kQkTile;  // token tiles per chunk
+  // grid: x = chunk x token tile, y = channel tile x term, z = head
+  const int n = blockIdx.x / tpc, t0 = (blockIdx.x % tpc) * kQkTile;
+  const long bh = blockIdx.z;
+  const int which = blockIdx.y & 1;  // 0: A1 (do, H), 1: A2 (v, dH)
+  const int c0 = (blockIdx.y >> 1) * kQkTile;
+  const long KV = (long)d.K * d.V;
+  const T *X = which ? v : dout;
+  const float *M = which ? dHs + (bh * d.N + n) * KV : Hs + (bh * (d.N + 1) + n) * KV;
+  const float *El = Ec ? Ec + (bh * d.Tp + (long)n * d.C + d.C - 1) * d.V : nullptr;
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  float acc[4][4] = {};
+  for (int j0 = 0; j0 < d.V; j0 += kQkRed) {
+    for (int idx = threadIdx.x; idx < kQkTile * kQkRed; idx += 256) {
+      const int r = idx / kQkRed, j = idx % kQkRed;
+      const int ti = t0 + r;
+      const long t = (long)n * d.C + ti;
+      float x = 0.f;
+      if (ti < d.C && t < d.T && j0 + j < d.V) {
+        x = ld(X + (bh * d.T + t) * d.V + j0 + j);
+        if (Ec) {
+          const float Et = Ec[(bh * d.Tp + t) * d.V + j0 + j];
+          x *= __expf(which ? El[j0 + j] - Et : Et);
+        }
+      }
+      Xs[j][r] = x;
+      Ys[j][r] = (c0 + r < d.K && j0 + j < d.V) ? M[(long)(c0 + r) * d.V + j0 + j] : 0.f;
+    }
+    __syncthreads();
+#pragma unroll 8
+    for (int j = 0; j < kQkRed; ++j) {
+      float xa[4], ya[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) xa[u] = Xs[j][4 * ty + u], ya[u] = Ys[j][4 * tx + u];
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int w = 0; w < 4; ++w) acc[u][w] += xa[u] * ya[w];
+    }
+    __syncthreads();
+  }
+  float *A = which ? A2 : A1;
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int ti = t0 + 4 * ty + u;
+    if (ti >= d.C) continue;
+    const long t = (long)n * d.C + ti;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      const int c = c0 + 4 * tx + w;
+      if (c < d.K) A[(bh * d.Tp + t) * d.K + c] = acc[u][w];
+    }
+  }
+}
+
 // One block per (chunk, head), one thread per key channel c:
 //   dq_t = e^{B_t} (do_t H[n]^T) + sum_{s<=t} dP[t,s] k_s e^{B_t - B_s}
 //   dk_t = e^{B_last - B_t} (v_t dH[n]^T) + sum_{s>=t} dP[s,t] q_s e^{B_s - B_t}
+// with the two contractions over d_v (A1, A2) from k_inter_qk
 //   dlog b_t = q_t dq_t - k_t dk_t   (closed form, section 4.3)
 //   dlog alpha_t = sum_{i >= t in chunk} dlog b_i + G_n,  G_n[c] = sum_v S_n[c,v] dS_n[c,v]
 // (S_n = H[n+1] the state after chunk n, dS_n = dH[n] its adjoint), which is the
 // suffix of dlog b beyond the chunk, so no cross-chunk scan is needed.
 template <typename T>
-__global__ void k_dqk(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
-                      const T *__restrict__ dout, const float *__restrict__ Bc, const float *__restrict__ Ec,
-                      const float *__restrict__ Hs, const float *__restrict__ dHs, const float *__restrict__ dP,
-                      Dims d, T *__restrict__ dq, T *__restrict__ dk, float *__restrict__ dgv) {
+__global__ void k_dqk(const T *__restrict__ q, const T *__restrict__ k,
+                      const float *__restrict__ Bc, const float *__restrict__ Hs, const float *__restrict__ dHs,
+                      const float *__restrict__ dP, const float *__restrict__ A1, const float *__restrict__ A2, Dims d,
+                      T *__restrict__ dq, T *__restrict__ dk, float *__restrict__ dgv) {
   const int c = threadIdx.x;
   if (c >= d.K) return;
   const long bh = blockIdx.y;
   const int n = blockIdx.x;
   const long KV = (long)d.K * d.V;
-  const float *H = Hs + (bh * (d.N + 1) + n) * KV + (long)c * d.V;
   const float *Hn = Hs + (bh * (d.N + 1) + n + 1) * KV + (long)c * d.V;
   const float *dH = dHs + (bh * d.N + n) * KV + (long)c * d.V;
   const float *dPc = dP + (bh * d.N + n) * (long)d.C * d.C;
@@ -254,20 +385,7 @@ __global__ void k_dqk(const T *__restrict__ q, const T *__restrict__ k, const T 
     const long t = (long)n * d.C + ti;
     if (t >= d.T) break;
     const float Bt = Bc[(bh * d.Tp + t) * d.K + c];
-    float a1 = 0.f, a2 = 0.f;
-    if (Ec) {
-      const float *Et = Ec + (bh * d.Tp + t) * d.V;
-      const float *El = Ec + (bh * d.Tp + (long)n * d.C + d.C - 1) * d.V;
-      for (int j = 0; j < d.V; ++j) {
-        a1 += ld(dout + (bh * d.T + t) * d.V + j) * H[j] * __expf(Et[j]);
-        a2 += ld(v + (bh * d.T + t) * d.V + j) * dH[j] * __expf(El[j] - Et[j]);
-      }
-    } else {
-      for (int j = 0; j < d.V; ++j) {
-        a1 += ld(dout + (bh * d.T + t) * d.V + j) * H[j];
-        a2 += ld(v + (bh * d.T + t) * d.V + j) * dH[j];
-      }
-    }
+    const float a1 = A1[(bh * d.Tp + t) * d.K + c], a2 = A2[(bh * d.Tp + t) * d.K + c];
     float dqv = __expf(Bt) * a1;
     float dkv = __expf(blast - Bt) * a2;
     for (int si = 0; si <= ti; ++si) {
@@ -378,7 +496,7 @@ __global__ void k_dg_out(const float *__restrict__ dgv, Dims d, float *__restric
 Dims dims_of(const Problem &p) { return Dims{p.T, p.K, p.V, p.C, p.N, p.gate, p.Tp}; }
 
 struct F32Ws {
-  float *Bc, *Hs, *P, *dHs, *dP, *dgv;
+  float *Bc, *Hs, *P, *dHs, *dP, *dgv, *A1, *A2;
   float *Ec, *of, *dvf;  // general gate only
   size_t bytes;
 };
@@ -393,6 +511,8 @@ F32Ws carve(const Problem &p, void *ws, bool bwd, bool general) {
     w.dHs = cv.take<float>((size_t)p.BH * p.N * p.K * p.V);
     w.dP = cv.take<float>((size_t)p.BH * p.N * p.C * p.C);
     w.dgv = cv.take<float>((size_t)p.BH * p.Tp * p.K);
+    w.A1 = cv.take<float>((size_t)p.BH * p.Tp * p.K);
+    w.A2 = cv.take<float>((size_t)p.BH * p.Tp * p.K);
   }
   if (general) {
     w.Ec = cv.take<float>((size_t)p.BH * p.Tp * p.V);
@@ -405,6 +525,30 @@ F32Ws carve(const Problem &p, void *ws, bool bwd, bool general) {
   return w;
 }
 
+// States (Hs, and h_final if hT) and state adjoints (dHs, dh0): per-chunk GEMMs, then scans.
+template <typename T>
+int launch_states(const Problem &p, const Dims &d, const T *k, const T *v, const F32Ws &w, const float *h0,
+                  float *hT, cudaStream_t st) {
+  const dim3 grid(p.N, ((p.K + kQkTile - 1) / kQkTile) * ((p.V + kQkTile - 1) / kQkTile), p.BH);
+  GLA_LAUNCH(K_F32_STATES, st, (k_chunk_kv<T, 0><<<grid, 256, 0, st>>>(k, v, w.Bc, w.Ec, d, w.Hs)));
+  const long KV = (long)p.K * p.V;
+  GLA_LAUNCH(K_F32_STATES, st,
+             (k_states_scan<<<dim3((unsigned)((KV + 255) / 256), p.BH), 256, 0, st>>>(w.Bc, w.Ec, h0, d, w.Hs, hT)));
+  return GLA_OK;
+}
+
+template <typename T>
+int launch_dstates(const Problem &p, const Dims &d, const T *q, const T *dout, const F32Ws &w, const float *dhT,
+                   float *dh0, cudaStream_t st) {
+  const dim3 grid(p.N, ((p.K + kQkTile - 1) / kQkTile) * ((p.V + kQkTile - 1) / kQkTile), p.BH);
+  GLA_LAUNCH(K_F32_DSTATES, st, (k_chunk_kv<T, 1><<<grid, 256, 0, st>>>(q, dout, w.Bc, w.Ec, d, w.dHs)));
+  const long KV = (long)p.K * p.V;
+  GLA_LAUNCH(K_F32_DSTATES, st,
+             (k_dstates_scan<<<dim3((unsigned)((KV + 255) / 256), p.BH), 256, 0, st>>>(w.Bc, w.Ec, dhT, d, w.dHs,
+                                                                                       dh0)));
+  return GLA_OK;
+}
+
 template <typename T>
 int fwd_impl(const Problem &p, const T *q, const T *k, const T *v, const float *la, const float *lb, const float *h0,
              T *o, float *hT, void *ws, cudaStream_t st) {
@@ -413,9 +557,7 @@ int fwd_impl(const Problem &p, const T *q, const T *k, const T *v, const float *
   const int kth = (p.K + 31) / 32 * 32;
   GLA_LAUNCH(K_F32_PREP, st, (k_prep<<<dim3(p.N, p.BH), kth, 0, st>>>(la, d, w.Bc)));
   if (lb) GLA_LAUNCH(K_F32_PREP, st, (k_prep_beta<<<dim3(p.N, p.BH), 256, 0, st>>>(lb, d, w.Ec)));
-  GLA_LAUNCH(K_F32_STATES, st,
-             (k_states<T><<<dim3((p.V + 31) / 32, (p.K + 7) / 8, p.BH), dim3(32, 8), 0, st>>>(k, v, w.Bc, w.Ec, h0, d,
-                                                                                              w.Hs, hT)));
+  if (const int r = launch_states<T>(p, d, k, v, w, h0, hT, st)) return r;
   GLA_LAUNCH(K_F32_SCORES, st, (k_scores<T><<<dim3(p.N, p.BH), 256, 0, st>>>(q, k, w.Bc, d, w.P)));
   GLA_LAUNCH(K_F32_OUT, st,
              (k_out<T, T><<<dim3((p.V + 63) / 64, p.N, p.BH), dim3(64, 4), 0, st>>>(q, v, w.Bc, w.Ec, w.Hs, w.P, d,
@@ -432,16 +574,15 @@ int bwd_impl(const Problem &p, const T *q, const T *k, const T *v, const float *
   const int kth = (p.K + 31) / 32 * 32;
   GLA_LAUNCH(K_F32_PREP, st, (k_prep<<<dim3(p.N, p.BH), kth, 0, st>>>(la, d, w.Bc)));
   if (lb) GLA_LAUNCH(K_F32_PREP, st, (k_prep_beta<<<dim3(p.N, p.BH), 256, 0, st>>>(lb, d, w.Ec)));
-  GLA_LAUNCH(K_F32_STATES, st,
-             (k_states<T><<<dim3((p.V + 31) / 32, (p.K + 7) / 8, p.BH), dim3(32, 8), 0, st>>>(k, v, w.Bc, w.Ec, h0, d,
-                                                                                              w.Hs, nullptr)));
+  if (const int r = launch_states<T>(p, d, k, v, w, h0, nullptr, st)) return r;
   GLA_LAUNCH(K_F32_SCORES, st, (k_scores<T><<<dim3(p.N, p.BH), 256, 0, st>>>(q, k, w.Bc, d, w.P)));
-  GLA_LAUNCH(K_F32_DSTATES, st,
-             (k_dstates<T><<<dim3((p.V + 31) / 32, (p.K + 7) / 8, p.BH), dim3(32, 8), 0, st>>>(q, dout, w.Bc, w.Ec,
-                                                                                               dhT, d, w.dHs, dh0)));
+  if (const int r = launch_dstates<T>(p, d, q, dout, w, dhT, dh0, st)) return r;
   GLA_LAUNCH(K_F32_DSCORES, st, (k_dscores<T><<<dim3(p.N, p.BH), 256, 0, st>>>(dout, v, w.Ec, d, w.dP)));
   GLA_LAUNCH(K_F32_DQK, st,
-             (k_dqk<T><<<dim3(p.N, p.BH), kth, 0, st>>>(q, k, v, dout, w.Bc, w.Ec, w.Hs, w.dHs, w.dP, d, dq, dk,
+             (k_inter_qk<T><<<dim3(p.N * ((p.C + kQkTile - 1) / kQkTile), 2 * ((p.K + kQkTile - 1) / kQkTile), p.BH), 256,
+                              0, st>>>(dout, v, w.Ec, w.Hs, w.dHs, d, w.A1, w.A2)));
+  GLA_LAUNCH(K_F32_DQK, st,
+             (k_dqk<T><<<dim3(p.N, p.BH), kth, 0, st>>>(q, k, w.Bc, w.Hs, w.dHs, w.dP, w.A1, w.A2, d, dq, dk,
                                                          w.dgv)));
   GLA_LAUNCH(K_F32_DV, st,
              (k_dv<T><<<dim3((p.V + 63) / 64, p.N, p.BH), dim3(64, 4), 0, st>>>(k, dout, w.Bc, w.Ec, w.dHs, w.P, d, dv,
