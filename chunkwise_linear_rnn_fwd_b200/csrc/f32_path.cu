@@ -12,7 +12,7 @@
 //   prep     B[t,c]   chunk-local inclusive cumsum of log_alpha
 //   states   H[n]     state before chunk n (H[N] = final state): each chunk's
 //                     contribution as a tiled fp32 GEMM over its tokens, then a scan
-//   scores   P[n]     C x C causal intra-chunk scores
+//   scores   P[n]     C x C causal intra-chunk scores (pairs staged in shared memory)
 //   out      o        (q (.) e^B) H[n] + P V
 //   dstates  dH[n]    adjoint of the state after chunk n (GEMMs, then a reverse scan)
 //   dscores  dP[n]    dO V^T (causal part)
@@ -207,56 +207,174 @@ __global__ void k_dstates_scan(const float *__restrict__ Bc, const float *__rest
   if (dh0) dh0[bh * KV + i] = dS;
 }
 
-// P[bh, n, t, s] = sum_c q_t[c] k_s[c] exp(B_t[c] - B_s[c]) for s <= t, else 0.
-template <typename T>
-__global__ void k_scores(const T *__restrict__ q, const T *__restrict__ k, const float *__restrict__ Bc,
-                         Dims d, float *__restrict__ P) {
+// Causal pair sums of one chunk, staged in shared memory:
+//   MODE 0 (scores):  P[t, s]  = sum_c q_t[c] k_s[c] e^{B_t[c] - B_s[c]}      (c < d_k)
+//   MODE 1 (dscores): dP[t, s] = sum_v do_t[v] v_s[v] (e^{E_t[v] - E_s[v]})   (v < d_v)
+// for s <= t (0 elsewhere), every pair in log space as before.  CTA = a 64 x 64 tile
+// of the chunk's (t, s) pairs; slices of 32 channels of both operands and of the
+// cumulative gates staged with coalesced loads; 256 threads, 4 x 4 pairs each; tiles
+// and micro-tiles wholly above the diagonal skip the arithmetic.
+template <typename T, int MODE>
+__global__ void __launch_bounds__(256) k_pairs(const T *__restrict__ a, const T *__restrict__ b,
+                                               const float *__restrict__ G, Dims d, float *__restrict__ out) {
+  __shared__ float As[kQkRed][kQkTile + 1], Bs[kQkRed][kQkTile + 1];  // [channel][row]
+  __shared__ float Ga[kQkRed][kQkTile + 1], Gb[kQkRed][kQkTile + 1];
+  const int W = MODE == 0 ? d.K : d.V;
+  const int tiles = (d.C + kQkTile - 1) / kQkTile;
+  const int n = blockIdx.x / (tiles * tiles);
+  const int t0 = ((blockIdx.x / tiles) % tiles) * kQkTile, s0 = (blockIdx.x % tiles) * kQkTile;
   const long bh = blockIdx.y;
-  const int n = blockIdx.x;
-  for (int idx = threadIdx.x; idx < d.C * d.C; idx += blockDim.x) {
-    const int ti = idx / d.C, si = idx % d.C;
-    const long t = (long)n * d.C + ti, s = (long)n * d.C + si;
-    float acc = 0.f;
-    if (si <= ti && t < d.T) {
-      for (int c = 0; c < d.K; ++c) {
-        const float e = __expf(Bc[(bh * d.Tp + t) * d.K + c] - Bc[(bh * d.Tp + s) * d.K + c]);
-        acc += ld(q + (bh * d.T + t) * d.K + c) * ld(k + (bh * d.T + s) * d.K + c) * e;
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  float *Pc = out + (bh * d.N + n) * (long)d.C * d.C;
+  float acc[4][4] = {};
+  const bool tile_live = s0 <= t0 + kQkTile - 1;
+  const bool live = tile_live && s0 + 4 * tx <= t0 + 4 * ty + 3;
+  if (tile_live) {
+    for (int c0 = 0; c0 < W; c0 += kQkRed) {
+      for (int idx = threadIdx.x; idx < kQkTile * kQkRed; idx += 256) {
+        const int r = idx / kQkRed, c = idx % kQkRed;
+        const long t = (long)n * d.C + t0 + r, s = (long)n * d.C + s0 + r;
+        const bool okc = c0 + c < W;
+        const bool okt = okc && t0 + r < d.C && t < d.T, oks = okc && s0 + r < d.C && s < d.T;
+        As[c][r] = okt ? ld(a + (bh * d.T + t) * W + c0 + c) : 0.f;
+        Bs[c][r] = oks ? ld(b + (bh * d.T + s) * W + c0 + c) : 0.f;
+        if (G) {
+          Ga[c][r] = okt ? G[(bh * d.Tp + t) * W + c0 + c] : 0.f;
+          Gb[c][r] = oks ? G[(bh * d.Tp + s) * W + c0 + c] : 0.f;
+        }
       }
+      __syncthreads();
+      if (live) {
+#pragma unroll 4
+        for (int c = 0; c < kQkRed; ++c) {
+          float xa[4], xb[4], ga[4], gb[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            xa[u] = As[c][4 * ty + u];
+            xb[u] = Bs[c][4 * tx + u];
+            ga[u] = G ? Ga[c][4 * ty + u] : 0.f;
+            gb[u] = G ? Gb[c][4 * tx + u] : 0.f;
+          }
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+#pragma unroll
+            for (int w = 0; w < 4; ++w) acc[u][w] += G ? xa[u] * xb[w] * __expf(ga[u] - gb[w]) : xa[u] * xb[w];
+        }
+      }
+      __syncthreads();
     }
-    P[((bh * d.N + n) * d.C + ti) * d.C + si] = acc;
+  }
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int ti = t0 + 4 * ty + u;
+    if (ti >= d.C) continue;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      const int si = s0 + 4 * tx + w;
+      if (si < d.C) Pc[(long)ti * d.C + si] = (si <= ti && (long)n * d.C + ti < d.T) ? acc[u][w] : 0.f;
+    }
   }
 }
 
-// o[t, v] = sum_c q_t[c] e^{B_t[c]} H[n][c, v] + sum_{s<=t} P[t, s] v_s[v]
-// (general gate: the first term times e^{E_t[v]}, the pairs times e^{E_t[v] - E_s[v]})
+// o[t, v] = e^{E_t[v]} sum_c q_t[c] e^{B_t[c]} H[n][c, v]
+//         + sum_{s<=t} P[t, s] v_s[v] e^{E_t[v] - E_s[v]}          (E null: no E factors)
+// CTA = 64 tokens x 64 value channels of one chunk; the first term a staged GEMM over
+// d_k, the second over the chunk's tokens with P, v and E staged; the causal mask is
+// applied before the exponential (for s > t, E_t - E_s > 0 could overflow).  256
+// threads, 4 x 4 outputs each.  grid: x = chunk x token tile x value tile, y = head.
 template <typename T, typename TO>
-__global__ void k_out(const T *__restrict__ q, const T *__restrict__ v, const float *__restrict__ Bc,
-                      const float *__restrict__ Ec, const float *__restrict__ Hs, const float *__restrict__ P,
-                      Dims d, TO *__restrict__ o) {
-  const int vi = blockIdx.x * blockDim.x + threadIdx.x;
-  const int n = blockIdx.y;
-  const long bh = blockIdx.z;
-  if (vi >= d.V) return;
+__global__ void __launch_bounds__(256) k_out(const T *__restrict__ q, const T *__restrict__ v,
+                                             const float *__restrict__ Bc, const float *__restrict__ Ec,
+                                             const float *__restrict__ Hs, const float *__restrict__ P, Dims d,
+                                             TO *__restrict__ o) {
+  __shared__ float Xs[kQkRed][kQkTile + 1], Ys[kQkRed][kQkTile + 1], Zs[kQkRed][kQkTile + 1];
+  const int ttiles = (d.C + kQkTile - 1) / kQkTile, vtiles = (d.V + kQkTile - 1) / kQkTile;
+  const int n = blockIdx.x / (ttiles * vtiles);
+  const int t0 = ((blockIdx.x / vtiles) % ttiles) * kQkTile, v0 = (blockIdx.x % vtiles) * kQkTile;
+  const long bh = blockIdx.y;
   const long KV = (long)d.K * d.V;
   const float *H = Hs + (bh * (d.N + 1) + n) * KV;
-  for (int ti = threadIdx.y; ti < d.C; ti += blockDim.y) {
-    const long t = (long)n * d.C + ti;
-    if (t >= d.T) break;
-    float acc = 0.f;
-    for (int c = 0; c < d.K; ++c)
-      acc += ld(q + (bh * d.T + t) * d.K + c) * __expf(Bc[(bh * d.Tp + t) * d.K + c]) * H[(long)c * d.V + vi];
-    const float *Pr = P + ((bh * d.N + n) * d.C + ti) * d.C;
-    if (Ec) {
-      const float Et = Ec[(bh * d.Tp + t) * d.V + vi];
-      acc *= __expf(Et);
-      for (int si = 0; si <= ti; ++si) {
-        const long s = (long)n * d.C + si;
-        acc += Pr[si] * ld(v + (bh * d.T + s) * d.V + vi) * __expf(Et - Ec[(bh * d.Tp + s) * d.V + vi]);
-      }
-    } else {
-      for (int si = 0; si <= ti; ++si) acc += Pr[si] * ld(v + (bh * d.T + (long)n * d.C + si) * d.V + vi);
+  const float *Pc = P + (bh * d.N + n) * (long)d.C * d.C;
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  float acc[4][4] = {};
+  // inter: staged q e^{B} [c][t] and H [c][v]
+  for (int c0 = 0; c0 < d.K; c0 += kQkRed) {
+    for (int idx = threadIdx.x; idx < kQkTile * kQkRed; idx += 256) {
+      const int r = idx / kQkRed, c = idx % kQkRed;
+      const long t = (long)n * d.C + t0 + r;
+      const bool okc = c0 + c < d.K;
+      Xs[c][r] = (okc && t0 + r < d.C && t < d.T)
+                     ? ld(q + (bh * d.T + t) * d.K + c0 + c) * __expf(Bc[(bh * d.Tp + t) * d.K + c0 + c])
+                     : 0.f;
+      const int cc = idx / kQkTile, vv = idx % kQkTile;  // H slice, coalesced along v
+      Ys[cc][vv] = (c0 + cc < d.K && v0 + vv < d.V) ? H[(long)(c0 + cc) * d.V + v0 + vv] : 0.f;
     }
-    st(o + (bh * d.T + t) * d.V + vi, acc);
+    __syncthreads();
+#pragma unroll 8
+    for (int c = 0; c < kQkRed; ++c) {
+      float xa[4], ya[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) xa[u] = Xs[c][4 * ty + u], ya[u] = Ys[c][4 * tx + u];
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int w = 0; w < 4; ++w) acc[u][w] += xa[u] * ya[w];
+    }
+    __syncthreads();
+  }
+  float Et[4][4] = {};
+  if (Ec) {
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const long t = (long)n * d.C + t0 + 4 * ty + u;
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        const int vv = v0 + 4 * tx + w;
+        Et[u][w] = (t0 + 4 * ty + u < d.C && t < d.T && vv < d.V) ? Ec[(bh * d.Tp + t) * d.V + vv] : 0.f;
+        acc[u][w] *= __expf(Et[u][w]);
+      }
+    }
+  }
+  // intra: staged P [s][t], v [s][v] and E [s][v] over the chunk's tokens s
+  const int s_end = min(d.C, t0 + kQkTile);
+  for (int s0 = 0; s0 < s_end; s0 += kQkRed) {
+    for (int idx = threadIdx.x; idx < kQkTile * kQkRed; idx += 256) {
+      const int r = idx % kQkTile, j = idx / kQkTile;  // P slice: row t = t0 + r, column s0 + j
+      const int sj = s0 + j;
+      const long sg = (long)n * d.C + sj;
+      Xs[j][r] = (sj < d.C && t0 + r < d.C) ? Pc[(long)(t0 + r) * d.C + sj] : 0.f;
+      const bool oks = sj < d.C && sg < d.T && v0 + r < d.V;
+      Ys[j][r] = oks ? ld(v + (bh * d.T + sg) * d.V + v0 + r) : 0.f;
+      // an absent token's factor e^{E_t - E_s} must be 0, not 0 * overflow
+      if (Ec) Zs[j][r] = oks ? Ec[(bh * d.Tp + sg) * d.V + v0 + r] : INFINITY;
+    }
+    __syncthreads();
+#pragma unroll 4
+    for (int j = 0; j < kQkRed; ++j) {
+      const int sj = s0 + j;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        if (sj > t0 + 4 * ty + u) continue;  // causal: s <= t
+        const float pv = Xs[j][4 * ty + u];
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+          const float x = pv * Ys[j][4 * tx + w];
+          acc[u][w] += Ec ? x * __expf(Et[u][w] - Zs[j][4 * tx + w]) : x;
+        }
+      }
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int ti = t0 + 4 * ty + u;
+    const long t = (long)n * d.C + ti;
+    if (ti >= d.C || t >= d.T) continue;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      const int vv = v0 + 4 * tx + w;
+      if (vv < d.V) st(o + (bh * d.T + t) * d.V + vv, acc[u][w]);
+    }
   }
 }
 
@@ -264,28 +382,6 @@ __global__ void k_out(const T *__restrict__ q, const T *__restrict__ v, const fl
 
 // dH[bh, n] = adjoint of the state after chunk n (through chunks > n and dh_final):
 // the chunk contributions by k_chunk_kv<MODE 1>, composed by k_dstates_scan.
-
-// dP[bh, n, t, s] = sum_v do_t[v] v_s[v] (e^{E_t[v] - E_s[v]}) for s <= t, else 0.
-template <typename T>
-__global__ void k_dscores(const T *__restrict__ dout, const T *__restrict__ v, const float *__restrict__ Ec, Dims d,
-                          float *__restrict__ dP) {
-  const long bh = blockIdx.y;
-  const int n = blockIdx.x;
-  for (int idx = threadIdx.x; idx < d.C * d.C; idx += blockDim.x) {
-    const int ti = idx / d.C, si = idx % d.C;
-    const long t = (long)n * d.C + ti, s = (long)n * d.C + si;
-    float acc = 0.f;
-    if (si <= ti && t < d.T) {
-      if (Ec)
-        for (int j = 0; j < d.V; ++j)
-          acc += ld(dout + (bh * d.T + t) * d.V + j) * ld(v + (bh * d.T + s) * d.V + j) *
-                 __expf(Ec[(bh * d.Tp + t) * d.V + j] - Ec[(bh * d.Tp + s) * d.V + j]);
-      else
-        for (int j = 0; j < d.V; ++j) acc += ld(dout + (bh * d.T + t) * d.V + j) * ld(v + (bh * d.T + s) * d.V + j);
-    }
-    dP[((bh * d.N + n) * d.C + ti) * d.C + si] = acc;
-  }
-}
 
 // Inter-chunk terms of dq and dk, contractions over the d_v channels per chunk n:
 //   A1[t, c] = sum_v do_t[v] e^{E_t[v]} H[n][c, v]
@@ -411,45 +507,104 @@ __global__ void k_dqk(const T *__restrict__ q, const T *__restrict__ k,
   }
 }
 
-// dv_t = (k_t (.) e^{B_last - B_t}) dH[n] + sum_{s>=t} P[s,t] do_s
-// (general gate: the first term times e^{E_last[v] - E_t[v]}, the pairs times
-// e^{E_s[v] - E_t[v]}; dvf, if not null, receives dv in fp32 for the beta gradient)
+// dv_t = e^{E_last - E_t} (k_t (.) e^{B_last - B_t}) dH[n] + sum_{s>=t} P[s,t] do_s e^{E_s - E_t}
+// (E null: no E factors), tiled like k_out: the first term a staged GEMM over d_k, the
+// second over the chunk's tokens s >= t (mask before the exponential).  dvf, if not
+// null, receives dv in fp32 for the beta gradient.
 template <typename T>
-__global__ void k_dv(const T *__restrict__ k, const T *__restrict__ dout, const float *__restrict__ Bc,
-                     const float *__restrict__ Ec, const float *__restrict__ dHs, const float *__restrict__ P, Dims d,
-                     T *__restrict__ dv, float *__restrict__ dvf) {
-  const int vi = blockIdx.x * blockDim.x + threadIdx.x;
-  const int n = blockIdx.y;
-  const long bh = blockIdx.z;
-  if (vi >= d.V) return;
+__global__ void __launch_bounds__(256) k_dv(const T *__restrict__ k, const T *__restrict__ dout,
+                                            const float *__restrict__ Bc, const float *__restrict__ Ec,
+                                            const float *__restrict__ dHs, const float *__restrict__ P, Dims d,
+                                            T *__restrict__ dv, float *__restrict__ dvf) {
+  __shared__ float Xs[kQkRed][kQkTile + 1], Ys[kQkRed][kQkTile + 1], Zs[kQkRed][kQkTile + 1];
+  const int ttiles = (d.C + kQkTile - 1) / kQkTile, vtiles = (d.V + kQkTile - 1) / kQkTile;
+  const int n = blockIdx.x / (ttiles * vtiles);
+  const int t0 = ((blockIdx.x / vtiles) % ttiles) * kQkTile, v0 = (blockIdx.x % vtiles) * kQkTile;
+  const long bh = blockIdx.y;
   const long KV = (long)d.K * d.V;
   const float *dH = dHs + (bh * d.N + n) * KV;
   const float *Pc = P + (bh * d.N + n) * (long)d.C * d.C;
-  for (int ti = threadIdx.y; ti < d.C; ti += blockDim.y) {
+  const long last = bh * d.Tp + (long)n * d.C + d.C - 1;
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  float acc[4][4] = {};
+  for (int c0 = 0; c0 < d.K; c0 += kQkRed) {
+    for (int idx = threadIdx.x; idx < kQkTile * kQkRed; idx += 256) {
+      const int r = idx / kQkRed, c = idx % kQkRed;
+      const long t = (long)n * d.C + t0 + r;
+      Xs[c][r] = (c0 + c < d.K && t0 + r < d.C && t < d.T)
+                     ? ld(k + (bh * d.T + t) * d.K + c0 + c) *
+                           __expf(Bc[last * d.K + c0 + c] - Bc[(bh * d.Tp + t) * d.K + c0 + c])
+                     : 0.f;
+      const int cc = idx / kQkTile, vv = idx % kQkTile;
+      Ys[cc][vv] = (c0 + cc < d.K && v0 + vv < d.V) ? dH[(long)(c0 + cc) * d.V + v0 + vv] : 0.f;
+    }
+    __syncthreads();
+#pragma unroll 8
+    for (int c = 0; c < kQkRed; ++c) {
+      float xa[4], ya[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) xa[u] = Xs[c][4 * ty + u], ya[u] = Ys[c][4 * tx + u];
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int w = 0; w < 4; ++w) acc[u][w] += xa[u] * ya[w];
+    }
+    __syncthreads();
+  }
+  float Et[4][4] = {};
+  if (Ec) {
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const long t = (long)n * d.C + t0 + 4 * ty + u;
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        const int vv = v0 + 4 * tx + w;
+        const bool ok = t0 + 4 * ty + u < d.C && t < d.T && vv < d.V;
+        Et[u][w] = ok ? Ec[(bh * d.Tp + t) * d.V + vv] : 0.f;
+        acc[u][w] *= ok ? __expf(Ec[last * d.V + vv] - Et[u][w]) : 0.f;
+      }
+    }
+  }
+  for (int s0 = t0; s0 < d.C; s0 += kQkRed) {
+    for (int idx = threadIdx.x; idx < kQkTile * kQkRed; idx += 256) {
+      const int r = idx % kQkTile, j = idx / kQkTile;  // P slice: row s0 + j, column t0 + r
+      const int sj = s0 + j;
+      const long sg = (long)n * d.C + sj;
+      Xs[j][r] = (sj < d.C && t0 + r < d.C) ? Pc[(long)sj * d.C + t0 + r] : 0.f;
+      const bool oks = sj < d.C && sg < d.T && v0 + r < d.V;
+      Ys[j][r] = oks ? ld(dout + (bh * d.T + sg) * d.V + v0 + r) : 0.f;
+      // an absent token's factor e^{E_s - E_t} must be 0, not 0 * overflow
+      if (Ec) Zs[j][r] = oks ? Ec[(bh * d.Tp + sg) * d.V + v0 + r] : -INFINITY;
+    }
+    __syncthreads();
+#pragma unroll 4
+    for (int j = 0; j < kQkRed; ++j) {
+      const int sj = s0 + j;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        if (sj < t0 + 4 * ty + u) continue;  // s >= t
+        const float pv = Xs[j][4 * ty + u];
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+          const float x = pv * Ys[j][4 * tx + w];
+          acc[u][w] += Ec ? x * __expf(Zs[j][4 * tx + w] - Et[u][w]) : x;
+        }
+      }
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int ti = t0 + 4 * ty + u;
     const long t = (long)n * d.C + ti;
-    if (t >= d.T) break;
-    float acc = 0.f;
-    for (int c = 0; c < d.K; ++c) {
-      const float blast = Bc[(bh * d.Tp + (long)n * d.C + d.C - 1) * d.K + c];
-      acc += ld(k + (bh * d.T + t) * d.K + c) * __expf(blast - Bc[(bh * d.Tp + t) * d.K + c]) * dH[(long)c * d.V + vi];
+    if (ti >= d.C || t >= d.T) continue;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      const int vv = v0 + 4 * tx + w;
+      if (vv >= d.V) continue;
+      st(dv + (bh * d.T + t) * d.V + vv, acc[u][w]);
+      if (dvf) dvf[(bh * d.T + t) * d.V + vv] = acc[u][w];
     }
-    if (Ec) {
-      const float Et = Ec[(bh * d.Tp + t) * d.V + vi];
-      acc *= __expf(Ec[(bh * d.Tp + (long)n * d.C + d.C - 1) * d.V + vi] - Et);
-      for (int si = ti; si < d.C; ++si) {
-        const long s = (long)n * d.C + si;
-        if (s >= d.T) break;
-        acc += Pc[si * d.C + ti] * ld(dout + (bh * d.T + s) * d.V + vi) * __expf(Ec[(bh * d.Tp + s) * d.V + vi] - Et);
-      }
-    } else {
-      for (int si = ti; si < d.C; ++si) {
-        const long s = (long)n * d.C + si;
-        if (s >= d.T) break;
-        acc += Pc[si * d.C + ti] * ld(dout + (bh * d.T + s) * d.V + vi);
-      }
-    }
-    st(dv + (bh * d.T + t) * d.V + vi, acc);
-    if (dvf) dvf[(bh * d.T + t) * d.V + vi] = acc;
   }
 }
 
@@ -525,6 +680,18 @@ F32Ws carve(const Problem &p, void *ws, bool bwd, bool general) {
   return w;
 }
 
+// Grid of k_out / k_dv: x = chunk x 64-token tile x 64-channel value tile, y = head.
+dim3 tv_grid(const Problem &p) {
+  const int ttiles = (p.C + kQkTile - 1) / kQkTile, vtiles = (p.V + kQkTile - 1) / kQkTile;
+  return dim3((unsigned)(p.N * ttiles * vtiles), (unsigned)p.BH);
+}
+
+// Grid of k_pairs: x = chunk x 64 x 64 pair tile, y = head.
+dim3 pair_grid(const Problem &p) {
+  const int tiles = (p.C + kQkTile - 1) / kQkTile;
+  return dim3((unsigned)(p.N * tiles * tiles), (unsigned)p.BH);
+}
+
 // States (Hs, and h_final if hT) and state adjoints (dHs, dh0): per-chunk GEMMs, then scans.
 template <typename T>
 int launch_states(const Problem &p, const Dims &d, const T *k, const T *v, const F32Ws &w, const float *h0,
@@ -558,10 +725,9 @@ int fwd_impl(const Problem &p, const T *q, const T *k, const T *v, const float *
   GLA_LAUNCH(K_F32_PREP, st, (k_prep<<<dim3(p.N, p.BH), kth, 0, st>>>(la, d, w.Bc)));
   if (lb) GLA_LAUNCH(K_F32_PREP, st, (k_prep_beta<<<dim3(p.N, p.BH), 256, 0, st>>>(lb, d, w.Ec)));
   if (const int r = launch_states<T>(p, d, k, v, w, h0, hT, st)) return r;
-  GLA_LAUNCH(K_F32_SCORES, st, (k_scores<T><<<dim3(p.N, p.BH), 256, 0, st>>>(q, k, w.Bc, d, w.P)));
+  GLA_LAUNCH(K_F32_SCORES, st, (k_pairs<T, 0><<<pair_grid(p), 256, 0, st>>>(q, k, w.Bc, d, w.P)));
   GLA_LAUNCH(K_F32_OUT, st,
-             (k_out<T, T><<<dim3((p.V + 63) / 64, p.N, p.BH), dim3(64, 4), 0, st>>>(q, v, w.Bc, w.Ec, w.Hs, w.P, d,
-                                                                                     o)));
+             (k_out<T, T><<<tv_grid(p), 256, 0, st>>>(q, v, w.Bc, w.Ec, w.Hs, w.P, d, o)));
   return GLA_OK;
 }
 
@@ -575,9 +741,9 @@ int bwd_impl(const Problem &p, const T *q, const T *k, const T *v, const float *
   GLA_LAUNCH(K_F32_PREP, st, (k_prep<<<dim3(p.N, p.BH), kth, 0, st>>>(la, d, w.Bc)));
   if (lb) GLA_LAUNCH(K_F32_PREP, st, (k_prep_beta<<<dim3(p.N, p.BH), 256, 0, st>>>(lb, d, w.Ec)));
   if (const int r = launch_states<T>(p, d, k, v, w, h0, nullptr, st)) return r;
-  GLA_LAUNCH(K_F32_SCORES, st, (k_scores<T><<<dim3(p.N, p.BH), 256, 0, st>>>(q, k, w.Bc, d, w.P)));
+  GLA_LAUNCH(K_F32_SCORES, st, (k_pairs<T, 0><<<pair_grid(p), 256, 0, st>>>(q, k, w.Bc, d, w.P)));
   if (const int r = launch_dstates<T>(p, d, q, dout, w, dhT, dh0, st)) return r;
-  GLA_LAUNCH(K_F32_DSCORES, st, (k_dscores<T><<<dim3(p.N, p.BH), 256, 0, st>>>(dout, v, w.Ec, d, w.dP)));
+  GLA_LAUNCH(K_F32_DSCORES, st, (k_pairs<T, 1><<<pair_grid(p), 256, 0, st>>>(dout, v, w.Ec, d, w.dP)));
   GLA_LAUNCH(K_F32_DQK, st,
              (k_inter_qk<T><<<dim3(p.N * ((p.C + kQkTile - 1) / kQkTile), 2 * ((p.K + kQkTile - 1) / kQkTile), p.BH), 256,
                               0, st>>>(dout, v, w.Ec, w.Hs, w.dHs, d, w.A1, w.A2)));
@@ -585,15 +751,13 @@ int bwd_impl(const Problem &p, const T *q, const T *k, const T *v, const float *
              (k_dqk<T><<<dim3(p.N, p.BH), kth, 0, st>>>(q, k, w.Bc, w.Hs, w.dHs, w.dP, w.A1, w.A2, d, dq, dk,
                                                          w.dgv)));
   GLA_LAUNCH(K_F32_DV, st,
-             (k_dv<T><<<dim3((p.V + 63) / 64, p.N, p.BH), dim3(64, 4), 0, st>>>(k, dout, w.Bc, w.Ec, w.dHs, w.P, d, dv,
-                                                                                w.dvf)));
+             (k_dv<T><<<tv_grid(p), 256, 0, st>>>(k, dout, w.Bc, w.Ec, w.dHs, w.P, d, dv, w.dvf)));
   if (p.gate != GLA_GATE_NONE)
     GLA_LAUNCH(K_F32_DG_SCALAR, st, (k_dg_out<<<dim3((p.T + 127) / 128, p.BH), 128, 0, st>>>(w.dgv, d, dla)));
   if (lb) {
     // o in fp32 for the beta gradient, then the closed form
     GLA_LAUNCH(K_F32_OUT, st,
-               (k_out<T, float><<<dim3((p.V + 63) / 64, p.N, p.BH), dim3(64, 4), 0, st>>>(q, v, w.Bc, w.Ec, w.Hs, w.P,
-                                                                                          d, w.of)));
+               (k_out<T, float><<<tv_grid(p), 256, 0, st>>>(q, v, w.Bc, w.Ec, w.Hs, w.P, d, w.of)));
     GLA_LAUNCH(K_F32_DLB, st,
                (k_dlb<T><<<dim3((p.V + 63) / 64, p.N, p.BH), 64, 0, st>>>(v, dout, w.of, w.dvf, w.Hs, w.dHs, d, dlb)));
   }
