@@ -442,9 +442,18 @@ def measure_general_gate(args, w, dev, stream, seed=0):
     e1.record(stream)
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / n
+    # bound "alu": fp32 FMA on CUDA cores; peak from the unit counts and the clock
+    # (148 SMs x 128 fp32 lanes x 2 FLOP x SM clock), the contraction FLOPs counted as
+    # for the alpha-only step (the beta factors add only elementwise work)
+    flops = B * H * T * (4 * K * V + w["C"] * (K + V) + 10 * K * V + w["C"] * (3 * K + 2 * V))
+    peak = 148 * 128 * 2 * FALLBACK_PEAKS["sm_max_mhz"] * 1e6 / 1e12
+    achieved = flops / (ms / 1e3) / 1e12
     return {"workload": f"general gate, B={B} H={H} T={T} d_k={K} d_v={V} bf16 in/out, {w['gate']} alpha + vector beta",
             "path": "CUDA cores, fp32 arithmetic, materialised chunk states", "ms_per_step": ms,
-            "tokens_per_s": B * T / (ms / 1e3)}
+            "tokens_per_s": B * T / (ms / 1e3),
+            "roofline": {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                         "frac": achieved / peak,
+                         "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 FLOP x 1965 MHz"}}
 
 
 def run_ours(args, w):
