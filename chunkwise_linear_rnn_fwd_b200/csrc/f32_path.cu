@@ -465,17 +465,30 @@ __global__ void k_dqk(const T *__restrict__ q, const T *__restrict__ k,
                       const float *__restrict__ Bc, const float *__restrict__ Hs, const float *__restrict__ dHs,
                       const float *__restrict__ dP, const float *__restrict__ A1, const float *__restrict__ A2, Dims d,
                       T *__restrict__ dq, T *__restrict__ dk, float *__restrict__ dgv) {
+  __shared__ float Gs[256];  // d_k <= 256
   const int c = threadIdx.x;
-  if (c >= d.K) return;
   const long bh = blockIdx.y;
   const int n = blockIdx.x;
   const long KV = (long)d.K * d.V;
-  const float *Hn = Hs + (bh * (d.N + 1) + n + 1) * KV + (long)c * d.V;
-  const float *dH = dHs + (bh * d.N + n) * KV + (long)c * d.V;
+  // G[c] = sum_v S_n[c, v] dS_n[c, v]: each warp reduces whole rows, lanes along v
+  // (coalesced), every thread of the block taking part
+  {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    const float *Hn = Hs + (bh * (d.N + 1) + n + 1) * KV;
+    const float *dH = dHs + (bh * d.N + n) * KV;
+    for (int r = warp; r < d.K; r += nw) {
+      float acc = 0.f;
+      for (int j = lane; j < d.V; j += 32) acc += Hn[(long)r * d.V + j] * dH[(long)r * d.V + j];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+      if (lane == 0) Gs[r] = acc;
+    }
+  }
+  __syncthreads();
+  if (c >= d.K) return;
   const float *dPc = dP + (bh * d.N + n) * (long)d.C * d.C;
   const float blast = Bc[(bh * d.Tp + (long)n * d.C + d.C - 1) * d.K + c];
-  float G = 0.f;
-  for (int j = 0; j < d.V; ++j) G += Hn[j] * dH[j];
+  const float G = Gs[c];
   // pass 1: dlog b per token into dgv, dq and dk stored
   for (int ti = 0; ti < d.C; ++ti) {
     const long t = (long)n * d.C + ti;

@@ -494,15 +494,13 @@ __global__ void __launch_bounds__(kBwdKH, 2)
 
 template <int K>
 int launch_bwd_main_k(const Problem &p, const BwdArgs &a, const CUtensorMap *maps, cudaStream_t st) {
-  static int smem = 0;
-  if (!smem) {
-    const int want = BwdSmem::kBytes + 1024;
+  static DeviceSlots slots;
+  const int smem = per_device(slots, [] {
     if (cudaFuncSetAttribute(k_bwd_main<K>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem) != cudaSuccess)
-      return GLA_ERR_CUDA;
-    const int got = smem_for_tmem(k_bwd_main<K>, kBwdKH, want, 256);
-    if (got < 0) return GLA_ERR_CUDA;
-    smem = got;
-  }
+      return -1;
+    return smem_for_tmem(k_bwd_main<K>, kBwdKH, BwdSmem::kBytes + 1024, 256);
+  });
+  if (smem < 0) return GLA_ERR_CUDA;
   GLA_LAUNCH(K_TC_BWD, st,
              if (launch_pdl(k_bwd_main<K>, dim3(K / kBwdKH, p.N, p.BH), dim3(kBwdKH), smem, st, a, maps[0], maps[1],
                             maps[2], maps[3]) != cudaSuccess) return GLA_ERR_CUDA);

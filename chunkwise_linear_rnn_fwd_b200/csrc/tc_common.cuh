@@ -15,6 +15,8 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "internal.h"
 
 namespace gla {
@@ -334,6 +336,29 @@ constexpr int kMaxDynSmem = 232448;
 // TMEM than its SM has left gets no usable allocation.  So every TMEM-using
 // kernel is launched with enough dynamic shared memory that at most
 // 512 / tmem_cols of its CTAs can be resident on one SM.
+template <typename Kern>
+inline int smem_for_tmem(Kern kernel, int threads, int smem, int tmem_cols);
+
+// Host-side cache of a positive launch-setup value per device (0 = not yet
+// computed): function attributes and device properties belong to the device that
+// was current when the value was computed.  Racing first calls compute the same
+// value; each store is atomic.
+constexpr int kMaxDevices = 64;
+struct DeviceSlots {
+  std::atomic<int> v[kMaxDevices];  // static storage: zero-initialised
+};
+template <typename F>
+inline int per_device(DeviceSlots &slots, F compute) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return compute();
+  int x = slots.v[dev].load(std::memory_order_acquire);
+  if (x <= 0) {
+    x = compute();
+    if (x > 0) slots.v[dev].store(x, std::memory_order_release);
+  }
+  return x;
+}
+
 template <typename Kern>
 inline int smem_for_tmem(Kern kernel, int threads, int smem, int tmem_cols) {
   const int max_ctas = 512 / tmem_cols;

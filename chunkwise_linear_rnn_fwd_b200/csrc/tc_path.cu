@@ -58,29 +58,26 @@ bool tc::map3_bf16(CUtensorMap *m, const void *base, uint64_t d0, uint64_t d1, u
 
 namespace {
 
+// 1 if the current device is sm_100 (per device: 1 = yes, 2 = no).
 int device_ok() {
-  static int state = -1;
-  static std::once_flag once;
-  std::call_once(once, [] {
+  static DeviceSlots slots;
+  return per_device(slots, [] {
     int dev = 0, major = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
-      state = 0;
-    else
-      state = (major == 10) ? 1 : 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+      return 2;
+    return major == 10 ? 1 : 2;
   });
-  return state;
 }
 
 int sm_count() {
-  static int n = 0;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    int dev = 0;
+  static DeviceSlots slots;
+  return per_device(slots, [] {
+    int dev = 0, n = 0;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    if (n <= 0) n = 148;
+    return n > 0 ? n : 148;
   });
-  return n;
 }
 
 int bv_of(const Problem &p) { return (p.K == 256 || p.V % 128 != 0) ? 64 : 128; }
@@ -161,15 +158,13 @@ int launch_prep(const Problem &p, const bf16 *q, const bf16 *k, const float *la,
   if (!map3(&mq, q, p.K, p.T, (uint64_t)p.BH, 64, 64) || !map3(&mk, k, p.K, p.T, (uint64_t)p.BH, 64, 64) ||
       !map3(&mqg, w.qg, p.K, p.Tp, (uint64_t)p.BH, 64, 64) || !map3(&mkg, w.kg, p.K, p.Tp, (uint64_t)p.BH, 64, 64))
     return GLA_ERR_CUDA;
-  static int smem = 0;
-  if (!smem) {
-    const int want = tc::PrepSmem<K>::kBytes + 1024;
+  static DeviceSlots slots;
+  const int smem = per_device(slots, [] {
     if (cudaFuncSetAttribute(tc::k_prep<K>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem) != cudaSuccess)
-      return GLA_ERR_CUDA;
-    const int got = smem_for_tmem(tc::k_prep<K>, 256, want, 64);
-    if (got < 0) return GLA_ERR_CUDA;
-    smem = got;
-  }
+      return -1;
+    return smem_for_tmem(tc::k_prep<K>, 256, tc::PrepSmem<K>::kBytes + 1024, 64);
+  });
+  if (smem < 0) return GLA_ERR_CUDA;
   GLA_LAUNCH(K_TC_PREP, st,
              if (launch_pdl(tc::k_prep<K>, dim3(p.N, p.BH), dim3(256), smem, st, a, mq, mk, mqg, mkg) != cudaSuccess)
                  return GLA_ERR_CUDA);
@@ -184,13 +179,14 @@ template <int K, int BV>
 int launch_walk(const Problem &p, const tc::WalkArgs &a, const WalkMaps &m, int P, cudaStream_t st) {
   using W = tc::WalkSmem<K, BV>;
   constexpr int kTmemCols = ((K / 128) * BV + BV <= 256) ? 256 : 512;
-  static bool attr = false;
-  if (!attr) {
-    if (cudaFuncSetAttribute(tc::k_walk<K, BV>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem) !=
-        cudaSuccess)
-      return GLA_ERR_CUDA;
-    attr = true;
-  }
+  static DeviceSlots attr;  // the attribute belongs to the current device
+  if (per_device(attr, [] {
+        return cudaFuncSetAttribute(tc::k_walk<K, BV>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem) ==
+                       cudaSuccess
+                   ? 1
+                   : -1;
+      }) < 0)
+    return GLA_ERR_CUDA;
   const int smem = smem_for_tmem(tc::k_walk<K, BV>, K, W::bytes(a.do_out != 0, a.do_out != 0), kTmemCols);
   if (smem < 0) return GLA_ERR_CUDA;
   GLA_LAUNCH(K_TC_WALK, st,
