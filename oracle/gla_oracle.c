@@ -51,7 +51,11 @@
  *  1: output read before the state update (o_t = q_t S_{t-1})
  *  2: gate applied after the outer product (S_t = diag(alpha)(S_{t-1} + k^T v))
  *  3: gate gradient taken with S_t in place of S_{t-1}
- *  4: dk taken before the output term q_t^T do_t is added to dS            */
+ *  4: dk taken before the output term q_t^T do_t is added to dS
+ *  5: (general gate) beta applied after the outer product
+ *     (S_t = diag(alpha) S_{t-1} diag(beta) + k^T v diag(beta))
+ *  6: (general gate) dlog beta accumulated without the alpha factor
+ *  7: (general gate) the adjoint propagated without beta (dS <- diag(alpha) dS) */
 #ifndef GLA_ORACLE_MUTANT
 #define GLA_ORACLE_MUTANT 0
 #endif
@@ -71,7 +75,11 @@ static void step_state(double *S, const double *lbt, const double *kt, const dou
     for (int c = 0; c < K; ++c) {
       const double a = exp(gate_log(la, mode, t, K, c));
       double *row = S + (long)c * V;
+#if GLA_ORACLE_MUTANT == 5
+      for (int j = 0; j < V; ++j) row[j] = (a * row[j] + kt[c] * vt[j]) * exp(lbt[j]);
+#else
       for (int j = 0; j < V; ++j) row[j] = a * row[j] * exp(lbt[j]) + kt[c] * vt[j];
+#endif
     }
     return;
   }
@@ -236,7 +244,11 @@ void gla_oracle_bwd_general(int B, int H, long T, int K, int V, int mode,
             dvh[t * V + j] += kt[c] * drow[j];
             const double bj = lbt ? exp(lbt[j]) : 1.0;
             accg += prow[j] * bj * drow[j];
+#if GLA_ORACLE_MUTANT == 6
+            if (dlbh) dlbh[t * V + j] += prow[j] * bj * drow[j];
+#else
             if (dlbh) dlbh[t * V + j] += a * prow[j] * bj * drow[j];
+#endif
           }
 #if GLA_ORACLE_MUTANT == 4
           dkh[t * K + c] = dla_vec[c];
@@ -261,7 +273,11 @@ void gla_oracle_bwd_general(int B, int H, long T, int K, int V, int mode,
         for (int c = 0; c < K; ++c) {
           const double a = exp(gate_log(lah, mode, t, K, c));
           double *drow = dS + (long)c * V;
+#if GLA_ORACLE_MUTANT == 7
+          if (0)
+#else
           if (lbt)
+#endif
             for (int j = 0; j < V; ++j) drow[j] *= a * exp(lbt[j]);
           else
             for (int j = 0; j < V; ++j) drow[j] *= a;

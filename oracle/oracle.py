@@ -198,3 +198,9 @@ class Mutant:
 
     def bwd(self, *a, **kw):
         return bwd(*a, _lib_override=self._lib, **kw)
+
+    def fwd_general(self, *a, **kw):
+        return fwd_general(*a, _lib_override=self._lib, **kw)
+
+    def bwd_general(self, *a, **kw):
+        return bwd_general(*a, _lib_override=self._lib, **kw)

@@ -462,3 +462,27 @@ def test_general_gate_closed_form_gate_gradients(oracle_mod):
     clb = rev(o * do - v * dv) + (hT * dhT).sum(axis=2)[:, :, None, :]
     np.testing.assert_allclose(dla, cla, rtol=1e-10, atol=1e-10)
     np.testing.assert_allclose(dlb, clb, rtol=1e-10, atol=1e-10)
+
+
+def _general_pins_pass(orc):
+    """The general-gate pins above against an oracle-like object."""
+    try:
+        test_general_gate_parallel_form(orc)
+        test_general_gate_transpose_symmetry(orc)
+        test_general_gate_finite_differences(orc)
+        test_general_gate_closed_form_gate_gradients(orc)
+    except AssertionError:
+        return False
+    return True
+
+
+def test_general_pins_pass_on_oracle(oracle_mod):
+    assert _general_pins_pass(oracle_mod)
+
+
+@pytest.mark.parametrize("mutant", [5, 6, 7])
+def test_general_pins_catch_planted_mistakes(mutant):
+    """Each planted general-gate mistake (beta after the outer product; dlog beta
+    without alpha; the adjoint propagated without beta) fails a pin."""
+    from oracle.oracle import Mutant
+    assert not _general_pins_pass(Mutant(mutant))

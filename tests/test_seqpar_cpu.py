@@ -133,7 +133,7 @@ def _worker(rank, world, port, T, cuts, gate, out):
 
 
 @pytest.mark.parametrize("world,cuts,gate", [(2, [0, 64, 150], "vector"), (3, [0, 50, 51, 150], "scalar"),
-                                             (2, [0, 77, 150], "none")])
+                                             (2, [0, 77, 150], "none"), (4, [0, 30, 31, 100, 150], "vector")])
 def test_sequence_parallel_matches_whole_sequence(oracle_mod, world, cuts, gate):
     T = 150
     port = _free_port()
