@@ -22,7 +22,6 @@ enum KernelId : int {
   K_F32_DG_SCALAR,
   K_TC_PREP,
   K_TC_WALK,
-  K_TC_SCAN,
   K_TC_BWD,
   K_STATUS_CLEAR,
   K_DECODE,
