@@ -155,3 +155,49 @@ def test_sequence_parallel_matches_whole_sequence(oracle_mod, world, cuts, gate)
         close(cat("dla"), dla)
     close(out[world - 1]["h_out"], hT)
     close(out[0]["dh_in"], dh0)
+
+
+def test_library_ops_reuse_chain(monkeypatch):
+    """seqpar.LibraryOps passes each call exactly the reuse flags that an earlier call
+    on its workspace has earned: fwd_state -> fwd reuses prep and segments; bwd_state
+    reuses prep only after fwd; bwd reuses prep and saved states only after fwd and
+    segments only after bwd_state; a call on a new shape starts over.  The CUDA
+    binding is replaced by a recorder (no GPU)."""
+    from chunkwise_linear_rnn_fwd_b200 import gla as G
+    from chunkwise_linear_rnn_fwd_b200 import seqpar
+    calls = []
+    monkeypatch.setattr(G, "workspace_size", lambda *a, **k: 256)
+    monkeypatch.setattr(G, "alloc_workspace", lambda n, dev: torch.empty(n, dtype=torch.uint8))
+
+    def rec(name):
+        def f(*a, **kw):
+            calls.append((name, {k: v for k, v in kw.items() if k in ("save_states", "reuse_prep", "reuse_segments",
+                                                                          "saved_states")}))
+            return (None, None) if name in ("fwd_state", "bwd_state", "fwd") else (None,) * 5
+        return f
+
+    for name in ("fwd_state", "bwd_state"):
+        monkeypatch.setattr(G, "gla_" + name, rec(name))
+    monkeypatch.setattr(G, "gla_fwd", rec("fwd"))
+    monkeypatch.setattr(G, "gla_bwd", rec("bwd"))
+    q = torch.zeros(1, 1, 8, 4)
+    v = torch.zeros(1, 1, 8, 4)
+    la = torch.zeros(1, 1, 8, 4)
+    ops = seqpar.LibraryOps()
+    ops.fwd_state(q, q, v, la, None)
+    ops.fwd(q, q, v, la, None)
+    ops.bwd_state(q, q, la, v, None)
+    ops.bwd(q, q, v, la, v, None, None)
+    ops.bwd(q, q, v, la, v, None, None)          # nothing left to reuse
+    ops.fwd(q, q, v, la, None)                   # a forward without its summary
+    q2 = torch.zeros(1, 1, 9, 4)
+    ops.bwd_state(q2, q2, torch.zeros(1, 1, 9, 4), torch.zeros(1, 1, 9, 4), None)  # new shape: new workspace
+    assert calls == [
+        ("fwd_state", {"save_states": True}),
+        ("fwd", {"save_states": True, "reuse_prep": True, "reuse_segments": True}),
+        ("bwd_state", {"reuse_prep": True}),
+        ("bwd", {"reuse_prep": True, "saved_states": True, "reuse_segments": True}),
+        ("bwd", {"reuse_prep": False, "saved_states": False, "reuse_segments": False}),
+        ("fwd", {"save_states": True, "reuse_prep": False, "reuse_segments": False}),
+        ("bwd_state", {"reuse_prep": False}),
+    ], calls
