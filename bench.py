@@ -192,6 +192,26 @@ def oracle_sample_rate(w, T_sample=1024, seed=0, min_seconds=0.0):
     return reps * w["B"] * T_sample / dt, dt, threads, desc
 
 
+def host_cpu():
+    """The host the oracle ran on: cores available to this process and the CPU model.
+    `cores` in cpu_baseline is the number of threads the oracle actually used (its
+    OpenMP loop runs over the B*H heads, so it cannot use more threads than heads)."""
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    try:
+        avail = len(os.sched_getaffinity(0))
+    except (AttributeError, OSError):
+        avail = os.cpu_count()
+    return {"host_cores_available": avail, "cpu_model": model}
+
+
 def run_reference(args, w):
     rank, world, _ = dist_env()
     if rank != 0:
@@ -210,7 +230,8 @@ def run_reference(args, w):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / max(1, args.steps),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": bench_config(w, world),
-        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": desc},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": desc,
+                         **host_cpu()},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -247,7 +268,8 @@ def kernel_io_bytes(name, w, sms=148):
         # forward: pre-pass + output walk that also stores h_n (saved states);
         # backward: reverse pre-pass + adjoint walk storing dh_n
         fwd_out = 2 * kx + vy + pt + seg + vy + BH * K * V * 4 + states
-        dh_walk = kx + vy + seg + states
+        # reverse walk: qg, dO (the adjoint) and kg, P^T (dv) in; dh_n and dv out
+        dh_walk = 2 * kx + vy + pt + seg + states + vy
         launches = 2 * (2 if P > 1 else 1)
         total = 2 * (pre if P > 1 else 0) + fwd_out + dh_walk
         return total / launches
@@ -258,6 +280,28 @@ def kernel_io_bytes(name, w, sms=148):
         return (BH * N * K * V * 2 * 2 + BH * T * (2 * V * 2 + 2 * K * 2 + g) + BH * Tp * 2 * K
                 + BH * N * 2 * C * C + BH * T * (2 * K * 2 + 2 * V + g))
     return None
+
+
+# Which of the step's algorithmic tensors (inputs and outputs of the forward and the
+# backward, each counted once per pass as in algorithmic_bytes) each kernel moves
+# between HBM and the chip: a kernel's algorithmic share of the step.
+KERNEL_ALG_TENSORS = {
+    "tc_prep": ("q", "k", "la"),                          # the forward's reads of q, k, log alpha
+    "tc_walk": ("v", "o", "h_final", "do", "dv"),         # forward: v in, o, h_final out; reverse: dO in, dv out
+    "tc_bwd": ("q", "k", "la", "v", "dq", "dk", "dla"),   # the backward's reads of q, k, log alpha, v and its outputs
+}
+
+
+def kernel_alg_bytes(name, w):
+    """Algorithmic bytes per step that kernel `name` is responsible for (its share of
+    algorithmic_bytes: the tensors of KERNEL_ALG_TENSORS, no workspace)."""
+    B, H, T, K, V = w["B"], w["H"], w["T"], w["K"], w["V"]
+    th = B * H * T
+    g = 4 * K if w["gate"] == "vector" else (4 if w["gate"] == "scalar" else 0)
+    size = {"q": th * 2 * K, "k": th * 2 * K, "v": th * 2 * V, "la": th * g, "o": th * 2 * V, "do": th * 2 * V,
+            "dq": th * 2 * K, "dk": th * 2 * K, "dv": th * 2 * V, "dla": th * g, "h_final": B * H * K * V * 4}
+    names = KERNEL_ALG_TENSORS.get(name)
+    return None if names is None else sum(size[n] for n in names)
 
 
 DECODE_WORKLOAD = dict(B=128, H=4, K=256, V=512)
@@ -456,6 +500,113 @@ def measure_general_gate(args, w, dev, stream, seed=0):
                          "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 FLOP x 1965 MHz"}}
 
 
+def _time_steps(fn, stream, steps, warmup=3):
+    """Mean device time of fn() over `steps` calls (CUDA events on the launch stream)."""
+    import torch
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        fn()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / steps
+
+
+def measure_variants(args, w, dev, stream, seed=0):
+    """The forward/backward variants of the workload, each a whole fwd+bwd step:
+    saved_states  the forward stores its bf16 chunk states, the backward reads them;
+    recompute     the backward recomputes the chunk states with a forward walk of its own;
+    materialized  the MATERIALIZED forward (every chunk state in fp32, then all chunk
+                  outputs in parallel), the backward reading the saved bf16 states.
+    All reuse the forward's prep outputs in the backward."""
+    import torch
+
+    import chunkwise_linear_rnn_fwd_b200 as pkg
+    from chunkwise_linear_rnn_fwd_b200.synth import make_inputs
+
+    B, H, T, K, V, C = w["B"], w["H"], w["T"], w["K"], w["V"], w["C"]
+    x = make_inputs(B, H, T, K, V, dtype=torch.bfloat16, gate=w["gate"], seed=seed, z_mean=w["z_mean"])
+    q, k, v, la, do = (t.to(dev) for t in (x.q, x.k, x.v, x.log_alpha, x.do))
+    o = torch.empty(B, H, T, V, dtype=torch.bfloat16, device=dev)
+    dq, dk, dv, dla = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v), torch.empty_like(la)
+    out = {}
+    n = max(5, min(args.steps, 20))
+    for name, save, variant in (("saved_states", True, "auto"), ("recompute", False, "auto"),
+                                ("materialized", True, "materialized")):
+        flags = pkg.FLAG_REUSE_PREP | (pkg.FLAG_SAVE_STATES if save else 0)
+        ws = pkg.alloc_workspace(pkg.workspace_size(B, H, T, K, V, torch.bfloat16, w["gate"], C, True, flags=flags,
+                                                    variant=variant), dev)
+
+        def fwd():
+            pkg.gla_fwd(q, k, v, la, None, chunk=C, o=o, want_final=False, workspace=ws, stream=stream,
+                        save_states=save, variant=variant)
+
+        def step():
+            fwd()
+            pkg.gla_bwd(q, k, v, la, do, None, None, chunk=C, dq=dq, dk=dk, dv=dv, dlog_alpha=dla, want_dh0=False,
+                        workspace=ws, stream=stream, reuse_prep=True, saved_states=save, variant=variant)
+
+        out[name] = {"step_ms": _time_steps(step, stream, n), "fwd_ms": _time_steps(fwd, stream, n)}
+        del ws
+    out["workload"] = (f"B={B} H={H} T={T} d_k={K} d_v={V} C={C} bf16, {w['gate']} gates; fwd+bwd and fwd alone, "
+                       "device time per call")
+    return out
+
+
+SWEEP_T = [dict(name=f"config 5: fwd+bwd, B*T=32768 H=4 d_k=256 d_v=512, T={T}", B=32768 // T, H=4, T=T, K=256,
+                V=512, gate=g, z_mean=0.0, bwd=True)
+           for T in (1024, 2048, 4096, 8192, 16384) for g in ("vector", "scalar", "none")]
+
+
+def time_workload(c, args, dev, stream, peaks, C=64):
+    """Device time of one workload configuration `c` (dict with B, H, T, K, V, gate,
+    z_mean, bwd): the forward (and backward) as bench.py's step launches them, inputs
+    drawn on the device with the workload's distributions (timing only; parity is in
+    tests/)."""
+    import torch
+
+    import chunkwise_linear_rnn_fwd_b200 as pkg
+
+    B, H, T, K, V = c["B"], c["H"], c["T"], c["K"], c["V"]
+    g = torch.Generator(device=dev)
+    g.manual_seed(0)
+    q = torch.randn(B, H, T, K, device=dev, generator=g).to(torch.bfloat16)
+    k = (torch.randn(B, H, T, K, device=dev, generator=g) / K ** 0.5).to(torch.bfloat16)
+    v = torch.randn(B, H, T, V, device=dev, generator=g).to(torch.bfloat16)
+    do = torch.randn(B, H, T, V, device=dev, generator=g).to(torch.bfloat16)
+    shape = {"vector": (B, H, T, K), "scalar": (B, H, T)}.get(c["gate"])
+    la = None if shape is None else torch.nn.functional.logsigmoid(
+        torch.randn(*shape, device=dev, generator=g) + c["z_mean"]) / 16
+    o = torch.empty_like(v)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    dla = None if la is None else torch.empty_like(la)
+    flags = pkg.FLAG_REUSE_PREP | pkg.FLAG_SAVE_STATES if c["bwd"] else 0
+    ws = pkg.alloc_workspace(pkg.workspace_size(B, H, T, K, V, torch.bfloat16, c["gate"], C, c["bwd"],
+                                                flags=flags), dev)
+
+    def step():
+        pkg.gla_fwd(q, k, v, la, None, chunk=C, gate=c["gate"], o=o, want_final=False, workspace=ws,
+                    stream=stream, save_states=c["bwd"])
+        if c["bwd"]:
+            pkg.gla_bwd(q, k, v, la, do, None, None, chunk=C, gate=c["gate"], dq=dq, dk=dk, dv=dv,
+                        dlog_alpha=dla, want_dh0=False, workspace=ws, stream=stream, reuse_prep=True,
+                        saved_states=True)
+
+    ms = _time_steps(step, stream, args.steps, max(3, args.warmup))
+    th = B * H * T
+    flops = th * (4 * K * V + C * (K + V)) + (th * (10 * K * V + C * (3 * K + 2 * V)) if c["bwd"] else 0)
+    abytes = algorithmic_bytes(B, H, T, K, V, c["gate"]) if c["bwd"] else th * (4 * K + 4 * V) + (
+        th * 4 * K if c["gate"] == "vector" else (th * 4 if c["gate"] == "scalar" else 0))
+    peak_t = float(peaks.get("bf16_tflops", 1590)) * 1e12
+    peak_b = float(peaks["hbm_gbs"]) * 1e9
+    return {"workload": c["name"], "gate": c["gate"], "ms_per_step": ms, "tokens_per_s": B * T / (ms / 1e3),
+            "tflops": flops / (ms / 1e3) / 1e12, "frac_of_tensor_peak": flops / (ms / 1e3) / peak_t,
+            "frac_of_roofline": max(flops / peak_t, abytes / peak_b) / (ms / 1e3)}
+
+
 def run_ours(args, w):
     import torch
     import torch.distributed as dist
@@ -568,13 +719,22 @@ def run_ours(args, w):
     if dom is not None:
         n_l, tot = per_kernel[dom]
         avg_ms = tot / n_l
+        launches_per_step = n_l / args.steps
+        alg = kernel_alg_bytes(dom, w)
         io = kernel_io_bytes(dom, w, torch.cuda.get_device_properties(dev).multi_processor_count)
-        if io is not None:
-            achieved = io / (avg_ms / 1e3) / 1e9
+        if alg is not None:
+            # achieved = the kernel's algorithmic bytes per launch / its mean launch time
+            alg_launch = alg / launches_per_step
+            achieved = alg_launch / (avg_ms / 1e3) / 1e9
             peak = float(peaks["hbm_gbs"])
             roofline = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peak, "unit": "GB/s",
                         "frac": achieved / peak, "traffic": measured_traffic(dom), "peak_source": peak_src,
-                        "bytes_per_launch": io, "avg_launch_ms": avg_ms}
+                        "bytes_per_launch": alg_launch, "bytes_source": "algorithmic share (no workspace)",
+                        "launches_per_step": launches_per_step, "avg_launch_ms": avg_ms}
+            if io is not None:
+                # the same kernel's own input + output bytes, workspace included
+                roofline["bytes_per_launch_incl_workspace"] = io
+                roofline["frac_incl_workspace"] = io / (avg_ms / 1e3) / 1e9 / peak
     flops = counted_flops(B, H, T, K, V, C)
     abytes = algorithmic_bytes(B, H, T, K, V, w["gate"])
     t_tensor = flops / (float(peaks.get("bf16_tflops", 1590)) * 1e12)
@@ -590,13 +750,17 @@ def run_ours(args, w):
     decode = measure_decode(args, dev, stream, peaks, peak_src, seed=rank)
     epilogue = measure_epilogue(args, w, dev, stream, peaks, peak_src, seed=rank)
     seqpar = measure_seqpar(args, w, dev, stream, seed=rank)
+    variants = measure_variants(args, w, dev, stream, seed=rank)
+    sweep_args = argparse.Namespace(steps=5, warmup=2)
+    sweep_T = [time_workload(c, sweep_args, dev, stream, peaks) for c in SWEEP_T]
     general = measure_general_gate(args, w, dev, stream, seed=rank)
     general["vs_alpha_only_step"] = general["ms_per_step"] / ms_per_step
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         r, dt, threads, desc = oracle_sample_rate(w, T_sample=w["T"], min_seconds=args.cpu_seconds)
-        cpu = {"value": r, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": desc, "seconds": dt}
+        cpu = {"value": r, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": desc, "seconds": dt,
+               **host_cpu()}
 
     if rank == 0:
         line = {
@@ -611,7 +775,9 @@ def run_ours(args, w):
             "kernel_timing": "separate pass of the same K steps with a CUDA-event pair around each launch",
             "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "clocks": clocks, "cpu_baseline": cpu, "decode_step": decode, "layer_epilogue": epilogue,
-            "sequence_parallel": seqpar, "general_gate": general,
+            "sequence_parallel": seqpar, "general_gate": general, "variants": variants,
+            "sweep_vs_T": {"workloads": sweep_T, "steps": 5, "peak_source": peak_src,
+                           "l2": "inputs larger than L2 (B*T = 32768 tokens, >= 1 GB per step)"},
         }
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -626,15 +792,11 @@ SWEEP = ([dict(name="config 2: fwd, B=8 H=4 T=2048 d_k=128 d_v=256", B=8, H=4, T
                  gate="vector", z_mean=0.0, bwd=True)]
          + [dict(name="config 4: fwd+bwd, B=2 H=4 T=4096 d_k=256 d_v=512", B=2, H=4, T=4096, K=256, V=512,
                  gate="vector", z_mean=-1.0, bwd=True)]
-         + [dict(name=f"config 5: fwd+bwd, B*T=32768 H=4 d_k=256 d_v=512, T={T}", B=32768 // T, H=4, T=T, K=256,
-                 V=512, gate=g, z_mean=0.0, bwd=True)
-            for T in (1024, 2048, 4096, 8192, 16384) for g in ("vector", "scalar", "none")])
+         + SWEEP_T)
 
 
 def run_sweep(args):
-    """Device time of every workload configuration (one JSON line, --sweep): the forward
-    (and backward) as bench.py's step launches them, inputs drawn once per shape on the
-    device with the workload's distributions (timing only; parity is in tests/)."""
+    """Device time of every workload configuration (one JSON line, --sweep)."""
     import torch
 
     import chunkwise_linear_rnn_fwd_b200 as pkg
@@ -644,49 +806,7 @@ def run_sweep(args):
     pkg.load()
     peaks, peak_src = load_peaks()
     stream = torch.cuda.current_stream()
-    g = torch.Generator(device=dev)
-    g.manual_seed(0)
-    out = []
-    for c in SWEEP:
-        B, H, T, K, V, C = c["B"], c["H"], c["T"], c["K"], c["V"], 64
-        q = torch.randn(B, H, T, K, device=dev, generator=g).to(torch.bfloat16)
-        k = (torch.randn(B, H, T, K, device=dev, generator=g) / K ** 0.5).to(torch.bfloat16)
-        v = torch.randn(B, H, T, V, device=dev, generator=g).to(torch.bfloat16)
-        do = torch.randn(B, H, T, V, device=dev, generator=g).to(torch.bfloat16)
-        shape = {"vector": (B, H, T, K), "scalar": (B, H, T)}.get(c["gate"])
-        la = None if shape is None else torch.nn.functional.logsigmoid(
-            torch.randn(*shape, device=dev, generator=g) + c["z_mean"]) / 16
-        o = torch.empty_like(v)
-        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-        dla = None if la is None else torch.empty_like(la)
-        flags = pkg.FLAG_REUSE_PREP | pkg.FLAG_SAVE_STATES if c["bwd"] else 0
-        ws = pkg.alloc_workspace(pkg.workspace_size(B, H, T, K, V, torch.bfloat16, c["gate"], C, c["bwd"],
-                                                    flags=flags), dev)
-
-        def step():
-            pkg.gla_fwd(q, k, v, la, None, chunk=C, gate=c["gate"], o=o, want_final=False, workspace=ws,
-                        stream=stream, save_states=c["bwd"])
-            if c["bwd"]:
-                pkg.gla_bwd(q, k, v, la, do, None, None, chunk=C, gate=c["gate"], dq=dq, dk=dk, dv=dv,
-                            dlog_alpha=dla, want_dh0=False, workspace=ws, stream=stream, reuse_prep=True,
-                            saved_states=True)
-
-        for _ in range(args.warmup):
-            step()
-        torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(args.steps):
-            step()
-        e1.record(stream)
-        torch.cuda.synchronize()
-        ms = e0.elapsed_time(e1) / args.steps
-        th = B * H * T
-        flops = th * (4 * K * V + C * (K + V)) + (th * (10 * K * V + C * (3 * K + 2 * V)) if c["bwd"] else 0)
-        out.append({"workload": c["name"], "gate": c["gate"], "ms_per_step": ms, "tokens_per_s": B * T / (ms / 1e3),
-                    "tflops": flops / (ms / 1e3) / 1e12,
-                    "frac_of_tensor_peak": flops / (ms / 1e3) / (float(peaks.get("bf16_tflops", 1590)) * 1e12)})
-        del q, k, v, do, la, o, dq, dk, dv, dla, ws
+    out = [time_workload(c, args, dev, stream, peaks) for c in SWEEP]
     print(json.dumps({"metric": METRIC, "sweep": out, "peak_source": peak_src}), flush=True)
     return 0
 

@@ -282,7 +282,8 @@ int gla_fwd_state(const gla_desc *desc, const void *q, const void *k, const void
   GLA_TRY(check_opt(h0));
   GLA_TRY(check_req(delta));
   GLA_TRY(check_req(gamma));
-  GLA_TRY(check_ws(desc, p, false));
+  // with GLA_FLAG_SAVE_STATES the summary uses the backward's (larger) layout
+  GLA_TRY(check_ws(desc, p, (p.flags & GLA_FLAG_SAVE_STATES) != 0));
   cudaStream_t st = (cudaStream_t)stream;
   GLA_TRY(clear_status(desc, st));
   return tc_fwd_state(p, q, k, v, log_alpha, h0, delta, gamma, desc->workspace, st);

@@ -15,7 +15,10 @@
 //     on g_scratch and must be serialised by the caller;
 //   * the first call on a device resolves the array's device address with
 //     cudaGetSymbolAddress (once per device, with that device current); make
-//     that first call before any stream capture.
+//     that first call before any stream capture;
+//   * the status word at the start of g_scratch (a bounded wait that ran out, a
+//     gate beyond the bf16 range) is read and cleared by
+//     gla_poll_status_noalloc, the counterpart of gla_poll_status.
 #include <mutex>
 
 #include "internal.h"
@@ -51,10 +54,14 @@ extern "C" int gla_fwd_noalloc(const gla_desc *desc, const void *q, const void *
                                const float *log_alpha, const float *h0, void *o, float *h_final, int chunk,
                                void *stream) {
   if (!desc) return GLA_ERR_INVALID_ARG;
+  // Nothing but an earlier no-allocation forward writes g_scratch, and that call's
+  // intermediates are not a promise to the next one: a flag that would make this
+  // call read them instead of computing them is refused.
+  if (desc->flags & (GLA_FLAG_REUSE_PREP | GLA_FLAG_REUSE_SEGMENTS)) return GLA_ERR_INVALID_ARG;
   gla_desc d = *desc;
   d.workspace = nullptr;
   d.workspace_bytes = 0;
-  const size_t need = gla_workspace_size(&d, chunk, 0);
+  const size_t need = gla_workspace_size(&d, chunk, (d.flags & GLA_FLAG_SAVE_STATES) ? 1 : 0);
   if (need == 0) return gla_check(&d, chunk);
   if (need > kScratchBytes) return GLA_ERR_WORKSPACE_TOO_SMALL;
   void *scratch = nullptr;
@@ -63,4 +70,16 @@ extern "C" int gla_fwd_noalloc(const gla_desc *desc, const void *q, const void *
   d.workspace = scratch;
   d.workspace_bytes = kScratchBytes;
   return gla_fwd(&d, q, k, v, log_alpha, h0, o, h_final, chunk, stream);
+}
+
+// Counterpart of gla_poll_status for the no-allocation forward: the status word
+// sits at the start of g_scratch, which a caller cannot name.
+extern "C" int gla_poll_status_noalloc(void *stream) {
+  void *scratch = nullptr;
+  const int r = scratch_address(&scratch);
+  if (r != GLA_OK) return r;
+  gla_desc d{};
+  d.workspace = scratch;
+  d.workspace_bytes = kScratchBytes;
+  return gla_poll_status(&d, stream);
 }

@@ -8,6 +8,7 @@ call fails, an exception is raised.  PyTorch is used only to own device memory
 from __future__ import annotations
 
 import ctypes
+import functools
 import os
 from typing import Optional
 
@@ -32,7 +33,7 @@ EXPORTS = ["gla_workspace_size", "gla_check", "gla_fwd", "gla_bwd", "gla_poll_st
            "gla_timing_enable", "gla_timing_collect", "gla_kernel_name", "gla_build_info", "gla_fwd_noalloc",
            "gla_decode_step", "gla_selftest_timeout", "gla_epilogue_workspace_size", "gla_epilogue_fwd",
            "gla_epilogue_bwd", "gla_fwd_state", "gla_bwd_state", "gla_state_scan", "gla_general_workspace_size",
-           "gla_fwd_general", "gla_bwd_general"]
+           "gla_fwd_general", "gla_bwd_general", "gla_poll_status_noalloc"]
 
 
 class GLAError(RuntimeError):
@@ -69,6 +70,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.gla_fwd.restype = i
     lib.gla_fwd_noalloc.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, i, vp]
     lib.gla_fwd_noalloc.restype = i
+    lib.gla_poll_status_noalloc.argtypes = [vp]
+    lib.gla_poll_status_noalloc.restype = i
     lib.gla_decode_step.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp]
     lib.gla_decode_step.restype = i
     lib.gla_selftest_timeout.argtypes = [vp, ctypes.c_uint, vp]
@@ -128,6 +131,22 @@ def _stream_handle(stream) -> ctypes.c_void_p:
     return ctypes.c_void_p(int(stream.cuda_stream))
 
 
+def _on_stream(fn):
+    """Run a binding with `stream` (keyword argument) as torch's current stream, so that
+    the tensors the binding allocates (outputs the caller did not pass, a temporary
+    workspace) belong to the stream the library launches on: the caching allocator
+    then cannot hand a temporary workspace to other work while the kernels that use
+    it are still queued on that stream."""
+    @functools.wraps(fn)
+    def wrapper(*args, **kwargs):
+        stream = kwargs.get("stream")
+        if stream is None or stream == torch.cuda.current_stream(stream.device):
+            return fn(*args, **kwargs)
+        with torch.cuda.stream(stream):
+            return fn(*args, **kwargs)
+    return wrapper
+
+
 def _gate_of(log_alpha, gate):
     if gate is not None:
         return gate
@@ -170,6 +189,7 @@ def alloc_workspace(nbytes: int, device) -> torch.Tensor:
     return torch.empty(int(nbytes), dtype=torch.uint8, device=device)
 
 
+@_on_stream
 def gla_fwd(q, k, v, log_alpha=None, h0=None, *, chunk=64, gate=None, subchunk=16, variant="auto", segments=0,
             o=None, h_final=None, want_final=True, workspace=None, stream=None, save_states=False,
             reuse_prep=False, reuse_segments=False):
@@ -210,6 +230,7 @@ def general_workspace_size(B, H, T, dk, dv, dtype, gate, chunk=64, for_bwd=False
     return int(n)
 
 
+@_on_stream
 def gla_fwd_general(q, k, v, log_alpha, log_beta, h0=None, *, chunk=64, gate=None, o=None, h_final=None,
                     want_final=True, workspace=None, stream=None):
     """Forward with the general gate alpha_t^T beta_t (log_beta [B,H,T,d_v]).
@@ -232,6 +253,7 @@ def gla_fwd_general(q, k, v, log_alpha, log_beta, h0=None, *, chunk=64, gate=Non
     return o, h_final
 
 
+@_on_stream
 def gla_bwd_general(q, k, v, log_alpha, log_beta, do, h0=None, dh_final=None, *, chunk=64, gate=None,
                     want_dh0=True, workspace=None, stream=None):
     """Backward of gla_fwd_general: (dq, dk, dv, dlog_alpha or None, dlog_beta, dh0 or None)."""
@@ -254,6 +276,7 @@ def gla_bwd_general(q, k, v, log_alpha, log_beta, do, h0=None, dh_final=None, *,
     return dq, dk, dv, dla, dlb, dh0
 
 
+@_on_stream
 def gla_fwd_state(q, k, v, log_alpha=None, h0=None, *, chunk=64, gate=None, subchunk=16, segments=0,
                   delta=None, gamma=None, workspace=None, stream=None, save_states=False, reuse_prep=False):
     """Summary of this piece of the sequence: (delta, gamma) = (the state after the
@@ -281,6 +304,7 @@ def gla_fwd_state(q, k, v, log_alpha=None, h0=None, *, chunk=64, gate=None, subc
     return delta, gamma
 
 
+@_on_stream
 def gla_bwd_state(q, k, log_alpha, do, dh_final=None, *, chunk=64, gate=None, subchunk=16, segments=0,
                   ddelta=None, gamma=None, want_gamma=True, workspace=None, stream=None, reuse_prep=False):
     """Reverse summary of this piece: (ddelta, gamma or None) = (the state adjoint
@@ -306,6 +330,7 @@ def gla_bwd_state(q, k, log_alpha, do, dh_final=None, *, chunk=64, gate=None, su
     return ddelta, gamma
 
 
+@_on_stream
 def gla_state_scan(gammas, deltas, seg, *, reverse=False, init=None, out=None, stream=None):
     """Fold of gathered piece summaries: gammas [P,B,H,dk], deltas [P,B,H,dk,dv] fp32.
     reverse=False: the state entering piece `seg` (pieces 0 .. seg-1 over init);
@@ -322,6 +347,7 @@ def gla_state_scan(gammas, deltas, seg, *, reverse=False, init=None, out=None, s
     return out
 
 
+@_on_stream
 def gla_fwd_noalloc(q, k, v, log_alpha=None, h0=None, *, chunk=64, gate=None, subchunk=16, variant="auto",
                     segments=0, o=None, h_final=None, want_final=True, stream=None):
     """Forward without a workspace, for callers that cannot allocate device memory:
@@ -343,6 +369,13 @@ def gla_fwd_noalloc(q, k, v, log_alpha=None, h0=None, *, chunk=64, gate=None, su
     return o, h_final
 
 
+def poll_status_noalloc(stream=None) -> int:
+    """Synchronise and read/clear the status word of gla_fwd_noalloc's scratch on the
+    current device (GLA_OK = 0, GLA_ERR_TIMEOUT = -6, GLA_ERR_GATE_RANGE = -7)."""
+    return int(load().gla_poll_status_noalloc(_stream_handle(stream)))
+
+
+@_on_stream
 def gla_decode_step(q, k, v, log_alpha, state, *, gate=None, o=None, stream=None):
     """One recurrent decode step per (batch, head): state <- diag(alpha) state + k^T v
     (in place), o = q state.  q, k [B,H,d_k]; v [B,H,d_v]; log_alpha [B,H,d_k] or
@@ -368,6 +401,7 @@ def epilogue_workspace_size(B, H, T, dv, dtype) -> int:
     return int(load().gla_epilogue_workspace_size(ctypes.byref(d)))
 
 
+@_on_stream
 def gla_epilogue_fwd(o, r, w=None, b=None, *, eps=1e-5, y=None, workspace=None, stream=None):
     """y = LayerNorm(o; w, b, eps) * Swish(r) per (batch, head, token) over d_v.
     o, r [B,H,T,d_v]; w, b [d_v] fp32 or None.  See include/gla.h."""
@@ -385,6 +419,7 @@ def gla_epilogue_fwd(o, r, w=None, b=None, *, eps=1e-5, y=None, workspace=None, 
     return y
 
 
+@_on_stream
 def gla_epilogue_bwd(o, r, dy, w=None, b=None, *, eps=1e-5, want_dwb=True, workspace=None, stream=None):
     """Backward of gla_epilogue_fwd: (do, dr, dw or None, db or None)."""
     lib = load()
@@ -404,6 +439,7 @@ def gla_epilogue_bwd(o, r, dy, w=None, b=None, *, eps=1e-5, want_dwb=True, works
     return do_, dr, dw, db
 
 
+@_on_stream
 def gla_bwd(q, k, v, log_alpha, do, h0=None, dh_final=None, *, chunk=64, gate=None, subchunk=16, dq=None, dk=None,
             dv=None, dlog_alpha=None, dh0=None, want_dh0=True, workspace=None, stream=None, reuse_prep=False,
             saved_states=False, reuse_segments=False, segments=0, variant="auto"):

@@ -25,6 +25,7 @@ fp32 per head), so there is nothing to overlap with.
 """
 from __future__ import annotations
 
+import contextlib
 from typing import Optional
 
 import torch
@@ -54,7 +55,11 @@ class LibraryOps:
         if key != self._key:
             B, H, T, dk = q.shape
             n = G.workspace_size(B, H, T, dk, dv, q.dtype, gate, self.chunk, True, flags=G.FLAG_SAVE_STATES)
-            self.ws, self._key = G.alloc_workspace(n, q.device), key
+            # the old workspace may still be in use by kernels queued on self.stream:
+            # allocate (and so later free) on that stream
+            ctx = torch.cuda.stream(self.stream) if self.stream is not None else contextlib.nullcontext()
+            with ctx:
+                self.ws, self._key = G.alloc_workspace(n, q.device), key
             self._state = self._fwd = self._bstate = False
         return self.ws
 

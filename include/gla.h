@@ -151,8 +151,10 @@ int gla_fwd(const gla_desc *desc, const void *q, const void *k, const void *v,
             void *stream);
 
 /* Backward (Algorithms 4 and 6 of Appendix B by title; closed-form gate
- * gradient of section 4.3).  Chunk states are recomputed, not read from the
- * forward.  The loss gradient enters through do [B,H,T,d_v] and dh_final
+ * gradient of section 4.3).  The chunk states are recomputed by a forward walk
+ * of the backward itself, unless desc->flags has GLA_FLAG_SAVE_STATES: then they
+ * are read from the workspace, where the preceding gla_fwd call with that flag
+ * stored them.  The loss gradient enters through do [B,H,T,d_v] and dh_final
  * (dL/dS_T, NULL = 0).  Outputs: dq, dk [B,H,T,d_k], dv [B,H,T,d_v],
  * dlog_alpha (gate layout; NULL iff gate == NONE), dh0 (dL/dh0; NULL = not
  * written).  With a SCALAR gate dlog_alpha_t is the sum over key channels. */
@@ -242,7 +244,11 @@ int gla_bwd_general(const gla_desc *desc, const void *q, const void *k, const vo
  *   starting from h0 (NULL = zero), i.e. the h_final of gla_fwd, without computing
  *   o; gamma [B,H,dk] fp32 = prod over the piece's tokens of alpha_t (exp of the
  *   summed log_alpha; all ones for GLA_GATE_NONE, the scalar gate broadcast over
- *   dk).  Workspace: gla_workspace_size(desc, chunk, 0).
+ *   dk).  Workspace: gla_workspace_size(desc, chunk, 0), or
+ *   gla_workspace_size(desc, chunk, 1) when desc->flags has GLA_FLAG_SAVE_STATES
+ *   (the summary then uses the backward's layout, so that a following gla_fwd
+ *   with that flag finds its segment contributions); a smaller workspace is
+ *   rejected with GLA_ERR_WORKSPACE_TOO_SMALL.
  * gla_bwd_state: ddelta [B,H,dk,dv] fp32 = the state adjoint before the piece's
  *   first token given dh_final (NULL = zero) after its last, i.e. the dh0 of
  *   gla_bwd, without the token gradients; gamma (NULL = not written) as above.
@@ -281,12 +287,22 @@ int gla_state_scan(const gla_desc *desc, int nseg, int seg, int reverse, const f
  *     serialise them.  Each call clears the status word it needs zeroed.
  *   - The first call on a device looks up the array's address for that device
  *     (cudaGetSymbolAddress); make that first call before any stream capture.
- *   - gla_poll_status cannot reach this scratch; errors found on the device
- *     are not reported by this entry point. */
+ *   - desc->flags may hold GLA_FLAG_SAVE_STATES (the workspace size is then
+ *     the backward's), but not GLA_FLAG_REUSE_PREP or GLA_FLAG_REUSE_SEGMENTS:
+ *     nothing leaves intermediates in this scratch for a later call to reuse,
+ *     so those flags are rejected with GLA_ERR_INVALID_ARG.
+ *   - Errors found on the device (a bounded wait that ran out, a gate beyond
+ *     the bf16 range) are recorded in a status word at the start of the
+ *     scratch, which gla_poll_status_noalloc reads and clears.
+ * gla_poll_status_noalloc: like gla_poll_status, for that status word on the
+ * current device: synchronises `stream`, reads and clears the word, and returns
+ * GLA_OK, GLA_ERR_TIMEOUT or GLA_ERR_GATE_RANGE (GLA_ERR_CUDA if the stream
+ * failed).  Its first call on a device resolves the scratch address as above. */
 #define GLA_NOALLOC_SCRATCH_BYTES (64u << 20)
 int gla_fwd_noalloc(const gla_desc *desc, const void *q, const void *k, const void *v,
                     const float *log_alpha, const float *h0, void *o, float *h_final, int chunk,
                     void *stream);
+int gla_poll_status_noalloc(void *stream);
 
 /* Synchronise `stream`, then read and clear the device status word kept in
  * desc->workspace.  Returns GLA_OK, GLA_ERR_TIMEOUT or GLA_ERR_GATE_RANGE (or

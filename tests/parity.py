@@ -13,6 +13,11 @@ import torch
 
 TOL = {torch.float32: 5e-3, torch.bfloat16: 2e-2}
 
+# Every run_case result of this session, (case description, tensor-scale errors,
+# element-wise errors); tests/conftest.py prints them in pytest's terminal summary
+# so that a run's log keeps both metrics.
+RECORDS: list = []
+
 
 def rel_err(x, ref) -> float:
     """max|x - ref| / max(1, max|ref|)"""
@@ -90,6 +95,9 @@ def run_case(B, H, T, K, V, *, dtype=torch.bfloat16, gate="vector", chunk=64, se
         errs[k] = rel_err(a, r)
         elem[k] = elem_err(a, r)
     errs["_elementwise"] = elem
+    RECORDS.append((f"B={B} H={H} T={T} dk={K} dv={V} {str(dtype).replace('torch.', '')} gate={gate} "
+                    f"variant={variant} seed={seed}" + (" save_states" if save_states else ""),
+                    {k: v for k, v in errs.items() if k != "_elementwise"}, dict(elem)))
     print("parity", {k: f"{v:.2e}" for k, v in errs.items() if k != "_elementwise"},
           "elementwise", {k: f"{v:.2e}" for k, v in elem.items()})
     return errs

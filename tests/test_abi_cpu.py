@@ -242,3 +242,30 @@ def test_general_gate_validation_enqueues_nothing(lib):
     d.workspace_bytes = 16
     assert f(ctypes.byref(d), a, a, a, a, a, None, a, None, 64, None) == -4         # workspace too small
     assert b(ctypes.byref(d), a, a, a, a, a, None, a, None, a, a, a, a, a, None, 64, None) == -4
+
+
+def test_saved_state_summary_needs_backward_workspace(lib):
+    """gla_fwd_state with GLA_FLAG_SAVE_STATES lays out the backward's workspace; a
+    workspace of the forward's size is refused before anything is enqueued."""
+    vp = ctypes.c_void_p
+    a = vp(4096)
+    d = desc(T=4096, dk=256, dv=512, flags=2)
+    fwd = lib.gla_workspace_size(ctypes.byref(d), 64, 0)
+    bwd = lib.gla_workspace_size(ctypes.byref(d), 64, 1)
+    assert 0 < fwd < bwd
+    d.workspace = 1 << 20
+    d.workspace_bytes = fwd
+    assert lib.gla_fwd_state(ctypes.byref(d), a, a, a, a, None, a, a, 64, None) == -4
+    d.workspace_bytes = bwd - 1
+    assert lib.gla_fwd_state(ctypes.byref(d), a, a, a, a, None, a, a, 64, None) == -4
+
+
+def test_noalloc_rejects_reuse_flags(lib):
+    """The no-allocation forward's scratch holds nothing a later call may reuse: the
+    reuse flags are refused before anything is enqueued (no GPU is touched)."""
+    vp = ctypes.c_void_p
+    a = vp(4096)
+    for flags in (1, 4, 5, 3):
+        d = desc(T=64, dk=128, dv=128, flags=flags)
+        assert lib.gla_fwd_noalloc(ctypes.byref(d), a, a, a, a, None, a, None, 64, None) == -1
+    assert lib.gla_fwd_noalloc(None, a, a, a, a, None, a, None, 64, None) == -1
