@@ -11,8 +11,8 @@
 //
 //   k_fold_segments  a piece's summary from the walk's segment contributions: the
 //                    zero-state pre-pass runs every segment of the piece in parallel
-//                    (contributions delta_p in the walk's float4-column layout, gate
-//                    products gseg_p); out = fold over p of S <- diag(gseg_p) S + delta_p
+//                    (contributions delta_p [BH][P][K][V], gate products gseg_p);
+//                    out = fold over p of S <- diag(gseg_p) S + delta_p
 //                    from h0 (dh_final in reverse), gamma = prod_p gseg_p
 //   k_state_scan     out = fold over the selected pieces of S <- diag(gamma_s) S + D_s
 //                    (elementwise per (bh, c, v), HBM-bound: one read of every D_s)
@@ -21,18 +21,18 @@
 namespace gla {
 namespace {
 
-// Thread (bh, v4, c), c fastest: the float4-column contributions
-// delta[bh][p][v4][c] are read coalesced; out[bh][c][4 v4 .. 4 v4 + 3].
+// Thread (bh, c, v4), v4 fastest: delta[bh][p][c][4 v4 .. 4 v4 + 3] and
+// out[bh][c][4 v4 .. 4 v4 + 3] are read and written coalesced.
 __global__ void __launch_bounds__(256) k_fold_segments(long BH, int K, int V, int P, int reverse,
                                                        const float *__restrict__ gseg,
                                                        const float4 *__restrict__ delta,
                                                        const float *__restrict__ h0, float *__restrict__ out,
                                                        float *__restrict__ gamma) {
   const int V4 = V / 4;
-  const long i = (long)blockIdx.x * blockDim.x + threadIdx.x;
+  const long i = (long)blockIdx.x * blockDim.x + threadIdx.x;  // float4 index in [BH][K][V/4]
   if (i >= BH * V4 * K) return;
-  const int c = (int)(i % K);
-  const int v4 = (int)((i / K) % V4);
+  const int v4 = (int)(i % V4);
+  const int c = (int)((i / V4) % K);
   const long bh = i / ((long)K * V4);
   const long o = (bh * K + c) * (long)V + 4 * v4;
   float4 S = h0 ? __ldg(reinterpret_cast<const float4 *>(h0 + o)) : make_float4(0.f, 0.f, 0.f, 0.f);
@@ -44,7 +44,7 @@ __global__ void __launch_bounds__(256) k_fold_segments(long BH, int K, int V, in
     for (int u = 0; u < 4; ++u) {
       const int j = j0 + u, p = reverse ? P - 1 - j : j;
       g[u] = j < P ? __ldg(gseg + (bh * P + p) * K + c) : 1.f;
-      d[u] = j < P ? __ldg(delta + ((bh * P + p) * V4 + v4) * K + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+      d[u] = j < P ? __ldg(delta + ((bh * P + p) * K + c) * V4 + v4) : make_float4(0.f, 0.f, 0.f, 0.f);
     }
 #pragma unroll
     for (int u = 0; u < 4; ++u) {

@@ -2,9 +2,10 @@
 //
 // One CTA per (chunk n, head, half of the key channels): 128 threads, one per key
 // channel c of its half.  Inputs: the chunk state h_n (state before chunk n) and
-// adjoint dh_n (gradient w.r.t. the state after chunk n), both bf16 in the
-// chunk-state layout [K/128][V/8][128][8]; gam from the prep kernel; q, k, V, dO
-// and log_alpha.  (dv comes from the reverse walk, which holds dh_n on chip.)
+// adjoint dh_n (gradient w.r.t. the state after chunk n), both bf16 in the walk's
+// chunk-state layout (state_chunk_off: per 64-column d_v tile and channel half a
+// contiguous 16 KB block, [2 channel blocks][64 v][64 c] 128-byte swizzled); gam
+// from the prep kernel; q, k, V, dO and log_alpha.  (dv comes from the reverse walk, which holds dh_n on chip.)
 // With B the chunk-local cumulative log-gate:
 //   phase 1 (loop over d_v tiles of 64, accumulating in TMEM):
 //     dqh^T = h_n dO^T          dkh^T = dh_n V^T         dP = dO V^T
@@ -57,7 +58,7 @@ struct BwdArgs {
 
 struct BwdSmem {
   static constexpr int BVb = 64;
-  static constexpr int kTileH = kBwdKH * BVb * 2;         // h or dh half-tile, [8][128][8] bf16
+  static constexpr int kTileH = kBwdKH * BVb * 2;         // h or dh half-tile, [2][64 v][64 c] bf16, SW128
   static constexpr int kTileV = 64 * BVb * 2;             // V or dO tile, SW128
   static constexpr int kStage = 2 * kTileH + 2 * kTileV;  // h, dh, V, dO
   static constexpr int kPhase1End = 2 * kStage;
@@ -72,16 +73,10 @@ struct BwdSmem {
   static constexpr int kKt = kQt + 64 * kBwdKH * 2;           // k tile [64][128] bf16
   static constexpr int kPhase2End = kKt + 64 * kBwdKH * 2;
   static constexpr int kRed = (kPhase1End > kPhase2End ? kPhase1End : kPhase2End);  // scalar-gate sums [4][64]
-  static constexpr int kBar = kRed + 4 * 64 * 4;
+  static constexpr int kRed2 = kRed + 4 * 64 * 4;            // partial sums of h (.) dh [8 row groups][128]
+  static constexpr int kBar = kRed2 + 8 * kBwdKH * 4;
   static constexpr int kBytes = kBar + 128;
 };
-
-__device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
-  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-                   dev::smem_u32(dst)),
-               "l"(src), "r"(bytes), "r"(dev::smem_u32(bar))
-               : "memory");
-}
 
 template <int K>
 __global__ void __launch_bounds__(kBwdKH, 2)
@@ -137,18 +132,19 @@ __global__ void __launch_bounds__(kBwdKH, 2)
   dev::tc_fence_after();
   const uint32_t tmem = *tslot;
 
-  // this CTA's 128 rows of h_n / dh_n for d_v tile i: 16 contiguous KB
-  const long half_tile = (long)kBwdKH * BVb;  // bf16 elements
-  const bf16 *h_src = a.hb + (hrow * kH + half) * (long)a.V * kBwdKH;
-  const bf16 *dh_src = a.dhb + (hrow * kH + half) * (long)a.V * kBwdKH;
+  // this CTA's 128 channels of h_n / dh_n for d_v tile i: 16 contiguous KB at
+  // ((hrow * V/64 + i) * K/64 + 2 half) * 64 * 64 elements
+  const long half_tile = (long)K * BVb;  // bf16 elements from one d_v tile to the next
+  const bf16 *h_src = a.hb + (hrow * (a.V / 64) * K / 64 + 2 * half) * 4096;
+  const bf16 *dh_src = a.dhb + (hrow * (a.V / 64) * K / 64 + 2 * half) * 4096;
   auto stage = [&](int s) { return smem + s * L::kStage; };
   auto issue_tile = [&](int i) {
     const int s = i & 1;
     uint8_t *st = stage(s);
     const int v0 = i * BVb;
     dev::mbar_arrive_expect_tx(&full[s], (uint32_t)L::kStage);
-    bulk_load(st, h_src + i * half_tile, (uint32_t)L::kTileH, &full[s]);
-    bulk_load(st + L::kTileH, dh_src + i * half_tile, (uint32_t)L::kTileH, &full[s]);
+    dev::bulk_load(st, h_src + i * half_tile, (uint32_t)L::kTileH, &full[s]);
+    dev::bulk_load(st + L::kTileH, dh_src + i * half_tile, (uint32_t)L::kTileH, &full[s]);
     dev::tma_load_3d(st + 2 * L::kTileH, &tmV, v0, n * kC, (int)bh, &full[s]);
     dev::tma_load_3d(st + 2 * L::kTileH + L::kTileV, &tmDO, v0, n * kC, (int)bh, &full[s]);
   };
@@ -159,7 +155,12 @@ __global__ void __launch_bounds__(kBwdKH, 2)
 
   const int cl = tid;     // key channel within this CTA's half
   const int c = c0 + cl;  // key channel
-  float R = 0.f;          // sum_v h[c,v] dh[c,v]
+  // partial sums of h (.) dh: thread -> 16-byte column chunk cc (channels 8 cc .. 8 cc + 7
+  // of this half), rows v = rg + 8 r of every d_v tile (in the swizzled tile, row v's
+  // chunk cc sits at position (cc % 8) ^ (v % 8) = (cc % 8) ^ rg of block cc / 8)
+  const int cc = tid & 15, rg = tid >> 4;
+  const uint32_t r_off = (uint32_t)((cc >> 3) * 8192 + rg * 128 + (((cc & 7) ^ rg) << 4));
+  float Racc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
   bool ok = true;
 
   // ============================ phase 1 ============================
@@ -172,17 +173,17 @@ __global__ void __launch_bounds__(kBwdKH, 2)
     // the same shared-memory tiles while they run
     if (lane == 0 && warp < 3 && ok) {
       const uint32_t sH = dev::smem_u32(st), sDH = sH + L::kTileH, sV = sDH + L::kTileH, sDO = sV + L::kTileV;
-      constexpr uint32_t id_kk128 = dev::idesc_bf16(128, 64, false, false);
+      constexpr uint32_t id_kk128 = dev::idesc_bf16(128, 64, true, false);  // A = h / dh MN-major
       constexpr uint32_t id_kk64 = dev::idesc_bf16(64, 64, false, false);
 #pragma unroll
       for (int kk = 0; kk < BVb / 16; ++kk) {
         const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
         if (warp == 0)
-          dev::umma_bf16(tmem + cDQ, dev::desc_state_kmajor(sH, kBwdKH, 0, kk * 16),
-                         dev::desc_kmajor(sDO, 64, 0, kk * 16), id_kk128, acc);
+          dev::umma_bf16(tmem + cDQ, dev::desc_mnmajor(sH, 64, kk * 16, 0), dev::desc_kmajor(sDO, 64, 0, kk * 16),
+                         id_kk128, acc);
         else if (warp == 1)
-          dev::umma_bf16(tmem + cDK, dev::desc_state_kmajor(sDH, kBwdKH, 0, kk * 16),
-                         dev::desc_kmajor(sV, 64, 0, kk * 16), id_kk128, acc);
+          dev::umma_bf16(tmem + cDK, dev::desc_mnmajor(sDH, 64, kk * 16, 0), dev::desc_kmajor(sV, 64, 0, kk * 16),
+                         id_kk128, acc);
         else
           dev::umma_bf16(tmem + cDP, dev::desc_kmajor(sDO, 64, 0, kk * 16), dev::desc_kmajor(sV, 64, 0, kk * 16),
                          id_kk64, acc);
@@ -190,22 +191,23 @@ __global__ void __launch_bounds__(kBwdKH, 2)
       dev::umma_commit(mma_bar);
     }
     {
-      const uint32_t sh = dev::smem_u32(st), sdh = sh + L::kTileH;
+      const uint32_t sh = dev::smem_u32(st) + r_off, sdh = sh + L::kTileH;
 #pragma unroll
-      for (int c8 = 0; c8 < BVb / 8; ++c8) {
+      for (int r = 0; r < 8; ++r) {
         uint4 x, y;
         asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];"
                      : "=r"(x.x), "=r"(x.y), "=r"(x.z), "=r"(x.w)
-                     : "r"(sh + (uint32_t)(c8 * kBwdKH + cl) * 16u));
+                     : "r"(sh + (uint32_t)(r * 1024)));
         asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];"
                      : "=r"(y.x), "=r"(y.y), "=r"(y.z), "=r"(y.w)
-                     : "r"(sdh + (uint32_t)(c8 * kBwdKH + cl) * 16u));
+                     : "r"(sdh + (uint32_t)(r * 1024)));
         const __nv_bfloat162 *xh = reinterpret_cast<const __nv_bfloat162 *>(&x);
         const __nv_bfloat162 *yh = reinterpret_cast<const __nv_bfloat162 *>(&y);
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const float2 xf = __bfloat1622float2(xh[e]), yf = __bfloat1622float2(yh[e]);
-          R += xf.x * yf.x + xf.y * yf.y;
+          Racc[2 * e] += xf.x * yf.x;
+          Racc[2 * e + 1] += xf.y * yf.y;
         }
       }
     }
@@ -214,6 +216,15 @@ __global__ void __launch_bounds__(kBwdKH, 2)
     __syncthreads();  // every thread has finished reading stage s (R sums)
     if (tid == 0 && ok && i + 2 < nvt) issue_tile(i + 2);
   }
+
+  // R[c] = sum_v h[c,v] dh[c,v]: the row groups' partial sums meet in shared memory
+  float *red2 = (float *)(smem + L::kRed2);
+#pragma unroll
+  for (int e = 0; e < 8; ++e) red2[rg * kBwdKH + 8 * cc + e] = Racc[e];
+  __syncthreads();
+  float R = 0.f;
+#pragma unroll
+  for (int g8 = 0; g8 < 8; ++g8) R += red2[g8 * kBwdKH + cl];
 
   // ============================ phase 2 ============================
   // q and k columns of this half into the space phase 1 no longer uses

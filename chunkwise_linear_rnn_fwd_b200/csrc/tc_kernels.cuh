@@ -305,390 +305,34 @@ __global__ void __launch_bounds__(256, 1)
 }
 
 // ============================================================================
-// Walk: per (d_v tile, segment, head); carries the fp32 state tile S (K x BV)
-// in TMEM across the chunks of one segment.  Per chunk n (forward):
-//     [state out]  h_n = S                       (bf16 via TMA, or fp32)
-//     [output]     O_n = qg_n S_bf16 + A_n V_n   (tcgen05, M = 64)
-//     S = diag(gam_n) S + kg_n^T V_n             (tcgen05, M = 128 per 128 key rows)
-// Reverse (adjoint) walks run the chunks backwards with (qg, dO) in place of
-// (kg, V): dS_{n-1} = diag(gam_n) dS_n + qg_n^T dO_n.
+// Arguments of the state walk (tc_walk.cuh): per (d_v tile, segment, head) the
+// fp32 state tile is carried across the chunks of one segment.  Forward walks
+// run S = diag(gam_n) S + kg_n^T V_n and, with outputs, O_n = qg_n S_{n-1} + A_n V_n;
+// reverse (adjoint) walks run the chunks backwards with (qg, dO) in place of
+// (kg, V): dS_{n-1} = diag(gam_n) dS_n + qg_n^T dO_n, dv_n = kg_n dS_n + A_n^T dO_n.
 // ============================================================================
 struct WalkArgs {
   int T, N, V, L;  // L = chunks per segment
   int P;           // segments per sequence (the grid covers segments seg0 .. seg0 + gridDim.y - 1)
   int seg0;
   int end_seg;     // -1: every segment writes end[BH][P][K][V]; s >= 0: only segment s writes end[BH][K][V]
-  int reverse, do_out, state_mode;  // state_mode: 0 none, 1 bf16 (TMA store), 2 fp32
+  int reverse, do_out, state_mode;  // state_mode: 0 none, 1 bf16 chunk states, 2 fp32 chunk states
   int p_kmajor;                     // output intra term: 0 = P V (forward), 1 = P^T dO (reverse: dv)
   const float *gam;                 // [BH][N][K]
   const float *start;               // [BH][P][K][V] fp32 start states or null
-  const float *delta;               // [BH][P][V/4][K] float4 segment contributions from a zero state (or null):
+  const float *delta;               // [BH][P][K][V] segment contributions from a zero state (or null):
                                     // the start state is then composed in the kernel from h0 and the
                                     // contributions of the segments before this one (after it, reverse)
   const float *h0;                  // initial state of the whole walk (h0, or dh_final in reverse) or null
-  float *end;                       // state after the segment or null: end_seg < 0: [BH][P][V/4][K] float4
+  float *end;                       // state after the segment or null: end_seg < 0: [BH][P][K][V]
                                     // (the delta layout); else [BH][K][V] fp32
   float *gseg;                      // [BH][P][K] product of gam over the segment (written by d_v tile 0) or null
   const float *gseg_in;             // the same products, read when composing start states
   float *h32;                       // [BH][N][K][V] fp32 states (state_mode 2)
-  bf16 *hb;                         // [BH][N][K/128][V/8][128][8] bf16 states (state_mode 1)
+  bf16 *hb;                         // bf16 states (state_mode 1), layout of state_chunk_off (tc_walk.cuh)
   bf16 *out;                        // [BH][T][V]
   unsigned *status;
 };
-
-// Shared-memory layout of a walk CTA.  Output walks stage (kg, V, qg, P^T) once
-// (two CTAs share an SM); state-only walks double-buffer (kg or qg, V or dO).
-template <int K, int BV>
-struct WalkSmem {
-  static constexpr int kTileX = 64 * K * 2;   // kg or qg chunk tile
-  static constexpr int kTileY = 64 * BV * 2;  // V or dO tile
-  static constexpr int kTileQ = 64 * K * 2;   // qg for the output
-  static constexpr int kTileP = 64 * 64 * 2;  // P^T
-  __host__ __device__ static constexpr int stages(bool out) { return out ? 1 : 2; }
-  __host__ __device__ static constexpr int stage_bytes(bool out) {
-    return kTileX + kTileY + (out ? kTileQ + kTileP : 0);
-  }
-  __host__ __device__ static constexpr int sb_off(bool out) { return stages(out) * stage_bytes(out); }
-  __host__ __device__ static constexpr int bar_off(bool out, bool sb) { return sb_off(out) + (sb ? K * BV * 2 : 0); }
-  __host__ __device__ static constexpr int bytes(bool out, bool sb) { return bar_off(out, sb) + 64; }
-};
-
-template <int K, int BV>
-__global__ void __launch_bounds__(K, 2)
-    k_walk(WalkArgs a, const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmY,
-           const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmP) {
-  using L = WalkSmem<K, BV>;
-  constexpr int kThreads = K;
-  constexpr int kMB = K / 128;         // 128-row blocks of the state
-  constexpr int kColO = kMB * BV;      // TMEM column of the output accumulator
-  constexpr int kTmemCols = (kColO + BV <= 256) ? 256 : 512;
-  // The dynamic shared-memory window is allocated without alignment slack (two
-  // CTAs must fit on one SM); its base is 1024-byte aligned when the kernel has
-  // no static shared memory.  Checked: a misaligned base would break the
-  // 128-byte swizzle, so the CTA reports it and does nothing.
-  extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t *smem = smem_raw;
-  if ((dev::smem_u32(smem_raw) & 1023u) != 0) {
-    if (threadIdx.x == 0) atomicOr(a.status, (unsigned)ST_SMEM_ALIGN);
-    return;
-  }
-  const bool need_sb = a.do_out != 0;
-  const int nst = L::stages(a.do_out);
-  const int kStage = L::stage_bytes(a.do_out);
-  uint64_t *full = (uint64_t *)(smem + L::bar_off(a.do_out, need_sb));
-  uint64_t *mma_bar = full + 2;
-  uint32_t *tslot = (uint32_t *)(full + 3);
-  uint8_t *sb_ptr = smem + L::sb_off(a.do_out);
-  const uint32_t sSb = dev::smem_u32(sb_ptr);
-
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int vt = blockIdx.x, seg = blockIdx.y + a.seg0;
-  const long bh = blockIdx.z;
-  const int v0 = vt * BV;
-  const int n_begin = seg * a.L;
-  const int n_end = min(a.N, n_begin + a.L);
-  const int nloc = n_end - n_begin;
-  const int P = a.P;
-
-  if (tid == 0) {
-    dev::mbar_init(&full[0], 1);
-    dev::mbar_init(&full[1], 1);
-    dev::mbar_init(mma_bar, 1);
-    dev::fence_mbar_init();
-    dev::prefetch_tmap(&tmX);
-    dev::prefetch_tmap(&tmY);
-    if (a.do_out) {
-      dev::prefetch_tmap(&tmQ);
-      dev::prefetch_tmap(&tmP);
-    }
-  }
-  dev::pdl_launch_dependents();
-  dev::pdl_wait();
-  if (warp == 0) dev::tmem_alloc(tslot, kTmemCols);
-  dev::tc_fence_before();
-  __syncthreads();
-  dev::tc_fence_after();
-  const uint32_t tmem = *tslot;
-
-  auto chunk_of = [&](int i) { return a.reverse ? (n_end - 1 - i) : (n_begin + i); };
-  auto stage_ptr = [&](int s) { return smem + s * kStage; };
-  const uint32_t tx_bytes = (uint32_t)kStage;
-
-  auto issue_loads = [&](int i) {
-    const int s = i % nst;
-    const int n = chunk_of(i);
-    uint8_t *st = stage_ptr(s);
-    dev::mbar_arrive_expect_tx(&full[s], tx_bytes);
-#pragma unroll
-    for (int cb = 0; cb < K / 64; ++cb) dev::tma_load_3d(st + cb * 64 * 128, &tmX, cb * 64, n * kC, (int)bh, &full[s]);
-#pragma unroll
-    for (int cb = 0; cb < BV / 64; ++cb)
-      dev::tma_load_3d(st + L::kTileX + cb * 64 * 128, &tmY, v0 + cb * 64, n * kC, (int)bh, &full[s]);
-    if (a.do_out) {
-#pragma unroll
-      for (int cb = 0; cb < K / 64; ++cb)
-        dev::tma_load_3d(st + L::kTileX + L::kTileY + cb * 64 * 128, &tmQ, cb * 64, n * kC, (int)bh, &full[s]);
-      dev::tma_load_3d(st + L::kTileX + L::kTileY + L::kTileQ, &tmP, 0, 0, (int)(bh * a.N + n), &full[s]);
-    }
-  };
-
-  if (tid == 0)
-    for (int i = 0; i < nst && i < nloc; ++i) issue_loads(i);
-
-  // thread -> state row c; TMEM lane block of its warp
-  const int mb = warp >> 2;
-  const int c = tid;  // state row (key channel)
-  const uint32_t tS = dev::tmem_addr(tmem, 32 * (warp & 3), mb * BV);
-  const long KV = (long)K * a.V;
-
-  // ---- initial state into TMEM --------------------------------------------
-  // Composed segment start: S = h0; then for every earlier segment p (later, in
-  // reverse) S = diag(gseg_p) S + delta_p -- the scan over segments, done per row.
-  // Done in 16-column blocks so that the loads of up to four segments are in
-  // flight together (the per-row chain is a sequence of dependent global loads).
-  {
-    const bool compose = (a.delta != nullptr);
-    const float *src = nullptr;
-    if (a.start) src = a.start + ((bh * P + seg) * K + c) * (long)a.V + v0;
-    else if (a.h0 && (compose || seg == (a.reverse ? P - 1 : 0))) src = a.h0 + bh * KV + (long)c * a.V + v0;
-    const int np = compose ? (a.reverse ? (P - 1 - seg) : seg) : 0;
-    auto seg_of = [&](int i) { return a.reverse ? (P - 1 - i) : i; };
-#pragma unroll 1
-    for (int cb = 0; cb < BV / 16; ++cb) {
-      float S[16];
-#pragma unroll
-      for (int x = 0; x < 4; ++x) {
-        const float4 v4 =
-            src ? __ldg(reinterpret_cast<const float4 *>(src + cb * 16) + x) : make_float4(0.f, 0.f, 0.f, 0.f);
-        S[4 * x] = v4.x;
-        S[4 * x + 1] = v4.y;
-        S[4 * x + 2] = v4.z;
-        S[4 * x + 3] = v4.w;
-      }
-      int i = 0;
-#pragma unroll 1
-      for (; i + 4 <= np; i += 4) {
-        float gs[4];
-        float4 d[4][4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int p = seg_of(i + u);
-          gs[u] = __ldg(a.gseg_in + (bh * P + p) * K + c);
-          const float4 *d4 = reinterpret_cast<const float4 *>(a.delta) +
-                             ((bh * P + p) * (a.V / 4) + v0 / 4 + cb * 4) * K + c;
-#pragma unroll
-          for (int x = 0; x < 4; ++x) d[u][x] = __ldg(d4 + (long)x * K);
-        }
-#pragma unroll
-        for (int u = 0; u < 4; ++u)
-#pragma unroll
-          for (int x = 0; x < 4; ++x) {
-            S[4 * x] = gs[u] * S[4 * x] + d[u][x].x;
-            S[4 * x + 1] = gs[u] * S[4 * x + 1] + d[u][x].y;
-            S[4 * x + 2] = gs[u] * S[4 * x + 2] + d[u][x].z;
-            S[4 * x + 3] = gs[u] * S[4 * x + 3] + d[u][x].w;
-          }
-      }
-      if (i < np) {  // 1 to 3 remaining segments, loads issued together
-        float gs[3];
-        float4 d[3][4];
-#pragma unroll
-        for (int u = 0; u < 3; ++u) {
-          if (i + u < np) {
-            const int p = seg_of(i + u);
-            gs[u] = __ldg(a.gseg_in + (bh * P + p) * K + c);
-            const float4 *d4 = reinterpret_cast<const float4 *>(a.delta) +
-                               ((bh * P + p) * (a.V / 4) + v0 / 4 + cb * 4) * K + c;
-#pragma unroll
-            for (int x = 0; x < 4; ++x) d[u][x] = __ldg(d4 + (long)x * K);
-          } else {
-            gs[u] = 1.f;
-#pragma unroll
-            for (int x = 0; x < 4; ++x) d[u][x] = make_float4(0.f, 0.f, 0.f, 0.f);
-          }
-        }
-#pragma unroll
-        for (int u = 0; u < 3; ++u)
-#pragma unroll
-          for (int x = 0; x < 4; ++x) {
-            S[4 * x] = gs[u] * S[4 * x] + d[u][x].x;
-            S[4 * x + 1] = gs[u] * S[4 * x + 1] + d[u][x].y;
-            S[4 * x + 2] = gs[u] * S[4 * x + 2] + d[u][x].z;
-            S[4 * x + 3] = gs[u] * S[4 * x + 3] + d[u][x].w;
-          }
-      }
-      dev::tmem_st16(tS + cb * 16, S);
-    }
-    dev::tmem_wait_st();
-  }
-
-  bool ok = true;
-  float gprod = 1.f;
-  // Output accumulator: two TMEM buffers when the columns allow, so that chunk
-  // i-1's output epilogue overlaps chunk i's MMAs.
-  constexpr bool kDoubleO = (kColO + 2 * BV <= kTmemCols);
-  auto o_col = [&](int i) { return (uint32_t)(kColO + (kDoubleO ? (i & 1) * BV : 0)); };
-  // rows t of the chunk (M = 64 TMEM layout: lanes 32*sub + [0,16)), bf16 to out[t][v0 + ...]
-  auto out_epilogue = [&](int i) {
-    constexpr int kWarps = kThreads / 32;
-    constexpr int kColsPerWarp = (kWarps >= 8) ? BV / 2 : BV;
-    const int sub = warp & 3;
-    const int col0 = (kWarps >= 8 && warp >= 4) ? BV / 2 : 0;
-    const int t = 16 * sub + lane;
-    const long tgl = (long)chunk_of(i) * kC + t;
-#pragma unroll
-    for (int cb = 0; cb < kColsPerWarp / 16; ++cb) {
-      float v[16];
-      dev::tmem_ld16(dev::tmem_addr(tmem, 32 * sub, o_col(i) + col0 + cb * 16), v);
-      dev::tmem_wait_ld();
-      if (lane < 16 && tgl < a.T && ok) {
-        uint4 p0, p1;
-        p0.x = dev::pack_bf16(v[0], v[1]);
-        p0.y = dev::pack_bf16(v[2], v[3]);
-        p0.z = dev::pack_bf16(v[4], v[5]);
-        p0.w = dev::pack_bf16(v[6], v[7]);
-        p1.x = dev::pack_bf16(v[8], v[9]);
-        p1.y = dev::pack_bf16(v[10], v[11]);
-        p1.z = dev::pack_bf16(v[12], v[13]);
-        p1.w = dev::pack_bf16(v[14], v[15]);
-        uint4 *dst = reinterpret_cast<uint4 *>(a.out + (bh * a.T + tgl) * (long)a.V + v0 + col0 + cb * 16);
-        dst[0] = p0;
-        dst[1] = p1;
-      }
-    }
-  };
-  float g_next = (nloc > 0) ? __ldg(a.gam + (bh * a.N + chunk_of(0)) * K + c) : 1.f;
-  for (int i = 0; i < nloc; ++i) {
-    const int s = i % nst;
-    const int n = chunk_of(i);
-    uint8_t *st = stage_ptr(s);
-    const float g = g_next;
-    if (i + 1 < nloc) g_next = __ldg(a.gam + (bh * a.N + chunk_of(i + 1)) * K + c);
-    gprod *= g;
-
-    // ---- S-pass: read S, publish bf16/fp32 copy, scale by gamma ---------------
-    // (needs only the previous chunk's MMAs: it runs while this chunk's tiles load)
-#pragma unroll
-    for (int cb = 0; cb < BV / 32; ++cb) {
-      float v[32];
-      dev::tmem_ld32(tS + cb * 32, v);
-      dev::tmem_wait_ld();
-      if (a.do_out || a.state_mode == 1) {
-        uint4 pk[4];
-#pragma unroll
-        for (int h = 0; h < 4; ++h)
-          pk[h] = make_uint4(dev::pack_bf16(v[8 * h], v[8 * h + 1]), dev::pack_bf16(v[8 * h + 2], v[8 * h + 3]),
-                             dev::pack_bf16(v[8 * h + 4], v[8 * h + 5]), dev::pack_bf16(v[8 * h + 6], v[8 * h + 7]));
-        if (a.do_out) {
-#pragma unroll
-          for (int h = 0; h < 4; ++h)
-            dev::st_shared_v4(sSb + dev::sw128_chunk(K, c, cb * 4 + h), pk[h].x, pk[h].y, pk[h].z, pk[h].w);
-        }
-        if (a.state_mode == 1) {
-          // chunk state h_n in the [K/128][V/8][128][8] layout: a warp stores 512
-          // contiguous bytes, and a 128-channel half of a 64-column tile is 16 KB
-          uint4 *dst = reinterpret_cast<uint4 *>(a.hb) +
-                       (((bh * a.N + n) * (K / 128) + (c >> 7)) * (a.V / 8) + (v0 + cb * 32) / 8) * 128 + (c & 127);
-#pragma unroll
-          for (int h = 0; h < 4; ++h) dst[h * 128] = pk[h];
-        }
-      }
-      if (a.state_mode == 2) {
-        float4 *dst = reinterpret_cast<float4 *>(a.h32 + ((bh * a.N + n) * K + c) * (long)a.V + v0 + cb * 32);
-#pragma unroll
-        for (int h = 0; h < 8; ++h) dst[h] = make_float4(v[4 * h], v[4 * h + 1], v[4 * h + 2], v[4 * h + 3]);
-      }
-#pragma unroll
-      for (int e = 0; e < 32; ++e) v[e] *= g;
-      dev::tmem_st16(tS + cb * 32, v);
-      dev::tmem_st16(tS + cb * 32 + 16, v + 16);
-    }
-    dev::tmem_wait_st();
-    dev::fence_proxy_async_smem();
-    if (ok) ok = dev::mbar_wait(&full[s], (uint32_t)((i / nst) & 1), a.status);
-    dev::tc_fence_before();
-    __syncthreads();
-    dev::tc_fence_after();
-
-    // ---- MMA issue ---------------------------------------------------------
-    if (tid == 0 && ok) {
-      const uint32_t sX = dev::smem_u32(st);
-      const uint32_t sY = sX + L::kTileX;
-      const uint32_t sQ = sY + L::kTileY;
-      const uint32_t sP = sQ + L::kTileQ;
-      if (a.do_out) {
-        const uint32_t tO = tmem + o_col(i);
-        constexpr uint32_t id_qs = dev::idesc_bf16(64, BV, false, true);
-#pragma unroll
-        for (int kk = 0; kk < K / 16; ++kk)
-          dev::umma_bf16(tO, dev::desc_kmajor(sQ, 64, 0, kk * 16), dev::desc_mnmajor(sSb, K, kk * 16, 0), id_qs,
-                         kk > 0 ? 1u : 0u);
-        if (!a.p_kmajor) {
-          // O += A V with A[t][s] = P^T tile [s][t]: MN-major A
-          constexpr uint32_t id_pv = dev::idesc_bf16(64, BV, true, true);
-#pragma unroll
-          for (int kk = 0; kk < kC / 16; ++kk)
-            dev::umma_bf16(tO, dev::desc_mnmajor(sP, 64, kk * 16, 0), dev::desc_mnmajor(sY, 64, kk * 16, 0), id_pv,
-                           1u);
-        } else {
-          // dv += A^T dO with A^T[s][t] = P^T tile [s][t]: K-major A
-          constexpr uint32_t id_pt = dev::idesc_bf16(64, BV, false, true);
-#pragma unroll
-          for (int kk = 0; kk < kC / 16; ++kk)
-            dev::umma_bf16(tO, dev::desc_kmajor(sP, 64, 0, kk * 16), dev::desc_mnmajor(sY, 64, kk * 16, 0), id_pt,
-                           1u);
-        }
-      }
-      constexpr uint32_t id_st = dev::idesc_bf16(128, BV, true, true);
-#pragma unroll
-      for (int m = 0; m < kMB; ++m)
-#pragma unroll
-        for (int kk = 0; kk < kC / 16; ++kk)
-          dev::umma_bf16(tmem + m * BV, dev::desc_mnmajor(sX, 64, kk * 16, 128 * m),
-                         dev::desc_mnmajor(sY, 64, kk * 16, 0), id_st, 1u);
-      dev::umma_commit(mma_bar);
-    }
-    // the previous chunk's output is read out while this chunk's MMAs run
-    if (a.do_out && kDoubleO && i > 0) out_epilogue(i - 1);
-    if (ok) ok = dev::mbar_wait(mma_bar, i & 1, a.status);
-    dev::tc_fence_after();
-    if (tid == 0 && ok && i + nst < nloc) issue_loads(i + nst);
-    if (a.do_out && !kDoubleO) out_epilogue(i);
-    dev::tc_fence_before();
-    __syncthreads();
-    dev::tc_fence_after();
-  }
-  if (a.do_out && kDoubleO && nloc > 0) {
-    out_epilogue(nloc - 1);
-    dev::tc_fence_before();
-    __syncthreads();
-    dev::tc_fence_after();
-  }
-
-  // ---- final state of the segment ---------------------------------------------
-  if (a.gseg && vt == 0) a.gseg[(bh * P + seg) * K + c] = gprod;
-  if (a.end && (a.end_seg < 0 || a.end_seg == seg)) {
-#pragma unroll
-    for (int cb = 0; cb < BV / 16; ++cb) {
-      float v[16];
-      dev::tmem_ld16(tS + cb * 16, v);
-      dev::tmem_wait_ld();
-      if (a.end_seg < 0) {
-        // segment contribution, float4-column layout (coalesced across the warp)
-        float4 *d4 = reinterpret_cast<float4 *>(a.end) + ((bh * P + seg) * (a.V / 4) + v0 / 4 + cb * 4) * K + c;
-#pragma unroll
-        for (int x = 0; x < 4; ++x) d4[(long)x * K] = make_float4(v[4 * x], v[4 * x + 1], v[4 * x + 2], v[4 * x + 3]);
-      } else {
-        float4 *d4 = reinterpret_cast<float4 *>(a.end + (bh * K + c) * (long)a.V + v0 + cb * 16);
-#pragma unroll
-        for (int x = 0; x < 4; ++x) d4[x] = make_float4(v[4 * x], v[4 * x + 1], v[4 * x + 2], v[4 * x + 3]);
-      }
-    }
-  }
-  dev::tc_fence_before();
-  __syncthreads();
-  if (warp == 0) dev::tmem_dealloc(tmem, kTmemCols);
-}
 
 }  // namespace tc
 }  // namespace gla

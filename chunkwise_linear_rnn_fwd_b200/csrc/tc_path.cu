@@ -18,6 +18,7 @@
 #include "tc_bwd.cuh"
 #include "tc_kernels.cuh"
 #include "tc_path.h"
+#include "tc_walk.cuh"
 
 namespace gla {
 namespace {
@@ -80,16 +81,18 @@ int sm_count() {
   });
 }
 
-int bv_of(const Problem &p) { return (p.K == 256 || p.V % 128 != 0) ? 64 : 128; }
+// d_v tiles of a walk (128 columns each; a last tile of 64 columns is padded by
+// the TMA loads' zero fill and masked on store)
+int walk_tiles(const Problem &p) { return (p.V + tc::kWalkBV - 1) / tc::kWalkBV; }
 
 // Segment count for the FUSED forward: as many segments as one wave of walk
-// CTAs (two per SM) can hold.
+// CTAs (one per SM) can hold.
 int segments_of(const Problem &p, int nvt) {
   if (p.variant == GLA_VARIANT_MATERIALIZED) return 1;
   int P = p.segments;
   if (P <= 0) {
     const long ctas = p.BH * nvt;
-    P = (int)std::max<long>(1, (2L * sm_count()) / ctas);
+    P = (int)std::max<long>(1, (long)sm_count() / ctas);
   }
   P = std::min(P, p.N);
   const int L = (p.N + P - 1) / P;
@@ -99,11 +102,11 @@ int segments_of(const Problem &p, int nvt) {
 struct TcWs {
   bf16 *qg, *kg, *PT;
   float *gam;
-  float *delta;          // [BH][P][V/4][K] float4 segment contributions
+  float *delta;          // [BH][P][K][V] segment contributions from a zero state
   float *gseg;           // [BH][P][K] per-segment gate products
   float *h32;            // materialised fp32 chunk states [BH][N][K][V]
   // backward
-  bf16 *hb, *dhb;        // bf16 chunk states and adjoints [BH][N][K/128][V/8][128][8]
+  bf16 *hb, *dhb;        // bf16 chunk states and adjoints, tc::state_chunk_off layout
   float *ddelta;
   size_t bytes;
 };
@@ -123,7 +126,7 @@ int bwd_segments(const Problem &p, int nvt) {
 TcWs carve(const Problem &p, void *ws, bool bwd) {
   Carve cv(ws);
   TcWs w{};
-  const int nvt = p.V / bv_of(p);
+  const int nvt = walk_tiles(p);
   w.qg = cv.take<bf16>((size_t)p.BH * p.Tp * p.K);
   w.kg = cv.take<bf16>((size_t)p.BH * p.Tp * p.K);
   w.PT = cv.take<bf16>((size_t)p.BH * p.N * tc::kC * tc::kC);
@@ -175,32 +178,29 @@ struct WalkMaps {
   CUtensorMap X, Y, Q, P;
 };
 
-template <int K, int BV>
+// P here is the number of segments this launch covers (a.seg0 .. a.seg0 + P - 1).
+template <int K>
 int launch_walk(const Problem &p, const tc::WalkArgs &a, const WalkMaps &m, int P, cudaStream_t st) {
-  using W = tc::WalkSmem<K, BV>;
-  constexpr int kTmemCols = ((K / 128) * BV + BV <= 256) ? 256 : 512;
+  constexpr int smem = tc::WalkTSmem<K>::kBytes + 1024;
+  static_assert(smem <= kMaxDynSmem, "walk shared memory");
   static DeviceSlots attr;  // the attribute belongs to the current device
   if (per_device(attr, [] {
-        return cudaFuncSetAttribute(tc::k_walk<K, BV>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem) ==
+        return cudaFuncSetAttribute(tc::k_walkT<K>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) ==
                        cudaSuccess
                    ? 1
                    : -1;
       }) < 0)
     return GLA_ERR_CUDA;
-  const int smem = smem_for_tmem(tc::k_walk<K, BV>, K, W::bytes(a.do_out != 0, a.do_out != 0), kTmemCols);
-  if (smem < 0) return GLA_ERR_CUDA;
   GLA_LAUNCH(K_TC_WALK, st,
-             if (launch_pdl(tc::k_walk<K, BV>, dim3(p.V / BV, P, p.BH), dim3(K), smem, st, a, m.X, m.Y, m.Q, m.P) !=
-                 cudaSuccess) return GLA_ERR_CUDA);
-  // P here is the number of segments this launch covers (a.seg0 .. a.seg0 + P - 1)
+             if (launch_pdl(tc::k_walkT<K>, dim3(walk_tiles(p), P, p.BH), dim3(tc::kWalkThreads), smem, st, a, m.X,
+                            m.Y, m.Q, m.P) != cudaSuccess) return GLA_ERR_CUDA);
   return GLA_OK;
 }
 
 int launch_walk_any(const Problem &p, const tc::WalkArgs &a, const WalkMaps &m, int P, cudaStream_t st) {
-  const int BV = bv_of(p);
-  if (p.K == 256 && BV == 64) return launch_walk<256, 64>(p, a, m, P, st);
-  if (p.K == 128 && BV == 128) return launch_walk<128, 128>(p, a, m, P, st);
-  if (p.K == 128 && BV == 64) return launch_walk<128, 64>(p, a, m, P, st);
+  if (P < 1 || P > 65535) return GLA_ERR_UNSUPPORTED_SHAPE;
+  if (p.K == 256) return launch_walk<256>(p, a, m, P, st);
+  if (p.K == 128) return launch_walk<128>(p, a, m, P, st);
   return GLA_ERR_UNSUPPORTED_SHAPE;
 }
 
@@ -252,8 +252,7 @@ int tc_fwd(const Problem &p, const void *q, const void *k, const void *v, const 
   unsigned *status = (unsigned *)ws;
   if (!(p.flags & GLA_FLAG_REUSE_PREP)) TRY(launch_prep_any(p, (const bf16 *)q, (const bf16 *)k, la, w, status, st));
 
-  const int BV = bv_of(p);
-  const int nvt = p.V / BV;
+  const int nvt = walk_tiles(p);
   WalkMaps m;
   const uint64_t BH = (uint64_t)p.BH;
   bool okm = map3(&m.X, w.kg, p.K, p.Tp, BH, 64, 64) && map3(&m.Y, v, p.V, p.T, BH, 64, 64) &&
@@ -331,8 +330,7 @@ int tc_bwd(const Problem &p, const void *q, const void *k, const void *v, const 
   // so a forward run on this workspace can hand them over
   if (!(p.flags & GLA_FLAG_REUSE_PREP)) TRY(launch_prep_any(p, (const bf16 *)q, (const bf16 *)k, la, w, status, st));
   const bool saved = (p.flags & GLA_FLAG_SAVE_STATES) != 0;
-  const int BV = bv_of(p);
-  const int nvt = p.V / BV;
+  const int nvt = walk_tiles(p);
   const int P = bwd_segments(p, nvt);
   const int L = (p.N + P - 1) / P;
   const uint64_t BH = (uint64_t)p.BH;
@@ -425,7 +423,7 @@ int tc_fwd_state(const Problem &p, const void *q, const void *k, const void *v, 
   TcWs w = carve(pf, ws, save);
   unsigned *status = (unsigned *)ws;
   if (!(p.flags & GLA_FLAG_REUSE_PREP)) TRY(launch_prep_any(pf, (const bf16 *)q, (const bf16 *)k, la, w, status, st));
-  const int nvt = p.V / bv_of(p);
+  const int nvt = walk_tiles(p);
   const int P = save ? bwd_segments(pf, nvt) : segments_of(pf, nvt);
   const uint64_t BH = (uint64_t)p.BH;
   WalkMaps m;
@@ -464,7 +462,7 @@ int tc_bwd_state(const Problem &p, const void *q, const void *k, const float *la
   TcWs w = carve(p, ws, true);
   unsigned *status = (unsigned *)ws;
   if (!(p.flags & GLA_FLAG_REUSE_PREP)) TRY(launch_prep_any(p, (const bf16 *)q, (const bf16 *)k, la, w, status, st));
-  const int nvt = p.V / bv_of(p);
+  const int nvt = walk_tiles(p);
   const int P = bwd_segments(p, nvt);
   const uint64_t BH = (uint64_t)p.BH;
   WalkMaps m;

@@ -1,0 +1,373 @@
+// tc_walk.cuh -- the inter-chunk state walk of the bf16 tensor-core path (sm_100a).
+//
+// One CTA per (128-column tile of d_v, segment, head) carries the fp32 state of
+// its tile across the chunks of one segment (section 3.3 / 4.2 of "Gated Linear
+// Attention Transformers with Hardware-Efficient Training": the chunk-level
+// recurrence S_n = diag(gam_n) S_{n-1} + kg_n^T V_n).  The state is kept
+// transposed, S^T [v][c], in the registers of 256 threads: thread (v, h) holds
+// row v of S^T for the key channels [h K/2, (h+1) K/2).  Per chunk n:
+//
+//   dS^T  = V_n^T kg_n                        tcgen05 M = 128 (v), N = K (c), K = 64 tokens
+//   S^T  <- gam_n (.) S^T + dS^T               CUDA cores, fp32, in registers
+//   O_n^T = S_{n-1}^T qg_n^T + V_n^T P_n^T     tcgen05 M = 128 (v), N = 64 (tokens);
+//           S_{n-1}^T is the A operand straight from TMEM (bf16, written there by the
+//           threads that hold it), so the state never passes through shared memory
+//
+// and the reverse (adjoint) walk runs the chunks backwards with (qg, dO) in place
+// of (kg, V) and dv_n^T = dS^T kg_n^T + dO_n^T P_n.  Warp roles: warps 0-7 hold
+// the state (and drain the output accumulator), warp 8 issues the TMA loads into
+// two rings (the key-side tiles kg / qg; the value-side tile with the intra-chunk
+// scores and the chunk's decay row), warp 9 issues the MMAs.  Every wait is
+// bounded (the status word records a timeout; the kernel then skips the dependent
+// work and ends).
+#pragma once
+
+#include "tc_kernels.cuh"
+
+namespace gla {
+namespace tc {
+
+constexpr int kWalkBV = 128;       // d_v columns per walk CTA
+constexpr int kWalkThreads = 320;  // 8 state warps + producer warp + MMA warp
+
+template <int K>
+struct WalkTSmem {
+  static constexpr int kXSlot = 64 * K * 2;             // kg or qg chunk tile [64][K] bf16, SW128
+  static constexpr int kYTile = 64 * kWalkBV * 2;       // V or dO tile [64][128] bf16, SW128
+  static constexpr int kPTile = 64 * 64 * 2;            // P^T [64][64] bf16, SW128
+  static constexpr int kYSlot = kYTile + kPTile + 1024;  // + the chunk's decay row gam [K] fp32
+  static constexpr int NX = (K == 256) ? 4 : 6;
+  static constexpr int NY = 3;
+  static constexpr int kY0 = NX * kXSlot;
+  static constexpr int kBar = kY0 + NY * kYSlot;
+  static constexpr int kBytes = kBar + 512;
+  static_assert(K * 4 <= 1024, "decay row fits its slot");
+};
+
+// Byte offset of the 16-byte chunk (value column vg, key channels 8 c8 .. 8 c8 + 7)
+// of a bf16 chunk state in the layout the backward reads:
+//   [BH*N][V/64][K/64][64 v][64 c], every [64][64] tile 128-byte swizzled (chunk
+//   j8 of row v at position j8 ^ (v % 8)),
+// so that the 128 channels of one half and one 64-column d_v tile are a contiguous
+// 16 KB block that, copied as is to a 1024-byte aligned address, is the SW128
+// layout of an MN-major operand (rows v, columns c).
+template <int K>
+__device__ __forceinline__ size_t state_chunk_off(long bhn, int V, int vg, int c8) {
+  const int vb = vg >> 6, vr = vg & 63, cb = c8 >> 3, j8 = c8 & 7;
+  return ((((size_t)bhn * (V / 64) + vb) * (K / 64) + cb) * 64 + vr) * 128 + (size_t)((j8 ^ (vr & 7)) << 4);
+}
+
+template <int K>
+// 320 threads, one CTA per SM: up to 200 registers per thread (the state rows
+// take K/2 of them)
+__global__ void __maxnreg__(200)
+    k_walkT(WalkArgs a, const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmY,
+            const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmP) {
+  using L = WalkTSmem<K>;
+  constexpr int BV = kWalkBV;
+  constexpr int KH = K / 2;  // key channels per state thread
+  constexpr int NX = L::NX, NY = L::NY;
+  constexpr int kStateWarps = 8;
+  constexpr int kTmemCols = 512;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint64_t *bars = (uint64_t *)(smem + L::kBar);
+  uint64_t *xfull = bars;             // [NX]
+  uint64_t *xempty = xfull + NX;      // [NX]
+  uint64_t *yfull = xempty + NX;      // [NY]
+  uint64_t *yempty = yfull + NY;      // [NY]  MMA commit + one arrival per state warp
+  uint64_t *dsfull = yempty + NY;     // [2]
+  uint64_t *dsempty = dsfull + 2;     // [2]   one arrival per state warp
+  uint64_t *afull = dsempty + 2;      // [1]   one arrival per state warp
+  uint64_t *ofull = afull + 1;        // [2]
+  uint64_t *oempty = ofull + 2;       // [2]   one arrival per state warp
+  uint64_t *done = oempty + 2;        // [1]   the MMA thread's last commit
+  uint32_t *tslot = (uint32_t *)(done + 1);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int vt = blockIdx.x, seg = blockIdx.y + a.seg0;
+  const long bh = blockIdx.z;
+  const int v0 = vt * BV;
+  const int n_begin = seg * a.L;
+  const int n_end = min(a.N, n_begin + a.L);
+  const int nloc = max(0, n_end - n_begin);
+  const int P = a.P;
+  const bool out = a.do_out != 0;
+  // dS buffers: two when the columns allow (every state-only walk; K = 128 with outputs)
+  const int nds = (!out || 2 * K + K / 2 + 128 <= kTmemCols) ? 2 : 1;
+  const uint32_t colA = (uint32_t)(nds * K);               // S^T (bf16) as the output MMA's A operand
+  auto colO = [&](int b) { return colA + (uint32_t)(K / 2 + 64 * b); };  // O^T accumulators (64 columns each)
+
+  if (tid == 0) {
+    for (int i = 0; i < NX; ++i) {
+      dev::mbar_init(&xfull[i], 1);
+      dev::mbar_init(&xempty[i], 1);
+    }
+    for (int i = 0; i < NY; ++i) {
+      dev::mbar_init(&yfull[i], 1);
+      dev::mbar_init(&yempty[i], 1 + kStateWarps);
+    }
+    for (int i = 0; i < 2; ++i) {
+      dev::mbar_init(&dsfull[i], 1);
+      dev::mbar_init(&dsempty[i], kStateWarps);
+      dev::mbar_init(&ofull[i], 1);
+      dev::mbar_init(&oempty[i], kStateWarps);
+    }
+    dev::mbar_init(afull, kStateWarps);
+    dev::mbar_init(done, 1);
+    dev::fence_mbar_init();
+    dev::prefetch_tmap(&tmX);
+    dev::prefetch_tmap(&tmY);
+    if (out) {
+      dev::prefetch_tmap(&tmQ);
+      dev::prefetch_tmap(&tmP);
+    }
+  }
+  dev::pdl_launch_dependents();
+  dev::pdl_wait();
+  if (warp == 0) dev::tmem_alloc(tslot, kTmemCols);
+  dev::tc_fence_before();
+  __syncthreads();
+  dev::tc_fence_after();
+  const uint32_t tmem = *tslot;
+
+  auto chunk_of = [&](int i) { return a.reverse ? (n_end - 1 - i) : (n_begin + i); };
+  auto xslot = [&](int s) { return smem + s * L::kXSlot; };
+  auto yslot = [&](int s) { return smem + L::kY0 + s * L::kYSlot; };
+
+  if (warp == kStateWarps) {
+    // ============================ TMA producer ============================
+    if (lane == 0) {
+      bool ok = true;
+      int xi = 0, yi = 0;  // loads issued into each ring
+      auto load_x = [&](const CUtensorMap *map, int n) {
+        const int s = xi % NX;
+        if (xi >= NX && ok) ok = dev::mbar_wait(&xempty[s], (uint32_t)(((xi / NX) - 1) & 1), a.status);
+        if (!ok) return;
+        dev::mbar_arrive_expect_tx(&xfull[s], (uint32_t)L::kXSlot);
+#pragma unroll
+        for (int cb = 0; cb < K / 64; ++cb)
+          dev::tma_load_3d(xslot(s) + cb * 8192, map, cb * 64, n * kC, (int)bh, &xfull[s]);
+        ++xi;
+      };
+      for (int i = 0; i < nloc && ok; ++i) {
+        const int n = chunk_of(i);
+        load_x(&tmX, n);
+        const int sy = i % NY;
+        if (i >= NY && ok) ok = dev::mbar_wait(&yempty[sy], (uint32_t)(((i / NY) - 1) & 1), a.status);
+        if (ok) {
+          ++yi;
+          uint8_t *y = yslot(sy);
+          dev::mbar_arrive_expect_tx(&yfull[sy], (uint32_t)(L::kYTile + (out ? L::kPTile : 0) + K * 4));
+#pragma unroll
+          for (int cb = 0; cb < BV / 64; ++cb)
+            dev::tma_load_3d(y + cb * 8192, &tmY, v0 + cb * 64, n * kC, (int)bh, &yfull[sy]);
+          if (out) dev::tma_load_3d(y + L::kYTile, &tmP, 0, 0, (int)(bh * a.N + n), &yfull[sy]);
+          dev::bulk_load(y + L::kYTile + L::kPTile, a.gam + (bh * a.N + n) * K, (uint32_t)(K * 4), &yfull[sy]);
+        }
+        if (out) load_x(&tmQ, n);
+      }
+      // every load issued has landed before the CTA may end (the consumers normally
+      // waited for them already; after a timeout nobody else does)
+      for (int j = max(0, xi - NX); j < xi; ++j) (void)dev::mbar_wait(&xfull[j % NX], (uint32_t)((j / NX) & 1), a.status);
+      for (int j = max(0, yi - NY); j < yi; ++j)
+        (void)dev::mbar_wait(&yfull[j % NY], (uint32_t)((j / NY) & 1), a.status);
+    }
+    __syncwarp();
+    // the product of the segment's chunk decays, per key channel (tile 0 only)
+    if (a.gseg && vt == 0) {
+      for (int c = lane; c < K; c += 32) {
+        float gp = 1.f;
+        for (int i = 0; i < nloc; ++i) gp *= __ldg(a.gam + (bh * a.N + chunk_of(i)) * K + c);
+        a.gseg[(bh * P + seg) * K + c] = gp;
+      }
+    }
+  } else if (warp == kStateWarps + 1) {
+    // ============================ MMA issuer ============================
+    if (lane == 0) {
+      bool ok = true;
+      int xi = 0;
+      constexpr uint32_t id_ds = dev::idesc_bf16(128, K, true, true);   // A = Y^T (MN), B = X (MN)
+      constexpr uint32_t id_o = dev::idesc_bf16(128, 64, false, false);  // A = S^T (TMEM), B = Q (K-major)
+      const uint32_t id_pv = a.p_kmajor ? dev::idesc_bf16(128, 64, true, false)  // B = P   (reverse)
+                                        : dev::idesc_bf16(128, 64, true, true);  // B = P^T (forward)
+      for (int i = 0; i < nloc && ok; ++i) {
+        const int sx = xi % NX, sy = i % NY, d = i % nds;
+        ok = dev::mbar_wait(&xfull[sx], (uint32_t)((xi / NX) & 1), a.status) &&
+             dev::mbar_wait(&yfull[sy], (uint32_t)((i / NY) & 1), a.status);
+        if (ok && i >= nds) ok = dev::mbar_wait(&dsempty[d], (uint32_t)(((i / nds) - 1) & 1), a.status);
+        if (!ok) break;
+        dev::tc_fence_after();
+        const uint32_t sX = dev::smem_u32(xslot(sx)), sY = dev::smem_u32(yslot(sy));
+#pragma unroll
+        for (int kk = 0; kk < kC / 16; ++kk)
+          dev::umma_bf16(tmem + (uint32_t)(d * K), dev::desc_mnmajor(sY, 64, kk * 16, 0),
+                         dev::desc_mnmajor(sX, 64, kk * 16, 0), id_ds, kk > 0 ? 1u : 0u);
+        dev::umma_commit(&dsfull[d]);
+        dev::umma_commit(&xempty[sx]);
+        ++xi;
+        if (out) {
+          const int sq = xi % NX;
+          ok = dev::mbar_wait(&xfull[sq], (uint32_t)((xi / NX) & 1), a.status) &&
+               dev::mbar_wait(afull, (uint32_t)(i & 1), a.status);
+          if (ok && i >= 2) ok = dev::mbar_wait(&oempty[i & 1], (uint32_t)(((i >> 1) - 1) & 1), a.status);
+          if (!ok) break;
+          dev::tc_fence_after();
+          const uint32_t sQ = dev::smem_u32(xslot(sq)), sP = sY + L::kYTile;
+          const uint32_t tO = tmem + colO(i & 1);
+#pragma unroll
+          for (int kk = 0; kk < K / 16; ++kk)
+            dev::umma_bf16_ts(tO, tmem + colA + (uint32_t)(kk * 8), dev::desc_kmajor(sQ, 64, 0, kk * 16), id_o,
+                              kk > 0 ? 1u : 0u);
+#pragma unroll
+          for (int kk = 0; kk < kC / 16; ++kk)
+            dev::umma_bf16(tO, dev::desc_mnmajor(sY, 64, kk * 16, 0),
+                           a.p_kmajor ? dev::desc_kmajor(sP, 64, 0, kk * 16) : dev::desc_mnmajor(sP, 64, kk * 16, 0),
+                           id_pv, 1u);
+          dev::umma_commit(&ofull[i & 1]);
+          dev::umma_commit(&xempty[sq]);
+          ++xi;
+        }
+        dev::umma_commit(&yempty[sy]);
+      }
+      // all MMAs of this thread have completed before TMEM is released
+      dev::umma_commit(done);
+      (void)dev::mbar_wait(done, 0, a.status);
+    }
+  } else {
+    // ============================ state threads ============================
+    const int q4 = warp & 3, hh = warp >> 2;
+    const int v = 32 * q4 + lane;  // TMEM lane = row of S^T
+    const int c0 = hh * KH;
+    const int vg = v0 + v;
+    const bool vok = vg < a.V;
+    const uint32_t lane_base = tmem + ((uint32_t)(32 * q4) << 16);
+    const long KV = (long)K * a.V;
+    float S[KH];
+
+    // ---- start state: h0 (or a materialised state), then the contributions of
+    // the earlier segments (later ones in reverse): S <- diag(gseg_p) S + delta_p
+    {
+      const float *src = nullptr;
+      if (a.start) src = a.start + (bh * P + seg) * KV;
+      else if (a.h0 && (a.delta != nullptr || seg == (a.reverse ? P - 1 : 0))) src = a.h0 + bh * KV;
+#pragma unroll
+      for (int j = 0; j < KH; ++j) S[j] = (src && vok) ? __ldg(src + (long)(c0 + j) * a.V + vg) : 0.f;
+      const int np = a.delta ? (a.reverse ? (P - 1 - seg) : seg) : 0;
+      for (int u = 0; u < np; ++u) {
+        const int p = a.reverse ? (P - 1 - u) : u;
+        const float *gp = a.gseg_in + (bh * P + p) * K + c0;
+        const float *dp = a.delta + (bh * P + p) * KV + vg;
+#pragma unroll
+        for (int j = 0; j < KH; ++j) S[j] = __ldg(gp + j) * S[j] + (vok ? __ldg(dp + (long)(c0 + j) * a.V) : 0.f);
+      }
+    }
+
+    bool ok = true;
+    // O_i^T (TMEM, lanes v, columns tokens) -> out[t][vg]; warp half hh takes tokens 32 hh ..
+    auto epilogue = [&](int i) {
+      float o[32];
+      dev::tmem_ld32(lane_base + colO(i & 1) + (uint32_t)(32 * hh), o);
+      dev::tmem_wait_ld();
+      dev::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) dev::mbar_arrive(&oempty[i & 1]);
+      const long t0 = (long)chunk_of(i) * kC + 32 * hh;
+      if (vok && ok) {
+        bf16 *dst = a.out + (bh * a.T + t0) * (long)a.V + vg;
+#pragma unroll
+        for (int e = 0; e < 32; ++e)
+          if (t0 + e < a.T) dst[(long)e * a.V] = __float2bfloat16_rn(o[e]);
+      }
+    };
+
+    for (int i = 0; i < nloc; ++i) {
+      const int n = chunk_of(i);
+      // ---- publish S_{i-1}: TMEM A operand of O_i, bf16 chunk state, fp32 state ----
+      if (out || a.state_mode != 0) {
+        if (out && i >= 1) {
+          if (ok) ok = dev::mbar_wait(&ofull[(i - 1) & 1], (uint32_t)(((i - 1) >> 1) & 1), a.status);
+          dev::tc_fence_after();
+        }
+        if (out || a.state_mode == 1) {
+          // 32 channels at a time: 16 packed bf16 pairs to the TMEM A operand and,
+          // for the backward, 4 x 16 bytes to the chunk-state layout
+          const bool st_hb = a.state_mode == 1 && ok && vok;
+          uint8_t *hb = reinterpret_cast<uint8_t *>(a.hb);
+          const long bhn = bh * a.N + n;
+#pragma unroll
+          for (int jb = 0; jb < KH / 32; ++jb) {
+            uint32_t w[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) w[e] = dev::pack_bf16(S[32 * jb + 2 * e], S[32 * jb + 2 * e + 1]);
+            if (out) dev::tmem_st16u(lane_base + colA + (uint32_t)(c0 / 2 + 16 * jb), w);
+            if (st_hb) {
+#pragma unroll
+              for (int x = 0; x < 4; ++x)
+                *reinterpret_cast<uint4 *>(hb + state_chunk_off<K>(bhn, a.V, vg, c0 / 8 + 4 * jb + x)) =
+                    make_uint4(w[4 * x], w[4 * x + 1], w[4 * x + 2], w[4 * x + 3]);
+            }
+          }
+          if (out) {
+            dev::tmem_wait_st();
+            dev::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) dev::mbar_arrive(afull);
+          }
+        }
+        if (a.state_mode == 2 && vok && ok) {
+          float *dst = a.h32 + (bh * a.N + n) * KV + vg;
+#pragma unroll
+          for (int j = 0; j < KH; ++j) dst[(long)(c0 + j) * a.V] = S[j];
+        }
+        if (out && i >= 1) epilogue(i - 1);
+      }
+      // ---- S_i = gam_i (.) S_{i-1} + dS_i ----------------------------------------
+      const int sy = i % NY, d = i % nds;
+      if (ok) ok = dev::mbar_wait(&yfull[sy], (uint32_t)((i / NY) & 1), a.status);
+      if (ok) ok = dev::mbar_wait(&dsfull[d], (uint32_t)((i / nds) & 1), a.status);
+      dev::tc_fence_after();
+      const float *g = reinterpret_cast<const float *>(yslot(sy) + L::kYTile + L::kPTile) + c0;
+#pragma unroll
+      for (int j = 0; j < KH / 32; ++j) {
+        float dsv[32];
+        dev::tmem_ld32(lane_base + (uint32_t)(d * K + c0 + 32 * j), dsv);
+        dev::tmem_wait_ld();
+#pragma unroll
+        for (int e4 = 0; e4 < 8; ++e4) {
+          const float4 g4 = *reinterpret_cast<const float4 *>(g + 32 * j + 4 * e4);
+          S[32 * j + 4 * e4 + 0] = g4.x * S[32 * j + 4 * e4 + 0] + dsv[4 * e4 + 0];
+          S[32 * j + 4 * e4 + 1] = g4.y * S[32 * j + 4 * e4 + 1] + dsv[4 * e4 + 1];
+          S[32 * j + 4 * e4 + 2] = g4.z * S[32 * j + 4 * e4 + 2] + dsv[4 * e4 + 2];
+          S[32 * j + 4 * e4 + 3] = g4.w * S[32 * j + 4 * e4 + 3] + dsv[4 * e4 + 3];
+        }
+      }
+      dev::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        dev::mbar_arrive(&dsempty[d]);
+        dev::mbar_arrive(&yempty[sy]);
+      }
+    }
+    if (out && nloc > 0) {
+      if (ok) ok = dev::mbar_wait(&ofull[(nloc - 1) & 1], (uint32_t)(((nloc - 1) >> 1) & 1), a.status);
+      dev::tc_fence_after();
+      epilogue(nloc - 1);
+    }
+
+    // ---- state after the segment ----------------------------------------------
+    if (a.end && (a.end_seg < 0 || a.end_seg == seg) && vok && ok) {
+      // end_seg < 0: segment contribution [BH][P][K][V]; else [BH][K][V]
+      float *dst = (a.end_seg < 0 ? a.end + (bh * P + seg) * KV : a.end + bh * KV) + vg;
+#pragma unroll
+      for (int j = 0; j < KH; ++j) dst[(long)(c0 + j) * a.V] = S[j];
+    }
+  }
+
+  dev::tc_fence_before();
+  __syncthreads();
+  if (warp == 0) dev::tmem_dealloc(tmem, kTmemCols);
+}
+
+}  // namespace tc
+}  // namespace gla
