@@ -1,5 +1,6 @@
 // gla_api.cu -- the C ABI of include/gla.h: validation, workspace sizing,
 // dispatch to the kernel paths, the device status word and launch timing.
+#include <atomic>
 #include <mutex>
 #include <vector>
 
@@ -18,6 +19,12 @@ const char *kernel_name(int id) {
   if (id < 0 || id >= K_COUNT) return "unknown";
   return names[id];
 }
+
+namespace {
+std::atomic<int> g_last_cuda_error{0};
+}  // namespace
+
+void note_cuda_error(cudaError_t e) { g_last_cuda_error.store((int)e, std::memory_order_relaxed); }
 
 // ------------------------------------------------------------------ timing
 namespace {
@@ -455,6 +462,11 @@ int gla_selftest_timeout(void *status_word, unsigned limit_us, void *stream) {
   if (!status_word || limit_us < 1 || limit_us > 1000000) return GLA_ERR_INVALID_ARG;
   if (((uintptr_t)status_word & 3u) != 0) return GLA_ERR_MISALIGNED;
   return gla::selftest_timeout((unsigned *)status_word, limit_us, (cudaStream_t)stream);
+}
+
+const char *gla_last_cuda_error(void) {
+  const int e = gla::g_last_cuda_error.load(std::memory_order_relaxed);
+  return e == 0 ? "no error" : cudaGetErrorString((cudaError_t)e);
 }
 
 const char *gla_build_info(void) {

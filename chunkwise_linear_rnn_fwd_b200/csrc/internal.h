@@ -36,6 +36,10 @@ enum KernelId : int {
 
 const char *kernel_name(int id);
 
+// The most recent CUDA runtime error that made a call return GLA_ERR_CUDA
+// (gla_last_cuda_error reports its text).
+void note_cuda_error(cudaError_t e);
+
 // Launch bracketing for gla_timing_* (no-ops unless enabled).
 void timing_begin(int kid, cudaStream_t s);
 void timing_end(int kid, cudaStream_t s);
@@ -99,10 +103,14 @@ int epilogue_bwd(const gla_desc *d, const void *o, const void *r, const float *w
 
 }  // namespace gla
 
-#define GLA_LAUNCH(kid, stream, launch_expr)                     \
-  do {                                                           \
-    gla::timing_begin((kid), (stream));                          \
-    launch_expr;                                                 \
-    gla::timing_end((kid), (stream));                            \
-    if (cudaGetLastError() != cudaSuccess) return GLA_ERR_CUDA;  \
+#define GLA_LAUNCH(kid, stream, launch_expr)         \
+  do {                                               \
+    gla::timing_begin((kid), (stream));              \
+    launch_expr;                                     \
+    gla::timing_end((kid), (stream));                \
+    const cudaError_t _le = cudaGetLastError();      \
+    if (_le != cudaSuccess) {                        \
+      gla::note_cuda_error(_le);                     \
+      return GLA_ERR_CUDA;                           \
+    }                                                \
   } while (0)

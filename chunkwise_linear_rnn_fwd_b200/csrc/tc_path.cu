@@ -185,10 +185,9 @@ int launch_walk(const Problem &p, const tc::WalkArgs &a, const WalkMaps &m, int 
   static_assert(smem <= kMaxDynSmem, "walk shared memory");
   static DeviceSlots attr;  // the attribute belongs to the current device
   if (per_device(attr, [] {
-        return cudaFuncSetAttribute(tc::k_walkT<K>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) ==
-                       cudaSuccess
-                   ? 1
-                   : -1;
+        const cudaError_t e = cudaFuncSetAttribute(tc::k_walkT<K>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) note_cuda_error(e);
+        return e == cudaSuccess ? 1 : -1;
       }) < 0)
     return GLA_ERR_CUDA;
   GLA_LAUNCH(K_TC_WALK, st,

@@ -58,9 +58,9 @@ __device__ __forceinline__ size_t state_chunk_off(long bhn, int V, int vg, int c
 }
 
 template <int K>
-// 320 threads, one CTA per SM: up to 200 registers per thread (the state rows
+// 320 threads, one CTA per SM: up to 192 registers per thread (the state rows
 // take K/2 of them)
-__global__ void __maxnreg__(200)
+__global__ void __maxnreg__(192)
     k_walkT(WalkArgs a, const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmY,
             const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmP) {
   using L = WalkTSmem<K>;

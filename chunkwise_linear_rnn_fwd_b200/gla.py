@@ -33,13 +33,16 @@ EXPORTS = ["gla_workspace_size", "gla_check", "gla_fwd", "gla_bwd", "gla_poll_st
            "gla_timing_enable", "gla_timing_collect", "gla_kernel_name", "gla_build_info", "gla_fwd_noalloc",
            "gla_decode_step", "gla_selftest_timeout", "gla_epilogue_workspace_size", "gla_epilogue_fwd",
            "gla_epilogue_bwd", "gla_fwd_state", "gla_bwd_state", "gla_state_scan", "gla_general_workspace_size",
-           "gla_fwd_general", "gla_bwd_general", "gla_poll_status_noalloc"]
+           "gla_fwd_general", "gla_bwd_general", "gla_poll_status_noalloc", "gla_last_cuda_error"]
 
 
 class GLAError(RuntimeError):
     def __init__(self, code: int, where: str):
         self.code = code
-        super().__init__(f"{where} failed: {STATUS.get(code, code)} ({status_string(code)})")
+        extra = ""
+        if code == -5:  # GLA_ERR_CUDA: name the CUDA error behind it
+            extra = f"; CUDA: {load().gla_last_cuda_error().decode()}"
+        super().__init__(f"{where} failed: {STATUS.get(code, code)} ({status_string(code)}{extra})")
 
 
 class gla_desc(ctypes.Structure):
@@ -109,6 +112,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.gla_kernel_name.restype = ctypes.c_char_p
     lib.gla_build_info.argtypes = []
     lib.gla_build_info.restype = ctypes.c_char_p
+    lib.gla_last_cuda_error.argtypes = []
+    lib.gla_last_cuda_error.restype = ctypes.c_char_p
     _lib = lib
     return lib
 

@@ -331,6 +331,11 @@ const char *gla_kernel_name(int kernel_id);
  * usable; it exists so that the timeout path can be tested. */
 int gla_selftest_timeout(void *status_word, unsigned limit_us, void *stream);
 
+/* Text of the most recent CUDA runtime error behind a GLA_ERR_CUDA return of
+ * any call in this process ("no error" if there was none; static storage).
+ * Host-only. */
+const char *gla_last_cuda_error(void);
+
 /* Build information: a static string naming the kernels and architecture. */
 const char *gla_build_info(void);
 
