@@ -17,7 +17,8 @@
 // of (kg, V) and dv_n^T = dS^T kg_n^T + dO_n^T P_n.  Warp roles: warps 0-7 hold
 // the state (and drain the output accumulator), warp 8 issues the TMA loads into
 // two rings (the key-side tiles kg / qg; the value-side tile with the intra-chunk
-// scores and the chunk's decay row), warp 9 issues the MMAs.  Every wait is
+// scores and the chunk's decay row), warp 9 issues the MMAs, warp 10 forms the
+// segment's decay product.  Every wait is
 // bounded (the status word records a timeout; the kernel then skips the dependent
 // work and ends).
 #pragma once
@@ -28,7 +29,16 @@ namespace gla {
 namespace tc {
 
 constexpr int kWalkBV = 128;       // d_v columns per walk CTA
-constexpr int kWalkThreads = 320;  // 8 state warps + producer warp + MMA warp
+constexpr int kWalkThreads = 384;  // two state warpgroups + one warpgroup for the TMA producer and MMA issuer
+// Register budgets.  Launched with 384 threads, one CTA per SM, a thread gets 168
+// registers (three warps share each of the SM's four 16K-register partitions);
+// the state warpgroups then take 224 (their state rows alone hold K/2 = 128) and
+// the producer/MMA warpgroup keeps 56: 256 x 224 + 128 x 56 = 64512 = 384 x 168.
+constexpr int kWalkRegsLaunch = 168;
+constexpr int kWalkRegsState = 224;
+constexpr int kWalkRegsRole = 56;
+static_assert(256 * kWalkRegsState + 128 * kWalkRegsRole <= kWalkThreads * kWalkRegsLaunch,
+              "register budgets exceed the launch allocation");
 
 template <int K>
 struct WalkTSmem {
@@ -58,9 +68,7 @@ __device__ __forceinline__ size_t state_chunk_off(long bhn, int V, int vg, int c
 }
 
 template <int K>
-// 320 threads, one CTA per SM: up to 192 registers per thread (the state rows
-// take K/2 of them)
-__global__ void __maxnreg__(192)
+__global__ void __launch_bounds__(kWalkThreads, 1)
     k_walkT(WalkArgs a, const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmY,
             const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmP) {
   using L = WalkTSmem<K>;
@@ -135,7 +143,9 @@ __global__ void __maxnreg__(192)
   auto xslot = [&](int s) { return smem + s * L::kXSlot; };
   auto yslot = [&](int s) { return smem + L::kY0 + s * L::kYSlot; };
 
-  if (warp == kStateWarps) {
+  if (warp >= kStateWarps) {
+    dev::regs_dec<kWalkRegsRole>();
+    if (warp == kStateWarps) {
     // ============================ TMA producer ============================
     if (lane == 0) {
       bool ok = true;
@@ -173,7 +183,7 @@ __global__ void __maxnreg__(192)
       for (int j = max(0, yi - NY); j < yi; ++j)
         (void)dev::mbar_wait(&yfull[j % NY], (uint32_t)((j / NY) & 1), a.status);
     }
-    __syncwarp();
+    } else if (warp == kStateWarps + 2) {
     // the product of the segment's chunk decays, per key channel (tile 0 only)
     if (a.gseg && vt == 0) {
       for (int c = lane; c < K; c += 32) {
@@ -182,7 +192,7 @@ __global__ void __maxnreg__(192)
         a.gseg[(bh * P + seg) * K + c] = gp;
       }
     }
-  } else if (warp == kStateWarps + 1) {
+    } else if (warp == kStateWarps + 1) {
     // ============================ MMA issuer ============================
     if (lane == 0) {
       bool ok = true;
@@ -234,7 +244,9 @@ __global__ void __maxnreg__(192)
       dev::umma_commit(done);
       (void)dev::mbar_wait(done, 0, a.status);
     }
+    }
   } else {
+    dev::regs_inc<kWalkRegsState>();
     // ============================ state threads ============================
     const int q4 = warp & 3, hh = warp >> 2;
     const int v = 32 * q4 + lane;  // TMEM lane = row of S^T
