@@ -747,17 +747,19 @@ def run_ours(args, w):
         "flops_per_step": flops, "algorithmic_bytes_per_step": abytes, "peak_source": peak_src,
     }
 
-    decode = measure_decode(args, dev, stream, peaks, peak_src, seed=rank)
-    epilogue = measure_epilogue(args, w, dev, stream, peaks, peak_src, seed=rank)
-    seqpar = measure_seqpar(args, w, dev, stream, seed=rank)
-    variants = measure_variants(args, w, dev, stream, seed=rank)
-    sweep_args = argparse.Namespace(steps=5, warmup=2)
-    sweep_T = [time_workload(c, sweep_args, dev, stream, peaks) for c in SWEEP_T]
-    general = measure_general_gate(args, w, dev, stream, seed=rank)
-    general["vs_alpha_only_step"] = general["ms_per_step"] / ms_per_step
+    decode = epilogue = seqpar = variants = general = sweep_T = None
+    if not args.step_only:
+        decode = measure_decode(args, dev, stream, peaks, peak_src, seed=rank)
+        epilogue = measure_epilogue(args, w, dev, stream, peaks, peak_src, seed=rank)
+        seqpar = measure_seqpar(args, w, dev, stream, seed=rank)
+        variants = measure_variants(args, w, dev, stream, seed=rank)
+        sweep_args = argparse.Namespace(steps=5, warmup=2)
+        sweep_T = [time_workload(c, sweep_args, dev, stream, peaks) for c in SWEEP_T]
+        general = measure_general_gate(args, w, dev, stream, seed=rank)
+        general["vs_alpha_only_step"] = general["ms_per_step"] / ms_per_step
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.step_only:
         r, dt, threads, desc = oracle_sample_rate(w, T_sample=w["T"], min_seconds=args.cpu_seconds)
         cpu = {"value": r, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": desc, "seconds": dt,
                **host_cpu()}
@@ -776,8 +778,9 @@ def run_ours(args, w):
             "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "clocks": clocks, "cpu_baseline": cpu, "decode_step": decode, "layer_epilogue": epilogue,
             "sequence_parallel": seqpar, "general_gate": general, "variants": variants,
-            "sweep_vs_T": {"workloads": sweep_T, "steps": 5, "peak_source": peak_src,
-                           "l2": "inputs larger than L2 (B*T = 32768 tokens, >= 1 GB per step)"},
+            "sweep_vs_T": None if sweep_T is None else {
+                "workloads": sweep_T, "steps": 5, "peak_source": peak_src,
+                "l2": "inputs larger than L2 (B*T = 32768 tokens, >= 1 GB per step)"},
         }
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -824,6 +827,9 @@ def main():
     ap.add_argument("--heads", type=int, default=None, help="override H")
     ap.add_argument("--seqlen", type=int, default=None, help="override T")
     ap.add_argument("--sweep", action="store_true", help="time every workload configuration (one JSON line)")
+    ap.add_argument("--step-only", action="store_true",
+                    help="time the fwd+bwd step alone (no decode, epilogue, sequence-parallel, variant, sweep, "
+                         "general-gate or CPU measurements): the command line of the profiler captures")
     ap.add_argument("--epilogue-once", action="store_true",
                     help="run the layer epilogue forward and backward twice on the workload's output shape and "
                          "exit (a small case for profiler captures; prints no bench line)")

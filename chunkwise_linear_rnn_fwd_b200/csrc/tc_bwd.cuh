@@ -3,9 +3,10 @@
 // One CTA per (chunk n, head, half of the key channels): 128 threads, one per key
 // channel c of its half.  Inputs: the chunk state h_n (state before chunk n) and
 // adjoint dh_n (gradient w.r.t. the state after chunk n), both bf16 in the walk's
-// chunk-state layout (state_chunk_off: per 64-column d_v tile and channel half a
-// contiguous 16 KB block, [2 channel blocks][64 v][64 c] 128-byte swizzled); gam
-// from the prep kernel; q, k, V, dO and log_alpha.  (dv comes from the reverse walk, which holds dh_n on chip.)
+// chunk-state layout [BH*N][K/8][V][8] (state_chunk_off), fetched per 64-column
+// d_v tile as one 4-D TMA box [16 channel groups][64 v][8 c] (no swizzle: the
+// MN-major operand layout of 8 x 8 core matrices); gam from the prep kernel; q, k,
+// V, dO and log_alpha.  (dv comes from the reverse walk, which holds dh_n on chip.)
 // With B the chunk-local cumulative log-gate:
 //   phase 1 (loop over d_v tiles of 64, accumulating in TMEM):
 //     dqh^T = h_n dO^T          dkh^T = dh_n V^T         dP = dO V^T
@@ -58,7 +59,7 @@ struct BwdArgs {
 
 struct BwdSmem {
   static constexpr int BVb = 64;
-  static constexpr int kTileH = kBwdKH * BVb * 2;         // h or dh half-tile, [2][64 v][64 c] bf16, SW128
+  static constexpr int kTileH = kBwdKH * BVb * 2;         // h or dh half-tile, [16][64 v][8 c] bf16
   static constexpr int kTileV = 64 * BVb * 2;             // V or dO tile, SW128
   static constexpr int kStage = 2 * kTileH + 2 * kTileV;  // h, dh, V, dO
   static constexpr int kPhase1End = 2 * kStage;
@@ -73,15 +74,16 @@ struct BwdSmem {
   static constexpr int kKt = kQt + 64 * kBwdKH * 2;           // k tile [64][128] bf16
   static constexpr int kPhase2End = kKt + 64 * kBwdKH * 2;
   static constexpr int kRed = (kPhase1End > kPhase2End ? kPhase1End : kPhase2End);  // scalar-gate sums [4][64]
-  static constexpr int kRed2 = kRed + 4 * 64 * 4;            // partial sums of h (.) dh [8 row groups][128]
-  static constexpr int kBar = kRed2 + 8 * kBwdKH * 4;
+  static constexpr int kRed2 = kRed + 4 * 64 * 4;            // sums of h (.) dh [128]
+  static constexpr int kBar = kRed2 + kBwdKH * 4;
   static constexpr int kBytes = kBar + 128;
 };
 
 template <int K>
 __global__ void __launch_bounds__(kBwdKH, 2)
     k_bwd_main(BwdArgs a, const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
-               const __grid_constant__ CUtensorMap tmQin, const __grid_constant__ CUtensorMap tmKin) {
+               const __grid_constant__ CUtensorMap tmQin, const __grid_constant__ CUtensorMap tmKin,
+               const __grid_constant__ CUtensorMap tmH, const __grid_constant__ CUtensorMap tmDH) {
   using L = BwdSmem;
   constexpr int BVb = L::BVb;
   constexpr int kH = K / kBwdKH;  // CTAs per chunk
@@ -116,6 +118,8 @@ __global__ void __launch_bounds__(kBwdKH, 2)
     dev::fence_mbar_init();
     dev::prefetch_tmap(&tmV);
     dev::prefetch_tmap(&tmDO);
+    dev::prefetch_tmap(&tmH);
+    dev::prefetch_tmap(&tmDH);
   }
   dev::pdl_launch_dependents();
   {
@@ -132,19 +136,15 @@ __global__ void __launch_bounds__(kBwdKH, 2)
   dev::tc_fence_after();
   const uint32_t tmem = *tslot;
 
-  // this CTA's 128 channels of h_n / dh_n for d_v tile i: 16 contiguous KB at
-  // ((hrow * V/64 + i) * K/64 + 2 half) * 64 * 64 elements
-  const long half_tile = (long)K * BVb;  // bf16 elements from one d_v tile to the next
-  const bf16 *h_src = a.hb + (hrow * (a.V / 64) * K / 64 + 2 * half) * 4096;
-  const bf16 *dh_src = a.dhb + (hrow * (a.V / 64) * K / 64 + 2 * half) * 4096;
   auto stage = [&](int s) { return smem + s * L::kStage; };
   auto issue_tile = [&](int i) {
     const int s = i & 1;
     uint8_t *st = stage(s);
     const int v0 = i * BVb;
     dev::mbar_arrive_expect_tx(&full[s], (uint32_t)L::kStage);
-    dev::bulk_load(st, h_src + i * half_tile, (uint32_t)L::kTileH, &full[s]);
-    dev::bulk_load(st + L::kTileH, dh_src + i * half_tile, (uint32_t)L::kTileH, &full[s]);
+    // the 16 channel groups of this half, value columns v0 .. v0 + 63 of chunk row hrow
+    dev::tma_load_4d(st, &tmH, 0, v0, (kBwdKH / 8) * half, (int)hrow, &full[s]);
+    dev::tma_load_4d(st + L::kTileH, &tmDH, 0, v0, (kBwdKH / 8) * half, (int)hrow, &full[s]);
     dev::tma_load_3d(st + 2 * L::kTileH, &tmV, v0, n * kC, (int)bh, &full[s]);
     dev::tma_load_3d(st + 2 * L::kTileH + L::kTileV, &tmDO, v0, n * kC, (int)bh, &full[s]);
   };
@@ -155,11 +155,11 @@ __global__ void __launch_bounds__(kBwdKH, 2)
 
   const int cl = tid;     // key channel within this CTA's half
   const int c = c0 + cl;  // key channel
-  // partial sums of h (.) dh: thread -> 16-byte column chunk cc (channels 8 cc .. 8 cc + 7
-  // of this half), rows v = rg + 8 r of every d_v tile (in the swizzled tile, row v's
-  // chunk cc sits at position (cc % 8) ^ (v % 8) = (cc % 8) ^ rg of block cc / 8)
-  const int cc = tid & 15, rg = tid >> 4;
-  const uint32_t r_off = (uint32_t)((cc >> 3) * 8192 + rg * 128 + (((cc & 7) ^ rg) << 4));
+  // partial sums of h (.) dh: thread -> channel group cg = 4 warp + lane / 8 (channels
+  // 8 cg .. 8 cg + 7 of this half) and value columns v = lane % 8 + 8 r of every d_v
+  // tile; the 8 lanes of a group read 128 contiguous bytes (no bank conflict)
+  const int cg = 4 * warp + (lane >> 3), vs = lane & 7;
+  const uint32_t r_off = (uint32_t)(cg * 1024 + vs * 16);
   float Racc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
   bool ok = true;
 
@@ -178,12 +178,14 @@ __global__ void __launch_bounds__(kBwdKH, 2)
 #pragma unroll
       for (int kk = 0; kk < BVb / 16; ++kk) {
         const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
+        // h / dh as MN-major A without swizzle: 8 (v) x 16-byte (8 c) core matrices,
+        // 1024 bytes apart along c (leading byte offset), 128 apart along v (stride byte offset)
         if (warp == 0)
-          dev::umma_bf16(tmem + cDQ, dev::desc_mnmajor(sH, 64, kk * 16, 0), dev::desc_kmajor(sDO, 64, 0, kk * 16),
-                         id_kk128, acc);
+          dev::umma_bf16(tmem + cDQ, dev::sdesc_noswz(sH + (uint32_t)(kk * 256), 1024u, 128u),
+                         dev::desc_kmajor(sDO, 64, 0, kk * 16), id_kk128, acc);
         else if (warp == 1)
-          dev::umma_bf16(tmem + cDK, dev::desc_mnmajor(sDH, 64, kk * 16, 0), dev::desc_kmajor(sV, 64, 0, kk * 16),
-                         id_kk128, acc);
+          dev::umma_bf16(tmem + cDK, dev::sdesc_noswz(sDH + (uint32_t)(kk * 256), 1024u, 128u),
+                         dev::desc_kmajor(sV, 64, 0, kk * 16), id_kk128, acc);
         else
           dev::umma_bf16(tmem + cDP, dev::desc_kmajor(sDO, 64, 0, kk * 16), dev::desc_kmajor(sV, 64, 0, kk * 16),
                          id_kk64, acc);
@@ -197,10 +199,10 @@ __global__ void __launch_bounds__(kBwdKH, 2)
         uint4 x, y;
         asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];"
                      : "=r"(x.x), "=r"(x.y), "=r"(x.z), "=r"(x.w)
-                     : "r"(sh + (uint32_t)(r * 1024)));
+                     : "r"(sh + (uint32_t)(r * 128)));
         asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];"
                      : "=r"(y.x), "=r"(y.y), "=r"(y.z), "=r"(y.w)
-                     : "r"(sdh + (uint32_t)(r * 1024)));
+                     : "r"(sdh + (uint32_t)(r * 128)));
         const __nv_bfloat162 *xh = reinterpret_cast<const __nv_bfloat162 *>(&x);
         const __nv_bfloat162 *yh = reinterpret_cast<const __nv_bfloat162 *>(&y);
 #pragma unroll
@@ -217,14 +219,19 @@ __global__ void __launch_bounds__(kBwdKH, 2)
     if (tid == 0 && ok && i + 2 < nvt) issue_tile(i + 2);
   }
 
-  // R[c] = sum_v h[c,v] dh[c,v]: the row groups' partial sums meet in shared memory
+  // R[c] = sum_v h[c,v] dh[c,v]: the 8 lanes of a channel group add their partial
+  // sums, then each channel's thread reads its total
   float *red2 = (float *)(smem + L::kRed2);
 #pragma unroll
-  for (int e = 0; e < 8; ++e) red2[rg * kBwdKH + 8 * cc + e] = Racc[e];
+  for (int e = 0; e < 8; ++e) {
+    float x = Racc[e];
+    x += __shfl_xor_sync(0xffffffffu, x, 1);
+    x += __shfl_xor_sync(0xffffffffu, x, 2);
+    x += __shfl_xor_sync(0xffffffffu, x, 4);
+    if (vs == 0) red2[8 * cg + e] = x;
+  }
   __syncthreads();
-  float R = 0.f;
-#pragma unroll
-  for (int g8 = 0; g8 < 8; ++g8) R += red2[g8 * kBwdKH + cl];
+  const float R = red2[cl];
 
   // ============================ phase 2 ============================
   // q and k columns of this half into the space phase 1 no longer uses
@@ -514,20 +521,24 @@ int launch_bwd_main_k(const Problem &p, const BwdArgs &a, const CUtensorMap *map
   if (smem < 0) return GLA_ERR_CUDA;
   GLA_LAUNCH(K_TC_BWD, st,
              if (launch_pdl(k_bwd_main<K>, dim3(K / kBwdKH, p.N, p.BH), dim3(kBwdKH), smem, st, a, maps[0], maps[1],
-                            maps[2], maps[3]) != cudaSuccess) return GLA_ERR_CUDA);
+                            maps[2], maps[3], maps[4], maps[5]) != cudaSuccess) return GLA_ERR_CUDA);
   return GLA_OK;
 }
 
 bool map3_bf16(CUtensorMap *m, const void *base, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t b0, uint32_t b1);
+// The chunk states [BH*N][K/8][V][8] bf16 as a 4-D map (8, V, K/8, BH*N), box
+// (8, 64, 16, 1), no swizzle.
+bool map_states(CUtensorMap *m, const void *base, uint64_t V, uint64_t K, uint64_t rows);
 
 inline int launch_bwd_main(const Problem &p, const bf16 *q, const bf16 *k, const bf16 *v, const float *la,
                            const bf16 *dout, bf16 *dq, bf16 *dk, float *dla, const float *gam, const bf16 *hb,
                            const bf16 *dhb, unsigned *status, cudaStream_t st) {
   if (p.V % 64 != 0 || p.K % kBwdKH != 0) return GLA_ERR_UNSUPPORTED_SHAPE;
-  CUtensorMap maps[4];
+  CUtensorMap maps[6];
   const uint64_t BH = (uint64_t)p.BH;
   const bool ok = map3_bf16(&maps[0], v, p.V, p.T, BH, 64, 64) && map3_bf16(&maps[1], dout, p.V, p.T, BH, 64, 64) &&
-                  map3_bf16(&maps[2], q, p.K, p.T, BH, 64, 64) && map3_bf16(&maps[3], k, p.K, p.T, BH, 64, 64);
+                  map3_bf16(&maps[2], q, p.K, p.T, BH, 64, 64) && map3_bf16(&maps[3], k, p.K, p.T, BH, 64, 64) &&
+                  map_states(&maps[4], hb, p.V, p.K, BH * p.N) && map_states(&maps[5], dhb, p.V, p.K, BH * p.N);
   if (!ok) return GLA_ERR_CUDA;
   // with a scalar gate and two channel halves, dlog alpha is summed by atomic adds
   if (p.gate == GLA_GATE_SCALAR && p.K > kBwdKH)

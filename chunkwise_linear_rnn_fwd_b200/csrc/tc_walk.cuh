@@ -56,15 +56,14 @@ struct WalkTSmem {
 
 // Byte offset of the 16-byte chunk (value column vg, key channels 8 c8 .. 8 c8 + 7)
 // of a bf16 chunk state in the layout the backward reads:
-//   [BH*N][V/64][K/64][64 v][64 c], every [64][64] tile 128-byte swizzled (chunk
-//   j8 of row v at position j8 ^ (v % 8)),
-// so that the 128 channels of one half and one 64-column d_v tile are a contiguous
-// 16 KB block that, copied as is to a 1024-byte aligned address, is the SW128
-// layout of an MN-major operand (rows v, columns c).
+//   [BH*N][K/8][V][8]  (8 consecutive key channels of one value column per 16 bytes)
+// A warp of the walk (32 consecutive value columns) stores 512 contiguous bytes per
+// instruction, and the backward fetches a (64-column d_v tile, 128-channel half) as
+// one 4-D TMA box, [16 channel groups][64 v][8 c], the no-swizzle MN-major operand
+// layout (core matrices of 8 v x 8 c).
 template <int K>
 __device__ __forceinline__ size_t state_chunk_off(long bhn, int V, int vg, int c8) {
-  const int vb = vg >> 6, vr = vg & 63, cb = c8 >> 3, j8 = c8 & 7;
-  return ((((size_t)bhn * (V / 64) + vb) * (K / 64) + cb) * 64 + vr) * 128 + (size_t)((j8 ^ (vr & 7)) << 4);
+  return (((size_t)bhn * (K / 8) + c8) * (size_t)V + vg) * 16;
 }
 
 template <int K>
