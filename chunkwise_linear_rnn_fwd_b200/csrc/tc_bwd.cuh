@@ -178,13 +178,14 @@ __global__ void __launch_bounds__(kBwdKH, 2)
 #pragma unroll
       for (int kk = 0; kk < BVb / 16; ++kk) {
         const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
-        // h / dh as MN-major A without swizzle: 8 (v) x 16-byte (8 c) core matrices,
-        // 1024 bytes apart along c (leading byte offset), 128 apart along v (stride byte offset)
+        // h / dh as MN-major A without swizzle: 8 (v) x 16-byte (8 c) core matrices;
+        // in this layout type the leading byte offset steps along K (8 v rows: 128
+        // bytes) and the stride byte offset along M (8 channels: 1024 bytes)
         if (warp == 0)
-          dev::umma_bf16(tmem + cDQ, dev::sdesc_noswz(sH + (uint32_t)(kk * 256), 1024u, 128u),
+          dev::umma_bf16(tmem + cDQ, dev::sdesc_noswz(sH + (uint32_t)(kk * 256), 128u, 1024u),
                          dev::desc_kmajor(sDO, 64, 0, kk * 16), id_kk128, acc);
         else if (warp == 1)
-          dev::umma_bf16(tmem + cDK, dev::sdesc_noswz(sDH + (uint32_t)(kk * 256), 1024u, 128u),
+          dev::umma_bf16(tmem + cDK, dev::sdesc_noswz(sDH + (uint32_t)(kk * 256), 128u, 1024u),
                          dev::desc_kmajor(sV, 64, 0, kk * 16), id_kk128, acc);
         else
           dev::umma_bf16(tmem + cDP, dev::desc_kmajor(sDO, 64, 0, kk * 16), dev::desc_kmajor(sV, 64, 0, kk * 16),

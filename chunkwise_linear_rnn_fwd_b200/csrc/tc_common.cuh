@@ -273,7 +273,8 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo_bytes, ui
 
 // Shared-memory matrix descriptor without swizzle (layout type 0), version 1:
 // 8-row x 16-byte core matrices; lbo = byte distance between core matrices
-// adjacent along K, sbo = between core matrices adjacent along M/N.
+// adjacent along K, sbo = between core matrices adjacent along M/N (for K-major
+// operands, whose core-matrix rows are M/N, and for MN-major ones, whose rows are K).
 __device__ __forceinline__ uint64_t sdesc_noswz(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
   uint64_t d = 0;
   d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
