@@ -3,10 +3,10 @@
 // One CTA per (chunk n, head, half of the key channels): 128 threads, one per key
 // channel c of its half.  Inputs: the chunk state h_n (state before chunk n) and
 // adjoint dh_n (gradient w.r.t. the state after chunk n), both bf16 in the walk's
-// chunk-state layout [BH*N][K/8][V][8] (state_chunk_off), fetched per 64-column
-// d_v tile as one 4-D TMA box [16 channel groups][64 v][8 c] (no swizzle: the
-// MN-major operand layout of 8 x 8 core matrices); gam from the prep kernel; q, k,
-// V, dO and log_alpha.  (dv comes from the reverse walk, which holds dh_n on chip.)
+// chunk-state layout (state_chunk_off): per 64-column d_v tile and channel half a
+// contiguous 16 KB block of 8 x 8 core matrices [8 v-groups][16 c-groups][8 v][8 c],
+// fetched with one bulk copy and read as the no-swizzle MN-major operand; gam from
+// the prep kernel; q, k, V, dO and log_alpha.  (dv comes from the reverse walk, which holds dh_n on chip.)
 // With B the chunk-local cumulative log-gate:
 //   phase 1 (loop over d_v tiles of 64, accumulating in TMEM):
 //     dqh^T = h_n dO^T          dkh^T = dh_n V^T         dP = dO V^T
@@ -59,7 +59,7 @@ struct BwdArgs {
 
 struct BwdSmem {
   static constexpr int BVb = 64;
-  static constexpr int kTileH = kBwdKH * BVb * 2;         // h or dh half-tile, [16][64 v][8 c] bf16
+  static constexpr int kTileH = kBwdKH * BVb * 2;         // h or dh half-tile, [8][16][8 v][8 c] bf16
   static constexpr int kTileV = 64 * BVb * 2;             // V or dO tile, SW128
   static constexpr int kStage = 2 * kTileH + 2 * kTileV;  // h, dh, V, dO
   static constexpr int kPhase1End = 2 * kStage;
@@ -82,8 +82,7 @@ struct BwdSmem {
 template <int K>
 __global__ void __launch_bounds__(kBwdKH, 2)
     k_bwd_main(BwdArgs a, const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
-               const __grid_constant__ CUtensorMap tmQin, const __grid_constant__ CUtensorMap tmKin,
-               const __grid_constant__ CUtensorMap tmH, const __grid_constant__ CUtensorMap tmDH) {
+               const __grid_constant__ CUtensorMap tmQin, const __grid_constant__ CUtensorMap tmKin) {
   using L = BwdSmem;
   constexpr int BVb = L::BVb;
   constexpr int kH = K / kBwdKH;  // CTAs per chunk
@@ -118,8 +117,6 @@ __global__ void __launch_bounds__(kBwdKH, 2)
     dev::fence_mbar_init();
     dev::prefetch_tmap(&tmV);
     dev::prefetch_tmap(&tmDO);
-    dev::prefetch_tmap(&tmH);
-    dev::prefetch_tmap(&tmDH);
   }
   dev::pdl_launch_dependents();
   {
@@ -136,15 +133,18 @@ __global__ void __launch_bounds__(kBwdKH, 2)
   dev::tc_fence_after();
   const uint32_t tmem = *tslot;
 
+  // this CTA's 16 KB block of h_n / dh_n for d_v tile i: ((hrow * V/64 + i) * K/128 + half) * 8192 elements
+  const bf16 *h_src = a.hb + (hrow * (a.V / 64) * kH + half) * (long)(kBwdKH * BVb);
+  const bf16 *dh_src = a.dhb + (hrow * (a.V / 64) * kH + half) * (long)(kBwdKH * BVb);
+  const long tile_step = (long)K * BVb;  // elements from one d_v tile to the next
   auto stage = [&](int s) { return smem + s * L::kStage; };
   auto issue_tile = [&](int i) {
     const int s = i & 1;
     uint8_t *st = stage(s);
     const int v0 = i * BVb;
     dev::mbar_arrive_expect_tx(&full[s], (uint32_t)L::kStage);
-    // the 16 channel groups of this half, value columns v0 .. v0 + 63 of chunk row hrow
-    dev::tma_load_4d(st, &tmH, 0, v0, (kBwdKH / 8) * half, (int)hrow, &full[s]);
-    dev::tma_load_4d(st + L::kTileH, &tmDH, 0, v0, (kBwdKH / 8) * half, (int)hrow, &full[s]);
+    dev::bulk_load(st, h_src + i * tile_step, (uint32_t)L::kTileH, &full[s]);
+    dev::bulk_load(st + L::kTileH, dh_src + i * tile_step, (uint32_t)L::kTileH, &full[s]);
     dev::tma_load_3d(st + 2 * L::kTileH, &tmV, v0, n * kC, (int)bh, &full[s]);
     dev::tma_load_3d(st + 2 * L::kTileH + L::kTileV, &tmDO, v0, n * kC, (int)bh, &full[s]);
   };
@@ -156,10 +156,10 @@ __global__ void __launch_bounds__(kBwdKH, 2)
   const int cl = tid;     // key channel within this CTA's half
   const int c = c0 + cl;  // key channel
   // partial sums of h (.) dh: thread -> channel group cg = 4 warp + lane / 8 (channels
-  // 8 cg .. 8 cg + 7 of this half) and value columns v = lane % 8 + 8 r of every d_v
-  // tile; the 8 lanes of a group read 128 contiguous bytes (no bank conflict)
+  // 8 cg .. 8 cg + 7 of this half) and value columns v = 8 r + lane % 8 of every d_v
+  // tile (core matrix (r, cg)); a warp reads 512 contiguous bytes (no bank conflict)
   const int cg = 4 * warp + (lane >> 3), vs = lane & 7;
-  const uint32_t r_off = (uint32_t)(cg * 1024 + vs * 16);
+  const uint32_t r_off = (uint32_t)(cg * 128 + vs * 16);
   float Racc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
   bool ok = true;
 
@@ -179,13 +179,13 @@ __global__ void __launch_bounds__(kBwdKH, 2)
       for (int kk = 0; kk < BVb / 16; ++kk) {
         const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
         // h / dh as MN-major A without swizzle: 8 (v) x 16-byte (8 c) core matrices;
-        // in this layout type the leading byte offset steps along K (8 v rows: 128
-        // bytes) and the stride byte offset along M (8 channels: 1024 bytes)
+        // in this layout type the leading byte offset steps along K (8 value
+        // columns: 2048 bytes) and the stride byte offset along M (8 channels: 128)
         if (warp == 0)
-          dev::umma_bf16(tmem + cDQ, dev::sdesc_noswz(sH + (uint32_t)(kk * 256), 128u, 1024u),
+          dev::umma_bf16(tmem + cDQ, dev::sdesc_noswz(sH + (uint32_t)(kk * 4096), 2048u, 128u),
                          dev::desc_kmajor(sDO, 64, 0, kk * 16), id_kk128, acc);
         else if (warp == 1)
-          dev::umma_bf16(tmem + cDK, dev::sdesc_noswz(sDH + (uint32_t)(kk * 256), 128u, 1024u),
+          dev::umma_bf16(tmem + cDK, dev::sdesc_noswz(sDH + (uint32_t)(kk * 4096), 2048u, 128u),
                          dev::desc_kmajor(sV, 64, 0, kk * 16), id_kk128, acc);
         else
           dev::umma_bf16(tmem + cDP, dev::desc_kmajor(sDO, 64, 0, kk * 16), dev::desc_kmajor(sV, 64, 0, kk * 16),
@@ -200,10 +200,10 @@ __global__ void __launch_bounds__(kBwdKH, 2)
         uint4 x, y;
         asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];"
                      : "=r"(x.x), "=r"(x.y), "=r"(x.z), "=r"(x.w)
-                     : "r"(sh + (uint32_t)(r * 128)));
+                     : "r"(sh + (uint32_t)(r * 2048)));
         asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];"
                      : "=r"(y.x), "=r"(y.y), "=r"(y.z), "=r"(y.w)
-                     : "r"(sdh + (uint32_t)(r * 128)));
+                     : "r"(sdh + (uint32_t)(r * 2048)));
         const __nv_bfloat162 *xh = reinterpret_cast<const __nv_bfloat162 *>(&x);
         const __nv_bfloat162 *yh = reinterpret_cast<const __nv_bfloat162 *>(&y);
 #pragma unroll
@@ -522,24 +522,20 @@ int launch_bwd_main_k(const Problem &p, const BwdArgs &a, const CUtensorMap *map
   if (smem < 0) return GLA_ERR_CUDA;
   GLA_LAUNCH(K_TC_BWD, st,
              if (launch_pdl(k_bwd_main<K>, dim3(K / kBwdKH, p.N, p.BH), dim3(kBwdKH), smem, st, a, maps[0], maps[1],
-                            maps[2], maps[3], maps[4], maps[5]) != cudaSuccess) return GLA_ERR_CUDA);
+                            maps[2], maps[3]) != cudaSuccess) return GLA_ERR_CUDA);
   return GLA_OK;
 }
 
 bool map3_bf16(CUtensorMap *m, const void *base, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t b0, uint32_t b1);
-// The chunk states [BH*N][K/8][V][8] bf16 as a 4-D map (8, V, K/8, BH*N), box
-// (8, 64, 16, 1), no swizzle.
-bool map_states(CUtensorMap *m, const void *base, uint64_t V, uint64_t K, uint64_t rows);
 
 inline int launch_bwd_main(const Problem &p, const bf16 *q, const bf16 *k, const bf16 *v, const float *la,
                            const bf16 *dout, bf16 *dq, bf16 *dk, float *dla, const float *gam, const bf16 *hb,
                            const bf16 *dhb, unsigned *status, cudaStream_t st) {
   if (p.V % 64 != 0 || p.K % kBwdKH != 0) return GLA_ERR_UNSUPPORTED_SHAPE;
-  CUtensorMap maps[6];
+  CUtensorMap maps[4];
   const uint64_t BH = (uint64_t)p.BH;
   const bool ok = map3_bf16(&maps[0], v, p.V, p.T, BH, 64, 64) && map3_bf16(&maps[1], dout, p.V, p.T, BH, 64, 64) &&
-                  map3_bf16(&maps[2], q, p.K, p.T, BH, 64, 64) && map3_bf16(&maps[3], k, p.K, p.T, BH, 64, 64) &&
-                  map_states(&maps[4], hb, p.V, p.K, BH * p.N) && map_states(&maps[5], dhb, p.V, p.K, BH * p.N);
+                  map3_bf16(&maps[2], q, p.K, p.T, BH, 64, 64) && map3_bf16(&maps[3], k, p.K, p.T, BH, 64, 64);
   if (!ok) return GLA_ERR_CUDA;
   // with a scalar gate and two channel halves, dlog alpha is summed by atomic adds
   if (p.gate == GLA_GATE_SCALAR && p.K > kBwdKH)

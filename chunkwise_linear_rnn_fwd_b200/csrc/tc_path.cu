@@ -57,18 +57,6 @@ bool tc::map3_bf16(CUtensorMap *m, const void *base, uint64_t d0, uint64_t d1, u
   return map3(m, base, d0, d1, d2, b0, b1);
 }
 
-bool tc::map_states(CUtensorMap *m, const void *base, uint64_t V, uint64_t K, uint64_t rows) {
-  auto fn = encode_fn();
-  if (!fn) return false;
-  cuuint64_t dims[4] = {8, V, K / 8, rows};
-  cuuint64_t strides[3] = {16, V * 16, V * K * 2};
-  cuuint32_t box[4] = {8, 64, 16, 1};
-  cuuint32_t es[4] = {1, 1, 1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box, es,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 namespace {
 
 // 1 if the current device is sm_100 (per device: 1 = yes, 2 = no).

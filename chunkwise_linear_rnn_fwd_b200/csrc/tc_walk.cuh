@@ -18,7 +18,7 @@
 // the state (and drain the output accumulator), warp 8 issues the TMA loads into
 // two rings (the key-side tiles kg / qg; the value-side tile with the intra-chunk
 // scores and the chunk's decay row), warp 9 issues the MMAs, warp 10 forms the
-// segment's decay product.  Every wait is
+// segment's decay product from the staged decay rows.  Every wait is
 // bounded (the status word records a timeout; the kernel then skips the dependent
 // work and ends).
 #pragma once
@@ -55,15 +55,18 @@ struct WalkTSmem {
 };
 
 // Byte offset of the 16-byte chunk (value column vg, key channels 8 c8 .. 8 c8 + 7)
-// of a bf16 chunk state in the layout the backward reads:
-//   [BH*N][K/8][V][8]  (8 consecutive key channels of one value column per 16 bytes)
-// A warp of the walk (32 consecutive value columns) stores 512 contiguous bytes per
-// instruction, and the backward fetches a (64-column d_v tile, 128-channel half) as
-// one 4-D TMA box, [16 channel groups][64 v][8 c], the no-swizzle MN-major operand
-// layout (core matrices of 8 v x 8 c).
+// of a bf16 chunk state in the layout the backward reads: per chunk row, d_v tile
+// of 64 columns and half of 128 key channels a contiguous 16 KB block
+//   [BH*N][V/64][K/128][8 v-groups][16 c-groups][8 v][8 c],
+// i.e. 8 x 8 core matrices (8 value columns x 16 bytes of channels) laid out
+// channel-group-fastest.  It is the no-swizzle MN-major operand layout of the
+// backward's MMAs (core matrices adjacent along the channels, 2 KB apart along
+// the value columns), fetched with one bulk copy; a warp of the walk (32
+// consecutive value columns) stores four full 128-byte lines per instruction.
 template <int K>
 __device__ __forceinline__ size_t state_chunk_off(long bhn, int V, int vg, int c8) {
-  return (((size_t)bhn * (K / 8) + c8) * (size_t)V + vg) * 16;
+  const int tile = vg >> 6, v8 = (vg >> 3) & 7, vr = vg & 7, half = c8 >> 4, cg = c8 & 15;
+  return (((((size_t)bhn * (V / 64) + tile) * (K / 128) + half) * 8 + v8) * 16 + cg) * 128 + (size_t)(vr * 16);
 }
 
 template <int K>
@@ -82,7 +85,7 @@ __global__ void __launch_bounds__(kWalkThreads, 1)
   uint64_t *xfull = bars;             // [NX]
   uint64_t *xempty = xfull + NX;      // [NX]
   uint64_t *yfull = xempty + NX;      // [NY]
-  uint64_t *yempty = yfull + NY;      // [NY]  MMA commit + one arrival per state warp
+  uint64_t *yempty = yfull + NY;      // [NY]  MMA commit + one arrival per state warp + warp 10
   uint64_t *dsfull = yempty + NY;     // [2]
   uint64_t *dsempty = dsfull + 2;     // [2]   one arrival per state warp
   uint64_t *afull = dsempty + 2;      // [1]   one arrival per state warp
@@ -112,7 +115,7 @@ __global__ void __launch_bounds__(kWalkThreads, 1)
     }
     for (int i = 0; i < NY; ++i) {
       dev::mbar_init(&yfull[i], 1);
-      dev::mbar_init(&yempty[i], 1 + kStateWarps);
+      dev::mbar_init(&yempty[i], 2 + kStateWarps);
     }
     for (int i = 0; i < 2; ++i) {
       dev::mbar_init(&dsfull[i], 1);
@@ -183,14 +186,28 @@ __global__ void __launch_bounds__(kWalkThreads, 1)
         (void)dev::mbar_wait(&yfull[j % NY], (uint32_t)((j / NY) & 1), a.status);
     }
     } else if (warp == kStateWarps + 2) {
-    // the product of the segment's chunk decays, per key channel (tile 0 only)
-    if (a.gseg && vt == 0) {
-      for (int c = lane; c < K; c += 32) {
-        float gp = 1.f;
-        for (int i = 0; i < nloc; ++i) gp *= __ldg(a.gam + (bh * a.N + chunk_of(i)) * K + c);
-        a.gseg[(bh * P + seg) * K + c] = gp;
+      // the product of the segment's chunk decays per key channel (lane: channels
+      // lane + 32 j), from the decay rows the producer stages with each chunk
+      const bool want = a.gseg && vt == 0;
+      float gp[K / 32];
+#pragma unroll
+      for (int j = 0; j < K / 32; ++j) gp[j] = 1.f;
+      bool ok = true;
+      for (int i = 0; i < nloc; ++i) {
+        const int sy = i % NY;
+        if (ok) ok = dev::mbar_wait(&yfull[sy], (uint32_t)((i / NY) & 1), a.status);
+        if (want) {
+          const float *g = reinterpret_cast<const float *>(yslot(sy) + L::kYTile + L::kPTile);
+#pragma unroll
+          for (int j = 0; j < K / 32; ++j) gp[j] *= g[lane + 32 * j];
+        }
+        __syncwarp();
+        if (lane == 0) dev::mbar_arrive(&yempty[sy]);
       }
-    }
+      if (want && ok) {
+#pragma unroll
+        for (int j = 0; j < K / 32; ++j) a.gseg[(bh * P + seg) * K + lane + 32 * j] = gp[j];
+      }
     } else if (warp == kStateWarps + 1) {
     // ============================ MMA issuer ============================
     if (lane == 0) {
