@@ -315,19 +315,17 @@ struct WalkArgs {
   int T, N, V, L;  // L = chunks per segment
   int P;           // segments per sequence (the grid covers segments seg0 .. seg0 + gridDim.y - 1)
   int seg0;
-  int end_seg;     // -1: every segment writes end[BH][P][K][V]; s >= 0: only segment s writes end[BH][K][V]
+  int end_seg;     // -1: every segment writes end[BH][P][V][K]; s >= 0: only segment s writes end[BH][K][V]
   int reverse, do_out, state_mode;  // state_mode: 0 none, 1 bf16 chunk states, 2 fp32 chunk states
   int p_kmajor;                     // output intra term: 0 = P V (forward), 1 = P^T dO (reverse: dv)
   const float *gam;                 // [BH][N][K]
-  const float *start;               // [BH][P][K][V] fp32 start states or null
-  const float *delta;               // [BH][P][K][V] segment contributions from a zero state (or null):
-                                    // the start state is then composed in the kernel from h0 and the
-                                    // contributions of the segments before this one (after it, reverse)
+  const float *start;               // [BH][P][K][V] fp32 start states (materialised chunk states) or null
+  const float *start_v;             // [BH][P][V][K] fp32 start states of the segments after the first
+                                    // (before it, reverse) or null; the first starts from h0
   const float *h0;                  // initial state of the whole walk (h0, or dh_final in reverse) or null
-  float *end;                       // state after the segment or null: end_seg < 0: [BH][P][K][V]
-                                    // (the delta layout); else [BH][K][V] fp32
+  float *end;                       // state after the segment or null: end_seg < 0: [BH][P][V][K]
+                                    // (segment contributions); else [BH][K][V] fp32
   float *gseg;                      // [BH][P][K] product of gam over the segment (written by d_v tile 0) or null
-  const float *gseg_in;             // the same products, read when composing start states
   float *h32;                       // [BH][N][K][V] fp32 states (state_mode 2)
   bf16 *hb;                         // bf16 states (state_mode 1), layout of state_chunk_off (tc_walk.cuh)
   bf16 *out;                        // [BH][T][V]

@@ -273,21 +273,26 @@ __global__ void __launch_bounds__(kWalkThreads, 1)
     const long KV = (long)K * a.V;
     float S[KH];
 
-    // ---- start state: h0 (or a materialised state), then the contributions of
-    // the earlier segments (later ones in reverse): S <- diag(gseg_p) S + delta_p
+    // ---- start state: h0 for the first segment (the last, reverse), else the
+    // segment's start state [V][K] (row vg contiguous) or a materialised [K][V] state
     {
-      const float *src = nullptr;
-      if (a.start) src = a.start + (bh * P + seg) * KV;
-      else if (a.h0 && (a.delta != nullptr || seg == (a.reverse ? P - 1 : 0))) src = a.h0 + bh * KV;
+      const bool first = seg == (a.reverse ? P - 1 : 0);
+      if (a.start_v && !first) {
+        const float4 *src = reinterpret_cast<const float4 *>(a.start_v + ((bh * P + seg) * (long)a.V + vg) * K + c0);
 #pragma unroll
-      for (int j = 0; j < KH; ++j) S[j] = (src && vok) ? __ldg(src + (long)(c0 + j) * a.V + vg) : 0.f;
-      const int np = a.delta ? (a.reverse ? (P - 1 - seg) : seg) : 0;
-      for (int u = 0; u < np; ++u) {
-        const int p = a.reverse ? (P - 1 - u) : u;
-        const float *gp = a.gseg_in + (bh * P + p) * K + c0;
-        const float *dp = a.delta + (bh * P + p) * KV + vg;
+        for (int j4 = 0; j4 < KH / 4; ++j4) {
+          const float4 x = vok ? __ldg(src + j4) : make_float4(0.f, 0.f, 0.f, 0.f);
+          S[4 * j4] = x.x;
+          S[4 * j4 + 1] = x.y;
+          S[4 * j4 + 2] = x.z;
+          S[4 * j4 + 3] = x.w;
+        }
+      } else {
+        const float *src = nullptr;
+        if (a.start) src = a.start + (bh * P + seg) * KV;
+        else if (a.h0 && first) src = a.h0 + bh * KV;
 #pragma unroll
-        for (int j = 0; j < KH; ++j) S[j] = __ldg(gp + j) * S[j] + (vok ? __ldg(dp + (long)(c0 + j) * a.V) : 0.f);
+        for (int j = 0; j < KH; ++j) S[j] = (src && vok) ? __ldg(src + (long)(c0 + j) * a.V + vg) : 0.f;
       }
     }
 
@@ -384,9 +389,16 @@ __global__ void __launch_bounds__(kWalkThreads, 1)
     }
 
     // ---- state after the segment ----------------------------------------------
-    if (a.end && (a.end_seg < 0 || a.end_seg == seg) && vok && ok) {
-      // end_seg < 0: segment contribution [BH][P][K][V]; else [BH][K][V]
-      float *dst = (a.end_seg < 0 ? a.end + (bh * P + seg) * KV : a.end + bh * KV) + vg;
+    if (a.end && a.end_seg < 0 && vok && ok) {
+      // segment contribution, [BH][P][V][K]: this thread's row, 16 bytes at a time
+      float4 *dst = reinterpret_cast<float4 *>(a.end + ((bh * P + seg) * (long)a.V + vg) * K + c0);
+#pragma unroll
+      for (int j4 = 0; j4 < KH / 4; ++j4)
+        dst[j4] = make_float4(S[4 * j4], S[4 * j4 + 1], S[4 * j4 + 2], S[4 * j4 + 3]);
+    }
+    if (a.end && a.end_seg == seg && vok && ok) {
+      // the walk's final state, [BH][K][V] (a warp stores 128 contiguous bytes per channel)
+      float *dst = a.end + bh * KV + vg;
 #pragma unroll
       for (int j = 0; j < KH; ++j) dst[(long)(c0 + j) * a.V] = S[j];
     }
