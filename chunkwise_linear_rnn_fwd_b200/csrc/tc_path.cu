@@ -51,6 +51,19 @@ bool map3(CUtensorMap *m, const void *base, uint64_t d0, uint64_t d1, uint64_t d
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The same without swizzle (row-major staging tiles, e.g. the walk's output blocks).
+bool map3_plain(CUtensorMap *m, const void *base, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t b0, uint32_t b1) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {d0 * 2, d0 * d1 * 2};
+  cuuint32_t box[3] = {b0, b1, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace
 
 bool tc::map3_bf16(CUtensorMap *m, const void *base, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t b0, uint32_t b1) {
@@ -178,7 +191,7 @@ int launch_prep(const Problem &p, const bf16 *q, const bf16 *k, const float *la,
 }
 
 struct WalkMaps {
-  CUtensorMap X, Y, Q, P;
+  CUtensorMap X, Y, Q, P, O;  // O: the output [BH][T][V] in [32 t][32 v] boxes (output walks)
 };
 
 // P here is the number of segments this launch covers (a.seg0 .. a.seg0 + P - 1).
@@ -195,7 +208,7 @@ int launch_walk(const Problem &p, const tc::WalkArgs &a, const WalkMaps &m, int 
     return GLA_ERR_CUDA;
   GLA_LAUNCH(K_TC_WALK, st,
              if (launch_pdl(tc::k_walkT<K>, dim3(walk_tiles(p), P, p.BH), dim3(tc::kWalkThreads), smem, st, a, m.X,
-                            m.Y, m.Q, m.P) != cudaSuccess) return GLA_ERR_CUDA);
+                            m.Y, m.Q, m.P, m.O) != cudaSuccess) return GLA_ERR_CUDA);
   return GLA_OK;
 }
 
@@ -258,7 +271,8 @@ int tc_fwd(const Problem &p, const void *q, const void *k, const void *v, const 
   WalkMaps m;
   const uint64_t BH = (uint64_t)p.BH;
   bool okm = map3(&m.X, w.kg, p.K, p.Tp, BH, 64, 64) && map3(&m.Y, v, p.V, p.T, BH, 64, 64) &&
-             map3(&m.Q, w.qg, p.K, p.Tp, BH, 64, 64) && map3(&m.P, w.PT, 64, 64, BH * p.N, 64, 64);
+             map3(&m.Q, w.qg, p.K, p.Tp, BH, 64, 64) && map3(&m.P, w.PT, 64, 64, BH * p.N, 64, 64) &&
+             map3_plain(&m.O, o, p.V, p.T, BH, 32, 32);
   if (!okm) return GLA_ERR_CUDA;
 
   tc::WalkArgs a{};
@@ -345,7 +359,9 @@ int tc_bwd(const Problem &p, const void *q, const void *k, const void *v, const 
   // ---- chunk adjoints dh_n (bf16) and dv = kg_n dh_n + P_n^T dO_n ------------------
   WalkMaps mr;
   okm = okm && map3(&mr.X, w.qg, p.K, p.Tp, BH, 64, 64) && map3(&mr.Y, dout, p.V, p.T, BH, 64, 64) &&
-        map3(&mr.Q, w.kg, p.K, p.Tp, BH, 64, 64) && map3(&mr.P, w.PT, 64, 64, BH * p.N, 64, 64);
+        map3(&mr.Q, w.kg, p.K, p.Tp, BH, 64, 64) && map3(&mr.P, w.PT, 64, 64, BH * p.N, 64, 64) &&
+        map3_plain(&mr.O, dv, p.V, p.T, BH, 32, 32);
+  mf.O = mf.X;
   if (!okm) return GLA_ERR_CUDA;
 
   tc::WalkArgs a{};
@@ -432,6 +448,7 @@ int tc_fwd_state(const Problem &p, const void *q, const void *k, const void *v, 
   if (!(map3(&m.X, w.kg, p.K, p.Tp, BH, 64, 64) && map3(&m.Y, v, p.V, p.T, BH, 64, 64))) return GLA_ERR_CUDA;
   m.Q = m.X;
   m.P = m.X;
+  m.O = m.X;
   tc::WalkArgs a{};
   a.T = p.T;
   a.N = p.N;
@@ -471,6 +488,7 @@ int tc_bwd_state(const Problem &p, const void *q, const void *k, const float *la
   if (!(map3(&m.X, w.qg, p.K, p.Tp, BH, 64, 64) && map3(&m.Y, dout, p.V, p.T, BH, 64, 64))) return GLA_ERR_CUDA;
   m.Q = m.X;
   m.P = m.X;
+  m.O = m.X;
   tc::WalkArgs r{};
   r.T = p.T;
   r.N = p.N;

@@ -49,7 +49,8 @@ struct WalkTSmem {
   static constexpr int NX = (K == 256) ? 4 : 6;
   static constexpr int NY = 3;
   static constexpr int kY0 = NX * kXSlot;
-  static constexpr int kBar = kY0 + NY * kYSlot;
+  static constexpr int kOst = kY0 + NY * kYSlot;          // output staging, [8 warps][32 t][32 v] bf16
+  static constexpr int kBar = kOst + 8 * 32 * 32 * 2;
   static constexpr int kBytes = kBar + 512;
   static_assert(K * 4 <= 1024, "decay row fits its slot");
 };
@@ -72,7 +73,8 @@ __device__ __forceinline__ size_t state_chunk_off(long bhn, int V, int vg, int c
 template <int K>
 __global__ void __launch_bounds__(kWalkThreads, 1)
     k_walkT(WalkArgs a, const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmY,
-            const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmP) {
+            const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmP,
+            const __grid_constant__ CUtensorMap tmO) {
   using L = WalkTSmem<K>;
   constexpr int BV = kWalkBV;
   constexpr int KH = K / 2;  // key channels per state thread
@@ -131,6 +133,7 @@ __global__ void __launch_bounds__(kWalkThreads, 1)
     if (out) {
       dev::prefetch_tmap(&tmQ);
       dev::prefetch_tmap(&tmP);
+      dev::prefetch_tmap(&tmO);
     }
   }
   dev::pdl_launch_dependents();
@@ -297,63 +300,77 @@ __global__ void __launch_bounds__(kWalkThreads, 1)
     }
 
     bool ok = true;
-    // O_i^T (TMEM, lanes v, columns tokens) -> out[t][vg]; warp half hh takes tokens 32 hh ..
+    // O_i^T (TMEM, lanes v, columns tokens) -> out[t][v]: this warp's [32 t][32 v]
+    // block (tokens 32 hh .., columns 32 q4 ..) goes through a shared-memory tile to
+    // one TMA store (the store clips rows beyond T and columns beyond V)
+    uint8_t *ost = smem + L::kOst + warp * 2048;
     auto epilogue = [&](int i) {
       float o[32];
       dev::tmem_ld32(lane_base + colO(i & 1) + (uint32_t)(32 * hh), o);
       dev::tmem_wait_ld();
       dev::tc_fence_before();
       __syncwarp();
-      if (lane == 0) dev::mbar_arrive(&oempty[i & 1]);
-      const long t0 = (long)chunk_of(i) * kC + 32 * hh;
-      if (vok && ok) {
-        bf16 *dst = a.out + (bh * a.T + t0) * (long)a.V + vg;
+      if (lane == 0) {
+        dev::mbar_arrive(&oempty[i & 1]);
+        dev::tma_store_wait_read();  // this warp's previous store has read the tile
+      }
+      __syncwarp();
+      const uint32_t so = dev::smem_u32(ost) + (uint32_t)(lane * 2);
 #pragma unroll
-        for (int e = 0; e < 32; ++e)
-          if (t0 + e < a.T) dst[(long)e * a.V] = __float2bfloat16_rn(o[e]);
+      for (int e = 0; e < 32; ++e) {
+        const bf16 b = __float2bfloat16_rn(o[e]);
+        dev::st_shared_u16(so + (uint32_t)(e * 64), *reinterpret_cast<const uint16_t *>(&b));
+      }
+      dev::fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0 && ok) {
+        dev::tma_store_3d(&tmO, ost, v0 + 32 * q4, chunk_of(i) * kC + 32 * hh, (int)bh);
+        dev::tma_store_commit();
       }
     };
+    // bf16 chunk state of this thread's row -> the backward's layout (4 x 16 bytes per 32 channels)
+    uint8_t *hb = reinterpret_cast<uint8_t *>(a.hb);
+    auto store_hb = [&](int n, int jb, const uint32_t *w) {
+      const long bhn = bh * a.N + n;
+#pragma unroll
+      for (int x = 0; x < 4; ++x)
+        *reinterpret_cast<uint4 *>(hb + state_chunk_off<K>(bhn, a.V, vg, c0 / 8 + 4 * jb + x)) =
+            make_uint4(w[4 * x], w[4 * x + 1], w[4 * x + 2], w[4 * x + 3]);
+    };
+    const bool st_hb = a.state_mode == 1 && vok;
 
     for (int i = 0; i < nloc; ++i) {
       const int n = chunk_of(i);
-      // ---- publish S_{i-1}: TMEM A operand of O_i, bf16 chunk state, fp32 state ----
-      if (out || a.state_mode != 0) {
-        if (out && i >= 1) {
+      // ---- publish S_{i-1} as the A operand of O_i (the MMA warp waits on afull) ----
+      if (out) {
+        if (i >= 1) {
           if (ok) ok = dev::mbar_wait(&ofull[(i - 1) & 1], (uint32_t)(((i - 1) >> 1) & 1), a.status);
           dev::tc_fence_after();
         }
-        if (out || a.state_mode == 1) {
-          // 32 channels at a time: 16 packed bf16 pairs to the TMEM A operand and,
-          // for the backward, 4 x 16 bytes to the chunk-state layout
-          const bool st_hb = a.state_mode == 1 && ok && vok;
-          uint8_t *hb = reinterpret_cast<uint8_t *>(a.hb);
-          const long bhn = bh * a.N + n;
 #pragma unroll
-          for (int jb = 0; jb < KH / 32; ++jb) {
-            uint32_t w[16];
+        for (int jb = 0; jb < KH / 32; ++jb) {
+          uint32_t w[16];
 #pragma unroll
-            for (int e = 0; e < 16; ++e) w[e] = dev::pack_bf16(S[32 * jb + 2 * e], S[32 * jb + 2 * e + 1]);
-            if (out) dev::tmem_st16u(lane_base + colA + (uint32_t)(c0 / 2 + 16 * jb), w);
-            if (st_hb) {
-#pragma unroll
-              for (int x = 0; x < 4; ++x)
-                *reinterpret_cast<uint4 *>(hb + state_chunk_off<K>(bhn, a.V, vg, c0 / 8 + 4 * jb + x)) =
-                    make_uint4(w[4 * x], w[4 * x + 1], w[4 * x + 2], w[4 * x + 3]);
-            }
-          }
-          if (out) {
-            dev::tmem_wait_st();
-            dev::tc_fence_before();
-            __syncwarp();
-            if (lane == 0) dev::mbar_arrive(afull);
-          }
+          for (int e = 0; e < 16; ++e) w[e] = dev::pack_bf16(S[32 * jb + 2 * e], S[32 * jb + 2 * e + 1]);
+          dev::tmem_st16u(lane_base + colA + (uint32_t)(c0 / 2 + 16 * jb), w);
         }
-        if (a.state_mode == 2 && vok && ok) {
-          float *dst = a.h32 + (bh * a.N + n) * KV + vg;
+        dev::tmem_wait_st();
+        dev::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) dev::mbar_arrive(afull);
+      } else if (st_hb && ok) {
 #pragma unroll
-          for (int j = 0; j < KH; ++j) dst[(long)(c0 + j) * a.V] = S[j];
+        for (int jb = 0; jb < KH / 32; ++jb) {
+          uint32_t w[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) w[e] = dev::pack_bf16(S[32 * jb + 2 * e], S[32 * jb + 2 * e + 1]);
+          store_hb(n, jb, w);
         }
-        if (out && i >= 1) epilogue(i - 1);
+      }
+      if (a.state_mode == 2 && vok && ok) {
+        float *dst = a.h32 + (bh * a.N + n) * KV + vg;
+#pragma unroll
+        for (int j = 0; j < KH; ++j) dst[(long)(c0 + j) * a.V] = S[j];
       }
       // ---- S_i = gam_i (.) S_{i-1} + dS_i ----------------------------------------
       const int sy = i % NY, d = i % nds;
@@ -381,6 +398,18 @@ __global__ void __launch_bounds__(kWalkThreads, 1)
         dev::mbar_arrive(&dsempty[d]);
         dev::mbar_arrive(&yempty[sy]);
       }
+      // ---- off the chain: S_{i-1} (still the A operand in TMEM) to the backward's
+      // layout, then the previous chunk's output -------------------------------------
+      if (out && st_hb && ok) {
+#pragma unroll
+        for (int jb = 0; jb < KH / 32; ++jb) {
+          float wf[16];
+          dev::tmem_ld16(lane_base + colA + (uint32_t)(c0 / 2 + 16 * jb), wf);
+          dev::tmem_wait_ld();
+          store_hb(n, jb, reinterpret_cast<const uint32_t *>(wf));
+        }
+      }
+      if (out && i >= 1) epilogue(i - 1);
     }
     if (out && nloc > 0) {
       if (ok) ok = dev::mbar_wait(&ofull[(nloc - 1) & 1], (uint32_t)(((nloc - 1) >> 1) & 1), a.status);
@@ -404,6 +433,7 @@ __global__ void __launch_bounds__(kWalkThreads, 1)
     }
   }
 
+  if (warp < kStateWarps && lane == 0) dev::tma_store_wait_all();  // output stores complete
   dev::tc_fence_before();
   __syncthreads();
   if (warp == 0) dev::tmem_dealloc(tmem, kTmemCols);
