@@ -87,16 +87,27 @@ __global__ void __launch_bounds__(256) k_segment_starts(long BH, int K, int V, i
     const long o = (bh * K + 4 * c4) * (long)V + v;
     S = make_float4(__ldg(h0 + o), __ldg(h0 + o + V), __ldg(h0 + o + 2L * V), __ldg(h0 + o + 3L * V));
   }
-  for (int j = 0; j + 1 < P; ++j) {
-    const int p = reverse ? P - 1 - j : j;         // segment folded in
-    const int nxt = reverse ? p - 1 : p + 1;       // segment it starts
-    const float4 g = __ldg(reinterpret_cast<const float4 *>(gseg + (bh * P + p) * K) + c4);
-    const float4 d = __ldg(delta + ((bh * P + p) * V + v) * K4 + c4);
-    S.x = g.x * S.x + d.x;
-    S.y = g.y * S.y + d.y;
-    S.z = g.z * S.z + d.z;
-    S.w = g.w * S.w + d.w;
-    starts[((bh * P + nxt) * V + v) * K4 + c4] = S;
+  for (int j0 = 0; j0 + 1 < P; j0 += 4) {  // the loads of four segments in flight together
+    float4 g[4], d[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int j = j0 + u, p = reverse ? P - 1 - j : j;
+      if (j + 1 < P) {
+        g[u] = __ldg(reinterpret_cast<const float4 *>(gseg + (bh * P + p) * K) + c4);
+        d[u] = __ldg(delta + ((bh * P + p) * V + v) * K4 + c4);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int j = j0 + u, p = reverse ? P - 1 - j : j;  // segment folded in
+      if (j + 1 < P) {
+        S.x = g[u].x * S.x + d[u].x;
+        S.y = g[u].y * S.y + d[u].y;
+        S.z = g[u].z * S.z + d[u].z;
+        S.w = g[u].w * S.w + d[u].w;
+        starts[((bh * P + (reverse ? p - 1 : p + 1)) * V + v) * K4 + c4] = S;  // the segment it starts
+      }
+    }
   }
 }
 // Pieces s in [s_lo, s_hi), ascending (forward) or descending (reverse).

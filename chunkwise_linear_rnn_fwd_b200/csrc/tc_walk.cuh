@@ -378,18 +378,20 @@ __global__ void __launch_bounds__(kWalkThreads, 1)
       if (ok) ok = dev::mbar_wait(&dsfull[d], (uint32_t)((i / nds) & 1), a.status);
       dev::tc_fence_after();
       const float *g = reinterpret_cast<const float *>(yslot(sy) + L::kYTile + L::kPTile) + c0;
+      // 64 columns of dS per TMEM round trip (two loads, one wait)
 #pragma unroll
-      for (int j = 0; j < KH / 32; ++j) {
-        float dsv[32];
-        dev::tmem_ld32(lane_base + (uint32_t)(d * K + c0 + 32 * j), dsv);
+      for (int j = 0; j < KH / 64; ++j) {
+        float dsv[64];
+        dev::tmem_ld32(lane_base + (uint32_t)(d * K + c0 + 64 * j), dsv);
+        dev::tmem_ld32(lane_base + (uint32_t)(d * K + c0 + 64 * j + 32), dsv + 32);
         dev::tmem_wait_ld();
 #pragma unroll
-        for (int e4 = 0; e4 < 8; ++e4) {
-          const float4 g4 = *reinterpret_cast<const float4 *>(g + 32 * j + 4 * e4);
-          S[32 * j + 4 * e4 + 0] = g4.x * S[32 * j + 4 * e4 + 0] + dsv[4 * e4 + 0];
-          S[32 * j + 4 * e4 + 1] = g4.y * S[32 * j + 4 * e4 + 1] + dsv[4 * e4 + 1];
-          S[32 * j + 4 * e4 + 2] = g4.z * S[32 * j + 4 * e4 + 2] + dsv[4 * e4 + 2];
-          S[32 * j + 4 * e4 + 3] = g4.w * S[32 * j + 4 * e4 + 3] + dsv[4 * e4 + 3];
+        for (int e4 = 0; e4 < 16; ++e4) {
+          const float4 g4 = *reinterpret_cast<const float4 *>(g + 64 * j + 4 * e4);
+          S[64 * j + 4 * e4 + 0] = g4.x * S[64 * j + 4 * e4 + 0] + dsv[4 * e4 + 0];
+          S[64 * j + 4 * e4 + 1] = g4.y * S[64 * j + 4 * e4 + 1] + dsv[4 * e4 + 1];
+          S[64 * j + 4 * e4 + 2] = g4.z * S[64 * j + 4 * e4 + 2] + dsv[4 * e4 + 2];
+          S[64 * j + 4 * e4 + 3] = g4.w * S[64 * j + 4 * e4 + 3] + dsv[4 * e4 + 3];
         }
       }
       dev::tc_fence_before();
