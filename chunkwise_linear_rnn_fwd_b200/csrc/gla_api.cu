@@ -14,7 +14,7 @@ const char *kernel_name(int id) {
       "f32_prep",     "f32_states",   "f32_scores",      "f32_out",    "f32_dstates",   "f32_dscores",
       "f32_dqk",      "f32_dv",       "f32_dg_out",      "tc_prep",    "tc_walk",       "tc_bwd",
       "status_clear", "decode",       "epilogue_fwd",    "epilogue_bwd", "epilogue_reduce", "state_scan",
-      "fold_segments", "f32_dlog_beta"};
+      "fold_segments", "f32_dlog_beta", "segment_starts"};
   static_assert(sizeof(names) / sizeof(names[0]) == K_COUNT, "one name per KernelId");
   if (id < 0 || id >= K_COUNT) return "unknown";
   return names[id];

@@ -31,6 +31,7 @@ enum KernelId : int {
   K_STATE_SCAN,
   K_FOLD_SEGMENTS,
   K_F32_DLB,
+  K_SEG_STARTS,
   K_COUNT
 };
 
@@ -96,7 +97,9 @@ int fold_segments(long BH, int K, int V, int P, int reverse, const float *gseg, 
                   float *out, float *gamma, cudaStream_t st);
 int state_scan(long BH, int K, int V, int nseg, int seg, int reverse, const float *gammas, const float *deltas,
                const float *init, float *out, cudaStream_t st);
-
+// start states of a walk's segments from their contributions (tc path)
+int segment_starts(long BH, int K, int V, int P, int reverse, const float *gseg, const float *delta, const float *h0,
+                   float *starts, cudaStream_t st);
 int epilogue_fwd(const gla_desc *d, const void *o, const void *r, const float *w, const float *b, float eps,
                  void *y, cudaStream_t st);
 int epilogue_bwd(const gla_desc *d, const void *o, const void *r, const float *w, const float *b, float eps,

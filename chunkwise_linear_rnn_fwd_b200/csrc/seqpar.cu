@@ -13,6 +13,9 @@
 //                    zero-state pre-pass runs every segment of the piece in parallel
 //                    (contributions delta_p [BH][P][V][K], gate products gseg_p);
 //                    out = fold over p of S <- diag(gseg_p) S + delta_p
+//   k_segment_starts the start state of every segment of a walk from the same
+//                    contributions: S = h0; S <- diag(gseg_p) S + delta_p, stored after
+//                    each p as the start of the next segment ([BH][P][V][K])
 //                    from h0 (dh_final in reverse), gamma = prod_p gseg_p
 //   k_state_scan     out = fold over the selected pieces of S <- diag(gamma_s) S + D_s
 //                    (elementwise per (bh, c, v), HBM-bound: one read of every D_s)
@@ -65,6 +68,48 @@ __global__ void __launch_bounds__(256) k_fold_segments(long BH, int K, int V, in
   if (gamma && v == 0) *reinterpret_cast<float4 *>(gamma + bh * K + 4 * c4) = gp;
 }
 
+// Start states of the segments of one walk: thread (bh, v, c4) folds the
+// contributions in walk order (forward: 0 .. P-2; reverse: P-1 .. 1) from h0
+// ([BH][K][V] or zero) and stores the state after each as the next segment's
+// start, starts[bh][p][v][4 c4 ..] (the segment that begins from h0 is not written).
+__global__ void __launch_bounds__(256) k_segment_starts(long BH, int K, int V, int P, int reverse,
+                                                        const float *__restrict__ gseg,
+                                                        const float4 *__restrict__ delta,
+                                                        const float *__restrict__ h0, float4 *__restrict__ starts) {
+  const int K4 = K / 4;
+  const long i = (long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= BH * V * K4) return;
+  const int c4 = (int)(i % K4);
+  const int v = (int)((i / K4) % V);
+  const long bh = i / ((long)K4 * V);
+  float4 S = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (h0) {
+    const long o = (bh * K + 4 * c4) * (long)V + v;
+    S = make_float4(__ldg(h0 + o), __ldg(h0 + o + V), __ldg(h0 + o + 2L * V), __ldg(h0 + o + 3L * V));
+  }
+  for (int j0 = 0; j0 + 1 < P; j0 += 4) {  // the loads of four segments in flight together
+    float4 g[4], d[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int j = j0 + u, p = reverse ? P - 1 - j : j;
+      if (j + 1 < P) {
+        g[u] = __ldg(reinterpret_cast<const float4 *>(gseg + (bh * P + p) * K) + c4);
+        d[u] = __ldg(delta + ((bh * P + p) * V + v) * K4 + c4);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int j = j0 + u, p = reverse ? P - 1 - j : j;  // segment folded in
+      if (j + 1 < P) {
+        S.x = g[u].x * S.x + d[u].x;
+        S.y = g[u].y * S.y + d[u].y;
+        S.z = g[u].z * S.z + d[u].z;
+        S.w = g[u].w * S.w + d[u].w;
+        starts[((bh * P + (reverse ? p - 1 : p + 1)) * V + v) * K4 + c4] = S;  // the segment it starts
+      }
+    }
+  }
+}
 // Pieces s in [s_lo, s_hi), ascending (forward) or descending (reverse).
 __global__ void __launch_bounds__(256) k_state_scan(long BH, int K, int V, int s_lo, int s_hi, int reverse,
                                                     const float *__restrict__ gammas,
@@ -104,6 +149,16 @@ int fold_segments(long BH, int K, int V, int P, int reverse, const float *gseg, 
   GLA_LAUNCH(K_FOLD_SEGMENTS, st,
              (k_fold_segments<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(BH, K, V, P, reverse, gseg,
                                                                           (const float4 *)delta, h0, out, gamma)));
+  return GLA_OK;
+}
+
+int segment_starts(long BH, int K, int V, int P, int reverse, const float *gseg, const float *delta, const float *h0,
+                   float *starts, cudaStream_t st) {
+  const long n = BH * V * (K / 4);
+  GLA_LAUNCH(K_SEG_STARTS, st,
+             (k_segment_starts<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(BH, K, V, P, reverse, gseg,
+                                                                           (const float4 *)delta, h0,
+                                                                           (float4 *)starts)));
   return GLA_OK;
 }
 

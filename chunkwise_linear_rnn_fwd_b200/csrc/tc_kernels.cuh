@@ -320,14 +320,12 @@ struct WalkArgs {
   int p_kmajor;                     // output intra term: 0 = P V (forward), 1 = P^T dO (reverse: dv)
   const float *gam;                 // [BH][N][K]
   const float *start;               // [BH][P][K][V] fp32 start states (materialised chunk states) or null
-  const float *delta;               // [BH][P][V][K] segment contributions from a zero state (or null):
-                                    // the start state is then composed in the kernel from h0 and the
-                                    // contributions of the segments before this one (after it, reverse)
+  const float *start_v;             // [BH][P][V][K] fp32 start states of the segments after the first
+                                    // (before it, reverse) or null; the first starts from h0
   const float *h0;                  // initial state of the whole walk (h0, or dh_final in reverse) or null
   float *end;                       // state after the segment or null: end_seg < 0: [BH][P][V][K]
                                     // (segment contributions); else [BH][K][V] fp32
   float *gseg;                      // [BH][P][K] product of gam over the segment (written by d_v tile 0) or null
-  const float *gseg_in;             // the same products, read when composing start states
   float *h32;                       // [BH][N][K][V] fp32 states (state_mode 2)
   bf16 *hb;                         // bf16 states (state_mode 1), layout of state_chunk_off (tc_walk.cuh)
   bf16 *out;                        // [BH][T][V]

@@ -3,9 +3,9 @@
 // Forward (section 4.2 chunkwise form, section 3.3 Figure 1 variants):
 //   prep                      qg, kg, gam, P^T per chunk (parallel over chunks)
 //   FUSED, P segments:        walk(no output) over segments 0..P-2 from 0 -> delta_p,
-//                             walk(output) per segment, each CTA composing its start
-//                             state from h0 and the earlier delta_p; the last segment
-//                             writes h_final (P = 1: a single walk from h0)
+//                             the fold of h0 and the delta_p into every segment's
+//                             start state, walk(output) per segment from its start;
+//                             the last segment writes h_final (P = 1: one walk from h0)
 //   MATERIALIZED:             walk(fp32 chunk states) over whole sequences, then
 //                             walk(output, one chunk per CTA) from those states.
 // Backward: chunk states h_n (saved by the forward, or a forward walk), a reverse
@@ -117,6 +117,7 @@ struct TcWs {
   float *gam;
   float *delta;          // [BH][P][V][K] segment contributions from a zero state
   float *gseg;           // [BH][P][K] per-segment gate products
+  float *starts;         // [BH][P][V][K] segment start states (folded from h0 and the contributions)
   float *h32;            // materialised fp32 chunk states [BH][N][K][V]
   // backward
   bf16 *hb, *dhb;        // bf16 chunk states and adjoints, tc::state_chunk_off layout
@@ -151,12 +152,14 @@ TcWs carve(const Problem &p, void *ws, bool bwd) {
     } else if (P > 1) {
       w.delta = cv.take<float>((size_t)p.BH * P * p.K * p.V);
       w.gseg = cv.take<float>((size_t)p.BH * P * p.K);
+      w.starts = cv.take<float>((size_t)p.BH * P * p.K * p.V);
     }
   } else {
     const int P = bwd_segments(p, nvt);
     w.delta = cv.take<float>((size_t)p.BH * P * p.K * p.V);
     w.ddelta = cv.take<float>((size_t)p.BH * P * p.K * p.V);
     w.gseg = cv.take<float>((size_t)p.BH * P * p.K);
+    w.starts = cv.take<float>((size_t)p.BH * P * p.K * p.V);
     w.hb = cv.take<bf16>((size_t)p.BH * p.N * p.K * p.V);
     w.dhb = cv.take<bf16>((size_t)p.BH * p.N * p.K * p.V);
     if (p.variant == GLA_VARIANT_MATERIALIZED && (p.flags & GLA_FLAG_SAVE_STATES))
@@ -327,8 +330,8 @@ int tc_fwd(const Problem &p, const void *q, const void *k, const void *v, const 
     pre.gseg = w.gseg;
     TRY(launch_walk_any(p, pre, m, P - 1, st));
   }
-  a.delta = w.delta;
-  a.gseg_in = w.gseg;
+  TRY(segment_starts(p.BH, p.K, p.V, P, 0, w.gseg, w.delta, h0, w.starts, st));
+  a.start_v = w.starts;
   a.h0 = h0;
   return launch_walk_any(p, a, m, P, st);
 }
@@ -376,8 +379,8 @@ int tc_bwd(const Problem &p, const void *q, const void *k, const void *v, const 
       pre.end = w.delta;
       pre.gseg = w.gseg;
       TRY(launch_walk_any(p, pre, mf, P - 1, st));
-      a.delta = w.delta;
-      a.gseg_in = w.gseg;
+      TRY(segment_starts(p.BH, p.K, p.V, P, 0, w.gseg, w.delta, h0, w.starts, st));
+      a.start_v = w.starts;
     }
     a.h0 = h0;
     a.state_mode = 1;
@@ -405,8 +408,8 @@ int tc_bwd(const Problem &p, const void *q, const void *k, const void *v, const 
       pre.gseg = w.gseg;
       TRY(launch_walk_any(p, pre, mr, P - 1, st));
     }
-    r.delta = w.ddelta;
-    r.gseg_in = w.gseg;
+    TRY(segment_starts(p.BH, p.K, p.V, P, 1, w.gseg, w.ddelta, dhT, w.starts, st));
+    r.start_v = w.starts;
   }
   r.h0 = dhT;
   r.state_mode = 1;

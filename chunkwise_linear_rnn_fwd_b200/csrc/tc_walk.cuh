@@ -276,30 +276,26 @@ __global__ void __launch_bounds__(kWalkThreads, 1)
     const long KV = (long)K * a.V;
     float S[KH];
 
-    // ---- start state: h0 (the first segment: the last, reverse) or a materialised
-    // state, then, with segment contributions, the fold over the earlier segments
-    // (later, reverse): S <- diag(gseg_p) S + delta_p, delta_p [V][K] read as this
-    // thread's row, 16 bytes at a time
+    // ---- start state: h0 for the first segment (the last, reverse), else the
+    // segment's start state [V][K] (row vg contiguous) or a materialised [K][V] state
     {
-      const float *src = nullptr;
-      if (a.start) src = a.start + (bh * P + seg) * KV;
-      else if (a.h0 && (a.delta != nullptr || seg == (a.reverse ? P - 1 : 0))) src = a.h0 + bh * KV;
-#pragma unroll
-      for (int j = 0; j < KH; ++j) S[j] = (src && vok) ? __ldg(src + (long)(c0 + j) * a.V + vg) : 0.f;
-      const int np = a.delta ? (a.reverse ? (P - 1 - seg) : seg) : 0;
-      for (int u = 0; u < np; ++u) {
-        const int p = a.reverse ? (P - 1 - u) : u;
-        const float4 *gp = reinterpret_cast<const float4 *>(a.gseg_in + (bh * P + p) * K + c0);
-        const float4 *dp = reinterpret_cast<const float4 *>(a.delta + ((bh * P + p) * (long)a.V + vg) * K + c0);
+      const bool first = seg == (a.reverse ? P - 1 : 0);
+      if (a.start_v && !first) {
+        const float4 *src = reinterpret_cast<const float4 *>(a.start_v + ((bh * P + seg) * (long)a.V + vg) * K + c0);
 #pragma unroll
         for (int j4 = 0; j4 < KH / 4; ++j4) {
-          const float4 g4 = __ldg(gp + j4);
-          const float4 d4 = vok ? __ldg(dp + j4) : make_float4(0.f, 0.f, 0.f, 0.f);
-          S[4 * j4] = g4.x * S[4 * j4] + d4.x;
-          S[4 * j4 + 1] = g4.y * S[4 * j4 + 1] + d4.y;
-          S[4 * j4 + 2] = g4.z * S[4 * j4 + 2] + d4.z;
-          S[4 * j4 + 3] = g4.w * S[4 * j4 + 3] + d4.w;
+          const float4 x = vok ? __ldg(src + j4) : make_float4(0.f, 0.f, 0.f, 0.f);
+          S[4 * j4] = x.x;
+          S[4 * j4 + 1] = x.y;
+          S[4 * j4 + 2] = x.z;
+          S[4 * j4 + 3] = x.w;
         }
+      } else {
+        const float *src = nullptr;
+        if (a.start) src = a.start + (bh * P + seg) * KV;
+        else if (a.h0 && first) src = a.h0 + bh * KV;
+#pragma unroll
+        for (int j = 0; j < KH; ++j) S[j] = (src && vok) ? __ldg(src + (long)(c0 + j) * a.V + vg) : 0.f;
       }
     }
 
