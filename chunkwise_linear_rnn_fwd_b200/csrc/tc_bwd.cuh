@@ -163,6 +163,61 @@ __global__ void __launch_bounds__(kBwdKH, 2)
   float Racc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
   bool ok = true;
 
+  // per key channel: sub-chunk boundary values of the cumulative log-gate (their 64
+  // gate loads are issued here, so that they complete while phase 1 streams); the 16
+  // values inside sub-chunk j are rebuilt from log_alpha when needed
+  float z[5], Gam[4], E[4], Gafter[4];
+  const long qrow0 = bh * a.T + (long)n * kC;  // first token row of this chunk
+  const uint32_t sQt = dev::smem_u32(smem + L::kQt), sKt = dev::smem_u32(smem + L::kKt);
+  auto qk_at = [&](int t, float &qf, float &kf) {
+    uint16_t qb, kb;
+    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(qb) : "r"(sQt + dev::sw128_off(64, t, cl)));
+    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(kb) : "r"(sKt + dev::sw128_off(64, t, cl)));
+    qf = __bfloat162float(*reinterpret_cast<const bf16 *>(&qb));
+    kf = __bfloat162float(*reinterpret_cast<const bf16 *>(&kb));
+  };
+  // log_alpha of token t of this chunk (0 beyond T)
+  auto gate_at = [&](int t) -> float {
+    if ((long)n * kC + t >= a.T) return 0.f;
+    if (a.gate == GLA_GATE_VECTOR) return __ldg(a.la + (qrow0 + t) * K + c);
+    if (a.gate == GLA_GATE_SCALAR) return __ldg(a.la + qrow0 + t);
+    return 0.f;
+  };
+  // g[e] = log_alpha of token 16 j + e; Bc[e] = z_j + g[0] + ... + g[e] (cumulative log-gate)
+  auto load16 = [&](int j, float *g) {
+#pragma unroll
+    for (int e = 0; e < 16; ++e) g[e] = gate_at(16 * j + e);
+  };
+  auto cumsum16 = [&](const float *g, float zj, float *Bc) {
+    float acc = zj;
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      acc += g[e];
+      Bc[e] = acc;
+    }
+  };
+  const uint32_t lanebase = 32 * warp;
+  {
+    float g[kC];
+#pragma unroll
+    for (int t = 0; t < kC; ++t) g[t] = gate_at(t);
+    float acc = 0.f;
+    z[0] = 0.f;
+#pragma unroll
+    for (int t = 0; t < kC; ++t) {
+      acc += g[t];
+      if ((t & 15) == 15) z[(t >> 4) + 1] = acc;
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      Gam[j] = __expf(z[j + 1] - z[j]);
+      E[j] = __expf(z[j]);
+    }
+    Gafter[3] = 1.f;
+    Gafter[2] = Gam[3];
+    Gafter[1] = Gam[3] * Gam[2];
+    Gafter[0] = Gam[3] * Gam[2] * Gam[1];
+  }
   // ============================ phase 1 ============================
   for (int i = 0; i < nvt; ++i) {
     const int s = i & 1;
@@ -277,60 +332,6 @@ __global__ void __launch_bounds__(kBwdKH, 2)
     }
   }
 
-  // per key channel: sub-chunk boundary values of the cumulative log-gate; the 16
-  // values inside sub-chunk j are rebuilt from log_alpha when needed
-  float z[5], Gam[4], E[4], Gafter[4];
-  const long qrow0 = bh * a.T + (long)n * kC;  // first token row of this chunk
-  const uint32_t sQt = dev::smem_u32(smem + L::kQt), sKt = dev::smem_u32(smem + L::kKt);
-  auto qk_at = [&](int t, float &qf, float &kf) {
-    uint16_t qb, kb;
-    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(qb) : "r"(sQt + dev::sw128_off(64, t, cl)));
-    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(kb) : "r"(sKt + dev::sw128_off(64, t, cl)));
-    qf = __bfloat162float(*reinterpret_cast<const bf16 *>(&qb));
-    kf = __bfloat162float(*reinterpret_cast<const bf16 *>(&kb));
-  };
-  // log_alpha of token t of this chunk (0 beyond T)
-  auto gate_at = [&](int t) -> float {
-    if ((long)n * kC + t >= a.T) return 0.f;
-    if (a.gate == GLA_GATE_VECTOR) return __ldg(a.la + (qrow0 + t) * K + c);
-    if (a.gate == GLA_GATE_SCALAR) return __ldg(a.la + qrow0 + t);
-    return 0.f;
-  };
-  // g[e] = log_alpha of token 16 j + e; Bc[e] = z_j + g[0] + ... + g[e] (cumulative log-gate)
-  auto load16 = [&](int j, float *g) {
-#pragma unroll
-    for (int e = 0; e < 16; ++e) g[e] = gate_at(16 * j + e);
-  };
-  auto cumsum16 = [&](const float *g, float zj, float *Bc) {
-    float acc = zj;
-#pragma unroll
-    for (int e = 0; e < 16; ++e) {
-      acc += g[e];
-      Bc[e] = acc;
-    }
-  };
-  const uint32_t lanebase = 32 * warp;
-  {
-    float g[kC];
-#pragma unroll
-    for (int t = 0; t < kC; ++t) g[t] = gate_at(t);
-    float acc = 0.f;
-    z[0] = 0.f;
-#pragma unroll
-    for (int t = 0; t < kC; ++t) {
-      acc += g[t];
-      if ((t & 15) == 15) z[(t >> 4) + 1] = acc;
-    }
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      Gam[j] = __expf(z[j + 1] - z[j]);
-      E[j] = __expf(z[j]);
-    }
-    Gafter[3] = 1.f;
-    Gafter[2] = Gam[3];
-    Gafter[1] = Gam[3] * Gam[2];
-    Gafter[0] = Gam[3] * Gam[2] * Gam[1];
-  }
   if (!dev::mbar_wait(qk_bar, 0, a.status)) ok = false;
 
   // window construction + boundary term G_n = gam_n R + sum_t k_t dk_inter_t
