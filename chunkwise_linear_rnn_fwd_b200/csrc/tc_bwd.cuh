@@ -197,27 +197,10 @@ __global__ void __launch_bounds__(kBwdKH, 2)
     }
   };
   const uint32_t lanebase = 32 * warp;
-  {
-    float g[kC];
+  // the 64 gate loads are issued now and first used after phase 1
+  float gpre[kC];
 #pragma unroll
-    for (int t = 0; t < kC; ++t) g[t] = gate_at(t);
-    float acc = 0.f;
-    z[0] = 0.f;
-#pragma unroll
-    for (int t = 0; t < kC; ++t) {
-      acc += g[t];
-      if ((t & 15) == 15) z[(t >> 4) + 1] = acc;
-    }
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      Gam[j] = __expf(z[j + 1] - z[j]);
-      E[j] = __expf(z[j]);
-    }
-    Gafter[3] = 1.f;
-    Gafter[2] = Gam[3];
-    Gafter[1] = Gam[3] * Gam[2];
-    Gafter[0] = Gam[3] * Gam[2] * Gam[1];
-  }
+  for (int t = 0; t < kC; ++t) gpre[t] = gate_at(t);
   // ============================ phase 1 ============================
   for (int i = 0; i < nvt; ++i) {
     const int s = i & 1;
@@ -288,6 +271,25 @@ __global__ void __launch_bounds__(kBwdKH, 2)
   }
   __syncthreads();
   const float R = red2[cl];
+
+  {
+    float acc = 0.f;
+    z[0] = 0.f;
+#pragma unroll
+    for (int t = 0; t < kC; ++t) {
+      acc += gpre[t];
+      if ((t & 15) == 15) z[(t >> 4) + 1] = acc;
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      Gam[j] = __expf(z[j + 1] - z[j]);
+      E[j] = __expf(z[j]);
+    }
+    Gafter[3] = 1.f;
+    Gafter[2] = Gam[3];
+    Gafter[1] = Gam[3] * Gam[2];
+    Gafter[0] = Gam[3] * Gam[2] * Gam[1];
+  }
 
   // ============================ phase 2 ============================
   // q and k columns of this half into the space phase 1 no longer uses
