@@ -19,7 +19,7 @@
 //                    from h0 (dh_final in reverse), gamma = prod_p gseg_p
 //   k_state_scan     out = fold over the selected pieces of S <- diag(gamma_s) S + D_s
 //                    (elementwise per (bh, c, v), HBM-bound: one read of every D_s)
-#include "internal.h"
+#include "tc_common.cuh"
 
 namespace gla {
 namespace {
@@ -76,6 +76,10 @@ __global__ void __launch_bounds__(256) k_segment_starts(long BH, int K, int V, i
                                                         const float *__restrict__ gseg,
                                                         const float4 *__restrict__ delta,
                                                         const float *__restrict__ h0, float4 *__restrict__ starts) {
+  // launched with programmatic stream serialization: wait for the walk that wrote
+  // the contributions, let the next walk's CTAs be scheduled early
+  dev::pdl_launch_dependents();
+  dev::pdl_wait();
   const int K4 = K / 4;
   const long i = (long)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= BH * V * K4) return;
@@ -156,9 +160,9 @@ int segment_starts(long BH, int K, int V, int P, int reverse, const float *gseg,
                    float *starts, cudaStream_t st) {
   const long n = BH * V * (K / 4);
   GLA_LAUNCH(K_SEG_STARTS, st,
-             (k_segment_starts<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(BH, K, V, P, reverse, gseg,
-                                                                           (const float4 *)delta, h0,
-                                                                           (float4 *)starts)));
+             if (launch_pdl(k_segment_starts, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, st, BH, K, V, P,
+                            reverse, gseg, (const float4 *)delta, h0, (float4 *)starts) != cudaSuccess)
+                 return GLA_ERR_CUDA);
   return GLA_OK;
 }
 
