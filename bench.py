@@ -7,8 +7,12 @@ inputs resident in HBM.  Prints one JSON line (rank 0).
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
 For N > 1 launch with torchrun; every rank runs its own replica of the workload
-(weak scaling, no collective on the data path).  --impl reference times the
-float64 CPU oracle (the only reference implementation) on a bounded sample.
+(weak scaling, no collective on the data path), and the line also reports the
+same sequence split across the ranks (sequence_parallel.ranks).  --seqpar makes
+that split the headline (strong scaling: each rank runs its piece of one
+sequence, with one NCCL all-gather of the pieces' state summaries per direction).
+--impl reference times the float64 CPU oracle (the only reference
+implementation) on a bounded sample.
 """
 from __future__ import annotations
 
@@ -455,6 +459,184 @@ def measure_seqpar(args, w, dev, stream, seed=0, pieces=8):
             "allgather_bytes_per_rank_per_direction": (B * H * K * V + B * H * K) * 4}
 
 
+# --------------------------------------------------------- sequence parallelism across ranks
+def seqpar_bounds(T, world, chunk=64):
+    """Token range [cuts[r], cuts[r+1]) of rank r's piece of a T-token sequence:
+    consecutive pieces of whole chunks, as equal as the chunk count allows; the last
+    piece takes the ragged tail.  Every piece holds at least one chunk."""
+    n = -(-T // chunk)
+    if n < world:
+        raise ValueError(f"{T} tokens make {n} chunks of {chunk}: fewer than {world} pieces")
+    cuts = [min(T, (n * r // world) * chunk) for r in range(world)] + [T]
+    return cuts
+
+
+def seqpar_step(ops, piece, h0=None, dh_final=None, group=None):
+    """One training step of this rank's piece through seqpar's protocol: the forward
+    (one all-gather of the pieces' summaries) then the backward (one more).  piece =
+    (q, k, v, log_alpha, do) of this rank; h0 / dh_final are read on the first / the
+    last rank only.  Returns (o, dq, dk, dv, dlog_alpha, h_out, dh_in)."""
+    from chunkwise_linear_rnn_fwd_b200 import seqpar
+    q, k, v, la, do = piece
+    o, h_out, h_in = seqpar.sp_gla_fwd(q, k, v, la, h0, group=group, ops=ops)
+    dq, dk, dv, dla, dh_in = seqpar.sp_gla_bwd(q, k, v, la, do, h_in, dh_final, group=group, ops=ops)
+    return o, dq, dk, dv, dla, h_out, dh_in
+
+
+def gather_pieces(t, cuts, group=None):
+    """The whole sequence's [B, H, T, ...] tensor, on every rank, from each rank's piece
+    t (token dimension 2): one all-gather of the pieces zero-padded to the longest."""
+    import torch
+    import torch.distributed as dist
+    world = len(cuts) - 1
+    lens = [cuts[r + 1] - cuts[r] for r in range(world)]
+    pad = t.new_zeros(*t.shape[:2], max(lens), *t.shape[3:])
+    pad[:, :, :t.shape[2]] = t
+    parts = [torch.empty_like(pad) for _ in range(world)]
+    dist.all_gather(parts, pad, group=group)
+    return torch.cat([p[:, :, :n] for p, n in zip(parts, lens)], dim=2)
+
+
+def tensor_rel_err(a, b):
+    """max |a - b| / max |b| over the whole tensor (0 for two empty or zero tensors)."""
+    a, b = a.float(), b.float()
+    den = b.abs().max().item() if b.numel() else 0.0
+    num = (a - b).abs().max().item() if b.numel() else 0.0
+    return num / den if den > 0 else num
+
+
+def measure_seqpar_ranks(args, w, dev, stream, rank, world):
+    """The workload's one sequence split across the job's ranks (strong scaling): rank r
+    runs seqpar_step on its piece through seqpar.LibraryOps, with one NCCL all-gather
+    of the pieces' summaries per direction; every rank draws the same whole-sequence
+    inputs.  Returns the step's device time (max over ranks, events on the launch
+    stream), the all-gather's own time and bytes, the per-kernel durations of one
+    rank, the end-to-end time with this rank's piece in pinned host memory, and the
+    gathered pieces compared on rank 0 with the single-GPU gla_fwd / gla_bwd of the
+    whole sequence (the same library; its parity with the oracle is in tests/)."""
+    import torch
+    import torch.distributed as dist
+
+    import chunkwise_linear_rnn_fwd_b200 as pkg
+    from chunkwise_linear_rnn_fwd_b200 import seqpar
+    from chunkwise_linear_rnn_fwd_b200.synth import make_inputs
+
+    B, H, T, K, V, C = w["B"], w["H"], w["T"], w["K"], w["V"], w["C"]
+    cuts = seqpar_bounds(T, world, C)
+    lo, hi = cuts[rank], cuts[rank + 1]
+    x = make_inputs(B, H, T, K, V, dtype=torch.bfloat16, gate=w["gate"], seed=0, z_mean=w["z_mean"])
+    whole = [None if t is None else t.to(dev) for t in (x.q, x.k, x.v, x.log_alpha, x.do)]
+    piece = [None if t is None else t[:, :, lo:hi].contiguous() for t in whole]
+    ops = seqpar.LibraryOps(C, stream)
+    group = None
+
+    def step():
+        return seqpar_step(ops, piece, group=group)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    n = max(5, args.steps)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(n):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = reduce_max_ms(e0.elapsed_time(e1), world, dev) / n
+
+    # the exchange alone: one all-gather of (gamma, delta) as the protocol packs them
+    gam = torch.rand(B, H, K, device=dev)
+    dlt = torch.randn(B, H, K, V, device=dev)
+    ag_ms = 0.0
+    if world > 1:
+        for _ in range(3):
+            seqpar.gather_summaries(gam, dlt, group)
+        torch.cuda.synchronize()
+        dist.barrier()
+        e0.record(stream)
+        for _ in range(n):
+            seqpar.gather_summaries(gam, dlt, group)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ag_ms = reduce_max_ms(e0.elapsed_time(e1), world, dev) / n
+
+    # this rank's kernels, one event pair per launch (a second pass of the same steps)
+    pkg.timing_enable(True)
+    pkg.timing_collect()
+    for _ in range(n):
+        step()
+    torch.cuda.synchronize()
+    launches = pkg.timing_collect()
+    pkg.timing_enable(False)
+    per_kernel = {}
+    for name, t in launches:
+        d = per_kernel.setdefault(name, [0, 0.0])
+        d[0] += 1
+        d[1] += t / n
+
+    # end to end: this rank's piece from pinned host memory, its gradients and output back
+    outs = step()
+    host_in = [None if t is None else t.cpu().pin_memory() for t in piece]
+    host_out = [None if t is None else torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in outs[:5]]
+    h2d = sum(t.numel() * t.element_size() for t in host_in if t is not None)
+    d2h = sum(t.numel() * t.element_size() for t in host_out if t is not None)
+
+    def e2e_step():
+        for dst, src in zip(piece, host_in):
+            if dst is not None:
+                dst.copy_(src, non_blocking=True)
+        res = step()
+        for dst, src in zip(host_out, res[:5]):
+            if dst is not None:
+                dst.copy_(src, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0.record(stream)
+    for _ in range(n):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = reduce_max_ms(e0.elapsed_time(e1), world, dev) / n
+
+    # the gathered pieces against the whole sequence on one GPU (rank 0 compares;
+    # every rank takes part in the gathers)
+    outs = step()
+    gathered = [None if t is None else gather_pieces(t, cuts, group) for t in outs[:5]]
+    h_final = outs[5].contiguous()
+    if world > 1:
+        dist.broadcast(h_final, src=world - 1, group=group)
+    check = None
+    if rank == 0:
+        q, k, v, la, do = whole
+        o, hT = pkg.gla_fwd(q, k, v, la, None, chunk=C, stream=stream)
+        dq, dk, dv, dla, _ = pkg.gla_bwd(q, k, v, la, do, None, None, chunk=C, stream=stream, want_dh0=False)
+        torch.cuda.synchronize()
+        names = ("o", "dq", "dk", "dv", "dlog_alpha")
+        check = {nm: tensor_rel_err(g, r) for nm, g, r in zip(names, gathered, (o, dq, dk, dv, dla))
+                 if g is not None}
+        check["h_final"] = tensor_rel_err(h_final, hT)
+        check["measure"] = "max |pieces - whole| / max |whole| per tensor (tensor scale)"
+    if world > 1:
+        dist.barrier()
+    return {
+        "ms_per_step": ms, "tokens_per_step": B * T, "pieces": cuts, "piece_tokens": hi - lo,
+        "allgather_ms": ag_ms, "allgathers_per_step": 2 if world > 1 else 0,
+        "allgather_bytes_per_rank_per_direction": (B * H * K + B * H * K * V) * 4 if world > 1 else 0,
+        "kernels_ms_per_step": {k2: v2[1] for k2, v2 in per_kernel.items()},
+        "gpu_launches_per_step": sum(v2[0] for v2 in per_kernel.values()) / n,
+        "e2e_ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+        "vs_whole_sequence": check,
+    }
+
+
 def measure_general_gate(args, w, dev, stream, seed=0):
     """The general gate alpha_t^T beta_t (CUDA-core path, fp32 arithmetic) on the
     bench workload with log beta drawn like log alpha: forward + backward step time
@@ -752,6 +934,9 @@ def run_ours(args, w):
         decode = measure_decode(args, dev, stream, peaks, peak_src, seed=rank)
         epilogue = measure_epilogue(args, w, dev, stream, peaks, peak_src, seed=rank)
         seqpar = measure_seqpar(args, w, dev, stream, seed=rank)
+        if world > 1:
+            # the same job, one sequence split across its ranks (all ranks take part)
+            seqpar["ranks"] = measure_seqpar_ranks(args, w, dev, stream, rank, world)
         variants = measure_variants(args, w, dev, stream, seed=rank)
         sweep_args = argparse.Namespace(steps=5, warmup=2)
         sweep_T = [time_workload(c, sweep_args, dev, stream, peaks) for c in SWEEP_T]
@@ -781,6 +966,64 @@ def run_ours(args, w):
             "sweep_vs_T": None if sweep_T is None else {
                 "workloads": sweep_T, "steps": 5, "peak_source": peak_src,
                 "l2": "inputs larger than L2 (B*T = 32768 tokens, >= 1 GB per step)"},
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def run_seqpar(args, w):
+    """--seqpar: one JSON line for the workload's sequence split across the job's ranks
+    (strong scaling; value = the sequence's tokens per second of the slowest rank)."""
+    import torch
+    import torch.distributed as dist
+
+    import chunkwise_linear_rnn_fwd_b200 as pkg
+
+    rank, world, local = dist_env()
+    if world > 1:
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pkg.load()
+    stream = torch.cuda.current_stream()
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    r = measure_seqpar_ranks(args, w, dev, stream, rank, world)
+    clocks = sampler.stop()
+    peaks, peak_src = load_peaks()
+    ms = r["ms_per_step"]
+    B, H, T, K, V, C = w["B"], w["H"], w["T"], w["K"], w["V"], w["C"]
+    kms = r["kernels_ms_per_step"]
+    roofline = None
+    if kms:
+        dom = max(kms, key=kms.get)
+        wp = dict(w, T=r["piece_tokens"])
+        alg = kernel_alg_bytes(dom, wp)
+        if alg is not None:
+            achieved = alg / (kms[dom] / 1e3) / 1e9
+            peak = float(peaks["hbm_gbs"])
+            roofline = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peak, "unit": "GB/s",
+                        "frac": achieved / peak, "traffic": None, "peak_source": peak_src,
+                        "bytes_source": "algorithmic share of rank 0's piece (no workspace)",
+                        "ms_per_step": kms[dom]}
+    flops = counted_flops(B, H, T, K, V, C)
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": B * T / (ms / 1e3), "unit": "tokens/s", "n_gpus": world,
+            "steps": max(5, args.steps), "warmup": max(3, args.warmup), "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "strong", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": dict(bench_config(w, 1), parallelism=f"sequence x{world}",
+                           pieces=r["pieces"]),
+            "tflops": flops / (ms / 1e3) / 1e12, "roofline": roofline,
+            "gpu_launches": int(round(r["gpu_launches_per_step"] * max(5, args.steps))),
+            "e2e": {"value": B * T / (r["e2e_ms_per_step"] / 1e3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": r["h2d_bytes_per_step"] * world,
+                    "d2h_bytes_per_step": r["d2h_bytes_per_step"] * world},
+            "clocks": clocks, "cpu_baseline": None, "sequence_parallel_ranks": r,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -827,6 +1070,9 @@ def main():
     ap.add_argument("--heads", type=int, default=None, help="override H")
     ap.add_argument("--seqlen", type=int, default=None, help="override T")
     ap.add_argument("--sweep", action="store_true", help="time every workload configuration (one JSON line)")
+    ap.add_argument("--seqpar", action="store_true",
+                    help="split the workload's sequence across the job's ranks (sequence parallelism, one NCCL "
+                         "all-gather per direction; strong scaling) instead of running a replica per rank")
     ap.add_argument("--step-only", action="store_true",
                     help="time the fwd+bwd step alone (no decode, epilogue, sequence-parallel, variant, sweep, "
                          "general-gate or CPU measurements): the command line of the profiler captures")
@@ -846,6 +1092,8 @@ def main():
         return run_sweep(args)
     if args.epilogue_once:
         return run_epilogue_once(w)
+    if args.seqpar:
+        return run_seqpar(args, w)
     return run_ours(args, w)
 
 

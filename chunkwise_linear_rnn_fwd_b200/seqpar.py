@@ -99,7 +99,7 @@ class LibraryOps:
         return G.gla_state_scan(gammas, deltas, seg, reverse=reverse, stream=self.stream)
 
 
-def _gather_summaries(gamma: torch.Tensor, delta: torch.Tensor, group) -> tuple[torch.Tensor, torch.Tensor]:
+def gather_summaries(gamma: torch.Tensor, delta: torch.Tensor, group) -> tuple[torch.Tensor, torch.Tensor]:
     """One all-gather of the packed (gamma, delta) of every rank: [P, *gamma.shape],
     [P, *delta.shape], piece-major."""
     world = dist.get_world_size(group)
@@ -126,7 +126,7 @@ def sp_gla_fwd(q, k, v, log_alpha=None, h0: Optional[torch.Tensor] = None, *, gr
         o, h_out = ops.fwd(q, k, v, log_alpha, h0)
         return o, h_out, h0
     delta, gamma = ops.fwd_state(q, k, v, log_alpha, h0 if rank == 0 else None)
-    gammas, deltas = _gather_summaries(gamma, delta, group)
+    gammas, deltas = gather_summaries(gamma, delta, group)
     h_in = h0 if rank == 0 else ops.state_scan(gammas, deltas, rank, False)
     o, h_out = ops.fwd(q, k, v, log_alpha, h_in)
     return o, h_out, h_in
@@ -144,6 +144,6 @@ def sp_gla_bwd(q, k, v, log_alpha, do, h_in: Optional[torch.Tensor], dh_final: O
         return ops.bwd(q, k, v, log_alpha, do, h_in, dh_final)
     last = rank == world - 1
     ddelta, gamma = ops.bwd_state(q, k, log_alpha, do, dh_final if last else None)
-    gammas, ddeltas = _gather_summaries(gamma, ddelta, group)
+    gammas, ddeltas = gather_summaries(gamma, ddelta, group)
     dh_out = dh_final if last else ops.state_scan(gammas, ddeltas, rank, True)
     return ops.bwd(q, k, v, log_alpha, do, h_in, dh_out)
