@@ -392,6 +392,44 @@ def measure_epilogue(args, w, dev, stream, peaks, peak_src, seed=0):
                      "frac_of_hbm": gbs / float(peaks["hbm_gbs"]), "l2": "flushed before every call"}
     res["workload"] = f"layer epilogue, B={B} H={H} T={T} d_v={V}, bf16 (fwd: o, r -> y; bwd: o, r, dy -> do, dr, dw, db)"
     res["peak_source"] = peak_src
+    res["fused_forward"] = measure_fused_epilogue(args, w, dev, stream, r, wt, bs, res["fwd"]["ms"], seed=seed)
+    return res
+
+
+def measure_fused_epilogue(args, w, dev, stream, r, wt, bs, separate_ms, seed=0):
+    """The forward with the epilogue fused into its output store (gla_fwd_epilogue)
+    against the plain forward (gla_fwd) on the bench workload: the fused store's
+    extra device time beside the separate pass's."""
+    import torch
+
+    import chunkwise_linear_rnn_fwd_b200 as pkg
+    from chunkwise_linear_rnn_fwd_b200.synth import make_inputs
+
+    B, H, T, K, V, C = w["B"], w["H"], w["T"], w["K"], w["V"], w["C"]
+    x = make_inputs(B, H, T, K, V, dtype=torch.bfloat16, gate=w["gate"], seed=seed, z_mean=w["z_mean"])
+    q, k, v, la = (t.to(dev) for t in (x.q, x.k, x.v, x.log_alpha))
+    o, y = torch.empty_like(v), torch.empty_like(v)
+    ws = pkg.alloc_workspace(pkg.workspace_size(B, H, T, K, V, torch.bfloat16, w["gate"], C, False), dev)
+    n = max(10, args.steps)
+    plain = lambda: pkg.gla_fwd(q, k, v, la, None, chunk=C, o=o, want_final=False, workspace=ws, stream=stream)
+    fused = lambda: pkg.gla_fwd_epilogue(q, k, v, la, r, wt, bs, chunk=C, o=o, y=y, want_final=False, workspace=ws,
+                                         stream=stream)
+    res = {"plain_fwd_ms": _time_steps(plain, stream, n, max(3, args.warmup)),
+           "fused_fwd_ms": _time_steps(fused, stream, n, max(3, args.warmup))}
+    pkg.timing_enable(True)
+    pkg.timing_collect()
+    for _ in range(n):
+        fused()
+    torch.cuda.synchronize()
+    per = {}
+    for kname, kms in pkg.timing_collect():
+        per[kname] = per.get(kname, 0.0) + kms / n
+    pkg.timing_enable(False)
+    res["fused_kernels_ms"] = per
+    res["extra_ms"] = res["fused_fwd_ms"] - res["plain_fwd_ms"]
+    res["separate_pass_ms"] = separate_ms
+    res["workload"] = (f"gla_fwd vs gla_fwd_epilogue, B={B} H={H} T={T} d_k={K} d_v={V}, bf16, "
+                       f"{w['gate']} gates; o and y both written")
     return res
 
 
@@ -489,6 +527,8 @@ def gather_pieces(t, cuts, group=None):
     import torch
     import torch.distributed as dist
     world = len(cuts) - 1
+    if world == 1:
+        return t
     lens = [cuts[r + 1] - cuts[r] for r in range(world)]
     pad = t.new_zeros(*t.shape[:2], max(lens), *t.shape[3:])
     pad[:, :, :t.shape[2]] = t

@@ -6,10 +6,10 @@ sequence over the ranks of a torch.distributed group.
 """
 from .gla import (FLAG_REUSE_PREP, FLAG_REUSE_SEGMENTS, FLAG_SAVE_STATES, GLAError, alloc_workspace, build_info,
                   epilogue_workspace_size, general_workspace_size, gla_bwd, gla_bwd_general, gla_bwd_state, gla_decode_step, gla_epilogue_bwd,
-                  gla_epilogue_fwd, gla_fwd, gla_fwd_general, gla_fwd_noalloc, gla_fwd_state, gla_state_scan, load, poll_status, poll_status_noalloc,
+                  gla_epilogue_fwd, gla_fwd, gla_fwd_epilogue, gla_fwd_general, gla_fwd_noalloc, gla_fwd_state, gla_state_scan, load, poll_status, poll_status_noalloc,
                   selftest_timeout, timing_collect, timing_enable, workspace_size)
 
 __all__ = ["FLAG_REUSE_PREP", "FLAG_REUSE_SEGMENTS", "FLAG_SAVE_STATES", "GLAError", "alloc_workspace", "build_info",
            "epilogue_workspace_size", "general_workspace_size", "gla_bwd", "gla_bwd_general", "gla_bwd_state", "gla_decode_step", "gla_epilogue_bwd",
-           "gla_epilogue_fwd", "gla_fwd", "gla_fwd_general", "gla_fwd_noalloc", "gla_fwd_state", "gla_state_scan", "load",
+           "gla_epilogue_fwd", "gla_fwd", "gla_fwd_epilogue", "gla_fwd_general", "gla_fwd_noalloc", "gla_fwd_state", "gla_state_scan", "load",
            "poll_status", "poll_status_noalloc", "selftest_timeout", "timing_collect", "timing_enable", "workspace_size"]

@@ -549,8 +549,8 @@ size_t epilogue_workspace(const gla_desc *d) {
 }
 
 int epilogue_fwd(const gla_desc *d, const void *o, const void *r, const float *w, const float *b, float eps,
-                 void *y, cudaStream_t st) {
-  if (cudaMemsetAsync(d->workspace, 0, kStatusBytes, st) != cudaSuccess) return GLA_ERR_CUDA;
+                 void *y, cudaStream_t st, bool clear_status) {
+  if (clear_status && cudaMemsetAsync(d->workspace, 0, kStatusBytes, st) != cudaSuccess) return GLA_ERR_CUDA;
   switch ((d->dv + 255) / 256) {
     case 1: return epi_fwd_t<1>(d, o, r, w, b, eps, y, st);
     case 2: return epi_fwd_t<2>(d, o, r, w, b, eps, y, st);

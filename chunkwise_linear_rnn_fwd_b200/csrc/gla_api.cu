@@ -14,7 +14,7 @@ const char *kernel_name(int id) {
       "f32_prep",     "f32_states",   "f32_scores",      "f32_out",    "f32_dstates",   "f32_dscores",
       "f32_dqk",      "f32_dv",       "f32_dg_out",      "tc_prep",    "tc_walk",       "tc_bwd",
       "status_clear", "decode",       "epilogue_fwd",    "epilogue_bwd", "epilogue_reduce", "state_scan",
-      "fold_segments", "f32_dlog_beta", "segment_starts"};
+      "fold_segments", "f32_dlog_beta", "segment_starts", "tc_walk_epi"};
   static_assert(sizeof(names) / sizeof(names[0]) == K_COUNT, "one name per KernelId");
   if (id < 0 || id >= K_COUNT) return "unknown";
   return names[id];
@@ -439,6 +439,41 @@ int gla_epilogue_fwd(const gla_desc *desc, const void *o, const void *r, const f
   GLA_TRY(check_opt(b));
   GLA_TRY(check_epilogue_ws(desc, false));
   return gla::epilogue_fwd(desc, o, r, w, b, eps, y, (cudaStream_t)stream);
+}
+
+int gla_fwd_epilogue(const gla_desc *desc, const void *q, const void *k, const void *v, const float *log_alpha,
+                     const float *h0, const void *r, const float *w, const float *b, float eps, void *o, void *y,
+                     float *h_final, int chunk, void *stream) {
+  Problem p;
+  GLA_TRY(make_problem(desc, chunk, &p));
+  if (p.flags & GLA_FLAG_REUSE_SEGMENTS) return GLA_ERR_INVALID_ARG;
+  GLA_TRY(check_req(q));
+  GLA_TRY(check_req(k));
+  GLA_TRY(check_req(v));
+  GLA_TRY(check_req(o));
+  GLA_TRY(check_req(r));
+  GLA_TRY(check_req(y));
+  GLA_TRY(check_gate_ptr(p, log_alpha));
+  GLA_TRY(check_opt(h0));
+  GLA_TRY(check_opt(h_final));
+  GLA_TRY(check_opt(w));
+  GLA_TRY(check_opt(b));
+  GLA_TRY(check_eps(eps));
+  GLA_TRY(check_ws(desc, p, (p.flags & GLA_FLAG_SAVE_STATES) != 0));
+  const bool fused = tc_epilogue_fusable(p);
+  if (!fused) GLA_TRY(check_epilogue_desc(desc));
+  cudaStream_t st = (cudaStream_t)stream;
+  GLA_TRY(clear_status(desc, st));
+  if (fused) {
+    const TcEpilogue epi{r, w, b, eps, y};
+    return tc_fwd_epilogue(p, q, k, v, log_alpha, h0, o, h_final, epi, desc->workspace, st);
+  }
+  // two passes: the forward, then the epilogue over its bf16 / fp32 output (the
+  // second pass keeps the status word, so a device error of either stays reported)
+  const int rf = p.dtype == GLA_DTYPE_BF16 ? tc_fwd(p, q, k, v, log_alpha, h0, o, h_final, desc->workspace, st)
+                                           : f32_fwd(p, q, k, v, log_alpha, nullptr, h0, o, h_final, desc->workspace, st);
+  if (rf != GLA_OK) return rf;
+  return gla::epilogue_fwd(desc, o, r, w, b, eps, y, st, false);
 }
 
 int gla_epilogue_bwd(const gla_desc *desc, const void *o, const void *r, const float *w, const float *b, float eps,

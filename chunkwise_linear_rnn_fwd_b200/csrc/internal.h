@@ -32,6 +32,7 @@ enum KernelId : int {
   K_FOLD_SEGMENTS,
   K_F32_DLB,
   K_SEG_STARTS,
+  K_TC_WALK_EPI,
   K_COUNT
 };
 
@@ -100,8 +101,9 @@ int state_scan(long BH, int K, int V, int nseg, int seg, int reverse, const floa
 // start states of a walk's segments from their contributions (tc path)
 int segment_starts(long BH, int K, int V, int P, int reverse, const float *gseg, const float *delta, const float *h0,
                    float *starts, cudaStream_t st);
+// clear_status = false: keep the status word (a second pass after a forward in the same call)
 int epilogue_fwd(const gla_desc *d, const void *o, const void *r, const float *w, const float *b, float eps,
-                 void *y, cudaStream_t st);
+                 void *y, cudaStream_t st, bool clear_status = true);
 int epilogue_bwd(const gla_desc *d, const void *o, const void *r, const float *w, const float *b, float eps,
                  const void *dy, void *dout, void *dr, float *dw, float *db, cudaStream_t st);
 

@@ -330,6 +330,11 @@ struct WalkArgs {
   bf16 *hb;                         // bf16 states (state_mode 1), layout of state_chunk_off (tc_walk.cuh)
   bf16 *out;                        // [BH][T][V]
   unsigned *status;
+  // layer epilogue fused into the output store (k_walkT<K, true> only): per-head
+  // LayerNorm over d_v with weight / bias (null: ones / zeros) and epsilon, times
+  // the Swish gate of r (read through its tensor map); y through its own map
+  const float *ln_w, *ln_b;
+  float eps;
 };
 
 }  // namespace tc

@@ -192,24 +192,74 @@ int launch_prep(const Problem &p, const bf16 *q, const bf16 *k, const float *la,
 
 struct WalkMaps {
   CUtensorMap X, Y, Q, P, O;  // O: the output [BH][T][V] in [32 t][32 v] boxes (output walks)
+  CUtensorMap R, Yo;          // fused epilogue: gate r (as Y) and the epilogue output y (as O)
 };
+
+template <int K, bool EPI>
+int walk_smem_attr() {
+  constexpr int smem = tc::WalkTSmem<K, EPI>::kBytes + 1024;
+  static_assert(smem <= kMaxDynSmem, "walk shared memory");
+  static DeviceSlots attr;  // the attribute belongs to the current device
+  if (per_device(attr, [] {
+        const cudaError_t e =
+            cudaFuncSetAttribute(tc::k_walkT<K, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) note_cuda_error(e);
+        return e == cudaSuccess ? 1 : -1;
+      }) < 0)
+    return -1;
+  return smem;
+}
 
 // P here is the number of segments this launch covers (a.seg0 .. a.seg0 + P - 1).
 template <int K>
 int launch_walk(const Problem &p, const tc::WalkArgs &a, const WalkMaps &m, int P, cudaStream_t st) {
-  constexpr int smem = tc::WalkTSmem<K>::kBytes + 1024;
-  static_assert(smem <= kMaxDynSmem, "walk shared memory");
-  static DeviceSlots attr;  // the attribute belongs to the current device
-  if (per_device(attr, [] {
-        const cudaError_t e = cudaFuncSetAttribute(tc::k_walkT<K>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (e != cudaSuccess) note_cuda_error(e);
-        return e == cudaSuccess ? 1 : -1;
-      }) < 0)
-    return GLA_ERR_CUDA;
+  const int smem = walk_smem_attr<K, false>();
+  if (smem < 0) return GLA_ERR_CUDA;
   GLA_LAUNCH(K_TC_WALK, st,
-             if (launch_pdl(tc::k_walkT<K>, dim3(walk_tiles(p), P, p.BH), dim3(tc::kWalkThreads), smem, st, a, m.X,
-                            m.Y, m.Q, m.P, m.O) != cudaSuccess) return GLA_ERR_CUDA);
+             if (launch_pdl(tc::k_walkT<K, false>, dim3(walk_tiles(p), P, p.BH), dim3(tc::kWalkThreads), smem, st, a,
+                            m.X, m.Y, m.Q, m.P, m.O, m.O, m.O) != cudaSuccess) return GLA_ERR_CUDA);
   return GLA_OK;
+}
+
+// The output walk with the fused layer epilogue: clusters of the walk_tiles(p)
+// CTAs of one (segment, head), which exchange row statistics through DSMEM.
+template <int K>
+int launch_walk_epi(const Problem &p, const tc::WalkArgs &a, const WalkMaps &m, int P, cudaStream_t st) {
+  const int smem = walk_smem_attr<K, true>();
+  if (smem < 0) return GLA_ERR_CUDA;
+  GLA_LAUNCH(K_TC_WALK_EPI, st,
+             if (launch_pdl_cluster(tc::k_walkT<K, true>, dim3(walk_tiles(p), P, p.BH), dim3(tc::kWalkThreads), smem,
+                                    st, (unsigned)walk_tiles(p), a, m.X, m.Y, m.Q, m.P, m.O, m.R,
+                                    m.Yo) != cudaSuccess) return GLA_ERR_CUDA);
+  return GLA_OK;
+}
+
+// Clusters of `nvt` fused-epilogue walk CTAs that fit on the device at once (0 on error).
+template <int K>
+int epi_max_clusters(int nvt) {
+  static DeviceSlots slots[4];
+  if (nvt < 1 || nvt > 4) return 0;
+  return per_device(slots[nvt - 1], [nvt] {
+    const int smem = walk_smem_attr<K, true>();
+    if (smem < 0) return 0;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(nvt, 1, 1);
+    cfg.blockDim = dim3(tc::kWalkThreads);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = nvt;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, tc::k_walkT<K, true>, &cfg) != cudaSuccess) {
+      (void)cudaGetLastError();
+      return 0;
+    }
+    return n;
+  });
 }
 
 int launch_walk_any(const Problem &p, const tc::WalkArgs &a, const WalkMaps &m, int P, cudaStream_t st) {
@@ -259,8 +309,14 @@ int tc_check(const Problem &p) {
 
 size_t tc_workspace(const Problem &p, bool bwd) { return carve(p, nullptr, bwd).bytes; }
 
-int tc_fwd(const Problem &p, const void *q, const void *k, const void *v, const float *la, const float *h0, void *o,
-           float *hT, void *ws, cudaStream_t st) {
+bool tc_epilogue_fusable(const Problem &p) {
+  return tc_check(p) == GLA_OK && p.dtype == GLA_DTYPE_BF16 && p.V % tc::kWalkBV == 0 &&
+         p.V / tc::kWalkBV <= 4 && p.variant != GLA_VARIANT_MATERIALIZED && !(p.flags & GLA_FLAG_REUSE_SEGMENTS);
+}
+
+namespace {
+int tc_fwd_impl(const Problem &p, const void *q, const void *k, const void *v, const float *la, const float *h0,
+                void *o, float *hT, void *ws, cudaStream_t st, const TcEpilogue *epi) {
   if (device_ok() != 1) return GLA_ERR_NO_DEVICE;
   const bool save = (p.flags & GLA_FLAG_SAVE_STATES) != 0;
   TcWs w = carve(p, ws, save);
@@ -273,6 +329,8 @@ int tc_fwd(const Problem &p, const void *q, const void *k, const void *v, const 
   bool okm = map3(&m.X, w.kg, p.K, p.Tp, BH, 64, 64) && map3(&m.Y, v, p.V, p.T, BH, 64, 64) &&
              map3(&m.Q, w.qg, p.K, p.Tp, BH, 64, 64) && map3(&m.P, w.PT, 64, 64, BH * p.N, 64, 64) &&
              map3_plain(&m.O, o, p.V, p.T, BH, 32, 32);
+  if (epi)
+    okm = okm && map3(&m.R, epi->r, p.V, p.T, BH, 64, 64) && map3_plain(&m.Yo, epi->y, p.V, p.T, BH, 32, 32);
   if (!okm) return GLA_ERR_CUDA;
 
   tc::WalkArgs a{};
@@ -307,7 +365,23 @@ int tc_fwd(const Problem &p, const void *q, const void *k, const void *v, const 
     return launch_walk_any(p, b, m, p.N, st);
   }
 
-  const int P = save ? bwd_segments(p, nvt) : segments_of(p, nvt);
+  int P = save ? bwd_segments(p, nvt) : segments_of(p, nvt);
+  if (epi) {
+    // every cluster of the fused output walk resident at once: at most as many
+    // segments per head as the device holds clusters (fewer than the workspace has room for)
+    const int mc = p.K == 256 ? epi_max_clusters<256>(nvt) : epi_max_clusters<128>(nvt);
+    if (mc < 1) return GLA_ERR_CUDA;
+    if ((long)P * p.BH > mc) P = (int)std::max<long>(1, mc / p.BH);
+    const int Lp = (p.N + P - 1) / P;
+    P = (p.N + Lp - 1) / Lp;
+    a.ln_w = epi->w;
+    a.ln_b = epi->b;
+    a.eps = epi->eps;
+  }
+  auto out_walk = [&](const tc::WalkArgs &wa, int nseg) {
+    if (!epi) return launch_walk_any(p, wa, m, nseg, st);
+    return p.K == 256 ? launch_walk_epi<256>(p, wa, m, nseg, st) : launch_walk_epi<128>(p, wa, m, nseg, st);
+  };
   const int L = (p.N + P - 1) / P;
   a.L = L;
   a.P = P;
@@ -317,7 +391,7 @@ int tc_fwd(const Problem &p, const void *q, const void *k, const void *v, const 
   a.end_seg = P - 1;
   if (P == 1) {
     a.h0 = h0;
-    return launch_walk_any(p, a, m, 1, st);
+    return out_walk(a, 1);
   }
   // pre-pass: the contribution of segments 0 .. P-2 from a zero state (already in
   // the workspace after gla_fwd_state with GLA_FLAG_REUSE_SEGMENTS)
@@ -333,7 +407,19 @@ int tc_fwd(const Problem &p, const void *q, const void *k, const void *v, const 
   TRY(segment_starts(p.BH, p.K, p.V, P, 0, w.gseg, w.delta, h0, w.starts, st));
   a.start_v = w.starts;
   a.h0 = h0;
-  return launch_walk_any(p, a, m, P, st);
+  return out_walk(a, P);
+}
+}  // namespace
+
+int tc_fwd(const Problem &p, const void *q, const void *k, const void *v, const float *la, const float *h0, void *o,
+           float *hT, void *ws, cudaStream_t st) {
+  return tc_fwd_impl(p, q, k, v, la, h0, o, hT, ws, st, nullptr);
+}
+
+int tc_fwd_epilogue(const Problem &p, const void *q, const void *k, const void *v, const float *la, const float *h0,
+                    void *o, float *hT, const TcEpilogue &epi, void *ws, cudaStream_t st) {
+  if (!tc_epilogue_fusable(p)) return GLA_ERR_UNSUPPORTED_SHAPE;
+  return tc_fwd_impl(p, q, k, v, la, h0, o, hT, ws, st, &epi);
 }
 
 int tc_bwd(const Problem &p, const void *q, const void *k, const void *v, const float *la, const float *h0,

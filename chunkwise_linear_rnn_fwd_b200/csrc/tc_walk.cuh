@@ -40,20 +40,50 @@ constexpr int kWalkRegsRole = 56;
 static_assert(256 * kWalkRegsState + 128 * kWalkRegsRole <= kWalkThreads * kWalkRegsLaunch,
               "register budgets exceed the launch allocation");
 
-template <int K>
+// EPI: the output walk with the layer epilogue fused into its output store (one
+// ring slot fewer on each side, room for the gate tiles r and the row statistics).
+template <int K, bool EPI = false>
 struct WalkTSmem {
   static constexpr int kXSlot = 64 * K * 2;             // kg or qg chunk tile [64][K] bf16, SW128
   static constexpr int kYTile = 64 * kWalkBV * 2;       // V or dO tile [64][128] bf16, SW128
   static constexpr int kPTile = 64 * 64 * 2;            // P^T [64][64] bf16, SW128
   static constexpr int kYSlot = kYTile + kPTile + 1024;  // + the chunk's decay row gam [K] fp32
-  static constexpr int NX = (K == 256) ? 4 : 6;
-  static constexpr int NY = 3;
+  static constexpr int NX = EPI ? ((K == 256) ? 3 : 6) : ((K == 256) ? 4 : 6);
+  static constexpr int NY = EPI ? 2 : 3;
   static constexpr int kY0 = NX * kXSlot;
-  static constexpr int kOst = kY0 + NY * kYSlot;          // output staging, [8 warps][32 t][32 v] bf16
+  static constexpr int kR0 = kY0 + NY * kYSlot;           // EPI: gate tiles r [2][64 t][128 v] bf16, SW128
+  static constexpr int kRTile = 64 * kWalkBV * 2;
+  static constexpr int kXch = kR0 + (EPI ? 2 * kRTile : 0);  // EPI: row statistics [2][4 ranks][4 q4][64 t] float2
+  static constexpr int kXchBuf = 4 * 4 * 64 * 8;
+  static constexpr int kOst = kXch + (EPI ? 2 * kXchBuf : 0);  // output staging, [8 warps][32 t][32 v] bf16
   static constexpr int kBar = kOst + 8 * 32 * 32 * 2;
   static constexpr int kBytes = kBar + 512;
   static_assert(K * 4 <= 1024, "decay row fits its slot");
 };
+
+// In-register transpose-and-add across a warp: v[e] on every lane in, out on
+// lane l the sum over the warp's lanes of their v[l] (v is overwritten).  Five
+// exchange rounds; in each, a lane keeps the half of its entries its partner
+// drops and adds the partner's copy of them.
+__device__ __forceinline__ float warp_transpose_sum32(float (&v)[32], int lane) {
+#pragma unroll
+  for (int w = 16; w >= 1; w >>= 1) {
+    const bool up = (lane & w) != 0;
+#pragma unroll
+    for (int j = 0; j < w; ++j) {
+      const float send = up ? v[j] : v[j + w];
+      const float keep = up ? v[j + w] : v[j];
+      v[j] = keep + __shfl_xor_sync(0xffffffffu, send, w);
+    }
+  }
+  return v[0];
+}
+
+__device__ __forceinline__ float tanh_approx_f(float x) {
+  float y;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 
 // Byte offset of the 16-byte chunk (value column vg, key channels 8 c8 .. 8 c8 + 7)
 // of a bf16 chunk state in the layout the backward reads: per chunk row, d_v tile
@@ -70,12 +100,13 @@ __device__ __forceinline__ size_t state_chunk_off(long bhn, int V, int vg, int c
   return (((((size_t)bhn * (V / 64) + tile) * (K / 128) + half) * 8 + v8) * 16 + cg) * 128 + (size_t)(vr * 16);
 }
 
-template <int K>
+template <int K, bool EPI>
 __global__ void __launch_bounds__(kWalkThreads, 1)
     k_walkT(WalkArgs a, const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmY,
             const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmP,
-            const __grid_constant__ CUtensorMap tmO) {
-  using L = WalkTSmem<K>;
+            const __grid_constant__ CUtensorMap tmO, const __grid_constant__ CUtensorMap tmR,
+            const __grid_constant__ CUtensorMap tmYo) {
+  using L = WalkTSmem<K, EPI>;
   constexpr int BV = kWalkBV;
   constexpr int KH = K / 2;  // key channels per state thread
   constexpr int NX = L::NX, NY = L::NY;
@@ -94,7 +125,10 @@ __global__ void __launch_bounds__(kWalkThreads, 1)
   uint64_t *ofull = afull + 1;        // [2]
   uint64_t *oempty = ofull + 2;       // [2]   one arrival per state warp
   uint64_t *done = oempty + 2;        // [1]   the MMA thread's last commit
-  uint32_t *tslot = (uint32_t *)(done + 1);
+  uint64_t *rfull = done + 1;         // [2]   EPI: gate tile r of the chunk
+  uint64_t *rempty = rfull + 2;       // [2]   EPI: one arrival per state warp
+  uint64_t *xchf = rempty + 2;        // [2]   EPI: row statistics of every warp of every CTA of the cluster
+  uint32_t *tslot = (uint32_t *)(xchf + 2);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int vt = blockIdx.x, seg = blockIdx.y + a.seg0;
@@ -127,6 +161,13 @@ __global__ void __launch_bounds__(kWalkThreads, 1)
     }
     dev::mbar_init(afull, kStateWarps);
     dev::mbar_init(done, 1);
+    if (EPI) {
+      for (int i = 0; i < 2; ++i) {
+        dev::mbar_init(&rfull[i], 1);
+        dev::mbar_init(&rempty[i], kStateWarps);
+        dev::mbar_init(&xchf[i], kStateWarps * gridDim.x);  // the cluster spans grid x
+      }
+    }
     dev::fence_mbar_init();
     dev::prefetch_tmap(&tmX);
     dev::prefetch_tmap(&tmY);
@@ -135,6 +176,10 @@ __global__ void __launch_bounds__(kWalkThreads, 1)
       dev::prefetch_tmap(&tmP);
       dev::prefetch_tmap(&tmO);
     }
+    if (EPI) {
+      dev::prefetch_tmap(&tmR);
+      dev::prefetch_tmap(&tmYo);
+    }
   }
   dev::pdl_launch_dependents();
   dev::pdl_wait();
@@ -142,6 +187,9 @@ __global__ void __launch_bounds__(kWalkThreads, 1)
   dev::tc_fence_before();
   __syncthreads();
   dev::tc_fence_after();
+  // EPI: the other CTAs of the cluster write into this CTA's shared memory; its
+  // barriers are initialised before any of them may start
+  if (EPI) dev::cluster_sync();
   const uint32_t tmem = *tslot;
 
   auto chunk_of = [&](int i) { return a.reverse ? (n_end - 1 - i) : (n_begin + i); };
@@ -154,7 +202,7 @@ __global__ void __launch_bounds__(kWalkThreads, 1)
     // ============================ TMA producer ============================
     if (lane == 0) {
       bool ok = true;
-      int xi = 0, yi = 0;  // loads issued into each ring
+      int xi = 0, yi = 0, ri = 0;  // loads issued into each ring
       auto load_x = [&](const CUtensorMap *map, int n) {
         const int s = xi % NX;
         if (xi >= NX && ok) ok = dev::mbar_wait(&xempty[s], (uint32_t)(((xi / NX) - 1) & 1), a.status);
@@ -181,12 +229,26 @@ __global__ void __launch_bounds__(kWalkThreads, 1)
           dev::bulk_load(y + L::kYTile + L::kPTile, a.gam + (bh * a.N + n) * K, (uint32_t)(K * 4), &yfull[sy]);
         }
         if (out) load_x(&tmQ, n);
+        if (EPI && ok) {
+          // the gate tile r of the chunk, held until its output rows are written
+          const int sr = i & 1;
+          if (i >= 2) ok = dev::mbar_wait(&rempty[sr], (uint32_t)(((i >> 1) - 1) & 1), a.status);
+          if (ok) {
+            ++ri;
+            uint8_t *rs = smem + L::kR0 + sr * L::kRTile;
+            dev::mbar_arrive_expect_tx(&rfull[sr], (uint32_t)L::kRTile);
+#pragma unroll
+            for (int cb = 0; cb < BV / 64; ++cb)
+              dev::tma_load_3d(rs + cb * 8192, &tmR, v0 + cb * 64, n * kC, (int)bh, &rfull[sr]);
+          }
+        }
       }
       // every load issued has landed before the CTA may end (the consumers normally
       // waited for them already; after a timeout nobody else does)
       for (int j = max(0, xi - NX); j < xi; ++j) (void)dev::mbar_wait(&xfull[j % NX], (uint32_t)((j / NX) & 1), a.status);
       for (int j = max(0, yi - NY); j < yi; ++j)
         (void)dev::mbar_wait(&yfull[j % NY], (uint32_t)((j / NY) & 1), a.status);
+      for (int j = max(0, ri - 2); j < ri; ++j) (void)dev::mbar_wait(&rfull[j & 1], (uint32_t)((j >> 1) & 1), a.status);
     }
     } else if (warp == kStateWarps + 2) {
       // the product of the segment's chunk decays per key channel (lane: channels
@@ -328,6 +390,108 @@ __global__ void __launch_bounds__(kWalkThreads, 1)
         dev::tma_store_commit();
       }
     };
+    // ---- EPI: the layer epilogue on the output rows (LayerNorm over the d_v
+    // columns of a token, which the cluster's CTAs share out in 128-column tiles,
+    // times the Swish gate r sigmoid(r)) -------------------------------------------
+    const float ln_w = (EPI && a.ln_w && vok) ? __ldg(a.ln_w + vg) : 1.f;
+    const float ln_b = (EPI && a.ln_b && vok) ? __ldg(a.ln_b + vg) : 0.f;
+    const uint32_t my_rank = EPI ? dev::cluster_ctarank() : 0u;
+    const int ncta = EPI ? (int)gridDim.x : 1;
+    // (A) chunk i's output block of this warp (tokens 32 hh .., columns 32 q4 ..):
+    // the bf16 output through the staging tile, and per token the mean and the sum
+    // of squared deviations over the warp's 32 columns, sent to every CTA of the
+    // cluster (slot [rank][q4][token] of the chunk's exchange buffer)
+    auto epi_a = [&](int i) {
+      float x[32];
+      const uint32_t tO = lane_base + colO(i & 1) + (uint32_t)(32 * hh);
+      dev::tmem_ld32(tO, x);
+      dev::tmem_wait_ld();
+      if (lane == 0) dev::tma_store_wait_read();
+      __syncwarp();
+      const uint32_t so = dev::smem_u32(ost) + (uint32_t)(lane * 2);
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        const bf16 b = __float2bfloat16_rn(x[e]);
+        dev::st_shared_u16(so + (uint32_t)(e * 64), *reinterpret_cast<const uint16_t *>(&b));
+      }
+      dev::fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0 && ok) {
+        dev::tma_store_3d(&tmO, ost, v0 + 32 * q4, chunk_of(i) * kC + 32 * hh, (int)bh);
+        dev::tma_store_commit();
+      }
+      const float mean = warp_transpose_sum32(x, lane) * (1.f / 32.f);  // of token 32 hh + lane
+      dev::tmem_ld32(tO, x);
+      dev::tmem_wait_ld();
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        const float d = x[e] - __shfl_sync(0xffffffffu, mean, e);
+        x[e] = d * d;
+      }
+      const float m2 = warp_transpose_sum32(x, lane);
+      const uint32_t slot = dev::smem_u32(smem + L::kXch + (i & 1) * L::kXchBuf) +
+                            (uint32_t)((((int)my_rank * 4 + q4) * 64 + 32 * hh + lane) * 8);
+      if (ok)
+        for (int r = 0; r < ncta; ++r) dev::st_cluster_f2(dev::mapa(slot, (uint32_t)r), mean, m2);
+      dev::fence_acq_rel_cluster();
+      __syncwarp();
+      if (lane < ncta && ok) dev::mbar_arrive_remote(dev::mapa(dev::smem_u32(&xchf[i & 1]), (uint32_t)lane));
+    };
+    // (B) once every warp of the cluster has sent chunk i's statistics: the token's
+    // mean and 1/sqrt(variance + eps) from the 4 ncta partials of 32 columns each
+    // (Chan's pairwise combination of means and squared deviations), then
+    // y = (w (o - mean) rstd + b) r sigmoid(r) through the staging tile
+    auto epi_b = [&](int i) {
+      if (ok) ok = dev::mbar_wait_cluster(&xchf[i & 1], (uint32_t)((i >> 1) & 1), a.status);
+      const float2 *xb = reinterpret_cast<const float2 *>(smem + L::kXch + (i & 1) * L::kXchBuf) + 32 * hh + lane;
+      const int np = 4 * ncta;
+      float mu = 0.f;
+      for (int p = 0; p < np; ++p) mu += xb[p * 64].x;
+      mu *= 1.f / (float)np;
+      float m2 = 0.f;
+      for (int p = 0; p < np; ++p) {
+        const float2 pr = xb[p * 64];
+        const float d = pr.x - mu;
+        m2 += fmaf(32.f * d, d, pr.y);
+      }
+      const float rstd = rsqrtf(m2 / (32.f * (float)np) + a.eps);
+      float x[32];
+      dev::tmem_ld32(lane_base + colO(i & 1) + (uint32_t)(32 * hh), x);
+      dev::tmem_wait_ld();
+      dev::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) dev::mbar_arrive(&oempty[i & 1]);
+      if (ok) ok = dev::mbar_wait(&rfull[i & 1], (uint32_t)((i >> 1) & 1), a.status);
+      const uint32_t rs = dev::smem_u32(smem + L::kR0 + (i & 1) * L::kRTile);
+      const int vl = 32 * q4 + lane;  // column within the 128-column tile
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        uint16_t rb;
+        asm volatile("ld.shared.u16 %0, [%1];" : "=h"(rb) : "r"(rs + dev::sw128_off(64, 32 * hh + e, vl)));
+        const float hr = 0.5f * __bfloat162float(*reinterpret_cast<const bf16 *>(&rb));
+        const float g = fmaf(hr, tanh_approx_f(hr), hr);  // r sigmoid(r) = h + h tanh(h), h = r / 2
+        const float m_e = __shfl_sync(0xffffffffu, mu, e), s_e = __shfl_sync(0xffffffffu, rstd, e);
+        x[e] = fmaf(ln_w * (x[e] - m_e), s_e, ln_b) * g;
+      }
+      __syncwarp();
+      if (lane == 0) {
+        dev::mbar_arrive(&rempty[i & 1]);
+        dev::tma_store_wait_read();  // the output block's store has read the staging tile
+      }
+      __syncwarp();
+      const uint32_t so = dev::smem_u32(ost) + (uint32_t)(lane * 2);
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        const bf16 b = __float2bfloat16_rn(x[e]);
+        dev::st_shared_u16(so + (uint32_t)(e * 64), *reinterpret_cast<const uint16_t *>(&b));
+      }
+      dev::fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0 && ok) {
+        dev::tma_store_3d(&tmYo, ost, v0 + 32 * q4, chunk_of(i) * kC + 32 * hh, (int)bh);
+        dev::tma_store_commit();
+      }
+    };
     // bf16 chunk state of this thread's row -> the backward's layout (4 x 16 bytes per 32 channels)
     uint8_t *hb = reinterpret_cast<uint8_t *>(a.hb);
     auto store_hb = [&](int n, int jb, const uint32_t *w) {
@@ -402,21 +566,31 @@ __global__ void __launch_bounds__(kWalkThreads, 1)
       }
       // ---- off the chain: S_{i-1} (still the A operand in TMEM) to the backward's
       // layout, then the previous chunk's output -------------------------------------
+      if (EPI && i >= 1) epi_a(i - 1);
       if (out && st_hb && ok) {
+        // the whole row in one TMEM round trip, then its 16-byte stores back to back
+        float wf[KH / 2];
 #pragma unroll
-        for (int jb = 0; jb < KH / 32; ++jb) {
-          float wf[16];
-          dev::tmem_ld16(lane_base + colA + (uint32_t)(c0 / 2 + 16 * jb), wf);
-          dev::tmem_wait_ld();
-          store_hb(n, jb, reinterpret_cast<const uint32_t *>(wf));
-        }
+        for (int jb = 0; jb < KH / 32; ++jb) dev::tmem_ld16(lane_base + colA + (uint32_t)(c0 / 2 + 16 * jb), wf + 16 * jb);
+        dev::tmem_wait_ld();
+#pragma unroll
+        for (int jb = 0; jb < KH / 32; ++jb) store_hb(n, jb, reinterpret_cast<const uint32_t *>(wf + 16 * jb));
       }
-      if (out && i >= 1) epilogue(i - 1);
+      if (EPI) {
+        if (i >= 1) epi_b(i - 1);
+      } else if (out && i >= 1) {
+        epilogue(i - 1);
+      }
     }
     if (out && nloc > 0) {
       if (ok) ok = dev::mbar_wait(&ofull[(nloc - 1) & 1], (uint32_t)(((nloc - 1) >> 1) & 1), a.status);
       dev::tc_fence_after();
-      epilogue(nloc - 1);
+      if (EPI) {
+        epi_a(nloc - 1);
+        epi_b(nloc - 1);
+      } else {
+        epilogue(nloc - 1);
+      }
     }
 
     // ---- state after the segment ----------------------------------------------
@@ -438,6 +612,8 @@ __global__ void __launch_bounds__(kWalkThreads, 1)
   if (warp < kStateWarps && lane == 0) dev::tma_store_wait_all();  // output stores complete
   dev::tc_fence_before();
   __syncthreads();
+  // EPI: no CTA leaves while another may still read its statistics or write its buffers
+  if (EPI) dev::cluster_sync();
   if (warp == 0) dev::tmem_dealloc(tmem, kTmemCols);
 }
 

@@ -33,7 +33,8 @@ EXPORTS = ["gla_workspace_size", "gla_check", "gla_fwd", "gla_bwd", "gla_poll_st
            "gla_timing_enable", "gla_timing_collect", "gla_kernel_name", "gla_build_info", "gla_fwd_noalloc",
            "gla_decode_step", "gla_selftest_timeout", "gla_epilogue_workspace_size", "gla_epilogue_fwd",
            "gla_epilogue_bwd", "gla_fwd_state", "gla_bwd_state", "gla_state_scan", "gla_general_workspace_size",
-           "gla_fwd_general", "gla_bwd_general", "gla_poll_status_noalloc", "gla_last_cuda_error"]
+           "gla_fwd_general", "gla_bwd_general", "gla_poll_status_noalloc", "gla_last_cuda_error",
+           "gla_fwd_epilogue"]
 
 
 class GLAError(RuntimeError):
@@ -84,6 +85,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.gla_epilogue_workspace_size.restype = ctypes.c_size_t
     lib.gla_epilogue_fwd.argtypes = [dp, vp, vp, vp, vp, f, vp, vp]
     lib.gla_epilogue_fwd.restype = i
+    lib.gla_fwd_epilogue.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp, f, vp, vp, vp, i, vp]
+    lib.gla_fwd_epilogue.restype = i
     lib.gla_epilogue_bwd.argtypes = [dp, vp, vp, vp, vp, f, vp, vp, vp, vp, vp, vp]
     lib.gla_epilogue_bwd.restype = i
     lib.gla_fwd_state.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, i, vp]
@@ -422,6 +425,37 @@ def gla_epilogue_fwd(o, r, w=None, b=None, *, eps=1e-5, y=None, workspace=None, 
     if r_ != GLA_OK:
         raise GLAError(r_, "gla_epilogue_fwd")
     return y
+
+
+@_on_stream
+def gla_fwd_epilogue(q, k, v, log_alpha, r, w=None, b=None, h0=None, *, eps=1e-5, chunk=64, gate=None, subchunk=16,
+                     variant="auto", segments=0, o=None, y=None, h_final=None, want_final=True, workspace=None,
+                     stream=None, save_states=False, reuse_prep=False):
+    """Forward with the layer epilogue fused into its output store.  Returns
+    (o, y, h_final or None): o and h_final as gla_fwd, y = LayerNorm(o; w, b, eps)
+    * Swish(r).  r [B,H,T,d_v] like v; w, b [d_v] fp32 or None.  See include/gla.h."""
+    lib = load()
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    gate = _gate_of(log_alpha, gate)
+    if o is None:
+        o = torch.empty(B, H, T, dv, dtype=q.dtype, device=q.device)
+    if y is None:
+        y = torch.empty(B, H, T, dv, dtype=q.dtype, device=q.device)
+    if h_final is None and want_final:
+        h_final = torch.empty(B, H, dk, dv, dtype=torch.float32, device=q.device)
+    flags = (FLAG_SAVE_STATES if save_states else 0) | (FLAG_REUSE_PREP if reuse_prep else 0)
+    if workspace is None:
+        workspace = alloc_workspace(workspace_size(B, H, T, dk, dv, q.dtype, gate, chunk, save_states,
+                                                   subchunk=subchunk, variant=variant, segments=segments,
+                                                   flags=flags), q.device)
+    d = make_desc(B, H, T, dk, dv, q.dtype, gate, subchunk=subchunk, variant=variant, segments=segments,
+                  flags=flags, workspace=workspace)
+    r_ = lib.gla_fwd_epilogue(ctypes.byref(d), _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(h0), _ptr(r), _ptr(w),
+                              _ptr(b), float(eps), _ptr(o), _ptr(y), _ptr(h_final), int(chunk), _stream_handle(stream))
+    if r_ != GLA_OK:
+        raise GLAError(r_, "gla_fwd_epilogue")
+    return o, y, h_final
 
 
 @_on_stream

@@ -99,6 +99,14 @@ class LibraryOps:
         return G.gla_state_scan(gammas, deltas, seg, reverse=reverse, stream=self.stream)
 
 
+def _rank_world(group) -> tuple[int, int]:
+    """(rank, world size) of `group`; without an initialised process group the
+    sequence is one piece on this process (0, 1)."""
+    if not (dist.is_available() and dist.is_initialized()):
+        return 0, 1
+    return dist.get_rank(group), dist.get_world_size(group)
+
+
 def gather_summaries(gamma: torch.Tensor, delta: torch.Tensor, group) -> tuple[torch.Tensor, torch.Tensor]:
     """One all-gather of the packed (gamma, delta) of every rank: [P, *gamma.shape],
     [P, *delta.shape], piece-major."""
@@ -121,7 +129,7 @@ def sp_gla_fwd(q, k, v, log_alpha=None, h0: Optional[torch.Tensor] = None, *, gr
     to sp_gla_bwd).  ops: the compute steps (a LibraryOps, kept for the backward of
     the same piece so that it reuses this call's work)."""
     ops = ops or LibraryOps(chunk, stream)
-    rank, world = dist.get_rank(group), dist.get_world_size(group)
+    rank, world = _rank_world(group)
     if world == 1:
         o, h_out = ops.fwd(q, k, v, log_alpha, h0)
         return o, h_out, h0
@@ -139,7 +147,7 @@ def sp_gla_bwd(q, k, v, log_alpha, do, h_in: Optional[torch.Tensor], dh_final: O
     (dq, dk, dv, dlog_alpha, dh_in): the piece's gradients and the adjoint of the
     state entering it (the sequence's dh0 on rank 0)."""
     ops = ops or LibraryOps(chunk, stream)
-    rank, world = dist.get_rank(group), dist.get_world_size(group)
+    rank, world = _rank_world(group)
     if world == 1:
         return ops.bwd(q, k, v, log_alpha, do, h_in, dh_final)
     last = rank == world - 1

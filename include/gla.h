@@ -209,6 +209,31 @@ int gla_epilogue_fwd(const gla_desc *desc, const void *o, const void *r, const f
 int gla_epilogue_bwd(const gla_desc *desc, const void *o, const void *r, const float *w, const float *b,
                      float eps, const void *dy, void *do_, void *dr, float *dw, float *db, void *stream);
 
+/* Forward with the layer epilogue fused into its output store ("Gated Linear
+ * Attention Transformers with Hardware-Efficient Training", the GLA layer of
+ * section 4.4: head-wise LayerNorm, then the Swish output gate).  Computes what
+ * gla_fwd followed by gla_epilogue_fwd computes: o and h_final exactly as
+ * gla_fwd, and y = (w (.) (o - mean(o)) / sqrt(var(o) + eps) + b) (.) r sigmoid(r)
+ * over the d_v channels of every (batch, head, token).
+ *   q, k, v, log_alpha, h0, o, h_final, chunk: as gla_fwd (o is still written:
+ *   the epilogue's backward reads it);  r, y [B,H,T,d_v] of desc->dtype;
+ *   w, b [d_v] fp32 or NULL (ones / zeros);  0 < eps < 1.
+ *   desc->workspace: as gla_fwd (gla_workspace_size(desc, chunk, 0), or the
+ *   backward size under GLA_FLAG_SAVE_STATES); GLA_FLAG_REUSE_PREP and
+ *   GLA_FLAG_SAVE_STATES as for gla_fwd; GLA_FLAG_REUSE_SEGMENTS is rejected
+ *   (GLA_ERR_INVALID_ARG: the fused walk may split the sequence into fewer segments).
+ * On the bf16 tensor-core path with d_v a multiple of 128 up to 512 and the fused
+ * variant, the statistics come from the fp32 output before its rounding to bf16:
+ * the output walk's CTAs of one head and segment form a thread-block cluster and
+ * exchange every token's per-tile mean and sum of squared deviations through
+ * distributed shared memory.  Any other valid descriptor runs gla_fwd and then the
+ * epilogue as a second pass over the bf16 o (d_v a multiple of 8, at most 1024).
+ * Returns GLA_OK or an error code; on error nothing was enqueued.  The status word
+ * (gla_poll_status) reports device-side errors as for gla_fwd. */
+int gla_fwd_epilogue(const gla_desc *desc, const void *q, const void *k, const void *v, const float *log_alpha,
+                     const float *h0, const void *r, const float *w, const float *b, float eps, void *o, void *y,
+                     float *h_final, int chunk, void *stream);
+
 /* ---- general gate (value-side gate beta) -------------------------------------------
  * "Gated Linear Attention Transformers with Hardware-Efficient Training",
  * appendix C: the gate G_t = alpha_t^T beta_t, an outer product of a key-side

@@ -269,3 +269,38 @@ def test_noalloc_rejects_reuse_flags(lib):
         d = desc(T=64, dk=128, dv=128, flags=flags)
         assert lib.gla_fwd_noalloc(ctypes.byref(d), a, a, a, a, None, a, None, 64, None) == -1
     assert lib.gla_fwd_noalloc(None, a, a, a, a, None, a, None, 64, None) == -1
+
+
+def test_fused_epilogue_validation_enqueues_nothing(lib):
+    """gla_fwd_epilogue checks the forward's and the epilogue's arguments before any
+    launch (every call below fails validation: none reaches a kernel)."""
+    vp = ctypes.c_void_p
+    a = vp(4096)
+    mis = vp(4096 + 4)
+    f = lib.gla_fwd_epilogue
+    d = desc(T=64, dk=128, dv=256)
+    d.workspace = 1 << 20
+    d.workspace_bytes = 1 << 40
+
+    def call(q=a, r=a, w=None, b=None, eps=1e-5, o=a, y=a, dd=d):
+        return f(ctypes.byref(dd), q, a, a, a, None, r, w, b, eps, o, y, None, 64, None)
+
+    assert call(q=None) == -1                      # q NULL
+    assert call(r=None) == -1                      # gate input r NULL
+    assert call(y=None) == -1                      # y NULL
+    assert call(y=mis) == -3                       # y misaligned
+    assert call(w=mis) == -3                       # LayerNorm weight misaligned
+    assert call(eps=0.0) == -1                     # eps must be positive
+    assert call(eps=1.5) == -1
+    d.flags = G.FLAG_REUSE_SEGMENTS
+    assert call() == -1                            # segment contributions are not reused
+    d.flags = 0
+    d.workspace_bytes = 16
+    assert call() == -4                            # workspace too small
+    d.workspace_bytes = 1 << 40
+    # shapes the fused walk does not take run two passes, so the epilogue's own
+    # limits apply: fp32 with d_v = 12 (not a multiple of 8)
+    e = desc(T=64, dk=64, dv=12, dtype=1)
+    e.workspace = 1 << 20
+    e.workspace_bytes = 1 << 40
+    assert call(dd=e) == -2

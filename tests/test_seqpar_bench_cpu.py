@@ -78,3 +78,18 @@ def test_bench_seqpar_step_matches_whole_sequence(oracle_mod, world, T, gate):
     np.testing.assert_allclose(out[world - 1]["h_out"], hT.numpy(), rtol=1e-10, atol=1e-10)
     np.testing.assert_allclose(out[0]["dh_in"], dh0.numpy(), rtol=1e-10, atol=1e-10)
     assert out[0]["cuts"][-1] == T and len(out[0]["cuts"]) == world + 1
+
+
+def test_bench_seqpar_step_without_process_group(oracle_mod):
+    """One process and no process group: the sequence is one piece and the step is
+    the plain forward and backward."""
+    import bench
+    q, k, v, la, do, h0, dhT = _inputs(100, "vector", seed=2)
+    ops = oracle_ops("vector")
+    o, dq, dk, dv, dla, h_out, dh_in = bench.seqpar_step(ops, (q, k, v, la, do), h0, dhT)
+    ro, rh = ops.fwd(q, k, v, la, h0)
+    rdq, rdk, rdv, rdla, rdh0 = ops.bwd(q, k, v, la, do, h0, dhT)
+    for a, b in ((o, ro), (h_out, rh), (dq, rdq), (dk, rdk), (dv, rdv), (dla, rdla), (dh_in, rdh0)):
+        np.testing.assert_allclose(a.numpy(), b.numpy(), rtol=0, atol=0)
+    cuts = bench.seqpar_bounds(100, 1, 16)
+    assert bench.gather_pieces(o, cuts) is o
