@@ -7,8 +7,11 @@
 //     y = (w (.) (o - mean) / sqrt(var + eps) + b) (.) r sigmoid(r)
 // with one weight w and bias b of size d_v shared by every head.  The walk that
 // produces o tiles d_v across CTAs, so the row statistics cannot be formed in its
-// output store; the epilogue is its own pass, bound by HBM bandwidth (read o and
-// r once, write y once; the backward reads o, r, dy and writes do, dr).
+// output store alone; this file is the epilogue as its own pass, bound by HBM
+// bandwidth (read o and r once, write y once; the backward reads o, r, dy and
+// writes do, dr).  gla_fwd_epilogue fuses the forward into the output walk where
+// the shape allows (its CTAs of one head form a cluster that exchanges the row
+// statistics); this pass serves the backward and the other shapes.
 //
 // Persistent grid (SMs x resident CTAs); every warp owns the rows
 // gw, gw + nw, gw + 2 nw, ... (gw its global warp index, nw the warp count) and a
@@ -55,48 +58,18 @@ __device__ __forceinline__ float warp_sum(float x) {
   return x;
 }
 
-// tanh, one-instruction approximation (relative error about 2^-11, below the
-// bf16 rounding of the epilogue's outputs)
-__device__ __forceinline__ float tanh_approx(float x) {
-  float y;
-  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
+// packed fp32 pairs and the one-instruction tanh (tc_common.cuh)
+using dev::add2;
+using dev::bf16pair;
+using dev::f2;
+using dev::fma2;
+using dev::hsum;
+using dev::mul2;
+using dev::pk;
+using dev::tanh_approx;
+using dev::upk;
 
-// ---- packed fp32 pairs (sm_100 f32x2 arithmetic: one instruction per two values)
-using f2 = uint64_t;
-__device__ __forceinline__ f2 pk(float lo, float hi) {
-  f2 r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-  return r;
-}
-__device__ __forceinline__ void upk(f2 v, float &lo, float &hi) {
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-}
-__device__ __forceinline__ f2 add2(f2 a, f2 b) {
-  f2 d;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
-__device__ __forceinline__ f2 mul2(f2 a, f2 b) {
-  f2 d;
-  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
-__device__ __forceinline__ f2 fma2(f2 a, f2 b, f2 c) {
-  f2 d;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-  return d;
-}
-__device__ __forceinline__ float hsum(f2 v) {
-  float lo, hi;
-  upk(v, lo, hi);
-  return lo + hi;
-}
 // 8 consecutive elements as 4 pairs: from shared memory (the staged row) ...
-__device__ __forceinline__ f2 bf16pair(uint32_t w) {  // element 2i in the low half
-  return pk(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
-}
 __device__ __forceinline__ void lds8p(const __nv_bfloat16 *p, f2 *x) {
   const uint4 u = *reinterpret_cast<const uint4 *>(p);
   x[0] = bf16pair(u.x);

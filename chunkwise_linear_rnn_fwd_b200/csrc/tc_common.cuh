@@ -370,6 +370,49 @@ __device__ __forceinline__ void st_shared_u16(uint32_t addr, uint16_t v) {
   asm volatile("st.shared.u16 [%0], %1;" ::"r"(addr), "h"(v) : "memory");
 }
 
+// ------------------------------------------------ packed fp32 pairs (sm_100 f32x2)
+// One add / mul / fma instruction per two values; a pair lives in one 64-bit register.
+using f2 = uint64_t;
+__device__ __forceinline__ f2 pk(float lo, float hi) {
+  f2 r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void upk(f2 v, float &lo, float &hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ f2 add2(f2 a, f2 b) {
+  f2 d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ f2 mul2(f2 a, f2 b) {
+  f2 d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ f2 fma2(f2 a, f2 b, f2 c) {
+  f2 d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ float hsum(f2 v) {
+  float lo, hi;
+  upk(v, lo, hi);
+  return lo + hi;
+}
+// two bf16 values packed in a 32-bit word (element 2i in the low half) as a pair
+__device__ __forceinline__ f2 bf16pair(uint32_t w) {
+  return pk(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
+// tanh, one-instruction approximation (relative error about 2^-11, below the bf16
+// rounding of the outputs it feeds)
+__device__ __forceinline__ float tanh_approx(float x) {
+  float y;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // ------------------------------------------------ thread-block clusters (DSMEM)
 __device__ __forceinline__ uint32_t cluster_ctarank() {
   uint32_t r;

@@ -64,6 +64,20 @@ bool map3_plain(CUtensorMap *m, const void *base, uint64_t d0, uint64_t d1, uint
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The same with the 64-byte swizzle (the fused epilogue's staging tiles: [32][32]
+// boxes, 64-byte rows).
+bool map3_sw64(CUtensorMap *m, const void *base, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t b0, uint32_t b1) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {d0 * 2, d0 * d1 * 2};
+  cuuint32_t box[3] = {b0, b1, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace
 
 bool tc::map3_bf16(CUtensorMap *m, const void *base, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t b0, uint32_t b1) {
@@ -329,8 +343,9 @@ int tc_fwd_impl(const Problem &p, const void *q, const void *k, const void *v, c
   bool okm = map3(&m.X, w.kg, p.K, p.Tp, BH, 64, 64) && map3(&m.Y, v, p.V, p.T, BH, 64, 64) &&
              map3(&m.Q, w.qg, p.K, p.Tp, BH, 64, 64) && map3(&m.P, w.PT, 64, 64, BH * p.N, 64, 64) &&
              map3_plain(&m.O, o, p.V, p.T, BH, 32, 32);
-  if (epi)
-    okm = okm && map3(&m.R, epi->r, p.V, p.T, BH, 64, 64) && map3_plain(&m.Yo, epi->y, p.V, p.T, BH, 32, 32);
+  if (epi)  // the fused epilogue stages o and y with the 64-byte swizzle
+    okm = okm && map3(&m.R, epi->r, p.V, p.T, BH, 64, 64) && map3_sw64(&m.O, o, p.V, p.T, BH, 32, 32) &&
+          map3_sw64(&m.Yo, epi->y, p.V, p.T, BH, 32, 32);
   if (!okm) return GLA_ERR_CUDA;
 
   tc::WalkArgs a{};

@@ -21,6 +21,17 @@
 // segment's decay product from the staged decay rows.  Every wait is
 // bounded (the status word records a timeout; the kernel then skips the dependent
 // work and ends).
+//
+// k_walkT<K, true> is the forward output walk with the GLA layer's epilogue fused
+// into its output store (section 4.4: per-head LayerNorm over d_v, then the Swish
+// output gate r sigmoid(r)).  The walk_tiles CTAs of one (segment, head) form a
+// thread-block cluster.  The state warps stage each chunk's bf16 output tile in
+// shared memory (two buffers) and hand it to warps 10 and 11, which store it,
+// take every token row's mean and squared deviations over the tile's 128 columns,
+// exchange them with the other CTAs of the cluster through distributed shared
+// memory, combine them over all d_v columns, and overwrite the tile with
+// y = (w (o - mean) / sqrt(var + eps) + b) r sigmoid(r) for its second store.  The
+// epilogue thus runs beside the state chain instead of on it.
 #pragma once
 
 #include "tc_kernels.cuh"
@@ -53,10 +64,12 @@ struct WalkTSmem {
   static constexpr int kY0 = NX * kXSlot;
   static constexpr int kR0 = kY0 + NY * kYSlot;           // EPI: gate tiles r [2][64 t][128 v] bf16, SW128
   static constexpr int kRTile = 64 * kWalkBV * 2;
-  static constexpr int kXch = kR0 + (EPI ? 2 * kRTile : 0);  // EPI: row statistics [2][4 ranks][4 q4][64 t] float2
-  static constexpr int kXchBuf = 4 * 4 * 64 * 8;
-  static constexpr int kOst = kXch + (EPI ? 2 * kXchBuf : 0);  // output staging, [8 warps][32 t][32 v] bf16
-  static constexpr int kBar = kOst + 8 * 32 * 32 * 2;
+  static constexpr int kXch = kR0 + (EPI ? 2 * kRTile : 0);  // EPI: row statistics [4][4 ranks][64 t] float2
+  static constexpr int kXchBuf = 4 * 64 * 8;
+  static constexpr int kWB = kXch + (EPI ? 4 * kXchBuf : 0);   // EPI: LayerNorm weight and bias of the tile [2][128] fp32
+  static constexpr int kOst = kWB + (EPI ? 1024 : 0);          // output staging, [8 warps][32 t][32 v] bf16
+  static constexpr int kOstBuf = 8 * 32 * 32 * 2;              // (EPI: two, SW64, handed to the epilogue warps)
+  static constexpr int kBar = kOst + (EPI ? 2 : 1) * kOstBuf;
   static constexpr int kBytes = kBar + 512;
   static_assert(K * 4 <= 1024, "decay row fits its slot");
 };
@@ -79,11 +92,7 @@ __device__ __forceinline__ float warp_transpose_sum32(float (&v)[32], int lane) 
   return v[0];
 }
 
-__device__ __forceinline__ float tanh_approx_f(float x) {
-  float y;
-  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
+
 
 // Byte offset of the 16-byte chunk (value column vg, key channels 8 c8 .. 8 c8 + 7)
 // of a bf16 chunk state in the layout the backward reads: per chunk row, d_v tile
@@ -125,10 +134,12 @@ __global__ void __launch_bounds__(kWalkThreads, 1)
   uint64_t *ofull = afull + 1;        // [2]
   uint64_t *oempty = ofull + 2;       // [2]   one arrival per state warp
   uint64_t *done = oempty + 2;        // [1]   the MMA thread's last commit
-  uint64_t *rfull = done + 1;         // [2]   EPI: gate tile r of the chunk
-  uint64_t *rempty = rfull + 2;       // [2]   EPI: one arrival per state warp
-  uint64_t *xchf = rempty + 2;        // [2]   EPI: row statistics of every warp of every CTA of the cluster
-  uint32_t *tslot = (uint32_t *)(xchf + 2);
+  uint64_t *rfull = done + 1;         // [2]   EPI: gate tile r of the chunk (one per epilogue warp)
+  uint64_t *rempty = rfull + 2;       // [2]   (unused)
+  uint64_t *xchf = rempty + 2;        // [4]   EPI: row statistics of a chunk from every CTA of the cluster
+  uint64_t *ostaged = xchf + 4;       // [2]   EPI: one arrival per state warp (the chunk's output tile is staged)
+  uint64_t *ofree = ostaged + 2;      // [2]   EPI: the epilogue warp is done with the staging tile
+  uint32_t *tslot = (uint32_t *)(ofree + 2);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int vt = blockIdx.x, seg = blockIdx.y + a.seg0;
@@ -151,7 +162,7 @@ __global__ void __launch_bounds__(kWalkThreads, 1)
     }
     for (int i = 0; i < NY; ++i) {
       dev::mbar_init(&yfull[i], 1);
-      dev::mbar_init(&yempty[i], 2 + kStateWarps);
+      dev::mbar_init(&yempty[i], 1 + kStateWarps + (EPI ? 0 : 1));  // MMA commit, state warps, warp 10
     }
     for (int i = 0; i < 2; ++i) {
       dev::mbar_init(&dsfull[i], 1);
@@ -164,8 +175,11 @@ __global__ void __launch_bounds__(kWalkThreads, 1)
     if (EPI) {
       for (int i = 0; i < 2; ++i) {
         dev::mbar_init(&rfull[i], 1);
-        dev::mbar_init(&rempty[i], kStateWarps);
-        dev::mbar_init(&xchf[i], kStateWarps * gridDim.x);  // the cluster spans grid x
+        dev::mbar_init(&ostaged[i], kStateWarps);
+        dev::mbar_init(&ofree[i], 1);
+      }
+      for (int i = 0; i < 4; ++i) dev::mbar_init(&xchf[i], gridDim.x);  // the cluster spans grid x
+      {
       }
     }
     dev::fence_mbar_init();
@@ -202,7 +216,7 @@ __global__ void __launch_bounds__(kWalkThreads, 1)
     // ============================ TMA producer ============================
     if (lane == 0) {
       bool ok = true;
-      int xi = 0, yi = 0, ri = 0;  // loads issued into each ring
+      int xi = 0, yi = 0;  // loads issued into each ring
       auto load_x = [&](const CUtensorMap *map, int n) {
         const int s = xi % NX;
         if (xi >= NX && ok) ok = dev::mbar_wait(&xempty[s], (uint32_t)(((xi / NX) - 1) & 1), a.status);
@@ -229,27 +243,202 @@ __global__ void __launch_bounds__(kWalkThreads, 1)
           dev::bulk_load(y + L::kYTile + L::kPTile, a.gam + (bh * a.N + n) * K, (uint32_t)(K * 4), &yfull[sy]);
         }
         if (out) load_x(&tmQ, n);
-        if (EPI && ok) {
-          // the gate tile r of the chunk, held until its output rows are written
-          const int sr = i & 1;
-          if (i >= 2) ok = dev::mbar_wait(&rempty[sr], (uint32_t)(((i >> 1) - 1) & 1), a.status);
-          if (ok) {
-            ++ri;
-            uint8_t *rs = smem + L::kR0 + sr * L::kRTile;
-            dev::mbar_arrive_expect_tx(&rfull[sr], (uint32_t)L::kRTile);
-#pragma unroll
-            for (int cb = 0; cb < BV / 64; ++cb)
-              dev::tma_load_3d(rs + cb * 8192, &tmR, v0 + cb * 64, n * kC, (int)bh, &rfull[sr]);
-          }
-        }
       }
       // every load issued has landed before the CTA may end (the consumers normally
       // waited for them already; after a timeout nobody else does)
       for (int j = max(0, xi - NX); j < xi; ++j) (void)dev::mbar_wait(&xfull[j % NX], (uint32_t)((j / NX) & 1), a.status);
       for (int j = max(0, yi - NY); j < yi; ++j)
         (void)dev::mbar_wait(&yfull[j % NY], (uint32_t)((j / NY) & 1), a.status);
-      for (int j = max(0, ri - 2); j < ri; ++j) (void)dev::mbar_wait(&rfull[j & 1], (uint32_t)((j >> 1) & 1), a.status);
     }
+    } else if (EPI && warp >= kStateWarps + 2) {
+      // ============================ epilogue warps (EPI) ============================
+      // Warp 10 + ew takes the chunks i with i % 2 == ew (staging buffer and gate
+      // buffer ew); lane l the token rows l and l + 32 of the chunk's 128-column
+      // output tile.  Per chunk: store the staged output, each row's mean and
+      // squared deviations over the tile to every CTA of the cluster, their
+      // combination over the d_v columns, y in place of o and its store.
+      const int ew = warp - (kStateWarps + 2);
+      float *sW = reinterpret_cast<float *>(smem + L::kWB);
+      float *sB = sW + BV;
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int c = 32 * ew + lane + 64 * u;
+        sW[c] = a.ln_w ? __ldg(a.ln_w + v0 + c) : 1.f;
+        sB[c] = a.ln_b ? __ldg(a.ln_b + v0 + c) : 0.f;
+      }
+      asm volatile("bar.sync 1, 64;" ::: "memory");  // both epilogue warps
+      const uint32_t my_rank = dev::cluster_ctarank();
+      const int ncta = (int)gridDim.x;
+      const float inv_n = 1.f / (float)(BV * ncta);
+      const dev::f2 half2 = dev::pk(0.5f, 0.5f);
+      bool ok = true;
+      uint8_t *stg = smem + L::kOst + ew * L::kOstBuf;
+      uint8_t *rt = smem + L::kR0 + ew * L::kRTile;
+      auto load_r = [&](int i) {
+        dev::mbar_arrive_expect_tx(&rfull[ew], (uint32_t)L::kRTile);
+#pragma unroll
+        for (int cb = 0; cb < BV / 64; ++cb)
+          dev::tma_load_3d(rt + cb * 8192, &tmR, v0 + cb * 64, chunk_of(i) * kC, (int)bh, &rfull[ew]);
+      };
+      if (lane == 0 && ew < nloc) load_r(ew);
+      int last_r = ew;  // the last chunk whose gate tile this warp loaded
+      // 16-byte unit j of block q of row 32 hr + lane (64-byte rows, 64-byte swizzle)
+      auto oaddr = [&](int hr, int q, int j) {
+        return dev::smem_u32(stg) + (uint32_t)((4 * hr + q) * 2048 + lane * 64 + ((j ^ ((lane >> 1) & 3)) << 4));
+      };
+      auto ld4p = [&](uint32_t addr, dev::f2 *x) {  // 8 bf16 as 4 pairs
+        uint4 u;
+        asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];" : "=r"(u.x), "=r"(u.y), "=r"(u.z), "=r"(u.w) : "r"(addr));
+        x[0] = dev::bf16pair(u.x);
+        x[1] = dev::bf16pair(u.y);
+        x[2] = dev::bf16pair(u.z);
+        x[3] = dev::bf16pair(u.w);
+      };
+      for (int i = ew; i < nloc; i += 2) {
+        const uint32_t par = (uint32_t)((i >> 1) & 1);
+        if (ok) ok = dev::mbar_wait(&ostaged[ew], par, a.status);
+        // the output tile: eight [32 t][32 v] blocks
+        if (lane == 0 && ok) {
+#pragma unroll
+          for (int hr = 0; hr < 2; ++hr)
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              dev::tma_store_3d(&tmO, stg + (4 * hr + q) * 2048, v0 + 32 * q, chunk_of(i) * kC + 32 * hr, (int)bh);
+          dev::tma_store_commit();
+        }
+        // row statistics in one pass, shifted by the row's first value: sums of
+        // d = o - s and d^2 over the tile's 128 columns (both rows side by side)
+        float mean[2], m2[2];
+        {
+          dev::f2 sh[2], sd[2], sq[2];
+#pragma unroll
+          for (int hr = 0; hr < 2; ++hr) {
+            dev::f2 x[4];
+            ld4p(oaddr(hr, 0, 0), x);
+            float lo, hi;
+            dev::upk(x[0], lo, hi);
+            sh[hr] = dev::pk(-lo, -lo);
+            sd[hr] = dev::pk(0.f, 0.f);
+            sq[hr] = dev::pk(0.f, 0.f);
+          }
+#pragma unroll 2
+          for (int c16 = 0; c16 < 16; ++c16) {
+#pragma unroll
+            for (int hr = 0; hr < 2; ++hr) {
+              dev::f2 x[4];
+              ld4p(oaddr(hr, c16 >> 2, c16 & 3), x);
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const dev::f2 d = dev::add2(x[e], sh[hr]);
+                sd[hr] = dev::add2(sd[hr], d);
+                sq[hr] = dev::fma2(d, d, sq[hr]);
+              }
+            }
+          }
+#pragma unroll
+          for (int hr = 0; hr < 2; ++hr) {
+            float s0, s1;
+            dev::upk(sh[hr], s0, s1);
+            const float sdv = dev::hsum(sd[hr]);
+            mean[hr] = sdv * (1.f / (float)BV) - s0;
+            m2[hr] = fmaxf(dev::hsum(sq[hr]) - sdv * sdv * (1.f / (float)BV), 0.f);
+          }
+        }
+        // to slots [rank][t] of buffer i % 4 of every CTA, then one arrival per CTA
+        const int xb4 = i & 3;
+        const uint32_t slot = dev::smem_u32(smem + L::kXch + xb4 * L::kXchBuf) + (uint32_t)(((int)my_rank * 64 + lane) * 8);
+        if (ok)
+          for (int r = 0; r < ncta; ++r) {
+            const uint32_t rs = dev::mapa(slot, (uint32_t)r);
+            dev::st_cluster_f2(rs, mean[0], m2[0]);
+            dev::st_cluster_f2(rs + 32 * 8, mean[1], m2[1]);
+          }
+        dev::fence_acq_rel_cluster();
+        __syncwarp();
+        if (lane < ncta && ok) dev::mbar_arrive_remote(dev::mapa(dev::smem_u32(&xchf[xb4]), (uint32_t)lane));
+        if (ok) ok = dev::mbar_wait_cluster(&xchf[xb4], (uint32_t)((i >> 2) & 1), a.status);
+        // Chan's combination of the ncta partials of BV columns each, per row
+        dev::f2 nmu2[2], rs2[2];
+#pragma unroll
+        for (int hr = 0; hr < 2; ++hr) {
+          const float2 *xb = reinterpret_cast<const float2 *>(smem + L::kXch + xb4 * L::kXchBuf) + 32 * hr + lane;
+          float mu = 0.f;
+          for (int r = 0; r < ncta; ++r) mu += xb[r * 64].x;
+          mu *= 1.f / (float)ncta;
+          float M2 = 0.f;
+          for (int r = 0; r < ncta; ++r) {
+            const float2 pr = xb[r * 64];
+            const float d = pr.x - mu;
+            M2 += fmaf((float)BV * d, d, pr.y);
+          }
+          const float rstd = rsqrtf(M2 * inv_n + a.eps);
+          nmu2[hr] = dev::pk(-mu, -mu);
+          rs2[hr] = dev::pk(rstd, rstd);
+        }
+        // y over o in the staging tile, once the output's stores have read it
+        if (lane == 0) dev::tma_store_wait_read();
+        __syncwarp();
+        if (ok) ok = dev::mbar_wait(&rfull[ew], par, a.status);
+#pragma unroll 1
+        for (int c16 = 0; c16 < 16; ++c16) {  // columns 8 c16 .. 8 c16 + 7 of the tile
+          dev::f2 w2[4], b2[4];
+          {
+            const ulonglong2 w01 = *reinterpret_cast<const ulonglong2 *>(sW + 8 * c16);
+            const ulonglong2 w23 = *reinterpret_cast<const ulonglong2 *>(sW + 8 * c16 + 4);
+            const ulonglong2 b01 = *reinterpret_cast<const ulonglong2 *>(sB + 8 * c16);
+            const ulonglong2 b23 = *reinterpret_cast<const ulonglong2 *>(sB + 8 * c16 + 4);
+            w2[0] = w01.x, w2[1] = w01.y, w2[2] = w23.x, w2[3] = w23.y;
+            b2[0] = b01.x, b2[1] = b01.y, b2[2] = b23.x, b2[3] = b23.y;
+          }
+#pragma unroll
+          for (int hr = 0; hr < 2; ++hr) {
+            const int t = 32 * hr + lane;
+            dev::f2 x[4], r[4];
+            const uint32_t oa = oaddr(hr, c16 >> 2, c16 & 3);
+            ld4p(oa, x);
+            ld4p(dev::smem_u32(rt) + (uint32_t)((c16 >> 3) * 8192 + t * 128 + (((c16 & 7) ^ (t & 7)) << 4)), r);
+            uint32_t pkd[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const dev::f2 nrm = dev::fma2(dev::mul2(dev::add2(x[e], nmu2[hr]), rs2[hr]), w2[e], b2[e]);
+              const dev::f2 h = dev::mul2(r[e], half2);
+              float hl, hh2;
+              dev::upk(h, hl, hh2);
+              const dev::f2 g = dev::fma2(h, dev::pk(dev::tanh_approx(hl), dev::tanh_approx(hh2)), h);  // r sigmoid(r)
+              float y0, y1;
+              dev::upk(dev::mul2(nrm, g), y0, y1);
+              pkd[e] = dev::pack_bf16(y0, y1);
+            }
+            asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(oa), "r"(pkd[0]), "r"(pkd[1]), "r"(pkd[2]),
+                         "r"(pkd[3])
+                         : "memory");
+          }
+        }
+        dev::fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          if (ok) {
+#pragma unroll
+            for (int hr = 0; hr < 2; ++hr)
+#pragma unroll
+              for (int q = 0; q < 4; ++q)
+                dev::tma_store_3d(&tmYo, stg + (4 * hr + q) * 2048, v0 + 32 * q, chunk_of(i) * kC + 32 * hr, (int)bh);
+            dev::tma_store_commit();
+          }
+          // the next gate tile of this warp (every lane has read this one)
+          if (i + 2 < nloc && ok) {
+            load_r(i + 2);
+            last_r = i + 2;
+          }
+          dev::tma_store_wait_read();  // the tile goes back to the state warps
+          dev::mbar_arrive(&ofree[ew]);
+        }
+      }
+      if (lane == 0) {
+        dev::tma_store_wait_all();
+        // the last gate tile load of this warp has landed before the CTA may end
+        if (last_r < nloc) (void)dev::mbar_wait(&rfull[ew], (uint32_t)((last_r >> 1) & 1), a.status);
+      }
     } else if (warp == kStateWarps + 2) {
       // the product of the segment's chunk decays per key channel (lane: channels
       // lane + 32 j), from the decay rows the producer stages with each chunk
@@ -372,6 +561,25 @@ __global__ void __launch_bounds__(kWalkThreads, 1)
       dev::tmem_wait_ld();
       dev::tc_fence_before();
       __syncwarp();
+      if (EPI) {
+        // the tile of chunk i - 2 went through the epilogue warps and its stores
+        if (lane == 0) dev::mbar_arrive(&oempty[i & 1]);
+        if (i >= 2 && ok) ok = dev::mbar_wait(&ofree[i & 1], (uint32_t)(((i >> 1) - 1) & 1), a.status);
+        // block (q4, hh) of the chunk's staging tile, 64-byte rows with the 64-byte
+        // swizzle (16-byte unit j of row e at unit j ^ ((e >> 1) & 3))
+        const uint32_t blk = dev::smem_u32(smem + L::kOst + (i & 1) * L::kOstBuf) + (uint32_t)(warp * 2048);
+        const uint32_t cb = (uint32_t)(lane * 2);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const bf16 b = __float2bfloat16_rn(o[e]);
+          const uint32_t off = (uint32_t)(e * 64) + ((((cb >> 4) ^ (uint32_t)((e >> 1) & 3))) << 4) + (cb & 15u);
+          dev::st_shared_u16(blk + off, *reinterpret_cast<const uint16_t *>(&b));
+        }
+        dev::fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) dev::mbar_arrive(&ostaged[i & 1]);
+        return;
+      }
       if (lane == 0) {
         dev::mbar_arrive(&oempty[i & 1]);
         dev::tma_store_wait_read();  // this warp's previous store has read the tile
@@ -387,108 +595,6 @@ __global__ void __launch_bounds__(kWalkThreads, 1)
       __syncwarp();
       if (lane == 0 && ok) {
         dev::tma_store_3d(&tmO, ost, v0 + 32 * q4, chunk_of(i) * kC + 32 * hh, (int)bh);
-        dev::tma_store_commit();
-      }
-    };
-    // ---- EPI: the layer epilogue on the output rows (LayerNorm over the d_v
-    // columns of a token, which the cluster's CTAs share out in 128-column tiles,
-    // times the Swish gate r sigmoid(r)) -------------------------------------------
-    const float ln_w = (EPI && a.ln_w && vok) ? __ldg(a.ln_w + vg) : 1.f;
-    const float ln_b = (EPI && a.ln_b && vok) ? __ldg(a.ln_b + vg) : 0.f;
-    const uint32_t my_rank = EPI ? dev::cluster_ctarank() : 0u;
-    const int ncta = EPI ? (int)gridDim.x : 1;
-    // (A) chunk i's output block of this warp (tokens 32 hh .., columns 32 q4 ..):
-    // the bf16 output through the staging tile, and per token the mean and the sum
-    // of squared deviations over the warp's 32 columns, sent to every CTA of the
-    // cluster (slot [rank][q4][token] of the chunk's exchange buffer)
-    auto epi_a = [&](int i) {
-      float x[32];
-      const uint32_t tO = lane_base + colO(i & 1) + (uint32_t)(32 * hh);
-      dev::tmem_ld32(tO, x);
-      dev::tmem_wait_ld();
-      if (lane == 0) dev::tma_store_wait_read();
-      __syncwarp();
-      const uint32_t so = dev::smem_u32(ost) + (uint32_t)(lane * 2);
-#pragma unroll
-      for (int e = 0; e < 32; ++e) {
-        const bf16 b = __float2bfloat16_rn(x[e]);
-        dev::st_shared_u16(so + (uint32_t)(e * 64), *reinterpret_cast<const uint16_t *>(&b));
-      }
-      dev::fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0 && ok) {
-        dev::tma_store_3d(&tmO, ost, v0 + 32 * q4, chunk_of(i) * kC + 32 * hh, (int)bh);
-        dev::tma_store_commit();
-      }
-      const float mean = warp_transpose_sum32(x, lane) * (1.f / 32.f);  // of token 32 hh + lane
-      dev::tmem_ld32(tO, x);
-      dev::tmem_wait_ld();
-#pragma unroll
-      for (int e = 0; e < 32; ++e) {
-        const float d = x[e] - __shfl_sync(0xffffffffu, mean, e);
-        x[e] = d * d;
-      }
-      const float m2 = warp_transpose_sum32(x, lane);
-      const uint32_t slot = dev::smem_u32(smem + L::kXch + (i & 1) * L::kXchBuf) +
-                            (uint32_t)((((int)my_rank * 4 + q4) * 64 + 32 * hh + lane) * 8);
-      if (ok)
-        for (int r = 0; r < ncta; ++r) dev::st_cluster_f2(dev::mapa(slot, (uint32_t)r), mean, m2);
-      dev::fence_acq_rel_cluster();
-      __syncwarp();
-      if (lane < ncta && ok) dev::mbar_arrive_remote(dev::mapa(dev::smem_u32(&xchf[i & 1]), (uint32_t)lane));
-    };
-    // (B) once every warp of the cluster has sent chunk i's statistics: the token's
-    // mean and 1/sqrt(variance + eps) from the 4 ncta partials of 32 columns each
-    // (Chan's pairwise combination of means and squared deviations), then
-    // y = (w (o - mean) rstd + b) r sigmoid(r) through the staging tile
-    auto epi_b = [&](int i) {
-      if (ok) ok = dev::mbar_wait_cluster(&xchf[i & 1], (uint32_t)((i >> 1) & 1), a.status);
-      const float2 *xb = reinterpret_cast<const float2 *>(smem + L::kXch + (i & 1) * L::kXchBuf) + 32 * hh + lane;
-      const int np = 4 * ncta;
-      float mu = 0.f;
-      for (int p = 0; p < np; ++p) mu += xb[p * 64].x;
-      mu *= 1.f / (float)np;
-      float m2 = 0.f;
-      for (int p = 0; p < np; ++p) {
-        const float2 pr = xb[p * 64];
-        const float d = pr.x - mu;
-        m2 += fmaf(32.f * d, d, pr.y);
-      }
-      const float rstd = rsqrtf(m2 / (32.f * (float)np) + a.eps);
-      float x[32];
-      dev::tmem_ld32(lane_base + colO(i & 1) + (uint32_t)(32 * hh), x);
-      dev::tmem_wait_ld();
-      dev::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) dev::mbar_arrive(&oempty[i & 1]);
-      if (ok) ok = dev::mbar_wait(&rfull[i & 1], (uint32_t)((i >> 1) & 1), a.status);
-      const uint32_t rs = dev::smem_u32(smem + L::kR0 + (i & 1) * L::kRTile);
-      const int vl = 32 * q4 + lane;  // column within the 128-column tile
-#pragma unroll
-      for (int e = 0; e < 32; ++e) {
-        uint16_t rb;
-        asm volatile("ld.shared.u16 %0, [%1];" : "=h"(rb) : "r"(rs + dev::sw128_off(64, 32 * hh + e, vl)));
-        const float hr = 0.5f * __bfloat162float(*reinterpret_cast<const bf16 *>(&rb));
-        const float g = fmaf(hr, tanh_approx_f(hr), hr);  // r sigmoid(r) = h + h tanh(h), h = r / 2
-        const float m_e = __shfl_sync(0xffffffffu, mu, e), s_e = __shfl_sync(0xffffffffu, rstd, e);
-        x[e] = fmaf(ln_w * (x[e] - m_e), s_e, ln_b) * g;
-      }
-      __syncwarp();
-      if (lane == 0) {
-        dev::mbar_arrive(&rempty[i & 1]);
-        dev::tma_store_wait_read();  // the output block's store has read the staging tile
-      }
-      __syncwarp();
-      const uint32_t so = dev::smem_u32(ost) + (uint32_t)(lane * 2);
-#pragma unroll
-      for (int e = 0; e < 32; ++e) {
-        const bf16 b = __float2bfloat16_rn(x[e]);
-        dev::st_shared_u16(so + (uint32_t)(e * 64), *reinterpret_cast<const uint16_t *>(&b));
-      }
-      dev::fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0 && ok) {
-        dev::tma_store_3d(&tmYo, ost, v0 + 32 * q4, chunk_of(i) * kC + 32 * hh, (int)bh);
         dev::tma_store_commit();
       }
     };
@@ -566,7 +672,6 @@ __global__ void __launch_bounds__(kWalkThreads, 1)
       }
       // ---- off the chain: S_{i-1} (still the A operand in TMEM) to the backward's
       // layout, then the previous chunk's output -------------------------------------
-      if (EPI && i >= 1) epi_a(i - 1);
       if (out && st_hb && ok) {
         // the whole row in one TMEM round trip, then its 16-byte stores back to back
         float wf[KH / 2];
@@ -576,21 +681,12 @@ __global__ void __launch_bounds__(kWalkThreads, 1)
 #pragma unroll
         for (int jb = 0; jb < KH / 32; ++jb) store_hb(n, jb, reinterpret_cast<const uint32_t *>(wf + 16 * jb));
       }
-      if (EPI) {
-        if (i >= 1) epi_b(i - 1);
-      } else if (out && i >= 1) {
-        epilogue(i - 1);
-      }
+      if (out && i >= 1) epilogue(i - 1);
     }
     if (out && nloc > 0) {
       if (ok) ok = dev::mbar_wait(&ofull[(nloc - 1) & 1], (uint32_t)(((nloc - 1) >> 1) & 1), a.status);
       dev::tc_fence_after();
-      if (EPI) {
-        epi_a(nloc - 1);
-        epi_b(nloc - 1);
-      } else {
-        epilogue(nloc - 1);
-      }
+      epilogue(nloc - 1);
     }
 
     // ---- state after the segment ----------------------------------------------
