@@ -50,6 +50,11 @@ constexpr int kWalkRegsState = 224;
 constexpr int kWalkRegsRole = 56;
 static_assert(256 * kWalkRegsState + 128 * kWalkRegsRole <= kWalkThreads * kWalkRegsLaunch,
               "register budgets exceed the launch allocation");
+// The fused-epilogue walk moves 8 registers per state thread to its epilogue warps.
+constexpr int kWalkRegsStateEpi = 216;
+constexpr int kWalkRegsRoleEpi = 72;
+static_assert(256 * kWalkRegsStateEpi + 128 * kWalkRegsRoleEpi <= kWalkThreads * kWalkRegsLaunch,
+              "register budgets exceed the launch allocation");
 
 // EPI: the output walk with the layer epilogue fused into its output store (one
 // ring slot fewer on each side, room for the gate tiles r and the row statistics).
@@ -211,7 +216,7 @@ __global__ void __launch_bounds__(kWalkThreads, 1)
   auto yslot = [&](int s) { return smem + L::kY0 + s * L::kYSlot; };
 
   if (warp >= kStateWarps) {
-    dev::regs_dec<kWalkRegsRole>();
+    dev::regs_dec<EPI ? kWalkRegsRoleEpi : kWalkRegsRole>();
     if (warp == kStateWarps) {
     // ============================ TMA producer ============================
     if (lane == 0) {
@@ -286,13 +291,10 @@ __global__ void __launch_bounds__(kWalkThreads, 1)
       auto oaddr = [&](int hr, int q, int j) {
         return dev::smem_u32(stg) + (uint32_t)((4 * hr + q) * 2048 + lane * 64 + ((j ^ ((lane >> 1) & 3)) << 4));
       };
-      auto ld4p = [&](uint32_t addr, dev::f2 *x) {  // 8 bf16 as 4 pairs
+      auto lds16 = [&](uint32_t addr) {
         uint4 u;
         asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];" : "=r"(u.x), "=r"(u.y), "=r"(u.z), "=r"(u.w) : "r"(addr));
-        x[0] = dev::bf16pair(u.x);
-        x[1] = dev::bf16pair(u.y);
-        x[2] = dev::bf16pair(u.z);
-        x[3] = dev::bf16pair(u.w);
+        return u;
       };
       for (int i = ew; i < nloc; i += 2) {
         const uint32_t par = (uint32_t)((i >> 1) & 1);
@@ -307,41 +309,45 @@ __global__ void __launch_bounds__(kWalkThreads, 1)
           dev::tma_store_commit();
         }
         // row statistics in one pass, shifted by the row's first value: sums of
-        // d = o - s and d^2 over the tile's 128 columns (both rows side by side)
+        // d = o - s and d^2 over the tile's 128 columns (both rows side by side, two
+        // accumulators each, a block's eight 16-byte loads issued together)
         float mean[2], m2[2];
         {
-          dev::f2 sh[2], sd[2], sq[2];
+          dev::f2 sh[2], sd[2][2], sq[2][2];
 #pragma unroll
           for (int hr = 0; hr < 2; ++hr) {
-            dev::f2 x[4];
-            ld4p(oaddr(hr, 0, 0), x);
-            float lo, hi;
-            dev::upk(x[0], lo, hi);
-            sh[hr] = dev::pk(-lo, -lo);
-            sd[hr] = dev::pk(0.f, 0.f);
-            sq[hr] = dev::pk(0.f, 0.f);
+            const uint4 u = lds16(oaddr(hr, 0, 0));
+            const float s0 = __uint_as_float(u.x << 16);
+            sh[hr] = dev::pk(-s0, -s0);
+            sd[hr][0] = sd[hr][1] = sq[hr][0] = sq[hr][1] = dev::pk(0.f, 0.f);
           }
-#pragma unroll 2
-          for (int c16 = 0; c16 < 16; ++c16) {
+#pragma unroll 1
+          for (int q = 0; q < 4; ++q) {
+            uint4 u[2][4];
 #pragma unroll
-            for (int hr = 0; hr < 2; ++hr) {
-              dev::f2 x[4];
-              ld4p(oaddr(hr, c16 >> 2, c16 & 3), x);
+            for (int hr = 0; hr < 2; ++hr)
 #pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const dev::f2 d = dev::add2(x[e], sh[hr]);
-                sd[hr] = dev::add2(sd[hr], d);
-                sq[hr] = dev::fma2(d, d, sq[hr]);
+              for (int j = 0; j < 4; ++j) u[hr][j] = lds16(oaddr(hr, q, j));
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+#pragma unroll
+              for (int hr = 0; hr < 2; ++hr) {
+                const uint32_t w4[4] = {u[hr][j].x, u[hr][j].y, u[hr][j].z, u[hr][j].w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  const dev::f2 d = dev::add2(dev::bf16pair(w4[e]), sh[hr]);
+                  sd[hr][e & 1] = dev::add2(sd[hr][e & 1], d);
+                  sq[hr][e & 1] = dev::fma2(d, d, sq[hr][e & 1]);
+                }
               }
-            }
           }
 #pragma unroll
           for (int hr = 0; hr < 2; ++hr) {
             float s0, s1;
             dev::upk(sh[hr], s0, s1);
-            const float sdv = dev::hsum(sd[hr]);
+            const float sdv = dev::hsum(dev::add2(sd[hr][0], sd[hr][1]));
             mean[hr] = sdv * (1.f / (float)BV) - s0;
-            m2[hr] = fmaxf(dev::hsum(sq[hr]) - sdv * sdv * (1.f / (float)BV), 0.f);
+            m2[hr] = fmaxf(dev::hsum(dev::add2(sq[hr][0], sq[hr][1])) - sdv * sdv * (1.f / (float)BV), 0.f);
           }
         }
         // to slots [rank][t] of buffer i % 4 of every CTA, then one arrival per CTA
@@ -379,8 +385,27 @@ __global__ void __launch_bounds__(kWalkThreads, 1)
         if (lane == 0) dev::tma_store_wait_read();
         __syncwarp();
         if (ok) ok = dev::mbar_wait(&rfull[ew], par, a.status);
+        // columns 8 c16 .. 8 c16 + 7 of the tile per step; the next step's o and r
+        // are loaded before this step's results are stored
+        auto raddr = [&](int hr, int c16) {
+          const int t = 32 * hr + lane;
+          return dev::smem_u32(rt) + (uint32_t)((c16 >> 3) * 8192 + t * 128 + (((c16 & 7) ^ (t & 7)) << 4));
+        };
+        uint4 ou[2], ru[2];
+#pragma unroll
+        for (int hr = 0; hr < 2; ++hr) {
+          ou[hr] = lds16(oaddr(hr, 0, 0));
+          ru[hr] = lds16(raddr(hr, 0));
+        }
 #pragma unroll 1
-        for (int c16 = 0; c16 < 16; ++c16) {  // columns 8 c16 .. 8 c16 + 7 of the tile
+        for (int c16 = 0; c16 < 16; ++c16) {
+          uint4 on[2], rn[2];
+          const int cn = c16 < 15 ? c16 + 1 : c16;
+#pragma unroll
+          for (int hr = 0; hr < 2; ++hr) {
+            on[hr] = lds16(oaddr(hr, cn >> 2, cn & 3));
+            rn[hr] = lds16(raddr(hr, cn));
+          }
           dev::f2 w2[4], b2[4];
           {
             const ulonglong2 w01 = *reinterpret_cast<const ulonglong2 *>(sW + 8 * c16);
@@ -390,28 +415,33 @@ __global__ void __launch_bounds__(kWalkThreads, 1)
             w2[0] = w01.x, w2[1] = w01.y, w2[2] = w23.x, w2[3] = w23.y;
             b2[0] = b01.x, b2[1] = b01.y, b2[2] = b23.x, b2[3] = b23.y;
           }
+          uint32_t pkd[2][4];
 #pragma unroll
           for (int hr = 0; hr < 2; ++hr) {
-            const int t = 32 * hr + lane;
-            dev::f2 x[4], r[4];
-            const uint32_t oa = oaddr(hr, c16 >> 2, c16 & 3);
-            ld4p(oa, x);
-            ld4p(dev::smem_u32(rt) + (uint32_t)((c16 >> 3) * 8192 + t * 128 + (((c16 & 7) ^ (t & 7)) << 4)), r);
-            uint32_t pkd[4];
+            const uint32_t xo[4] = {ou[hr].x, ou[hr].y, ou[hr].z, ou[hr].w};
+            const uint32_t xr[4] = {ru[hr].x, ru[hr].y, ru[hr].z, ru[hr].w};
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              const dev::f2 nrm = dev::fma2(dev::mul2(dev::add2(x[e], nmu2[hr]), rs2[hr]), w2[e], b2[e]);
-              const dev::f2 h = dev::mul2(r[e], half2);
+              const dev::f2 nrm =
+                  dev::fma2(dev::mul2(dev::add2(dev::bf16pair(xo[e]), nmu2[hr]), rs2[hr]), w2[e], b2[e]);
+              const dev::f2 h = dev::mul2(dev::bf16pair(xr[e]), half2);
               float hl, hh2;
               dev::upk(h, hl, hh2);
               const dev::f2 g = dev::fma2(h, dev::pk(dev::tanh_approx(hl), dev::tanh_approx(hh2)), h);  // r sigmoid(r)
               float y0, y1;
               dev::upk(dev::mul2(nrm, g), y0, y1);
-              pkd[e] = dev::pack_bf16(y0, y1);
+              pkd[hr][e] = dev::pack_bf16(y0, y1);
             }
-            asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(oa), "r"(pkd[0]), "r"(pkd[1]), "r"(pkd[2]),
-                         "r"(pkd[3])
+          }
+#pragma unroll
+          for (int hr = 0; hr < 2; ++hr)
+            asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(oaddr(hr, c16 >> 2, c16 & 3)), "r"(pkd[hr][0]),
+                         "r"(pkd[hr][1]), "r"(pkd[hr][2]), "r"(pkd[hr][3])
                          : "memory");
+#pragma unroll
+          for (int hr = 0; hr < 2; ++hr) {
+            ou[hr] = on[hr];
+            ru[hr] = rn[hr];
           }
         }
         dev::fence_proxy_async_smem();
@@ -516,7 +546,7 @@ __global__ void __launch_bounds__(kWalkThreads, 1)
     }
     }
   } else {
-    dev::regs_inc<kWalkRegsState>();
+    dev::regs_inc<EPI ? kWalkRegsStateEpi : kWalkRegsState>();
     // ============================ state threads ============================
     const int q4 = warp & 3, hh = warp >> 2;
     const int v = 32 * q4 + lane;  // TMEM lane = row of S^T
