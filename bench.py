@@ -244,11 +244,12 @@ def run_reference(args, w):
 
 # ------------------------------------------------------------------------------------ ours
 def walk_segments(w, sms):
-    """Segment count the library picks for the walks (one wave of two CTAs per SM)."""
+    """Segment count the library picks for the walks (one wave of one CTA per SM over
+    the heads' 128-column d_v tiles)."""
     B, H, T, K, V, C = w["B"], w["H"], w["T"], w["K"], w["V"], w["C"]
     N = -(-T // C)
-    bv = 64 if (K == 256 or V % 128) else 128
-    P = max(1, (2 * sms) // (B * H * (V // bv)))
+    nvt = -(-V // 128)
+    P = max(1, sms // (B * H * nvt))
     P = min(P, N)
     L = -(-N // P)
     return -(-N // L)
@@ -829,6 +830,84 @@ def time_workload(c, args, dev, stream, peaks, C=64):
             "frac_of_roofline": max(flops / peak_t, abytes / peak_b) / (ms / 1e3)}
 
 
+def measure_e2e(args, x, step_on, dev_in, dev_out, stream, world, dev):
+    """The step end to end through the public API with the inputs in pinned host
+    memory and the results read back to it, every step: a copy-in stream, the compute
+    stream and a copy-out stream with two sets of device buffers, so that step j's
+    computation overlaps the copy-in of step j + 1 and the copy-out of step j - 1
+    (each on its own copy engine).  Timed with events from the first copy-in to the
+    last copy-out (max over ranks).  Also the same steps with the copies and the
+    computation in one stream (serial_ms_per_step), for comparison."""
+    import torch
+    import torch.distributed as dist
+
+    pin = lambda t: t.cpu().pin_memory()
+    h_in = [pin(t) for t in (x.q, x.k, x.v, x.log_alpha, x.do)]
+    h_out = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in dev_out]
+    h2d = sum(t.numel() * t.element_size() for t in h_in)
+    d2h = sum(t.numel() * t.element_size() for t in h_out)
+    ins = [list(dev_in), [torch.empty_like(t) for t in dev_in]]
+    outs = [list(dev_out), [torch.empty_like(t) for t in dev_out]]
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    in_ready, done, out_copied = [ev(), ev()], [ev(), ev()], [ev(), ev()]
+    for b in range(2):  # every buffer starts free
+        done[b].record(stream)
+        out_copied[b].record(stream)
+
+    def run(n):
+        for j in range(n):
+            b = j & 1
+            s_in.wait_event(done[b])  # step j - 2 has read these inputs
+            with torch.cuda.stream(s_in):
+                for dst, src in zip(ins[b], h_in):
+                    dst.copy_(src, non_blocking=True)
+            in_ready[b].record(s_in)
+            stream.wait_event(in_ready[b])
+            stream.wait_event(out_copied[b])  # step j - 2's results have left these outputs
+            step_on(ins[b], outs[b], stream)
+            done[b].record(stream)
+            s_out.wait_event(done[b])
+            with torch.cuda.stream(s_out):
+                for dst, src in zip(h_out, outs[b]):
+                    dst.copy_(src, non_blocking=True)
+            out_copied[b].record(s_out)
+
+    run(2)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    n = max(2, args.steps // 2)
+    f0, f1 = ev(), ev()
+    f0.record(s_in)
+    run(n)
+    f1.record(s_out)
+    torch.cuda.synchronize()
+    ms_total = reduce_max_ms(f0.elapsed_time(f1), world, dev)
+
+    # the serial form: copy-in, step, copy-out on the compute stream
+    def serial():
+        for dst, src in zip(ins[0], h_in):
+            dst.copy_(src, non_blocking=True)
+        step_on(ins[0], outs[0], stream)
+        for dst, src in zip(h_out, outs[0]):
+            dst.copy_(src, non_blocking=True)
+
+    serial()
+    torch.cuda.synchronize()
+    g0, g1 = ev(), ev()
+    g0.record(stream)
+    for _ in range(n):
+        serial()
+    g1.record(stream)
+    torch.cuda.synchronize()
+    serial_ms = reduce_max_ms(g0.elapsed_time(g1), world, dev) / n
+    return {"steps": n, "ms_total": ms_total, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "serial_ms_per_step": serial_ms,
+            "pipeline": "copy-in, compute and copy-out streams, two device buffer sets: step j overlaps the "
+                        "copy-in of step j+1 and the copy-out of step j-1"}
+
+
 def run_ours(args, w):
     import torch
     import torch.distributed as dist
@@ -857,10 +936,17 @@ def run_ours(args, w):
     ws = pkg.alloc_workspace(pkg.workspace_size(B, H, T, K, V, torch.bfloat16, w["gate"], C, True, flags=flags), dev)
     stream = torch.cuda.current_stream()
 
-    def step(qq=q, kk=k, vv=v, ll=la, dd=do):
-        pkg.gla_fwd(qq, kk, vv, ll, None, chunk=C, o=o, h_final=hT, workspace=ws, stream=stream, save_states=True)
-        pkg.gla_bwd(qq, kk, vv, ll, dd, None, None, chunk=C, dq=dq, dk=dk, dv=dv, dlog_alpha=dla, want_dh0=False,
-                    workspace=ws, stream=stream, reuse_prep=True, saved_states=True)
+    def step_on(ins, outs, st):
+        """One training step of the workload: gla_fwd then gla_bwd on `st`, inputs
+        (q, k, v, log_alpha, do) and outputs (o, dq, dk, dv, dlog_alpha) as given."""
+        qq, kk, vv, ll, dd = ins
+        oo, dqq, dkk, dvv, dll = outs
+        pkg.gla_fwd(qq, kk, vv, ll, None, chunk=C, o=oo, h_final=hT, workspace=ws, stream=st, save_states=True)
+        pkg.gla_bwd(qq, kk, vv, ll, dd, None, None, chunk=C, dq=dqq, dk=dkk, dv=dvv, dlog_alpha=dll, want_dh0=False,
+                    workspace=ws, stream=st, reuse_prep=True, saved_states=True)
+
+    def step():
+        step_on((q, k, v, la, do), (o, dq, dk, dv, dla), stream)
 
     for _ in range(args.warmup):
         step()
@@ -899,35 +985,8 @@ def run_ours(args, w):
     value = aggregate_value(B * T, world, args.steps, ms)
 
     # ---- end to end through the public API with host buffers ----------------------------
-    pin = lambda t: t.cpu().pin_memory()
-    hq, hk, hv, hla, hdo = pin(x.q), pin(x.k), pin(x.v), pin(x.log_alpha), pin(x.do)
-    ho = torch.empty(o.shape, dtype=o.dtype).pin_memory()
-    hdq, hdk, hdv = (torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (dq, dk, dv))
-    hdla = torch.empty(dla.shape, dtype=dla.dtype).pin_memory()
-    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hla, hdo))
-    d2h = sum(t.numel() * t.element_size() for t in (ho, hdq, hdk, hdv, hdla))
-
-    def e2e_step():
-        for dst, src in ((q, hq), (k, hk), (v, hv), (la, hla), (do, hdo)):
-            dst.copy_(src, non_blocking=True)
-        step()
-        for dst, src in ((ho, o), (hdq, dq), (hdk, dk), (hdv, dv), (hdla, dla)):
-            dst.copy_(src, non_blocking=True)
-
-    for _ in range(2):
-        e2e_step()
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    f0.record(stream)
-    n_e2e = max(1, args.steps // 2)
-    for _ in range(n_e2e):
-        e2e_step()
-    f1.record(stream)
-    torch.cuda.synchronize()
-    ems = reduce_max_ms(f0.elapsed_time(f1), world, dev)
-    e2e_value = aggregate_value(B * T, world, n_e2e, ems)
+    e2e = measure_e2e(args, x, step_on, (q, k, v, la, do), (o, dq, dk, dv, dla), stream, world, dev)
+    e2e_value = aggregate_value(B * T, world, e2e["steps"], e2e["ms_total"])
 
     # ---- roofline of the dominant kernel --------------------------------------------------
     peaks, peak_src = load_peaks()
@@ -1000,7 +1059,9 @@ def run_ours(args, w):
                         for k2, v2 in sorted(per_kernel.items(), key=lambda kv: -kv[1][1])},
             "gpu_launches": len(launches),
             "kernel_timing": "separate pass of the same K steps with a CUDA-event pair around each launch",
-            "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": e2e["h2d_bytes_per_step"],
+                    "d2h_bytes_per_step": e2e["d2h_bytes_per_step"], "ms_per_step": e2e["ms_total"] / e2e["steps"],
+                    "pipeline": e2e["pipeline"], "serial_ms_per_step": e2e["serial_ms_per_step"]},
             "clocks": clocks, "cpu_baseline": cpu, "decode_step": decode, "layer_epilogue": epilogue,
             "sequence_parallel": seqpar, "general_gate": general, "variants": variants,
             "sweep_vs_T": None if sweep_T is None else {
