@@ -11,11 +11,11 @@
 //
 //   k_fold_segments  a piece's summary from the walk's segment contributions: the
 //                    zero-state pre-pass runs every segment of the piece in parallel
-//                    (contributions delta_p [BH][P][V][K], gate products gseg_p);
+//                    (contributions delta_p [BH][P][K/4][V][4], gate products gseg_p);
 //                    out = fold over p of S <- diag(gseg_p) S + delta_p
 //   k_segment_starts the start state of every segment of a walk from the same
 //                    contributions: S = h0; S <- diag(gseg_p) S + delta_p, stored after
-//                    each p as the start of the next segment ([BH][P][V][K])
+//                    each p as the start of the next segment ([BH][P][K/4][V][4])
 //                    from h0 (dh_final in reverse), gamma = prod_p gseg_p
 //   k_state_scan     out = fold over the selected pieces of S <- diag(gamma_s) S + D_s
 //                    (elementwise per (bh, c, v), HBM-bound: one read of every D_s)
@@ -24,20 +24,22 @@
 namespace gla {
 namespace {
 
-// Thread (bh, v, c4), c4 fastest: delta[bh][p][v][4 c4 .. 4 c4 + 3] is read
-// coalesced; out[bh][4 c4 .. 4 c4 + 3][v] and h0 are strided (one pass).
+// Segment contributions and start states are [BH][P][K/4][V] float4 groups (the
+// four channels 4 c4 .. 4 c4 + 3 of value column v in one float4, as the walk
+// stores them).  Thread (bh, c4, v), v fastest: those are read and written as
+// 512 contiguous bytes per warp, the [K][V] states (h0, out) as 128 per channel.
 __global__ void __launch_bounds__(256) k_fold_segments(long BH, int K, int V, int P, int reverse,
-                                                       const float *__restrict__ gseg,
+                                                       const float4 *__restrict__ gseg,
                                                        const float4 *__restrict__ delta,
                                                        const float *__restrict__ h0, float *__restrict__ out,
-                                                       float *__restrict__ gamma) {
+                                                       float4 *__restrict__ gamma) {
   const int K4 = K / 4;
-  const long i = (long)blockIdx.x * blockDim.x + threadIdx.x;  // float4 index in [BH][V][K/4]
-  if (i >= BH * V * K4) return;
-  const int c4 = (int)(i % K4);
-  const int v = (int)((i / K4) % V);
-  const long bh = i / ((long)K4 * V);
-  const long o = (bh * K + 4 * c4) * (long)V + v;  // element (c = 4 c4, v) of [BH][K][V]
+  const long i = (long)blockIdx.x * blockDim.x + threadIdx.x;  // index in [BH][K/4][V]
+  if (i >= BH * K4 * V) return;
+  const int v = (int)(i % V);
+  const int c4 = (int)((i / V) % K4);
+  const long bh = i / ((long)V * K4);
+  const long o = (bh * K + 4 * c4) * (long)V + v;  // element (4 c4, v) of [BH][K][V]
   float4 S = make_float4(0.f, 0.f, 0.f, 0.f);
   if (h0) S = make_float4(__ldg(h0 + o), __ldg(h0 + o + V), __ldg(h0 + o + 2L * V), __ldg(h0 + o + 3L * V));
   float4 gp = make_float4(1.f, 1.f, 1.f, 1.f);
@@ -46,8 +48,8 @@ __global__ void __launch_bounds__(256) k_fold_segments(long BH, int K, int V, in
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       const int j = j0 + u, p = reverse ? P - 1 - j : j;
-      g[u] = j < P ? __ldg(reinterpret_cast<const float4 *>(gseg + (bh * P + p) * K) + c4) : make_float4(1.f, 1.f, 1.f, 1.f);
-      d[u] = j < P ? __ldg(delta + ((bh * P + p) * V + v) * K4 + c4) : make_float4(0.f, 0.f, 0.f, 0.f);
+      g[u] = j < P ? __ldg(gseg + (bh * P + p) * K4 + c4) : make_float4(1.f, 1.f, 1.f, 1.f);
+      d[u] = j < P ? __ldg(delta + ((bh * P + p) * K4 + c4) * V + v) : make_float4(0.f, 0.f, 0.f, 0.f);
     }
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
@@ -65,15 +67,15 @@ __global__ void __launch_bounds__(256) k_fold_segments(long BH, int K, int V, in
   out[o + V] = S.y;
   out[o + 2L * V] = S.z;
   out[o + 3L * V] = S.w;
-  if (gamma && v == 0) *reinterpret_cast<float4 *>(gamma + bh * K + 4 * c4) = gp;
+  if (gamma && v == 0) gamma[bh * K4 + c4] = gp;
 }
 
-// Start states of the segments of one walk: thread (bh, v, c4) folds the
+// Start states of the segments of one walk: thread (bh, c4, v) folds the
 // contributions in walk order (forward: 0 .. P-2; reverse: P-1 .. 1) from h0
 // ([BH][K][V] or zero) and stores the state after each as the next segment's
-// start, starts[bh][p][v][4 c4 ..] (the segment that begins from h0 is not written).
+// start (the segment that begins from h0 is not written).
 __global__ void __launch_bounds__(256) k_segment_starts(long BH, int K, int V, int P, int reverse,
-                                                        const float *__restrict__ gseg,
+                                                        const float4 *__restrict__ gseg,
                                                         const float4 *__restrict__ delta,
                                                         const float *__restrict__ h0, float4 *__restrict__ starts) {
   // launched with programmatic stream serialization: wait for the walk that wrote
@@ -81,11 +83,11 @@ __global__ void __launch_bounds__(256) k_segment_starts(long BH, int K, int V, i
   dev::pdl_launch_dependents();
   dev::pdl_wait();
   const int K4 = K / 4;
-  const long i = (long)blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= BH * V * K4) return;
-  const int c4 = (int)(i % K4);
-  const int v = (int)((i / K4) % V);
-  const long bh = i / ((long)K4 * V);
+  const long i = (long)blockIdx.x * blockDim.x + threadIdx.x;  // index in [BH][K/4][V]
+  if (i >= BH * K4 * V) return;
+  const int v = (int)(i % V);
+  const int c4 = (int)((i / V) % K4);
+  const long bh = i / ((long)V * K4);
   float4 S = make_float4(0.f, 0.f, 0.f, 0.f);
   if (h0) {
     const long o = (bh * K + 4 * c4) * (long)V + v;
@@ -97,8 +99,8 @@ __global__ void __launch_bounds__(256) k_segment_starts(long BH, int K, int V, i
     for (int u = 0; u < 4; ++u) {
       const int j = j0 + u, p = reverse ? P - 1 - j : j;
       if (j + 1 < P) {
-        g[u] = __ldg(reinterpret_cast<const float4 *>(gseg + (bh * P + p) * K) + c4);
-        d[u] = __ldg(delta + ((bh * P + p) * V + v) * K4 + c4);
+        g[u] = __ldg(gseg + (bh * P + p) * K4 + c4);
+        d[u] = __ldg(delta + ((bh * P + p) * K4 + c4) * V + v);
       }
     }
 #pragma unroll
@@ -109,7 +111,7 @@ __global__ void __launch_bounds__(256) k_segment_starts(long BH, int K, int V, i
         S.y = g[u].y * S.y + d[u].y;
         S.z = g[u].z * S.z + d[u].z;
         S.w = g[u].w * S.w + d[u].w;
-        starts[((bh * P + (reverse ? p - 1 : p + 1)) * V + v) * K4 + c4] = S;  // the segment it starts
+        starts[((bh * P + (reverse ? p - 1 : p + 1)) * K4 + c4) * V + v] = S;  // the segment it starts
       }
     }
   }
@@ -149,19 +151,19 @@ __global__ void __launch_bounds__(256) k_state_scan(long BH, int K, int V, int s
 
 int fold_segments(long BH, int K, int V, int P, int reverse, const float *gseg, const float *delta, const float *h0,
                   float *out, float *gamma, cudaStream_t st) {
-  const long n = BH * V * (K / 4);
+  const long n = BH * (K / 4) * V;
   GLA_LAUNCH(K_FOLD_SEGMENTS, st,
-             (k_fold_segments<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(BH, K, V, P, reverse, gseg,
-                                                                          (const float4 *)delta, h0, out, gamma)));
+             (k_fold_segments<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(
+                 BH, K, V, P, reverse, (const float4 *)gseg, (const float4 *)delta, h0, out, (float4 *)gamma)));
   return GLA_OK;
 }
 
 int segment_starts(long BH, int K, int V, int P, int reverse, const float *gseg, const float *delta, const float *h0,
                    float *starts, cudaStream_t st) {
-  const long n = BH * V * (K / 4);
+  const long n = BH * (K / 4) * V;
   GLA_LAUNCH(K_SEG_STARTS, st,
              if (launch_pdl(k_segment_starts, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, st, BH, K, V, P,
-                            reverse, gseg, (const float4 *)delta, h0, (float4 *)starts) != cudaSuccess)
+                            reverse, (const float4 *)gseg, (const float4 *)delta, h0, (float4 *)starts) != cudaSuccess)
                  return GLA_ERR_CUDA);
   return GLA_OK;
 }

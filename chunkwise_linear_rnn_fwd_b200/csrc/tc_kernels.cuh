@@ -315,15 +315,15 @@ struct WalkArgs {
   int T, N, V, L;  // L = chunks per segment
   int P;           // segments per sequence (the grid covers segments seg0 .. seg0 + gridDim.y - 1)
   int seg0;
-  int end_seg;     // -1: every segment writes end[BH][P][V][K]; s >= 0: only segment s writes end[BH][K][V]
+  int end_seg;     // -1: every segment writes end[BH][P][K/4][V][4]; s >= 0: only segment s writes end[BH][K][V]
   int reverse, do_out, state_mode;  // state_mode: 0 none, 1 bf16 chunk states, 2 fp32 chunk states
   int p_kmajor;                     // output intra term: 0 = P V (forward), 1 = P^T dO (reverse: dv)
   const float *gam;                 // [BH][N][K]
   const float *start;               // [BH][P][K][V] fp32 start states (materialised chunk states) or null
-  const float *start_v;             // [BH][P][V][K] fp32 start states of the segments after the first
+  const float *start_v;             // [BH][P][K/4][V][4] fp32 start states of the segments after the first
                                     // (before it, reverse) or null; the first starts from h0
   const float *h0;                  // initial state of the whole walk (h0, or dh_final in reverse) or null
-  float *end;                       // state after the segment or null: end_seg < 0: [BH][P][V][K]
+  float *end;                       // state after the segment or null: end_seg < 0: [BH][P][K/4][V][4]
                                     // (segment contributions); else [BH][K][V] fp32
   float *gseg;                      // [BH][P][K] product of gam over the segment (written by d_v tile 0) or null
   float *h32;                       // [BH][N][K][V] fp32 states (state_mode 2)

@@ -129,9 +129,9 @@ int segments_of(const Problem &p, int nvt) {
 struct TcWs {
   bf16 *qg, *kg, *PT;
   float *gam;
-  float *delta;          // [BH][P][V][K] segment contributions from a zero state
+  float *delta;          // [BH][P][K/4][V][4] segment contributions from a zero state
   float *gseg;           // [BH][P][K] per-segment gate products
-  float *starts;         // [BH][P][V][K] segment start states (folded from h0 and the contributions)
+  float *starts;         // [BH][P][K/4][V][4] segment start states (folded from h0 and the contributions)
   float *h32;            // materialised fp32 chunk states [BH][N][K][V]
   // backward
   bf16 *hb, *dhb;        // bf16 chunk states and adjoints, tc::state_chunk_off layout

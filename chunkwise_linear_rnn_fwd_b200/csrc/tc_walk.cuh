@@ -558,14 +558,15 @@ __global__ void __launch_bounds__(kWalkThreads, 1)
     float S[KH];
 
     // ---- start state: h0 for the first segment (the last, reverse), else the
-    // segment's start state [V][K] (row vg contiguous) or a materialised [K][V] state
+    // segment's start state ([K/4][V] float4 groups of four channels: a warp reads
+    // 512 contiguous bytes per group) or a materialised [K][V] chunk state
     {
       const bool first = seg == (a.reverse ? P - 1 : 0);
       if (a.start_v && !first) {
-        const float4 *src = reinterpret_cast<const float4 *>(a.start_v + ((bh * P + seg) * (long)a.V + vg) * K + c0);
+        const float4 *src = reinterpret_cast<const float4 *>(a.start_v) + ((bh * P + seg) * (K / 4) + c0 / 4) * a.V + vg;
 #pragma unroll
         for (int j4 = 0; j4 < KH / 4; ++j4) {
-          const float4 x = vok ? __ldg(src + j4) : make_float4(0.f, 0.f, 0.f, 0.f);
+          const float4 x = vok ? __ldg(src + (long)j4 * a.V) : make_float4(0.f, 0.f, 0.f, 0.f);
           S[4 * j4] = x.x;
           S[4 * j4 + 1] = x.y;
           S[4 * j4 + 2] = x.z;
@@ -721,11 +722,12 @@ __global__ void __launch_bounds__(kWalkThreads, 1)
 
     // ---- state after the segment ----------------------------------------------
     if (a.end && a.end_seg < 0 && vok && ok) {
-      // segment contribution, [BH][P][V][K]: this thread's row, 16 bytes at a time
-      float4 *dst = reinterpret_cast<float4 *>(a.end + ((bh * P + seg) * (long)a.V + vg) * K + c0);
+      // segment contribution, [BH][P][K/4][V] float4 groups (a warp stores 512
+      // contiguous bytes per group of four channels)
+      float4 *dst = reinterpret_cast<float4 *>(a.end) + ((bh * P + seg) * (K / 4) + c0 / 4) * a.V + vg;
 #pragma unroll
       for (int j4 = 0; j4 < KH / 4; ++j4)
-        dst[j4] = make_float4(S[4 * j4], S[4 * j4 + 1], S[4 * j4 + 2], S[4 * j4 + 3]);
+        dst[(long)j4 * a.V] = make_float4(S[4 * j4], S[4 * j4 + 1], S[4 * j4 + 2], S[4 * j4 + 3]);
     }
     if (a.end && a.end_seg == seg && vok && ok) {
       // the walk's final state, [BH][K][V] (a warp stores 128 contiguous bytes per channel)
