@@ -73,6 +73,13 @@ struct BwdSmem {
   static constexpr int kQt = kdPd + 64 * 16 * 4;              // q tile [64][128] bf16 (TMA, after phase 1)
   static constexpr int kKt = kQt + 64 * kBwdKH * 2;           // k tile [64][128] bf16
   static constexpr int kPhase2End = kKt + 64 * kBwdKH * 2;
+  // epilogue (aliases the windows and dP tiles, dead once the phase-2 MMAs are done):
+  // dq, dk [2 column halves][64 t][64 c] bf16 and dlog alpha [2][64 t][64 c] fp32,
+  // each column half one TMA store box
+  static constexpr int kSDq = 0;
+  static constexpr int kSDk = kSDq + 64 * kBwdKH * 2;
+  static constexpr int kSDla = kSDk + 64 * kBwdKH * 2;
+  static_assert(kSDla + 64 * kBwdKH * 4 <= kdPd, "epilogue staging stays clear of the diagonal blocks");
   static constexpr int kRed = (kPhase1End > kPhase2End ? kPhase1End : kPhase2End);  // scalar-gate sums [4][64]
   static constexpr int kRed2 = kRed + 4 * 64 * 4;            // sums of h (.) dh [128]
   static constexpr int kBar = kRed2 + kBwdKH * 4;
@@ -82,7 +89,9 @@ struct BwdSmem {
 template <int K>
 __global__ void __launch_bounds__(kBwdKH, 2)
     k_bwd_main(BwdArgs a, const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
-               const __grid_constant__ CUtensorMap tmQin, const __grid_constant__ CUtensorMap tmKin) {
+               const __grid_constant__ CUtensorMap tmQin, const __grid_constant__ CUtensorMap tmKin,
+               const __grid_constant__ CUtensorMap tmDQ, const __grid_constant__ CUtensorMap tmDK,
+               const __grid_constant__ CUtensorMap tmDLA) {
   using L = BwdSmem;
   constexpr int BVb = L::BVb;
   constexpr int kH = K / kBwdKH;  // CTAs per chunk
@@ -417,7 +426,10 @@ __global__ void __launch_bounds__(kBwdKH, 2)
   dev::tc_fence_after();
 
   // ============================ epilogue ============================
-  // reverse over sub-chunks and tokens: dq, dk, dlog b and its suffix sum
+  // reverse over sub-chunks and tokens: dq, dk, dlog b and its suffix sum, staged in
+  // shared memory for three TMA stores
+  const uint32_t sDq = dev::smem_u32(smem + L::kSDq), sDk = dev::smem_u32(smem + L::kSDk),
+                 sDla = dev::smem_u32(smem + L::kSDla);
   float run = Gb;
   float gnext[16];
   load16(3, gnext);
@@ -483,10 +495,15 @@ __global__ void __launch_bounds__(kBwdKH, 2)
       const float dqr = uu[e] * (Ej * xq[e] + offq_on * xqi[e]);
       const float dkr = ww[e] * (GAj * xk[e] + offk_on * xki[e]);
       run += (qv[e] * dqr - kv[e] * dkr) + (qv[e] * dqd_e - kv[e] * dkd_e);
-      if (tg < a.T && ok) {
-        a.dq[(qrow0 + t) * K + c] = __float2bfloat16_rn(dqr + dqd_e);
-        a.dk[(qrow0 + t) * K + c] = __float2bfloat16_rn(dkr + dkd_e);
-        if (a.gate == GLA_GATE_VECTOR) a.dla[(qrow0 + t) * K + c] = run;
+      {
+        // into the staging tiles (rows beyond T are clipped by the stores)
+        const uint32_t e16 = (uint32_t)((cl >> 6) * 4096 + t * 64 + (cl & 63));
+        const bf16 bq = __float2bfloat16_rn(dqr + dqd_e), bk = __float2bfloat16_rn(dkr + dkd_e);
+        dev::st_shared_u16(sDq + 2u * e16, *reinterpret_cast<const uint16_t *>(&bq));
+        dev::st_shared_u16(sDk + 2u * e16, *reinterpret_cast<const uint16_t *>(&bk));
+        if (a.gate == GLA_GATE_VECTOR)
+          asm volatile("st.shared.f32 [%0], %1;" ::"r"(sDla + 4u * e16), "f"(run) : "memory");
+        (void)tg;
       }
       if (a.gate == GLA_GATE_SCALAR) {
         float x = run;
@@ -496,8 +513,19 @@ __global__ void __launch_bounds__(kBwdKH, 2)
       }
     }
   }
+  dev::fence_proxy_async_smem();
+  __syncthreads();
+  if (tid == 0 && ok) {
+#pragma unroll
+    for (int hc = 0; hc < kBwdKH / 64; ++hc) {
+      dev::tma_store_3d(&tmDQ, smem + L::kSDq + hc * 8192, c0 + 64 * hc, n * kC, (int)bh);
+      dev::tma_store_3d(&tmDK, smem + L::kSDk + hc * 8192, c0 + 64 * hc, n * kC, (int)bh);
+      if (a.gate == GLA_GATE_VECTOR)
+        dev::tma_store_3d(&tmDLA, smem + L::kSDla + hc * 16384, c0 + 64 * hc, n * kC, (int)bh);
+    }
+    dev::tma_store_commit();
+  }
   if (a.gate == GLA_GATE_SCALAR) {
-    __syncthreads();
     if (tid < kC) {
       float ssum = 0.f;
 #pragma unroll
@@ -509,6 +537,7 @@ __global__ void __launch_bounds__(kBwdKH, 2)
       }
     }
   }
+  if (tid == 0) dev::tma_store_wait_all();  // the stores have read their tiles before the CTA ends
   dev::tc_fence_before();
   __syncthreads();
   if (warp == 0) dev::tmem_dealloc(tmem, kTmemCols);
@@ -525,20 +554,27 @@ int launch_bwd_main_k(const Problem &p, const BwdArgs &a, const CUtensorMap *map
   if (smem < 0) return GLA_ERR_CUDA;
   GLA_LAUNCH(K_TC_BWD, st,
              if (launch_pdl(k_bwd_main<K>, dim3(K / kBwdKH, p.N, p.BH), dim3(kBwdKH), smem, st, a, maps[0], maps[1],
-                            maps[2], maps[3]) != cudaSuccess) return GLA_ERR_CUDA);
+                            maps[2], maps[3], maps[4], maps[5], maps[6]) != cudaSuccess) return GLA_ERR_CUDA);
   return GLA_OK;
 }
 
 bool map3_bf16(CUtensorMap *m, const void *base, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t b0, uint32_t b1);
+// row-major staging tile -> tensor (no swizzle), bf16 or fp32 elements
+bool map3_store(CUtensorMap *m, const void *base, bool fp32, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t b0,
+                uint32_t b1);
 
 inline int launch_bwd_main(const Problem &p, const bf16 *q, const bf16 *k, const bf16 *v, const float *la,
                            const bf16 *dout, bf16 *dq, bf16 *dk, float *dla, const float *gam, const bf16 *hb,
                            const bf16 *dhb, unsigned *status, cudaStream_t st) {
   if (p.V % 64 != 0 || p.K % kBwdKH != 0) return GLA_ERR_UNSUPPORTED_SHAPE;
-  CUtensorMap maps[4];
+  CUtensorMap maps[7];
   const uint64_t BH = (uint64_t)p.BH;
-  const bool ok = map3_bf16(&maps[0], v, p.V, p.T, BH, 64, 64) && map3_bf16(&maps[1], dout, p.V, p.T, BH, 64, 64) &&
-                  map3_bf16(&maps[2], q, p.K, p.T, BH, 64, 64) && map3_bf16(&maps[3], k, p.K, p.T, BH, 64, 64);
+  bool ok = map3_bf16(&maps[0], v, p.V, p.T, BH, 64, 64) && map3_bf16(&maps[1], dout, p.V, p.T, BH, 64, 64) &&
+            map3_bf16(&maps[2], q, p.K, p.T, BH, 64, 64) && map3_bf16(&maps[3], k, p.K, p.T, BH, 64, 64) &&
+            map3_store(&maps[4], dq, false, p.K, p.T, BH, 64, 64) && map3_store(&maps[5], dk, false, p.K, p.T, BH, 64, 64);
+  // dlog alpha through a tile store for vector gates (the map is unused otherwise)
+  ok = ok && (p.gate == GLA_GATE_VECTOR ? map3_store(&maps[6], dla, true, p.K, p.T, BH, 64, 64)
+                                        : map3_store(&maps[6], dq, false, p.K, p.T, BH, 64, 64));
   if (!ok) return GLA_ERR_CUDA;
   // with a scalar gate and two channel halves, dlog alpha is summed by atomic adds
   if (p.gate == GLA_GATE_SCALAR && p.K > kBwdKH)

@@ -84,6 +84,20 @@ bool tc::map3_bf16(CUtensorMap *m, const void *base, uint64_t d0, uint64_t d1, u
   return map3(m, base, d0, d1, d2, b0, b1);
 }
 
+bool tc::map3_store(CUtensorMap *m, const void *base, bool fp32, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t b0,
+                    uint32_t b1) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const uint64_t es = fp32 ? 4 : 2;
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {d0 * es, d0 * d1 * es};
+  cuuint32_t box[3] = {b0, b1, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, fp32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base),
+            dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 namespace {
 
 // 1 if the current device is sm_100 (per device: 1 = yes, 2 = no).
