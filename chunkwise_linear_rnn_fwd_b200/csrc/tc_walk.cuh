@@ -648,17 +648,24 @@ __global__ void __launch_bounds__(kWalkThreads, 1)
           if (ok) ok = dev::mbar_wait(&ofull[(i - 1) & 1], (uint32_t)(((i - 1) >> 1) & 1), a.status);
           dev::tc_fence_after();
         }
+        uint32_t w[KH / 2];  // the bf16 row, kept for the chunk-state stores
 #pragma unroll
         for (int jb = 0; jb < KH / 32; ++jb) {
-          uint32_t w[16];
 #pragma unroll
-          for (int e = 0; e < 16; ++e) w[e] = dev::pack_bf16(S[32 * jb + 2 * e], S[32 * jb + 2 * e + 1]);
-          dev::tmem_st16u(lane_base + colA + (uint32_t)(c0 / 2 + 16 * jb), w);
+          for (int e = 0; e < 16; ++e)
+            w[16 * jb + e] = dev::pack_bf16(S[32 * jb + 2 * e], S[32 * jb + 2 * e + 1]);
+          dev::tmem_st16u(lane_base + colA + (uint32_t)(c0 / 2 + 16 * jb), w + 16 * jb);
         }
         dev::tmem_wait_st();
         dev::tc_fence_before();
         __syncwarp();
         if (lane == 0) dev::mbar_arrive(afull);
+        // S_{i-1} to the backward's layout from the same registers, after the MMA warp
+        // has been released
+        if (st_hb && ok) {
+#pragma unroll
+          for (int jb = 0; jb < KH / 32; ++jb) store_hb(n, jb, w + 16 * jb);
+        }
       } else if (st_hb && ok) {
 #pragma unroll
         for (int jb = 0; jb < KH / 32; ++jb) {
@@ -703,15 +710,6 @@ __global__ void __launch_bounds__(kWalkThreads, 1)
       }
       // ---- off the chain: S_{i-1} (still the A operand in TMEM) to the backward's
       // layout, then the previous chunk's output -------------------------------------
-      if (out && st_hb && ok) {
-        // the whole row in one TMEM round trip, then its 16-byte stores back to back
-        float wf[KH / 2];
-#pragma unroll
-        for (int jb = 0; jb < KH / 32; ++jb) dev::tmem_ld16(lane_base + colA + (uint32_t)(c0 / 2 + 16 * jb), wf + 16 * jb);
-        dev::tmem_wait_ld();
-#pragma unroll
-        for (int jb = 0; jb < KH / 32; ++jb) store_hb(n, jb, reinterpret_cast<const uint32_t *>(wf + 16 * jb));
-      }
       if (out && i >= 1) epilogue(i - 1);
     }
     if (out && nloc > 0) {
