@@ -52,15 +52,15 @@ def algorithmic_bytes(B, H, T, K, V, gate="vector"):
 # DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) measured by ncu on
 # the full-size workload, with the sha256 of the kernel sources it was measured on.  It is
 # reported only while the sources are unchanged (a changed kernel has unknown traffic).
-NCU_TRAFFIC = {"src_sha256": "f0d3f88407fbaa217cd54af5eceb3848d9c3c7f8c9024922510d954f28e2b6de",
-               "per_launch_bytes": {"tc_walk": 117555328, "tc_bwd": 448334336, "tc_prep": 73070848}}
+NCU_TRAFFIC = {"src_sha256": "cdee8da559628cfc47ae53331168aec32159d565ba6b25d6d0ad903d9718a49c",
+               "per_launch_bytes": {"tc_walk": 116625216, "tc_bwd": 461712256, "tc_prep": 71790848, "segment_starts": 12621184}}
 
 
 def kernel_src_sha256():
-    """sha256 over the sources of the tensor-core kernels (the tc_* files)."""
+    """sha256 over the sources of the step's kernels (the tc_* files and seqpar.cu)."""
     d = os.path.join(ROOT, "chunkwise_linear_rnn_fwd_b200", "csrc")
     h = hashlib.sha256()
-    for f in sorted(x for x in os.listdir(d) if x.startswith("tc_")):
+    for f in sorted(x for x in os.listdir(d) if x.startswith("tc_") or x == "seqpar.cu"):
         h.update(f.encode())
         with open(os.path.join(d, f), "rb") as fh:
             h.update(fh.read())
