@@ -118,3 +118,32 @@ def test_fused_epilogue_reports_gate_range():
     ws = pkg.alloc_workspace(pkg.workspace_size(B, H, T, K, V, torch.bfloat16, "vector", 64, False), dev)
     pkg.gla_fwd_epilogue(q, k, v, la, r, workspace=ws)
     assert pkg.poll_status(ws) == -7  # GLA_ERR_GATE_RANGE
+
+
+def test_fused_epilogue_forward_feeds_the_backward():
+    """A training step through the fused forward: gla_fwd_epilogue saving the chunk
+    states, then gla_bwd reading them and the forward's prep outputs from the same
+    workspace.  The gradients match the oracle's back-propagation of the plain
+    recurrence (the epilogue's own backward is the separate pass, tested elsewhere)."""
+    import chunkwise_linear_rnn_fwd_b200 as pkg
+    from chunkwise_linear_rnn_fwd_b200.synth import make_inputs
+    from oracle import oracle
+    B, H, T, K, V = 1, 4, 1100, 256, 512
+    x = make_inputs(B, H, T, K, V, dtype=torch.bfloat16, gate="vector", seed=17, z_mean=-1.0)
+    dev = torch.device("cuda")
+    q, k, v, la, do = (t.to(dev) for t in (x.q, x.k, x.v, x.log_alpha, x.do))
+    r = torch.randn(B, H, T, V, generator=torch.Generator().manual_seed(3)).to(torch.bfloat16).to(dev)
+    flags = pkg.FLAG_SAVE_STATES | pkg.FLAG_REUSE_PREP
+    ws = pkg.alloc_workspace(pkg.workspace_size(B, H, T, K, V, torch.bfloat16, "vector", 64, True, flags=flags), dev)
+    o, y, _ = pkg.gla_fwd_epilogue(q, k, v, la, r, workspace=ws, save_states=True)
+    dq, dk, dv, dla, _ = pkg.gla_bwd(q, k, v, la, do, None, None, workspace=ws, reuse_prep=True, saved_states=True,
+                                     want_dh0=False)
+    torch.cuda.synchronize()
+    assert pkg.poll_status(ws) == 0
+    n = lambda t: t.double().numpy()
+    ro, _ = oracle.fwd(n(x.q), n(x.k), n(x.v), n(x.log_alpha), gate="vector")
+    rdq, rdk, rdv, rdla, _ = oracle.bwd(n(x.q), n(x.k), n(x.v), n(x.log_alpha), n(x.do), None, None, gate="vector")
+    errs = {"o": rel_err(_np(o), ro), "dq": rel_err(_np(dq), rdq), "dk": rel_err(_np(dk), rdk),
+            "dv": rel_err(_np(dv), rdv), "dlog_alpha": rel_err(_np(dla), rdla)}
+    print("fused forward -> backward", {k2: f"{e:.2e}" for k2, e in errs.items()})
+    assert all(e <= TOL[torch.bfloat16] for e in errs.values()), errs
