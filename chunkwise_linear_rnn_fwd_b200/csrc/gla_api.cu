@@ -73,9 +73,8 @@ namespace {
 
 bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
 
-// tensor_path: bf16 descriptors also pass the tensor-core path's shape limits
-// (false for the general gate, which runs on CUDA cores for both dtypes).
-int make_problem(const gla_desc *d, int chunk, Problem *p, bool tensor_path = true) {
+// The descriptor's limits common to both paths (on_tc picks the path).
+int make_problem(const gla_desc *d, int chunk, Problem *p) {
   if (!d) return GLA_ERR_INVALID_ARG;
   if (d->B < 1 || d->H < 1 || d->T < 1 || d->dk < 1 || d->dv < 1) return GLA_ERR_INVALID_ARG;
   if (d->dtype != GLA_DTYPE_BF16 && d->dtype != GLA_DTYPE_FP32) return GLA_ERR_INVALID_ARG;
@@ -106,15 +105,16 @@ int make_problem(const gla_desc *d, int chunk, Problem *p, bool tensor_path = tr
   p->BH = (long)d->B * d->H;
   p->N = (d->T + chunk - 1) / chunk;
   p->Tp = (long)p->N * chunk;
-  if (p->dtype == GLA_DTYPE_BF16 && tensor_path) {
-    const int r = tc_check(*p);
-    if (r != GLA_OK) return r;
-  }
   return GLA_OK;
 }
 
+// bf16 inputs run on the tensor-core path when it takes the shape (d_k 128 or 256,
+// d_v a multiple of 64, chunk 64 with sub-chunk 16); every other shape, and fp32
+// inputs, on the CUDA-core path (fp32 arithmetic, any element type)
+bool on_tc(const Problem &p) { return p.dtype == GLA_DTYPE_BF16 && tc_check(p) == GLA_OK; }
+
 size_t ws_bytes(const Problem &p, bool bwd) {
-  if (p.dtype == GLA_DTYPE_BF16) return tc_workspace(p, bwd);
+  if (on_tc(p)) return tc_workspace(p, bwd);
   return f32_workspace(p, bwd);
 }
 
@@ -189,7 +189,7 @@ int gla_fwd(const gla_desc *desc, const void *q, const void *k, const void *v, c
   GLA_TRY(check_ws(desc, p, (p.flags & GLA_FLAG_SAVE_STATES) != 0));
   cudaStream_t st = (cudaStream_t)stream;
   GLA_TRY(clear_status(desc, st));
-  if (p.dtype == GLA_DTYPE_BF16) return tc_fwd(p, q, k, v, log_alpha, h0, o, h_final, desc->workspace, st);
+  if (on_tc(p)) return tc_fwd(p, q, k, v, log_alpha, h0, o, h_final, desc->workspace, st);
   return f32_fwd(p, q, k, v, log_alpha, nullptr, h0, o, h_final, desc->workspace, st);
 }
 
@@ -217,7 +217,7 @@ int gla_bwd(const gla_desc *desc, const void *q, const void *k, const void *v, c
   GLA_TRY(check_ws(desc, p, true));
   cudaStream_t st = (cudaStream_t)stream;
   GLA_TRY(clear_status(desc, st));
-  if (p.dtype == GLA_DTYPE_BF16)
+  if (on_tc(p))
     return tc_bwd(p, q, k, v, log_alpha, h0, do_, dh_final, dq, dk, dv, dlog_alpha, dh0, desc->workspace, st);
   return f32_bwd(p, q, k, v, log_alpha, nullptr, h0, do_, dh_final, dq, dk, dv, dlog_alpha, nullptr, dh0,
                  desc->workspace, st);
@@ -225,14 +225,14 @@ int gla_bwd(const gla_desc *desc, const void *q, const void *k, const void *v, c
 
 size_t gla_general_workspace_size(const gla_desc *desc, int chunk, int for_bwd) {
   Problem p;
-  if (make_problem(desc, chunk, &p, false) != GLA_OK) return 0;
+  if (make_problem(desc, chunk, &p) != GLA_OK) return 0;
   return f32_general_workspace(p, for_bwd != 0);
 }
 
 int gla_fwd_general(const gla_desc *desc, const void *q, const void *k, const void *v, const float *log_alpha,
                     const float *log_beta, const float *h0, void *o, float *h_final, int chunk, void *stream) {
   Problem p;
-  GLA_TRY(make_problem(desc, chunk, &p, false));
+  GLA_TRY(make_problem(desc, chunk, &p));
   GLA_TRY(check_req(q));
   GLA_TRY(check_req(k));
   GLA_TRY(check_req(v));
@@ -251,7 +251,7 @@ int gla_bwd_general(const gla_desc *desc, const void *q, const void *k, const vo
                     const float *log_beta, const float *h0, const void *do_, const float *dh_final, void *dq,
                     void *dk, void *dv, float *dlog_alpha, float *dlog_beta, float *dh0, int chunk, void *stream) {
   Problem p;
-  GLA_TRY(make_problem(desc, chunk, &p, false));
+  GLA_TRY(make_problem(desc, chunk, &p));
   GLA_TRY(check_req(q));
   GLA_TRY(check_req(k));
   GLA_TRY(check_req(v));
@@ -281,7 +281,7 @@ int gla_fwd_state(const gla_desc *desc, const void *q, const void *k, const void
                   const float *h0, float *delta, float *gamma, int chunk, void *stream) {
   Problem p;
   GLA_TRY(make_problem(desc, chunk, &p));
-  if (p.dtype != GLA_DTYPE_BF16) return GLA_ERR_UNSUPPORTED_SHAPE;
+  if (!on_tc(p)) return GLA_ERR_UNSUPPORTED_SHAPE;  // the summaries exist on the tensor-core path
   GLA_TRY(check_req(q));
   GLA_TRY(check_req(k));
   GLA_TRY(check_req(v));
@@ -300,7 +300,7 @@ int gla_bwd_state(const gla_desc *desc, const void *q, const void *k, const floa
                   const float *dh_final, float *ddelta, float *gamma, int chunk, void *stream) {
   Problem p;
   GLA_TRY(make_problem(desc, chunk, &p));
-  if (p.dtype != GLA_DTYPE_BF16) return GLA_ERR_UNSUPPORTED_SHAPE;
+  if (!on_tc(p)) return GLA_ERR_UNSUPPORTED_SHAPE;  // the summaries exist on the tensor-core path
   GLA_TRY(check_req(q));
   GLA_TRY(check_req(k));
   GLA_TRY(check_gate_ptr(p, log_alpha));
@@ -470,7 +470,7 @@ int gla_fwd_epilogue(const gla_desc *desc, const void *q, const void *k, const v
   }
   // two passes: the forward, then the epilogue over its bf16 / fp32 output (the
   // second pass keeps the status word, so a device error of either stays reported)
-  const int rf = p.dtype == GLA_DTYPE_BF16 ? tc_fwd(p, q, k, v, log_alpha, h0, o, h_final, desc->workspace, st)
+  const int rf = on_tc(p) ? tc_fwd(p, q, k, v, log_alpha, h0, o, h_final, desc->workspace, st)
                                            : f32_fwd(p, q, k, v, log_alpha, nullptr, h0, o, h_final, desc->workspace, st);
   if (rf != GLA_OK) return rf;
   return gla::epilogue_fwd(desc, o, r, w, b, eps, y, st, false);

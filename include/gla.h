@@ -144,7 +144,10 @@ int gla_check(const gla_desc *desc, int chunk);
 /* Forward (sections 4.2-4.3; Algorithms 3 and 5 of Appendix B by title).
  *   q, k [B,H,T,d_k], v [B,H,T,d_v], log_alpha (see layout), h0 [B,H,d_k,d_v] or NULL
  *   o [B,H,T,d_v] (written), h_final [B,H,d_k,d_v] or NULL (written: S_T)
- * chunk: C (64 for the bf16 tensor-core path; 16/32/64/128 for fp32).
+ * chunk: C in {16, 32, 64, 128}.  bf16 inputs run on the tensor-core path when
+ * d_k is 128 or 256, d_v a multiple of 64, C = 64 and the sub-chunk 16; every
+ * other shape, and fp32 inputs, run on the CUDA-core path (fp32 arithmetic,
+ * pairwise log-space intra-chunk terms; the workspace sizes follow the path).
  * Returns GLA_OK or an error code; on error nothing was enqueued. */
 int gla_fwd(const gla_desc *desc, const void *q, const void *k, const void *v,
             const float *log_alpha, const float *h0, void *o, float *h_final, int chunk,
@@ -263,7 +266,8 @@ int gla_bwd_general(const gla_desc *desc, const void *q, const void *k, const vo
  * state it produces.  One exchange of the summaries (an all-gather), a fold, and
  * every piece reruns gla_fwd / gla_bwd with its incoming state.  Each call below
  * describes one piece: desc->T is the piece's token count, the tensors hold only
- * the piece's tokens.  bf16 path only (fp32 descriptors: GLA_ERR_UNSUPPORTED_SHAPE).
+ * the piece's tokens.  Tensor-core path only (fp32 descriptors, and bf16 shapes that
+ * path does not take: GLA_ERR_UNSUPPORTED_SHAPE).
  *
  * gla_fwd_state: delta [B,H,dk,dv] fp32 = the state after the piece's tokens
  *   starting from h0 (NULL = zero), i.e. the h_final of gla_fwd, without computing

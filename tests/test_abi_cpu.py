@@ -304,3 +304,21 @@ def test_fused_epilogue_validation_enqueues_nothing(lib):
     e.workspace = 1 << 20
     e.workspace_bytes = 1 << 40
     assert call(dd=e) == -2
+
+
+def test_bf16_shapes_outside_the_tensor_core_path(lib):
+    """bf16 descriptors the tensor-core path does not take (chunk 16, 32, 128; d_k 64;
+    d_v not a multiple of 64) are valid and sized for the CUDA-core path; the
+    sequence summaries, which exist on the tensor-core path only, refuse them."""
+    vp = ctypes.c_void_p
+    a = vp(4096)
+    for kw, chunk in ((dict(), 16), (dict(), 32), (dict(), 128), (dict(dk=64), 64), (dict(dv=200), 64)):
+        d = desc(**kw)
+        assert lib.gla_check(ctypes.byref(d), chunk) == 0, (kw, chunk)
+        assert lib.gla_workspace_size(ctypes.byref(d), chunk, 1) > 0
+        d.workspace = 1 << 20
+        d.workspace_bytes = 1 << 40
+        assert lib.gla_fwd_state(ctypes.byref(d), a, a, a, a, None, a, a, chunk, None) == -2
+    # the same bf16 shape sizes its workspace by the path that runs it
+    d64, d128 = desc(), desc()
+    assert lib.gla_workspace_size(ctypes.byref(d64), 64, 0) != lib.gla_workspace_size(ctypes.byref(d128), 128, 0)

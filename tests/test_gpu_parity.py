@@ -143,3 +143,12 @@ def test_saved_states_k128():
     errs = run_case(1, 3, 300, 128, 256, dtype=BF16, gate="scalar", chunk=64, seed=10, with_h0=True,
                     reuse_prep=True, save_states=True)
     assert_parity(errs, BF16)
+
+
+@pytest.mark.parametrize("chunk,K,V", [(16, 128, 128), (32, 128, 256), (128, 256, 128), (64, 64, 96)])
+def test_bf16_shapes_on_the_cuda_core_path(chunk, K, V):
+    """bf16 inputs in shapes the tensor-core path does not take (chunk 16, 32 or 128;
+    d_k = 64 with d_v = 96) run on the CUDA-core path: fwd+bwd parity at the bf16
+    tolerance, ragged T."""
+    errs = run_case(1, 2, 300, K, V, dtype=BF16, gate="vector", chunk=chunk, bwd=True, seed=chunk + K)
+    assert_parity(errs, BF16)
