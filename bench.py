@@ -1177,6 +1177,10 @@ def main():
     ap.add_argument("--step-only", action="store_true",
                     help="time the fwd+bwd step alone (no decode, epilogue, sequence-parallel, variant, sweep, "
                          "general-gate or CPU measurements): the command line of the profiler captures")
+    ap.add_argument("--fused-epilogue-once", action="store_true",
+                    help="run gla_fwd_epilogue (the forward with the layer epilogue fused into its output store) "
+                         "three times on the workload and exit (a small case for profiler captures; prints no "
+                         "bench line)")
     ap.add_argument("--epilogue-once", action="store_true",
                     help="run the layer epilogue forward and backward twice on the workload's output shape and "
                          "exit (a small case for profiler captures; prints no bench line)")
@@ -1193,9 +1197,36 @@ def main():
         return run_sweep(args)
     if args.epilogue_once:
         return run_epilogue_once(w)
+    if args.fused_epilogue_once:
+        return run_fused_epilogue_once(w)
     if args.seqpar:
         return run_seqpar(args, w)
     return run_ours(args, w)
+
+
+def run_fused_epilogue_once(w):
+    """Three calls of gla_fwd_epilogue on the workload (inputs drawn on the device),
+    then the device status word.  Launch order per call: prep, pre-pass walk, start
+    fold, fused output walk."""
+    import torch
+
+    import chunkwise_linear_rnn_fwd_b200 as pkg
+
+    dev = torch.device("cuda", 0)
+    B, H, T, K, V, C = w["B"], w["H"], w["T"], w["K"], w["V"], w["C"]
+    g = torch.Generator(device=dev)
+    g.manual_seed(0)
+    q = torch.randn(B, H, T, K, device=dev, generator=g).to(torch.bfloat16)
+    k = (torch.randn(B, H, T, K, device=dev, generator=g) / K ** 0.5).to(torch.bfloat16)
+    v, r = (torch.randn(B, H, T, V, device=dev, generator=g).to(torch.bfloat16) for _ in range(2))
+    la = torch.nn.functional.logsigmoid(torch.randn(B, H, T, K, device=dev, generator=g) + w["z_mean"]) / 16
+    ws = pkg.alloc_workspace(pkg.workspace_size(B, H, T, K, V, torch.bfloat16, w["gate"], C, False), dev)
+    for _ in range(3):
+        pkg.gla_fwd_epilogue(q, k, v, la, r, workspace=ws, chunk=C)
+    torch.cuda.synchronize()
+    st = pkg.poll_status(ws)
+    print(json.dumps({"fused_epilogue_once": {"B": B, "H": H, "T": T, "d_k": K, "d_v": V, "status": st}}))
+    return 0 if st == 0 else 1
 
 
 def run_epilogue_once(w):
