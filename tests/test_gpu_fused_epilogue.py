@@ -58,6 +58,8 @@ def _case(B, H, T, K, V, *, dtype=torch.bfloat16, gate="vector", seed=0, z_mean=
     (1, 3, 65, 128, 128, "none", 0, False, True),       # clusters of 1 (one tile per token)
     (1, 1, 1, 256, 384, "vector", 0, True, True),       # a single token, clusters of 3
     (2, 1, 1000, 256, 512, "vector", 5, False, True),   # five segments of four chunk tiles each
+    (1, 3, 200, 128, 512, "vector", 0, True, True),     # d_k = 128 with clusters of 4
+    (1, 2, 4096, 256, 512, "vector", 0, False, True),   # more segments than resident clusters: capped
 ])
 def test_fused_epilogue_parity(B, H, T, K, V, gate, segments, with_h0, affine):
     errs, (o, hT, o_plain, hT_plain, _) = _case(B, H, T, K, V, gate=gate, seed=T + V, segments=segments,
